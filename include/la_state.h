@@ -1,0 +1,201 @@
+/*
+ * la_state.h -- C ABI of liblastate.so: the fixed-size recurrent-state step of linear
+ * attention (Gated DeltaNet family) on NVIDIA B200 (sm_100a).
+ *
+ * What the library computes.  Per state head the state S is a d_k x d_v matrix.  For
+ * each token, with gate g and write strength beta:
+ *
+ *   u = b * (v - c * S^T k)          write (delta) vector, length d_v
+ *   S <- a * S + k u^T               decay plus rank-one correction
+ *   o = scale * S^T q                readout by the query, from the UPDATED state
+ *
+ *   rule         a   b     c       source
+ *   linear       1   1     0       "basic additive"
+ *   gated        g   1     0       "exponential decay"
+ *   delta        1   beta  1       "delta rule without decay"
+ *   gated_delta  g   beta  g       S <- g (I - beta k k^T) S + beta k v^T (the default)
+ *
+ * The rule names, their one-line meanings and the default are those of the ONNX
+ * LinearAttention operator described in "Seven Architectures Replacing KV Cache With
+ * Bounded Mutable State" (section "ONNX LinearAttention / FlashInfer"); the
+ * gated_delta recurrence is the one of the "Gated DeltaNet" glossary page (Technical
+ * definition: decay by a gate, rank-one delta-rule correction, projection by the
+ * query) and of the KDA formula in the "Kimi Linear" section of the same article,
+ * read with a scalar gate.  The kernels compute the readout in the rearranged form of
+ * the "Gated DeltaNet" page (Engineering details),
+ *   o = scale * ( a * (S_old^T q) + (k . q) * u ),
+ * so that the update and the readout share one pass over S.  All arithmetic is FP32;
+ * the state is stored in FP32 or BF16 (rounded to nearest even), as in the "Recurrent
+ * state" glossary page (Why it matters: BF16 storage, FP32 compute).
+ *
+ * Layouts (row-major, last index contiguous; all device memory):
+ *   state pool   [n_slots, H_v, d_k, d_v]       (the ONNX past_state / present_state
+ *                                                shape (B, H_kv, d_k, d_v) with B -> slots)
+ *   q, k         [B or T, H_qk, d_k]   io dtype  state head h reads q/k head h / (H_v/H_qk)
+ *   v, o         [B or T, H_v,  d_v]   io dtype
+ *   g, beta      [B or T, H_v]         float32
+ * Supported (d_k, d_v): (16,16), (64,64), (128,64), (128,128).
+ *
+ * Slots.  A request reads its state from read_slot[b] of the source pool and writes
+ * the new state to write_slot[b] of the destination pool ("Recurrent state" and "Gated
+ * DeltaNet" glossary pages: separate slots for reading a prefix-cache checkpoint and
+ * writing live state, so the checkpoint survives).  A NULL slot array means slot b for
+ * request b ("dense" mode: the source pool is past_state, the destination pool is
+ * present_state, and they may be the same pool for an in-place update).
+ *
+ * Conventions for every entry point.
+ *   - Ownership: all buffers belong to the caller.  The library allocates, frees and
+ *     synchronizes nothing; work is enqueued asynchronously on `stream` (a
+ *     cudaStream_t; NULL = the legacy default stream).
+ *   - Host-side errors (LA_ERR_*) are returned before anything is launched.
+ *   - Device-side errors never trap: a tile with an out-of-range slot, or a sequence
+ *     with inconsistent cu_seqlens, is skipped (its outputs and destination are left
+ *     untouched) and a bit is OR-ed into *err_word (device int32, required).  The
+ *     caller reads it after synchronizing.  Bits are LA_DEVERR_*.
+ *   - Preconditions (not checked on the device; la_state_check_slots checks them on the
+ *     host): write slots are distinct, and no write slot equals another request's read
+ *     slot.  Read slots may repeat; a request may read and write the same slot.
+ *   - Pointers to the pool, q, k, v, o and dense buffers must be 16-byte aligned;
+ *     g, beta and int32 arrays 4-byte aligned.
+ */
+#ifndef LA_STATE_H
+#define LA_STATE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LA_ABI_VERSION 1
+
+typedef enum {
+    LA_RULE_LINEAR = 0,
+    LA_RULE_GATED = 1,
+    LA_RULE_DELTA = 2,
+    LA_RULE_GATED_DELTA = 3
+} la_rule;
+
+typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_NULL = 1,        /* a required pointer is NULL */
+    LA_ERR_SHAPE = 2,       /* a size is negative / zero where it must not be, or inconsistent */
+    LA_ERR_UNSUPPORTED = 3, /* (d_k, d_v), dtype or rule outside the supported set */
+    LA_ERR_ALIGN = 4,       /* a pointer violates the alignment rule above */
+    LA_ERR_ALIAS = 5,       /* la_state_check_slots: slot preconditions violated */
+    LA_ERR_CUDA = 6         /* the CUDA runtime refused the launch (see la_last_cuda_error) */
+} la_status;
+
+/* Bits OR-ed into *err_word by the kernels. */
+#define LA_DEVERR_READ_SLOT 1u  /* a read / source slot index outside [0, n_slots) */
+#define LA_DEVERR_WRITE_SLOT 2u /* a write / destination slot index outside [0, n_slots) */
+#define LA_DEVERR_CU_SEQLENS 4u /* cu_seqlens not non-decreasing within [0, total_tokens], or a bad seq_order entry */
+#define LA_DEVERR_TIMEOUT 8u    /* an internal pipeline wait gave up (should never happen) */
+
+typedef struct {
+    int32_t n_qk_heads; /* H_qk: heads of q and k */
+    int32_t n_v_heads;  /* H_v: heads of v, o and of the state; a multiple of H_qk */
+    int32_t d_k;
+    int32_t d_v;
+} la_shape;
+
+/* A slot pool: n_slots states of `shape`, contiguous, [n_slots, H_v, d_k, d_v]. */
+typedef struct {
+    void *data;     /* device pointer, 16-byte aligned */
+    int32_t dtype;  /* la_dtype of the stored state */
+    int32_t n_slots;
+    la_shape shape;
+} la_pool;
+
+/* Bytes of one slot (one request's state for one layer): H_v * d_k * d_v * sizeof(dtype).
+ * Pure host function; returns 0 for an invalid shape or dtype.  For 64 heads of 128 x 128
+ * at 2 bytes this is 2 MiB, the per-request figure of the ONNX section of "Seven
+ * Architectures ..."; for 128 heads of 128 x 64 at BF16 it is 2 MiB, the Nemotron-H-8B
+ * per-layer figure of "SSM / linear-RNN decode: the constant-size recurrent state update". */
+size_t la_state_bytes(const la_shape *shape, la_dtype dtype);
+
+/* 1 if (d_k, d_v) is one of the compiled tile shapes, else 0.  Pure host function. */
+int la_shape_supported(int32_t d_k, int32_t d_v);
+
+/* One batched decode step (one token per request) for B requests and all H_v heads.
+ *   src, dst     pools with identical shape and dtype (they may be the same pool)
+ *   read_slot    device int32 [B] or NULL (request b reads src slot b)
+ *   write_slot   device int32 [B] or NULL (request b writes dst slot b)
+ *   q, k         [B, H_qk, d_k] io dtype;  v, o: [B, H_v, d_v] io dtype
+ *   g            float32 [B, H_v]; required for gated / gated_delta, ignored otherwise
+ *   beta         float32 [B, H_v]; required for delta / gated_delta, ignored otherwise
+ *   scale        multiplies the readout (1.0 for pre-normalised queries)
+ *   err_word     device int32, required; bits LA_DEVERR_* are OR-ed in
+ * B == 0 is a no-op returning LA_OK.  With a NULL slot array, B must not exceed that
+ * pool's n_slots (LA_ERR_SHAPE). */
+la_status la_state_step(la_rule rule, const la_pool *src, const int32_t *read_slot,
+                        const la_pool *dst, const int32_t *write_slot, int32_t B,
+                        const void *q, const void *k, const void *v, la_dtype io,
+                        const float *g, const float *beta, float scale, void *o,
+                        int32_t *err_word, void *stream);
+
+/* Token-serial scan (prefill) over n_seqs packed variable-length sequences.  The state
+ * of each (sequence, head) stays on chip in FP32 across all of the sequence's tokens;
+ * it is read once at the start and stored once at the end.
+ *   src, read_slot  initial state: src slot read_slot[s]; if read_slot is NULL the
+ *                   initial state is zero and src may be NULL.  src may have another
+ *                   dtype than dst, but the same shape.
+ *   dst, write_slot final state goes to dst slot write_slot[s] (NULL: slot s)
+ *   cu_seqlens      device int32 [n_seqs + 1]: sequence s is tokens
+ *                   [cu_seqlens[s], cu_seqlens[s+1]) of the packed arrays
+ *   total_tokens    T, the leading size of q, k, v, g, beta, o
+ *   seq_order       device int32 [n_seqs] or NULL: the order in which sequences are
+ *                   handed to the SMs (longest first balances the load best); each
+ *                   sequence must appear exactly once.  NULL = 0, 1, 2, ...
+ *   q, k            [T, H_qk, d_k];  v, o: [T, H_v, d_v];  g, beta: [T, H_v]
+ * Empty sequences are allowed (their initial state is copied to the destination).
+ * n_seqs == 0 is a no-op returning LA_OK. */
+la_status la_state_scan(la_rule rule, const la_pool *src, const int32_t *read_slot,
+                        const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
+                        const int32_t *cu_seqlens, int32_t total_tokens, const int32_t *seq_order,
+                        const void *q, const void *k, const void *v, la_dtype io,
+                        const float *g, const float *beta, float scale, void *o,
+                        int32_t *err_word, void *stream);
+
+/* Slot-pool maintenance, bit-exact whole-slot copies ("Recurrent state" glossary: slot
+ * allocation and prefix-cache checkpoints; "Seven Architectures ...", ONNX section:
+ * snapshots saved and restored for speculative-decoding rollback, migrated between
+ * places).  n == 0 is a no-op.  Slot arrays are device int32 [n].
+ *   copy     pool[dst_slots[i]] <- pool[src_slots[i]]; the destination set must not
+ *            intersect the source set (except a slot copied onto itself)
+ *   gather   dense[i] <- pool[slots[i]]          dense: [n, H_v, d_k, d_v], pool dtype
+ *   scatter  pool[slots[i]] <- dense[i]
+ *   zero     pool[slots[i]] <- 0 */
+la_status la_state_pool_copy(const la_pool *pool, int32_t n, const int32_t *src_slots,
+                             const int32_t *dst_slots, int32_t *err_word, void *stream);
+la_status la_state_pool_gather(const la_pool *pool, int32_t n, const int32_t *slots, void *dense,
+                               int32_t *err_word, void *stream);
+la_status la_state_pool_scatter(const la_pool *pool, int32_t n, const int32_t *slots,
+                                const void *dense, int32_t *err_word, void *stream);
+la_status la_state_pool_zero(const la_pool *pool, int32_t n, const int32_t *slots,
+                             int32_t *err_word, void *stream);
+
+/* Host-side check of the slot preconditions of la_state_step / la_state_scan on HOST
+ * copies of the slot arrays (either may be NULL = identity): every index in [0, n_slots),
+ * write slots distinct, no write slot equal to another request's read slot.  Returns
+ * LA_OK, LA_ERR_SHAPE (index out of range) or LA_ERR_ALIAS. */
+la_status la_state_check_slots(int32_t B, const int32_t *read_slot_host,
+                               const int32_t *write_slot_host, int32_t n_slots);
+
+/* Human-readable name of a status. */
+const char *la_status_str(la_status status);
+
+/* The cudaError_t of the most recent LA_ERR_CUDA returned on the calling thread (0 if none). */
+int32_t la_last_cuda_error(void);
+
+/* LA_ABI_VERSION of the loaded library. */
+int32_t la_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_STATE_H */

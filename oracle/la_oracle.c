@@ -1,0 +1,365 @@
+/*
+ * la_oracle.c -- plain, slow, obviously correct CPU oracle for the recurrent-state
+ * step of linear attention.  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and
+ * the benchmark's CPU-baseline leg call it; the product library never does, and this
+ * file shares no code, header or constant generator with the CUDA path.
+ *
+ * What it computes (written from the pages, not from any listing):
+ *
+ *   "Gated DeltaNet" (inferencex glossary), Technical definition: at each step the
+ *   running state is decayed by a gate, corrected by a rank-one delta-rule term and
+ *   projected by the query.
+ *   "Seven Architectures Replacing KV Cache With Bounded Mutable State", section
+ *   "ONNX LinearAttention / FlashInfer": update_rule in {linear (basic additive),
+ *   gated (exponential decay), delta (delta rule without decay), gated_delta}; state
+ *   tensors past_state / present_state of shape (B, H_kv, d_k, d_v).
+ *   Same page, section "Kimi Linear": S_t = Diag(a) S_{t-1} + b k (v - Diag(a) S_{t-1}^T k)^T,
+ *   read here with a scalar gate (the Gated DeltaNet special case).
+ *
+ * Per state head, with S (d_k x d_v), per token t:
+ *
+ *   u_t = b_t * (v_t - c_t * S_{t-1}^T k_t)
+ *   S_t = a_t * S_{t-1} + k_t u_t^T
+ *   o_t = scale * S_t^T q_t                 (readout from the UPDATED state)
+ *
+ *   rule         a_t   b_t    c_t
+ *   linear       1     1      0
+ *   gated        g_t   1      0
+ *   delta        1     beta_t 1
+ *   gated_delta  g_t   beta_t g_t
+ *
+ * Arithmetic is IEEE double throughout.  Rounding happens only where the method
+ * stores a value ("Recurrent state" glossary, Why it matters: state stored in BF16
+ * while computed in a wider type): the state after each decode step, the state at the
+ * end of a scan, and each output o_t (to the io type).  Storage types: 0 = f64 (no
+ * rounding), 1 = f32, 2 = bf16 (round-to-nearest-even from the IEEE definition).
+ *
+ * Layouts (row-major, last index contiguous):
+ *   pool   [n_slots, H_v, d_k, d_v]
+ *   q, k   [B or T, H_qk, d_k]        state head h reads q/k head h / (H_v / H_qk)
+ *   v, o   [B or T, H_v, d_v]
+ *   g, beta[B or T, H_v]
+ *
+ * Slots ("Recurrent state" glossary, Engineering details / Why it matters; "Gated
+ * DeltaNet" glossary, Why it matters): a request reads its state from read_slot[b]
+ * (NULL: slot b) and writes it to write_slot[b] (NULL: slot b), so a checkpoint slot
+ * survives a step that continues from it.  A request whose slot index is outside the
+ * pool is skipped (its outputs and destination are left untouched) and an error bit
+ * is returned: 1 = read slot, 2 = write slot, 4 = bad cu_seqlens.
+ */
+#include "la_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define LAO_ERR_READ_SLOT 1
+#define LAO_ERR_WRITE_SLOT 2
+#define LAO_ERR_CU_SEQLENS 4
+
+/* ---- rounding to a storage type ------------------------------------------------ */
+
+/* Largest finite bfloat16: (2 - 2^-7) * 2^127. */
+static const double BF16_MAX = 3.38953138925153547590470800371487866880e38;
+
+/* Round x to the nearest bfloat16 value, ties to even.  bfloat16 has 8 significant
+ * bits, the binary32 exponent range, and subnormals down to 2^-133.  The quantum of
+ * the binade holding |x| is 2^(e-8) where |x| = m 2^e, m in [0.5, 1); below the
+ * normal range the quantum stays 2^-133.  x / quantum is exact in double, rint()
+ * rounds it half-to-even, and the product is exact again.  A result beyond the
+ * largest finite value overflows to infinity.  NaN stays NaN. */
+double lao_round_bf16(double x)
+{
+    if (isnan(x) || isinf(x) || x == 0.0) return x;
+    int e;
+    frexp(fabs(x), &e);
+    int qe = e - 8;
+    if (qe < -133) qe = -133;
+    double y = ldexp(rint(ldexp(x, -qe)), qe);
+    if (fabs(y) > BF16_MAX) return copysign(INFINITY, x);
+    return y;
+}
+
+double lao_round_to(double x, int dtype)
+{
+    if (dtype == LAO_F32) return (double)(float)x;
+    if (dtype == LAO_BF16) return lao_round_bf16(x);
+    return x;
+}
+
+/* ---- one state head, one token ------------------------------------------------- */
+
+static void rule_coefficients(int rule, double g, double beta, double *a, double *b, double *c)
+{
+    switch (rule) {
+    case LAO_RULE_LINEAR:      *a = 1.0; *b = 1.0;  *c = 0.0; break;
+    case LAO_RULE_GATED:       *a = g;   *b = 1.0;  *c = 0.0; break;
+    case LAO_RULE_DELTA:       *a = 1.0; *b = beta; *c = 1.0; break;
+    default: /* gated_delta */ *a = g;   *b = beta; *c = g;   break;
+    }
+}
+
+/* S (dk x dv, in/out) <- a S + k u^T with u = b (v - c S^T k); o = scale * S_new^T q.
+ * u is scratch of length dv. */
+static void token_update(int rule, int dk, int dv, double *S, const double *q, const double *k,
+                         const double *v, double g, double beta, double scale, double *o, double *u)
+{
+    double a, b, c;
+    rule_coefficients(rule, g, beta, &a, &b, &c);
+    for (int j = 0; j < dv; ++j) {
+        double pj = 0.0; /* (S^T k)_j */
+        for (int i = 0; i < dk; ++i) pj += S[(size_t)i * dv + j] * k[i];
+        u[j] = b * (v[j] - c * pj);
+    }
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j)
+            S[(size_t)i * dv + j] = a * S[(size_t)i * dv + j] + k[i] * u[j];
+    for (int j = 0; j < dv; ++j) {
+        double oj = 0.0; /* (S_new^T q)_j */
+        for (int i = 0; i < dk; ++i) oj += S[(size_t)i * dv + j] * q[i];
+        o[j] = scale * oj;
+    }
+}
+
+static int head_group(int n_qk_heads, int n_v_heads, int h)
+{
+    return h / (n_v_heads / n_qk_heads);
+}
+
+/* ---- batched decode step -------------------------------------------------------- */
+
+int lao_step(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+             const double *src_pool, int src_slots,
+             double *dst_pool, int dst_slots, int dst_dtype,
+             const int *read_slot, const int *write_slot, int B,
+             const double *q, const double *k, const double *v, int io_dtype,
+             const double *g, const double *beta, double scale, double *o)
+{
+    const size_t tile = (size_t)dk * dv;
+    const size_t slot = (size_t)n_v_heads * tile;
+    int err = 0;
+    /* New states are computed for every request before any is written, so a request
+     * that reads and writes the same slot sees its old state. */
+    double *next = (double *)malloc(sizeof(double) * (B > 0 ? (size_t)B : 1) * slot);
+    unsigned char *ok = (unsigned char *)calloc(B > 0 ? (size_t)B : 1, 1);
+    if (!next || !ok) { free(next); free(ok); return -1; }
+
+    for (int b = 0; b < B; ++b) {
+        int rs = read_slot ? read_slot[b] : b;
+        int ws = write_slot ? write_slot[b] : b;
+        if (rs < 0 || rs >= src_slots) { err |= LAO_ERR_READ_SLOT; continue; }
+        if (ws < 0 || ws >= dst_slots) { err |= LAO_ERR_WRITE_SLOT; continue; }
+        ok[b] = 1;
+    }
+
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < n_v_heads; ++h) {
+            if (!ok[b]) continue;
+            int rs = read_slot ? read_slot[b] : b;
+            int hq = head_group(n_qk_heads, n_v_heads, h);
+            double *S = next + (size_t)b * slot + (size_t)h * tile;
+            double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+            memcpy(S, src_pool + (size_t)rs * slot + (size_t)h * tile, sizeof(double) * tile);
+            double *ob = o + ((size_t)b * n_v_heads + h) * dv;
+            token_update(rule, dk, dv, S,
+                         q + ((size_t)b * n_qk_heads + hq) * dk,
+                         k + ((size_t)b * n_qk_heads + hq) * dk,
+                         v + ((size_t)b * n_v_heads + h) * dv,
+                         g ? g[(size_t)b * n_v_heads + h] : 1.0,
+                         beta ? beta[(size_t)b * n_v_heads + h] : 1.0,
+                         scale, ob, u);
+            for (int j = 0; j < dv; ++j) ob[j] = lao_round_to(ob[j], io_dtype);
+            for (size_t e = 0; e < tile; ++e) S[e] = lao_round_to(S[e], dst_dtype);
+            free(u);
+        }
+    }
+
+    for (int b = 0; b < B; ++b) {
+        if (!ok[b]) continue;
+        int ws = write_slot ? write_slot[b] : b;
+        memcpy(dst_pool + (size_t)ws * slot, next + (size_t)b * slot, sizeof(double) * slot);
+    }
+    free(next);
+    free(ok);
+    return err;
+}
+
+/* The readout of one decode step written in the rearranged form of the "Gated DeltaNet"
+ * glossary (Engineering details): the decayed state times the query plus the current
+ * token's contribution, a scalar (k . q) times the write vector u.
+ *   o = scale * ( a * (S_{t-1}^T q) + (k . q) * u ).
+ * Used only to check the identity against the direct readout of lao_step.  Dense mode
+ * (request b reads slot b of src_pool); state is not written. */
+void lao_readout_rearranged(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+                            const double *src_pool, int B,
+                            const double *q, const double *k, const double *v,
+                            const double *g, const double *beta, double scale, double *o)
+{
+    const size_t tile = (size_t)dk * dv;
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < n_v_heads; ++h) {
+            int hq = head_group(n_qk_heads, n_v_heads, h);
+            const double *S = src_pool + ((size_t)b * n_v_heads + h) * tile;
+            const double *qb = q + ((size_t)b * n_qk_heads + hq) * dk;
+            const double *kb = k + ((size_t)b * n_qk_heads + hq) * dk;
+            const double *vb = v + ((size_t)b * n_v_heads + h) * dv;
+            double a, bc, c;
+            rule_coefficients(rule, g ? g[(size_t)b * n_v_heads + h] : 1.0,
+                              beta ? beta[(size_t)b * n_v_heads + h] : 1.0, &a, &bc, &c);
+            double kq = 0.0;
+            for (int i = 0; i < dk; ++i) kq += kb[i] * qb[i];
+            for (int j = 0; j < dv; ++j) {
+                double pj = 0.0, rj = 0.0;
+                for (int i = 0; i < dk; ++i) {
+                    pj += S[(size_t)i * dv + j] * kb[i];
+                    rj += S[(size_t)i * dv + j] * qb[i];
+                }
+                double uj = bc * (vb[j] - c * pj);
+                o[((size_t)b * n_v_heads + h) * dv + j] = scale * (a * rj + kq * uj);
+            }
+        }
+    }
+}
+
+/* ---- token-serial scan over packed variable-length sequences -------------------- */
+
+int lao_scan(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+             const double *src_pool, int src_slots, const int *read_slot,
+             double *dst_pool, int dst_slots, int dst_dtype, const int *write_slot,
+             int n_seqs, const int *cu_seqlens, int total_tokens,
+             const double *q, const double *k, const double *v, int io_dtype,
+             const double *g, const double *beta, double scale, double *o)
+{
+    const size_t tile = (size_t)dk * dv;
+    const size_t slot = (size_t)n_v_heads * tile;
+    int err = 0;
+    double *next = (double *)malloc(sizeof(double) * (n_seqs > 0 ? (size_t)n_seqs : 1) * slot);
+    unsigned char *ok = (unsigned char *)calloc(n_seqs > 0 ? (size_t)n_seqs : 1, 1);
+    if (!next || !ok) { free(next); free(ok); return -1; }
+
+    if (n_seqs > 0 && cu_seqlens[0] != 0) err |= LAO_ERR_CU_SEQLENS;
+    for (int s = 0; s < n_seqs; ++s) {
+        int t0 = cu_seqlens[s], t1 = cu_seqlens[s + 1];
+        if (t0 < 0 || t1 < t0 || t1 > total_tokens) { err |= LAO_ERR_CU_SEQLENS; continue; }
+        if (read_slot && (read_slot[s] < 0 || read_slot[s] >= src_slots)) { err |= LAO_ERR_READ_SLOT; continue; }
+        int ws = write_slot ? write_slot[s] : s;
+        if (ws < 0 || ws >= dst_slots) { err |= LAO_ERR_WRITE_SLOT; continue; }
+        ok[s] = 1;
+    }
+
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int s = 0; s < n_seqs; ++s) {
+        for (int h = 0; h < n_v_heads; ++h) {
+            if (!ok[s]) continue;
+            int hq = head_group(n_qk_heads, n_v_heads, h);
+            double *S = next + (size_t)s * slot + (size_t)h * tile;
+            double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+            if (read_slot)
+                memcpy(S, src_pool + (size_t)read_slot[s] * slot + (size_t)h * tile, sizeof(double) * tile);
+            else
+                memset(S, 0, sizeof(double) * tile);
+            for (int t = cu_seqlens[s]; t < cu_seqlens[s + 1]; ++t) {
+                double *ot = o + ((size_t)t * n_v_heads + h) * dv;
+                token_update(rule, dk, dv, S,
+                             q + ((size_t)t * n_qk_heads + hq) * dk,
+                             k + ((size_t)t * n_qk_heads + hq) * dk,
+                             v + ((size_t)t * n_v_heads + h) * dv,
+                             g ? g[(size_t)t * n_v_heads + h] : 1.0,
+                             beta ? beta[(size_t)t * n_v_heads + h] : 1.0,
+                             scale, ot, u);
+                for (int j = 0; j < dv; ++j) ot[j] = lao_round_to(ot[j], io_dtype);
+            }
+            for (size_t e = 0; e < tile; ++e) S[e] = lao_round_to(S[e], dst_dtype);
+            free(u);
+        }
+    }
+
+    for (int s = 0; s < n_seqs; ++s) {
+        if (!ok[s]) continue;
+        int ws = write_slot ? write_slot[s] : s;
+        memcpy(dst_pool + (size_t)ws * slot, next + (size_t)s * slot, sizeof(double) * slot);
+    }
+    free(next);
+    free(ok);
+    return err;
+}
+
+/* ---- slot pool: whole-slot byte copies ------------------------------------------ */
+/* Checkpoints and snapshots ("Recurrent state" glossary, Why it matters; "Seven
+ * Architectures", ONNX section on saving and restoring state snapshots) are plain byte
+ * copies of whole slots.  All sources are read before any destination is written. */
+
+int lao_pool_copy(unsigned char *pool, size_t slot_bytes, int n_slots, int n,
+                  const int *src_slots, const int *dst_slots)
+{
+    int err = 0;
+    unsigned char *tmp = (unsigned char *)malloc(slot_bytes * (n > 0 ? (size_t)n : 1));
+    if (!tmp) return -1;
+    for (int i = 0; i < n; ++i) {
+        if (src_slots[i] < 0 || src_slots[i] >= n_slots) { err |= LAO_ERR_READ_SLOT; continue; }
+        memcpy(tmp + (size_t)i * slot_bytes, pool + (size_t)src_slots[i] * slot_bytes, slot_bytes);
+    }
+    for (int i = 0; i < n; ++i) {
+        if (src_slots[i] < 0 || src_slots[i] >= n_slots) continue;
+        if (dst_slots[i] < 0 || dst_slots[i] >= n_slots) { err |= LAO_ERR_WRITE_SLOT; continue; }
+        memcpy(pool + (size_t)dst_slots[i] * slot_bytes, tmp + (size_t)i * slot_bytes, slot_bytes);
+    }
+    free(tmp);
+    return err;
+}
+
+int lao_pool_gather(const unsigned char *pool, size_t slot_bytes, int n_slots, int n,
+                    const int *slots, unsigned char *dense)
+{
+    int err = 0;
+    for (int i = 0; i < n; ++i) {
+        if (slots[i] < 0 || slots[i] >= n_slots) { err |= LAO_ERR_READ_SLOT; continue; }
+        memcpy(dense + (size_t)i * slot_bytes, pool + (size_t)slots[i] * slot_bytes, slot_bytes);
+    }
+    return err;
+}
+
+int lao_pool_scatter(unsigned char *pool, size_t slot_bytes, int n_slots, int n,
+                     const int *slots, const unsigned char *dense)
+{
+    int err = 0;
+    for (int i = 0; i < n; ++i) {
+        if (slots[i] < 0 || slots[i] >= n_slots) { err |= LAO_ERR_WRITE_SLOT; continue; }
+        memcpy(pool + (size_t)slots[i] * slot_bytes, dense + (size_t)i * slot_bytes, slot_bytes);
+    }
+    return err;
+}
+
+int lao_pool_zero(unsigned char *pool, size_t slot_bytes, int n_slots, int n, const int *slots)
+{
+    int err = 0;
+    for (int i = 0; i < n; ++i) {
+        if (slots[i] < 0 || slots[i] >= n_slots) { err |= LAO_ERR_WRITE_SLOT; continue; }
+        memset(pool + (size_t)slots[i] * slot_bytes, 0, slot_bytes);
+    }
+    return err;
+}
+
+/* ---- threads -------------------------------------------------------------------- */
+
+int lao_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void lao_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

@@ -1,0 +1,205 @@
+"""ctypes binding of the CPU oracle.  TEST INFRASTRUCTURE ONLY.
+
+Only tests/, the smoke check and the benchmark's CPU-baseline leg may import this.
+Arrays are numpy float64 (values already rounded to their storage / io type by the
+caller, which is exact in float64) and int32 slot / cu_seqlens arrays.  What each
+function computes, and which passage of the pages it follows, is in la_oracle.c.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+RULES = {"linear": 0, "gated": 1, "delta": 2, "gated_delta": 3}
+DTYPES = {"f64": 0, "f32": 1, "bf16": 2}
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        _lib = ctypes.CDLL(path)
+        d, i, p = ctypes.c_double, ctypes.c_int, ctypes.c_void_p
+        sz = ctypes.c_size_t
+        _lib.lao_round_bf16.argtypes = [d]
+        _lib.lao_round_bf16.restype = d
+        _lib.lao_round_to.argtypes = [d, i]
+        _lib.lao_round_to.restype = d
+        _lib.lao_step.argtypes = [i, i, i, i, i, p, i, p, i, i, p, p, i, p, p, p, i, p, p, d, p]
+        _lib.lao_step.restype = i
+        _lib.lao_readout_rearranged.argtypes = [i, i, i, i, i, p, i, p, p, p, p, p, d, p]
+        _lib.lao_readout_rearranged.restype = None
+        _lib.lao_scan.argtypes = [i, i, i, i, i, p, i, p, p, i, i, p, i, p, i, p, p, p, i, p, p, d, p]
+        _lib.lao_scan.restype = i
+        _lib.lao_pool_copy.argtypes = [p, sz, i, i, p, p]
+        _lib.lao_pool_gather.argtypes = [p, sz, i, i, p, p]
+        _lib.lao_pool_scatter.argtypes = [p, sz, i, i, p, p]
+        _lib.lao_pool_zero.argtypes = [p, sz, i, i, p]
+        for f in (_lib.lao_pool_copy, _lib.lao_pool_gather, _lib.lao_pool_scatter, _lib.lao_pool_zero):
+            f.restype = i
+        _lib.lao_num_threads.restype = i
+        _lib.lao_set_threads.argtypes = [i]
+    return _lib
+
+
+def use_library(path):
+    """Load the oracle from another shared object (used by the tests that plant a
+    mistake in a copy of the oracle and check the pins catch it).  Returns the previous
+    handle; pass it to restore_library() to switch back."""
+    global _lib
+    prev = lib()
+    _lib = None
+    saved = _build.LIB
+    _build.LIB = path
+    try:
+        _build.build = (lambda force=False, _p=path: _p)  # type: ignore[assignment]
+        lib()
+    finally:
+        _build.LIB = saved
+        _build.build = _BUILD
+    return prev
+
+
+def restore_library(handle):
+    global _lib
+    _lib = handle
+
+
+_BUILD = _build.build
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _i32(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.int32)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def round_bf16(x):
+    """Round each element of a float64 array to the nearest bfloat16 (ties to even)."""
+    f = lib().lao_round_bf16
+    x = _f64(x)
+    return np.array([f(float(e)) for e in x.ravel()], dtype=np.float64).reshape(x.shape)
+
+
+def round_to(x, dtype):
+    f = lib().lao_round_to
+    x = _f64(x)
+    code = DTYPES[dtype]
+    return np.array([f(float(e), code) for e in x.ravel()], dtype=np.float64).reshape(x.shape)
+
+
+def step(rule, n_qk_heads, src_pool, q, k, v, g=None, beta=None, scale=1.0, *,
+         dst_pool=None, dst_dtype="f64", io_dtype="f64", read_slot=None, write_slot=None):
+    """One decode step.  src_pool [n_src, H_v, d_k, d_v]; dst_pool (updated in place and
+    returned; defaults to a copy of src_pool).  Returns (dst_pool, o, err_bits)."""
+    src = _f64(src_pool)
+    dst = src.copy() if dst_pool is None else dst_pool
+    assert dst.dtype == np.float64 and dst.flags.c_contiguous
+    n_src, hv, dk, dv = src.shape
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B = q.shape[0]
+    g = None if g is None else _f64(g)
+    beta = None if beta is None else _f64(beta)
+    rs, ws = _i32(read_slot), _i32(write_slot)
+    o = np.zeros((B, hv, dv), dtype=np.float64)
+    err = lib().lao_step(RULES[rule], n_qk_heads, hv, dk, dv, _ptr(src), n_src,
+                         _ptr(dst), dst.shape[0], DTYPES[dst_dtype], _ptr(rs), _ptr(ws), B,
+                         _ptr(q), _ptr(k), _ptr(v), DTYPES[io_dtype], _ptr(g), _ptr(beta),
+                         float(scale), _ptr(o))
+    return dst, o, err
+
+
+def readout_rearranged(rule, n_qk_heads, state, q, k, v, g=None, beta=None, scale=1.0):
+    """o of one decode step in the rearranged form; state [B, H_v, d_k, d_v] (dense)."""
+    S = _f64(state)
+    B, hv, dk, dv = S.shape
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    g = None if g is None else _f64(g)
+    beta = None if beta is None else _f64(beta)
+    o = np.zeros((B, hv, dv), dtype=np.float64)
+    lib().lao_readout_rearranged(RULES[rule], n_qk_heads, hv, dk, dv, _ptr(S), B,
+                                 _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(o))
+    return o
+
+
+def scan(rule, n_qk_heads, cu_seqlens, q, k, v, g=None, beta=None, scale=1.0, *,
+         src_pool=None, read_slot=None, dst_pool=None, dst_dtype="f64", write_slot=None,
+         io_dtype="f64", n_v_heads=None, d_v=None):
+    """Token-serial scan over packed sequences.  Initial state from src_pool[read_slot]
+    (zero when read_slot is None).  Returns (dst_pool, o, err_bits)."""
+    cu = _i32(cu_seqlens)
+    n_seqs = cu.shape[0] - 1
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, _, dk = q.shape
+    hv, dv = v.shape[1], v.shape[2]
+    if dst_pool is None:
+        dst_pool = np.zeros((n_seqs, hv, dk, dv), dtype=np.float64)
+    assert dst_pool.dtype == np.float64 and dst_pool.flags.c_contiguous
+    src = None if src_pool is None else _f64(src_pool)
+    n_src = 0 if src is None else src.shape[0]
+    g = None if g is None else _f64(g)
+    beta = None if beta is None else _f64(beta)
+    o = np.zeros((T, hv, dv), dtype=np.float64)
+    err = lib().lao_scan(RULES[rule], n_qk_heads, hv, dk, dv, _ptr(src), n_src, _ptr(_i32(read_slot)),
+                         _ptr(dst_pool), dst_pool.shape[0], DTYPES[dst_dtype], _ptr(_i32(write_slot)),
+                         n_seqs, _ptr(cu), T, _ptr(q), _ptr(k), _ptr(v), DTYPES[io_dtype],
+                         _ptr(g), _ptr(beta), float(scale), _ptr(o))
+    return dst_pool, o, err
+
+
+def _u8(pool):
+    assert pool.flags.c_contiguous
+    return pool.view(np.uint8).reshape(pool.shape[0], -1)
+
+
+def pool_copy(pool, src_slots, dst_slots):
+    """Bit copy of whole slots, pool is any contiguous numpy array [n_slots, ...]."""
+    b = _u8(pool)
+    s, d = _i32(src_slots), _i32(dst_slots)
+    return lib().lao_pool_copy(_ptr(b), b.shape[1], b.shape[0], s.shape[0], _ptr(s), _ptr(d))
+
+
+def pool_gather(pool, slots):
+    b = _u8(pool)
+    s = _i32(slots)
+    dense = np.zeros((s.shape[0],) + pool.shape[1:], dtype=pool.dtype)
+    err = lib().lao_pool_gather(_ptr(b), b.shape[1], b.shape[0], s.shape[0], _ptr(s), _ptr(_u8(dense)))
+    return dense, err
+
+
+def pool_scatter(pool, slots, dense):
+    b = _u8(pool)
+    s = _i32(slots)
+    dense = np.ascontiguousarray(dense, dtype=pool.dtype)
+    return lib().lao_pool_scatter(_ptr(b), b.shape[1], b.shape[0], s.shape[0], _ptr(s), _ptr(_u8(dense)))
+
+
+def pool_zero(pool, slots):
+    b = _u8(pool)
+    s = _i32(slots)
+    return lib().lao_pool_zero(_ptr(b), b.shape[1], b.shape[0], s.shape[0], _ptr(s))
+
+
+def num_threads():
+    return lib().lao_num_threads()
+
+
+def set_threads(n):
+    lib().lao_set_threads(int(n))
+
+
+__all__ = ["round_bf16", "round_to", "step", "readout_rearranged", "scan", "pool_copy",
+           "pool_gather", "pool_scatter", "pool_zero", "num_threads", "set_threads", "RULES", "DTYPES"]
+
+if os.environ.get("LAO_THREADS"):
+    set_threads(int(os.environ["LAO_THREADS"]))
