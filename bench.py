@@ -1,0 +1,684 @@
+"""Benchmark of the recurrent-state step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode64|decode512|mamba2|prefill32] [--rows all|none]
+
+Prints ONE JSON line.  The headline workload is the batched decode step the metric is
+quoted on (decode64: B=64 requests, 16 q/k heads shared by 32 state heads, 128 x 128
+BF16 state in a 256-slot pool, gated_delta).  One step = one call of la_state_step over
+the batch (slot gather, load, S^T k / S^T q reductions, delta vector, update, readout,
+store: every row of the decode path).  `value` = algorithmic state-update bytes of all
+ranks / device time of one step (max over ranks), in GB/s; `e2e` is the same metric
+measured through the same C-ABI call with the step's inputs copied from pinned host
+memory and its output copied back inside the timed region.
+
+Timing: W untimed warm-up steps, then K steps back to back between CUDA events on the
+launching stream, bracketed by a barrier and a device synchronize.  The decode64 pool
+(256 MiB) is larger than L2 (126 MB): step i uses slot set i mod 4 of four disjoint
+sets of 64 slots, so each step's state was last touched three steps (384 MiB of
+traffic) earlier.  A second figure with an L2 flush (a 256 MiB write) before every step
+is reported beside it.
+
+With --gpus N (launched by torchrun) every rank runs its own replica of the workload
+on its own GPU: the step has no exchange between GPUs (every (request, head) tile is
+independent), so there is no collective on the data path; ranks only meet at the
+barriers and the final max-over-ranks of the elapsed time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "state-update HBM GB/s (% of B200 peak) and decode tokens/s per layer step"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_SM_MHZ = 1965.0
+FP32_LANES_PER_SM = 128
+
+# --------------------------------------------------------------------------------------
+# byte / flop model (algorithmic: what the method must move, no re-reads)
+
+
+def step_bytes_and_flops(*, B, n_qk_heads, n_v_heads, d_k, d_v, state_bytes, io_bytes, rule, state_only=False,
+                         slot_arrays=0):
+    """Bytes and flops of one decode step over B requests.
+
+    Bytes: the state is read and written once per (request, head) tile; q and k once
+    per q/k head; v and o once per state head; g and beta (4 bytes) where the rule uses
+    them; int32 slot ids.  Flops: 6 per state element (S^T k, S^T q and the update, 2
+    each), the count of the "SSM / linear-RNN decode" page."""
+    elems = B * n_v_heads * d_k * d_v
+    state = 2 * elems * state_bytes
+    flops = 6 * elems
+    if state_only:
+        return state, flops
+    qk = 2 * B * n_qk_heads * d_k * io_bytes
+    vo = 2 * B * n_v_heads * d_v * io_bytes
+    gates = B * n_v_heads * 4 * ((rule in ("gated", "gated_delta")) + (rule in ("delta", "gated_delta")))
+    return state + qk + vo + gates + 4 * B * slot_arrays, flops
+
+
+def scan_bytes_and_flops(*, T, n_seqs, n_qk_heads, n_v_heads, d_k, d_v, io_bytes, rule, final_state_bytes,
+                         init_state_bytes=0):
+    """Bytes and flops of one scan: every token's q, k (per q/k head), v, o (per state
+    head), gates; the final state stored once (and read once when initialised)."""
+    per_tok = 2 * n_qk_heads * d_k * io_bytes + 2 * n_v_heads * d_v * io_bytes
+    per_tok += n_v_heads * 4 * ((rule in ("gated", "gated_delta")) + (rule in ("delta", "gated_delta")))
+    state = n_seqs * n_v_heads * d_k * d_v * (final_state_bytes + init_state_bytes)
+    return T * per_tok + state + 4 * (n_seqs + 1), 6 * T * n_v_heads * d_k * d_v
+
+
+# --------------------------------------------------------------------------------------
+# peaks, clocks, traffic evidence
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", FALLBACK_SM_MHZ)),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": FALLBACK_SM_MHZ, "source": "fallback"}
+
+
+def fp32_alu_peak_tflops(sm_count, mhz):
+    """FP32 FMA roofline: SMs x 128 FP32 lanes x 2 flops x clock."""
+    return sm_count * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "gated_deltanet_recurrent_la_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {
+    "step": ["la_step.cuh", "la_device.cuh"],
+    "scan": ["la_scan.cuh", "la_device.cuh"],
+    "pool": ["la_pool.cu"],
+}
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json), or
+    None when there is none or the kernel source changed since it was captured."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
+            rec = json.load(fh).get(f"{kernel}/{workload}")
+    except Exception:
+        return None
+    if not rec or rec.get("source_hash") != kernel_source_hash(KERNEL_SOURCES[kernel]):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML (read only) in a
+    background thread; `window()` keeps the samples taken between mark_start/mark_end."""
+
+    HW_BAD = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+    def __init__(self, device_index, period_s=0.002):
+        self.samples = []
+        self.period = period_s
+        self.ok = False
+        self.t0 = self.t1 = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that, do not guess
+            self.err = str(e)
+        self._stop = threading.Event()
+        self._th = threading.Thread(target=self._run, daemon=True)
+
+    def _reasons(self, bits):
+        nv = self.nv
+        names = {"hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+                 "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+                 "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+                 "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+                 "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+                 "gpu_idle": getattr(nv, "nvmlClocksEventReasonGpuIdle", 0x1)}
+        return [k for k, v in names.items() if bits & v]
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    bits = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, bits))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._th.start()
+
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._th.join(timeout=2)
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "NVML unavailable"}
+        win = [s for s in self.samples if self.t0 is not None and self.t0 <= s[0] <= (self.t1 or s[0])]
+        if not win:  # region shorter than one poll: take the nearest samples
+            win = sorted(self.samples, key=lambda s: abs(s[0] - (self.t0 or 0)))[:3]
+        reasons = set()
+        for _, _, bits in win:
+            reasons.update(self._reasons(bits))
+        return {"sm_mhz": statistics.median([m for _, m, _ in win]) if win else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(win)}
+
+
+# --------------------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; replicas)
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(per_rank_units, max_ms, world):
+    """Whole-job throughput: units processed by all ranks / the slowest rank's time."""
+    return per_rank_units * world / (max_ms * 1e-3)
+
+
+# --------------------------------------------------------------------------------------
+# device workloads
+
+
+def to_dev(t):
+    return None if t is None else t.cuda().contiguous()
+
+
+class DecodeRunner:
+    """Holds one decode workload on the device and launches la_state_step on it, with
+    `n_sets` disjoint slot sets rotated from step to step."""
+
+    def __init__(self, inp, n_sets=1, seed=0):
+        import torch
+        from gated_deltanet_recurrent_la_b200 import lastate as L
+        self.L = L
+        self.inp = inp
+        self.pool_t = to_dev(inp.pool)
+        self.pool = L.Pool(self.pool_t, inp.n_qk_heads)
+        self.q, self.k, self.v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+        self.g, self.beta = to_dev(inp.g), to_dev(inp.beta)
+        B = inp.q.shape[0]
+        self.o = torch.empty(B, inp.n_v_heads, inp.d_v, dtype=inp.io_dtype, device="cuda")
+        self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.sets = []
+        if inp.read_slot is None:
+            self.sets = [(None, None)]
+        else:
+            n_slots = inp.pool.shape[0]
+            if n_sets > 1:
+                assert n_sets * B <= n_slots
+                rest = [s for s in range(n_slots) if s not in set(inp.write_slot.tolist()) | set(inp.read_slot.tolist())]
+                g = torch.Generator().manual_seed(seed + 101)
+                perm = torch.tensor(rest)[torch.randperm(len(rest), generator=g)]
+                self.sets.append((inp.read_slot, inp.write_slot))
+                for i in range(1, n_sets):
+                    s = perm[(i - 1) * B:i * B].to(torch.int32)
+                    self.sets.append((s, s))
+            else:
+                self.sets.append((inp.read_slot, inp.write_slot))
+            self.sets = [(to_dev(r), to_dev(w)) for r, w in self.sets]
+        self.B = B
+
+    def step(self, i=0, stream=None):
+        r, w = self.sets[i % len(self.sets)]
+        st = self.L.la_state_step(self.inp.rule, self.pool, r, self.pool, w, self.q, self.k, self.v, self.g,
+                                  self.beta, self.inp.scale, self.o, self.err, stream=stream)
+        if st != 0:
+            raise self.L.LAError(st)
+
+    def bytes_flops(self):
+        i = self.inp
+        return step_bytes_and_flops(B=self.B, n_qk_heads=i.n_qk_heads, n_v_heads=i.n_v_heads, d_k=i.d_k, d_v=i.d_v,
+                                    state_bytes=i.pool.element_size(), io_bytes=i.q.element_size(), rule=i.rule,
+                                    slot_arrays=0 if i.read_slot is None else 2)
+
+
+class ScanRunner:
+    def __init__(self, inp):
+        import torch
+        from gated_deltanet_recurrent_la_b200 import lastate as L
+        self.L = L
+        self.inp = inp
+        n_seqs = inp.cu_seqlens.numel() - 1
+        self.dst_t = torch.empty(n_seqs, inp.n_v_heads, inp.d_k, inp.d_v, dtype=inp.state_dtype, device="cuda")
+        self.dst = L.Pool(self.dst_t, inp.n_qk_heads)
+        self.src = None if inp.pool is None else L.Pool(to_dev(inp.pool), inp.n_qk_heads)
+        self.read_slot = to_dev(inp.read_slot)
+        self.cu = to_dev(inp.cu_seqlens)
+        lens = (inp.cu_seqlens[1:] - inp.cu_seqlens[:-1]).tolist()
+        order = sorted(range(n_seqs), key=lambda s: -lens[s])  # longest first
+        self.order = torch.tensor(order, dtype=torch.int32, device="cuda")
+        self.q, self.k, self.v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+        self.g, self.beta = to_dev(inp.g), to_dev(inp.beta)
+        self.o = torch.empty(inp.q.shape[0], inp.n_v_heads, inp.d_v, dtype=inp.io_dtype, device="cuda")
+        self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.T = int(inp.q.shape[0])
+        self.n_seqs = n_seqs
+
+    def step(self, i=0, stream=None):
+        st = self.L.la_state_scan(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu, self.q, self.k,
+                                  self.v, self.g, self.beta, self.inp.scale, self.o, self.err,
+                                  seq_order=self.order, stream=stream)
+        if st != 0:
+            raise self.L.LAError(st)
+
+    def bytes_flops(self):
+        i = self.inp
+        return scan_bytes_and_flops(T=self.T, n_seqs=self.n_seqs, n_qk_heads=i.n_qk_heads, n_v_heads=i.n_v_heads,
+                                    d_k=i.d_k, d_v=i.d_v, io_bytes=i.q.element_size(), rule=i.rule,
+                                    final_state_bytes=self.dst_t.element_size(),
+                                    init_state_bytes=0 if i.pool is None else i.pool.element_size())
+
+
+class PoolRunner:
+    """Checkpoint copies: the 64 live slots of the decode64 pool copied to 64 others."""
+
+    def __init__(self, decode: DecodeRunner):
+        import torch
+        self.d = decode
+        r0 = decode.sets[0][1]
+        r1 = decode.sets[1][1] if len(decode.sets) > 1 else decode.sets[0][1]
+        self.src, self.dst = r0, r1
+        self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step(self, i=0, stream=None):
+        L = self.d.L
+        a, b = (self.src, self.dst) if i % 2 == 0 else (self.dst, self.src)
+        st = L.la_state_pool_copy(self.d.pool, a, b, self.err, stream=stream)
+        if st != 0:
+            raise L.LAError(st)
+
+    def bytes_flops(self):
+        return 2 * self.src.numel() * self.d.pool_t[0].numel() * self.d.pool_t.element_size(), 0
+
+
+# --------------------------------------------------------------------------------------
+# timing
+
+
+class L2Flush:
+    def __init__(self):
+        import torch
+        props = torch.cuda.get_device_properties(torch.cuda.current_device())
+        self.buf = torch.empty(max(2 * props.L2_cache_size, 64 << 20), dtype=torch.uint8, device="cuda")
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def time_back_to_back(run, steps, warmup, world, sampler=None):
+    """W warm-up steps, then K steps back to back between two CUDA events on the current
+    stream; barrier + synchronize on both sides.  Returns ms per step (max over ranks)."""
+    import torch
+    for i in range(warmup):
+        run.step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.mark_start()
+    e0.record(s)
+    for i in range(steps):
+        run.step(warmup + i)
+    e1.record(s)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark_end()
+    barrier(world)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return max_over_ranks(ms, world)
+
+
+def time_flushed(run, steps, flush):
+    """Each step timed alone between events after an L2 flush (flush outside the events)."""
+    import torch
+    s = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i, (a, b) in enumerate(evs):
+        flush()
+        a.record(s)
+        run.step(i)
+        b.record(s)
+    torch.cuda.synchronize()
+    return statistics.median([a.elapsed_time(b) for a, b in evs])
+
+
+def time_e2e(run: DecodeRunner, steps, warmup, world):
+    """The decode step through the same C-ABI call with its inputs copied from pinned host
+    memory (q, k, v, g, beta and the slot ids, one packed copy) and o copied back, all
+    inside the timed region.  The state stays resident in the device pool."""
+    import torch
+    inp = run.inp
+    parts = [inp.q, inp.k, inp.v, inp.g, inp.beta]
+    slot_parts = [(r, w) for r, w in run.sets]
+    offs, total = [], 0
+    sizes = [p.numel() * p.element_size() for p in parts] + [run.B * 4, run.B * 4]
+    for sz in sizes:
+        offs.append(total)
+        total += (sz + 255) // 256 * 256
+    hosts = []
+    for r, w in slot_parts:
+        hb = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+        for p, off in zip(parts, offs):
+            hb[off:off + p.numel() * p.element_size()].copy_(p.contiguous().view(-1).view(torch.uint8))
+        if r is not None:
+            hb[offs[5]:offs[5] + run.B * 4].copy_(r.cpu().view(torch.uint8))
+            hb[offs[6]:offs[6] + run.B * 4].copy_(w.cpu().view(torch.uint8))
+        hosts.append(hb)
+    dev = torch.empty(total, dtype=torch.uint8, device="cuda")
+
+    def view(i, dtype, shape):
+        n = 1
+        for s in shape:
+            n *= s
+        return dev[offs[i]:offs[i] + n * torch.empty(0, dtype=dtype).element_size()].view(dtype).view(shape)
+
+    q = view(0, inp.q.dtype, inp.q.shape)
+    k = view(1, inp.k.dtype, inp.k.shape)
+    v = view(2, inp.v.dtype, inp.v.shape)
+    g = view(3, torch.float32, inp.g.shape)
+    beta = view(4, torch.float32, inp.beta.shape)
+    rs = view(5, torch.int32, (run.B,)) if inp.read_slot is not None else None
+    ws = view(6, torch.int32, (run.B,)) if inp.read_slot is not None else None
+    o_host = torch.empty(run.o.shape, dtype=run.o.dtype, pin_memory=True)
+    L = run.L
+
+    def one(i):
+        dev.copy_(hosts[i % len(hosts)], non_blocking=True)
+        st = L.la_state_step(inp.rule, run.pool, rs, run.pool, ws, q, k, v, g, beta, inp.scale, run.o, run.err)
+        if st != 0:
+            raise L.LAError(st)
+        o_host.copy_(run.o, non_blocking=True)
+
+    class R:
+        step = staticmethod(one)
+
+    ms = time_back_to_back(R, steps, warmup, world)
+    return ms, total, o_host.numel() * o_host.element_size()
+
+
+# --------------------------------------------------------------------------------------
+# oracle on the host cores (baseline only)
+
+
+def cpu_baseline_decode(inp, budget_s=10.0):
+    """The CPU oracle as it stands (fp64, OpenMP over tiles) on the decode workload: whole
+    steps repeated until about budget_s of wall time.  Returns (ms per step, threads,
+    sample description)."""
+    import oracle
+    import numpy as np
+    pool = inp.pool.double().numpy()
+    args = [inp.q.double().numpy(), inp.k.double().numpy(), inp.v.double().numpy(),
+            None if inp.g is None else inp.g.double().numpy(), None if inp.beta is None else inp.beta.double().numpy()]
+    rs = None if inp.read_slot is None else inp.read_slot.numpy().astype(np.int32)
+    ws = None if inp.write_slot is None else inp.write_slot.numpy().astype(np.int32)
+    st = "bf16" if inp.state_dtype.itemsize == 2 else "f32"
+    io = "bf16" if inp.io_dtype.itemsize == 2 else "f32"
+    dst = pool.copy()
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while time.perf_counter() < t_end or not times:
+        t0 = time.perf_counter()
+        oracle.step(inp.rule, inp.n_qk_heads, pool, *args, inp.scale, dst_pool=dst, dst_dtype=st, io_dtype=io,
+                    read_slot=rs, write_slot=ws)
+        times.append(time.perf_counter() - t0)
+    return 1e3 * statistics.median(times), oracle.num_threads(), f"{len(times)} whole decode steps of the workload"
+
+
+# --------------------------------------------------------------------------------------
+
+
+def build_runner(name, seed=0):
+    from gated_deltanet_recurrent_la_b200 import workloads as W
+    inp = W.WORKLOADS[name](seed)
+    if inp.kind == "scan":
+        return ScanRunner(inp), inp
+    n_sets = 4 if name == "decode64" else 1
+    return DecodeRunner(inp, n_sets=n_sets, seed=seed), inp
+
+
+def describe(name, inp):
+    d = {"workload": name, "rule": inp.rule, "n_qk_heads": inp.n_qk_heads, "n_v_heads": inp.n_v_heads,
+         "d_k": inp.d_k, "d_v": inp.d_v, "state": str(inp.state_dtype).replace("torch.", ""),
+         "io": str(inp.io_dtype).replace("torch.", "")}
+    if inp.kind == "step":
+        d.update(B=int(inp.q.shape[0]), pool_slots=int(inp.pool.shape[0]),
+                 slot_map="dense" if inp.read_slot is None else
+                 ("checkpoint" if not bool((inp.read_slot == inp.write_slot).all()) else "perm"))
+    else:
+        lens = (inp.cu_seqlens[1:] - inp.cu_seqlens[:-1])
+        d.update(n_seqs=int(lens.numel()), total_tokens=int(inp.cu_seqlens[-1]), min_len=int(lens.min()),
+                 max_len=int(lens.max()), init="slots" if inp.pool is not None else "zero",
+                 final_state=str(inp.state_dtype).replace("torch.", ""))
+    return d
+
+
+def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None):
+    run, inp = build_runner(name)
+    ms = time_back_to_back(run, steps, warmup, world)
+    nbytes, flops = run.bytes_flops()
+    row = {"config": describe(name, inp), "ms_per_step": ms, "gb_s": nbytes / (ms * 1e-3) / 1e9}
+    if inp.kind == "step":
+        row["tokens_per_s"] = run.B / (ms * 1e-3)
+        row["state_steps_per_s"] = run.B * inp.n_v_heads / (ms * 1e-3)
+        row["roofline"] = {"bound": "hbm", "achieved": row["gb_s"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": row["gb_s"] / peaks["hbm_gbs"], "traffic": recorded_traffic("step", name),
+                           "peak_source": peaks["source"]}
+        row["pct_of_spec_8000"] = 100 * row["gb_s"] / SPEC_HBM_GBS
+        if flush is not None:
+            row["ms_per_step_l2_flushed"] = time_flushed(run, max(10, min(steps, 50)), flush)
+    else:
+        alu = fp32_alu_peak_tflops(sm_count, peaks["sm_max_mhz"])
+        tf = flops / (ms * 1e-3) / 1e12
+        row["tokens_per_s"] = run.T / (ms * 1e-3)
+        row["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
+                           "traffic": recorded_traffic("scan", name), "hbm_gb_s": row["gb_s"],
+                           "effective_state_gb_s": run.T * inp.n_v_heads * 2 * inp.d_k * inp.d_v * 4 / (ms * 1e-3) / 1e9,
+                           "peak_note": "SMs x 128 FP32 lanes x 2 x max SM clock"}
+    del run
+    return row
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode64", choices=["decode64", "decode512", "mamba2", "prefill32"])
+    ap.add_argument("--rows", default="all", choices=["all", "none"])
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    a = ap.parse_args()
+    a.warmup = max(a.warmup, 3)
+
+    rank, world, local = dist_setup(a.gpus)
+    if a.impl == "reference":
+        return reference_arm(a, rank, world)
+
+    import torch
+    from gated_deltanet_recurrent_la_b200 import lastate as L
+    L.lib()  # fail loudly if the CUDA library is missing
+    peaks = measured_peaks()
+    sm_count = torch.cuda.get_device_properties(local).multi_processor_count
+    sampler = ClockSampler(local)
+    sampler.start()
+
+    run, inp = build_runner(a.workload)
+    nbytes, flops = run.bytes_flops()
+    ms = time_back_to_back(run, a.steps, a.warmup, world, sampler)
+    sampler.stop()
+    flush = L2Flush()
+    ms_flushed = time_flushed(run, min(a.steps, 50), flush) if inp.kind == "step" else None
+    value = aggregate(nbytes, ms, world) / 1e9
+    per_gpu = nbytes / (ms * 1e-3) / 1e9
+    out = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+           "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+           "data": "synthetic (seeded host generator; no dataset)",
+           "config": dict(describe(a.workload, inp), parallelism=f"replicas x{world}",
+                          l2="inputs larger than L2: 4 disjoint 64-slot sets of the 256 MiB pool rotated step to step"
+                          if a.workload == "decode64" else "inputs larger than L2")}
+    if inp.kind == "step":
+        out["pct_of_peak"] = 100 * per_gpu / peaks["hbm_gbs"]
+        out["pct_of_spec_8000"] = 100 * per_gpu / SPEC_HBM_GBS
+        out["tokens_per_s"] = world * run.B / (ms * 1e-3)
+        out["state_steps_per_s"] = world * run.B * inp.n_v_heads / (ms * 1e-3)
+        out["ms_per_step_l2_flushed"] = ms_flushed
+        out["roofline"] = {"bound": "hbm", "achieved": per_gpu, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": per_gpu / peaks["hbm_gbs"], "traffic": recorded_traffic("step", a.workload),
+                           "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] == "measured"
+                           else "fallback 6650 GB/s", "algorithmic_bytes_per_launch": nbytes, "kernel": "la::step_kernel"}
+    else:
+        alu = fp32_alu_peak_tflops(sm_count, peaks["sm_max_mhz"])
+        tf = flops / (ms * 1e-3) / 1e12
+        out["tokens_per_s"] = world * run.T / (ms * 1e-3)
+        out["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
+                           "traffic": recorded_traffic("scan", a.workload), "kernel": "la::scan_kernel"}
+    out["gpu_launches"] = a.steps
+    out["clocks"] = sampler.summary()
+
+    if inp.kind == "step":
+        e2e_ms, h2d, d2h = time_e2e(run, a.steps, a.warmup, world)
+        out["e2e"] = {"value": aggregate(nbytes, e2e_ms, world) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        out["gpu_launches"] += a.steps
+    del run
+    torch.cuda.empty_cache()
+
+    if a.rows == "all":
+        rows = {}
+        for name in ("decode512", "mamba2", "prefill32"):
+            if name == a.workload:
+                continue
+            k = a.steps if name != "prefill32" else max(3, min(a.steps, 20))
+            rows[name] = measure_row(name, min(k, 500), a.warmup, world, peaks, sm_count, flush)
+            torch.cuda.empty_cache()
+        prun, _ = build_runner("decode64")
+        pool_run = PoolRunner(prun)
+        pms = time_back_to_back(pool_run, min(a.steps, 500), a.warmup, world)
+        pb, _ = pool_run.bytes_flops()
+        rows["pool_copy64"] = {"ms_per_call": pms, "gb_s": pb / (pms * 1e-3) / 1e9,
+                               "roofline": {"bound": "hbm", "achieved": pb / (pms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                                            "unit": "GB/s", "frac": pb / (pms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                            "traffic": recorded_traffic("pool", "decode64")},
+                               "config": "64 slots x 1 MiB copied within the decode64 pool"}
+        del prun, pool_run
+        out["rows"] = rows
+
+    if rank == 0 and world == 1 or rank == 0:
+        if world == 1:
+            cms, cores, sample = cpu_baseline_decode(inp, a.cpu_budget) if inp.kind == "step" else (None, None, None)
+            if cms is not None:
+                out["cpu_baseline"] = {"value": nbytes / (cms * 1e-3) / 1e9, "unit": "GB/s", "cores": cores,
+                                       "kind": "oracle", "sample": sample, "ms_per_step": cms}
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def reference_arm(a, rank, world):
+    """The oracle (CPU, fp64, OpenMP) timed on the host cores on the same workload, as the
+    reference arm.  Under torchrun only rank 0 runs it; the other ranks exit."""
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
+    from gated_deltanet_recurrent_la_b200 import workloads as W
+    inp = W.WORKLOADS[a.workload](0)
+    if inp.kind != "step":
+        print(json.dumps({"impl": "reference", "unavailable": "the reference arm times decode workloads only"}))
+        return 0
+    nbytes, _ = step_bytes_and_flops(B=int(inp.q.shape[0]), n_qk_heads=inp.n_qk_heads, n_v_heads=inp.n_v_heads,
+                                     d_k=inp.d_k, d_v=inp.d_v, state_bytes=inp.pool.element_size(),
+                                     io_bytes=inp.q.element_size(), rule=inp.rule,
+                                     slot_arrays=0 if inp.read_slot is None else 2)
+    budget = max(5.0, min(60.0, 0.5 * (a.steps + a.warmup)))
+    cms, cores, sample = cpu_baseline_decode(inp, min(budget, a.cpu_budget * 3))
+    value = nbytes / (cms * 1e-3) / 1e9
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": a.steps,
+           "warmup": a.warmup, "ms_per_step": cms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f64", "data": "synthetic (seeded host generator; no dataset)",
+           "config": describe(a.workload, inp),
+           "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,313 @@
+// la_api.cu -- the extern "C" entry points of liblastate.so (declared and documented in
+// include/la_state.h): argument validation on the host, then one kernel launch on the
+// caller's stream.  Nothing here allocates, frees or synchronizes.
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <unordered_set>
+#include <utility>
+
+#include <cuda_runtime.h>
+
+#include "la_internal.h"
+#include "la_state.h"
+
+namespace la {
+
+namespace {
+
+thread_local int32_t g_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 128;
+int g_sm_count[kMaxDevices] = {0};
+std::mutex g_mutex;
+std::map<std::pair<const void*, int>, int> g_per_sm;
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+}  // namespace
+
+int device_sm_count() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 0;
+  int n = __atomic_load_n(&g_sm_count[dev], __ATOMIC_ACQUIRE);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    __atomic_store_n(&g_sm_count[dev], n, __ATOMIC_RELEASE);
+  }
+  return n;
+}
+
+int prepare_kernel(const void* func, int threads, int smem_bytes) {
+  const int dev = current_device();
+  if (dev < 0) return 0;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  auto key = std::make_pair(func, dev);
+  auto it = g_per_sm.find(key);
+  if (it != g_per_sm.end()) return it->second;
+  if (smem_bytes > 48 * 1024 &&
+      cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
+    return 0;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, func, threads, smem_bytes) != cudaSuccess) return 0;
+  g_per_sm[key] = n;
+  return n;
+}
+
+}  // namespace la
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int elem_bytes(int32_t dt) { return dt == LA_F32 ? 4 : dt == LA_BF16 ? 2 : 0; }
+
+bool shape_ok(const la_shape& s) {
+  return s.n_qk_heads > 0 && s.n_v_heads > 0 && s.d_k > 0 && s.d_v > 0 && s.n_v_heads % s.n_qk_heads == 0;
+}
+
+bool same_shape(const la_shape& a, const la_shape& b) {
+  return a.n_qk_heads == b.n_qk_heads && a.n_v_heads == b.n_v_heads && a.d_k == b.d_k && a.d_v == b.d_v;
+}
+
+la_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return LA_OK;
+  la::g_last_cuda_error = static_cast<int32_t>(e);
+  return LA_ERR_CUDA;
+}
+
+bool uses_gate(la_rule r) { return r == LA_RULE_GATED || r == LA_RULE_GATED_DELTA; }
+bool uses_beta(la_rule r) { return r == LA_RULE_DELTA || r == LA_RULE_GATED_DELTA; }
+
+la_status check_pool(const la_pool* p) {
+  if (!p || !p->data) return LA_ERR_NULL;
+  if (p->n_slots < 0 || !shape_ok(p->shape)) return LA_ERR_SHAPE;
+  if (!elem_bytes(p->dtype)) return LA_ERR_UNSUPPORTED;
+  if (!aligned(p->data, 16)) return LA_ERR_ALIGN;
+  return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t la_state_bytes(const la_shape* shape, la_dtype dtype) {
+  if (!shape || !shape_ok(*shape) || !elem_bytes(dtype)) return 0;
+  return (size_t)shape->n_v_heads * (size_t)shape->d_k * (size_t)shape->d_v * (size_t)elem_bytes(dtype);
+}
+
+int la_shape_supported(int32_t d_k, int32_t d_v) {
+  return (d_k == 16 && d_v == 16) || (d_k == 64 && d_v == 64) || (d_k == 128 && d_v == 64) ||
+         (d_k == 128 && d_v == 128);
+}
+
+la_status la_state_step(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
+                        const int32_t* write_slot, int32_t B, const void* q, const void* k, const void* v,
+                        la_dtype io, const float* g, const float* beta, float scale, void* o, int32_t* err_word,
+                        void* stream) {
+  if (rule < LA_RULE_LINEAR || rule > LA_RULE_GATED_DELTA) return LA_ERR_UNSUPPORTED;
+  if (!err_word) return LA_ERR_NULL;
+  if (B < 0) return LA_ERR_SHAPE;
+  la_status st = check_pool(src);
+  if (st != LA_OK) return st;
+  if ((st = check_pool(dst)) != LA_OK) return st;
+  if (B == 0) return LA_OK;
+  if (!q || !k || !v || !o) return LA_ERR_NULL;
+  if (uses_gate(rule) && !g) return LA_ERR_NULL;
+  if (uses_beta(rule) && !beta) return LA_ERR_NULL;
+  if (!same_shape(src->shape, dst->shape)) return LA_ERR_SHAPE;
+  if (src->dtype != dst->dtype || !elem_bytes(io)) return LA_ERR_UNSUPPORTED;
+  if (!la_shape_supported(src->shape.d_k, src->shape.d_v)) return LA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, 4) ||
+      !aligned(beta, 4) || !aligned(read_slot, 4) || !aligned(write_slot, 4) || !aligned(err_word, 4))
+    return LA_ERR_ALIGN;
+  if ((!read_slot && B > src->n_slots) || (!write_slot && B > dst->n_slots)) return LA_ERR_SHAPE;
+  if ((int64_t)B * src->shape.n_v_heads > INT32_MAX) return LA_ERR_SHAPE;
+
+  const la_shape& s = src->shape;
+  la::StepLaunchFn fn = (src->dtype == LA_F32) ? la::find_step_f32(rule, s.d_k, s.d_v, io)
+                                               : la::find_step_bf16(rule, s.d_k, s.d_v, io);
+  if (!fn) return LA_ERR_UNSUPPORTED;
+  la::StepParams p;
+  p.src = src->data;
+  p.src_slots = src->n_slots;
+  p.dst = dst->data;
+  p.dst_slots = dst->n_slots;
+  p.read_slot = read_slot;
+  p.write_slot = write_slot;
+  p.B = B;
+  p.n_qk_heads = s.n_qk_heads;
+  p.n_v_heads = s.n_v_heads;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.g = uses_gate(rule) ? g : nullptr;
+  p.beta = uses_beta(rule) ? beta : nullptr;
+  p.scale = scale;
+  p.o = o;
+  p.err = err_word;
+  return cuda_status(fn(p, static_cast<cudaStream_t>(stream)));
+}
+
+la_status la_state_scan(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
+                        const int32_t* write_slot, int32_t n_seqs, const int32_t* cu_seqlens, int32_t total_tokens,
+                        const int32_t* seq_order, const void* q, const void* k, const void* v, la_dtype io,
+                        const float* g, const float* beta, float scale, void* o, int32_t* err_word, void* stream) {
+  if (rule < LA_RULE_LINEAR || rule > LA_RULE_GATED_DELTA) return LA_ERR_UNSUPPORTED;
+  if (!err_word) return LA_ERR_NULL;
+  if (n_seqs < 0 || total_tokens < 0) return LA_ERR_SHAPE;
+  la_status st = check_pool(dst);
+  if (st != LA_OK) return st;
+  if (read_slot) {
+    if ((st = check_pool(src)) != LA_OK) return st;
+    if (!same_shape(src->shape, dst->shape)) return LA_ERR_SHAPE;
+  }
+  if (n_seqs == 0) return LA_OK;
+  if (!cu_seqlens) return LA_ERR_NULL;
+  if (total_tokens > 0) {
+    if (!q || !k || !v || !o) return LA_ERR_NULL;
+    if (uses_gate(rule) && !g) return LA_ERR_NULL;
+    if (uses_beta(rule) && !beta) return LA_ERR_NULL;
+  }
+  if (!elem_bytes(io)) return LA_ERR_UNSUPPORTED;
+  const la_shape& s = dst->shape;
+  if (!la_shape_supported(s.d_k, s.d_v)) return LA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, 4) ||
+      !aligned(beta, 4) || !aligned(read_slot, 4) || !aligned(write_slot, 4) || !aligned(cu_seqlens, 4) ||
+      !aligned(seq_order, 4) || !aligned(err_word, 4))
+    return LA_ERR_ALIGN;
+  if (!write_slot && n_seqs > dst->n_slots) return LA_ERR_SHAPE;
+  if ((int64_t)n_seqs * s.n_v_heads > INT32_MAX) return LA_ERR_SHAPE;
+
+  la::ScanLaunchFn fn = (io == LA_F32) ? la::find_scan_f32io(rule, s.d_k, s.d_v) : la::find_scan_bf16io(rule, s.d_k, s.d_v);
+  if (!fn) return LA_ERR_UNSUPPORTED;
+  la::ScanParams p;
+  p.src = read_slot ? src->data : nullptr;
+  p.src_slots = read_slot ? src->n_slots : 0;
+  p.src_dtype = read_slot ? src->dtype : dst->dtype;
+  p.read_slot = read_slot;
+  p.dst = dst->data;
+  p.dst_slots = dst->n_slots;
+  p.dst_dtype = dst->dtype;
+  p.write_slot = write_slot;
+  p.n_seqs = n_seqs;
+  p.cu_seqlens = cu_seqlens;
+  p.total_tokens = total_tokens;
+  p.seq_order = seq_order;
+  p.n_qk_heads = s.n_qk_heads;
+  p.n_v_heads = s.n_v_heads;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.g = uses_gate(rule) ? g : nullptr;
+  p.beta = uses_beta(rule) ? beta : nullptr;
+  p.scale = scale;
+  p.o = o;
+  p.err = err_word;
+  return cuda_status(fn(p, static_cast<cudaStream_t>(stream)));
+}
+
+static la_status pool_op(const la_pool* pool, int32_t n, const int32_t* src_slots, const int32_t* dst_slots,
+                         const void* src_dense, void* dst_dense, int zero, int32_t* err_word, void* stream) {
+  if (!err_word) return LA_ERR_NULL;
+  if (n < 0) return LA_ERR_SHAPE;
+  la_status st = check_pool(pool);
+  if (st != LA_OK) return st;
+  if (n == 0) return LA_OK;
+  if (!aligned(src_slots, 4) || !aligned(dst_slots, 4) || !aligned(err_word, 4) || !aligned(src_dense, 16) ||
+      !aligned(dst_dense, 16))
+    return LA_ERR_ALIGN;
+  la::PoolCopyParams p;
+  p.slot_bytes = (int64_t)la_state_bytes(&pool->shape, static_cast<la_dtype>(pool->dtype));
+  p.n = n;
+  p.zero = zero;
+  p.err = err_word;
+  if (src_dense) {  // scatter: dense -> pool
+    p.src = src_dense;
+    p.src_index = nullptr;
+    p.src_count = n;
+    p.dst = pool->data;
+    p.dst_index = dst_slots;
+    p.dst_count = pool->n_slots;
+  } else if (dst_dense) {  // gather: pool -> dense
+    p.src = pool->data;
+    p.src_index = src_slots;
+    p.src_count = pool->n_slots;
+    p.dst = dst_dense;
+    p.dst_index = nullptr;
+    p.dst_count = n;
+  } else {  // copy or zero within the pool
+    p.src = pool->data;
+    p.src_index = src_slots;
+    p.src_count = pool->n_slots;
+    p.dst = pool->data;
+    p.dst_index = dst_slots;
+    p.dst_count = pool->n_slots;
+  }
+  return cuda_status(la::launch_pool_copy(p, static_cast<cudaStream_t>(stream)));
+}
+
+la_status la_state_pool_copy(const la_pool* pool, int32_t n, const int32_t* src_slots, const int32_t* dst_slots,
+                             int32_t* err_word, void* stream) {
+  if (n > 0 && (!src_slots || !dst_slots)) return LA_ERR_NULL;
+  return pool_op(pool, n, src_slots, dst_slots, nullptr, nullptr, 0, err_word, stream);
+}
+
+la_status la_state_pool_gather(const la_pool* pool, int32_t n, const int32_t* slots, void* dense, int32_t* err_word,
+                               void* stream) {
+  if (n > 0 && (!slots || !dense)) return LA_ERR_NULL;
+  return pool_op(pool, n, slots, nullptr, nullptr, dense, 0, err_word, stream);
+}
+
+la_status la_state_pool_scatter(const la_pool* pool, int32_t n, const int32_t* slots, const void* dense,
+                                int32_t* err_word, void* stream) {
+  if (n > 0 && (!slots || !dense)) return LA_ERR_NULL;
+  return pool_op(pool, n, nullptr, slots, dense, nullptr, 0, err_word, stream);
+}
+
+la_status la_state_pool_zero(const la_pool* pool, int32_t n, const int32_t* slots, int32_t* err_word, void* stream) {
+  if (n > 0 && !slots) return LA_ERR_NULL;
+  return pool_op(pool, n, nullptr, slots, nullptr, nullptr, 1, err_word, stream);
+}
+
+la_status la_state_check_slots(int32_t B, const int32_t* read_slot_host, const int32_t* write_slot_host,
+                               int32_t n_slots) {
+  if (B < 0 || n_slots < 0) return LA_ERR_SHAPE;
+  std::unordered_set<int32_t> writes;
+  for (int32_t b = 0; b < B; ++b) {
+    const int32_t r = read_slot_host ? read_slot_host[b] : b;
+    const int32_t w = write_slot_host ? write_slot_host[b] : b;
+    if (r < 0 || r >= n_slots || w < 0 || w >= n_slots) return LA_ERR_SHAPE;
+    if (!writes.insert(w).second) return LA_ERR_ALIAS;
+  }
+  for (int32_t b = 0; b < B; ++b) {
+    const int32_t r = read_slot_host ? read_slot_host[b] : b;
+    const int32_t w = write_slot_host ? write_slot_host[b] : b;
+    if (r != w && writes.count(r)) return LA_ERR_ALIAS;  // reads a slot another request overwrites
+  }
+  return LA_OK;
+}
+
+const char* la_status_str(la_status status) {
+  switch (status) {
+    case LA_OK: return "LA_OK";
+    case LA_ERR_NULL: return "LA_ERR_NULL: a required pointer is NULL";
+    case LA_ERR_SHAPE: return "LA_ERR_SHAPE: invalid or inconsistent sizes";
+    case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: shape, dtype or rule not supported";
+    case LA_ERR_ALIGN: return "LA_ERR_ALIGN: pointer alignment";
+    case LA_ERR_ALIAS: return "LA_ERR_ALIAS: slot preconditions violated";
+    case LA_ERR_CUDA: return "LA_ERR_CUDA: the CUDA runtime refused the launch";
+  }
+  return "unknown la_status";
+}
+
+int32_t la_last_cuda_error(void) { return la::g_last_cuda_error; }
+
+int32_t la_abi_version(void) { return LA_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,338 @@
+// la_scan.cuh -- token-serial scan (prefill) over packed variable-length sequences.
+//
+// Same recurrence as the decode step (the "Gated DeltaNet" glossary page, Technical
+// definition, under the ONNX LinearAttention update rules of "Seven Architectures
+// Replacing KV Cache With Bounded Mutable State"), applied token after token with the
+// state held on chip in FP32 for the whole sequence: it is read once at the start and
+// stored once at the end (BF16 storage, FP32 compute, as on the "Recurrent state"
+// glossary page).  The pages give no prefill algorithm beyond "prefill" speed-ups; this
+// is the plain sequential form.
+//
+// Work unit: one (sequence, state head).  Each column of S evolves on its own given
+// the token's k, q, gate and beta, so the unit's d_v columns are spread over warps and
+// lanes with no exchange between columns:
+//   * a CTA of DV/32 warps owns one unit; warp w owns columns [32w, 32w+32);
+//   * lane = 4 * cg + rg owns columns 32w + 4cg + (0..3) and rows [rg*R, rg*R + R) with
+//     R = d_k / 4, i.e. 4 x R = 128 (d_k = 128) FP32 state values in registers;
+//   * per token, one fused pass over the lane's elements applies the previous token's
+//     update  S <- a S + k u^T  and accumulates  p = S^T k,  r = S^T q  for the current
+//     token (the readout rearrangement of the "Gated DeltaNet" page makes r the old
+//     state's product), then two xor-shuffles finish the d_k sums across the 4 lanes;
+//   * q, k (converted to FP32 in a bank-conflict-free padded layout), v, g, beta of 16
+//     upcoming tokens are staged in shared memory with cp.async double buffering;
+//   * units are dealt to persistent CTAs in the order given by seq_order (longest
+//     first balances best) in a boustrophedon pattern.
+#pragma once
+
+#include <cstdint>
+
+#include "la_device.cuh"
+#include "la_internal.h"
+
+namespace la {
+
+template <int DK, int DV, typename IT>
+struct ScanCfg {
+  static constexpr int kLG = 4;            // lanes sharing a column group (split d_k)
+  static constexpr int kC = 4;             // columns per lane
+  static constexpr int kR = DK / kLG;      // rows per lane
+  static constexpr int kWarps = DV >= 32 ? DV / 32 : 1;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kTC = 16;           // tokens per staged chunk
+  static constexpr int kIB = sizeof(IT);
+  static constexpr int kRowStride = kR + 4;        // padded row-block stride (floats)
+  static constexpr int kKP = kLG * kRowStride;     // padded FP32 key / query length
+  static constexpr int kQKVecs = DK * kIB / 16;    // 16-byte pieces per q or k row
+  static constexpr int kVVecs = DV * kIB / 16;
+  // raw (io dtype) staging, double buffered
+  static constexpr int kRawQ = 0;
+  static constexpr int kRawK = kRawQ + kTC * DK * kIB;
+  static constexpr int kRawV = kRawK + kTC * DK * kIB;
+  static constexpr int kRawG = kRawV + kTC * DV * kIB;
+  static constexpr int kRawB = kRawG + kTC * 4;
+  static constexpr int kRawBytes = kRawB + kTC * 4;
+  // converted FP32 keys / queries and k.q, double buffered
+  static constexpr int kCvtK = 0;
+  static constexpr int kCvtQ = kCvtK + kTC * kKP * 4;
+  static constexpr int kCvtKQ = kCvtQ + kTC * kKP * 4;
+  static constexpr int kCvtBytes = kCvtKQ + kTC * 4;
+  static constexpr int kOffCvt = 2 * kRawBytes;
+  static constexpr int kSmem = kOffCvt + 2 * kCvtBytes;
+
+  static_assert(DK % (4 * kLG) == 0, "rows per lane must be a multiple of 4");
+  static_assert(DV % kC == 0 && (DV >= 32 ? DV % 32 == 0 : 32 % DV == 0), "columns must tile the warps");
+  static_assert((DK * kIB) % 16 == 0 && (DV * kIB) % 16 == 0, "16-byte staging");
+  static_assert(kRawBytes % 16 == 0 && kCvtBytes % 16 == 0, "alignment of staging buffers");
+};
+
+template <int RULE, int DK, int DV, typename IT, int MIN_BLOCKS>
+__global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) scan_kernel(const ScanParams p) {
+  using C = ScanCfg<DK, DV, IT>;
+  constexpr int R = C::kR;
+  extern __shared__ __align__(128) unsigned char smem[];
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int rg = lane & 3;   // row group
+  const int cg = lane >> 2;  // column group within the warp
+  const int col0 = warp * 32 + cg * C::kC;
+  const bool col_active = col0 < DV;
+  const int H = p.n_v_heads;
+  const int ratio = H / p.n_qk_heads;
+  const int64_t units = (int64_t)p.n_seqs * H;
+  const int64_t G = gridDim.x;
+
+  const IT* qg = static_cast<const IT*>(p.q);
+  const IT* kg = static_cast<const IT*>(p.k);
+  const IT* vg = static_cast<const IT*>(p.v);
+  IT* og = static_cast<IT*>(p.o);
+
+  for (int64_t round = 0; round * G < units; ++round) {
+    const int64_t u = round * G + ((round & 1) ? (G - 1 - blockIdx.x) : blockIdx.x);
+    if (u >= units) continue;
+    const int64_t si = u / H;
+    const int h = (int)(u % H);
+    const int hq = h / ratio;
+    const int seq = p.seq_order ? __ldg(p.seq_order + si) : (int)si;
+    if (seq < 0 || seq >= p.n_seqs) {
+      if (tid == 0) report(p.err, LA_DEVERR_CU_SEQLENS);
+      continue;
+    }
+    const int t0 = __ldg(p.cu_seqlens + seq);
+    const int t1 = __ldg(p.cu_seqlens + seq + 1);
+    if (seq == 0 && h == 0 && t0 != 0 && tid == 0) report(p.err, LA_DEVERR_CU_SEQLENS);
+    if (t0 < 0 || t1 < t0 || t1 > p.total_tokens) {
+      if (tid == 0) report(p.err, LA_DEVERR_CU_SEQLENS);
+      continue;
+    }
+    const int rs = p.read_slot ? __ldg(p.read_slot + seq) : 0;
+    const int ws = p.write_slot ? __ldg(p.write_slot + seq) : seq;
+    const bool rs_ok = !p.read_slot || (rs >= 0 && rs < p.src_slots);
+    const bool ws_ok = ws >= 0 && ws < p.dst_slots;
+    if (!rs_ok || !ws_ok) {
+      if (tid == 0) report(p.err, (rs_ok ? 0u : LA_DEVERR_READ_SLOT) | (ws_ok ? 0u : LA_DEVERR_WRITE_SLOT));
+      continue;
+    }
+
+    // ---- initial state (rows rg*R .. rg*R+R-1, columns col0 .. col0+3)
+    float S[R][C::kC];
+    if (p.read_slot && col_active) {
+      const int64_t base = ((int64_t)rs * H + h) * (DK * DV);
+      if (p.src_dtype == LA_F32) {
+        const float* src = static_cast<const float*>(p.src) + base;
+#pragma unroll
+        for (int m = 0; m < R; ++m) {
+          const float4 x = *reinterpret_cast<const float4*>(src + (rg * R + m) * DV + col0);
+          S[m][0] = x.x; S[m][1] = x.y; S[m][2] = x.z; S[m][3] = x.w;
+        }
+      } else {
+        const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.src) + base;
+#pragma unroll
+        for (int m = 0; m < R; ++m) {
+          const uint2 x = *reinterpret_cast<const uint2*>(src + (rg * R + m) * DV + col0);
+          S[m][0] = bf16_lo(x.x); S[m][1] = bf16_hi(x.x); S[m][2] = bf16_lo(x.y); S[m][3] = bf16_hi(x.y);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int m = 0; m < R; ++m)
+#pragma unroll
+        for (int c = 0; c < C::kC; ++c) S[m][c] = 0.0f;
+    }
+
+    // ---- token loop
+    const int n_tok = t1 - t0;
+    const int n_chunks = (n_tok + C::kTC - 1) / C::kTC;
+    float ap = 1.0f;                 // pending update  S <- ap S + kp up^T
+    float up[C::kC] = {0.f, 0.f, 0.f, 0.f};
+    const float* kp = nullptr;       // pending key (padded FP32 row block), nullptr: none
+
+    auto issue = [&](int ch) {
+      unsigned char* raw = smem + (ch & 1) * C::kRawBytes;
+      const int tok0 = t0 + ch * C::kTC;
+      const int n = (t1 - tok0) < C::kTC ? (t1 - tok0) : C::kTC;
+      for (int idx = tid; idx < n * C::kQKVecs; idx += C::kThreads) {
+        const int tt = idx / C::kQKVecs, pc = idx % C::kQKVecs;
+        const int64_t row = ((int64_t)(tok0 + tt) * p.n_qk_heads + hq) * DK;
+        cp_async_16(raw + C::kRawQ + (tt * DK) * C::kIB + pc * 16,
+                    reinterpret_cast<const unsigned char*>(qg + row) + pc * 16);
+        cp_async_16(raw + C::kRawK + (tt * DK) * C::kIB + pc * 16,
+                    reinterpret_cast<const unsigned char*>(kg + row) + pc * 16);
+      }
+      for (int idx = tid; idx < n * C::kVVecs; idx += C::kThreads) {
+        const int tt = idx / C::kVVecs, pc = idx % C::kVVecs;
+        const int64_t row = ((int64_t)(tok0 + tt) * H + h) * DV;
+        cp_async_16(raw + C::kRawV + (tt * DV) * C::kIB + pc * 16,
+                    reinterpret_cast<const unsigned char*>(vg + row) + pc * 16);
+      }
+      for (int tt = tid; tt < n; tt += C::kThreads) {
+        const int64_t gi = (int64_t)(tok0 + tt) * H + h;
+        if (Rule<RULE>::kUsesGate) cp_async_4(raw + C::kRawG + tt * 4, p.g + gi);
+        if (Rule<RULE>::kUsesBeta) cp_async_4(raw + C::kRawB + tt * 4, p.beta + gi);
+      }
+      cp_async_commit();
+    };
+
+    if (n_chunks > 0) issue(0);
+    for (int ch = 0; ch < n_chunks; ++ch) {
+      const int buf = ch & 1;
+      if (ch + 1 < n_chunks) {
+        issue(ch + 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();
+
+      const unsigned char* raw = smem + buf * C::kRawBytes;
+      unsigned char* cvt = smem + C::kOffCvt + buf * C::kCvtBytes;
+      float* kf = reinterpret_cast<float*>(cvt + C::kCvtK);
+      float* qf = reinterpret_cast<float*>(cvt + C::kCvtQ);
+      float* kqs = reinterpret_cast<float*>(cvt + C::kCvtKQ);
+      const IT* kraw = reinterpret_cast<const IT*>(raw + C::kRawK);
+      const IT* qraw = reinterpret_cast<const IT*>(raw + C::kRawQ);
+      const int tok0 = t0 + ch * C::kTC;
+      const int n = (t1 - tok0) < C::kTC ? (t1 - tok0) : C::kTC;
+
+      // convert keys / queries to padded FP32, and k.q per token
+      for (int idx = tid; idx < n * DK; idx += C::kThreads) {
+        const int tt = idx / DK, i = idx % DK;
+        const int pi = tt * C::kKP + (i / R) * C::kRowStride + (i % R);
+        kf[pi] = io_load(kraw + idx);
+        qf[pi] = io_load(qraw + idx);
+      }
+      for (int tt = warp; tt < n; tt += C::kWarps) {
+        float d = 0.0f;
+        for (int i = lane; i < DK; i += 32) d = fmaf(io_load(kraw + tt * DK + i), io_load(qraw + tt * DK + i), d);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+        if (lane == 0) kqs[tt] = d;
+      }
+      __syncthreads();
+
+      const IT* vraw = reinterpret_cast<const IT*>(raw + C::kRawV);
+      const float* graw = reinterpret_cast<const float*>(raw + C::kRawG);
+      const float* braw = reinterpret_cast<const float*>(raw + C::kRawB);
+      for (int tt = 0; tt < n; ++tt) {
+        const float* kc = kf + tt * C::kKP + rg * C::kRowStride;
+        const float* qc = qf + tt * C::kKP + rg * C::kRowStride;
+        const float* kpp = kp ? kp : kc;  // no pending update before the first token
+        float pa[C::kC], ra[C::kC];
+#pragma unroll
+        for (int c = 0; c < C::kC; ++c) pa[c] = ra[c] = 0.0f;
+#pragma unroll
+        for (int m4 = 0; m4 < R / 4; ++m4) {
+          const float4 k4p = *reinterpret_cast<const float4*>(kpp + 4 * m4);
+          const float4 k4 = *reinterpret_cast<const float4*>(kc + 4 * m4);
+          const float4 q4 = *reinterpret_cast<const float4*>(qc + 4 * m4);
+          const float kpv[4] = {k4p.x, k4p.y, k4p.z, k4p.w};
+          const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+          const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+          for (int mm = 0; mm < 4; ++mm) {
+#pragma unroll
+            for (int c = 0; c < C::kC; ++c) {
+              float& x = S[4 * m4 + mm][c];
+              x = fmaf(kpv[mm], up[c], ap * x);
+              if (Rule<RULE>::kPredicts) pa[c] = fmaf(x, kv[mm], pa[c]);
+              ra[c] = fmaf(x, qv[mm], ra[c]);
+            }
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < C::kC; ++c) {
+          if (Rule<RULE>::kPredicts) {
+            pa[c] += __shfl_xor_sync(0xffffffffu, pa[c], 1);
+            pa[c] += __shfl_xor_sync(0xffffffffu, pa[c], 2);
+          }
+          ra[c] += __shfl_xor_sync(0xffffffffu, ra[c], 1);
+          ra[c] += __shfl_xor_sync(0xffffffffu, ra[c], 2);
+        }
+        const float gt = Rule<RULE>::kUsesGate ? graw[tt] : 1.0f;
+        const float bt = Rule<RULE>::kUsesBeta ? braw[tt] : 1.0f;
+        float a, bcoef, cdel;
+        Rule<RULE>::coeffs(gt, bt, a, bcoef, cdel);
+        const float kq = kqs[tt];
+        float vv[C::kC] = {0.f, 0.f, 0.f, 0.f};
+        if (col_active) {
+#pragma unroll
+          for (int c = 0; c < C::kC; ++c) vv[c] = io_load(vraw + tt * DV + col0 + c);
+        }
+        float oc[C::kC];
+#pragma unroll
+        for (int c = 0; c < C::kC; ++c) {
+          up[c] = bcoef * (vv[c] - cdel * pa[c]);
+          oc[c] = p.scale * fmaf(a, ra[c], kq * up[c]);
+        }
+        ap = a;
+        kp = kc;
+        if (col_active) {
+          const float mine = rg == 0 ? oc[0] : rg == 1 ? oc[1] : rg == 2 ? oc[2] : oc[3];
+          io_store(og + ((int64_t)(tok0 + tt) * H + h) * DV + col0 + rg, mine);
+        }
+      }
+      __syncthreads();
+    }
+
+    // ---- last pending update, then store the final state
+    if (kp) {
+#pragma unroll
+      for (int m4 = 0; m4 < R / 4; ++m4) {
+        const float4 k4p = *reinterpret_cast<const float4*>(kp + 4 * m4);
+        const float kpv[4] = {k4p.x, k4p.y, k4p.z, k4p.w};
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm)
+#pragma unroll
+          for (int c = 0; c < C::kC; ++c) S[4 * m4 + mm][c] = fmaf(kpv[mm], up[c], ap * S[4 * m4 + mm][c]);
+      }
+    }
+    if (col_active) {
+      const int64_t base = ((int64_t)ws * H + h) * (DK * DV);
+      if (p.dst_dtype == LA_F32) {
+        float* dst = static_cast<float*>(p.dst) + base;
+#pragma unroll
+        for (int m = 0; m < R; ++m)
+          *reinterpret_cast<float4*>(dst + (rg * R + m) * DV + col0) = make_float4(S[m][0], S[m][1], S[m][2], S[m][3]);
+      } else {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.dst) + base;
+#pragma unroll
+        for (int m = 0; m < R; ++m)
+          *reinterpret_cast<uint2*>(dst + (rg * R + m) * DV + col0) =
+              make_uint2(pack_bf16x2(S[m][0], S[m][1]), pack_bf16x2(S[m][2], S[m][3]));
+      }
+    }
+    // the next unit's staging must not overwrite what this unit still reads
+    __syncthreads();
+  }
+}
+
+template <int RULE, int DK, int DV, typename IT>
+cudaError_t launch_scan(const ScanParams& p, cudaStream_t stream) {
+  using C = ScanCfg<DK, DV, IT>;
+  constexpr int kMinBlocks = 2;
+  const void* fn = reinterpret_cast<const void*>(&scan_kernel<RULE, DK, DV, IT, kMinBlocks>);
+  const int per_sm = prepare_kernel(fn, C::kThreads, C::kSmem);
+  if (per_sm <= 0) return cudaErrorInvalidConfiguration;
+  const int64_t units = (int64_t)p.n_seqs * p.n_v_heads;
+  const int64_t cap = (int64_t)device_sm_count() * per_sm;
+  const int grid = (int)(units < cap ? units : cap);
+  scan_kernel<RULE, DK, DV, IT, kMinBlocks><<<grid, C::kThreads, C::kSmem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename IT>
+ScanLaunchFn find_scan_impl(int rule, int dk, int dv) {
+#define LA_SCAN_CASE(R, K, V) \
+  if (rule == R && dk == K && dv == V) return &launch_scan<R, K, V, IT>;
+#define LA_SCAN_SHAPES(R) LA_SCAN_CASE(R, 16, 16) LA_SCAN_CASE(R, 64, 64) LA_SCAN_CASE(R, 128, 64) LA_SCAN_CASE(R, 128, 128)
+  LA_SCAN_SHAPES(LA_RULE_LINEAR)
+  LA_SCAN_SHAPES(LA_RULE_GATED)
+  LA_SCAN_SHAPES(LA_RULE_DELTA)
+  LA_SCAN_SHAPES(LA_RULE_GATED_DELTA)
+#undef LA_SCAN_SHAPES
+#undef LA_SCAN_CASE
+  return nullptr;
+}
+
+}  // namespace la

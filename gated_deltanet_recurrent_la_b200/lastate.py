@@ -1,0 +1,204 @@
+"""Thin Python binding of liblastate.so (C ABI declared in include/la_state.h).
+
+Argument marshalling only: every function takes torch tensors, passes their device
+pointers and sizes to the C entry point of the same name, and returns its la_status.
+All arithmetic happens in the library's CUDA kernels; there is no fallback path.  If
+the shared library is missing, loading raises instead of degrading.
+
+    pool = Pool(tensor, n_qk_heads)          # tensor [n_slots, H_v, d_k, d_v], fp32 / bf16, CUDA
+    st = la_state_step("gated_delta", pool, read_slot, pool, write_slot, q, k, v, g, beta, 1.0, o, err)
+    check(st)                                # raises LAError unless LA_OK
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblastate.so")
+
+RULES = {"linear": 0, "gated": 1, "delta": 2, "gated_delta": 3}
+LA_F32, LA_BF16 = 0, 1
+STATUS = {0: "LA_OK", 1: "LA_ERR_NULL", 2: "LA_ERR_SHAPE", 3: "LA_ERR_UNSUPPORTED", 4: "LA_ERR_ALIGN",
+          5: "LA_ERR_ALIAS", 6: "LA_ERR_CUDA"}
+LA_OK, LA_ERR_NULL, LA_ERR_SHAPE, LA_ERR_UNSUPPORTED, LA_ERR_ALIGN, LA_ERR_ALIAS, LA_ERR_CUDA = range(7)
+DEVERR_READ_SLOT, DEVERR_WRITE_SLOT, DEVERR_CU_SEQLENS, DEVERR_TIMEOUT = 1, 2, 4, 8
+
+EXPORTS = ("la_state_bytes", "la_shape_supported", "la_state_step", "la_state_scan", "la_state_pool_copy",
+           "la_state_pool_gather", "la_state_pool_scatter", "la_state_pool_zero", "la_state_check_slots",
+           "la_status_str", "la_last_cuda_error", "la_abi_version")
+
+
+class LAError(RuntimeError):
+    def __init__(self, status: int):
+        self.status = status
+        msg = lib().la_status_str(status).decode() if status in STATUS else f"status {status}"
+        if status == LA_ERR_CUDA:
+            msg += f" (cudaError {lib().la_last_cuda_error()})"
+        super().__init__(msg)
+
+
+class la_shape(ctypes.Structure):
+    _fields_ = [("n_qk_heads", ctypes.c_int32), ("n_v_heads", ctypes.c_int32), ("d_k", ctypes.c_int32),
+                ("d_v", ctypes.c_int32)]
+
+
+class la_pool(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("n_slots", ctypes.c_int32),
+                ("shape", la_shape)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded liblastate.so.  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m gated_deltanet_recurrent_la_b200.build` (there is no fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+        PP = ctypes.POINTER(la_pool)
+        L.la_state_bytes.argtypes = [ctypes.POINTER(la_shape), I32]
+        L.la_state_bytes.restype = ctypes.c_size_t
+        L.la_shape_supported.argtypes = [I32, I32]
+        L.la_shape_supported.restype = ctypes.c_int
+        L.la_state_step.argtypes = [I32, PP, P, PP, P, I32, P, P, P, I32, P, P, F, P, P, P]
+        L.la_state_step.restype = I32
+        L.la_state_scan.argtypes = [I32, PP, P, PP, P, I32, P, I32, P, P, P, P, I32, P, P, F, P, P, P]
+        L.la_state_scan.restype = I32
+        L.la_state_pool_copy.argtypes = [PP, I32, P, P, P, P]
+        L.la_state_pool_gather.argtypes = [PP, I32, P, P, P, P]
+        L.la_state_pool_scatter.argtypes = [PP, I32, P, P, P, P]
+        L.la_state_pool_zero.argtypes = [PP, I32, P, P, P]
+        for f in (L.la_state_pool_copy, L.la_state_pool_gather, L.la_state_pool_scatter, L.la_state_pool_zero):
+            f.restype = I32
+        L.la_state_check_slots.argtypes = [I32, P, P, I32]
+        L.la_state_check_slots.restype = I32
+        L.la_status_str.argtypes = [I32]
+        L.la_status_str.restype = ctypes.c_char_p
+        L.la_last_cuda_error.restype = I32
+        L.la_abi_version.restype = I32
+        _lib = L
+    return _lib
+
+
+def check(status: int) -> None:
+    if status != LA_OK:
+        raise LAError(status)
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return LA_F32
+    if dt == torch.bfloat16:
+        return LA_BF16
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"expected {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class Pool:
+    """A slot pool: tensor [n_slots, H_v, d_k, d_v] (float32 or bfloat16) plus H_qk."""
+
+    def __init__(self, tensor: torch.Tensor, n_qk_heads: int):
+        if tensor.dim() != 4:
+            raise ValueError("pool tensor must be [n_slots, H_v, d_k, d_v]")
+        self.tensor = tensor
+        n, hv, dk, dv = tensor.shape
+        self.struct = la_pool(_ptr(tensor), dtype_code(tensor.dtype), n,
+                              la_shape(int(n_qk_heads), hv, dk, dv))
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+
+def la_state_bytes(n_qk_heads: int, n_v_heads: int, d_k: int, d_v: int, dtype: torch.dtype) -> int:
+    s = la_shape(n_qk_heads, n_v_heads, d_k, d_v)
+    return lib().la_state_bytes(ctypes.byref(s), dtype_code(dtype))
+
+
+def la_shape_supported(d_k: int, d_v: int) -> bool:
+    return bool(lib().la_shape_supported(d_k, d_v))
+
+
+def la_state_step(rule, src: Pool, read_slot, dst: Pool, write_slot, q, k, v, g, beta, scale, o, err_word,
+                  stream=None) -> int:
+    io = dtype_code(q.dtype)
+    return lib().la_state_step(RULES[rule] if isinstance(rule, str) else int(rule), src.ref,
+                               _ptr(read_slot, torch.int32), dst.ref, _ptr(write_slot, torch.int32),
+                               int(q.shape[0]), _ptr(q), _ptr(k, q.dtype), _ptr(v, q.dtype), io,
+                               _ptr(g, torch.float32), _ptr(beta, torch.float32), float(scale), _ptr(o, q.dtype),
+                               _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_state_scan(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens, q, k, v, g, beta,
+                  scale, o, err_word, seq_order=None, stream=None) -> int:
+    io = dtype_code(q.dtype)
+    return lib().la_state_scan(RULES[rule] if isinstance(rule, str) else int(rule),
+                               None if src is None else src.ref, _ptr(read_slot, torch.int32), dst.ref,
+                               _ptr(write_slot, torch.int32), int(cu_seqlens.numel() - 1),
+                               _ptr(cu_seqlens, torch.int32), int(q.shape[0]), _ptr(seq_order, torch.int32),
+                               _ptr(q), _ptr(k, q.dtype), _ptr(v, q.dtype), io, _ptr(g, torch.float32),
+                               _ptr(beta, torch.float32), float(scale), _ptr(o, q.dtype),
+                               _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_state_pool_copy(pool: Pool, src_slots, dst_slots, err_word, stream=None) -> int:
+    return lib().la_state_pool_copy(pool.ref, int(src_slots.numel()), _ptr(src_slots, torch.int32),
+                                    _ptr(dst_slots, torch.int32), _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_state_pool_gather(pool: Pool, slots, dense, err_word, stream=None) -> int:
+    return lib().la_state_pool_gather(pool.ref, int(slots.numel()), _ptr(slots, torch.int32),
+                                      _ptr(dense, pool.tensor.dtype), _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_state_pool_scatter(pool: Pool, slots, dense, err_word, stream=None) -> int:
+    return lib().la_state_pool_scatter(pool.ref, int(slots.numel()), _ptr(slots, torch.int32),
+                                       _ptr(dense, pool.tensor.dtype), _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_state_pool_zero(pool: Pool, slots, err_word, stream=None) -> int:
+    return lib().la_state_pool_zero(pool.ref, int(slots.numel()), _ptr(slots, torch.int32),
+                                    _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_state_check_slots(read_slot_host, write_slot_host, n_slots: int, B: Optional[int] = None) -> int:
+    """Host-side slot precondition check on CPU int32 tensors (or None = identity)."""
+    def hp(t):
+        if t is None:
+            return None
+        t = t.to(torch.int32).contiguous().cpu()
+        hp.keep.append(t)
+        return ctypes.c_void_p(t.data_ptr())
+    hp.keep = []
+    if B is None:
+        B = int((read_slot_host if read_slot_host is not None else write_slot_host).numel())
+    return lib().la_state_check_slots(int(B), hp(read_slot_host), hp(write_slot_host), int(n_slots))
+
+
+def la_abi_version() -> int:
+    return lib().la_abi_version()

@@ -1,0 +1,126 @@
+"""Helpers of the GPU parity tests: run a workload through the C ABI (liblastate.so) and
+through the CPU oracle on the same host-generated inputs, and compare."""
+import numpy as np
+import torch
+
+import oracle
+from gated_deltanet_recurrent_la_b200 import lastate as L
+
+F32, BF16 = torch.float32, torch.bfloat16
+
+
+def tolerances(state_dtype, io_dtype):
+    """max|err| <= tol * max|ref|: 1e-4 for FP32 state (and FP32 io), 2e-2 where BF16
+    storage or BF16 outputs are involved (the oracle rounds at the same points)."""
+    st = 1e-4 if state_dtype == F32 else 2e-2
+    o = 1e-4 if (state_dtype == F32 and io_dtype == F32) else 2e-2
+    return st, o
+
+
+def dname(dt):
+    return {torch.float32: "f32", torch.bfloat16: "bf16", torch.float64: "f64"}[dt]
+
+
+def assert_close(got, ref, tol, what):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    if ref.size == 0:
+        return
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    err = float(np.max(np.abs(got - ref)))
+    mx = float(np.max(np.abs(ref)))
+    assert err <= tol * max(mx, 1e-30), f"{what}: max|err| {err:.3e} > {tol:g} * max|ref| {mx:.3e}"
+
+
+def np64(t):
+    return None if t is None else t.detach().cpu().double().numpy()
+
+
+def dev(t):
+    return None if t is None else t.cuda().contiguous()
+
+
+def gpu_step(inp, *, pool_dev=None, read_slot=None, write_slot=None, guard=0):
+    """One la_state_step on the device.  Returns (pool after, o, err word) on the host.
+    `guard` > 0 surrounds o with sentinel elements and checks they survive."""
+    pool_t = dev(inp.pool) if pool_dev is None else pool_dev
+    pool = L.Pool(pool_t, inp.n_qk_heads)
+    rs = dev(inp.read_slot if read_slot is None else read_slot)
+    ws = dev(inp.write_slot if write_slot is None else write_slot)
+    B = inp.q.shape[0]
+    n = B * inp.n_v_heads * inp.d_v
+    o_buf = torch.full((n + 2 * guard,), 7.0, dtype=inp.io_dtype, device="cuda")
+    o = o_buf[guard:guard + n].view(B, inp.n_v_heads, inp.d_v)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = L.la_state_step(inp.rule, pool, rs, pool, ws, dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.g),
+                         dev(inp.beta), inp.scale, o, err)
+    L.check(st)
+    torch.cuda.synchronize()
+    if guard:
+        assert torch.all(o_buf[:guard] == 7.0) and torch.all(o_buf[guard + n:] == 7.0), "o guard band overwritten"
+    return pool_t.cpu(), o.cpu(), int(err.item())
+
+
+def oracle_step(inp, pool_host=None, rows=None):
+    """Oracle decode step on the requests `rows` (all by default), in dense mode on the
+    gathered source tiles.  Returns (new states [len(rows), H, dk, dv], o, err)."""
+    pool = inp.pool if pool_host is None else pool_host
+    B = inp.q.shape[0]
+    rows = np.arange(B) if rows is None else np.asarray(rows)
+    rs = np.arange(B) if inp.read_slot is None else inp.read_slot.numpy()
+    src = np64(pool[torch.as_tensor(rs[rows], dtype=torch.long)])
+    sl = torch.as_tensor(rows, dtype=torch.long)
+    new, o, err = oracle.step(inp.rule, inp.n_qk_heads, src, np64(inp.q[sl]), np64(inp.k[sl]), np64(inp.v[sl]),
+                              np64(None if inp.g is None else inp.g[sl]), np64(None if inp.beta is None else inp.beta[sl]),
+                              inp.scale, dst_dtype=dname(inp.state_dtype), io_dtype=dname(inp.io_dtype))
+    return new, o, err
+
+
+def check_step_against_oracle(inp, chunk=64, guard=16):
+    """Full comparison of one decode step: every request's new state and output, plus
+    bit-exact preservation of every slot that is not written."""
+    before = inp.pool.clone()
+    pool_after, o, err = gpu_step(inp, guard=guard)
+    assert err == 0, f"device error bits {err}"
+    B = inp.q.shape[0]
+    ws = np.arange(B) if inp.write_slot is None else inp.write_slot.numpy()
+    tol_s, tol_o = tolerances(inp.state_dtype, inp.io_dtype)
+    for c0 in range(0, B, chunk):
+        rows = np.arange(c0, min(B, c0 + chunk))
+        new, o_ref, e = oracle_step(inp, before, rows)
+        assert e == 0
+        assert_close(np64(pool_after[torch.as_tensor(ws[rows], dtype=torch.long)]), new, tol_s, f"state rows {c0}..")
+        assert_close(np64(o[torch.as_tensor(rows, dtype=torch.long)]), o_ref, tol_o, f"o rows {c0}..")
+    untouched = np.setdiff1d(np.arange(before.shape[0]), ws)
+    ut = torch.as_tensor(untouched, dtype=torch.long)
+    assert torch.equal(pool_after[ut].view(torch.int16) if before.dtype == BF16 else pool_after[ut].view(torch.int32),
+                       before[ut].view(torch.int16) if before.dtype == BF16 else before[ut].view(torch.int32)), \
+        "slots that are not written must stay bit-identical (checkpoints included)"
+    return pool_after, o
+
+
+def gpu_scan(inp, *, dst_dtype=None, seq_order=None, write_slot=None, n_dst=None, src_pool=None):
+    n_seqs = inp.cu_seqlens.numel() - 1
+    dst_dtype = inp.state_dtype if dst_dtype is None else dst_dtype
+    dst_t = torch.full((n_dst or n_seqs, inp.n_v_heads, inp.d_k, inp.d_v), 3.0, dtype=dst_dtype, device="cuda")
+    dst = L.Pool(dst_t, inp.n_qk_heads)
+    src_t = dev(inp.pool if src_pool is None else src_pool)
+    src = None if src_t is None else L.Pool(src_t, inp.n_qk_heads)
+    T = inp.q.shape[0]
+    o = torch.full((T, inp.n_v_heads, inp.d_v), 5.0, dtype=inp.io_dtype, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = L.la_state_scan(inp.rule, src, dev(inp.read_slot), dst, dev(write_slot), dev(inp.cu_seqlens), dev(inp.q),
+                         dev(inp.k), dev(inp.v), dev(inp.g), dev(inp.beta), inp.scale, o, err,
+                         seq_order=dev(seq_order))
+    L.check(st)
+    torch.cuda.synchronize()
+    return dst_t.cpu(), o.cpu(), int(err.item())
+
+
+def oracle_scan(inp, dst_dtype=None):
+    dst_dtype = inp.state_dtype if dst_dtype is None else dst_dtype
+    return oracle.scan(inp.rule, inp.n_qk_heads, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k), np64(inp.v),
+                       np64(inp.g), np64(inp.beta), inp.scale, src_pool=np64(inp.pool),
+                       read_slot=None if inp.read_slot is None else inp.read_slot.numpy(),
+                       dst_dtype=dname(dst_dtype), io_dtype=dname(inp.io_dtype))

@@ -1,0 +1,177 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol include/la_state.h
+declares, its pure host functions return the sizes the pages print, and invalid
+arguments are rejected on the host before anything is launched (no call in this file
+reaches a kernel launch)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from gated_deltanet_recurrent_la_b200 import lastate as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "la_state.h")
+GOLDEN = os.path.join(ROOT, "tests", "golden", "page_sizes.txt")
+
+
+def golden():
+    out = {}
+    for line in open(GOLDEN):
+        line = line.split("#", 1)[0].strip()
+        if line:
+            k, v = line.split()
+            out[k] = int(v)
+    return out
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(L.LIB_PATH):
+        from gated_deltanet_recurrent_la_b200 import build
+        build.build()
+    return L.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(la_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(L.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (la_[a-z_]+)\b", out))
+    missing = [f for f in declared_functions() if f not in exported]
+    assert not missing, missing
+    for f in declared_functions():
+        assert hasattr(lib, f)
+    assert lib.la_abi_version() == 1
+
+
+def test_state_bytes_match_page_figures(lib):
+    G = golden()
+    # 64 heads x 128 x 128 at 2 bytes (BF16 has the page's 2 bytes per value)
+    assert L.la_state_bytes(64, 64, 128, 128, torch.bfloat16) == G["onnx_64heads_128x128_2byte_state_bytes"]
+    # Nemotron-H-8B layer: 128 heads x (N=128) x (head dim 64)
+    nb = L.la_state_bytes(1, 128, 128, 64, torch.bfloat16)
+    assert nb == G["nemotron_layer_state_bytes_bf16"]
+    assert nb // 2 == G["nemotron_layer_state_elements"]
+    assert 48 * nb == G["nemotron_48_layer_state_bytes_bf16"]
+    assert L.la_state_bytes(16, 32, 128, 128, torch.float32) == 2 * L.la_state_bytes(16, 32, 128, 128, torch.bfloat16)
+    s = L.la_shape(16, 33, 128, 128)  # H_v not a multiple of H_qk
+    assert lib.la_state_bytes(ctypes.byref(s), 1) == 0
+    s = L.la_shape(1, 1, 128, 128)
+    assert lib.la_state_bytes(ctypes.byref(s), 7) == 0
+
+
+def test_byte_model_matches_page(lib):
+    from bench import step_bytes_and_flops
+    G = golden()
+    b, f = step_bytes_and_flops(B=1, n_qk_heads=1, n_v_heads=128, d_k=128, d_v=64, state_bytes=2, io_bytes=2,
+                                rule="gated", state_only=True)
+    assert b == G["nemotron_layer_step_state_bytes"]
+    assert f == G["nemotron_layer_step_flops"]
+
+
+def test_supported_shapes(lib):
+    for dk, dv in [(16, 16), (64, 64), (128, 64), (128, 128)]:
+        assert L.la_shape_supported(dk, dv)
+    for dk, dv in [(32, 32), (128, 256), (0, 0), (64, 128)]:
+        assert not L.la_shape_supported(dk, dv)
+
+
+# ---- host-side validation (fake, never dereferenced device addresses) ------------------
+
+A = 0x7f0000000000  # 16-byte aligned fake address
+
+
+def pool(dtype=1, n=8, shape=(2, 4, 128, 128), data=A):
+    return L.la_pool(ctypes.c_void_p(data), dtype, n, L.la_shape(*shape))
+
+
+def step(lib, rule=3, src=None, dst=None, rs=None, ws=None, B=4, q=A, k=A, v=A, io=1, g=A, beta=A, o=A, err=A):
+    src = src or pool()
+    dst = dst or src
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.la_state_step(rule, ctypes.byref(src), P(rs), ctypes.byref(dst), P(ws), B, P(q), P(k), P(v), io, P(g),
+                             P(beta), 1.0, P(o), P(err), None)
+
+
+def test_step_host_errors(lib):
+    assert step(lib, rule=9) == L.LA_ERR_UNSUPPORTED
+    assert step(lib, err=None) == L.LA_ERR_NULL
+    assert step(lib, B=-1) == L.LA_ERR_SHAPE
+    assert step(lib, B=0) == L.LA_OK  # empty batch: no-op, nothing launched
+    assert step(lib, q=None) == L.LA_ERR_NULL
+    assert step(lib, rule=1, g=None) == L.LA_ERR_NULL
+    assert step(lib, rule=2, beta=None) == L.LA_ERR_NULL
+    assert step(lib, rule=3, g=None) == L.LA_ERR_NULL
+    assert step(lib, src=pool(data=0)) == L.LA_ERR_NULL
+    assert step(lib, src=pool(shape=(3, 4, 128, 128))) == L.LA_ERR_SHAPE      # H_v % H_qk != 0
+    assert step(lib, src=pool(), dst=pool(shape=(2, 4, 128, 64))) == L.LA_ERR_SHAPE
+    assert step(lib, src=pool(dtype=0), dst=pool(dtype=1)) == L.LA_ERR_UNSUPPORTED
+    assert step(lib, src=pool(dtype=5)) == L.LA_ERR_UNSUPPORTED
+    assert step(lib, io=3) == L.LA_ERR_UNSUPPORTED
+    assert step(lib, src=pool(shape=(2, 4, 32, 32))) == L.LA_ERR_UNSUPPORTED
+    assert step(lib, q=A + 8) == L.LA_ERR_ALIGN
+    assert step(lib, o=A + 2) == L.LA_ERR_ALIGN
+    assert step(lib, src=pool(data=A + 4)) == L.LA_ERR_ALIGN
+    assert step(lib, g=A + 2) == L.LA_ERR_ALIGN
+    assert step(lib, B=9) == L.LA_ERR_SHAPE  # dense mode: B > n_slots
+
+
+def scan(lib, rule=3, src=None, rs=None, dst=None, ws=None, n=2, cu=A, T=10, order=None, q=A, io=1, g=A, err=A):
+    dst = dst or pool()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.la_state_scan(rule, None if src is None else ctypes.byref(src), P(rs), ctypes.byref(dst), P(ws), n,
+                             P(cu), T, P(order), P(q), P(A), P(A), io, P(g), P(A), 1.0, P(A), P(err), None)
+
+
+def test_scan_host_errors(lib):
+    assert scan(lib, rule=-1) == L.LA_ERR_UNSUPPORTED
+    assert scan(lib, err=None) == L.LA_ERR_NULL
+    assert scan(lib, n=-1) == L.LA_ERR_SHAPE
+    assert scan(lib, T=-1) == L.LA_ERR_SHAPE
+    assert scan(lib, n=0) == L.LA_OK
+    assert scan(lib, cu=None) == L.LA_ERR_NULL
+    assert scan(lib, q=None) == L.LA_ERR_NULL
+    assert scan(lib, rs=A, src=None) == L.LA_ERR_NULL
+    assert scan(lib, rs=A, src=pool(shape=(2, 4, 64, 64))) == L.LA_ERR_SHAPE
+    assert scan(lib, dst=pool(shape=(2, 4, 128, 96))) == L.LA_ERR_UNSUPPORTED
+    assert scan(lib, cu=A + 2) == L.LA_ERR_ALIGN
+    assert scan(lib, order=A + 1) == L.LA_ERR_ALIGN
+    assert scan(lib, n=9) == L.LA_ERR_SHAPE
+
+
+def test_pool_host_errors(lib):
+    p = pool()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    assert lib.la_state_pool_copy(ctypes.byref(p), 2, P(A), None, P(A), None) == L.LA_ERR_NULL
+    assert lib.la_state_pool_copy(ctypes.byref(p), 0, None, None, P(A), None) == L.LA_OK
+    assert lib.la_state_pool_gather(ctypes.byref(p), 2, P(A), P(A + 8), P(A), None) == L.LA_ERR_ALIGN
+    assert lib.la_state_pool_scatter(ctypes.byref(p), -1, P(A), P(A), P(A), None) == L.LA_ERR_SHAPE
+    assert lib.la_state_pool_zero(ctypes.byref(p), 1, P(A), None, None) == L.LA_ERR_NULL
+    bad = pool(dtype=9)
+    assert lib.la_state_pool_zero(ctypes.byref(bad), 1, P(A), P(A), None) == L.LA_ERR_UNSUPPORTED
+
+
+def test_check_slots(lib):
+    t = lambda x: torch.tensor(x, dtype=torch.int32)  # noqa: E731
+    assert L.la_state_check_slots(t([0, 1, 2]), t([0, 1, 2]), 4) == L.LA_OK
+    assert L.la_state_check_slots(t([5, 5, 6]), t([0, 1, 2]), 8) == L.LA_OK          # shared checkpoint reads
+    assert L.la_state_check_slots(t([0, 1]), t([2, 2]), 4) == L.LA_ERR_ALIAS          # duplicate write
+    assert L.la_state_check_slots(t([0, 1]), t([1, 3]), 4) == L.LA_ERR_ALIAS          # reads a slot another writes
+    assert L.la_state_check_slots(t([0, 4]), t([0, 1]), 4) == L.LA_ERR_SHAPE
+    assert L.la_state_check_slots(None, None, 4, B=3) == L.LA_OK
+
+
+def test_status_strings(lib):
+    for code, name in L.STATUS.items():
+        assert lib.la_status_str(code).decode().startswith(name)

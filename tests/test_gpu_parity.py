@@ -1,0 +1,361 @@
+"""GPU parity: the CUDA kernels, called through the C ABI, against the CPU oracle on the
+same seeded inputs (element by element), at small sizes spanning several tiles with
+ragged tails and at the full sizes of the named workloads.
+
+Tolerances (max|err| <= tol * max|ref|, outputs and states checked separately): 1e-4
+with FP32 state and io, 2e-2 where BF16 storage or BF16 io is involved; the oracle
+rounds at the same points (state after each decode step, at the end of a scan; o to
+the io type).  Slot operations and invariants are checked bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_deltanet_recurrent_la_b200 import lastate as L
+from gated_deltanet_recurrent_la_b200 import workloads as W
+from gpu_helpers import (BF16, F32, assert_close, check_step_against_oracle, dev, dname, gpu_scan, gpu_step,
+                         np64, oracle_scan, tolerances)
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(16, 16), (64, 64), (128, 64), (128, 128)]
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    L.lib()
+
+
+# ---- the tiny workload: all four rules, as 64 decode steps and as one scan ------------
+
+@pytest.mark.parametrize("rule", W.RULES)
+def test_tiny_sequential_steps(rule):
+    inp = W.tiny(rule)
+    cu = inp.cu_seqlens.numpy()
+    pool_t = torch.zeros(2, 2, 16, 16, dtype=F32, device="cuda")
+    ref = np.zeros((2, 2, 16, 16))
+    for t in range(64):
+        rows = torch.as_tensor(cu[:-1] + t, dtype=torch.long)
+        step_inp = W.Inputs("step", rule, 2, 2, 16, 16, F32, F32, inp.q[rows], inp.k[rows], inp.v[rows],
+                            inp.g[rows], inp.beta[rows], 1.0, pool_t)
+        after, o, err = gpu_step(step_inp, pool_dev=pool_t, guard=4)
+        assert err == 0
+        ref, o_ref, e = oracle.step(rule, 2, ref, np64(step_inp.q), np64(step_inp.k), np64(step_inp.v),
+                                    np64(step_inp.g), np64(step_inp.beta), dst_dtype="f32", io_dtype="f32")
+        assert e == 0
+        assert_close(np64(after), ref, 1e-4, f"{rule} state after step {t}")
+        assert_close(np64(o), o_ref, 1e-4, f"{rule} o at step {t}")
+
+
+@pytest.mark.parametrize("rule", W.RULES)
+def test_tiny_scan(rule):
+    inp = W.tiny(rule)
+    S, o, err = gpu_scan(inp)
+    assert err == 0
+    S_ref, o_ref, e = oracle_scan(inp)
+    assert e == 0
+    assert_close(np64(S), S_ref, 1e-4, f"{rule} final state")
+    assert_close(np64(o), o_ref, 1e-4, f"{rule} outputs")
+
+
+# ---- the full-size decode workloads ----------------------------------------------------
+
+def test_decode64_full():
+    check_step_against_oracle(W.decode64())
+
+
+def test_decode512_full_with_checkpoints():
+    inp = W.decode512()
+    rs, ws = inp.read_slot.numpy(), inp.write_slot.numpy()
+    assert (rs != ws).sum() == 256 and len(set(ws)) == 512
+    check_step_against_oracle(inp)  # also proves every checkpoint slot is bit-identical afterwards
+
+
+def test_mamba2_full():
+    check_step_against_oracle(W.mamba2())
+
+
+# ---- the full-size prefill workload, sampled ----------------------------------------------
+
+def test_prefill32_sampled():
+    inp = W.prefill32()
+    S, o, err = gpu_scan(inp)
+    assert err == 0
+    cu = inp.cu_seqlens.numpy()
+    lens = cu[1:] - cu[:-1]
+    order = np.argsort(lens)
+    picks = [(int(order[0]), 0), (int(order[0]), 31), (int(order[16]), 7), (int(order[-1]), 19)]
+    tol_s, tol_o = tolerances(inp.state_dtype, inp.io_dtype)
+    for s, h in picks:
+        t0, t1 = int(cu[s]), int(cu[s + 1])
+        sub = W.Inputs("scan", inp.rule, 1, 1, 128, 128, inp.state_dtype, inp.io_dtype, inp.q[t0:t1, h:h + 1],
+                       inp.k[t0:t1, h:h + 1], inp.v[t0:t1, h:h + 1], inp.g[t0:t1, h:h + 1],
+                       inp.beta[t0:t1, h:h + 1], 1.0, None, None, None, torch.tensor([0, t1 - t0], dtype=torch.int32))
+        S_ref, o_ref, e = oracle_scan(sub)
+        assert e == 0
+        assert_close(np64(S[s, h]), S_ref[0, 0], tol_s, f"seq {s} head {h} final state")
+        assert_close(np64(o[t0:t1, h]), o_ref[:, 0], tol_o, f"seq {s} head {h} outputs")
+    assert torch.isfinite(o.float()).all() and torch.isfinite(S.float()).all()
+
+
+# ---- every rule x tile shape x dtype, small batches -----------------------------------------
+
+@pytest.mark.parametrize("state", [F32, BF16], ids=["f32state", "bf16state"])
+@pytest.mark.parametrize("io", [F32, BF16], ids=["f32io", "bf16io"])
+@pytest.mark.parametrize("dk,dv", SHAPES, ids=[f"{a}x{b}" for a, b in SHAPES])
+@pytest.mark.parametrize("rule", W.RULES)
+def test_step_all_variants(rule, dk, dv, io, state):
+    inp = W.step_inputs(B=5, n_qk_heads=2, n_v_heads=4, d_k=dk, d_v=dv, rule=rule, n_slots=11, state_dtype=state,
+                        io_dtype=io, seed=dk + dv + len(rule), slot_map="perm", scale=0.9)
+    check_step_against_oracle(inp)
+
+
+@pytest.mark.parametrize("io", [F32, BF16], ids=["f32io", "bf16io"])
+@pytest.mark.parametrize("dk,dv", SHAPES, ids=[f"{a}x{b}" for a, b in SHAPES])
+@pytest.mark.parametrize("rule", W.RULES)
+def test_scan_all_variants(rule, dk, dv, io):
+    inp = W.scan_inputs(lengths=[3, 37, 0, 1, 16, 17], n_qk_heads=2, n_v_heads=4, d_k=dk, d_v=dv, rule=rule,
+                        state_dtype=BF16, io_dtype=io, seed=7 + dk, init="slots", init_dtype=F32, scale=1.1)
+    for dst in (F32, BF16):
+        S, o, err = gpu_scan(inp, dst_dtype=dst)
+        assert err == 0
+        S_ref, o_ref, e = oracle_scan(inp, dst_dtype=dst)
+        assert e == 0
+        tol_s, tol_o = tolerances(dst, io)
+        assert_close(np64(S), S_ref, tol_s, f"{rule} {dk}x{dv} final state ({dst})")
+        assert_close(np64(o), o_ref, tol_o, f"{rule} {dk}x{dv} outputs")
+
+
+def test_scan_ragged_multi_tile():
+    inp = W.scan_inputs(lengths=[1, 17, 100, 0, 333, 64, 15, 2], n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128,
+                        state_dtype=BF16, io_dtype=BF16, seed=21)
+    S, o, err = gpu_scan(inp, dst_dtype=F32)
+    assert err == 0
+    S_ref, o_ref, _ = oracle_scan(inp, dst_dtype=F32)
+    assert_close(np64(S), S_ref, 1e-4, "final FP32 state")
+    assert_close(np64(o), o_ref, 2e-2, "BF16 outputs")
+
+
+def test_scan_fp32_init_bf16_final():
+    """The prefill layout with an FP32 initial state read from slots and a BF16 final state."""
+    inp = W.scan_inputs(lengths=[1024, 1500, 1030], n_qk_heads=32, n_v_heads=32, d_k=128, d_v=128, seed=22,
+                        init="slots", init_dtype=F32)
+    S, o, err = gpu_scan(inp)
+    assert err == 0
+    S_ref, o_ref, _ = oracle_scan(inp)
+    assert_close(np64(S), S_ref, 2e-2, "final BF16 state")
+    assert_close(np64(o), o_ref, 2e-2, "outputs")
+
+
+# ---- invariants and structure, bit for bit where the algebra is exact -----------------------
+
+@pytest.mark.parametrize("state", [F32, BF16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("rule", ["delta", "gated_delta"])
+def test_beta0_g1_leaves_state_bit_identical(rule, state):
+    inp = W.step_inputs(B=6, n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128, rule=rule, n_slots=9, state_dtype=state,
+                        io_dtype=BF16, g_mode="one", beta_mode="zero", slot_map="perm", seed=3)
+    before = inp.pool.clone()
+    after, _, err = gpu_step(inp)
+    assert err == 0
+    assert torch.equal(after.view(torch.int16 if state == BF16 else torch.int32),
+                       before.view(torch.int16 if state == BF16 else torch.int32))
+    S, _, err = gpu_scan(W.scan_inputs(lengths=[5, 9], n_qk_heads=1, n_v_heads=2, d_k=64, d_v=64, rule=rule,
+                                       state_dtype=state, io_dtype=F32, g_mode="one", beta_mode="zero", init="slots",
+                                       init_dtype=state, seed=4))
+    assert err == 0
+
+
+def test_delta_unit_key_stores_value():
+    inp = W.step_inputs(B=8, n_qk_heads=4, n_v_heads=4, d_k=128, d_v=128, rule="delta", state_dtype=F32,
+                        io_dtype=F32, beta_mode="one", slot_map="dense", seed=5, pool_std=1.0)
+    inp.q = inp.k.clone()
+    after, o, err = gpu_step(inp)
+    assert err == 0
+    k = np64(inp.k)
+    k = k / np.linalg.norm(k, axis=-1, keepdims=True)
+    stk = np.einsum("bhij,bhi->bhj", np64(after), k)
+    assert_close(stk, np64(inp.v), 1e-5, "S^T k = v")
+    assert_close(np64(o), np64(inp.v), 1e-5, "o = v for q = k")
+
+
+def test_wide_gate_and_beta_ranges():
+    """g in [-1, 1], beta in [0, 2] are not clamped (decode and scan)."""
+    inp = W.step_inputs(B=7, n_qk_heads=1, n_v_heads=3, d_k=64, d_v=64, rule="gated_delta", n_slots=7,
+                        state_dtype=F32, io_dtype=F32, g_mode="uniform_pm1", beta_mode="uniform_0_2", seed=8)
+    check_step_against_oracle(inp)
+    sc = W.scan_inputs(lengths=[40, 7], n_qk_heads=1, n_v_heads=3, d_k=64, d_v=64, state_dtype=F32, io_dtype=F32,
+                       g_mode="uniform_pm1", beta_mode="uniform_0_2", seed=9, init="slots", init_dtype=F32)
+    S, o, err = gpu_scan(sc)
+    S_ref, o_ref, _ = oracle_scan(sc)
+    assert err == 0
+    assert_close(np64(S), S_ref, 1e-4, "wide-range scan state")
+    assert_close(np64(o), o_ref, 1e-4, "wide-range scan outputs")
+
+
+def test_gqa_heads_sharing_qk_agree_bitwise():
+    inp = W.step_inputs(B=3, n_qk_heads=2, n_v_heads=8, d_k=128, d_v=128, slot_map="dense", seed=10)
+    inp.v[:, 1] = inp.v[:, 0]
+    inp.g[:, 1] = inp.g[:, 0]
+    inp.beta[:, 1] = inp.beta[:, 0]
+    inp.pool[:, 1] = inp.pool[:, 0]
+    after, o, err = gpu_step(inp)
+    assert err == 0
+    assert torch.equal(after[:, 0], after[:, 1]) and torch.equal(o[:, 0], o[:, 1])
+    assert not torch.equal(after[:, 4], after[:, 0])
+
+
+def test_scan_equals_sequential_steps_fp32():
+    inp = W.scan_inputs(lengths=[48, 48, 48], n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128, state_dtype=F32,
+                        io_dtype=F32, seed=11)
+    S_scan, o_scan, err = gpu_scan(inp)
+    assert err == 0
+    cu = inp.cu_seqlens.numpy()
+    pool_t = torch.zeros(3, 4, 128, 128, dtype=F32, device="cuda")
+    outs = torch.zeros_like(o_scan)
+    for t in range(48):
+        rows = torch.as_tensor(cu[:-1] + t, dtype=torch.long)
+        si = W.Inputs("step", inp.rule, 2, 4, 128, 128, F32, F32, inp.q[rows], inp.k[rows], inp.v[rows],
+                      inp.g[rows], inp.beta[rows], 1.0, pool_t)
+        _, o, err = gpu_step(si, pool_dev=pool_t)
+        assert err == 0
+        outs[rows] = o
+    assert_close(np64(pool_t.cpu()), np64(S_scan), 1e-4, "scan vs steps, state")
+    assert_close(np64(outs), np64(o_scan), 1e-4, "scan vs steps, outputs")
+
+
+def test_scan_seq_order_is_only_a_schedule():
+    inp = W.scan_inputs(lengths=[30, 3, 0, 70, 12], n_qk_heads=2, n_v_heads=4, d_k=128, d_v=64, seed=12)
+    S0, o0, e0 = gpu_scan(inp)
+    S1, o1, e1 = gpu_scan(inp, seq_order=torch.tensor([3, 0, 4, 1, 2], dtype=torch.int32))
+    assert e0 == e1 == 0
+    assert torch.equal(S0, S1) and torch.equal(o0, o1)
+
+
+def test_dense_past_present_equals_in_place():
+    inp = W.step_inputs(B=4, n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128, slot_map="dense", seed=13)
+    past = dev(inp.pool)
+    present = torch.zeros_like(past)
+    o = torch.empty(4, 4, 128, dtype=BF16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = L.la_state_step("gated_delta", L.Pool(past, 2), None, L.Pool(present, 2), None, dev(inp.q), dev(inp.k),
+                         dev(inp.v), dev(inp.g), dev(inp.beta), 1.0, o, err)
+    L.check(st)
+    in_place, o2, _ = gpu_step(inp)
+    torch.cuda.synchronize()
+    assert torch.equal(past.cpu(), inp.pool), "past_state must not change"
+    assert torch.equal(present.cpu(), in_place) and torch.equal(o.cpu(), o2)
+
+
+def test_scan_write_slots_and_checkpoint_survives():
+    inp = W.scan_inputs(lengths=[20, 5], n_qk_heads=1, n_v_heads=2, d_k=128, d_v=128, seed=14, init="slots",
+                        init_dtype=BF16)
+    ws = torch.tensor([3, 0], dtype=torch.int32)
+    src = inp.pool.clone()  # slots 0, 1 hold the initial states (read_slot is a permutation of them)
+    S, o, err = gpu_scan(inp, write_slot=ws, n_dst=4)
+    assert err == 0
+    S_ref, o_ref, _ = oracle_scan(inp)
+    assert_close(np64(S[ws.long()]), S_ref, 2e-2, "final states at the write slots")
+    assert torch.equal(S[1], torch.full_like(S[1], 3.0)) and torch.equal(S[2], torch.full_like(S[2], 3.0))
+    assert torch.equal(inp.pool, src)
+
+
+# ---- device-side error reporting (never a trap) -------------------------------------------
+
+def test_step_bad_slots_are_skipped_and_reported():
+    inp = W.step_inputs(B=6, n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128, n_slots=10, slot_map="perm", seed=15)
+    good_ws = inp.write_slot.clone()
+    inp.read_slot[1] = 10       # out of range
+    inp.write_slot[4] = -1      # out of range
+    before = inp.pool.clone()
+    after, o, err = gpu_step(inp)
+    assert err == (L.DEVERR_READ_SLOT | L.DEVERR_WRITE_SLOT)
+    assert torch.all(o[1] == 7.0) and torch.all(o[4] == 7.0), "skipped requests leave o untouched"
+    assert torch.equal(after[good_ws[1].long()], before[good_ws[1].long()])
+    for b in (0, 2, 3, 5):
+        sl = torch.tensor([b])
+        one = W.Inputs("step", inp.rule, 2, 4, 128, 128, BF16, BF16, inp.q[sl], inp.k[sl], inp.v[sl], inp.g[sl],
+                       inp.beta[sl], 1.0, before, inp.read_slot[sl], inp.write_slot[sl])
+        new, o_ref, _ = oracle.step(one.rule, 2, np64(before[inp.read_slot[sl].long()]), np64(one.q), np64(one.k),
+                                    np64(one.v), np64(one.g), np64(one.beta), dst_dtype="bf16", io_dtype="bf16")
+        assert_close(np64(after[inp.write_slot[b].long()]), new[0], 2e-2, f"request {b}")
+        assert_close(np64(o[b]), o_ref[0], 2e-2, f"request {b} o")
+
+
+def test_scan_bad_cu_seqlens_and_order_reported():
+    inp = W.scan_inputs(lengths=[4, 6], n_qk_heads=1, n_v_heads=2, d_k=64, d_v=64, seed=16)
+    bad = inp.cu_seqlens.clone()
+    bad[1] = 11  # beyond total_tokens
+    inp2 = W.Inputs(**{**inp.__dict__, "cu_seqlens": bad})
+    _, _, err = gpu_scan(inp2)
+    assert err & L.DEVERR_CU_SEQLENS
+    _, _, err = gpu_scan(inp, seq_order=torch.tensor([0, 5], dtype=torch.int32))
+    assert err == L.DEVERR_CU_SEQLENS
+
+
+def test_empty_calls_are_noops():
+    pool_t = torch.zeros(2, 2, 64, 64, dtype=BF16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    e = torch.empty(0, 2, 64, dtype=BF16, device="cuda")
+    st = L.la_state_step("gated_delta", L.Pool(pool_t, 1), None, L.Pool(pool_t, 1), None,
+                         torch.empty(0, 1, 64, dtype=BF16, device="cuda"), torch.empty(0, 1, 64, dtype=BF16, device="cuda"),
+                         e, torch.empty(0, 2, device="cuda"), torch.empty(0, 2, device="cuda"), 1.0, e, err)
+    assert st == L.LA_OK
+    st = L.la_state_scan("gated_delta", None, None, L.Pool(pool_t, 1), None, torch.zeros(1, dtype=torch.int32, device="cuda"),
+                         torch.empty(0, 1, 64, dtype=BF16, device="cuda"), torch.empty(0, 1, 64, dtype=BF16, device="cuda"),
+                         e, torch.empty(0, 2, device="cuda"), torch.empty(0, 2, device="cuda"), 1.0, e, err)
+    assert st == L.LA_OK
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and not pool_t.any()
+
+
+# ---- slot pool operations, bit for bit ---------------------------------------------------
+
+@pytest.mark.parametrize("dtype", [F32, BF16], ids=["f32", "bf16"])
+def test_pool_ops_bit_exact(dtype):
+    g = torch.Generator().manual_seed(17)
+    host = torch.randn(12, 4, 128, 64, generator=g).to(dtype)
+    ints = torch.int16 if dtype == BF16 else torch.int32
+    pool_t = host.cuda()
+    pool = L.Pool(pool_t, 2)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    slots = torch.tensor([7, 2, 2, 11], dtype=torch.int32)
+    dense = torch.empty(4, 4, 128, 64, dtype=dtype, device="cuda")
+    L.check(L.la_state_pool_gather(pool, dev(slots), dense, err))
+    ref, e = oracle.pool_gather(host.view(ints).numpy(), slots.numpy())
+    assert e == 0 and np.array_equal(dense.cpu().view(ints).numpy(), ref)
+    new = torch.randn(2, 4, 128, 64, generator=g).to(dtype)
+    L.check(L.la_state_pool_scatter(pool, dev(torch.tensor([4, 9], dtype=torch.int32)), new.cuda(), err))
+    L.check(L.la_state_pool_copy(pool, dev(torch.tensor([1, 3], dtype=torch.int32)),
+                                 dev(torch.tensor([5, 0], dtype=torch.int32)), err))
+    L.check(L.la_state_pool_zero(pool, dev(torch.tensor([6], dtype=torch.int32)), err))
+    ref = host.view(ints).numpy().copy()
+    assert oracle.pool_scatter(ref, np.array([4, 9], dtype=np.int32), new.view(ints).numpy()) == 0
+    assert oracle.pool_copy(ref, np.array([1, 3], dtype=np.int32), np.array([5, 0], dtype=np.int32)) == 0
+    assert oracle.pool_zero(ref, np.array([6], dtype=np.int32)) == 0
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert np.array_equal(pool_t.cpu().view(ints).numpy(), ref)
+    # out-of-range slots: skipped and reported
+    L.check(L.la_state_pool_zero(pool, dev(torch.tensor([12], dtype=torch.int32)), err))
+    L.check(L.la_state_pool_gather(pool, dev(torch.tensor([-3], dtype=torch.int32)), dense[:1], err))
+    torch.cuda.synchronize()
+    assert int(err.item()) == (L.DEVERR_READ_SLOT | L.DEVERR_WRITE_SLOT)
+    assert np.array_equal(pool_t.cpu().view(ints).numpy(), ref)
+
+
+def test_pool_checkpoint_roundtrip_full_size():
+    """The decode64 pool: snapshot 64 live slots into checkpoint slots and back."""
+    inp = W.decode64()
+    pool_t = dev(inp.pool)
+    pool = L.Pool(pool_t, 16)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    live = inp.write_slot
+    others = torch.tensor([s for s in range(256) if s not in set(live.tolist())][:64], dtype=torch.int32)
+    L.check(L.la_state_pool_copy(pool, dev(live), dev(others), err))
+    torch.cuda.synchronize()
+    after = pool_t.cpu()
+    assert torch.equal(after[others.long()].view(torch.int16), inp.pool[live.long()].view(torch.int16))
+    assert torch.equal(after[live.long()].view(torch.int16), inp.pool[live.long()].view(torch.int16))
+    assert int(err.item()) == 0
