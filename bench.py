@@ -337,25 +337,31 @@ class ScanRunner:
 
 
 class PoolRunner:
-    """Checkpoint copies: the 64 live slots of the decode64 pool copied to 64 others."""
+    """Prefix-cache checkpoint copies of 64 slots of 1 MiB (the decode64 slot size) inside
+    a 1024-slot pool (1 GiB, larger than L2): call i copies slot set 2i mod 16 onto set
+    2i+1 mod 16 of 16 disjoint 64-slot sets, so no set is touched twice within 8 calls."""
 
-    def __init__(self, decode: DecodeRunner):
+    def __init__(self, n_sets=16, per_set=64, seed=0):
         import torch
-        self.d = decode
-        r0 = decode.sets[0][1]
-        r1 = decode.sets[1][1] if len(decode.sets) > 1 else decode.sets[0][1]
-        self.src, self.dst = r0, r1
+        from gated_deltanet_recurrent_la_b200 import lastate as L
+        self.L = L
+        g = torch.Generator(device="cuda").manual_seed(seed)
+        self.pool_t = torch.randint(-30000, 30000, (n_sets * per_set, 32, 128, 128), dtype=torch.int16,
+                                    device="cuda", generator=g).view(torch.bfloat16)
+        self.pool = L.Pool(self.pool_t, 16)
+        perm = torch.randperm(n_sets * per_set, generator=torch.Generator().manual_seed(seed)).to(torch.int32)
+        self.sets = [perm[i * per_set:(i + 1) * per_set].cuda() for i in range(n_sets)]
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     def step(self, i=0, stream=None):
-        L = self.d.L
-        a, b = (self.src, self.dst) if i % 2 == 0 else (self.dst, self.src)
-        st = L.la_state_pool_copy(self.d.pool, a, b, self.err, stream=stream)
+        n = len(self.sets)
+        st = self.L.la_state_pool_copy(self.pool, self.sets[(2 * i) % n], self.sets[(2 * i + 1) % n], self.err,
+                                       stream=stream)
         if st != 0:
-            raise L.LAError(st)
+            raise self.L.LAError(st)
 
     def bytes_flops(self):
-        return 2 * self.src.numel() * self.d.pool_t[0].numel() * self.d.pool_t.element_size(), 0
+        return 2 * self.sets[0].numel() * self.pool_t[0].numel() * self.pool_t.element_size(), 0
 
 
 # --------------------------------------------------------------------------------------
@@ -497,9 +503,9 @@ def cpu_baseline_decode(inp, budget_s=10.0):
 # --------------------------------------------------------------------------------------
 
 
-def build_runner(name, seed=0):
+def build_runner(name, seed=0, prefill_seqs=32):
     from gated_deltanet_recurrent_la_b200 import workloads as W
-    inp = W.WORKLOADS[name](seed)
+    inp = W.prefill32(seed, prefill_seqs) if name == "prefill32" else W.WORKLOADS[name](seed)
     if inp.kind == "scan":
         return ScanRunner(inp), inp
     n_sets = 4 if name == "decode64" else 1
@@ -557,6 +563,8 @@ def main():
     ap.add_argument("--workload", default="decode64", choices=["decode64", "decode512", "mamba2", "prefill32"])
     ap.add_argument("--rows", default="all", choices=["all", "none"])
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--prefill-seqs", type=int, default=32,
+                    help="sequences of the prefill workload (fewer only to profile a smaller case)")
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
 
@@ -572,7 +580,7 @@ def main():
     sampler = ClockSampler(local)
     sampler.start()
 
-    run, inp = build_runner(a.workload)
+    run, inp = build_runner(a.workload, prefill_seqs=a.prefill_seqs)
     nbytes, flops = run.bytes_flops()
     ms = time_back_to_back(run, a.steps, a.warmup, world, sampler)
     sampler.stop()
@@ -621,19 +629,19 @@ def main():
             k = a.steps if name != "prefill32" else max(3, min(a.steps, 20))
             rows[name] = measure_row(name, min(k, 500), a.warmup, world, peaks, sm_count, flush)
             torch.cuda.empty_cache()
-        prun, _ = build_runner("decode64")
-        pool_run = PoolRunner(prun)
+        pool_run = PoolRunner()
         pms = time_back_to_back(pool_run, min(a.steps, 500), a.warmup, world)
         pb, _ = pool_run.bytes_flops()
         rows["pool_copy64"] = {"ms_per_call": pms, "gb_s": pb / (pms * 1e-3) / 1e9,
                                "roofline": {"bound": "hbm", "achieved": pb / (pms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
                                             "unit": "GB/s", "frac": pb / (pms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                                            "traffic": recorded_traffic("pool", "decode64")},
-                               "config": "64 slots x 1 MiB copied within the decode64 pool"}
-        del prun, pool_run
+                                            "traffic": recorded_traffic("pool", "copy64")},
+                               "config": "64 slots x 1 MiB (32 heads x 128 x 128 BF16) copied to 64 others in a "
+                                         "1024-slot pool; 16 disjoint slot sets rotated"}
+        del pool_run
         out["rows"] = rows
 
-    if rank == 0 and world == 1 or rank == 0:
+    if rank == 0:
         if world == 1:
             cms, cores, sample = cpu_baseline_decode(inp, a.cpu_budget) if inp.kind == "step" else (None, None, None)
             if cms is not None:
