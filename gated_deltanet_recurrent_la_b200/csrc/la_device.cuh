@@ -128,6 +128,14 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ---- programmatic dependent launch ---------------------------------------------------
+
+// Blocks until the preceding kernel on the stream has completed and its memory is
+// visible (a no-op when the launch did not allow programmatic overlap).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel on the stream be scheduled (it still waits in griddep_wait).
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // ---- named barriers among a subset of warps ---------------------------------------
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
@@ -208,6 +216,86 @@ struct StateVec<__nv_bfloat16> {
                       pack_bf16x2(x[6], x[7]));
   }
 };
+
+// N consecutive io-type values -> FP32, with the widest aligned vector loads the byte
+// count allows (16 or 8 bytes; scalar otherwise).  `p` must be aligned to that width.
+template <typename IT, int N>
+__device__ __forceinline__ void load_f32(const IT* p, float* out) {
+  constexpr int kBytes = N * (int)sizeof(IT);
+  if constexpr (kBytes % 16 == 0) {
+    constexpr int kPer = 16 / sizeof(IT);
+#pragma unroll
+    for (int i = 0; i < N / kPer; ++i) {
+      const uint4 w = reinterpret_cast<const uint4*>(p)[i];
+      if constexpr (sizeof(IT) == 2) {
+        StateVec<__nv_bfloat16>::unpack(w, out + i * kPer);
+      } else {
+        StateVec<float>::unpack(w, out + i * kPer);
+      }
+    }
+  } else if constexpr (kBytes % 8 == 0) {
+    constexpr int kPer = 8 / sizeof(IT);
+#pragma unroll
+    for (int i = 0; i < N / kPer; ++i) {
+      const uint2 w = reinterpret_cast<const uint2*>(p)[i];
+      if constexpr (sizeof(IT) == 2) {
+        out[i * kPer + 0] = bf16_lo(w.x); out[i * kPer + 1] = bf16_hi(w.x);
+        out[i * kPer + 2] = bf16_lo(w.y); out[i * kPer + 3] = bf16_hi(w.y);
+      } else {
+        out[i * kPer + 0] = __uint_as_float(w.x); out[i * kPer + 1] = __uint_as_float(w.y);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) out[i] = io_load(p + i);
+  }
+}
+
+// N FP32 values -> N consecutive io-type values (BF16 rounded to nearest even).
+template <typename IT, int N>
+__device__ __forceinline__ void store_f32(IT* p, const float* in) {
+  constexpr int kBytes = N * (int)sizeof(IT);
+  if constexpr (kBytes % 16 == 0) {
+    constexpr int kPer = 16 / sizeof(IT);
+#pragma unroll
+    for (int i = 0; i < N / kPer; ++i) {
+      if constexpr (sizeof(IT) == 2) {
+        reinterpret_cast<uint4*>(p)[i] = StateVec<__nv_bfloat16>::pack(in + i * kPer);
+      } else {
+        reinterpret_cast<uint4*>(p)[i] = StateVec<float>::pack(in + i * kPer);
+      }
+    }
+  } else if constexpr (kBytes % 8 == 0 && sizeof(IT) == 2) {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i)
+      reinterpret_cast<uint2*>(p)[i] = make_uint2(pack_bf16x2(in[4 * i], in[4 * i + 1]), pack_bf16x2(in[4 * i + 2], in[4 * i + 3]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) io_store(p + i, in[i]);
+  }
+}
+
+// FP32 pair arithmetic.  sm_100 has packed FFMA2 / FMUL2, but in the register-heavy FMA
+// loops of these kernels it measured slower on B200 than two scalar FFMAs (identical
+// results), so the pairs are computed with scalar instructions unless LA_PACKED_FP32=1.
+#ifndef LA_PACKED_FP32
+#define LA_PACKED_FP32 0
+#endif
+__device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+#if LA_PACKED_FP32
+  return __ffma2_rn(a, b, c);
+#else
+  return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
+#endif
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+#if LA_PACKED_FP32
+  return __fmul2_rn(a, b);
+#else
+  return make_float2(a.x * b.x, a.y * b.y);
+#endif
+}
 
 // Coefficients (a, b, c) of a rule: S <- a S + k u^T, u = b (v - c S^T k).
 template <int RULE>

@@ -6,18 +6,22 @@
 // state held on chip in FP32 for the whole sequence: it is read once at the start and
 // stored once at the end (BF16 storage, FP32 compute, as on the "Recurrent state"
 // glossary page).  The pages give no prefill algorithm beyond "prefill" speed-ups; this
-// is the plain sequential form.
+// is the plain sequential form, bound by FP32 issue rather than by memory.
 //
 // Work unit: one (sequence, state head).  Each column of S evolves on its own given
 // the token's k, q, gate and beta, so the unit's d_v columns are spread over warps and
 // lanes with no exchange between columns:
-//   * a CTA of DV/32 warps owns one unit; warp w owns columns [32w, 32w+32);
-//   * lane = 4 * cg + rg owns columns 32w + 4cg + (0..3) and rows [rg*R, rg*R + R) with
-//     R = d_k / 4, i.e. 4 x R = 128 (d_k = 128) FP32 state values in registers;
+//   * a CTA of d_v / (8 kC) warps owns one unit; lane = 4 cg + rg owns kC columns
+//     (column group cg) and the rows [rg R, rg R + R), R = d_k / 4, in FP32 registers
+//     (kC = 4: 128 values per lane for 128 x 128);
+//   * the state is kept as S = gam * St with a running scalar gam (the product of the
+//     gates since the last fold), so the update costs one FMA per element:
+//     St <- St + k (u / gam)^T.  When gam leaves [2^-40, 2^40] (or reaches 0) it is
+//     folded into St; it is folded once more before the final store;
 //   * per token, one fused pass over the lane's elements applies the previous token's
-//     update  S <- a S + k u^T  and accumulates  p = S^T k,  r = S^T q  for the current
-//     token (the readout rearrangement of the "Gated DeltaNet" page makes r the old
-//     state's product), then two xor-shuffles finish the d_k sums across the 4 lanes;
+//     update and accumulates St^T k and St^T q for the current token (the readout
+//     rearrangement of the "Gated DeltaNet" page makes S^T q the old state's product):
+//     three FMAs per element; two xor-shuffles finish the d_k sums across the 4 lanes;
 //   * q, k (converted to FP32 in a bank-conflict-free padded layout), v, g, beta of 16
 //     upcoming tokens are staged in shared memory with cp.async double buffering;
 //   * units are dealt to persistent CTAs in the order given by seq_order (longest
@@ -29,20 +33,25 @@
 #include "la_device.cuh"
 #include "la_internal.h"
 
+#ifndef LA_SCAN_COLS
+#define LA_SCAN_COLS 4
+#endif
+
 namespace la {
 
 template <int DK, int DV, typename IT>
 struct ScanCfg {
-  static constexpr int kLG = 4;            // lanes sharing a column group (split d_k)
-  static constexpr int kC = 4;             // columns per lane
-  static constexpr int kR = DK / kLG;      // rows per lane
-  static constexpr int kWarps = DV >= 32 ? DV / 32 : 1;
+  static constexpr int kLG = 4;                        // lanes sharing a column group (split d_k)
+  static constexpr int kC = LA_SCAN_COLS;              // columns per lane
+  static constexpr int kWarpCols = (32 / kLG) * kC;    // columns per warp
+  static constexpr int kR = DK / kLG;                  // rows per lane
+  static constexpr int kWarps = DV >= kWarpCols ? DV / kWarpCols : 1;
   static constexpr int kThreads = kWarps * 32;
-  static constexpr int kTC = 16;           // tokens per staged chunk
+  static constexpr int kTC = 16;                       // tokens per staged chunk
   static constexpr int kIB = sizeof(IT);
-  static constexpr int kRowStride = kR + 4;        // padded row-block stride (floats)
-  static constexpr int kKP = kLG * kRowStride;     // padded FP32 key / query length
-  static constexpr int kQKVecs = DK * kIB / 16;    // 16-byte pieces per q or k row
+  static constexpr int kRowStride = kR + 4;            // padded row-block stride (floats)
+  static constexpr int kKP = kLG * kRowStride;         // padded FP32 key / query length
+  static constexpr int kQKVecs = DK * kIB / 16;        // 16-byte pieces per q or k row
   static constexpr int kVVecs = DV * kIB / 16;
   // raw (io dtype) staging, double buffered
   static constexpr int kRawQ = 0;
@@ -59,8 +68,10 @@ struct ScanCfg {
   static constexpr int kOffCvt = 2 * kRawBytes;
   static constexpr int kSmem = kOffCvt + 2 * kCvtBytes;
 
+  static_assert(kC == 2 || kC == 4, "columns per lane");
   static_assert(DK % (4 * kLG) == 0, "rows per lane must be a multiple of 4");
-  static_assert(DV % kC == 0 && (DV >= 32 ? DV % 32 == 0 : 32 % DV == 0), "columns must tile the warps");
+  static_assert(DV % kC == 0 && (DV >= kWarpCols ? DV % kWarpCols == 0 : kWarpCols % DV == 0),
+                "columns must tile the warps");
   static_assert((DK * kIB) % 16 == 0 && (DV * kIB) % 16 == 0, "16-byte staging");
   static_assert(kRawBytes % 16 == 0 && kCvtBytes % 16 == 0, "alignment of staging buffers");
 };
@@ -69,6 +80,7 @@ template <int RULE, int DK, int DV, typename IT, int MIN_BLOCKS>
 __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) scan_kernel(const ScanParams p) {
   using C = ScanCfg<DK, DV, IT>;
   constexpr int R = C::kR;
+  constexpr int KC = C::kC;
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int tid = threadIdx.x;
@@ -76,7 +88,7 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
   const int lane = tid & 31;
   const int rg = lane & 3;   // row group
   const int cg = lane >> 2;  // column group within the warp
-  const int col0 = warp * 32 + cg * C::kC;
+  const int col0 = warp * C::kWarpCols + cg * KC;
   const bool col_active = col0 < DV;
   const int H = p.n_v_heads;
   const int ratio = H / p.n_qk_heads;
@@ -88,6 +100,7 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
   const IT* vg = static_cast<const IT*>(p.v);
   IT* og = static_cast<IT*>(p.o);
 
+#pragma unroll 1
   for (int64_t round = 0; round * G < units; ++round) {
     const int64_t u = round * G + ((round & 1) ? (G - 1 - blockIdx.x) : blockIdx.x);
     if (u >= units) continue;
@@ -115,38 +128,34 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
       continue;
     }
 
-    // ---- initial state (rows rg*R .. rg*R+R-1, columns col0 .. col0+3)
-    float S[R][C::kC];
+    // ---- initial state: rows rg*R .. rg*R+R-1, columns col0 .. col0+KC-1
+    float S[R][KC];
     if (p.read_slot && col_active) {
       const int64_t base = ((int64_t)rs * H + h) * (DK * DV);
       if (p.src_dtype == LA_F32) {
         const float* src = static_cast<const float*>(p.src) + base;
 #pragma unroll
-        for (int m = 0; m < R; ++m) {
-          const float4 x = *reinterpret_cast<const float4*>(src + (rg * R + m) * DV + col0);
-          S[m][0] = x.x; S[m][1] = x.y; S[m][2] = x.z; S[m][3] = x.w;
-        }
+        for (int m = 0; m < R; ++m) load_f32<float, KC>(src + (rg * R + m) * DV + col0, S[m]);
       } else {
         const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.src) + base;
 #pragma unroll
-        for (int m = 0; m < R; ++m) {
-          const uint2 x = *reinterpret_cast<const uint2*>(src + (rg * R + m) * DV + col0);
-          S[m][0] = bf16_lo(x.x); S[m][1] = bf16_hi(x.x); S[m][2] = bf16_lo(x.y); S[m][3] = bf16_hi(x.y);
-        }
+        for (int m = 0; m < R; ++m) load_f32<__nv_bfloat16, KC>(src + (rg * R + m) * DV + col0, S[m]);
       }
     } else {
 #pragma unroll
       for (int m = 0; m < R; ++m)
 #pragma unroll
-        for (int c = 0; c < C::kC; ++c) S[m][c] = 0.0f;
+        for (int c = 0; c < KC; ++c) S[m][c] = 0.0f;
     }
 
     // ---- token loop
     const int n_tok = t1 - t0;
     const int n_chunks = (n_tok + C::kTC - 1) / C::kTC;
-    float ap = 1.0f;                 // pending update  S <- ap S + kp up^T
-    float up[C::kC] = {0.f, 0.f, 0.f, 0.f};
-    const float* kp = nullptr;       // pending key (padded FP32 row block), nullptr: none
+    float gam = 1.0f;       // S = gam * St  (the registers hold St)
+    float up[KC];           // pending update  St <- St + kp up^T
+#pragma unroll
+    for (int c = 0; c < KC; ++c) up[c] = 0.0f;
+    const float* kp = nullptr;  // pending key (padded FP32 row block); nullptr: none
 
     auto issue = [&](int ch) {
       unsigned char* raw = smem + (ch & 1) * C::kRawBytes;
@@ -175,6 +184,7 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
     };
 
     if (n_chunks > 0) issue(0);
+#pragma unroll 1
     for (int ch = 0; ch < n_chunks; ++ch) {
       const int buf = ch & 1;
       if (ch + 1 < n_chunks) {
@@ -214,13 +224,14 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
       const IT* vraw = reinterpret_cast<const IT*>(raw + C::kRawV);
       const float* graw = reinterpret_cast<const float*>(raw + C::kRawG);
       const float* braw = reinterpret_cast<const float*>(raw + C::kRawB);
+#pragma unroll 1
       for (int tt = 0; tt < n; ++tt) {
         const float* kc = kf + tt * C::kKP + rg * C::kRowStride;
         const float* qc = qf + tt * C::kKP + rg * C::kRowStride;
         const float* kpp = kp ? kp : kc;  // no pending update before the first token
-        float pa[C::kC], ra[C::kC];
+        float pa[KC], ra[KC];
 #pragma unroll
-        for (int c = 0; c < C::kC; ++c) pa[c] = ra[c] = 0.0f;
+        for (int c = 0; c < KC; ++c) pa[c] = ra[c] = 0.0f;
 #pragma unroll
         for (int m4 = 0; m4 < R / 4; ++m4) {
           const float4 k4p = *reinterpret_cast<const float4*>(kpp + 4 * m4);
@@ -232,16 +243,16 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
 #pragma unroll
           for (int mm = 0; mm < 4; ++mm) {
 #pragma unroll
-            for (int c = 0; c < C::kC; ++c) {
+            for (int c = 0; c < KC; ++c) {
               float& x = S[4 * m4 + mm][c];
-              x = fmaf(kpv[mm], up[c], ap * x);
+              x = fmaf(kpv[mm], up[c], x);
               if (Rule<RULE>::kPredicts) pa[c] = fmaf(x, kv[mm], pa[c]);
               ra[c] = fmaf(x, qv[mm], ra[c]);
             }
           }
         }
 #pragma unroll
-        for (int c = 0; c < C::kC; ++c) {
+        for (int c = 0; c < KC; ++c) {
           if (Rule<RULE>::kPredicts) {
             pa[c] += __shfl_xor_sync(0xffffffffu, pa[c], 1);
             pa[c] += __shfl_xor_sync(0xffffffffu, pa[c], 2);
@@ -254,28 +265,50 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
         float a, bcoef, cdel;
         Rule<RULE>::coeffs(gt, bt, a, bcoef, cdel);
         const float kq = kqs[tt];
-        float vv[C::kC] = {0.f, 0.f, 0.f, 0.f};
-        if (col_active) {
+        float vv[KC];
 #pragma unroll
-          for (int c = 0; c < C::kC; ++c) vv[c] = io_load(vraw + tt * DV + col0 + c);
-        }
-        float oc[C::kC];
+        for (int c = 0; c < KC; ++c) vv[c] = 0.0f;
+        if (col_active) load_f32<IT, KC>(vraw + tt * DV + col0, vv);
+        // u = b (v - c S^T k),  o = scale (a S^T q + (k.q) u),  with S = gam St
+        float uu[KC], oc[KC];
 #pragma unroll
-        for (int c = 0; c < C::kC; ++c) {
-          up[c] = bcoef * (vv[c] - cdel * pa[c]);
-          oc[c] = p.scale * fmaf(a, ra[c], kq * up[c]);
+        for (int c = 0; c < KC; ++c) {
+          uu[c] = bcoef * (vv[c] - cdel * (gam * pa[c]));
+          oc[c] = p.scale * fmaf(a, gam * ra[c], kq * uu[c]);
         }
-        ap = a;
-        kp = kc;
-        if (col_active) {
-          const float mine = rg == 0 ? oc[0] : rg == 1 ? oc[1] : rg == 2 ? oc[2] : oc[3];
+        if (col_active && rg < KC) {
+          float mine = oc[0];
+#pragma unroll
+          for (int c = 1; c < KC; ++c) mine = (rg == c) ? oc[c] : mine;
           io_store(og + ((int64_t)(tok0 + tt) * H + h) * DV + col0 + rg, mine);
         }
+        // S_t = a S_{t-1} + k u^T:  gam <- a gam,  St <- St + k (u / gam)^T (applied in
+        // the next token's pass).  A gate product outside [2^-40, 2^40] is folded now:
+        // the registers hold St_{t-1}, so St <- (a gam) St and gam <- 1.
+        if (Rule<RULE>::kUsesGate) {
+          const float gnew = a * gam;
+          if (!(fabsf(gnew) >= 0x1p-40f && fabsf(gnew) <= 0x1p40f)) {
+#pragma unroll
+            for (int m = 0; m < R; ++m)
+#pragma unroll
+              for (int c = 0; c < KC; ++c) S[m][c] *= gnew;
+            gam = 1.0f;
+          } else {
+            gam = gnew;
+          }
+          const float inv = __frcp_rn(gam);
+#pragma unroll
+          for (int c = 0; c < KC; ++c) up[c] = uu[c] * inv;
+        } else {
+#pragma unroll
+          for (int c = 0; c < KC; ++c) up[c] = uu[c];
+        }
+        kp = kc;
       }
       __syncthreads();
     }
 
-    // ---- last pending update, then store the final state
+    // ---- last pending update, fold gam, store the final state
     if (kp) {
 #pragma unroll
       for (int m4 = 0; m4 < R / 4; ++m4) {
@@ -284,22 +317,23 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
 #pragma unroll
         for (int mm = 0; mm < 4; ++mm)
 #pragma unroll
-          for (int c = 0; c < C::kC; ++c) S[4 * m4 + mm][c] = fmaf(kpv[mm], up[c], ap * S[4 * m4 + mm][c]);
+          for (int c = 0; c < KC; ++c) S[4 * m4 + mm][c] = fmaf(kpv[mm], up[c], S[4 * m4 + mm][c]);
       }
     }
     if (col_active) {
+#pragma unroll
+      for (int m = 0; m < R; ++m)
+#pragma unroll
+        for (int c = 0; c < KC; ++c) S[m][c] *= gam;
       const int64_t base = ((int64_t)ws * H + h) * (DK * DV);
       if (p.dst_dtype == LA_F32) {
         float* dst = static_cast<float*>(p.dst) + base;
 #pragma unroll
-        for (int m = 0; m < R; ++m)
-          *reinterpret_cast<float4*>(dst + (rg * R + m) * DV + col0) = make_float4(S[m][0], S[m][1], S[m][2], S[m][3]);
+        for (int m = 0; m < R; ++m) store_f32<float, KC>(dst + (rg * R + m) * DV + col0, S[m]);
       } else {
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.dst) + base;
 #pragma unroll
-        for (int m = 0; m < R; ++m)
-          *reinterpret_cast<uint2*>(dst + (rg * R + m) * DV + col0) =
-              make_uint2(pack_bf16x2(S[m][0], S[m][1]), pack_bf16x2(S[m][2], S[m][3]));
+        for (int m = 0; m < R; ++m) store_f32<__nv_bfloat16, KC>(dst + (rg * R + m) * DV + col0, S[m]);
       }
     }
     // the next unit's staging must not overwrite what this unit still reads
@@ -310,7 +344,7 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
 template <int RULE, int DK, int DV, typename IT>
 cudaError_t launch_scan(const ScanParams& p, cudaStream_t stream) {
   using C = ScanCfg<DK, DV, IT>;
-  constexpr int kMinBlocks = 2;
+  constexpr int kMinBlocks = 2;  // two CTAs (units) per SM
   const void* fn = reinterpret_cast<const void*>(&scan_kernel<RULE, DK, DV, IT, kMinBlocks>);
   const int per_sm = prepare_kernel(fn, C::kThreads, C::kSmem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;

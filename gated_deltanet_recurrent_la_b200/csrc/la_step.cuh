@@ -16,13 +16,18 @@
 //    t / H_v, head t % H_v);
 //  * warp specialisation: one producer warp streams each whole d_k x d_v state tile (a
 //    contiguous 8-64 KiB block of the pool) plus q, k, v into a shared-memory stage
-//    with 1-D bulk copies on the TMA engine, signalling an mbarrier; the "asynchronous
-//    state transfers" of the "Gated DeltaNet" page (How to read it), so several tiles
-//    are always in flight per SM;
-//  * eight consumer warps turn a stage into FP32 registers (16-byte vectors, 8 BF16 or
-//    4 FP32 state elements per thread per row), reduce S^T k and S^T q over d_k with
-//    shuffles plus one shared-memory pass, form u and o, release the stage, and store
-//    the new state with coalesced 16-byte stores (BF16 rounding to nearest even).
+//    with 1-D bulk copies on the TMA engine, signalling an mbarrier -- the
+//    "asynchronous state transfers" of the "Gated DeltaNet" page (How to read it) --
+//    so that several tiles are in flight per SM at all times;
+//  * every column of S evolves on its own, so each consumer warp owns a strip of up to
+//    32 columns of a tile for all d_k rows and needs nobody else: lanes split the strip
+//    into 16-byte column chunks x row blocks, hold the strip's 128 state values in FP32
+//    registers, finish S^T k and S^T q with xor-shuffles inside the warp, form u and o,
+//    release the stage on their own, and store the new state with 16-byte stores.
+//    Warps of different tiles run concurrently; there is no CTA-wide barrier.  Four
+//    consumer warps (plus the producer) keep every SM sub-partition at <= 2 warps so a
+//    thread may hold its 128 state values without spilling.
+//  * FP32 arithmetic in packed pairs (sm_100 FFMA2 / FMUL2).
 #pragma once
 
 #include <cstdint>
@@ -45,36 +50,46 @@ struct StepMeta {
   int64_t o_off;    // element offset of o[b, h, 0]
 };
 
+// Consumer warps per CTA and the widest column strip of one warp.  With 4 consumer
+// warps plus the producer no SM sub-partition holds more than 2 warps, so a thread may
+// use up to 255 registers (a strip of 32 x 128 holds 128 FP32 state values per lane).
+#ifndef LA_STEP_CONSUMER_WARPS
+#define LA_STEP_CONSUMER_WARPS 4
+#endif
+#ifndef LA_STEP_STRIP_COLS
+#define LA_STEP_STRIP_COLS 32
+#endif
+// Launch with programmatic stream serialization so that a step's prologue overlaps the
+// tail of the previous kernel on the stream.
+#ifndef LA_STEP_PDL
+#define LA_STEP_PDL 1
+#endif
+
 template <int DK, int DV, typename ST, typename IT>
 struct StepCfg {
   static constexpr int kSB = sizeof(ST);
-  static constexpr int kVec = StateVec<ST>::kElems;  // state elements per 16-byte vector
-  static constexpr int kTPR = DV / kVec;             // threads covering one row of the tile
-  static constexpr int kConsumerWarps = 8;
-  static constexpr int kConsumers = kConsumerWarps * 32;
-  static constexpr int kThreads = kConsumers + 32;   // + one producer warp
-  static constexpr int kUsed = cmin(DK * kTPR, kConsumers);  // consumer threads holding state
-  static constexpr int kUsedWarps = kUsed / 32;
-  static constexpr int kRowsPerPass = kUsed / kTPR;
-  static constexpr int kPasses = DK / kRowsPerPass;  // rows per thread
+  static constexpr int kVec = StateVec<ST>::kElems;     // state elements per 16-byte chunk
+  static constexpr int kCW = DV < LA_STEP_STRIP_COLS ? DV : LA_STEP_STRIP_COLS;  // strip width
+  static constexpr int kWPT = DV / kCW;                 // warps per tile
+  static constexpr int kNCH = kCW / kVec;               // 16-byte chunks per strip row
+  static constexpr int kRG = 32 / kNCH;                 // row blocks per warp
+  static constexpr int kRL = DK / kRG;                  // rows per lane
+  static constexpr int kConsumerWarps = kWPT > LA_STEP_CONSUMER_WARPS ? kWPT : LA_STEP_CONSUMER_WARPS;
+  static constexpr int kTeams = kConsumerWarps / kWPT;  // tiles in compute at once
+  static constexpr int kThreads = (kConsumerWarps + 1) * 32;
   static constexpr int kTileBytes = DK * DV * kSB;
   static constexpr int kQKBytes = DK * (int)sizeof(IT);
   static constexpr int kVBytes = DV * (int)sizeof(IT);
   static constexpr int kCopyBytes = kTileBytes + 2 * kQKBytes + kVBytes;
   static constexpr int kStageBytes = round_up(kCopyBytes, 128);
-  static constexpr int kStages = cmax(2, cmin(8, (200 * 1024) / kStageBytes));
-  // shared-memory layout
+  static constexpr int kStages = cmax(2, cmin(12, (204 * 1024) / kStageBytes));
   static constexpr int kOffMeta = kStages * kStageBytes;
-  static constexpr int kOffRedP = round_up(kOffMeta + kStages * (int)sizeof(StepMeta), 16);
-  static constexpr int kOffRedR = kOffRedP + kUsedWarps * DV * 4;
-  static constexpr int kOffU = kOffRedR + kUsedWarps * DV * 4;
-  static constexpr int kOffBars = round_up(kOffU + DV * 4, 8);
+  static constexpr int kOffBars = round_up(kOffMeta + kStages * (int)sizeof(StepMeta), 8);
   static constexpr int kSmem = kOffBars + 2 * kStages * 8;
 
-  static_assert(kTPR >= 1 && kTPR <= 32 && (32 % kTPR) == 0, "row must map onto a power-of-two lane group");
-  static_assert(kUsed % 32 == 0 && DK % kRowsPerPass == 0, "tile must map onto whole warps");
-  static_assert(kVec % 4 == 0 || kVec == 4, "vector width");
-  static_assert(DV <= kConsumers, "one finishing thread per column");
+  static_assert(kNCH >= 1 && kNCH <= 32 && (32 % kNCH) == 0, "strip row must map onto a power-of-two lane group");
+  static_assert(kRL >= 1 && DK % kRG == 0, "rows must split evenly over the row blocks");
+  static_assert(kConsumerWarps % kWPT == 0, "whole tiles per team");
   static_assert(kQKBytes % 16 == 0 && kVBytes % 16 == 0 && kTileBytes % 16 == 0, "bulk copies move 16-byte units");
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
@@ -84,9 +99,6 @@ __global__ void __launch_bounds__(StepCfg<DK, DV, ST, IT>::kThreads, 1) step_ker
   using C = StepCfg<DK, DV, ST, IT>;
   extern __shared__ __align__(128) unsigned char smem[];
   StepMeta* meta = reinterpret_cast<StepMeta*>(smem + C::kOffMeta);
-  float* red_p = reinterpret_cast<float*>(smem + C::kOffRedP);
-  float* red_r = reinterpret_cast<float*>(smem + C::kOffRedR);
-  float* ubuf = reinterpret_cast<float*>(smem + C::kOffU);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
   uint64_t* empty = full + C::kStages;
 
@@ -97,11 +109,17 @@ __global__ void __launch_bounds__(StepCfg<DK, DV, ST, IT>::kThreads, 1) step_ker
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], C::kWPT);
     }
     mbar_init_fence();
   }
   __syncthreads();
+#if LA_STEP_PDL
+  // Programmatic dependent launch: everything above overlapped the previous kernel on
+  // the stream; nothing global is read before that kernel has completed.
+  griddep_wait();
+  griddep_launch_dependents();
+#endif
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -193,17 +211,25 @@ __global__ void __launch_bounds__(StepCfg<DK, DV, ST, IT>::kThreads, 1) step_ker
   }
 
   // -------------------------------------------------------------------- consumers
-  const int tid = threadIdx.x;  // 0 .. kConsumers-1
-  const bool holds = tid < C::kUsed;
-  const int cc = tid % C::kTPR;  // 16-byte column chunk
-  const int r0 = tid / C::kTPR;  // first row
+  constexpr int RL = C::kRL;
+  constexpr int V = C::kVec;
+  const int team = warp / C::kWPT;
+  const int part = warp % C::kWPT;
+  const int ch = lane % C::kNCH;              // 16-byte column chunk within the strip
+  const int rb = lane / C::kNCH;              // row block
+  const int col0 = part * C::kCW + ch * V;    // first column held by this lane
+  const int row0 = rb * RL;                   // first row held by this lane
   ST* dst = static_cast<ST*>(p.dst);
   IT* out = static_cast<IT*>(p.o);
 
-  for (int64_t it = 0; it < n_my; ++it) {
+  for (int64_t it = team; it < n_my; it += C::kTeams) {
     const int stage = (int)(it % C::kStages);
     const uint32_t round = (uint32_t)(it / C::kStages);
     const bool arrived = mbar_wait(&full[stage], round & 1u);
+    if (!__all_sync(0xffffffffu, arrived)) {
+      if (lane == 0) report(p.err, LA_DEVERR_TIMEOUT);
+      return;
+    }
     const StepMeta m = meta[stage];
     const unsigned char* sb = smem + stage * C::kStageBytes;
     const ST* tile = reinterpret_cast<const ST*>(sb);
@@ -213,86 +239,87 @@ __global__ void __launch_bounds__(StepCfg<DK, DV, ST, IT>::kThreads, 1) step_ker
     float a, bcoef, c;
     Rule<RULE>::coeffs(m.g, m.beta, a, bcoef, c);
 
-    // k . q (every warp computes it; only the finishing threads use it)
-    float kq = 0.0f;
-    for (int i = lane; i < DK; i += 32) kq = fmaf(io_load(ks + i), io_load(qs + i), kq);
+    float s[RL][V];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    for (int r = 0; r < RL; ++r)
+      StateVec<ST>::unpack(*reinterpret_cast<const uint4*>(tile + (row0 + r) * DV + col0), s[r]);
 
-    float s[C::kPasses][C::kVec];
-    float kr[C::kPasses];
-    if (holds) {
-      float pp[C::kVec], rr[C::kVec];
+    // k.q, S^T k and S^T q over this lane's rows (k, q read from the stage in blocks of
+    // up to 8 rows), then across the row blocks
+    constexpr int KB = RL < 8 ? RL : 8;
+    float kq = 0.0f;
+    float2 pp[V / 2], rr[V / 2];
 #pragma unroll
-      for (int e = 0; e < C::kVec; ++e) pp[e] = rr[e] = 0.0f;
+    for (int j = 0; j < V / 2; ++j) pp[j] = rr[j] = f2(0.0f, 0.0f);
 #pragma unroll
-      for (int ps = 0; ps < C::kPasses; ++ps) {
-        const int row = r0 + ps * C::kRowsPerPass;
-        const uint4 w = *reinterpret_cast<const uint4*>(tile + row * DV + cc * C::kVec);
-        StateVec<ST>::unpack(w, s[ps]);
-        kr[ps] = io_load(ks + row);
-        const float qr = io_load(qs + row);
+    for (int r0 = 0; r0 < RL; r0 += KB) {
+      float kb[KB], qb[KB];
+      load_f32<IT, KB>(ks + row0 + r0, kb);
+      load_f32<IT, KB>(qs + row0 + r0, qb);
 #pragma unroll
-        for (int e = 0; e < C::kVec; ++e) {
-          if (Rule<RULE>::kPredicts) pp[e] = fmaf(s[ps][e], kr[ps], pp[e]);
-          rr[e] = fmaf(s[ps][e], qr, rr[e]);
-        }
-      }
+      for (int r = 0; r < KB; ++r) {
+        kq = fmaf(kb[r], qb[r], kq);
+        const float2 k2 = f2(kb[r], kb[r]);
+        const float2 q2 = f2(qb[r], qb[r]);
 #pragma unroll
-      for (int off = C::kTPR; off < 32; off <<= 1) {
-#pragma unroll
-        for (int e = 0; e < C::kVec; ++e) {
-          if (Rule<RULE>::kPredicts) pp[e] += __shfl_xor_sync(0xffffffffu, pp[e], off);
-          rr[e] += __shfl_xor_sync(0xffffffffu, rr[e], off);
-        }
-      }
-      if (lane < C::kTPR) {
-        float4* dp = reinterpret_cast<float4*>(red_p + warp * DV + cc * C::kVec);
-        float4* dr = reinterpret_cast<float4*>(red_r + warp * DV + cc * C::kVec);
-#pragma unroll
-        for (int e4 = 0; e4 < C::kVec / 4; ++e4) {
-          if (Rule<RULE>::kPredicts) dp[e4] = make_float4(pp[4 * e4], pp[4 * e4 + 1], pp[4 * e4 + 2], pp[4 * e4 + 3]);
-          dr[e4] = make_float4(rr[4 * e4], rr[4 * e4 + 1], rr[4 * e4 + 2], rr[4 * e4 + 3]);
+        for (int j = 0; j < V / 2; ++j) {
+          const float2 s2 = f2(s[r0 + r][2 * j], s[r0 + r][2 * j + 1]);
+          if (Rule<RULE>::kPredicts) pp[j] = fma2(s2, k2, pp[j]);
+          rr[j] = fma2(s2, q2, rr[j]);
         }
       }
     }
-    // Barrier 1 (consumers): partial sums are in shared memory.  It also ORs the
-    // "stage never arrived" flags so that every consumer leaves together.
-    if (named_bar_or(1, C::kConsumers, !arrived)) {
-      if (tid == 0) report(p.err, LA_DEVERR_TIMEOUT);
-      return;
-    }
-    if (tid < DV) {
-      float pj = 0.0f, rj = 0.0f;
 #pragma unroll
-      for (int w = 0; w < C::kUsedWarps; ++w) {
-        if (Rule<RULE>::kPredicts) pj += red_p[w * DV + tid];
-        rj += red_r[w * DV + tid];
-      }
-      const float u = bcoef * (io_load(vs + tid) - c * pj);
-      ubuf[tid] = u;
-      if (m.valid) io_store(out + m.o_off + tid, p.scale * fmaf(a, rj, kq * u));
-    }
-    // Barrier 2: u is in shared memory and nobody reads the stage any more.
-    named_bar_sync(2, C::kConsumers);
-    if (tid == 0) mbar_arrive(&empty[stage]);
-    if (holds && m.valid) {
-      float u[C::kVec];
+    for (int off = C::kNCH; off < 32; off <<= 1) {
+      kq += __shfl_xor_sync(0xffffffffu, kq, off);
 #pragma unroll
-      for (int e4 = 0; e4 < C::kVec / 4; ++e4) {
-        const float4 x = *reinterpret_cast<const float4*>(ubuf + cc * C::kVec + 4 * e4);
-        u[4 * e4] = x.x; u[4 * e4 + 1] = x.y; u[4 * e4 + 2] = x.z; u[4 * e4 + 3] = x.w;
+      for (int j = 0; j < V / 2; ++j) {
+        if (Rule<RULE>::kPredicts) {
+          pp[j].x += __shfl_xor_sync(0xffffffffu, pp[j].x, off);
+          pp[j].y += __shfl_xor_sync(0xffffffffu, pp[j].y, off);
+        }
+        rr[j].x += __shfl_xor_sync(0xffffffffu, rr[j].x, off);
+        rr[j].y += __shfl_xor_sync(0xffffffffu, rr[j].y, off);
       }
+    }
+
+    if (m.valid) {
+      // u = b (v - c p),  o = scale (a r + (k.q) u)
+      float vv[V], u[V], o[V];
+      load_f32<IT, V>(vs + col0, vv);
+#pragma unroll
+      for (int j = 0; j < V / 2; ++j) {
+        u[2 * j] = bcoef * (vv[2 * j] - c * pp[j].x);
+        u[2 * j + 1] = bcoef * (vv[2 * j + 1] - c * pp[j].y);
+        o[2 * j] = p.scale * fmaf(a, rr[j].x, kq * u[2 * j]);
+        o[2 * j + 1] = p.scale * fmaf(a, rr[j].y, kq * u[2 * j + 1]);
+      }
+      if (rb == 0) store_f32<IT, V>(out + m.o_off + col0, o);
+
+      // S' = a S + k u^T, stored with 16-byte vectors
       ST* dtile = dst + m.dst_off;
+      const float2 a2 = f2(a, a);
 #pragma unroll
-      for (int ps = 0; ps < C::kPasses; ++ps) {
-        const int row = r0 + ps * C::kRowsPerPass;
-        float y[C::kVec];
+      for (int r0 = 0; r0 < RL; r0 += KB) {
+        float kb[KB];
+        load_f32<IT, KB>(ks + row0 + r0, kb);
 #pragma unroll
-        for (int e = 0; e < C::kVec; ++e) y[e] = fmaf(kr[ps], u[e], a * s[ps][e]);
-        *reinterpret_cast<uint4*>(dtile + row * DV + cc * C::kVec) = StateVec<ST>::pack(y);
+        for (int r = 0; r < KB; ++r) {
+          const float2 k2 = f2(kb[r], kb[r]);
+          float y[V];
+#pragma unroll
+          for (int j = 0; j < V / 2; ++j) {
+            const float2 t =
+                fma2(k2, f2(u[2 * j], u[2 * j + 1]), mul2(a2, f2(s[r0 + r][2 * j], s[r0 + r][2 * j + 1])));
+            y[2 * j] = t.x;
+            y[2 * j + 1] = t.y;
+          }
+          *reinterpret_cast<uint4*>(dtile + (row0 + r0 + r) * DV + col0) = StateVec<ST>::pack(y);
+        }
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);  // this warp is done with the stage
   }
 }
 
@@ -305,7 +332,22 @@ cudaError_t launch_step(const StepParams& p, cudaStream_t stream) {
   const int64_t ntiles = (int64_t)p.B * p.n_v_heads;
   const int64_t cap = (int64_t)device_sm_count() * per_sm;
   const int grid = (int)(ntiles < cap ? ntiles : cap);
+#if LA_STEP_PDL
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, step_kernel<RULE, DK, DV, ST, IT>, p);
+  if (e != cudaSuccess) return e;
+#else
   step_kernel<RULE, DK, DV, ST, IT><<<grid, C::kThreads, C::kSmem, stream>>>(p);
+#endif
   return cudaGetLastError();
 }
 
