@@ -206,6 +206,9 @@ class ClockSampler:
 
 
 def dist_setup(n_gpus):
+    """One process per GPU from torchrun's environment (RANK, LOCAL_RANK, WORLD_SIZE,
+    MASTER_*).  NCCL when CUDA is present, gloo otherwise (the CPU tests of this logic).
+    The process group only carries barriers and the max-over-ranks of the elapsed time."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -213,9 +216,12 @@ def dist_setup(n_gpus):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return rank, world, local
@@ -232,7 +238,8 @@ def max_over_ranks(x, world):
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -419,57 +426,113 @@ def time_flushed(run, steps, flush):
 
 
 def time_e2e(run: DecodeRunner, steps, warmup, world):
-    """The decode step through the same C-ABI call with its inputs copied from pinned host
-    memory (q, k, v, g, beta and the slot ids, one packed copy) and o copied back, all
-    inside the timed region.  The state stays resident in the device pool."""
+    """The decode step through the same C-ABI call with every step's inputs (q, k, v, g,
+    beta and the slot ids, one packed buffer) copied from pinned host memory and its
+    output o copied back to pinned host memory, all inside the timed region.  The state
+    stays resident in the device pool.  Steps are pipelined the way a serving loop would
+    run them: device inputs and outputs are double buffered, the host-to-device copy of
+    step i+1 and the device-to-host copy of step i-1 run on their own streams while step i
+    computes, and chunks of steps are captured in a CUDA graph so that Python launch
+    overhead does not bound the loop.  Returns (ms per step, H2D bytes, D2H bytes)."""
     import torch
     inp = run.inp
+    L = run.L
     parts = [inp.q, inp.k, inp.v, inp.g, inp.beta]
-    slot_parts = [(r, w) for r, w in run.sets]
-    offs, total = [], 0
     sizes = [p.numel() * p.element_size() for p in parts] + [run.B * 4, run.B * 4]
+    offs, total = [], 0
     for sz in sizes:
         offs.append(total)
         total += (sz + 255) // 256 * 256
+    payload = sum(sizes[:5]) + (2 * run.B * 4 if inp.read_slot is not None else 0)
     hosts = []
-    for r, w in slot_parts:
-        hb = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    for r, w in run.sets:
+        hb = torch.zeros(total, dtype=torch.uint8, pin_memory=True)
         for p, off in zip(parts, offs):
             hb[off:off + p.numel() * p.element_size()].copy_(p.contiguous().view(-1).view(torch.uint8))
         if r is not None:
             hb[offs[5]:offs[5] + run.B * 4].copy_(r.cpu().view(torch.uint8))
             hb[offs[6]:offs[6] + run.B * 4].copy_(w.cpu().view(torch.uint8))
         hosts.append(hb)
-    dev = torch.empty(total, dtype=torch.uint8, device="cuda")
+    devs = [torch.empty(total, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    outs = [torch.empty_like(run.o) for _ in range(2)]
+    o_hosts = [torch.empty(run.o.shape, dtype=run.o.dtype, pin_memory=True) for _ in range(2)]
+    o_bytes = o_hosts[0].numel() * o_hosts[0].element_size()
 
-    def view(i, dtype, shape):
-        n = 1
-        for s in shape:
-            n *= s
-        return dev[offs[i]:offs[i] + n * torch.empty(0, dtype=dtype).element_size()].view(dtype).view(shape)
+    def views(dev):
+        def v(i, dtype, shape):
+            n = 1
+            for x in shape:
+                n *= x
+            return dev[offs[i]:offs[i] + n * torch.empty(0, dtype=dtype).element_size()].view(dtype).view(shape)
+        return (v(0, inp.q.dtype, inp.q.shape), v(1, inp.k.dtype, inp.k.shape), v(2, inp.v.dtype, inp.v.shape),
+                v(3, torch.float32, inp.g.shape), v(4, torch.float32, inp.beta.shape),
+                v(5, torch.int32, (run.B,)) if inp.read_slot is not None else None,
+                v(6, torch.int32, (run.B,)) if inp.read_slot is not None else None)
+    vs = [views(d) for d in devs]
+    sh, sd = torch.cuda.Stream(), torch.cuda.Stream()
 
-    q = view(0, inp.q.dtype, inp.q.shape)
-    k = view(1, inp.k.dtype, inp.k.shape)
-    v = view(2, inp.v.dtype, inp.v.shape)
-    g = view(3, torch.float32, inp.g.shape)
-    beta = view(4, torch.float32, inp.beta.shape)
-    rs = view(5, torch.int32, (run.B,)) if inp.read_slot is not None else None
-    ws = view(6, torch.int32, (run.B,)) if inp.read_slot is not None else None
-    o_host = torch.empty(run.o.shape, dtype=run.o.dtype, pin_memory=True)
-    L = run.L
+    def enqueue(n_steps, first):
+        """n_steps pipelined steps on the current stream (+ the two copy streams)."""
+        cs = torch.cuda.current_stream()
+        fork = torch.cuda.Event()
+        fork.record(cs)
+        sh.wait_event(fork)
+        sd.wait_event(fork)
+        kev, dev_free = [None, None], [None, None]
+        for j in range(n_steps):
+            b = j % 2
+            hev = torch.cuda.Event()
+            with torch.cuda.stream(sh):
+                if kev[b] is not None:
+                    sh.wait_event(kev[b])          # step j-2 no longer reads devs[b]
+                devs[b].copy_(hosts[(first + j) % len(hosts)], non_blocking=True)
+                hev.record(sh)
+            cs.wait_event(hev)
+            if dev_free[b] is not None:
+                cs.wait_event(dev_free[b])         # o of step j-2 has reached the host
+            q, k, v, g, beta, rs, ws = vs[b]
+            st = L.la_state_step(inp.rule, run.pool, rs, run.pool, ws, q, k, v, g, beta, inp.scale, outs[b], run.err)
+            if st != 0:
+                raise L.LAError(st)
+            kev[b] = torch.cuda.Event()
+            kev[b].record(cs)
+            with torch.cuda.stream(sd):
+                sd.wait_event(kev[b])
+                o_hosts[b].copy_(outs[b], non_blocking=True)
+                dev_free[b] = torch.cuda.Event()
+                dev_free[b].record(sd)
+        jh, jd = torch.cuda.Event(), torch.cuda.Event()
+        jh.record(sh)
+        jd.record(sd)
+        cs.wait_event(jh)
+        cs.wait_event(jd)
 
-    def one(i):
-        dev.copy_(hosts[i % len(hosts)], non_blocking=True)
-        st = L.la_state_step(inp.rule, run.pool, rs, run.pool, ws, q, k, v, g, beta, inp.scale, run.o, run.err)
-        if st != 0:
-            raise L.LAError(st)
-        o_host.copy_(run.o, non_blocking=True)
+    chunk = next(c for c in (16, 8, 4, 2, 1) if steps % c == 0)
+    graph = None
+    try:
+        enqueue(chunk, 0)  # warm-up outside capture
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            enqueue(chunk, 0)
+        torch.cuda.synchronize()
+    except Exception:
+        graph = None  # capture not available: enqueue the same pipeline eagerly
+        torch.cuda.synchronize()
 
     class R:
-        step = staticmethod(one)
+        @staticmethod
+        def step(i):
+            if i % chunk:
+                return
+            if graph is not None:
+                graph.replay()
+            else:
+                enqueue(chunk, i)
 
-    ms = time_back_to_back(R, steps, warmup, world)
-    return ms, total, o_host.numel() * o_host.element_size()
+    ms = time_back_to_back(R, steps, max(warmup, chunk), world)
+    del graph
+    return ms, payload, o_bytes
 
 
 # --------------------------------------------------------------------------------------
@@ -616,7 +679,10 @@ def main():
     if inp.kind == "step":
         e2e_ms, h2d, d2h = time_e2e(run, a.steps, a.warmup, world)
         out["e2e"] = {"value": aggregate(nbytes, e2e_ms, world) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
-                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                      "tokens_per_s": world * run.B / (e2e_ms * 1e-3),
+                      "how": "pinned host buffers; H2D of step i+1 and D2H of step i-1 overlap step i; "
+                             "chunks of 16 steps replayed as a CUDA graph"}
         out["gpu_launches"] += a.steps
     del run
     torch.cuda.empty_cache()
