@@ -307,7 +307,10 @@ class DecodeRunner:
 
 
 class ScanRunner:
-    def __init__(self, inp):
+    """A prefill workload on the device.  ckpt_every > 0: la_state_scan_checkpointed with a
+    checkpoint slot for every ckpt_every tokens of every sequence."""
+
+    def __init__(self, inp, ckpt_every=0):
         import torch
         from gated_deltanet_recurrent_la_b200 import lastate as L
         self.L = L
@@ -327,20 +330,40 @@ class ScanRunner:
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
         self.T = int(inp.q.shape[0])
         self.n_seqs = n_seqs
+        self.ckpt_every = ckpt_every
+        self.n_ckpt = 0
+        if ckpt_every > 0:
+            n_ck = [l // ckpt_every for l in lens]
+            self.n_ckpt = sum(n_ck)
+            cu = [0]
+            for n in n_ck:
+                cu.append(cu[-1] + n)
+            self.ckpt_cu = torch.tensor(cu, dtype=torch.int32, device="cuda")
+            self.ckpt_slots = torch.arange(n_seqs, n_seqs + self.n_ckpt, dtype=torch.int32, device="cuda")
+            self.dst_t = torch.empty(n_seqs + self.n_ckpt, inp.n_v_heads, inp.d_k, inp.d_v, dtype=inp.state_dtype,
+                                     device="cuda")
+            self.dst = L.Pool(self.dst_t, inp.n_qk_heads)
 
     def step(self, i=0, stream=None):
-        st = self.L.la_state_scan(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu, self.q, self.k,
-                                  self.v, self.g, self.beta, self.inp.scale, self.o, self.err,
-                                  seq_order=self.order, stream=stream)
+        if self.ckpt_every > 0:
+            st = self.L.la_state_scan_checkpointed(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu,
+                                                   self.q, self.k, self.v, self.g, self.beta, self.inp.scale, self.o,
+                                                   self.ckpt_every, self.ckpt_cu, self.ckpt_slots, self.err,
+                                                   seq_order=self.order, stream=stream)
+        else:
+            st = self.L.la_state_scan(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu, self.q,
+                                      self.k, self.v, self.g, self.beta, self.inp.scale, self.o, self.err,
+                                      seq_order=self.order, stream=stream)
         if st != 0:
             raise self.L.LAError(st)
 
     def bytes_flops(self):
         i = self.inp
-        return scan_bytes_and_flops(T=self.T, n_seqs=self.n_seqs, n_qk_heads=i.n_qk_heads, n_v_heads=i.n_v_heads,
+        b, f = scan_bytes_and_flops(T=self.T, n_seqs=self.n_seqs, n_qk_heads=i.n_qk_heads, n_v_heads=i.n_v_heads,
                                     d_k=i.d_k, d_v=i.d_v, io_bytes=i.q.element_size(), rule=i.rule,
                                     final_state_bytes=self.dst_t.element_size(),
                                     init_state_bytes=0 if i.pool is None else i.pool.element_size())
+        return b + self.n_ckpt * i.n_v_heads * i.d_k * i.d_v * self.dst_t.element_size(), f
 
 
 class PoolRunner:
@@ -566,11 +589,11 @@ def cpu_baseline_decode(inp, budget_s=10.0):
 # --------------------------------------------------------------------------------------
 
 
-def build_runner(name, seed=0, prefill_seqs=32):
+def build_runner(name, seed=0, prefill_seqs=32, ckpt_every=0):
     from gated_deltanet_recurrent_la_b200 import workloads as W
     inp = W.prefill32(seed, prefill_seqs) if name == "prefill32" else W.WORKLOADS[name](seed)
     if inp.kind == "scan":
-        return ScanRunner(inp), inp
+        return ScanRunner(inp, ckpt_every), inp
     n_sets = 4 if name == "decode64" else 1
     return DecodeRunner(inp, n_sets=n_sets, seed=seed), inp
 
@@ -591,8 +614,8 @@ def describe(name, inp):
     return d
 
 
-def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None):
-    run, inp = build_runner(name)
+def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_every=0):
+    run, inp = build_runner(name, ckpt_every=ckpt_every)
     ms = time_back_to_back(run, steps, warmup, world)
     nbytes, flops = run.bytes_flops()
     row = {"config": describe(name, inp), "ms_per_step": ms, "gb_s": nbytes / (ms * 1e-3) / 1e9}
@@ -609,6 +632,9 @@ def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None):
         alu = fp32_alu_peak_tflops(sm_count, peaks["sm_max_mhz"])
         tf = flops / (ms * 1e-3) / 1e12
         row["tokens_per_s"] = run.T / (ms * 1e-3)
+        if ckpt_every:
+            row["config"]["ckpt_every"] = ckpt_every
+            row["config"]["checkpoints"] = run.n_ckpt
         row["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
                            "traffic": recorded_traffic("scan", name), "hbm_gb_s": row["gb_s"],
                            "effective_state_gb_s": run.T * inp.n_v_heads * 2 * inp.d_k * inp.d_v * 4 / (ms * 1e-3) / 1e9,
@@ -695,6 +721,9 @@ def main():
             k = a.steps if name != "prefill32" else max(3, min(a.steps, 20))
             rows[name] = measure_row(name, min(k, 500), a.warmup, world, peaks, sm_count, flush)
             torch.cuda.empty_cache()
+        rows["prefill32_ckpt256"] = measure_row("prefill32", max(3, min(a.steps, 20)), a.warmup, world, peaks,
+                                                sm_count, None, ckpt_every=256)
+        torch.cuda.empty_cache()
         pool_run = PoolRunner()
         pms = time_back_to_back(pool_run, min(a.steps, 500), a.warmup, world)
         pb, _ = pool_run.bytes_flops()

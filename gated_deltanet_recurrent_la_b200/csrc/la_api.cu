@@ -154,10 +154,11 @@ la_status la_state_step(la_rule rule, const la_pool* src, const int32_t* read_sl
   return cuda_status(fn(p, static_cast<cudaStream_t>(stream)));
 }
 
-la_status la_state_scan(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
-                        const int32_t* write_slot, int32_t n_seqs, const int32_t* cu_seqlens, int32_t total_tokens,
-                        const int32_t* seq_order, const void* q, const void* k, const void* v, la_dtype io,
-                        const float* g, const float* beta, float scale, void* o, int32_t* err_word, void* stream) {
+static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
+                           const int32_t* write_slot, int32_t n_seqs, const int32_t* cu_seqlens, int32_t total_tokens,
+                           const int32_t* seq_order, const void* q, const void* k, const void* v, la_dtype io,
+                           const float* g, const float* beta, float scale, void* o, int32_t ckpt_every,
+                           const int32_t* ckpt_cu, const int32_t* ckpt_slots, int32_t* err_word, void* stream) {
   if (rule < LA_RULE_LINEAR || rule > LA_RULE_GATED_DELTA) return LA_ERR_UNSUPPORTED;
   if (!err_word) return LA_ERR_NULL;
   if (n_seqs < 0 || total_tokens < 0) return LA_ERR_SHAPE;
@@ -209,7 +210,31 @@ la_status la_state_scan(la_rule rule, const la_pool* src, const int32_t* read_sl
   p.scale = scale;
   p.o = o;
   p.err = err_word;
+  p.ckpt_every = ckpt_every;
+  p.ckpt_cu = ckpt_cu;
+  p.ckpt_slots = ckpt_slots;
   return cuda_status(fn(p, static_cast<cudaStream_t>(stream)));
+}
+
+la_status la_state_scan(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
+                        const int32_t* write_slot, int32_t n_seqs, const int32_t* cu_seqlens, int32_t total_tokens,
+                        const int32_t* seq_order, const void* q, const void* k, const void* v, la_dtype io,
+                        const float* g, const float* beta, float scale, void* o, int32_t* err_word, void* stream) {
+  return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, q, k, v, io,
+                   g, beta, scale, o, 0, nullptr, nullptr, err_word, stream);
+}
+
+la_status la_state_scan_checkpointed(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
+                                     const int32_t* write_slot, int32_t n_seqs, const int32_t* cu_seqlens,
+                                     int32_t total_tokens, const int32_t* seq_order, const void* q, const void* k,
+                                     const void* v, la_dtype io, const float* g, const float* beta, float scale,
+                                     void* o, int32_t ckpt_every, const int32_t* ckpt_cu, const int32_t* ckpt_slots,
+                                     int32_t* err_word, void* stream) {
+  if (ckpt_every <= 0) return LA_ERR_SHAPE;
+  if (n_seqs > 0 && (!ckpt_cu || !ckpt_slots)) return LA_ERR_NULL;
+  if (!aligned(ckpt_cu, 4) || !aligned(ckpt_slots, 4)) return LA_ERR_ALIGN;
+  return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, q, k, v, io,
+                   g, beta, scale, o, ckpt_every, ckpt_cu, ckpt_slots, err_word, stream);
 }
 
 static la_status pool_op(const la_pool* pool, int32_t n, const int32_t* src_slots, const int32_t* dst_slots,

@@ -52,6 +52,9 @@ struct ScanParams {
   float scale;
   void* o;
   int32_t* err;
+  int32_t ckpt_every;          // > 0: intermediate states every ckpt_every tokens
+  const int32_t* ckpt_cu;      // [n_seqs + 1] offsets into ckpt_slots
+  const int32_t* ckpt_slots;   // destination slots of the checkpoints
 };
 
 struct PoolCopyParams {

@@ -21,9 +21,13 @@
 //   * per token, one fused pass over the lane's elements applies the previous token's
 //     update and accumulates St^T k and St^T q for the current token (the readout
 //     rearrangement of the "Gated DeltaNet" page makes S^T q the old state's product):
-//     three FMAs per element; two xor-shuffles finish the d_k sums across the 4 lanes;
+//     three FMAs per element, the two sums kept as even / odd row partials for more
+//     independent chains; two xor-shuffles finish the d_k sums across the 4 lanes;
 //   * q, k (converted to FP32 in a bank-conflict-free padded layout), v, g, beta of 16
 //     upcoming tokens are staged in shared memory with cp.async double buffering;
+//   * optional checkpoints: every ckpt_every tokens the pending update is applied at
+//     once and the state is stored to a checkpoint slot (prefix caching at KV-block
+//     boundaries, "Gated DeltaNet" glossary, Why it matters);
 //   * units are dealt to persistent CTAs in the order given by seq_order (longest
 //     first balances best) in a boustrophedon pattern.
 #pragma once
@@ -128,6 +132,18 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
       continue;
     }
 
+    // ---- checkpoints of this sequence: after (j + 1) * ckpt_every tokens, j < n_ck
+    int n_ck = 0, ck_base = 0;
+    if (p.ckpt_every > 0) {
+      ck_base = __ldg(p.ckpt_cu + seq);
+      n_ck = __ldg(p.ckpt_cu + seq + 1) - ck_base;
+      const int fit = (t1 - t0) / p.ckpt_every;
+      if (n_ck < 0 || n_ck > fit) {
+        if (tid == 0) report(p.err, LA_DEVERR_CU_SEQLENS);
+        n_ck = n_ck < 0 ? 0 : fit;
+      }
+    }
+
     // ---- initial state: rows rg*R .. rg*R+R-1, columns col0 .. col0+KC-1
     float S[R][KC];
     if (p.read_slot && col_active) {
@@ -156,6 +172,32 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
 #pragma unroll
     for (int c = 0; c < KC; ++c) up[c] = 0.0f;
     const float* kp = nullptr;  // pending key (padded FP32 row block); nullptr: none
+    int ck_j = 0, ck_left = p.ckpt_every;  // next checkpoint, tokens until it
+
+    // stores gam * St (the state) to slot `slot` of the destination pool
+    auto store_state = [&](int slot) {
+      if (!col_active) return;
+      const int64_t base = ((int64_t)slot * H + h) * (DK * DV);
+      if (p.dst_dtype == LA_F32) {
+        float* dst = static_cast<float*>(p.dst) + base;
+#pragma unroll
+        for (int m = 0; m < R; ++m) {
+          float y[KC];
+#pragma unroll
+          for (int c = 0; c < KC; ++c) y[c] = gam * S[m][c];
+          store_f32<float, KC>(dst + (rg * R + m) * DV + col0, y);
+        }
+      } else {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.dst) + base;
+#pragma unroll
+        for (int m = 0; m < R; ++m) {
+          float y[KC];
+#pragma unroll
+          for (int c = 0; c < KC; ++c) y[c] = gam * S[m][c];
+          store_f32<__nv_bfloat16, KC>(dst + (rg * R + m) * DV + col0, y);
+        }
+      }
+    };
 
     auto issue = [&](int ch) {
       unsigned char* raw = smem + (ch & 1) * C::kRawBytes;
@@ -229,9 +271,9 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
         const float* kc = kf + tt * C::kKP + rg * C::kRowStride;
         const float* qc = qf + tt * C::kKP + rg * C::kRowStride;
         const float* kpp = kp ? kp : kc;  // no pending update before the first token
-        float pa[KC], ra[KC];
+        float pa[KC], ra[KC], pb[KC], rb2[KC];  // even / odd row partial sums
 #pragma unroll
-        for (int c = 0; c < KC; ++c) pa[c] = ra[c] = 0.0f;
+        for (int c = 0; c < KC; ++c) pa[c] = ra[c] = pb[c] = rb2[c] = 0.0f;
 #pragma unroll
         for (int m4 = 0; m4 < R / 4; ++m4) {
           const float4 k4p = *reinterpret_cast<const float4*>(kpp + 4 * m4);
@@ -246,13 +288,20 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
             for (int c = 0; c < KC; ++c) {
               float& x = S[4 * m4 + mm][c];
               x = fmaf(kpv[mm], up[c], x);
-              if (Rule<RULE>::kPredicts) pa[c] = fmaf(x, kv[mm], pa[c]);
-              ra[c] = fmaf(x, qv[mm], ra[c]);
+              if (mm & 1) {
+                if (Rule<RULE>::kPredicts) pb[c] = fmaf(x, kv[mm], pb[c]);
+                rb2[c] = fmaf(x, qv[mm], rb2[c]);
+              } else {
+                if (Rule<RULE>::kPredicts) pa[c] = fmaf(x, kv[mm], pa[c]);
+                ra[c] = fmaf(x, qv[mm], ra[c]);
+              }
             }
           }
         }
 #pragma unroll
         for (int c = 0; c < KC; ++c) {
+          pa[c] += pb[c];
+          ra[c] += rb2[c];
           if (Rule<RULE>::kPredicts) {
             pa[c] += __shfl_xor_sync(0xffffffffu, pa[c], 1);
             pa[c] += __shfl_xor_sync(0xffffffffu, pa[c], 2);
@@ -296,7 +345,7 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
           } else {
             gam = gnew;
           }
-          const float inv = __frcp_rn(gam);
+          const float inv = __fdividef(1.0f, gam);
 #pragma unroll
           for (int c = 0; c < KC; ++c) up[c] = uu[c] * inv;
         } else {
@@ -304,6 +353,29 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
           for (int c = 0; c < KC; ++c) up[c] = uu[c];
         }
         kp = kc;
+        if (ck_j < n_ck && --ck_left == 0) {
+          // checkpoint: apply this token's update now and store the state
+          ck_left = p.ckpt_every;
+#pragma unroll
+          for (int m4 = 0; m4 < R / 4; ++m4) {
+            const float4 k4 = *reinterpret_cast<const float4*>(kc + 4 * m4);
+            const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm)
+#pragma unroll
+              for (int c = 0; c < KC; ++c) S[4 * m4 + mm][c] = fmaf(kv[mm], up[c], S[4 * m4 + mm][c]);
+          }
+#pragma unroll
+          for (int c = 0; c < KC; ++c) up[c] = 0.0f;
+          kp = nullptr;
+          const int cs = __ldg(p.ckpt_slots + ck_base + ck_j);
+          if (cs >= 0 && cs < p.dst_slots) {
+            store_state(cs);
+          } else if (tid == 0) {
+            report(p.err, LA_DEVERR_WRITE_SLOT);
+          }
+          ++ck_j;
+        }
       }
       __syncthreads();
     }
@@ -320,22 +392,7 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
           for (int c = 0; c < KC; ++c) S[4 * m4 + mm][c] = fmaf(kpv[mm], up[c], S[4 * m4 + mm][c]);
       }
     }
-    if (col_active) {
-#pragma unroll
-      for (int m = 0; m < R; ++m)
-#pragma unroll
-        for (int c = 0; c < KC; ++c) S[m][c] *= gam;
-      const int64_t base = ((int64_t)ws * H + h) * (DK * DV);
-      if (p.dst_dtype == LA_F32) {
-        float* dst = static_cast<float*>(p.dst) + base;
-#pragma unroll
-        for (int m = 0; m < R; ++m) store_f32<float, KC>(dst + (rg * R + m) * DV + col0, S[m]);
-      } else {
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.dst) + base;
-#pragma unroll
-        for (int m = 0; m < R; ++m) store_f32<__nv_bfloat16, KC>(dst + (rg * R + m) * DV + col0, S[m]);
-      }
-    }
+    store_state(ws);
     // the next unit's staging must not overwrite what this unit still reads
     __syncthreads();
   }

@@ -160,6 +160,28 @@ la_status la_state_scan(la_rule rule, const la_pool *src, const int32_t *read_sl
                         const float *g, const float *beta, float scale, void *o,
                         int32_t *err_word, void *stream);
 
+/* The scan of la_state_scan that also stores intermediate states: the prefix-cache
+ * checkpoints "aligned to KV block boundaries" of the "Gated DeltaNet" glossary page (Why
+ * it matters), and state snapshots for speculative-decoding rollback ("Seven
+ * Architectures ...", Limitations and Open Questions).
+ *   ckpt_every  > 0; checkpoint j of sequence s is the state after the sequence's first
+ *               (j + 1) * ckpt_every tokens (the state the next token would start from)
+ *   ckpt_cu     device int32 [n_seqs + 1]: sequence s has checkpoints
+ *               ckpt_slots[ckpt_cu[s] .. ckpt_cu[s+1]), at most len(s) / ckpt_every of them
+ *   ckpt_slots  device int32: destination slots in dst (dst dtype), distinct from every
+ *               write slot and every read slot
+ * Other arguments and errors as la_state_scan.  A sequence with more checkpoints than fit
+ * reports LA_DEVERR_CU_SEQLENS (the ones that fit are written); an out-of-range
+ * checkpoint slot reports LA_DEVERR_WRITE_SLOT and is skipped.  Host errors: ckpt_every
+ * <= 0 (LA_ERR_SHAPE), NULL ckpt arrays (LA_ERR_NULL). */
+la_status la_state_scan_checkpointed(la_rule rule, const la_pool *src, const int32_t *read_slot,
+                                     const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
+                                     const int32_t *cu_seqlens, int32_t total_tokens,
+                                     const int32_t *seq_order, const void *q, const void *k,
+                                     const void *v, la_dtype io, const float *g, const float *beta,
+                                     float scale, void *o, int32_t ckpt_every, const int32_t *ckpt_cu,
+                                     const int32_t *ckpt_slots, int32_t *err_word, void *stream);
+
 /* Slot-pool maintenance, bit-exact whole-slot copies ("Recurrent state" glossary: slot
  * allocation and prefix-cache checkpoints; "Seven Architectures ...", ONNX section:
  * snapshots saved and restored for speculative-decoding rollback, migrated between

@@ -227,12 +227,21 @@ void lao_readout_rearranged(int rule, int n_qk_heads, int n_v_heads, int dk, int
 
 /* ---- token-serial scan over packed variable-length sequences -------------------- */
 
-int lao_scan(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
-             const double *src_pool, int src_slots, const int *read_slot,
-             double *dst_pool, int dst_slots, int dst_dtype, const int *write_slot,
-             int n_seqs, const int *cu_seqlens, int total_tokens,
-             const double *q, const double *k, const double *v, int io_dtype,
-             const double *g, const double *beta, double scale, double *o)
+/* Scan with intermediate checkpoints ("Gated DeltaNet" glossary, Why it matters:
+ * hybrid prefix caching keeps checkpoint slots aligned to KV block boundaries; "Seven
+ * Architectures ...", Limitations: state snapshots for speculative-decoding rollback).
+ * With ckpt_every > 0, checkpoint j of sequence s (j < ckpt_cu[s+1] - ckpt_cu[s]) is the
+ * state after the sequence's first (j + 1) * ckpt_every tokens, rounded to dst_dtype and
+ * stored to dst_pool slot ckpt_slots[ckpt_cu[s] + j].  A checkpoint position beyond the
+ * sequence is reported (bit 4) and skipped; an out-of-range checkpoint slot is reported
+ * (bit 2) and skipped.  ckpt_every <= 0: no checkpoints (lao_scan). */
+int lao_scan_ckpt(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+                  const double *src_pool, int src_slots, const int *read_slot,
+                  double *dst_pool, int dst_slots, int dst_dtype, const int *write_slot,
+                  int n_seqs, const int *cu_seqlens, int total_tokens,
+                  const double *q, const double *k, const double *v, int io_dtype,
+                  const double *g, const double *beta, double scale, double *o,
+                  int ckpt_every, const int *ckpt_cu, const int *ckpt_slots)
 {
     const size_t tile = (size_t)dk * dv;
     const size_t slot = (size_t)n_v_heads * tile;
@@ -249,6 +258,14 @@ int lao_scan(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
         int ws = write_slot ? write_slot[s] : s;
         if (ws < 0 || ws >= dst_slots) { err |= LAO_ERR_WRITE_SLOT; continue; }
         ok[s] = 1;
+        if (ckpt_every > 0) {
+            const int n_ck = ckpt_cu[s + 1] - ckpt_cu[s];
+            for (int j = 0; j < n_ck; ++j) {
+                if ((long long)(j + 1) * ckpt_every > (long long)(t1 - t0)) { err |= LAO_ERR_CU_SEQLENS; break; }
+                const int cs = ckpt_slots[ckpt_cu[s] + j];
+                if (cs < 0 || cs >= dst_slots) err |= LAO_ERR_WRITE_SLOT;
+            }
+        }
     }
 
 #pragma omp parallel for collapse(2) schedule(dynamic, 1)
@@ -272,6 +289,17 @@ int lao_scan(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
                              beta ? beta[(size_t)t * n_v_heads + h] : 1.0,
                              scale, ot, u);
                 for (int j = 0; j < dv; ++j) ot[j] = lao_round_to(ot[j], io_dtype);
+                const int pos = t - cu_seqlens[s] + 1; /* tokens of this sequence consumed */
+                if (ckpt_every > 0 && pos % ckpt_every == 0) {
+                    const int j = pos / ckpt_every - 1;
+                    if (j < ckpt_cu[s + 1] - ckpt_cu[s]) {
+                        const int cs = ckpt_slots[ckpt_cu[s] + j];
+                        if (cs >= 0 && cs < dst_slots) {
+                            double *D = dst_pool + (size_t)cs * slot + (size_t)h * tile;
+                            for (size_t e = 0; e < tile; ++e) D[e] = lao_round_to(S[e], dst_dtype);
+                        }
+                    }
+                }
             }
             for (size_t e = 0; e < tile; ++e) S[e] = lao_round_to(S[e], dst_dtype);
             free(u);
@@ -286,6 +314,18 @@ int lao_scan(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
     free(next);
     free(ok);
     return err;
+}
+
+int lao_scan(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+             const double *src_pool, int src_slots, const int *read_slot,
+             double *dst_pool, int dst_slots, int dst_dtype, const int *write_slot,
+             int n_seqs, const int *cu_seqlens, int total_tokens,
+             const double *q, const double *k, const double *v, int io_dtype,
+             const double *g, const double *beta, double scale, double *o)
+{
+    return lao_scan_ckpt(rule, n_qk_heads, n_v_heads, dk, dv, src_pool, src_slots, read_slot, dst_pool,
+                         dst_slots, dst_dtype, write_slot, n_seqs, cu_seqlens, total_tokens, q, k, v, io_dtype,
+                         g, beta, scale, o, 0, NULL, NULL);
 }
 
 /* ---- slot pool: whole-slot byte copies ------------------------------------------ */

@@ -35,6 +35,8 @@ def lib():
         _lib.lao_readout_rearranged.restype = None
         _lib.lao_scan.argtypes = [i, i, i, i, i, p, i, p, p, i, i, p, i, p, i, p, p, p, i, p, p, d, p]
         _lib.lao_scan.restype = i
+        _lib.lao_scan_ckpt.argtypes = _lib.lao_scan.argtypes + [i, p, p]
+        _lib.lao_scan_ckpt.restype = i
         _lib.lao_pool_copy.argtypes = [p, sz, i, i, p, p]
         _lib.lao_pool_gather.argtypes = [p, sz, i, i, p, p]
         _lib.lao_pool_scatter.argtypes = [p, sz, i, i, p, p]
@@ -134,9 +136,11 @@ def readout_rearranged(rule, n_qk_heads, state, q, k, v, g=None, beta=None, scal
 
 def scan(rule, n_qk_heads, cu_seqlens, q, k, v, g=None, beta=None, scale=1.0, *,
          src_pool=None, read_slot=None, dst_pool=None, dst_dtype="f64", write_slot=None,
-         io_dtype="f64", n_v_heads=None, d_v=None):
+         io_dtype="f64", n_v_heads=None, d_v=None, ckpt_every=0, ckpt_cu=None, ckpt_slots=None):
     """Token-serial scan over packed sequences.  Initial state from src_pool[read_slot]
-    (zero when read_slot is None).  Returns (dst_pool, o, err_bits)."""
+    (zero when read_slot is None).  With ckpt_every > 0, the state after every ckpt_every
+    tokens of sequence s goes to dst_pool[ckpt_slots[ckpt_cu[s] + j]] (see la_oracle.c).
+    Returns (dst_pool, o, err_bits)."""
     cu = _i32(cu_seqlens)
     n_seqs = cu.shape[0] - 1
     q, k, v = _f64(q), _f64(k), _f64(v)
@@ -150,10 +154,15 @@ def scan(rule, n_qk_heads, cu_seqlens, q, k, v, g=None, beta=None, scale=1.0, *,
     g = None if g is None else _f64(g)
     beta = None if beta is None else _f64(beta)
     o = np.zeros((T, hv, dv), dtype=np.float64)
-    err = lib().lao_scan(RULES[rule], n_qk_heads, hv, dk, dv, _ptr(src), n_src, _ptr(_i32(read_slot)),
-                         _ptr(dst_pool), dst_pool.shape[0], DTYPES[dst_dtype], _ptr(_i32(write_slot)),
-                         n_seqs, _ptr(cu), T, _ptr(q), _ptr(k), _ptr(v), DTYPES[io_dtype],
-                         _ptr(g), _ptr(beta), float(scale), _ptr(o))
+    args = (RULES[rule], n_qk_heads, hv, dk, dv, _ptr(src), n_src, _ptr(_i32(read_slot)),
+            _ptr(dst_pool), dst_pool.shape[0], DTYPES[dst_dtype], _ptr(_i32(write_slot)),
+            n_seqs, _ptr(cu), T, _ptr(q), _ptr(k), _ptr(v), DTYPES[io_dtype],
+            _ptr(g), _ptr(beta), float(scale), _ptr(o))
+    if ckpt_every > 0:
+        ccu, csl = _i32(ckpt_cu), _i32(ckpt_slots)
+        err = lib().lao_scan_ckpt(*args, int(ckpt_every), _ptr(ccu), _ptr(csl))
+    else:
+        err = lib().lao_scan(*args)
     return dst_pool, o, err
 
 

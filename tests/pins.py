@@ -439,7 +439,47 @@ def pin_pool_ops(orc):
     assert orc.pool_zero(p4, np.array([10], dtype=np.int32)) == 2
 
 
+def pin_scan_checkpoints(orc):
+    """Checkpoint j of a sequence is the state after its first (j + 1) * every tokens:
+    checked against the transition-product states at those positions, for every rule,
+    with a random initial state; a checkpoint beyond the sequence is reported (bit 4)."""
+    every = 4
+    for rule in W.RULES:
+        inp = W.scan_inputs(lengths=[21, 7, 0, 12], n_qk_heads=1, n_v_heads=2, d_k=16, d_v=16, rule=rule,
+                            state_dtype=torch.float32, io_dtype=torch.float32, seed=17)
+        init = np.random.default_rng(6).standard_normal((4, 2, 16, 16)) * 0.5
+        cu = inp.cu_seqlens.numpy()
+        lens = cu[1:] - cu[:-1]
+        n_ck = lens // every
+        ckpt_cu = np.concatenate([[0], np.cumsum(n_ck)]).astype(np.int32)
+        ckpt_slots = (4 + np.arange(ckpt_cu[-1])).astype(np.int32)
+        dst = np.zeros((4 + ckpt_cu[-1], 2, 16, 16))
+        S, o, err = orc.scan(rule, 1, cu, np64(inp.q), np64(inp.k), np64(inp.v), np64(inp.g), np64(inp.beta),
+                             src_pool=init, read_slot=np.arange(4, dtype=np.int32), dst_pool=dst,
+                             ckpt_every=every, ckpt_cu=ckpt_cu, ckpt_slots=ckpt_slots)
+        assert err == 0
+        q, k, v = np64(inp.q), np64(inp.k), np64(inp.v)
+        g, b = np64(inp.g), np64(inp.beta)
+        for sq in range(4):
+            t0, t1 = int(cu[sq]), int(cu[sq + 1])
+            for h in range(2):
+                states, _ = brute_force_head(rule, init[sq, h], q[t0:t1, 0], k[t0:t1, 0], v[t0:t1, h],
+                                             None if g is None else g[t0:t1, h], None if b is None else b[t0:t1, h])
+                for j in range(n_ck[sq]):
+                    close(S[ckpt_slots[ckpt_cu[sq] + j], h], states[(j + 1) * every - 1], 1e-9,
+                          f"{rule} seq {sq} head {h} checkpoint {j}")
+                close(S[sq, h], states[-1] if states else init[sq, h], 1e-9, f"{rule} final state")
+    # one checkpoint too many for sequence 1 (7 tokens, every 4): reported, the rest still written
+    bad_cu = ckpt_cu.copy()
+    bad_cu[2:] += 1
+    bad_slots = np.concatenate([ckpt_slots[:ckpt_cu[2]], [3], ckpt_slots[ckpt_cu[2]:]]).astype(np.int32)
+    _, _, err = orc.scan("gated_delta", 1, cu, np64(inp.q), np64(inp.k), np64(inp.v), np64(inp.g), np64(inp.beta),
+                         dst_pool=np.zeros_like(dst), ckpt_every=every, ckpt_cu=bad_cu, ckpt_slots=bad_slots)
+    assert err == 4
+
+
 ALL_PINS = [pin_bf16_rounding, pin_brute_force_all_rules, pin_gqa_grouping, pin_exact_rational,
             pin_linear_closed_form, pin_gated_closed_form, pin_beta0_g1_identity, pin_delta_stores_value,
             pin_rearranged_readout, pin_scan_structure, pin_wide_ranges_non_expansive,
-            pin_long_sequence_bounded, pin_storage_rounding_points, pin_slots, pin_pool_ops]
+            pin_long_sequence_bounded, pin_storage_rounding_points, pin_slots, pin_pool_ops,
+            pin_scan_checkpoints]

@@ -150,6 +150,19 @@ def test_scan_host_errors(lib):
     assert scan(lib, n=9) == L.LA_ERR_SHAPE
 
 
+def test_checkpointed_scan_host_errors(lib):
+    dst = pool()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+
+    def call(every=8, ccu=A, cs=A, n=2):
+        return lib.la_state_scan_checkpointed(3, None, None, ctypes.byref(dst), None, n, P(A), 10, None, P(A), P(A),
+                                              P(A), 1, P(A), P(A), 1.0, P(A), every, P(ccu), P(cs), P(A), None)
+    assert call(every=0) == L.LA_ERR_SHAPE
+    assert call(ccu=None) == L.LA_ERR_NULL
+    assert call(cs=A + 2) == L.LA_ERR_ALIGN
+    assert call(n=0) == L.LA_OK
+
+
 def test_pool_host_errors(lib):
     p = pool()
     P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731

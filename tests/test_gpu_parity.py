@@ -359,3 +359,65 @@ def test_pool_checkpoint_roundtrip_full_size():
     assert torch.equal(after[others.long()].view(torch.int16), inp.pool[live.long()].view(torch.int16))
     assert torch.equal(after[live.long()].view(torch.int16), inp.pool[live.long()].view(torch.int16))
     assert int(err.item()) == 0
+
+
+# ---- scan with intermediate checkpoints ------------------------------------------------
+
+def _ckpt_layout(lengths, every, extra_slot_base):
+    n_ck = [l // every for l in lengths]
+    cu = np.concatenate([[0], np.cumsum(n_ck)]).astype(np.int32)
+    slots = (extra_slot_base + np.arange(cu[-1])).astype(np.int32)
+    return cu, slots
+
+
+def _gpu_scan_ckpt(inp, every, ckpt_cu, ckpt_slots, n_dst, dst_dtype):
+    n_seqs = inp.cu_seqlens.numel() - 1
+    dst_t = torch.full((n_dst, inp.n_v_heads, inp.d_k, inp.d_v), 3.0, dtype=dst_dtype, device="cuda")
+    src = None if inp.pool is None else L.Pool(dev(inp.pool), inp.n_qk_heads)
+    o = torch.full((inp.q.shape[0], inp.n_v_heads, inp.d_v), 5.0, dtype=inp.io_dtype, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = L.la_state_scan_checkpointed(inp.rule, src, dev(inp.read_slot), L.Pool(dst_t, inp.n_qk_heads), None,
+                                      dev(inp.cu_seqlens), dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.g),
+                                      dev(inp.beta), inp.scale, o, every, dev(torch.as_tensor(ckpt_cu)),
+                                      dev(torch.as_tensor(ckpt_slots)), err)
+    L.check(st)
+    torch.cuda.synchronize()
+    assert n_seqs <= n_dst
+    return dst_t.cpu(), o.cpu(), int(err.item())
+
+
+@pytest.mark.parametrize("dst", [F32, BF16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("rule", W.RULES)
+def test_scan_checkpoints(rule, dst):
+    lengths, every = [37, 8, 0, 64, 5, 16], 8
+    inp = W.scan_inputs(lengths=lengths, n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128, rule=rule, io_dtype=BF16,
+                        seed=31, init="slots", init_dtype=F32)
+    ckpt_cu, ckpt_slots = _ckpt_layout(lengths, every, len(lengths))
+    n_dst = len(lengths) + int(ckpt_cu[-1])
+    S, o, err = _gpu_scan_ckpt(inp, every, ckpt_cu, ckpt_slots, n_dst, dst)
+    assert err == 0
+    ref_pool = np.zeros((n_dst, 4, 128, 128))
+    S_ref, o_ref, e = oracle.scan(rule, 2, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k), np64(inp.v),
+                                  np64(inp.g), np64(inp.beta), inp.scale, src_pool=np64(inp.pool),
+                                  read_slot=inp.read_slot.numpy(), dst_pool=ref_pool, dst_dtype=dname(dst),
+                                  io_dtype="bf16", ckpt_every=every, ckpt_cu=ckpt_cu, ckpt_slots=ckpt_slots)
+    assert e == 0
+    tol_s, tol_o = tolerances(dst, BF16)
+    assert_close(np64(S), S_ref, tol_s, f"{rule}: final states and checkpoints")
+    assert_close(np64(o), o_ref, tol_o, f"{rule}: outputs (unchanged by checkpointing)")
+    S_plain, o_plain, _ = gpu_scan(inp, dst_dtype=dst)
+    assert torch.equal(o, o_plain), "checkpoints must not change the outputs"
+
+
+def test_scan_checkpoint_errors_reported():
+    lengths, every = [9, 4], 4
+    inp = W.scan_inputs(lengths=lengths, n_qk_heads=1, n_v_heads=2, d_k=64, d_v=64, seed=32)
+    cu = np.array([0, 3, 4], dtype=np.int32)            # sequence 0 fits only 2 checkpoints
+    slots = np.array([2, 3, 4, 99], dtype=np.int32)      # slot 99 is outside the pool
+    S, o, err = _gpu_scan_ckpt(inp, every, cu, slots, 5, BF16)
+    assert err == (L.DEVERR_CU_SEQLENS | L.DEVERR_WRITE_SLOT)
+    S_ref, _, _ = oracle.scan("gated_delta", 1, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k), np64(inp.v),
+                              np64(inp.g), np64(inp.beta), dst_pool=np.zeros((5, 2, 64, 64)), dst_dtype="bf16",
+                              io_dtype="bf16", ckpt_every=every, ckpt_cu=np.array([0, 2, 3], dtype=np.int32),
+                              ckpt_slots=np.array([2, 3, 4], dtype=np.int32))
+    assert_close(np64(S[:4]), S_ref[:4], 2e-2, "checkpoints that fit are written")

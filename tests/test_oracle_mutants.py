@@ -33,6 +33,7 @@ MUTANTS = [
      "            free(u);\n        }\n    }\n\n    for (int b = 0;"),
     ("checkpoint_overwritten", "memcpy(dst_pool + (size_t)ws * slot, next + (size_t)b * slot, sizeof(double) * slot);",
      "memcpy(dst_pool + (size_t)(read_slot ? read_slot[b] : b) * slot, next + (size_t)b * slot, sizeof(double) * slot);"),
+    ("checkpoint_off_by_one", "const int pos = t - cu_seqlens[s] + 1;", "const int pos = t - cu_seqlens[s];"),
     ("gather_wrong_slot", "memcpy(dense + (size_t)i * slot_bytes, pool + (size_t)slots[i] * slot_bytes, slot_bytes);",
      "memcpy(dense + (size_t)i * slot_bytes, pool + (size_t)i * slot_bytes, slot_bytes);"),
 ]
