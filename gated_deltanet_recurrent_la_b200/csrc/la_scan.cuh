@@ -80,7 +80,7 @@ struct ScanCfg {
   static_assert(kRawBytes % 16 == 0 && kCvtBytes % 16 == 0, "alignment of staging buffers");
 };
 
-template <int RULE, int DK, int DV, typename IT, int MIN_BLOCKS>
+template <int RULE, int DK, int DV, typename IT, int MIN_BLOCKS, bool CKPT>
 __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) scan_kernel(const ScanParams p) {
   using C = ScanCfg<DK, DV, IT>;
   constexpr int R = C::kR;
@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
 
     // ---- checkpoints of this sequence: after (j + 1) * ckpt_every tokens, j < n_ck
     int n_ck = 0, ck_base = 0;
-    if (p.ckpt_every > 0) {
+    if (CKPT && p.ckpt_every > 0) {
       ck_base = __ldg(p.ckpt_cu + seq);
       n_ck = __ldg(p.ckpt_cu + seq + 1) - ck_base;
       const int fit = (t1 - t0) / p.ckpt_every;
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, IT>::kThreads, MIN_BLOCKS) sca
           for (int c = 0; c < KC; ++c) up[c] = uu[c];
         }
         kp = kc;
-        if (ck_j < n_ck && --ck_left == 0) {
+        if (CKPT && ck_j < n_ck && --ck_left == 0) {
           // checkpoint: apply this token's update now and store the state
           ck_left = p.ckpt_every;
 #pragma unroll
@@ -402,13 +402,20 @@ template <int RULE, int DK, int DV, typename IT>
 cudaError_t launch_scan(const ScanParams& p, cudaStream_t stream) {
   using C = ScanCfg<DK, DV, IT>;
   constexpr int kMinBlocks = 2;  // two CTAs (units) per SM
-  const void* fn = reinterpret_cast<const void*>(&scan_kernel<RULE, DK, DV, IT, kMinBlocks>);
+  // checkpoints are a separate instantiation so that the plain scan's loop carries no
+  // checkpoint bookkeeping
+  const bool ck = p.ckpt_every > 0;
+  const void* fn = ck ? reinterpret_cast<const void*>(&scan_kernel<RULE, DK, DV, IT, kMinBlocks, true>)
+                      : reinterpret_cast<const void*>(&scan_kernel<RULE, DK, DV, IT, kMinBlocks, false>);
   const int per_sm = prepare_kernel(fn, C::kThreads, C::kSmem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;
   const int64_t units = (int64_t)p.n_seqs * p.n_v_heads;
   const int64_t cap = (int64_t)device_sm_count() * per_sm;
   const int grid = (int)(units < cap ? units : cap);
-  scan_kernel<RULE, DK, DV, IT, kMinBlocks><<<grid, C::kThreads, C::kSmem, stream>>>(p);
+  if (ck)
+    scan_kernel<RULE, DK, DV, IT, kMinBlocks, true><<<grid, C::kThreads, C::kSmem, stream>>>(p);
+  else
+    scan_kernel<RULE, DK, DV, IT, kMinBlocks, false><<<grid, C::kThreads, C::kSmem, stream>>>(p);
   return cudaGetLastError();
 }
 
