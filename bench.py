@@ -310,7 +310,7 @@ class ScanRunner:
     """A prefill workload on the device.  ckpt_every > 0: la_state_scan_checkpointed with a
     checkpoint slot for every ckpt_every tokens of every sequence."""
 
-    def __init__(self, inp, ckpt_every=0):
+    def __init__(self, inp, ckpt_every=0, chunked=False):
         import torch
         from gated_deltanet_recurrent_la_b200 import lastate as L
         self.L = L
@@ -331,6 +331,7 @@ class ScanRunner:
         self.T = int(inp.q.shape[0])
         self.n_seqs = n_seqs
         self.ckpt_every = ckpt_every
+        self.chunked = chunked
         self.n_ckpt = 0
         if ckpt_every > 0:
             n_ck = [l // ckpt_every for l in lens]
@@ -345,7 +346,11 @@ class ScanRunner:
             self.dst = L.Pool(self.dst_t, inp.n_qk_heads)
 
     def step(self, i=0, stream=None):
-        if self.ckpt_every > 0:
+        if self.chunked:
+            st = self.L.la_state_scan_chunked(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu, self.q,
+                                              self.k, self.v, self.g, self.beta, self.inp.scale, self.o, self.err,
+                                              seq_order=self.order, stream=stream)
+        elif self.ckpt_every > 0:
             st = self.L.la_state_scan_checkpointed(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu,
                                                    self.q, self.k, self.v, self.g, self.beta, self.inp.scale, self.o,
                                                    self.ckpt_every, self.ckpt_cu, self.ckpt_slots, self.err,
@@ -589,11 +594,11 @@ def cpu_baseline_decode(inp, budget_s=10.0):
 # --------------------------------------------------------------------------------------
 
 
-def build_runner(name, seed=0, prefill_seqs=32, ckpt_every=0):
+def build_runner(name, seed=0, prefill_seqs=32, ckpt_every=0, chunked=False):
     from gated_deltanet_recurrent_la_b200 import workloads as W
     inp = W.prefill32(seed, prefill_seqs) if name == "prefill32" else W.WORKLOADS[name](seed)
     if inp.kind == "scan":
-        return ScanRunner(inp, ckpt_every), inp
+        return ScanRunner(inp, ckpt_every, chunked), inp
     n_sets = 4 if name == "decode64" else 1
     return DecodeRunner(inp, n_sets=n_sets, seed=seed), inp
 
@@ -614,8 +619,8 @@ def describe(name, inp):
     return d
 
 
-def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_every=0):
-    run, inp = build_runner(name, ckpt_every=ckpt_every)
+def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_every=0, chunked=False):
+    run, inp = build_runner(name, ckpt_every=ckpt_every, chunked=chunked)
     ms = time_back_to_back(run, steps, warmup, world)
     nbytes, flops = run.bytes_flops()
     row = {"config": describe(name, inp), "ms_per_step": ms, "gb_s": nbytes / (ms * 1e-3) / 1e9}
@@ -635,6 +640,11 @@ def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_ev
         if ckpt_every:
             row["config"]["ckpt_every"] = ckpt_every
             row["config"]["checkpoints"] = run.n_ckpt
+        if chunked:
+            row["config"]["algorithm"] = "chunked (64-token WY/UT form, BF16 tensor-core products)"
+            # the same algorithmic flops as the token-serial form (6 per state element per token);
+            # the chunked form executes more multiply-adds, on the tensor cores
+            row["hbm"] = {"achieved_gb_s": row["gb_s"], "frac_of_measured": row["gb_s"] / peaks["hbm_gbs"]}
         row["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
                            "traffic": recorded_traffic("scan", name), "hbm_gb_s": row["gb_s"],
                            "effective_state_gb_s": run.T * inp.n_v_heads * 2 * inp.d_k * inp.d_v * 4 / (ms * 1e-3) / 1e9,
@@ -723,6 +733,9 @@ def main():
             torch.cuda.empty_cache()
         rows["prefill32_ckpt256"] = measure_row("prefill32", max(3, min(a.steps, 20)), a.warmup, world, peaks,
                                                 sm_count, None, ckpt_every=256)
+        torch.cuda.empty_cache()
+        rows["prefill32_chunked"] = measure_row("prefill32", max(3, min(a.steps, 50)), a.warmup, world, peaks,
+                                                sm_count, None, chunked=True)
         torch.cuda.empty_cache()
         pool_run = PoolRunner()
         pms = time_back_to_back(pool_run, min(a.steps, 500), a.warmup, world)

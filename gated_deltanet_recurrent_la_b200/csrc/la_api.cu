@@ -158,7 +158,8 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
                            const int32_t* write_slot, int32_t n_seqs, const int32_t* cu_seqlens, int32_t total_tokens,
                            const int32_t* seq_order, const void* q, const void* k, const void* v, la_dtype io,
                            const float* g, const float* beta, float scale, void* o, int32_t ckpt_every,
-                           const int32_t* ckpt_cu, const int32_t* ckpt_slots, int32_t* err_word, void* stream) {
+                           const int32_t* ckpt_cu, const int32_t* ckpt_slots, int32_t* err_word, void* stream,
+                           bool chunked = false) {
   if (rule < LA_RULE_LINEAR || rule > LA_RULE_GATED_DELTA) return LA_ERR_UNSUPPORTED;
   if (!err_word) return LA_ERR_NULL;
   if (n_seqs < 0 || total_tokens < 0) return LA_ERR_SHAPE;
@@ -185,7 +186,13 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
   if (!write_slot && n_seqs > dst->n_slots) return LA_ERR_SHAPE;
   if ((int64_t)n_seqs * s.n_v_heads > INT32_MAX) return LA_ERR_SHAPE;
 
-  la::ScanLaunchFn fn = (io == LA_F32) ? la::find_scan_f32io(rule, s.d_k, s.d_v) : la::find_scan_bf16io(rule, s.d_k, s.d_v);
+  la::ScanLaunchFn fn = nullptr;
+  if (chunked) {
+    if (s.d_k != 128 || s.d_v != 128 || io != LA_BF16) return LA_ERR_UNSUPPORTED;
+    fn = la::find_chunk_scan(rule);
+  } else {
+    fn = (io == LA_F32) ? la::find_scan_f32io(rule, s.d_k, s.d_v) : la::find_scan_bf16io(rule, s.d_k, s.d_v);
+  }
   if (!fn) return LA_ERR_UNSUPPORTED;
   la::ScanParams p;
   p.src = read_slot ? src->data : nullptr;
@@ -222,6 +229,15 @@ la_status la_state_scan(la_rule rule, const la_pool* src, const int32_t* read_sl
                         const float* g, const float* beta, float scale, void* o, int32_t* err_word, void* stream) {
   return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, q, k, v, io,
                    g, beta, scale, o, 0, nullptr, nullptr, err_word, stream);
+}
+
+la_status la_state_scan_chunked(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
+                                const int32_t* write_slot, int32_t n_seqs, const int32_t* cu_seqlens,
+                                int32_t total_tokens, const int32_t* seq_order, const void* q, const void* k,
+                                const void* v, la_dtype io, const float* g, const float* beta, float scale, void* o,
+                                int32_t* err_word, void* stream) {
+  return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, q, k, v, io,
+                   g, beta, scale, o, 0, nullptr, nullptr, err_word, stream, true);
 }
 
 la_status la_state_scan_checkpointed(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,

@@ -80,6 +80,9 @@ StepLaunchFn find_step_bf16(int rule, int dk, int dv, int io);
 ScanLaunchFn find_scan_f32io(int rule, int dk, int dv);
 ScanLaunchFn find_scan_bf16io(int rule, int dk, int dv);
 
+// Chunked tensor-core prefill (d_k = d_v = 128, BF16 io); nullptr for an unknown rule.
+ScanLaunchFn find_chunk_scan(int rule);
+
 cudaError_t launch_pool_copy(const PoolCopyParams& p, cudaStream_t stream);
 
 // Streaming multiprocessors of the current device (cached per device).

@@ -27,7 +27,8 @@ STATUS = {0: "LA_OK", 1: "LA_ERR_NULL", 2: "LA_ERR_SHAPE", 3: "LA_ERR_UNSUPPORTE
 LA_OK, LA_ERR_NULL, LA_ERR_SHAPE, LA_ERR_UNSUPPORTED, LA_ERR_ALIGN, LA_ERR_ALIAS, LA_ERR_CUDA = range(7)
 DEVERR_READ_SLOT, DEVERR_WRITE_SLOT, DEVERR_CU_SEQLENS, DEVERR_TIMEOUT = 1, 2, 4, 8
 
-EXPORTS = ("la_state_bytes", "la_shape_supported", "la_state_step", "la_state_scan", "la_state_scan_checkpointed",
+EXPORTS = ("la_state_bytes", "la_shape_supported", "la_state_step", "la_state_scan", "la_state_scan_chunked",
+           "la_state_scan_checkpointed",
            "la_state_pool_copy",
            "la_state_pool_gather", "la_state_pool_scatter", "la_state_pool_zero", "la_state_check_slots",
            "la_status_str", "la_last_cuda_error", "la_abi_version")
@@ -73,6 +74,8 @@ def lib():
         L.la_state_step.restype = I32
         L.la_state_scan.argtypes = [I32, PP, P, PP, P, I32, P, I32, P, P, P, P, I32, P, P, F, P, P, P]
         L.la_state_scan.restype = I32
+        L.la_state_scan_chunked.argtypes = L.la_state_scan.argtypes
+        L.la_state_scan_chunked.restype = I32
         L.la_state_scan_checkpointed.argtypes = L.la_state_scan.argtypes[:-2] + [I32, P, P, P, P]
         L.la_state_scan_checkpointed.restype = I32
         L.la_state_pool_copy.argtypes = [PP, I32, P, P, P, P]
@@ -167,6 +170,18 @@ def la_state_scan(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, c
                                _ptr(q), _ptr(k, q.dtype), _ptr(v, q.dtype), io, _ptr(g, torch.float32),
                                _ptr(beta, torch.float32), float(scale), _ptr(o, q.dtype),
                                _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_state_scan_chunked(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens, q, k, v, g, beta,
+                          scale, o, err_word, seq_order=None, stream=None) -> int:
+    io = dtype_code(q.dtype)
+    return lib().la_state_scan_chunked(RULES[rule] if isinstance(rule, str) else int(rule),
+                                       None if src is None else src.ref, _ptr(read_slot, torch.int32), dst.ref,
+                                       _ptr(write_slot, torch.int32), int(cu_seqlens.numel() - 1),
+                                       _ptr(cu_seqlens, torch.int32), int(q.shape[0]), _ptr(seq_order, torch.int32),
+                                       _ptr(q), _ptr(k, q.dtype), _ptr(v, q.dtype), io, _ptr(g, torch.float32),
+                                       _ptr(beta, torch.float32), float(scale), _ptr(o, q.dtype),
+                                       _ptr(err_word, torch.int32), _stream(stream))
 
 
 def la_state_scan_checkpointed(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens, q, k, v, g,

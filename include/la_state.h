@@ -160,6 +160,22 @@ la_status la_state_scan(la_rule rule, const la_pool *src, const int32_t *read_sl
                         const float *g, const float *beta, float scale, void *o,
                         int32_t *err_word, void *stream);
 
+/* The scan of la_state_scan evaluated in chunks of 64 tokens on the tensor cores: the
+ * chunkwise-parallel form of the "Kimi Linear" section and the chunkwise WY algorithm of
+ * the "Gated DeltaNet-2" section of "Seven Architectures ...".  Within a chunk the
+ * delta-rule corrections are solved exactly with a triangular (UT) transform; the
+ * products run with BF16 operands and FP32 accumulation, and the state stays in FP32
+ * across the sequence.  Results agree with la_state_scan to BF16 precision (about 5e-3 of
+ * the largest output over thousands of tokens), not bit for bit.
+ * Arguments, outputs and errors as la_state_scan.  Supported: d_k = d_v = 128 with BF16
+ * q/k/v/o (LA_ERR_UNSUPPORTED otherwise); any rule; gates of either sign. */
+la_status la_state_scan_chunked(la_rule rule, const la_pool *src, const int32_t *read_slot,
+                                const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
+                                const int32_t *cu_seqlens, int32_t total_tokens, const int32_t *seq_order,
+                                const void *q, const void *k, const void *v, la_dtype io,
+                                const float *g, const float *beta, float scale, void *o,
+                                int32_t *err_word, void *stream);
+
 /* The scan of la_state_scan that also stores intermediate states: the prefix-cache
  * checkpoints "aligned to KV block boundaries" of the "Gated DeltaNet" glossary page (Why
  * it matters), and state snapshots for speculative-decoding rollback ("Seven

@@ -150,6 +150,18 @@ def test_scan_host_errors(lib):
     assert scan(lib, n=9) == L.LA_ERR_SHAPE
 
 
+def test_chunked_scan_supported_set(lib):
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+
+    def call(shape=(2, 4, 128, 128), io=1):
+        dst = pool(shape=shape)
+        return lib.la_state_scan_chunked(3, None, None, ctypes.byref(dst), None, 2, P(A), 10, None, P(A), P(A), P(A),
+                                         io, P(A), P(A), 1.0, P(A), P(A), None)
+    assert call(shape=(2, 4, 64, 64)) == L.LA_ERR_UNSUPPORTED
+    assert call(shape=(2, 4, 128, 64)) == L.LA_ERR_UNSUPPORTED
+    assert call(io=0) == L.LA_ERR_UNSUPPORTED
+
+
 def test_checkpointed_scan_host_errors(lib):
     dst = pool()
     P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731

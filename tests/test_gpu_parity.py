@@ -421,3 +421,58 @@ def test_scan_checkpoint_errors_reported():
                               io_dtype="bf16", ckpt_every=every, ckpt_cu=np.array([0, 2, 3], dtype=np.int32),
                               ckpt_slots=np.array([2, 3, 4], dtype=np.int32))
     assert_close(np64(S[:4]), S_ref[:4], 2e-2, "checkpoints that fit are written")
+
+
+# ---- chunked tensor-core prefill (BF16 operands: compared at the BF16 tolerance) ----------
+
+def _gpu_scan_chunked(inp, dst_dtype):
+    n_seqs = inp.cu_seqlens.numel() - 1
+    dst_t = torch.full((n_seqs, inp.n_v_heads, inp.d_k, inp.d_v), 3.0, dtype=dst_dtype, device="cuda")
+    src = None if inp.pool is None else L.Pool(dev(inp.pool), inp.n_qk_heads)
+    o = torch.full((inp.q.shape[0], inp.n_v_heads, inp.d_v), 5.0, dtype=inp.io_dtype, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = L.la_state_scan_chunked(inp.rule, src, dev(inp.read_slot), L.Pool(dst_t, inp.n_qk_heads), None,
+                                 dev(inp.cu_seqlens), dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.g), dev(inp.beta),
+                                 inp.scale, o, err)
+    L.check(st)
+    torch.cuda.synchronize()
+    return dst_t.cpu(), o.cpu(), int(err.item())
+
+
+@pytest.mark.parametrize("dst", [F32, BF16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("rule", W.RULES)
+def test_chunked_scan_vs_oracle(rule, dst):
+    inp = W.scan_inputs(lengths=[100, 64, 1, 0, 200, 63, 129], n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128,
+                        rule=rule, io_dtype=BF16, seed=41, init="slots", init_dtype=F32, scale=0.8)
+    S, o, err = _gpu_scan_chunked(inp, dst)
+    assert err == 0
+    S_ref, o_ref, e = oracle_scan(inp, dst_dtype=dst)
+    assert e == 0
+    assert_close(np64(S), S_ref, 2e-2, f"{rule}: final states")
+    assert_close(np64(o), o_ref, 2e-2, f"{rule}: outputs")
+
+
+def test_chunked_scan_wide_gate_and_beta_ranges():
+    inp = W.scan_inputs(lengths=[300, 70], n_qk_heads=1, n_v_heads=2, d_k=128, d_v=128, io_dtype=BF16, seed=42,
+                        g_mode="uniform_pm1", beta_mode="uniform_0_2", init="slots", init_dtype=F32)
+    S, o, err = _gpu_scan_chunked(inp, F32)
+    S_ref, o_ref, _ = oracle_scan(inp, dst_dtype=F32)
+    assert err == 0
+    assert_close(np64(S), S_ref, 2e-2, "wide-range final states")
+    assert_close(np64(o), o_ref, 2e-2, "wide-range outputs")
+
+
+def test_chunked_prefill32_sampled():
+    inp = W.prefill32()
+    S, o, err = _gpu_scan_chunked(inp, BF16)
+    assert err == 0
+    cu = inp.cu_seqlens.numpy()
+    order = np.argsort(cu[1:] - cu[:-1])
+    for s, h in [(int(order[0]), 3), (int(order[-1]), 29)]:
+        t0, t1 = int(cu[s]), int(cu[s + 1])
+        sub = W.Inputs("scan", inp.rule, 1, 1, 128, 128, BF16, BF16, inp.q[t0:t1, h:h + 1], inp.k[t0:t1, h:h + 1],
+                       inp.v[t0:t1, h:h + 1], inp.g[t0:t1, h:h + 1], inp.beta[t0:t1, h:h + 1], 1.0, None, None, None,
+                       torch.tensor([0, t1 - t0], dtype=torch.int32))
+        S_ref, o_ref, _ = oracle_scan(sub)
+        assert_close(np64(S[s, h]), S_ref[0, 0], 2e-2, f"seq {s} head {h} final state")
+        assert_close(np64(o[t0:t1, h]), o_ref[:, 0], 2e-2, f"seq {s} head {h} outputs")
