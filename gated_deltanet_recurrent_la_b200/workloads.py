@@ -9,7 +9,7 @@ either side sees them.
 Distributions (the workloads the pages describe; no dataset is involved):
   q, k ~ N(0, 1), each head vector L2-normalised     (delta-rule keys are unit vectors)
   v    ~ N(0, 1)
-  g    = exp(-softplus(N(0, 1)))                      gate in (0, 1)
+  g    = exp(-softplus(N(0, 1)))                      gate in (0, 1); kda: one per key channel
   beta = sigmoid(N(0, 1))                             write strength in (0, 1)
   pool = N(0, 0.05) initial states (decode workloads)
 
@@ -20,6 +20,7 @@ Named workloads (sizes from the "SSM / linear-RNN decode" page, the ONNX section
   decode512   B=512, same heads, 1024-slot pool, half the requests read a checkpoint slot
   prefill32   32 packed sequences, lengths U_int[1024, 8192], 32 heads, 128 x 128 scan
   mamba2      B=256 gated decode, 128 heads x 64, d_state 128 (Nemotron-H-8B layer sizes)
+  kda_decode64, kda_prefill32   the same shapes with the channel-wise (kda) gate
 """
 from __future__ import annotations
 
@@ -29,6 +30,8 @@ from typing import Optional
 import torch
 
 RULES = ("linear", "gated", "delta", "gated_delta")
+# kda: the channel-wise gate of Kimi Delta Attention (g holds d_k decays per token and head)
+ALL_RULES = RULES + ("kda",)
 
 
 def _gen(seed: int) -> torch.Generator:
@@ -55,7 +58,7 @@ class Inputs:
     q: torch.Tensor                # [B|T, H_qk, d_k] io dtype
     k: torch.Tensor
     v: torch.Tensor                # [B|T, H_v, d_v] io dtype
-    g: Optional[torch.Tensor]      # [B|T, H_v] float32
+    g: Optional[torch.Tensor]      # [B|T, H_v] float32 ([B|T, H_v, d_k] for kda)
     beta: Optional[torch.Tensor]
     scale: float = 1.0
     pool: Optional[torch.Tensor] = None        # source pool [n_slots, H_v, d_k, d_v]
@@ -70,21 +73,23 @@ class Inputs:
 
 
 def token_operands(n_tok, n_qk_heads, n_v_heads, d_k, d_v, io_dtype, gen, *, normalise_qk=True,
-                   g_mode="exp_neg_softplus", beta_mode="sigmoid"):
-    """q, k, v, g, beta for n_tok tokens (or requests), drawn in that order from gen."""
+                   g_mode="exp_neg_softplus", beta_mode="sigmoid", channel_gate=False):
+    """q, k, v, g, beta for n_tok tokens (or requests), drawn in that order from gen.
+    channel_gate: g has one decay per key channel, [n_tok, H_v, d_k] (kda)."""
     q = torch.randn(n_tok, n_qk_heads, d_k, generator=gen)
     k = torch.randn(n_tok, n_qk_heads, d_k, generator=gen)
     if normalise_qk:
         q, k = _unit(q), _unit(k)
     v = torch.randn(n_tok, n_v_heads, d_v, generator=gen)
-    zg = torch.randn(n_tok, n_v_heads, generator=gen)
+    gshape = (n_tok, n_v_heads, d_k) if channel_gate else (n_tok, n_v_heads)
+    zg = torch.randn(*gshape, generator=gen)
     zb = torch.randn(n_tok, n_v_heads, generator=gen)
     if g_mode == "exp_neg_softplus":
         g = torch.exp(-torch.nn.functional.softplus(zg))
     elif g_mode == "uniform_pm1":          # gate range [-1, 1] ("Complex KDA" section)
-        g = torch.rand(n_tok, n_v_heads, generator=gen) * 2 - 1
+        g = torch.rand(*gshape, generator=gen) * 2 - 1
     elif g_mode == "one":
-        g = torch.ones(n_tok, n_v_heads)
+        g = torch.ones(*gshape)
     else:
         raise ValueError(g_mode)
     if beta_mode == "sigmoid":
@@ -135,7 +140,8 @@ def step_inputs(*, B, n_qk_heads, n_v_heads, d_k, d_v, rule="gated_delta", n_slo
     elif slot_map != "dense":
         raise ValueError(slot_map)
     q, k, v, g, beta = token_operands(B, n_qk_heads, n_v_heads, d_k, d_v, io_dtype, gen,
-                                      normalise_qk=normalise_qk, g_mode=g_mode, beta_mode=beta_mode)
+                                      normalise_qk=normalise_qk, g_mode=g_mode, beta_mode=beta_mode,
+                                      channel_gate=rule == "kda")
     return Inputs("step", rule, n_qk_heads, n_v_heads, d_k, d_v, state_dtype, io_dtype, q, k, v, g, beta,
                   scale, pool, read_slot, write_slot)
 
@@ -160,7 +166,8 @@ def scan_inputs(*, lengths, n_qk_heads, n_v_heads, d_k, d_v, rule="gated_delta",
     elif init != "zero":
         raise ValueError(init)
     q, k, v, g, beta = token_operands(T, n_qk_heads, n_v_heads, d_k, d_v, io_dtype, gen,
-                                      normalise_qk=normalise_qk, g_mode=g_mode, beta_mode=beta_mode)
+                                      normalise_qk=normalise_qk, g_mode=g_mode, beta_mode=beta_mode,
+                                      channel_gate=rule == "kda")
     return Inputs("scan", rule, n_qk_heads, n_v_heads, d_k, d_v, state_dtype, io_dtype, q, k, v, g, beta,
                   scale, pool, read_slot, None, cu)
 
@@ -180,6 +187,12 @@ def decode64(seed: int = 0) -> Inputs:
                        slot_map="perm")
 
 
+def kda_decode64(seed: int = 0) -> Inputs:
+    """decode64 with the channel-wise gate of Kimi Delta Attention (d_k decays per head)."""
+    return step_inputs(B=64, n_qk_heads=16, n_v_heads=32, d_k=128, d_v=128, n_slots=256, seed=seed,
+                       slot_map="perm", rule="kda")
+
+
 def decode512(seed: int = 0) -> Inputs:
     """Large decode: B=512, same heads, 1024-slot pool; half the requests read a
     checkpoint slot and write a distinct live slot, the rest update in place."""
@@ -196,6 +209,12 @@ def prefill32(seed: int = 0, n_seqs: int = 32) -> Inputs:
     128 x 128, FP32 state on chip, zero initial state, BF16 final state and io."""
     return scan_inputs(lengths=prefill32_lengths(seed, n_seqs), n_qk_heads=32, n_v_heads=32, d_k=128,
                        d_v=128, seed=seed + 1)
+
+
+def kda_prefill32(seed: int = 0, n_seqs: int = 32) -> Inputs:
+    """prefill32 with the channel-wise gate of Kimi Delta Attention."""
+    return scan_inputs(lengths=prefill32_lengths(seed, n_seqs), n_qk_heads=32, n_v_heads=32, d_k=128,
+                       d_v=128, seed=seed + 1, rule="kda")
 
 
 def mamba2(seed: int = 0, B: int = 256) -> Inputs:
@@ -224,4 +243,6 @@ WORKLOADS = {
     "decode512": decode512,
     "prefill32": prefill32,
     "mamba2": mamba2,
+    "kda_decode64": kda_decode64,
+    "kda_prefill32": kda_prefill32,
 }

@@ -13,8 +13,9 @@
  *   "ONNX LinearAttention / FlashInfer": update_rule in {linear (basic additive),
  *   gated (exponential decay), delta (delta rule without decay), gated_delta}; state
  *   tensors past_state / present_state of shape (B, H_kv, d_k, d_v).
- *   Same page, section "Kimi Linear": S_t = Diag(a) S_{t-1} + b k (v - Diag(a) S_{t-1}^T k)^T,
- *   read here with a scalar gate (the Gated DeltaNet special case).
+ *   Same page, section "Kimi Linear": the channel-wise gate of Kimi Delta Attention,
+ *   S_t = Diag(alpha_t) S_{t-1} + beta_t k_t (v_t - (Diag(alpha_t) S_{t-1})^T k_t)^T with
+ *   alpha_t in R^{d_k} (rule kda); with a scalar gate it is the Gated DeltaNet rule.
  *
  * Per state head, with S (d_k x d_v), per token t:
  *
@@ -27,6 +28,11 @@
  *   gated        g_t   1      0
  *   delta        1     beta_t 1
  *   gated_delta  g_t   beta_t g_t
+ *   kda          Diag(alpha_t) beta_t, prediction from the decayed state Diag(alpha_t) S_{t-1}
+ *
+ * For kda the gate array holds d_k values per (token, head): row i of the state decays by
+ * alpha_t[i].  The formula's "Diag(alpha_t) S_{t-1}^T k_t" is read as the transpose of the
+ * decayed state times k (the only reading whose shapes agree when d_k != d_v).
  *
  * Arithmetic is IEEE double throughout.  Rounding happens only where the method
  * stores a value ("Recurrent state" glossary, Why it matters: state stored in BF16
@@ -38,7 +44,7 @@
  *   pool   [n_slots, H_v, d_k, d_v]
  *   q, k   [B or T, H_qk, d_k]        state head h reads q/k head h / (H_v / H_qk)
  *   v, o   [B or T, H_v, d_v]
- *   g, beta[B or T, H_v]
+ *   g, beta[B or T, H_v]               (kda: g is [B or T, H_v, d_k])
  *
  * Slots ("Recurrent state" glossary, Engineering details / Why it matters; "Gated
  * DeltaNet" glossary, Why it matters): a request reads its state from read_slot[b]
@@ -103,20 +109,26 @@ static void rule_coefficients(int rule, double g, double beta, double *a, double
 }
 
 /* S (dk x dv, in/out) <- a S + k u^T with u = b (v - c S^T k); o = scale * S_new^T q.
- * u is scratch of length dv. */
+ * For kda (alpha != NULL, dk values): S <- Diag(alpha) S + k u^T with
+ * u = beta (v - (Diag(alpha) S)^T k).  u is scratch of length dv. */
 static void token_update(int rule, int dk, int dv, double *S, const double *q, const double *k,
-                         const double *v, double g, double beta, double scale, double *o, double *u)
+                         const double *v, double g, const double *alpha, double beta, double scale,
+                         double *o, double *u)
 {
     double a, b, c;
     rule_coefficients(rule, g, beta, &a, &b, &c);
+    if (rule == LAO_RULE_KDA) { b = beta; c = 1.0; }
     for (int j = 0; j < dv; ++j) {
-        double pj = 0.0; /* (S^T k)_j */
-        for (int i = 0; i < dk; ++i) pj += S[(size_t)i * dv + j] * k[i];
+        double pj = 0.0; /* (S^T k)_j, or ((Diag(alpha) S)^T k)_j */
+        for (int i = 0; i < dk; ++i)
+            pj += (rule == LAO_RULE_KDA ? alpha[i] * S[(size_t)i * dv + j] : S[(size_t)i * dv + j]) * k[i];
         u[j] = b * (v[j] - c * pj);
     }
-    for (int i = 0; i < dk; ++i)
+    for (int i = 0; i < dk; ++i) {
+        const double ai = rule == LAO_RULE_KDA ? alpha[i] : a;
         for (int j = 0; j < dv; ++j)
-            S[(size_t)i * dv + j] = a * S[(size_t)i * dv + j] + k[i] * u[j];
+            S[(size_t)i * dv + j] = ai * S[(size_t)i * dv + j] + k[i] * u[j];
+    }
     for (int j = 0; j < dv; ++j) {
         double oj = 0.0; /* (S_new^T q)_j */
         for (int i = 0; i < dk; ++i) oj += S[(size_t)i * dv + j] * q[i];
@@ -169,7 +181,8 @@ int lao_step(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
                          q + ((size_t)b * n_qk_heads + hq) * dk,
                          k + ((size_t)b * n_qk_heads + hq) * dk,
                          v + ((size_t)b * n_v_heads + h) * dv,
-                         g ? g[(size_t)b * n_v_heads + h] : 1.0,
+                         g && rule != LAO_RULE_KDA ? g[(size_t)b * n_v_heads + h] : 1.0,
+                         rule == LAO_RULE_KDA ? g + ((size_t)b * n_v_heads + h) * dk : NULL,
                          beta ? beta[(size_t)b * n_v_heads + h] : 1.0,
                          scale, ob, u);
             for (int j = 0; j < dv; ++j) ob[j] = lao_round_to(ob[j], io_dtype);
@@ -207,16 +220,21 @@ void lao_readout_rearranged(int rule, int n_qk_heads, int n_v_heads, int dk, int
             const double *qb = q + ((size_t)b * n_qk_heads + hq) * dk;
             const double *kb = k + ((size_t)b * n_qk_heads + hq) * dk;
             const double *vb = v + ((size_t)b * n_v_heads + h) * dv;
+            const int kda = rule == LAO_RULE_KDA;
+            const double *al = kda ? g + ((size_t)b * n_v_heads + h) * dk : NULL;
             double a, bc, c;
-            rule_coefficients(rule, g ? g[(size_t)b * n_v_heads + h] : 1.0,
+            rule_coefficients(rule, g && !kda ? g[(size_t)b * n_v_heads + h] : 1.0,
                               beta ? beta[(size_t)b * n_v_heads + h] : 1.0, &a, &bc, &c);
+            if (kda) { a = 1.0; c = 1.0; }
             double kq = 0.0;
             for (int i = 0; i < dk; ++i) kq += kb[i] * qb[i];
             for (int j = 0; j < dv; ++j) {
+                /* kda: the decay sits on each row, so (Diag(alpha) S)^T k and (Diag(alpha) S)^T q */
                 double pj = 0.0, rj = 0.0;
                 for (int i = 0; i < dk; ++i) {
-                    pj += S[(size_t)i * dv + j] * kb[i];
-                    rj += S[(size_t)i * dv + j] * qb[i];
+                    const double sij = kda ? al[i] * S[(size_t)i * dv + j] : S[(size_t)i * dv + j];
+                    pj += sij * kb[i];
+                    rj += sij * qb[i];
                 }
                 double uj = bc * (vb[j] - c * pj);
                 o[((size_t)b * n_v_heads + h) * dv + j] = scale * (a * rj + kq * uj);
@@ -285,7 +303,8 @@ int lao_scan_ckpt(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
                              q + ((size_t)t * n_qk_heads + hq) * dk,
                              k + ((size_t)t * n_qk_heads + hq) * dk,
                              v + ((size_t)t * n_v_heads + h) * dv,
-                             g ? g[(size_t)t * n_v_heads + h] : 1.0,
+                             g && rule != LAO_RULE_KDA ? g[(size_t)t * n_v_heads + h] : 1.0,
+                             rule == LAO_RULE_KDA ? g + ((size_t)t * n_v_heads + h) * dk : NULL,
                              beta ? beta[(size_t)t * n_v_heads + h] : 1.0,
                              scale, ot, u);
                 for (int j = 0; j < dv; ++j) ot[j] = lao_round_to(ot[j], io_dtype);

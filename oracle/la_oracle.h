@@ -12,6 +12,7 @@
 #define LAO_RULE_GATED 1
 #define LAO_RULE_DELTA 2
 #define LAO_RULE_GATED_DELTA 3
+#define LAO_RULE_KDA 4
 
 #define LAO_F64 0
 #define LAO_F32 1

@@ -12,7 +12,7 @@ import numpy as np
 
 from . import build as _build
 
-RULES = {"linear": 0, "gated": 1, "delta": 2, "gated_delta": 3}
+RULES = {"linear": 0, "gated": 1, "delta": 2, "gated_delta": 3, "kda": 4}
 DTYPES = {"f64": 0, "f32": 1, "bf16": 2}
 
 _lib = None

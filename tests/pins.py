@@ -9,7 +9,9 @@ What the pins rest on (none of them re-types the oracle's recurrence):
   * the matrix (transition) form of each rule: gated_delta as
     S_t = g (I - beta k k^T) S_{t-1} + beta k v^T  ("Seven Architectures ...", section
     "Gated DeltaNet-2": b = w = beta with a scalar decay recovers Gated DeltaNet), delta
-    without the decay, gated as g S + k v^T and linear as S + k v^T (ONNX section),
+    without the decay, gated as g S + k v^T and linear as S + k v^T (ONNX section), and
+    kda as the diagonal-plus-low-rank transition (I - beta k k^T) Diag(alpha) S_{t-1} +
+    beta k v^T (section "Kimi Linear": a rank-one correction of the decayed state),
     evaluated as explicit products of d_k x d_k transition matrices in extended
     precision, and in exact rational arithmetic on the smallest shapes;
   * closed forms of the linear and gated rules (sums of outer products);
@@ -57,6 +59,9 @@ def transition(rule, k, v, g, beta, dtype=LD):
         return I - cast(beta) * kkT, cast(beta) * np.outer(k, v)
     if rule == "gated_delta":
         return cast(g) * (I - cast(beta) * kkT), cast(beta) * np.outer(k, v)
+    if rule == "kda":
+        D = np.diag(np.asarray([cast(x) for x in g], dtype=dtype))
+        return (I - cast(beta) * kkT).dot(D), cast(beta) * np.outer(k, v)
     raise ValueError(rule)
 
 
@@ -165,9 +170,9 @@ def brute_force_all(inp, init=None, dtype=LD):
 
 
 def pin_brute_force_all_rules(orc):
-    """All four rules on the tiny workload shapes (2 x 64 tokens, 2 heads, 16 x 16) with
+    """All five rules on the tiny workload shapes (2 x 64 tokens, 2 heads, 16 x 16) with
     a random initial state: oracle scan and oracle decode steps vs transition products."""
-    for rule in W.RULES:
+    for rule in W.ALL_RULES:
         inp = W.tiny(rule, seed=3)
         init = np.random.default_rng(1).standard_normal((2, 2, 16, 16)) * 0.3
         S_ref, o_ref = brute_force_all(inp, init)
@@ -201,16 +206,17 @@ def pin_exact_rational(orc):
     def dy(shape, den=8):
         return rng.integers(-8, 9, size=shape) / den
 
-    for rule in W.RULES:
+    for rule in W.ALL_RULES:
         K, Q, V = dy((T, dk)), dy((T, dk)), dy((T, dv))
-        G = rng.integers(1, 8, size=T) / 8.0
+        G = rng.integers(1, 8, size=(T, dk) if rule == "kda" else T) / 8.0
         Bt = rng.integers(0, 9, size=T) / 8.0
         S0 = dy((dk, dv), 4)
         F = lambda a: np.vectorize(Fraction)(a).astype(object)  # noqa: E731
         S = F(S0)
         outs = []
         for t in range(T):
-            A, Wm = transition(rule, F(K[t]), F(V[t]), Fraction(G[t]), Fraction(Bt[t]), dtype=object)
+            Gt = list(F(G[t])) if rule == "kda" else Fraction(G[t])
+            A, Wm = transition(rule, F(K[t]), F(V[t]), Gt, Fraction(Bt[t]), dtype=object)
             S = A.dot(S) + Wm
             outs.append(S.T.dot(F(Q[t])))
         inp = W.Inputs("scan", rule, 1, 1, dk, dv, torch.float64, torch.float64,
@@ -289,7 +295,7 @@ def pin_delta_stores_value(orc):
 def pin_rearranged_readout(orc):
     """o from the updated state equals the rearranged form a S_old^T q + (k.q) u (checked
     against the direct readout of the brute-force state)."""
-    for rule in W.RULES:
+    for rule in W.ALL_RULES:
         inp = W.step_inputs(B=3, n_qk_heads=1, n_v_heads=2, d_k=16, d_v=16, rule=rule, slot_map="dense",
                             state_dtype=torch.float64, io_dtype=torch.float64, seed=8, pool_std=0.5, scale=0.7)
         pool = np64(inp.pool)
@@ -301,7 +307,8 @@ def pin_rearranged_readout(orc):
         q, k, v = np64(inp.q), np64(inp.k), np64(inp.v)
         for b in range(3):
             for h in range(2):
-                A, Wm = transition(rule, k[b, 0], v[b, h], inp.g[b, h].item(), inp.beta[b, h].item(), np.float64)
+                gb = inp.g[b, h].tolist() if rule == "kda" else inp.g[b, h].item()
+                A, Wm = transition(rule, k[b, 0], v[b, h], gb, inp.beta[b, h].item(), np.float64)
                 S1 = A @ pool[b, h] + Wm
                 close(o_direct[b, h], 0.7 * S1.T @ q[b, 0], 1e-12, f"{rule} direct readout")
 
@@ -444,7 +451,7 @@ def pin_scan_checkpoints(orc):
     checked against the transition-product states at those positions, for every rule,
     with a random initial state; a checkpoint beyond the sequence is reported (bit 4)."""
     every = 4
-    for rule in W.RULES:
+    for rule in W.ALL_RULES:
         inp = W.scan_inputs(lengths=[21, 7, 0, 12], n_qk_heads=1, n_v_heads=2, d_k=16, d_v=16, rule=rule,
                             state_dtype=torch.float32, io_dtype=torch.float32, seed=17)
         init = np.random.default_rng(6).standard_normal((4, 2, 16, 16)) * 0.5
@@ -478,8 +485,59 @@ def pin_scan_checkpoints(orc):
     assert err == 4
 
 
+def pin_kda_reductions(orc):
+    """kda special cases: (1) every channel decaying by the same g is the gated_delta rule
+    with that scalar gate, checked against the scalar transition products; (2) beta = 0
+    leaves only the per-channel decay, S_T = Diag(prod_t alpha_t) S_0, and each output is
+    the decayed initial state read by q_t."""
+    inp = W.tiny("gated_delta", seed=19)
+    gk = np.repeat(np64(inp.g)[:, :, None], 16, axis=2)  # [T, H, d_k], equal channels
+    init = np.random.default_rng(8).standard_normal((2, 2, 16, 16)) * 0.5
+    S_ref, o_ref = brute_force_all(inp, init)
+    S, o, err = orc.scan("kda", 2, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k), np64(inp.v), gk,
+                         np64(inp.beta), src_pool=init, read_slot=np.arange(2, dtype=np.int32))
+    assert err == 0
+    close(S, S_ref, 1e-9, "kda with equal channels = gated_delta (state)")
+    close(o, o_ref, 1e-9, "kda with equal channels = gated_delta (output)")
+
+    inp = W.scan_inputs(lengths=[37], n_qk_heads=1, n_v_heads=2, d_k=16, d_v=8, rule="kda",
+                        state_dtype=torch.float32, io_dtype=torch.float32, seed=20, beta_mode="zero")
+    init = np.random.default_rng(9).standard_normal((1, 2, 16, 8))
+    S, o, err = run_scan_f64(orc, inp, init)
+    assert err == 0
+    a, q = np64(inp.g), np64(inp.q)
+    decay = np.cumprod(a, axis=0)  # [T, H, d_k]: prod_{s<=t} alpha_s per channel
+    for h in range(2):
+        close(S[0, h], decay[-1, h][:, None] * init[0, h], 1e-12, "kda beta = 0 state")
+        ref_o = np.einsum("ti,ij,ti->tj", decay[:, h], init[0, h], q[:, 0])
+        close(o[:, h], ref_o, 1e-12, "kda beta = 0 outputs")
+
+
+def pin_kda_wide_ranges_non_expansive(orc):
+    """kda with alpha ~ U[-1, 1] per channel and beta ~ U[0, 2] ("Complex KDA" ranges),
+    unit keys: the oracle follows the transition products, and because
+    ||(I - beta k k^T) Diag(alpha)||_2 <= 1 the state norm obeys
+    ||S_t||_F <= ||S_{t-1}||_F + beta ||v|| at every step."""
+    inp = W.scan_inputs(lengths=[40], n_qk_heads=1, n_v_heads=2, d_k=16, d_v=16, rule="kda",
+                        state_dtype=torch.float32, io_dtype=torch.float32, seed=21, g_mode="uniform_pm1",
+                        beta_mode="uniform_0_2")
+    init = np.random.default_rng(10).standard_normal((1, 2, 16, 16))
+    S_ref, o_ref = brute_force_all(inp, init)
+    S, o, err = run_scan_f64(orc, inp, init)
+    assert err == 0
+    close(S, S_ref, 1e-9, "kda wide-range state")
+    close(o, o_ref, 1e-9, "kda wide-range output")
+    pool = init.copy()
+    q, k, v, g, b = np64(inp.q), np64(inp.k), np64(inp.v), np64(inp.g), np64(inp.beta)
+    for t in range(40):
+        prev = np.linalg.norm(pool.reshape(2, -1), axis=1)
+        pool, _, _ = orc.step("kda", 1, pool, q[t:t + 1], k[t:t + 1], v[t:t + 1], g[t:t + 1], b[t:t + 1])
+        now = np.linalg.norm(pool.reshape(2, -1), axis=1)
+        assert np.all(now <= prev + b[t] * np.linalg.norm(v[t], axis=1) + 1e-12), t
+
+
 ALL_PINS = [pin_bf16_rounding, pin_brute_force_all_rules, pin_gqa_grouping, pin_exact_rational,
             pin_linear_closed_form, pin_gated_closed_form, pin_beta0_g1_identity, pin_delta_stores_value,
             pin_rearranged_readout, pin_scan_structure, pin_wide_ranges_non_expansive,
             pin_long_sequence_bounded, pin_storage_rounding_points, pin_slots, pin_pool_ops,
-            pin_scan_checkpoints]
+            pin_scan_checkpoints, pin_kda_reductions, pin_kda_wide_ranges_non_expansive]

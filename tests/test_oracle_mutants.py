@@ -20,8 +20,15 @@ MUTANTS = [
     ("gated_write_scaled", "case LAO_RULE_GATED:       *a = g;   *b = 1.0;",
      "case LAO_RULE_GATED:       *a = g;   *b = g;"),
     ("readout_by_key", "oj += S[(size_t)i * dv + j] * q[i];", "oj += S[(size_t)i * dv + j] * k[i];"),
-    ("transposed_prediction", "pj += S[(size_t)i * dv + j] * k[i];", "pj += S[(size_t)j * dv + i] * k[i];"),
-    ("transposed_outer", "a * S[(size_t)i * dv + j] + k[i] * u[j];", "a * S[(size_t)i * dv + j] + k[j] * u[i];"),
+    ("transposed_prediction", "alpha[i] * S[(size_t)i * dv + j] : S[(size_t)i * dv + j]) * k[i];",
+     "alpha[i] * S[(size_t)j * dv + i] : S[(size_t)j * dv + i]) * k[i];"),
+    ("transposed_outer", "ai * S[(size_t)i * dv + j] + k[i] * u[j];", "ai * S[(size_t)i * dv + j] + k[j] * u[i];"),
+    ("kda_undecayed_prediction", "(rule == LAO_RULE_KDA ? alpha[i] * S[(size_t)i * dv + j] :",
+     "(rule == LAO_RULE_KDA ? S[(size_t)i * dv + j] :"),
+    ("kda_channels_reversed", "const double ai = rule == LAO_RULE_KDA ? alpha[i] : a;",
+     "const double ai = rule == LAO_RULE_KDA ? alpha[dk - 1 - i] : a;"),
+    ("kda_readout_undecayed", "const double sij = kda ? al[i] * S[(size_t)i * dv + j] : S[(size_t)i * dv + j];",
+     "const double sij = S[(size_t)i * dv + j];"),
     ("gqa_interleaved", "return h / (n_v_heads / n_qk_heads);", "return h % n_qk_heads;"),
     ("scan_drops_last_token", "for (int t = cu_seqlens[s]; t < cu_seqlens[s + 1]; ++t) {",
      "for (int t = cu_seqlens[s]; t < cu_seqlens[s + 1] - 1; ++t) {"),
