@@ -66,6 +66,9 @@ class Inputs:
     write_slot: Optional[torch.Tensor] = None  # int32
     cu_seqlens: Optional[torch.Tensor] = None  # int32 [n_seqs + 1] (scan)
     extra: dict = field(default_factory=dict)
+    # > 0: the query-group direction of the ONNX operator -- k has one head per state head
+    # (n_qk_heads == n_v_heads), q and o have n_q_heads heads
+    n_q_heads: int = 0
 
     @property
     def batch(self) -> int:
@@ -114,10 +117,21 @@ def random_pool(n_slots, n_v_heads, d_k, d_v, dtype, gen, std=0.05):
     return out
 
 
+def _query_groups(inp: Inputs, n_q_heads: int, gen, normalise_qk: bool) -> Inputs:
+    """Switch inputs to the query-group direction: n_q_heads queries per row, drawn after
+    everything else (so the other operands are those of the default direction)."""
+    if n_q_heads:
+        assert inp.n_qk_heads == inp.n_v_heads and n_q_heads % inp.n_v_heads == 0
+        q = torch.randn(inp.q.shape[0], n_q_heads, inp.d_k, generator=gen)
+        inp.q = (_unit(q) if normalise_qk else q).to(inp.io_dtype).contiguous()
+        inp.n_q_heads = n_q_heads
+    return inp
+
+
 def step_inputs(*, B, n_qk_heads, n_v_heads, d_k, d_v, rule="gated_delta", n_slots=None,
                 state_dtype=torch.bfloat16, io_dtype=torch.bfloat16, seed=0, slot_map="perm",
                 pool_std=0.05, g_mode="exp_neg_softplus", beta_mode="sigmoid", normalise_qk=True,
-                scale=1.0) -> Inputs:
+                scale=1.0, n_q_heads=0) -> Inputs:
     """A decode step.  slot_map: "perm" (read = write = randperm(n_slots)[:B]),
     "dense" (no slot arrays), or "checkpoint" (half of the requests read a checkpoint slot
     and write a distinct live slot, the rest update in place)."""
@@ -142,14 +156,14 @@ def step_inputs(*, B, n_qk_heads, n_v_heads, d_k, d_v, rule="gated_delta", n_slo
     q, k, v, g, beta = token_operands(B, n_qk_heads, n_v_heads, d_k, d_v, io_dtype, gen,
                                       normalise_qk=normalise_qk, g_mode=g_mode, beta_mode=beta_mode,
                                       channel_gate=rule == "kda")
-    return Inputs("step", rule, n_qk_heads, n_v_heads, d_k, d_v, state_dtype, io_dtype, q, k, v, g, beta,
-                  scale, pool, read_slot, write_slot)
+    return _query_groups(Inputs("step", rule, n_qk_heads, n_v_heads, d_k, d_v, state_dtype, io_dtype, q, k, v, g,
+                                beta, scale, pool, read_slot, write_slot), n_q_heads, gen, normalise_qk)
 
 
 def scan_inputs(*, lengths, n_qk_heads, n_v_heads, d_k, d_v, rule="gated_delta",
                 state_dtype=torch.bfloat16, io_dtype=torch.bfloat16, seed=0, init="zero",
                 init_dtype=torch.float32, pool_std=0.05, g_mode="exp_neg_softplus",
-                beta_mode="sigmoid", normalise_qk=True, scale=1.0) -> Inputs:
+                beta_mode="sigmoid", normalise_qk=True, scale=1.0, n_q_heads=0) -> Inputs:
     """Packed varlen prefill.  init: "zero" (no read slots) or "slots" (initial states
     read from a pool of init_dtype, read_slot = randperm)."""
     gen = _gen(seed)
@@ -168,8 +182,8 @@ def scan_inputs(*, lengths, n_qk_heads, n_v_heads, d_k, d_v, rule="gated_delta",
     q, k, v, g, beta = token_operands(T, n_qk_heads, n_v_heads, d_k, d_v, io_dtype, gen,
                                       normalise_qk=normalise_qk, g_mode=g_mode, beta_mode=beta_mode,
                                       channel_gate=rule == "kda")
-    return Inputs("scan", rule, n_qk_heads, n_v_heads, d_k, d_v, state_dtype, io_dtype, q, k, v, g, beta,
-                  scale, pool, read_slot, None, cu)
+    return _query_groups(Inputs("scan", rule, n_qk_heads, n_v_heads, d_k, d_v, state_dtype, io_dtype, q, k, v, g,
+                                beta, scale, pool, read_slot, None, cu), n_q_heads, gen, normalise_qk)
 
 
 # ---- the named workloads ----------------------------------------------------------

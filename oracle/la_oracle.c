@@ -108,12 +108,13 @@ static void rule_coefficients(int rule, double g, double beta, double *a, double
     }
 }
 
-/* S (dk x dv, in/out) <- a S + k u^T with u = b (v - c S^T k); o = scale * S_new^T q.
+/* S (dk x dv, in/out) <- a S + k u^T with u = b (v - c S^T k); then, for each of the nq
+ * queries q_r = q + r * q_stride, o_r = scale * S_new^T q_r stored at o + r * o_stride.
  * For kda (alpha != NULL, dk values): S <- Diag(alpha) S + k u^T with
  * u = beta (v - (Diag(alpha) S)^T k).  u is scratch of length dv. */
-static void token_update(int rule, int dk, int dv, double *S, const double *q, const double *k,
-                         const double *v, double g, const double *alpha, double beta, double scale,
-                         double *o, double *u)
+static void token_update(int rule, int dk, int dv, double *S, int nq, const double *q, size_t q_stride,
+                         const double *k, const double *v, double g, const double *alpha, double beta,
+                         double scale, double *o, size_t o_stride, double *u)
 {
     double a, b, c;
     rule_coefficients(rule, g, beta, &a, &b, &c);
@@ -129,11 +130,12 @@ static void token_update(int rule, int dk, int dv, double *S, const double *q, c
         for (int j = 0; j < dv; ++j)
             S[(size_t)i * dv + j] = ai * S[(size_t)i * dv + j] + k[i] * u[j];
     }
-    for (int j = 0; j < dv; ++j) {
-        double oj = 0.0; /* (S_new^T q)_j */
-        for (int i = 0; i < dk; ++i) oj += S[(size_t)i * dv + j] * q[i];
-        o[j] = scale * oj;
-    }
+    for (int r = 0; r < nq; ++r, q += q_stride, o += o_stride)
+        for (int j = 0; j < dv; ++j) {
+            double oj = 0.0; /* (S_new^T q)_j */
+            for (int i = 0; i < dk; ++i) oj += S[(size_t)i * dv + j] * q[i];
+            o[j] = scale * oj;
+        }
 }
 
 static int head_group(int n_qk_heads, int n_v_heads, int h)
@@ -141,15 +143,50 @@ static int head_group(int n_qk_heads, int n_v_heads, int h)
     return h / (n_v_heads / n_qk_heads);
 }
 
+/* Head bookkeeping of one call.  Default direction (n_q_heads == 0): q and k have
+ * n_qk_heads heads and state head h reads q/k head h / (H_v / H_qk), one output per state
+ * head.  Query-group direction of the ONNX operator (n_q_heads > 0; "Seven Architectures
+ * ...", ONNX section: each KV head and its state shared by a group of query heads): k has
+ * one head per state head, q and o have n_q_heads heads, and query head i reads state head
+ * i / (n_q_heads / H_v); the state is updated once per state head. */
+typedef struct {
+    int nk;      /* k heads */
+    int nqh;     /* q heads */
+    int grp;     /* queries per state head (1 in the default direction) */
+    int no;      /* o heads */
+} heads_t;
+
+static heads_t heads_of(int n_qk_heads, int n_v_heads, int n_q_heads)
+{
+    heads_t hd;
+    if (n_q_heads > 0) {
+        hd.nk = n_v_heads; hd.nqh = n_q_heads; hd.grp = n_q_heads / n_v_heads; hd.no = n_q_heads;
+    } else {
+        hd.nk = n_qk_heads; hd.nqh = n_qk_heads; hd.grp = 1; hd.no = n_v_heads;
+    }
+    return hd;
+}
+
+/* q row of the first query of state head h, k row of state head h (token or request row t) */
+static size_t q_row(heads_t hd, int n_qk_heads, int n_v_heads, int n_q_heads, size_t t, int h)
+{
+    return t * hd.nqh + (n_q_heads > 0 ? (size_t)h * hd.grp : (size_t)head_group(n_qk_heads, n_v_heads, h));
+}
+static size_t k_row(heads_t hd, int n_qk_heads, int n_v_heads, int n_q_heads, size_t t, int h)
+{
+    return t * hd.nk + (n_q_heads > 0 ? (size_t)h : (size_t)head_group(n_qk_heads, n_v_heads, h));
+}
+
 /* ---- batched decode step -------------------------------------------------------- */
 
-int lao_step(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
-             const double *src_pool, int src_slots,
-             double *dst_pool, int dst_slots, int dst_dtype,
-             const int *read_slot, const int *write_slot, int B,
-             const double *q, const double *k, const double *v, int io_dtype,
-             const double *g, const double *beta, double scale, double *o)
+static int step_impl(int rule, int n_qk_heads, int n_v_heads, int n_q_heads, int dk, int dv,
+                     const double *src_pool, int src_slots,
+                     double *dst_pool, int dst_slots, int dst_dtype,
+                     const int *read_slot, const int *write_slot, int B,
+                     const double *q, const double *k, const double *v, int io_dtype,
+                     const double *g, const double *beta, double scale, double *o)
 {
+    const heads_t hd = heads_of(n_qk_heads, n_v_heads, n_q_heads);
     const size_t tile = (size_t)dk * dv;
     const size_t slot = (size_t)n_v_heads * tile;
     int err = 0;
@@ -172,20 +209,19 @@ int lao_step(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
         for (int h = 0; h < n_v_heads; ++h) {
             if (!ok[b]) continue;
             int rs = read_slot ? read_slot[b] : b;
-            int hq = head_group(n_qk_heads, n_v_heads, h);
             double *S = next + (size_t)b * slot + (size_t)h * tile;
             double *u = (double *)malloc(sizeof(double) * (size_t)dv);
             memcpy(S, src_pool + (size_t)rs * slot + (size_t)h * tile, sizeof(double) * tile);
-            double *ob = o + ((size_t)b * n_v_heads + h) * dv;
-            token_update(rule, dk, dv, S,
-                         q + ((size_t)b * n_qk_heads + hq) * dk,
-                         k + ((size_t)b * n_qk_heads + hq) * dk,
+            double *ob = o + ((size_t)b * hd.no + (size_t)h * hd.grp) * dv;
+            token_update(rule, dk, dv, S, hd.grp,
+                         q + q_row(hd, n_qk_heads, n_v_heads, n_q_heads, (size_t)b, h) * dk, (size_t)dk,
+                         k + k_row(hd, n_qk_heads, n_v_heads, n_q_heads, (size_t)b, h) * dk,
                          v + ((size_t)b * n_v_heads + h) * dv,
                          g && rule != LAO_RULE_KDA ? g[(size_t)b * n_v_heads + h] : 1.0,
                          rule == LAO_RULE_KDA ? g + ((size_t)b * n_v_heads + h) * dk : NULL,
                          beta ? beta[(size_t)b * n_v_heads + h] : 1.0,
-                         scale, ob, u);
-            for (int j = 0; j < dv; ++j) ob[j] = lao_round_to(ob[j], io_dtype);
+                         scale, ob, (size_t)dv, u);
+            for (int j = 0; j < dv * hd.grp; ++j) ob[j] = lao_round_to(ob[j], io_dtype);
             for (size_t e = 0; e < tile; ++e) S[e] = lao_round_to(S[e], dst_dtype);
             free(u);
         }
@@ -199,6 +235,30 @@ int lao_step(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
     free(next);
     free(ok);
     return err;
+}
+
+int lao_step(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+             const double *src_pool, int src_slots,
+             double *dst_pool, int dst_slots, int dst_dtype,
+             const int *read_slot, const int *write_slot, int B,
+             const double *q, const double *k, const double *v, int io_dtype,
+             const double *g, const double *beta, double scale, double *o)
+{
+    return step_impl(rule, n_qk_heads, n_v_heads, 0, dk, dv, src_pool, src_slots, dst_pool, dst_slots, dst_dtype,
+                     read_slot, write_slot, B, q, k, v, io_dtype, g, beta, scale, o);
+}
+
+/* Decode step in the query-group direction: k [B, H_v, d_k], q [B, n_q_heads, d_k],
+ * o [B, n_q_heads, d_v]; query head i reads the updated state of head i / (n_q_heads / H_v). */
+int lao_step_qgroups(int rule, int n_q_heads, int n_v_heads, int dk, int dv,
+                     const double *src_pool, int src_slots,
+                     double *dst_pool, int dst_slots, int dst_dtype,
+                     const int *read_slot, const int *write_slot, int B,
+                     const double *q, const double *k, const double *v, int io_dtype,
+                     const double *g, const double *beta, double scale, double *o)
+{
+    return step_impl(rule, n_v_heads, n_v_heads, n_q_heads, dk, dv, src_pool, src_slots, dst_pool, dst_slots,
+                     dst_dtype, read_slot, write_slot, B, q, k, v, io_dtype, g, beta, scale, o);
 }
 
 /* The readout of one decode step written in the rearranged form of the "Gated DeltaNet"
@@ -253,14 +313,15 @@ void lao_readout_rearranged(int rule, int n_qk_heads, int n_v_heads, int dk, int
  * stored to dst_pool slot ckpt_slots[ckpt_cu[s] + j].  A checkpoint position beyond the
  * sequence is reported (bit 4) and skipped; an out-of-range checkpoint slot is reported
  * (bit 2) and skipped.  ckpt_every <= 0: no checkpoints (lao_scan). */
-int lao_scan_ckpt(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
-                  const double *src_pool, int src_slots, const int *read_slot,
-                  double *dst_pool, int dst_slots, int dst_dtype, const int *write_slot,
-                  int n_seqs, const int *cu_seqlens, int total_tokens,
-                  const double *q, const double *k, const double *v, int io_dtype,
-                  const double *g, const double *beta, double scale, double *o,
-                  int ckpt_every, const int *ckpt_cu, const int *ckpt_slots)
+static int scan_impl(int rule, int n_qk_heads, int n_v_heads, int n_q_heads, int dk, int dv,
+                     const double *src_pool, int src_slots, const int *read_slot,
+                     double *dst_pool, int dst_slots, int dst_dtype, const int *write_slot,
+                     int n_seqs, const int *cu_seqlens, int total_tokens,
+                     const double *q, const double *k, const double *v, int io_dtype,
+                     const double *g, const double *beta, double scale, double *o,
+                     int ckpt_every, const int *ckpt_cu, const int *ckpt_slots)
 {
+    const heads_t hd = heads_of(n_qk_heads, n_v_heads, n_q_heads);
     const size_t tile = (size_t)dk * dv;
     const size_t slot = (size_t)n_v_heads * tile;
     int err = 0;
@@ -290,7 +351,6 @@ int lao_scan_ckpt(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
     for (int s = 0; s < n_seqs; ++s) {
         for (int h = 0; h < n_v_heads; ++h) {
             if (!ok[s]) continue;
-            int hq = head_group(n_qk_heads, n_v_heads, h);
             double *S = next + (size_t)s * slot + (size_t)h * tile;
             double *u = (double *)malloc(sizeof(double) * (size_t)dv);
             if (read_slot)
@@ -298,16 +358,16 @@ int lao_scan_ckpt(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
             else
                 memset(S, 0, sizeof(double) * tile);
             for (int t = cu_seqlens[s]; t < cu_seqlens[s + 1]; ++t) {
-                double *ot = o + ((size_t)t * n_v_heads + h) * dv;
-                token_update(rule, dk, dv, S,
-                             q + ((size_t)t * n_qk_heads + hq) * dk,
-                             k + ((size_t)t * n_qk_heads + hq) * dk,
+                double *ot = o + ((size_t)t * hd.no + (size_t)h * hd.grp) * dv;
+                token_update(rule, dk, dv, S, hd.grp,
+                             q + q_row(hd, n_qk_heads, n_v_heads, n_q_heads, (size_t)t, h) * dk, (size_t)dk,
+                             k + k_row(hd, n_qk_heads, n_v_heads, n_q_heads, (size_t)t, h) * dk,
                              v + ((size_t)t * n_v_heads + h) * dv,
                              g && rule != LAO_RULE_KDA ? g[(size_t)t * n_v_heads + h] : 1.0,
                              rule == LAO_RULE_KDA ? g + ((size_t)t * n_v_heads + h) * dk : NULL,
                              beta ? beta[(size_t)t * n_v_heads + h] : 1.0,
-                             scale, ot, u);
-                for (int j = 0; j < dv; ++j) ot[j] = lao_round_to(ot[j], io_dtype);
+                             scale, ot, (size_t)dv, u);
+                for (int j = 0; j < dv * hd.grp; ++j) ot[j] = lao_round_to(ot[j], io_dtype);
                 const int pos = t - cu_seqlens[s] + 1; /* tokens of this sequence consumed */
                 if (ckpt_every > 0 && pos % ckpt_every == 0) {
                     const int j = pos / ckpt_every - 1;
@@ -335,6 +395,19 @@ int lao_scan_ckpt(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
     return err;
 }
 
+int lao_scan_ckpt(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+                  const double *src_pool, int src_slots, const int *read_slot,
+                  double *dst_pool, int dst_slots, int dst_dtype, const int *write_slot,
+                  int n_seqs, const int *cu_seqlens, int total_tokens,
+                  const double *q, const double *k, const double *v, int io_dtype,
+                  const double *g, const double *beta, double scale, double *o,
+                  int ckpt_every, const int *ckpt_cu, const int *ckpt_slots)
+{
+    return scan_impl(rule, n_qk_heads, n_v_heads, 0, dk, dv, src_pool, src_slots, read_slot, dst_pool,
+                     dst_slots, dst_dtype, write_slot, n_seqs, cu_seqlens, total_tokens, q, k, v, io_dtype,
+                     g, beta, scale, o, ckpt_every, ckpt_cu, ckpt_slots);
+}
+
 int lao_scan(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
              const double *src_pool, int src_slots, const int *read_slot,
              double *dst_pool, int dst_slots, int dst_dtype, const int *write_slot,
@@ -345,6 +418,19 @@ int lao_scan(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
     return lao_scan_ckpt(rule, n_qk_heads, n_v_heads, dk, dv, src_pool, src_slots, read_slot, dst_pool,
                          dst_slots, dst_dtype, write_slot, n_seqs, cu_seqlens, total_tokens, q, k, v, io_dtype,
                          g, beta, scale, o, 0, NULL, NULL);
+}
+
+/* Scan in the query-group direction (layouts as lao_step_qgroups, T rows). */
+int lao_scan_qgroups(int rule, int n_q_heads, int n_v_heads, int dk, int dv,
+                     const double *src_pool, int src_slots, const int *read_slot,
+                     double *dst_pool, int dst_slots, int dst_dtype, const int *write_slot,
+                     int n_seqs, const int *cu_seqlens, int total_tokens,
+                     const double *q, const double *k, const double *v, int io_dtype,
+                     const double *g, const double *beta, double scale, double *o)
+{
+    return scan_impl(rule, n_v_heads, n_v_heads, n_q_heads, dk, dv, src_pool, src_slots, read_slot, dst_pool,
+                     dst_slots, dst_dtype, write_slot, n_seqs, cu_seqlens, total_tokens, q, k, v, io_dtype,
+                     g, beta, scale, o, 0, NULL, NULL);
 }
 
 /* ---- slot pool: whole-slot byte copies ------------------------------------------ */

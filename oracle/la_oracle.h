@@ -52,6 +52,20 @@ int lao_scan_ckpt(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
                   const double *g, const double *beta, double scale, double *o,
                   int ckpt_every, const int *ckpt_cu, const int *ckpt_slots);
 
+int lao_step_qgroups(int rule, int n_q_heads, int n_v_heads, int dk, int dv,
+                     const double *src_pool, int src_slots,
+                     double *dst_pool, int dst_slots, int dst_dtype,
+                     const int *read_slot, const int *write_slot, int B,
+                     const double *q, const double *k, const double *v, int io_dtype,
+                     const double *g, const double *beta, double scale, double *o);
+
+int lao_scan_qgroups(int rule, int n_q_heads, int n_v_heads, int dk, int dv,
+                     const double *src_pool, int src_slots, const int *read_slot,
+                     double *dst_pool, int dst_slots, int dst_dtype, const int *write_slot,
+                     int n_seqs, const int *cu_seqlens, int total_tokens,
+                     const double *q, const double *k, const double *v, int io_dtype,
+                     const double *g, const double *beta, double scale, double *o);
+
 int lao_pool_copy(unsigned char *pool, size_t slot_bytes, int n_slots, int n,
                   const int *src_slots, const int *dst_slots);
 int lao_pool_gather(const unsigned char *pool, size_t slot_bytes, int n_slots, int n,

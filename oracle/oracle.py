@@ -37,6 +37,10 @@ def lib():
         _lib.lao_scan.restype = i
         _lib.lao_scan_ckpt.argtypes = _lib.lao_scan.argtypes + [i, p, p]
         _lib.lao_scan_ckpt.restype = i
+        _lib.lao_step_qgroups.argtypes = _lib.lao_step.argtypes
+        _lib.lao_step_qgroups.restype = i
+        _lib.lao_scan_qgroups.argtypes = _lib.lao_scan.argtypes
+        _lib.lao_scan_qgroups.restype = i
         _lib.lao_pool_copy.argtypes = [p, sz, i, i, p, p]
         _lib.lao_pool_gather.argtypes = [p, sz, i, i, p, p]
         _lib.lao_pool_scatter.argtypes = [p, sz, i, i, p, p]
@@ -119,6 +123,53 @@ def step(rule, n_qk_heads, src_pool, q, k, v, g=None, beta=None, scale=1.0, *,
                          _ptr(q), _ptr(k), _ptr(v), DTYPES[io_dtype], _ptr(g), _ptr(beta),
                          float(scale), _ptr(o))
     return dst, o, err
+
+
+def step_qgroups(rule, n_q_heads, src_pool, q, k, v, g=None, beta=None, scale=1.0, *,
+                 dst_pool=None, dst_dtype="f64", io_dtype="f64", read_slot=None, write_slot=None):
+    """One decode step in the query-group direction of the ONNX operator: k [B, H_v, d_k]
+    (one key per state head), q [B, n_q_heads, d_k], o [B, n_q_heads, d_v]; query head i
+    reads state head i / (n_q_heads / H_v).  Returns (dst_pool, o, err_bits)."""
+    src = _f64(src_pool)
+    dst = src.copy() if dst_pool is None else dst_pool
+    assert dst.dtype == np.float64 and dst.flags.c_contiguous
+    n_src, hv, dk, dv = src.shape
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B = q.shape[0]
+    g = None if g is None else _f64(g)
+    beta = None if beta is None else _f64(beta)
+    rs, ws = _i32(read_slot), _i32(write_slot)
+    o = np.zeros((B, n_q_heads, dv), dtype=np.float64)
+    err = lib().lao_step_qgroups(RULES[rule], n_q_heads, hv, dk, dv, _ptr(src), n_src,
+                                 _ptr(dst), dst.shape[0], DTYPES[dst_dtype], _ptr(rs), _ptr(ws), B,
+                                 _ptr(q), _ptr(k), _ptr(v), DTYPES[io_dtype], _ptr(g), _ptr(beta),
+                                 float(scale), _ptr(o))
+    return dst, o, err
+
+
+def scan_qgroups(rule, n_q_heads, cu_seqlens, q, k, v, g=None, beta=None, scale=1.0, *,
+                 src_pool=None, read_slot=None, dst_pool=None, dst_dtype="f64", write_slot=None,
+                 io_dtype="f64"):
+    """Token-serial scan in the query-group direction (layouts as step_qgroups with T
+    rows).  Returns (dst_pool, o, err_bits)."""
+    cu = _i32(cu_seqlens)
+    n_seqs = cu.shape[0] - 1
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, hv, dk = k.shape
+    dv = v.shape[2]
+    if dst_pool is None:
+        dst_pool = np.zeros((n_seqs, hv, dk, dv), dtype=np.float64)
+    assert dst_pool.dtype == np.float64 and dst_pool.flags.c_contiguous
+    src = None if src_pool is None else _f64(src_pool)
+    n_src = 0 if src is None else src.shape[0]
+    g = None if g is None else _f64(g)
+    beta = None if beta is None else _f64(beta)
+    o = np.zeros((T, n_q_heads, dv), dtype=np.float64)
+    err = lib().lao_scan_qgroups(RULES[rule], n_q_heads, hv, dk, dv, _ptr(src), n_src, _ptr(_i32(read_slot)),
+                                 _ptr(dst_pool), dst_pool.shape[0], DTYPES[dst_dtype], _ptr(_i32(write_slot)),
+                                 n_seqs, _ptr(cu), T, _ptr(q), _ptr(k), _ptr(v), DTYPES[io_dtype],
+                                 _ptr(g), _ptr(beta), float(scale), _ptr(o))
+    return dst_pool, o, err
 
 
 def readout_rearranged(rule, n_qk_heads, state, q, k, v, g=None, beta=None, scale=1.0):
@@ -208,7 +259,8 @@ def set_threads(n):
 
 
 __all__ = ["round_bf16", "round_to", "step", "readout_rearranged", "scan", "pool_copy",
-           "pool_gather", "pool_scatter", "pool_zero", "num_threads", "set_threads", "RULES", "DTYPES"]
+           "pool_gather", "pool_scatter", "pool_zero", "num_threads", "set_threads", "RULES", "DTYPES",
+           "step_qgroups", "scan_qgroups"]
 
 if os.environ.get("LAO_THREADS"):
     set_threads(int(os.environ["LAO_THREADS"]))

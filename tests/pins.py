@@ -536,8 +536,48 @@ def pin_kda_wide_ranges_non_expansive(orc):
         assert np.all(now <= prev + b[t] * np.linalg.norm(v[t], axis=1) + 1e-12), t
 
 
+def pin_query_groups(orc):
+    """Query-group direction of the ONNX operator (each state head read by a group of query
+    heads): 2 state heads, 6 query heads.  Each state head's states come from transition
+    products of its own k, v; query head i reads the state of head i // 3 after the token.
+    Checked for the scan and for sequential decode steps, for gated_delta and kda; with one
+    query per state head it equals the default direction."""
+    for rule in ("gated_delta", "kda"):
+        inp = W.scan_inputs(lengths=[13, 6], n_qk_heads=2, n_v_heads=2, d_k=16, d_v=8, rule=rule,
+                            state_dtype=torch.float32, io_dtype=torch.float32, seed=22, n_q_heads=6)
+        init = np.random.default_rng(11).standard_normal((2, 2, 16, 8)) * 0.5
+        q, k, v = np64(inp.q), np64(inp.k), np64(inp.v)
+        g, b = np64(inp.g), np64(inp.beta)
+        cu = inp.cu_seqlens.numpy()
+        S, o, err = orc.scan_qgroups(rule, 6, cu, q, k, v, g, b, src_pool=init, read_slot=np.arange(2, dtype=np.int32))
+        assert err == 0 and o.shape == (19, 6, 8)
+        for sq in range(2):
+            t0, t1 = int(cu[sq]), int(cu[sq + 1])
+            for h in range(2):
+                states, _ = brute_force_head(rule, init[sq, h], q[t0:t1, 0], k[t0:t1, h], v[t0:t1, h], g[t0:t1, h],
+                                             b[t0:t1, h])
+                close(S[sq, h], states[-1], 1e-9, f"{rule} query-group state")
+                for i in range(3 * h, 3 * h + 3):
+                    ref = np.stack([states[t].T.astype(np.float64) @ q[t0 + t, i] for t in range(t1 - t0)])
+                    close(o[t0:t1, i], ref, 1e-9, f"{rule} query head {i}")
+        # the same tokens as decode steps (sequence 1's 6 tokens)
+        pool = init[1:2].copy()
+        for t in range(int(cu[1]), int(cu[2])):
+            pool, ot, err = orc.step_qgroups(rule, 6, pool, q[t:t + 1], k[t:t + 1], v[t:t + 1], g[t:t + 1], b[t:t + 1])
+            assert err == 0
+            close(ot[0], o[t], 1e-12, f"{rule} query-group step vs scan")
+        close(pool[0], S[1], 1e-12, f"{rule} query-group step state")
+    # one query per state head: identical to the default direction with H_qk = H_v
+    inp = W.scan_inputs(lengths=[9], n_qk_heads=2, n_v_heads=2, d_k=16, d_v=16, rule="gated_delta",
+                        state_dtype=torch.float32, io_dtype=torch.float32, seed=23)
+    S1, o1, _ = run_scan_f64(orc, inp)
+    S2, o2, _ = orc.scan_qgroups("gated_delta", 2, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k), np64(inp.v),
+                                 np64(inp.g), np64(inp.beta))
+    assert np.array_equal(S1, S2) and np.array_equal(o1, o2)
+
+
 ALL_PINS = [pin_bf16_rounding, pin_brute_force_all_rules, pin_gqa_grouping, pin_exact_rational,
             pin_linear_closed_form, pin_gated_closed_form, pin_beta0_g1_identity, pin_delta_stores_value,
             pin_rearranged_readout, pin_scan_structure, pin_wide_ranges_non_expansive,
             pin_long_sequence_bounded, pin_storage_rounding_points, pin_slots, pin_pool_ops,
-            pin_scan_checkpoints, pin_kda_reductions, pin_kda_wide_ranges_non_expansive]
+            pin_scan_checkpoints, pin_kda_reductions, pin_kda_wide_ranges_non_expansive, pin_query_groups]

@@ -30,6 +30,10 @@ MUTANTS = [
     ("kda_readout_undecayed", "const double sij = kda ? al[i] * S[(size_t)i * dv + j] : S[(size_t)i * dv + j];",
      "const double sij = S[(size_t)i * dv + j];"),
     ("gqa_interleaved", "return h / (n_v_heads / n_qk_heads);", "return h % n_qk_heads;"),
+    ("query_group_reads_wrong_queries", "return t * hd.nqh + (n_q_heads > 0 ? (size_t)h * hd.grp :",
+     "return t * hd.nqh + (n_q_heads > 0 ? (size_t)h :"),
+    ("query_group_output_misplaced", "double *ot = o + ((size_t)t * hd.no + (size_t)h * hd.grp) * dv;",
+     "double *ot = o + ((size_t)t * hd.no + (size_t)h) * dv;"),
     ("scan_drops_last_token", "for (int t = cu_seqlens[s]; t < cu_seqlens[s + 1]; ++t) {",
      "for (int t = cu_seqlens[s]; t < cu_seqlens[s + 1] - 1; ++t) {"),
     ("scan_ignores_initial_state", "memcpy(S, src_pool + (size_t)read_slot[s] * slot + (size_t)h * tile, sizeof(double) * tile);",
