@@ -38,7 +38,8 @@
  * stores a value ("Recurrent state" glossary, Why it matters: state stored in BF16
  * while computed in a wider type): the state after each decode step, the state at the
  * end of a scan, and each output o_t (to the io type).  Storage types: 0 = f64 (no
- * rounding), 1 = f32, 2 = bf16 (round-to-nearest-even from the IEEE definition).
+ * rounding), 1 = f32, 2 = bf16 (round-to-nearest-even from the IEEE definition), 3 = q8
+ * (the mixed INT8 / BF16 format below; state only).
  *
  * Layouts (row-major, last index contiguous):
  *   pool   [n_slots, H_v, d_k, d_v]
@@ -94,6 +95,155 @@ double lao_round_to(double x, int dtype)
     if (dtype == LAO_F32) return (double)(float)x;
     if (dtype == LAO_BF16) return lao_round_bf16(x);
     return x;
+}
+
+/* ---- mixed INT8 / BF16 state storage ------------------------------------------------
+ *
+ * "Seven Architectures ...", sections "ONNX LinearAttention / FlashInfer" and the
+ * Practical Implications: DAMP stores the recurrent state at about 9.9 bits per value,
+ * the high-risk key channels in a higher precision and the rest in INT8, a 69.1 %
+ * reduction of state storage.  The pages fix no layout; the reading taken here (format
+ * code 3, "q8"), per (slot, head) tile of d_k x d_v:
+ *   - a per-head mask of d_k bits marks the n_hp high-precision key channels (rows);
+ *   - every other row is stored as INT8 codes in groups of 32 consecutive columns, each
+ *     group with an FP32 scale s = absmax / 127 (absmax of the group's FP32 values);
+ *     code = clamp(rint(x * (127 / absmax)), -127, 127), decoded as code * s; a group of
+ *     zeros has s = 0 and codes 0;
+ *   - high-precision rows are stored in BF16 (round to nearest even).
+ * Byte layout of a tile: codes [d_k - n_hp][d_v] int8, then scales [d_k - n_hp][d_v / 32]
+ * float32, then BF16 rows [n_hp][d_v]; rows of each block in increasing row index.  The
+ * codes are decided in FP32 from the FP32 value (the value the kernels hold).  With
+ * n_hp = d_k / 8 the tile holds 9.875 bits per value. */
+
+size_t lao_q8_tile_bytes(int dk, int dv, int n_hp)
+{
+    const size_t n8 = (size_t)(dk - n_hp);
+    return n8 * (size_t)dv + n8 * (size_t)(dv / 32) * 4 + (size_t)n_hp * (size_t)dv * 2;
+}
+
+static int hp_row(const unsigned *mask, int i)
+{
+    return (int)((mask[i / 32] >> (i % 32)) & 1u);
+}
+
+static unsigned short bf16_bits(float x)
+{
+    float y = (float)lao_round_bf16((double)x);
+    unsigned u;
+    memcpy(&u, &y, 4);
+    return (unsigned short)(u >> 16);
+}
+
+static void q8_encode_tile(const float *x, int dk, int dv, int n_hp, const unsigned *mask, unsigned char *out)
+{
+    const int n8 = dk - n_hp, ng = dv / 32;
+    unsigned char *sc = out + (size_t)n8 * dv;
+    unsigned char *hp = sc + (size_t)n8 * ng * 4;
+    int r8 = 0, rh = 0;
+    for (int i = 0; i < dk; ++i) {
+        const float *row = x + (size_t)i * dv;
+        if (hp_row(mask, i)) {
+            for (int j = 0; j < dv; ++j) {
+                unsigned short b = bf16_bits(row[j]);
+                memcpy(hp + ((size_t)rh * dv + j) * 2, &b, 2);
+            }
+            ++rh;
+            continue;
+        }
+        for (int gi = 0; gi < ng; ++gi) {
+            float amax = 0.0f;
+            for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(row[gi * 32 + j]));
+            const float s = amax > 0.0f ? amax / 127.0f : 0.0f;
+            const float inv = amax > 0.0f ? 127.0f / amax : 0.0f;
+            memcpy(sc + ((size_t)r8 * ng + gi) * 4, &s, 4);
+            for (int j = 0; j < 32; ++j) {
+                const float c = fminf(fmaxf(rintf(row[gi * 32 + j] * inv), -127.0f), 127.0f);
+                out[(size_t)r8 * dv + gi * 32 + j] = (unsigned char)(signed char)c;
+            }
+        }
+        ++r8;
+    }
+}
+
+static void q8_decode_tile(const unsigned char *in, int dk, int dv, int n_hp, const unsigned *mask, float *x)
+{
+    const int n8 = dk - n_hp, ng = dv / 32;
+    const unsigned char *sc = in + (size_t)n8 * dv;
+    const unsigned char *hp = sc + (size_t)n8 * ng * 4;
+    int r8 = 0, rh = 0;
+    for (int i = 0; i < dk; ++i) {
+        float *row = x + (size_t)i * dv;
+        if (hp_row(mask, i)) {
+            for (int j = 0; j < dv; ++j) {
+                unsigned short b;
+                memcpy(&b, hp + ((size_t)rh * dv + j) * 2, 2);
+                unsigned u = (unsigned)b << 16;
+                memcpy(&row[j], &u, 4);
+            }
+            ++rh;
+            continue;
+        }
+        for (int gi = 0; gi < ng; ++gi) {
+            float s;
+            memcpy(&s, sc + ((size_t)r8 * ng + gi) * 4, 4);
+            for (int j = 0; j < 32; ++j)
+                row[gi * 32 + j] = (float)(signed char)in[(size_t)r8 * dv + gi * 32 + j] * s;
+        }
+        ++r8;
+    }
+}
+
+/* x [n][H][dk][dv] float <-> q8 slots [n][H][tile bytes]; masks [H][dk / 32].  Returns -1
+ * when a head's mask does not hold exactly n_hp rows, else 0. */
+static int q8_masks_ok(const unsigned *masks, int H, int dk, int n_hp)
+{
+    for (int h = 0; h < H; ++h) {
+        int c = 0;
+        for (int i = 0; i < dk; ++i) c += hp_row(masks + (size_t)h * (dk / 32), i);
+        if (c != n_hp) return 0;
+    }
+    return 1;
+}
+
+int lao_q8_encode(const float *x, int n, int H, int dk, int dv, int n_hp, const unsigned *masks,
+                  unsigned char *out)
+{
+    if (!q8_masks_ok(masks, H, dk, n_hp)) return -1;
+    const size_t tb = lao_q8_tile_bytes(dk, dv, n_hp);
+    for (int t = 0; t < n * H; ++t)
+        q8_encode_tile(x + (size_t)t * dk * dv, dk, dv, n_hp, masks + (size_t)(t % H) * (dk / 32), out + (size_t)t * tb);
+    return 0;
+}
+
+int lao_q8_decode(const unsigned char *in, int n, int H, int dk, int dv, int n_hp, const unsigned *masks, float *x)
+{
+    if (!q8_masks_ok(masks, H, dk, n_hp)) return -1;
+    const size_t tb = lao_q8_tile_bytes(dk, dv, n_hp);
+    for (int t = 0; t < n * H; ++t)
+        q8_decode_tile(in + (size_t)t * tb, dk, dv, n_hp, masks + (size_t)(t % H) * (dk / 32), x + (size_t)t * dk * dv);
+    return 0;
+}
+
+/* Rounds one tile to its storage type: elementwise for f64 / f32 / bf16; for q8 the
+ * FP32 value encoded and decoded again (mask: the head's d_k / 32 mask words). */
+static void round_tile(double *S, int dk, int dv, int dtype, const unsigned *mask)
+{
+    const size_t tile = (size_t)dk * dv;
+    if (dtype != LAO_Q8) {
+        for (size_t e = 0; e < tile; ++e) S[e] = lao_round_to(S[e], dtype);
+        return;
+    }
+    int n_hp = 0;
+    for (int i = 0; i < dk; ++i) n_hp += hp_row(mask, i);
+    float *x = (float *)malloc(sizeof(float) * (tile ? tile : 1));
+    unsigned char *b = (unsigned char *)malloc(lao_q8_tile_bytes(dk, dv, n_hp) + 1);
+    if (!x || !b || !tile) { free(x); free(b); return; }
+    for (size_t e = 0; e < tile; ++e) x[e] = (float)S[e];
+    q8_encode_tile(x, dk, dv, n_hp, mask, b);
+    q8_decode_tile(b, dk, dv, n_hp, mask, x);
+    for (size_t e = 0; e < tile; ++e) S[e] = (double)x[e];
+    free(x);
+    free(b);
 }
 
 /* ---- one state head, one token ------------------------------------------------- */
@@ -184,7 +334,7 @@ static int step_impl(int rule, int n_qk_heads, int n_v_heads, int n_q_heads, int
                      double *dst_pool, int dst_slots, int dst_dtype,
                      const int *read_slot, const int *write_slot, int B,
                      const double *q, const double *k, const double *v, int io_dtype,
-                     const double *g, const double *beta, double scale, double *o)
+                     const double *g, const double *beta, double scale, double *o, const unsigned *q8_masks)
 {
     const heads_t hd = heads_of(n_qk_heads, n_v_heads, n_q_heads);
     const size_t tile = (size_t)dk * dv;
@@ -222,7 +372,7 @@ static int step_impl(int rule, int n_qk_heads, int n_v_heads, int n_q_heads, int
                          beta ? beta[(size_t)b * n_v_heads + h] : 1.0,
                          scale, ob, (size_t)dv, u);
             for (int j = 0; j < dv * hd.grp; ++j) ob[j] = lao_round_to(ob[j], io_dtype);
-            for (size_t e = 0; e < tile; ++e) S[e] = lao_round_to(S[e], dst_dtype);
+            round_tile(S, dk, dv, dst_dtype, q8_masks ? q8_masks + (size_t)h * (dk / 32) : NULL);
             free(u);
         }
     }
@@ -245,7 +395,19 @@ int lao_step(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
              const double *g, const double *beta, double scale, double *o)
 {
     return step_impl(rule, n_qk_heads, n_v_heads, 0, dk, dv, src_pool, src_slots, dst_pool, dst_slots, dst_dtype,
-                     read_slot, write_slot, B, q, k, v, io_dtype, g, beta, scale, o);
+                     read_slot, write_slot, B, q, k, v, io_dtype, g, beta, scale, o, NULL);
+}
+
+/* Decode step whose destination is stored in the q8 format (masks [H_v][d_k / 32]); the
+ * source pool holds decoded values. */
+int lao_step_q8(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+                const double *src_pool, int src_slots, double *dst_pool, int dst_slots,
+                const int *read_slot, const int *write_slot, int B,
+                const double *q, const double *k, const double *v, int io_dtype,
+                const double *g, const double *beta, double scale, double *o, const unsigned *q8_masks)
+{
+    return step_impl(rule, n_qk_heads, n_v_heads, 0, dk, dv, src_pool, src_slots, dst_pool, dst_slots, LAO_Q8,
+                     read_slot, write_slot, B, q, k, v, io_dtype, g, beta, scale, o, q8_masks);
 }
 
 /* Decode step in the query-group direction: k [B, H_v, d_k], q [B, n_q_heads, d_k],
@@ -258,7 +420,7 @@ int lao_step_qgroups(int rule, int n_q_heads, int n_v_heads, int dk, int dv,
                      const double *g, const double *beta, double scale, double *o)
 {
     return step_impl(rule, n_v_heads, n_v_heads, n_q_heads, dk, dv, src_pool, src_slots, dst_pool, dst_slots,
-                     dst_dtype, read_slot, write_slot, B, q, k, v, io_dtype, g, beta, scale, o);
+                     dst_dtype, read_slot, write_slot, B, q, k, v, io_dtype, g, beta, scale, o, NULL);
 }
 
 /* The readout of one decode step written in the rearranged form of the "Gated DeltaNet"
@@ -319,7 +481,7 @@ static int scan_impl(int rule, int n_qk_heads, int n_v_heads, int n_q_heads, int
                      int n_seqs, const int *cu_seqlens, int total_tokens,
                      const double *q, const double *k, const double *v, int io_dtype,
                      const double *g, const double *beta, double scale, double *o,
-                     int ckpt_every, const int *ckpt_cu, const int *ckpt_slots)
+                     int ckpt_every, const int *ckpt_cu, const int *ckpt_slots, const unsigned *q8_masks)
 {
     const heads_t hd = heads_of(n_qk_heads, n_v_heads, n_q_heads);
     const size_t tile = (size_t)dk * dv;
@@ -375,12 +537,13 @@ static int scan_impl(int rule, int n_qk_heads, int n_v_heads, int n_q_heads, int
                         const int cs = ckpt_slots[ckpt_cu[s] + j];
                         if (cs >= 0 && cs < dst_slots) {
                             double *D = dst_pool + (size_t)cs * slot + (size_t)h * tile;
-                            for (size_t e = 0; e < tile; ++e) D[e] = lao_round_to(S[e], dst_dtype);
+                            memcpy(D, S, sizeof(double) * tile);
+                            round_tile(D, dk, dv, dst_dtype, q8_masks ? q8_masks + (size_t)h * (dk / 32) : NULL);
                         }
                     }
                 }
             }
-            for (size_t e = 0; e < tile; ++e) S[e] = lao_round_to(S[e], dst_dtype);
+            round_tile(S, dk, dv, dst_dtype, q8_masks ? q8_masks + (size_t)h * (dk / 32) : NULL);
             free(u);
         }
     }
@@ -405,7 +568,21 @@ int lao_scan_ckpt(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
 {
     return scan_impl(rule, n_qk_heads, n_v_heads, 0, dk, dv, src_pool, src_slots, read_slot, dst_pool,
                      dst_slots, dst_dtype, write_slot, n_seqs, cu_seqlens, total_tokens, q, k, v, io_dtype,
-                     g, beta, scale, o, ckpt_every, ckpt_cu, ckpt_slots);
+                     g, beta, scale, o, ckpt_every, ckpt_cu, ckpt_slots, NULL);
+}
+
+/* Scan whose final states (and checkpoints) are stored in the q8 format. */
+int lao_scan_q8(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+                const double *src_pool, int src_slots, const int *read_slot,
+                double *dst_pool, int dst_slots, const int *write_slot,
+                int n_seqs, const int *cu_seqlens, int total_tokens,
+                const double *q, const double *k, const double *v, int io_dtype,
+                const double *g, const double *beta, double scale, double *o,
+                int ckpt_every, const int *ckpt_cu, const int *ckpt_slots, const unsigned *q8_masks)
+{
+    return scan_impl(rule, n_qk_heads, n_v_heads, 0, dk, dv, src_pool, src_slots, read_slot, dst_pool,
+                     dst_slots, LAO_Q8, write_slot, n_seqs, cu_seqlens, total_tokens, q, k, v, io_dtype,
+                     g, beta, scale, o, ckpt_every, ckpt_cu, ckpt_slots, q8_masks);
 }
 
 int lao_scan(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
@@ -430,7 +607,7 @@ int lao_scan_qgroups(int rule, int n_q_heads, int n_v_heads, int dk, int dv,
 {
     return scan_impl(rule, n_v_heads, n_v_heads, n_q_heads, dk, dv, src_pool, src_slots, read_slot, dst_pool,
                      dst_slots, dst_dtype, write_slot, n_seqs, cu_seqlens, total_tokens, q, k, v, io_dtype,
-                     g, beta, scale, o, 0, NULL, NULL);
+                     g, beta, scale, o, 0, NULL, NULL, NULL);
 }
 
 /* ---- slot pool: whole-slot byte copies ------------------------------------------ */

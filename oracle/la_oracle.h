@@ -17,6 +17,7 @@
 #define LAO_F64 0
 #define LAO_F32 1
 #define LAO_BF16 2
+#define LAO_Q8 3
 
 #ifdef __cplusplus
 extern "C" {
@@ -65,6 +66,23 @@ int lao_scan_qgroups(int rule, int n_q_heads, int n_v_heads, int dk, int dv,
                      int n_seqs, const int *cu_seqlens, int total_tokens,
                      const double *q, const double *k, const double *v, int io_dtype,
                      const double *g, const double *beta, double scale, double *o);
+
+size_t lao_q8_tile_bytes(int dk, int dv, int n_hp);
+int lao_q8_encode(const float *x, int n, int H, int dk, int dv, int n_hp, const unsigned *masks,
+                  unsigned char *out);
+int lao_q8_decode(const unsigned char *in, int n, int H, int dk, int dv, int n_hp, const unsigned *masks, float *x);
+int lao_step_q8(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+                const double *src_pool, int src_slots, double *dst_pool, int dst_slots,
+                const int *read_slot, const int *write_slot, int B,
+                const double *q, const double *k, const double *v, int io_dtype,
+                const double *g, const double *beta, double scale, double *o, const unsigned *q8_masks);
+int lao_scan_q8(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+                const double *src_pool, int src_slots, const int *read_slot,
+                double *dst_pool, int dst_slots, const int *write_slot,
+                int n_seqs, const int *cu_seqlens, int total_tokens,
+                const double *q, const double *k, const double *v, int io_dtype,
+                const double *g, const double *beta, double scale, double *o,
+                int ckpt_every, const int *ckpt_cu, const int *ckpt_slots, const unsigned *q8_masks);
 
 int lao_pool_copy(unsigned char *pool, size_t slot_bytes, int n_slots, int n,
                   const int *src_slots, const int *dst_slots);

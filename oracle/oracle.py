@@ -37,6 +37,16 @@ def lib():
         _lib.lao_scan.restype = i
         _lib.lao_scan_ckpt.argtypes = _lib.lao_scan.argtypes + [i, p, p]
         _lib.lao_scan_ckpt.restype = i
+        _lib.lao_q8_tile_bytes.argtypes = [i, i, i]
+        _lib.lao_q8_tile_bytes.restype = sz
+        _lib.lao_q8_encode.argtypes = [p, i, i, i, i, i, p, p]
+        _lib.lao_q8_encode.restype = i
+        _lib.lao_q8_decode.argtypes = [p, i, i, i, i, i, p, p]
+        _lib.lao_q8_decode.restype = i
+        _lib.lao_step_q8.argtypes = [i, i, i, i, i, p, i, p, i, p, p, i, p, p, p, i, p, p, d, p, p]
+        _lib.lao_step_q8.restype = i
+        _lib.lao_scan_q8.argtypes = [i, i, i, i, i, p, i, p, p, i, p, i, p, i, p, p, p, i, p, p, d, p, i, p, p, p]
+        _lib.lao_scan_q8.restype = i
         _lib.lao_step_qgroups.argtypes = _lib.lao_step.argtypes
         _lib.lao_step_qgroups.restype = i
         _lib.lao_scan_qgroups.argtypes = _lib.lao_scan.argtypes
@@ -172,6 +182,78 @@ def scan_qgroups(rule, n_q_heads, cu_seqlens, q, k, v, g=None, beta=None, scale=
     return dst_pool, o, err
 
 
+def q8_tile_bytes(dk, dv, n_hp):
+    """Bytes of one (slot, head) tile in the mixed INT8 / BF16 ("q8") format."""
+    return int(lib().lao_q8_tile_bytes(dk, dv, n_hp))
+
+
+def _u32(masks):
+    return np.ascontiguousarray(masks, dtype=np.uint32)
+
+
+def q8_encode(x, n_hp, masks):
+    """x float32 [n, H, d_k, d_v] -> uint8 [n, H, tile bytes]; masks uint32 [H, d_k / 32]
+    (bit i of a head's mask: key channel i is kept in BF16)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    n, H, dk, dv = x.shape
+    out = np.zeros((n, H, q8_tile_bytes(dk, dv, n_hp)), dtype=np.uint8)
+    m = _u32(masks)
+    assert lib().lao_q8_encode(_ptr(x), n, H, dk, dv, n_hp, _ptr(m), _ptr(out)) == 0, "mask rows != n_hp"
+    return out
+
+
+def q8_decode(b, dk, dv, n_hp, masks):
+    """uint8 [n, H, tile bytes] -> float32 [n, H, d_k, d_v]."""
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    n, H, _ = b.shape
+    x = np.zeros((n, H, dk, dv), dtype=np.float32)
+    m = _u32(masks)
+    assert lib().lao_q8_decode(_ptr(b), n, H, dk, dv, n_hp, _ptr(m), _ptr(x)) == 0, "mask rows != n_hp"
+    return x
+
+
+def step_q8(rule, n_qk_heads, src_pool, q, k, v, g=None, beta=None, scale=1.0, *, masks,
+            dst_pool=None, io_dtype="f64", read_slot=None, write_slot=None):
+    """Decode step whose new states are stored in the q8 format (returned as decoded values)."""
+    src = _f64(src_pool)
+    dst = src.copy() if dst_pool is None else dst_pool
+    n_src, hv, dk, dv = src.shape
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B = q.shape[0]
+    g = None if g is None else _f64(g)
+    beta = None if beta is None else _f64(beta)
+    o = np.zeros((B, hv, dv), dtype=np.float64)
+    m = _u32(masks)
+    err = lib().lao_step_q8(RULES[rule], n_qk_heads, hv, dk, dv, _ptr(src), n_src, _ptr(dst), dst.shape[0],
+                            _ptr(_i32(read_slot)), _ptr(_i32(write_slot)), B, _ptr(q), _ptr(k), _ptr(v),
+                            DTYPES[io_dtype], _ptr(g), _ptr(beta), float(scale), _ptr(o), _ptr(m))
+    return dst, o, err
+
+
+def scan_q8(rule, n_qk_heads, cu_seqlens, q, k, v, g=None, beta=None, scale=1.0, *, masks,
+            src_pool=None, read_slot=None, dst_pool=None, write_slot=None, io_dtype="f64", ckpt_every=0,
+            ckpt_cu=None, ckpt_slots=None):
+    """Scan whose final states (and checkpoints) are stored in the q8 format."""
+    cu = _i32(cu_seqlens)
+    n_seqs = cu.shape[0] - 1
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, _, dk = q.shape
+    hv, dv = v.shape[1], v.shape[2]
+    if dst_pool is None:
+        dst_pool = np.zeros((n_seqs, hv, dk, dv), dtype=np.float64)
+    src = None if src_pool is None else _f64(src_pool)
+    n_src = 0 if src is None else src.shape[0]
+    g = None if g is None else _f64(g)
+    beta = None if beta is None else _f64(beta)
+    o = np.zeros((T, hv, dv), dtype=np.float64)
+    m = _u32(masks)
+    err = lib().lao_scan_q8(RULES[rule], n_qk_heads, hv, dk, dv, _ptr(src), n_src, _ptr(_i32(read_slot)),
+                            _ptr(dst_pool), dst_pool.shape[0], _ptr(_i32(write_slot)), n_seqs, _ptr(cu), T,
+                            _ptr(q), _ptr(k), _ptr(v), DTYPES[io_dtype], _ptr(g), _ptr(beta), float(scale), _ptr(o),
+                            int(ckpt_every), _ptr(_i32(ckpt_cu)), _ptr(_i32(ckpt_slots)), _ptr(m))
+    return dst_pool, o, err
+
+
 def readout_rearranged(rule, n_qk_heads, state, q, k, v, g=None, beta=None, scale=1.0):
     """o of one decode step in the rearranged form; state [B, H_v, d_k, d_v] (dense)."""
     S = _f64(state)
@@ -260,7 +342,7 @@ def set_threads(n):
 
 __all__ = ["round_bf16", "round_to", "step", "readout_rearranged", "scan", "pool_copy",
            "pool_gather", "pool_scatter", "pool_zero", "num_threads", "set_threads", "RULES", "DTYPES",
-           "step_qgroups", "scan_qgroups"]
+           "step_qgroups", "scan_qgroups", "q8_tile_bytes", "q8_encode", "q8_decode", "step_q8", "scan_q8"]
 
 if os.environ.get("LAO_THREADS"):
     set_threads(int(os.environ["LAO_THREADS"]))

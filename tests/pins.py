@@ -576,8 +576,112 @@ def pin_query_groups(orc):
     assert np.array_equal(S1, S2) and np.array_equal(o1, o2)
 
 
+# ---------------------------------------------------------------------------------
+# mixed INT8 / BF16 ("q8") state storage
+
+
+def _q8_masks(H, dk, n_hp, seed):
+    rng = np.random.default_rng(seed)
+    masks = np.zeros((H, dk // 32), dtype=np.uint32)
+    for h in range(H):
+        for i in rng.choice(dk, n_hp, replace=False):
+            masks[h, i // 32] |= np.uint32(1 << (i % 32))
+    return masks
+
+
+def _hp_rows(masks, h, dk):
+    return [i for i in range(dk) if (int(masks[h, i // 32]) >> (i % 32)) & 1]
+
+
+def pin_q8_page_figures(orc):
+    """With 1/8 of the key channels in BF16, the q8 tile of a 128 x 128 head holds
+    9.875 bits per value and saves 69.14 % of FP32 storage: the page's 9.9 bits and 69.1 %."""
+    G = {}
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "page_sizes.txt")
+    for line in open(path):
+        if line.strip() and not line.startswith("#"):
+            k, v = line.split()[:2]
+            G[k] = int(v)
+    nbytes = orc.q8_tile_bytes(128, 128, 16)
+    bits = 8.0 * nbytes / (128 * 128)
+    assert round(bits * 10) == G["damp_bits_per_value_x10"], bits
+    assert round((1 - bits / 32) * 1000) == G["damp_storage_reduction_pct_x10"], bits
+
+
+def pin_q8_codec(orc):
+    """The codec against its definition checked by properties: INT8 rows reproduce every
+    value within half a group step (s / 2, s = group absmax / 127), the group's largest
+    magnitude lands on code +-127, all-zero groups decode to zero, values k * 2^e of a
+    group whose absmax is 127 * 2^e come back exactly; BF16 rows equal torch's
+    round-to-nearest-even conversion bit for bit."""
+    rng = np.random.default_rng(12)
+    H, dk, dv, n_hp = 3, 64, 64, 8
+    masks = _q8_masks(H, dk, n_hp, 1)
+    x = (rng.standard_normal((2, H, dk, dv)) * 10.0 ** rng.integers(-6, 6, (2, H, dk, 1))).astype(np.float32)
+    x[0, 0, :, 32:] = 0.0                                                   # zero groups
+    e = rng.integers(-10, 10, (2, H, dk, 2))
+    x[1] = (rng.integers(-127, 128, (H, dk, dv)) * np.repeat(2.0 ** e[1], 32, axis=2)).astype(np.float32)
+    x[1, :, :, 0] = 127 * 2.0 ** e[1][:, :, 0]                             # absmax 127 * 2^e per group
+    x[1, :, :, 32] = -127 * 2.0 ** e[1][:, :, 1]
+    b = orc.q8_encode(x, n_hp, masks)
+    assert b.shape[2] == orc.q8_tile_bytes(dk, dv, n_hp)
+    y = orc.q8_decode(b, dk, dv, n_hp, masks)
+    for n in range(2):
+        for h in range(H):
+            hp = _hp_rows(masks, h, dk)
+            assert len(hp) == n_hp
+            ref = torch.tensor(x[n, h, hp]).to(torch.bfloat16).float().numpy()
+            assert np.array_equal(y[n, h, hp].view(np.uint32), ref.view(np.uint32)), "bf16 rows"
+            lo = [i for i in range(dk) if i not in hp]
+            xg = x[n, h, lo].reshape(len(lo), dv // 32, 32).astype(np.float64)
+            yg = y[n, h, lo].reshape(len(lo), dv // 32, 32).astype(np.float64)
+            amax = np.abs(xg).max(axis=2, keepdims=True)
+            step = amax / 127.0
+            assert np.all(np.abs(yg - xg) <= 0.5 * step * (1 + 1e-5) + 1e-45), "int8 rows within s / 2"
+            arg = np.abs(xg).argmax(axis=2)
+            top = np.take_along_axis(yg, arg[..., None], axis=2)[..., 0]
+            big = amax[..., 0] > 0
+            assert np.allclose(np.abs(top[big]), amax[..., 0][big], rtol=1e-6), "absmax on code 127"
+            assert np.all(yg[~big] == 0.0), "zero groups"
+            if n == 1:
+                assert np.array_equal(yg, xg), "exact dyadic groups"
+    # codes and scales sit where the layout says: row r8, group g -> scale at n8 * dv + 4 (r8 * ng + g)
+    n8, ng = dk - n_hp, dv // 32
+    scales = b[1, 0, n8 * dv:n8 * dv + 4 * n8 * ng].view(np.float32).reshape(n8, ng)
+    lo = [i for i in range(dk) if i not in _hp_rows(masks, 0, dk)]
+    assert np.array_equal(scales, (2.0 ** e[1][0][lo]).astype(np.float32)), "scale layout"
+    codes = b[1, 0, :n8 * dv].view(np.int8).reshape(n8, dv).astype(np.float64)
+    assert np.array_equal(codes * np.repeat(scales, 32, axis=1), x[1, 0, lo]), "code layout"
+
+
+def pin_q8_store_point(orc):
+    """Decode step and scan with q8 destinations: every stored tile is the codec applied to
+    the FP32-rounded state of the unquantised oracle, each head with its own mask."""
+    H, dk, dv, n_hp = 2, 64, 64, 8
+    masks = _q8_masks(H, dk, n_hp, 2)
+    inp = W.step_inputs(B=3, n_qk_heads=1, n_v_heads=H, d_k=dk, d_v=dv, rule="gated_delta", slot_map="dense",
+                        state_dtype=torch.float32, io_dtype=torch.float32, seed=24)
+    args = (np64(inp.q), np64(inp.k), np64(inp.v), np64(inp.g), np64(inp.beta))
+    ref, o_ref, _ = orc.step("gated_delta", 1, np64(inp.pool), *args, dst_dtype="f32")
+    got, o, err = orc.step_q8("gated_delta", 1, np64(inp.pool), *args, masks=masks)
+    assert err == 0 and np.array_equal(o, o_ref)
+    want = orc.q8_decode(orc.q8_encode(ref.astype(np.float32), n_hp, masks), dk, dv, n_hp, masks)
+    assert np.array_equal(got, want.astype(np.float64)), "step: q8 store"
+    sc = W.scan_inputs(lengths=[11, 4], n_qk_heads=1, n_v_heads=H, d_k=dk, d_v=dv, rule="kda",
+                       state_dtype=torch.float32, io_dtype=torch.float32, seed=25)
+    cu = sc.cu_seqlens.numpy()
+    args = (np64(sc.q), np64(sc.k), np64(sc.v), np64(sc.g), np64(sc.beta))
+    ref, _, _ = orc.scan("kda", 1, cu, *args, dst_dtype="f32")
+    got, _, err = orc.scan_q8("kda", 1, cu, *args, masks=masks)
+    assert err == 0
+    want = orc.q8_decode(orc.q8_encode(ref.astype(np.float32), n_hp, masks), dk, dv, n_hp, masks)
+    assert np.array_equal(got, want.astype(np.float64)), "scan: q8 store"
+
+
 ALL_PINS = [pin_bf16_rounding, pin_brute_force_all_rules, pin_gqa_grouping, pin_exact_rational,
             pin_linear_closed_form, pin_gated_closed_form, pin_beta0_g1_identity, pin_delta_stores_value,
             pin_rearranged_readout, pin_scan_structure, pin_wide_ranges_non_expansive,
             pin_long_sequence_bounded, pin_storage_rounding_points, pin_slots, pin_pool_ops,
-            pin_scan_checkpoints, pin_kda_reductions, pin_kda_wide_ranges_non_expansive, pin_query_groups]
+            pin_scan_checkpoints, pin_kda_reductions, pin_kda_wide_ranges_non_expansive, pin_query_groups,
+            pin_q8_page_figures, pin_q8_codec, pin_q8_store_point]
