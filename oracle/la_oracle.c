@@ -410,6 +410,111 @@ int lao_step_q8(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
                      read_slot, write_slot, B, q, k, v, io_dtype, g, beta, scale, o, q8_masks);
 }
 
+/* ---- short causal convolution fused ahead of the decode step ---------------------------
+ *
+ * "Gated DeltaNet" glossary, Engineering details: Conv1D is fused with the recurrence into
+ * one kernel.  The pages give nothing else; the reading taken: before the recurrence, the
+ * q, k and v projections of each token pass through a causal depthwise convolution of
+ * width W along time (per channel c: y_t = sum_{j<W} w[c][j] x_{t-W+1+j}, the W - 1 earlier
+ * inputs kept per request as the convolution state), optionally followed by SiLU
+ * (y / (1 + e^-y)), and q and k are optionally scaled to unit length per head
+ * (x / sqrt(|x|^2 + 1e-6)).  The convolution state is kept per state head: head h holds
+ * the histories of its q/k head's 2 d_k channels and of its own d_v v channels, so every
+ * state head owns its history (heads that share a q/k head hold equal copies).
+ *
+ * Layouts: xq, xk [B, H_qk, d_k], xv [B, H_v, d_v] (pre-convolution inputs, already in
+ * the io type); weights wq, wk [H_qk, d_k, W], wv [H_v, d_v, W]; convolution pools
+ * [n_slots, H_v, 2 d_k + d_v, W - 1] (q channels, then k, then v; oldest input first),
+ * read from read_slot[b] of conv_src and written to write_slot[b] of conv_dst like the
+ * recurrent state.  Post-convolution values are not rounded (the fused kernel keeps them
+ * in FP32 registers). */
+
+/* One (request, state head): post-convolution q, k (d_k each) and v (d_v) from the inputs
+ * and the history `hist` ([2 d_k + d_v][W - 1]); the new history goes to `hist_out`. */
+static void conv_head(int dk, int dv, int W, int act, int l2norm, const double *xq, const double *xk,
+                      const double *xv, const double *wq, const double *wk, const double *wv, const double *hist,
+                      double *hist_out, double *q, double *k, double *v)
+{
+    const int C = 2 * dk + dv;
+    for (int c = 0; c < C; ++c) {
+        const double *w = c < dk ? wq + (size_t)c * W : c < 2 * dk ? wk + (size_t)(c - dk) * W
+                                                                  : wv + (size_t)(c - 2 * dk) * W;
+        const double x = c < dk ? xq[c] : c < 2 * dk ? xk[c - dk] : xv[c - 2 * dk];
+        const double *h = hist + (size_t)c * (W - 1);
+        double y = w[W - 1] * x;
+        for (int j = 0; j < W - 1; ++j) y += w[j] * h[j];
+        if (act) y = y / (1.0 + exp(-y));
+        double *dstv = c < dk ? q + c : c < 2 * dk ? k + (c - dk) : v + (c - 2 * dk);
+        *dstv = y;
+        double *ho = hist_out + (size_t)c * (W - 1);
+        for (int j = 0; j < W - 2; ++j) ho[j] = h[j + 1];
+        if (W > 1) ho[W - 2] = x;
+    }
+    if (l2norm) {
+        double sq = 0.0, sk = 0.0;
+        for (int i = 0; i < dk; ++i) { sq += q[i] * q[i]; sk += k[i] * k[i]; }
+        const double rq = 1.0 / sqrt(sq + 1e-6), rk = 1.0 / sqrt(sk + 1e-6);
+        for (int i = 0; i < dk; ++i) { q[i] *= rq; k[i] *= rk; }
+    }
+}
+
+/* The convolution alone for B requests (dense: request b uses history b): post-convolution
+ * q, k [B, H_v, d_k] (per state head) and v [B, H_v, d_v]; the new histories to hist_out. */
+void lao_conv(int n_qk_heads, int n_v_heads, int dk, int dv, int W, int act, int l2norm, int B,
+              const double *xq, const double *xk, const double *xv, const double *wq, const double *wk,
+              const double *wv, const double *hist, double *hist_out, double *q, double *k, double *v)
+{
+    const size_t C = (size_t)(2 * dk + dv) * (W - 1);
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < n_v_heads; ++h) {
+            const int hq = head_group(n_qk_heads, n_v_heads, h);
+            const size_t t = (size_t)b * n_v_heads + h;
+            conv_head(dk, dv, W, act, l2norm, xq + ((size_t)b * n_qk_heads + hq) * dk,
+                      xk + ((size_t)b * n_qk_heads + hq) * dk, xv + t * dv, wq + (size_t)hq * dk * W,
+                      wk + (size_t)hq * dk * W, wv + (size_t)h * dv * W, hist + t * C, hist_out + t * C,
+                      q + t * dk, k + t * dk, v + t * dv);
+        }
+}
+
+/* Decode step with the convolution fused ahead of it: lao_conv on the histories of the
+ * read slots, then the step of lao_step with one q/k row per state head (H_qk = H_v for
+ * the recurrence); the new histories go to the write slots of conv_dst. */
+int lao_step_conv(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+                  const double *src_pool, int src_slots, double *dst_pool, int dst_slots, int dst_dtype,
+                  const int *read_slot, const int *write_slot, int B,
+                  const double *xq, const double *xk, const double *xv, int io_dtype,
+                  const double *g, const double *beta, double scale, double *o,
+                  int W, int act, int l2norm, const double *wq, const double *wk, const double *wv,
+                  const double *conv_src, double *conv_dst)
+{
+    const size_t C = (size_t)(2 * dk + dv) * (W - 1);
+    const size_t cslot = (size_t)n_v_heads * C;
+    int err = 0;
+    for (int b = 0; b < B; ++b) {
+        int rs = read_slot ? read_slot[b] : b, ws = write_slot ? write_slot[b] : b;
+        if (rs < 0 || rs >= src_slots) err |= LAO_ERR_READ_SLOT;
+        if (ws < 0 || ws >= dst_slots) err |= LAO_ERR_WRITE_SLOT;
+    }
+    if (err) return err;
+    double *hist = (double *)calloc((size_t)B * cslot + 1, sizeof(double));
+    double *hout = (double *)malloc(sizeof(double) * ((size_t)B * cslot + 1));
+    double *q = (double *)malloc(sizeof(double) * ((size_t)B * n_v_heads * dk + 1));
+    double *k = (double *)malloc(sizeof(double) * ((size_t)B * n_v_heads * dk + 1));
+    double *v = (double *)malloc(sizeof(double) * ((size_t)B * n_v_heads * dv + 1));
+    if (!hist || !hout || !q || !k || !v) { free(hist); free(hout); free(q); free(k); free(v); return -1; }
+    for (int b = 0; b < B; ++b)
+        memcpy(hist + (size_t)b * cslot, conv_src + (size_t)(read_slot ? read_slot[b] : b) * cslot,
+               sizeof(double) * cslot);
+    lao_conv(n_qk_heads, n_v_heads, dk, dv, W, act, l2norm, B, xq, xk, xv, wq, wk, wv, hist, hout, q, k, v);
+    err = step_impl(rule, n_v_heads, n_v_heads, 0, dk, dv, src_pool, src_slots, dst_pool, dst_slots, dst_dtype,
+                    read_slot, write_slot, B, q, k, v, io_dtype, g, beta, scale, o, NULL);
+    for (int b = 0; b < B; ++b)
+        memcpy(conv_dst + (size_t)(write_slot ? write_slot[b] : b) * cslot, hout + (size_t)b * cslot,
+               sizeof(double) * cslot);
+    free(hist); free(hout); free(q); free(k); free(v);
+    return err;
+}
+
 /* Decode step in the query-group direction: k [B, H_v, d_k], q [B, n_q_heads, d_k],
  * o [B, n_q_heads, d_v]; query head i reads the updated state of head i / (n_q_heads / H_v). */
 int lao_step_qgroups(int rule, int n_q_heads, int n_v_heads, int dk, int dv,

@@ -84,6 +84,17 @@ int lao_scan_q8(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
                 const double *g, const double *beta, double scale, double *o,
                 int ckpt_every, const int *ckpt_cu, const int *ckpt_slots, const unsigned *q8_masks);
 
+void lao_conv(int n_qk_heads, int n_v_heads, int dk, int dv, int W, int act, int l2norm, int B,
+              const double *xq, const double *xk, const double *xv, const double *wq, const double *wk,
+              const double *wv, const double *hist, double *hist_out, double *q, double *k, double *v);
+int lao_step_conv(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+                  const double *src_pool, int src_slots, double *dst_pool, int dst_slots, int dst_dtype,
+                  const int *read_slot, const int *write_slot, int B,
+                  const double *xq, const double *xk, const double *xv, int io_dtype,
+                  const double *g, const double *beta, double scale, double *o,
+                  int W, int act, int l2norm, const double *wq, const double *wk, const double *wv,
+                  const double *conv_src, double *conv_dst);
+
 int lao_pool_copy(unsigned char *pool, size_t slot_bytes, int n_slots, int n,
                   const int *src_slots, const int *dst_slots);
 int lao_pool_gather(const unsigned char *pool, size_t slot_bytes, int n_slots, int n,

@@ -47,6 +47,11 @@ def lib():
         _lib.lao_step_q8.restype = i
         _lib.lao_scan_q8.argtypes = [i, i, i, i, i, p, i, p, p, i, p, i, p, i, p, p, p, i, p, p, d, p, i, p, p, p]
         _lib.lao_scan_q8.restype = i
+        _lib.lao_conv.argtypes = [i, i, i, i, i, i, i, i, p, p, p, p, p, p, p, p, p, p, p]
+        _lib.lao_conv.restype = None
+        _lib.lao_step_conv.argtypes = [i, i, i, i, i, p, i, p, i, i, p, p, i, p, p, p, i, p, p, d, p,
+                                       i, i, i, p, p, p, p, p]
+        _lib.lao_step_conv.restype = i
         _lib.lao_step_qgroups.argtypes = _lib.lao_step.argtypes
         _lib.lao_step_qgroups.restype = i
         _lib.lao_scan_qgroups.argtypes = _lib.lao_scan.argtypes
@@ -254,6 +259,41 @@ def scan_q8(rule, n_qk_heads, cu_seqlens, q, k, v, g=None, beta=None, scale=1.0,
     return dst_pool, o, err
 
 
+def conv(n_qk_heads, xq, xk, xv, wq, wk, wv, hist, *, act=0, l2norm=0):
+    """The short causal convolution alone (see la_oracle.c): xq, xk [B, H_qk, d_k], xv
+    [B, H_v, d_v], weights [heads, channels, W], hist [B, H_v, 2 d_k + d_v, W - 1].
+    Returns (q, k [B, H_v, d_k], v [B, H_v, d_v], new hist)."""
+    xq, xk, xv, wq, wk, wv, hist = (_f64(a) for a in (xq, xk, xv, wq, wk, wv, hist))
+    B, hv, dv = xv.shape
+    dk = xq.shape[2]
+    W = wq.shape[2]
+    q = np.zeros((B, hv, dk)); k = np.zeros((B, hv, dk)); v = np.zeros((B, hv, dv))
+    out = np.zeros_like(hist)
+    lib().lao_conv(n_qk_heads, hv, dk, dv, W, int(act), int(l2norm), B, _ptr(xq), _ptr(xk), _ptr(xv), _ptr(wq),
+                   _ptr(wk), _ptr(wv), _ptr(hist), _ptr(out), _ptr(q), _ptr(k), _ptr(v))
+    return q, k, v, out
+
+
+def step_conv(rule, n_qk_heads, src_pool, xq, xk, xv, g, beta, scale, wq, wk, wv, conv_src, *, act=0, l2norm=0,
+              dst_pool=None, conv_dst=None, dst_dtype="f64", io_dtype="f64", read_slot=None, write_slot=None):
+    """Decode step with the convolution fused ahead of it.  Returns (dst_pool, conv_dst, o, err)."""
+    src = _f64(src_pool)
+    dst = src.copy() if dst_pool is None else dst_pool
+    csrc = _f64(conv_src)
+    cdst = csrc.copy() if conv_dst is None else conv_dst
+    n_src, hv, dk, dv = src.shape
+    xq, xk, xv, wq, wk, wv = (_f64(a) for a in (xq, xk, xv, wq, wk, wv))
+    B = xq.shape[0]
+    g = None if g is None else _f64(g)
+    beta = None if beta is None else _f64(beta)
+    o = np.zeros((B, hv, dv))
+    err = lib().lao_step_conv(RULES[rule], n_qk_heads, hv, dk, dv, _ptr(src), n_src, _ptr(dst), dst.shape[0],
+                              DTYPES[dst_dtype], _ptr(_i32(read_slot)), _ptr(_i32(write_slot)), B, _ptr(xq), _ptr(xk),
+                              _ptr(xv), DTYPES[io_dtype], _ptr(g), _ptr(beta), float(scale), _ptr(o), wq.shape[2],
+                              int(act), int(l2norm), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(csrc), _ptr(cdst))
+    return dst, cdst, o, err
+
+
 def readout_rearranged(rule, n_qk_heads, state, q, k, v, g=None, beta=None, scale=1.0):
     """o of one decode step in the rearranged form; state [B, H_v, d_k, d_v] (dense)."""
     S = _f64(state)
@@ -342,7 +382,8 @@ def set_threads(n):
 
 __all__ = ["round_bf16", "round_to", "step", "readout_rearranged", "scan", "pool_copy",
            "pool_gather", "pool_scatter", "pool_zero", "num_threads", "set_threads", "RULES", "DTYPES",
-           "step_qgroups", "scan_qgroups", "q8_tile_bytes", "q8_encode", "q8_decode", "step_q8", "scan_q8"]
+           "step_qgroups", "scan_qgroups", "q8_tile_bytes", "q8_encode", "q8_decode", "step_q8", "scan_q8", "conv",
+           "step_conv"]
 
 if os.environ.get("LAO_THREADS"):
     set_threads(int(os.environ["LAO_THREADS"]))

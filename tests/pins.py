@@ -679,9 +679,85 @@ def pin_q8_store_point(orc):
     assert np.array_equal(got, want.astype(np.float64)), "scan: q8 store"
 
 
+# ---------------------------------------------------------------------------------
+# short causal convolution ahead of the step
+
+
+def _conv_operands(seed, H_qk=1, H=2, dk=16, dv=8, W=4, T=9):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((T, H_qk, dk)), rng.standard_normal((T, H_qk, dk)), rng.standard_normal((T, H, dv)),
+            rng.standard_normal((H_qk, dk, W)), rng.standard_normal((H_qk, dk, W)), rng.standard_normal((H, dv, W)),
+            rng.standard_normal((1, H, 2 * dk + dv, W - 1)))
+
+
+def pin_conv_definition(orc):
+    """Token by token, the convolution equals numpy's full convolution of each channel's
+    input sequence (preceded by the W - 1 inputs of the initial history) with the reversed
+    weights; SiLU is y * expit(y); the q/k normalisation gives unit vectors; the history
+    after T tokens holds the last W - 1 inputs.  Two state heads over one q/k head both see
+    that head's channels (each keeps its own copy)."""
+    from scipy.special import expit
+    for W in (2, 4):
+        xq, xk, xv, wq, wk, wv, hist0 = _conv_operands(30 + W, W=W)
+        T, dk, dv = xq.shape[0], xq.shape[2], xv.shape[2]
+        for act, l2 in ((0, 0), (1, 0), (1, 1)):
+            hist = hist0.copy()
+            outs = []
+            for t in range(T):
+                q, k, v, hist = orc.conv(1, xq[t:t + 1], xk[t:t + 1], xv[t:t + 1], wq, wk, wv, hist, act=act,
+                                         l2norm=l2)
+                outs.append((q[0], k[0], v[0]))
+            for h in range(2):
+                for kind, xs, w, nch in (("q", xq[:, 0], wq[0], dk), ("k", xk[:, 0], wk[0], dk),
+                                         ("v", xv[:, h], wv[h], dv)):
+                    base = {"q": 0, "k": dk, "v": 2 * dk}[kind]
+                    for c in range(nch):
+                        seq = np.concatenate([hist0[0, h, base + c], xs[:, c]])
+                        y = np.convolve(seq, w[c][::-1])[W - 1:W - 1 + T]
+                        if act:
+                            y = y * expit(y)
+                        got = np.array([o[{"q": 0, "k": 1, "v": 2}[kind]][h, c] for o in outs])
+                        if l2 and kind != "v":
+                            ys = []
+                            for t in range(T):
+                                full = np.array([np.convolve(np.concatenate([hist0[0, h, base + cc], xs[:, cc]]),
+                                                             w[cc][::-1])[W - 1 + t] for cc in range(nch)])
+                                full = full * expit(full)
+                                ys.append(full[c] / np.sqrt(np.sum(full ** 2) + 1e-6))
+                            y = np.array(ys)
+                        close(got, y, 1e-12, f"conv W={W} act={act} l2={l2} {kind}{c} head {h}")
+                    last = np.concatenate([hist0[0, h, base:base + nch].T, xs.reshape(T, -1)[:, :nch]])[-(W - 1):].T
+                    close(hist[0, h, base:base + nch], last, 0.0 + 1e-300, f"history {kind}")
+
+
+def pin_conv_fused_step(orc):
+    """The fused step equals the convolution followed by the recurrence: states and outputs
+    against transition products of the post-convolution operands, and the histories go to
+    the write slots."""
+    xq, xk, xv, wq, wk, wv, hist = _conv_operands(40, T=3)
+    rng = np.random.default_rng(41)
+    B, H, dk, dv = 3, 2, 16, 8
+    pool = rng.standard_normal((5, H, dk, dv)) * 0.3
+    hists = rng.standard_normal((5, H, 2 * dk + dv, 3))
+    g, beta = rng.uniform(0.2, 1.0, (B, H)), rng.uniform(0.0, 1.0, (B, H))
+    rs, ws = np.array([4, 1, 2], np.int32), np.array([0, 1, 3], np.int32)
+    new, hnew, o, err = orc.step_conv("gated_delta", 1, pool, xq, xk, xv, g, beta, 0.9, wq, wk, wv, hists, act=1,
+                                      l2norm=1, read_slot=rs, write_slot=ws)
+    assert err == 0
+    q, k, v, hout = orc.conv(1, xq, xk, xv, wq, wk, wv, hists[rs], act=1, l2norm=1)
+    for b in range(B):
+        for h in range(H):
+            states, outs = brute_force_head("gated_delta", pool[rs[b], h], q[b, h][None], k[b, h][None],
+                                            v[b, h][None], g[b, h][None], beta[b, h][None], 0.9)
+            close(new[ws[b], h], states[0], 1e-12, "fused step state")
+            close(o[b, h], outs[0], 1e-12, "fused step output")
+    close(hnew[ws], hout, 1e-300, "histories to the write slots")
+    assert np.array_equal(hnew[4], hists[4]) and np.array_equal(new[4], pool[4]), "read-only slot untouched"
+
+
 ALL_PINS = [pin_bf16_rounding, pin_brute_force_all_rules, pin_gqa_grouping, pin_exact_rational,
             pin_linear_closed_form, pin_gated_closed_form, pin_beta0_g1_identity, pin_delta_stores_value,
             pin_rearranged_readout, pin_scan_structure, pin_wide_ranges_non_expansive,
             pin_long_sequence_bounded, pin_storage_rounding_points, pin_slots, pin_pool_ops,
             pin_scan_checkpoints, pin_kda_reductions, pin_kda_wide_ranges_non_expansive, pin_query_groups,
-            pin_q8_page_figures, pin_q8_codec, pin_q8_store_point]
+            pin_q8_page_figures, pin_q8_codec, pin_q8_store_point, pin_conv_definition, pin_conv_fused_step]

@@ -51,6 +51,13 @@ MUTANTS = [
     ("q8_mask_ignored", "return (int)((mask[i / 32] >> (i % 32)) & 1u);", "return 0 * (int)mask[i / 32];"),
     ("q8_first_head_mask", "round_tile(S, dk, dv, dst_dtype, q8_masks ? q8_masks + (size_t)h * (dk / 32) : NULL);\n            free(u);\n        }\n    }\n\n    for (int b",
      "round_tile(S, dk, dv, dst_dtype, q8_masks);\n            free(u);\n        }\n    }\n\n    for (int b"),
+    ("conv_window_shifted", "for (int j = 0; j < W - 1; ++j) y += w[j] * h[j];",
+     "for (int j = 0; j < W - 1; ++j) y += w[j + 1] * h[j];"),
+    ("conv_history_not_shifted", "for (int j = 0; j < W - 2; ++j) ho[j] = h[j + 1];",
+     "for (int j = 0; j < W - 2; ++j) ho[j] = h[j];"),
+    ("conv_silu_sign", "if (act) y = y / (1.0 + exp(-y));", "if (act) y = y / (1.0 + exp(y));"),
+    ("conv_norm_shared", "const double rq = 1.0 / sqrt(sq + 1e-6), rk = 1.0 / sqrt(sk + 1e-6);",
+     "const double rq = 1.0 / sqrt(sq + 1e-6), rk = rq;"),
     ("gather_wrong_slot", "memcpy(dense + (size_t)i * slot_bytes, pool + (size_t)slots[i] * slot_bytes, slot_bytes);",
      "memcpy(dense + (size_t)i * slot_bytes, pool + (size_t)i * slot_bytes, slot_bytes);"),
 ]
