@@ -10,8 +10,8 @@
  *   running state is decayed by a gate, corrected by a rank-one delta-rule term and
  *   projected by the query.
  *   "Seven Architectures Replacing KV Cache With Bounded Mutable State", section
- *   "ONNX LinearAttention / FlashInfer": update_rule in {linear (basic additive),
- *   gated (exponential decay), delta (delta rule without decay), gated_delta}; state
+ *   "ONNX LinearAttention / FlashInfer": update_rule in {linear (plain additive update),
+ *   gated (update decayed by a gate), delta (delta correction, no gate), gated_delta}; state
  *   tensors past_state / present_state of shape (B, H_kv, d_k, d_v).
  *   Same page, section "Kimi Linear": the channel-wise gate of Kimi Delta Attention,
  *   S_t = Diag(alpha_t) S_{t-1} + beta_t k_t (v_t - (Diag(alpha_t) S_{t-1})^T k_t)^T with
@@ -106,9 +106,10 @@ double lao_round_to(double x, int dtype)
  * code 3, "q8"), per (slot, head) tile of d_k x d_v:
  *   - a per-head mask of d_k bits marks the n_hp high-precision key channels (rows);
  *   - every other row is stored as INT8 codes in groups of 32 consecutive columns, each
- *     group with an FP32 scale s = absmax / 127 (absmax of the group's FP32 values);
- *     code = clamp(rint(x * (127 / absmax)), -127, 127), decoded as code * s; a group of
- *     zeros has s = 0 and codes 0;
+ *     group with an FP32 scale s = absmax * fl(1/127) (absmax of the group's FP32 values)
+ *     and inverse scale inv = fl(1/absmax) * 127 (every operation a correctly rounded FP32
+ *     one); code = rint(x * inv) clamped to [-127, 127] (NaN to 0), decoded as code * s;
+ *     a group of zeros has s = inv = 0 and codes 0;
  *   - high-precision rows are stored in BF16 (round to nearest even).
  * Byte layout of a tile: codes [d_k - n_hp][d_v] int8, then scales [d_k - n_hp][d_v / 32]
  * float32, then BF16 rows [n_hp][d_v]; rows of each block in increasing row index.  The
@@ -153,11 +154,13 @@ static void q8_encode_tile(const float *x, int dk, int dv, int n_hp, const unsig
         for (int gi = 0; gi < ng; ++gi) {
             float amax = 0.0f;
             for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(row[gi * 32 + j]));
-            const float s = amax > 0.0f ? amax / 127.0f : 0.0f;
-            const float inv = amax > 0.0f ? 127.0f / amax : 0.0f;
+            const float k127 = 1.0f / 127.0f;
+            const float s = amax > 0.0f ? amax * k127 : 0.0f;
+            const float inv = amax > 0.0f ? (1.0f / amax) * 127.0f : 0.0f;
             memcpy(sc + ((size_t)r8 * ng + gi) * 4, &s, 4);
             for (int j = 0; j < 32; ++j) {
-                const float c = fminf(fmaxf(rintf(row[gi * 32 + j] * inv), -127.0f), 127.0f);
+                const float y = rintf(row[gi * 32 + j] * inv);
+                const float c = isnan(y) ? 0.0f : fminf(fmaxf(y, -127.0f), 127.0f);
                 out[(size_t)r8 * dv + gi * 32 + j] = (unsigned char)(signed char)c;
             }
         }
@@ -573,7 +576,7 @@ void lao_readout_rearranged(int rule, int n_qk_heads, int n_v_heads, int dk, int
 /* ---- token-serial scan over packed variable-length sequences -------------------- */
 
 /* Scan with intermediate checkpoints ("Gated DeltaNet" glossary, Why it matters:
- * hybrid prefix caching keeps checkpoint slots aligned to KV block boundaries; "Seven
+ * hybrid prefix caching keeps checkpoint slots at KV-cache block boundaries; "Seven
  * Architectures ...", Limitations: state snapshots for speculative-decoding rollback).
  * With ckpt_every > 0, checkpoint j of sequence s (j < ckpt_cu[s+1] - ckpt_cu[s]) is the
  * state after the sequence's first (j + 1) * ckpt_every tokens, rounded to dst_dtype and

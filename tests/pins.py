@@ -611,7 +611,8 @@ def pin_q8_page_figures(orc):
 
 def pin_q8_codec(orc):
     """The codec against its definition checked by properties: INT8 rows reproduce every
-    value within half a group step (s / 2, s = group absmax / 127), the group's largest
+    value within half a group step (s / 2, s = group absmax / 127, plus the few FP32
+    roundings of s and of the inverse scale: 1e-4 s), the group's largest
     magnitude lands on code +-127, all-zero groups decode to zero, values k * 2^e of a
     group whose absmax is 127 * 2^e come back exactly; BF16 rows equal torch's
     round-to-nearest-even conversion bit for bit."""
@@ -638,7 +639,7 @@ def pin_q8_codec(orc):
             yg = y[n, h, lo].reshape(len(lo), dv // 32, 32).astype(np.float64)
             amax = np.abs(xg).max(axis=2, keepdims=True)
             step = amax / 127.0
-            assert np.all(np.abs(yg - xg) <= 0.5 * step * (1 + 1e-5) + 1e-45), "int8 rows within s / 2"
+            assert np.all(np.abs(yg - xg) <= step * (0.5 + 1e-4) + 1e-45), "int8 rows within s / 2"
             arg = np.abs(xg).argmax(axis=2)
             top = np.take_along_axis(yg, arg[..., None], axis=2)[..., 0]
             big = amax[..., 0] > 0

@@ -46,8 +46,7 @@ MUTANTS = [
      "memcpy(dst_pool + (size_t)(read_slot ? read_slot[b] : b) * slot, next + (size_t)b * slot, sizeof(double) * slot);"),
     ("checkpoint_off_by_one", "const int pos = t - cu_seqlens[s] + 1;", "const int pos = t - cu_seqlens[s];"),
     ("q8_truncates", "rintf(row[gi * 32 + j] * inv)", "truncf(row[gi * 32 + j] * inv)"),
-    ("q8_scale_by_128", "const float s = amax > 0.0f ? amax / 127.0f : 0.0f;",
-     "const float s = amax > 0.0f ? amax / 128.0f : 0.0f;"),
+    ("q8_scale_by_128", "const float k127 = 1.0f / 127.0f;", "const float k127 = 1.0f / 128.0f;"),
     ("q8_mask_ignored", "return (int)((mask[i / 32] >> (i % 32)) & 1u);", "return 0 * (int)mask[i / 32];"),
     ("q8_first_head_mask", "round_tile(S, dk, dv, dst_dtype, q8_masks ? q8_masks + (size_t)h * (dk / 32) : NULL);\n            free(u);\n        }\n    }\n\n    for (int b",
      "round_tile(S, dk, dv, dst_dtype, q8_masks);\n            free(u);\n        }\n    }\n\n    for (int b"),
