@@ -43,6 +43,7 @@ METRIC = "state-update HBM GB/s (% of B200 peak) and decode tokens/s per layer s
 SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_SM_MHZ = 1965.0
+FALLBACK_BF16_TFLOPS = 1590.0
 FP32_LANES_PER_SM = 128
 
 # --------------------------------------------------------------------------------------
@@ -50,22 +51,32 @@ FP32_LANES_PER_SM = 128
 
 
 def step_bytes_and_flops(*, B, n_qk_heads, n_v_heads, d_k, d_v, state_bytes, io_bytes, rule, state_only=False,
-                         slot_arrays=0):
+                         slot_arrays=0, n_q_heads=0):
     """Bytes and flops of one decode step over B requests.
 
     Bytes: the state is read and written once per (request, head) tile; q and k once
     per q/k head; v and o once per state head; g and beta (4 bytes) where the rule uses
-    them; int32 slot ids.  Flops: 6 per state element (S^T k, S^T q and the update, 2
-    each), the count of the "SSM / linear-RNN decode" page."""
+    them (kda: d_k decays of 4 bytes); int32 slot ids.  Flops: 6 per state element
+    (S^T k, S^T q and the update, 2 each), the count of the "SSM / linear-RNN decode"
+    page.  Query-group direction (n_q_heads > 0): k per state head, n_q_heads query and
+    output rows, 2 more flops per state element for each extra query of a group."""
     elems = B * n_v_heads * d_k * d_v
     state = 2 * elems * state_bytes
-    flops = 6 * elems
+    group = n_q_heads // n_v_heads if n_q_heads else 1
+    flops = (4 + 2 * group) * elems
     if state_only:
         return state, flops
-    qk = 2 * B * n_qk_heads * d_k * io_bytes
-    vo = 2 * B * n_v_heads * d_v * io_bytes
-    gates = B * n_v_heads * 4 * ((rule in ("gated", "gated_delta")) + (rule in ("delta", "gated_delta")))
-    return state + qk + vo + gates + 4 * B * slot_arrays, flops
+    n_q = n_q_heads if n_q_heads else n_qk_heads
+    n_o = n_q_heads if n_q_heads else n_v_heads
+    qk = B * (n_q + n_qk_heads) * d_k * io_bytes
+    vo = B * (n_v_heads + n_o) * d_v * io_bytes
+    return state + qk + vo + B * gate_bytes_per_head(rule, d_k) * n_v_heads + 4 * B * slot_arrays, flops
+
+
+def gate_bytes_per_head(rule, d_k):
+    """FP32 gate and beta bytes of one token and state head."""
+    g = {"gated": 4, "gated_delta": 4, "kda": 4 * d_k}.get(rule, 0)
+    return g + (4 if rule in ("delta", "gated_delta", "kda") else 0)
 
 
 def scan_bytes_and_flops(*, T, n_seqs, n_qk_heads, n_v_heads, d_k, d_v, io_bytes, rule, final_state_bytes,
@@ -73,7 +84,7 @@ def scan_bytes_and_flops(*, T, n_seqs, n_qk_heads, n_v_heads, d_k, d_v, io_bytes
     """Bytes and flops of one scan: every token's q, k (per q/k head), v, o (per state
     head), gates; the final state stored once (and read once when initialised)."""
     per_tok = 2 * n_qk_heads * d_k * io_bytes + 2 * n_v_heads * d_v * io_bytes
-    per_tok += n_v_heads * 4 * ((rule in ("gated", "gated_delta")) + (rule in ("delta", "gated_delta")))
+    per_tok += n_v_heads * gate_bytes_per_head(rule, d_k)
     state = n_seqs * n_v_heads * d_k * d_v * (final_state_bytes + init_state_bytes)
     return T * per_tok + state + 4 * (n_seqs + 1), 6 * T * n_v_heads * d_k * d_v
 
@@ -88,9 +99,10 @@ def measured_peaks():
         with open(path) as fh:
             d = json.load(fh)
         return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", FALLBACK_SM_MHZ)),
-                "source": "measured"}
+                "bf16_tflops": float(d.get("bf16_tflops", FALLBACK_BF16_TFLOPS)), "source": "measured"}
     except Exception:
-        return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": FALLBACK_SM_MHZ, "source": "fallback"}
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": FALLBACK_SM_MHZ, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "source": "fallback"}
 
 
 def fp32_alu_peak_tflops(sm_count, mhz):
@@ -265,13 +277,33 @@ class DecodeRunner:
         import torch
         from gated_deltanet_recurrent_la_b200 import lastate as L
         self.L = L
+        self.torch = torch
         self.inp = inp
-        self.pool_t = to_dev(inp.pool)
-        self.pool = L.Pool(self.pool_t, inp.n_qk_heads)
+        if inp.state_dtype == torch.uint8:
+            # q8 storage: the FP32 initial values are encoded into the pool by the library
+            n_hp, mask = inp.extra["n_hp"], to_dev(inp.extra["hp_mask"])
+            n, H, dk, dv = inp.pool.shape
+            self.pool_t = torch.zeros(n, H, L.q8_tile_bytes(dk, dv, n_hp), dtype=torch.uint8, device="cuda")
+            self.pool = L.Pool.q8(self.pool_t, inp.n_qk_heads, dk, dv, n_hp, mask)
+            err = torch.zeros(1, dtype=torch.int32, device="cuda")
+            L.check(L.la_state_pool_encode(self.pool, torch.arange(n, dtype=torch.int32, device="cuda"),
+                                           to_dev(inp.pool.float()), err))
+            torch.cuda.synchronize()
+            if int(err.item()):
+                raise RuntimeError(f"q8 encode reported {int(err.item())}")
+        else:
+            self.pool_t = to_dev(inp.pool)
+            self.pool = L.Pool(self.pool_t, inp.n_qk_heads)
+        self.conv = None
+        if "width" in inp.extra:  # the short causal convolution ahead of the step
+            x = inp.extra
+            self.hist_t = to_dev(x["hist"])
+            self.conv = L.Conv(to_dev(x["w_q"]), to_dev(x["w_k"]), to_dev(x["w_v"]), self.hist_t,
+                               activation=x["activation"], qk_l2norm=x["qk_l2norm"])
         self.q, self.k, self.v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
         self.g, self.beta = to_dev(inp.g), to_dev(inp.beta)
         B = inp.q.shape[0]
-        self.o = torch.empty(B, inp.n_v_heads, inp.d_v, dtype=inp.io_dtype, device="cuda")
+        self.o = torch.empty(B, inp.n_q_heads or inp.n_v_heads, inp.d_v, dtype=inp.io_dtype, device="cuda")
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
         self.sets = []
         if inp.read_slot is None:
@@ -292,18 +324,64 @@ class DecodeRunner:
             self.sets = [(to_dev(r), to_dev(w)) for r, w in self.sets]
         self.B = B
 
-    def step(self, i=0, stream=None):
-        r, w = self.sets[i % len(self.sets)]
-        st = self.L.la_state_step(self.inp.rule, self.pool, r, self.pool, w, self.q, self.k, self.v, self.g,
-                                  self.beta, self.inp.scale, self.o, self.err, stream=stream)
+    def call(self, r, w, q, k, v, g, beta, o, stream=None):
+        """One decode step through the C ABI (the query-group entry point when the
+        workload has query groups)."""
+        if self.conv is not None:
+            st = self.L.la_state_step_conv(self.inp.rule, self.pool, r, self.pool, w, self.conv, q, k, v, g, beta,
+                                           self.inp.scale, o, self.err, stream=stream)
+        else:
+            fn = self.L.la_state_step_qgroups if self.inp.n_q_heads else self.L.la_state_step
+            st = fn(self.inp.rule, self.pool, r, self.pool, w, q, k, v, g, beta, self.inp.scale, o, self.err,
+                    stream=stream)
         if st != 0:
             raise self.L.LAError(st)
 
+    def step(self, i=0, stream=None):
+        r, w = self.sets[i % len(self.sets)]
+        self.call(r, w, self.q, self.k, self.v, self.g, self.beta, self.o, stream)
+
     def bytes_flops(self):
         i = self.inp
-        return step_bytes_and_flops(B=self.B, n_qk_heads=i.n_qk_heads, n_v_heads=i.n_v_heads, d_k=i.d_k, d_v=i.d_v,
-                                    state_bytes=i.pool.element_size(), io_bytes=i.q.element_size(), rule=i.rule,
-                                    slot_arrays=0 if i.read_slot is None else 2)
+        b, f = step_bytes_and_flops(B=self.B, n_qk_heads=i.n_qk_heads, n_v_heads=i.n_v_heads, d_k=i.d_k, d_v=i.d_v,
+                                    state_bytes=state_bytes_per_value(i), io_bytes=i.q.element_size(), rule=i.rule,
+                                    slot_arrays=0 if i.read_slot is None else 2, n_q_heads=i.n_q_heads)
+        if self.conv is not None:
+            # histories read and written per (request, head); the weights once
+            x = i.extra
+            b += 2 * self.B * i.n_v_heads * (2 * i.d_k + i.d_v) * (x["width"] - 1) * i.q.element_size()
+            b += 4 * x["width"] * (2 * i.n_qk_heads * i.d_k + i.n_v_heads * i.d_v)
+            f += 2 * self.B * i.n_v_heads * (2 * i.d_k + i.d_v) * x["width"]
+        return b, f
+
+
+CHUNK = 64  # tokens per chunk of the tensor-core prefill
+
+
+def chunk_mma_flops(lengths, n_v_heads, d_k, d_v, rule):
+    """Tensor-core flops the chunked prefill executes (whole chunks, the last one padded):
+    per chunk and head Q K^T and (Q K^T . M) U (2 C^2 d_k and 2 C^2 d_v), Q S0 and the
+    state update K^T U (2 C d_k d_v each); the delta rules add K K^T, W = T K, U~ = T V and
+    W S0 (2 C^2 d_k, 2 C^2 d_k, 2 C^2 d_v, 2 C d_k d_v)."""
+    C = CHUNK
+    per = 2 * C * C * d_k + 2 * C * C * d_v + 4 * C * d_k * d_v
+    if rule in ("delta", "gated_delta"):
+        per += 4 * C * C * d_k + 2 * C * C * d_v + 2 * C * d_k * d_v
+    chunks = sum((int(n) + C - 1) // C for n in lengths)
+    return chunks * n_v_heads * per
+
+
+def tensor_roofline(run, inp, ms, peaks):
+    """Roofline object of the chunked prefill: executed MMA flops against the measured dense
+    BF16 peak (a cuBLAS GEMM, tcgen05); this kernel issues mma.sync."""
+    lens = (inp.cu_seqlens[1:] - inp.cu_seqlens[:-1]).tolist()
+    tf = chunk_mma_flops(lens, inp.n_v_heads, inp.d_k, inp.d_v, inp.rule) / (ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)
+    return {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+            "traffic": recorded_traffic("chunk", "prefill32"),
+            "peak_note": "measured dense BF16 GEMM (MEASURED_PEAKS.json bf16_tflops); the kernel uses mma.sync "
+                         "BF16 m16n8k16, whose own ceiling on this part is about a third of that",
+            "hbm_gb_s": run.bytes_flops()[0] / (ms * 1e-3) / 1e9, "kernel": "la::chunk_scan_kernel"}
 
 
 class ScanRunner:
@@ -519,9 +597,7 @@ def time_e2e(run: DecodeRunner, steps, warmup, world):
             if dev_free[b] is not None:
                 cs.wait_event(dev_free[b])         # o of step j-2 has reached the host
             q, k, v, g, beta, rs, ws = vs[b]
-            st = L.la_state_step(inp.rule, run.pool, rs, run.pool, ws, q, k, v, g, beta, inp.scale, outs[b], run.err)
-            if st != 0:
-                raise L.LAError(st)
+            run.call(rs, ws, q, k, v, g, beta, outs[b])
             kev[b] = torch.cuda.Event()
             kev[b].record(cs)
             with torch.cuda.stream(sd):
@@ -567,6 +643,15 @@ def time_e2e(run: DecodeRunner, steps, warmup, world):
 # oracle on the host cores (baseline only)
 
 
+def state_bytes_per_value(inp):
+    """Stored bytes per state value of a workload (q8: the tile bytes over d_k x d_v)."""
+    import torch
+    if inp.state_dtype == torch.uint8:
+        n_hp, dk, dv = inp.extra["n_hp"], inp.d_k, inp.d_v
+        return ((dk - n_hp) * dv + (dk - n_hp) * (dv // 32) * 4 + n_hp * dv * 2) / (dk * dv)
+    return inp.pool.element_size()
+
+
 def cpu_baseline_decode(inp, budget_s=10.0):
     """The CPU oracle as it stands (fp64, OpenMP over tiles) on the decode workload: whole
     steps repeated until about budget_s of wall time.  Returns (ms per step, threads,
@@ -581,12 +666,28 @@ def cpu_baseline_decode(inp, budget_s=10.0):
     st = "bf16" if inp.state_dtype.itemsize == 2 else "f32"
     io = "bf16" if inp.io_dtype.itemsize == 2 else "f32"
     dst = pool.copy()
+    if "width" in inp.extra:
+        hist = inp.extra["hist"].double().numpy()
+        hist_out = hist.copy()
     times = []
     t_end = time.perf_counter() + budget_s
     while time.perf_counter() < t_end or not times:
         t0 = time.perf_counter()
-        oracle.step(inp.rule, inp.n_qk_heads, pool, *args, inp.scale, dst_pool=dst, dst_dtype=st, io_dtype=io,
-                    read_slot=rs, write_slot=ws)
+        if "width" in inp.extra:
+            x = inp.extra
+            oracle.step_conv(inp.rule, inp.n_qk_heads, pool, *args, inp.scale, x["w_q"].double().numpy(),
+                             x["w_k"].double().numpy(), x["w_v"].double().numpy(), hist, act=x["activation"],
+                             l2norm=x["qk_l2norm"], dst_pool=dst, conv_dst=hist_out, dst_dtype=st, io_dtype=io,
+                             read_slot=rs, write_slot=ws)
+        elif inp.state_dtype.itemsize == 1:
+            oracle.step_q8(inp.rule, inp.n_qk_heads, pool, *args, inp.scale, dst_pool=dst, io_dtype=io,
+                           read_slot=rs, write_slot=ws, masks=inp.extra["hp_mask"].numpy().view(np.uint32))
+        elif inp.n_q_heads:
+            oracle.step_qgroups(inp.rule, inp.n_q_heads, pool, *args, inp.scale, dst_pool=dst, dst_dtype=st,
+                                io_dtype=io, read_slot=rs, write_slot=ws)
+        else:
+            oracle.step(inp.rule, inp.n_qk_heads, pool, *args, inp.scale, dst_pool=dst, dst_dtype=st, io_dtype=io,
+                        read_slot=rs, write_slot=ws)
         times.append(time.perf_counter() - t0)
     return 1e3 * statistics.median(times), oracle.num_threads(), f"{len(times)} whole decode steps of the workload"
 
@@ -596,17 +697,24 @@ def cpu_baseline_decode(inp, budget_s=10.0):
 
 def build_runner(name, seed=0, prefill_seqs=32, ckpt_every=0, chunked=False):
     from gated_deltanet_recurrent_la_b200 import workloads as W
-    inp = W.prefill32(seed, prefill_seqs) if name == "prefill32" else W.WORKLOADS[name](seed)
+    if name in ("prefill32", "kda_prefill32"):
+        inp = W.WORKLOADS[name](seed, prefill_seqs)
+    else:
+        inp = W.WORKLOADS[name](seed)
     if inp.kind == "scan":
         return ScanRunner(inp, ckpt_every, chunked), inp
-    n_sets = 4 if name == "decode64" else 1
+    n_sets = 4 if name in ("decode64", "kda_decode64", "qgroup_decode256", "q8_decode64", "conv_decode64") else 1
     return DecodeRunner(inp, n_sets=n_sets, seed=seed), inp
 
 
 def describe(name, inp):
     d = {"workload": name, "rule": inp.rule, "n_qk_heads": inp.n_qk_heads, "n_v_heads": inp.n_v_heads,
-         "d_k": inp.d_k, "d_v": inp.d_v, "state": str(inp.state_dtype).replace("torch.", ""),
+         "d_k": inp.d_k, "d_v": inp.d_v,
+         "state": (f"q8 (INT8 codes, FP32 scale per 32 columns, {inp.extra['n_hp']} of {inp.d_k} key channels "
+                   f"BF16)" if inp.state_dtype.itemsize == 1 else str(inp.state_dtype).replace("torch.", "")),
          "io": str(inp.io_dtype).replace("torch.", "")}
+    if inp.n_q_heads:
+        d["n_q_heads"] = inp.n_q_heads
     if inp.kind == "step":
         d.update(B=int(inp.q.shape[0]), pool_slots=int(inp.pool.shape[0]),
                  slot_map="dense" if inp.read_slot is None else
@@ -642,13 +750,15 @@ def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_ev
             row["config"]["checkpoints"] = run.n_ckpt
         if chunked:
             row["config"]["algorithm"] = "chunked (64-token WY/UT form, BF16 tensor-core products)"
-            # the same algorithmic flops as the token-serial form (6 per state element per token);
-            # the chunked form executes more multiply-adds, on the tensor cores
             row["hbm"] = {"achieved_gb_s": row["gb_s"], "frac_of_measured": row["gb_s"] / peaks["hbm_gbs"]}
-        row["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
-                           "traffic": recorded_traffic("scan", name), "hbm_gb_s": row["gb_s"],
-                           "effective_state_gb_s": run.T * inp.n_v_heads * 2 * inp.d_k * inp.d_v * 4 / (ms * 1e-3) / 1e9,
-                           "peak_note": "SMs x 128 FP32 lanes x 2 x max SM clock"}
+            row["token_serial_equivalent_tflops"] = tf  # 6 flops per state element per token, for comparison
+            row["roofline"] = tensor_roofline(run, inp, ms, peaks)
+        else:
+            row["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
+                               "traffic": recorded_traffic("scan", name), "hbm_gb_s": row["gb_s"],
+                               "effective_state_gb_s": run.T * inp.n_v_heads * 2 * inp.d_k * inp.d_v * 4 /
+                               (ms * 1e-3) / 1e9,
+                               "peak_note": "SMs x 128 FP32 lanes x 2 x max SM clock"}
     del run
     return row
 
@@ -659,9 +769,13 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode64", choices=["decode64", "decode512", "mamba2", "prefill32"])
+    ap.add_argument("--workload", default="decode64",
+                    choices=["decode64", "decode512", "mamba2", "prefill32", "kda_decode64", "kda_prefill32",
+                             "qgroup_decode256", "q8_decode64", "conv_decode64"])
     ap.add_argument("--rows", default="all", choices=["all", "none"])
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--scan-algo", default="serial", choices=["serial", "chunked"],
+                    help="prefill workload: token-serial scan or the chunked tensor-core form")
     ap.add_argument("--prefill-seqs", type=int, default=32,
                     help="sequences of the prefill workload (fewer only to profile a smaller case)")
     a = ap.parse_args()
@@ -679,7 +793,7 @@ def main():
     sampler = ClockSampler(local)
     sampler.start()
 
-    run, inp = build_runner(a.workload, prefill_seqs=a.prefill_seqs)
+    run, inp = build_runner(a.workload, prefill_seqs=a.prefill_seqs, chunked=a.scan_algo == "chunked")
     nbytes, flops = run.bytes_flops()
     ms = time_back_to_back(run, a.steps, a.warmup, world, sampler)
     sampler.stop()
@@ -707,8 +821,11 @@ def main():
         alu = fp32_alu_peak_tflops(sm_count, peaks["sm_max_mhz"])
         tf = flops / (ms * 1e-3) / 1e12
         out["tokens_per_s"] = world * run.T / (ms * 1e-3)
-        out["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
-                           "traffic": recorded_traffic("scan", a.workload), "kernel": "la::scan_kernel"}
+        if a.scan_algo == "chunked":
+            out["roofline"] = tensor_roofline(run, inp, ms, peaks)
+        else:
+            out["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
+                               "traffic": recorded_traffic("scan", a.workload), "kernel": "la::scan_kernel"}
     out["gpu_launches"] = a.steps
     out["clocks"] = sampler.summary()
 
@@ -725,10 +842,11 @@ def main():
 
     if a.rows == "all":
         rows = {}
-        for name in ("decode512", "mamba2", "prefill32"):
+        for name in ("decode512", "mamba2", "prefill32", "kda_decode64", "kda_prefill32", "qgroup_decode256",
+                     "q8_decode64", "conv_decode64"):
             if name == a.workload:
                 continue
-            k = a.steps if name != "prefill32" else max(3, min(a.steps, 20))
+            k = a.steps if "prefill" not in name else max(3, min(a.steps, 20))
             rows[name] = measure_row(name, min(k, 500), a.warmup, world, peaks, sm_count, flush)
             torch.cuda.empty_cache()
         rows["prefill32_ckpt256"] = measure_row("prefill32", max(3, min(a.steps, 20)), a.warmup, world, peaks,
@@ -777,9 +895,9 @@ def reference_arm(a, rank, world):
         print(json.dumps({"impl": "reference", "unavailable": "the reference arm times decode workloads only"}))
         return 0
     nbytes, _ = step_bytes_and_flops(B=int(inp.q.shape[0]), n_qk_heads=inp.n_qk_heads, n_v_heads=inp.n_v_heads,
-                                     d_k=inp.d_k, d_v=inp.d_v, state_bytes=inp.pool.element_size(),
+                                     d_k=inp.d_k, d_v=inp.d_v, state_bytes=state_bytes_per_value(inp),
                                      io_bytes=inp.q.element_size(), rule=inp.rule,
-                                     slot_arrays=0 if inp.read_slot is None else 2)
+                                     slot_arrays=0 if inp.read_slot is None else 2, n_q_heads=inp.n_q_heads)
     budget = max(5.0, min(60.0, 0.5 * (a.steps + a.warmup)))
     cms, cores, sample = cpu_baseline_decode(inp, min(budget, a.cpu_budget * 3))
     value = nbytes / (cms * 1e-3) / 1e9

@@ -81,15 +81,46 @@ la_status cuda_status(cudaError_t e) {
   return LA_ERR_CUDA;
 }
 
-bool uses_gate(la_rule r) { return r == LA_RULE_GATED || r == LA_RULE_GATED_DELTA; }
-bool uses_beta(la_rule r) { return r == LA_RULE_DELTA || r == LA_RULE_GATED_DELTA; }
+bool uses_gate(la_rule r) { return r == LA_RULE_GATED || r == LA_RULE_GATED_DELTA || r == LA_RULE_KDA; }
+bool uses_beta(la_rule r) { return r == LA_RULE_DELTA || r == LA_RULE_GATED_DELTA || r == LA_RULE_KDA; }
+// the gate array's alignment: kda's per-channel decays are moved in 16-byte pieces
+size_t gate_align(la_rule r) { return r == LA_RULE_KDA ? 16 : 4; }
+
+// Query-group direction: k has one head per state head (shape.n_qk_heads == n_v_heads)
+// and n_q_heads query heads are read in groups of n_q_heads / n_v_heads <= 8.
+la_status query_group(const la_shape& s, int32_t n_q_heads, int32_t* group) {
+  if (n_q_heads <= 0 || s.n_qk_heads != s.n_v_heads || n_q_heads % s.n_v_heads) return LA_ERR_SHAPE;
+  if (n_q_heads / s.n_v_heads > la::kMaxQueryGroup) return LA_ERR_UNSUPPORTED;
+  *group = n_q_heads / s.n_v_heads;
+  return LA_OK;
+}
+
+// q8 pools: d_v a multiple of the 32-column group, (d_k, d_v) one of the q8 tile shapes,
+// an even number of BF16 channels of at most d_k / 4, and a channel mask.
+bool q8_shape_ok(const la_shape& s) {
+  return (s.d_k == 64 && s.d_v == 64) || (s.d_k == 128 && s.d_v == 64) || (s.d_k == 128 && s.d_v == 128);
+}
 
 la_status check_pool(const la_pool* p) {
   if (!p || !p->data) return LA_ERR_NULL;
   if (p->n_slots < 0 || !shape_ok(p->shape)) return LA_ERR_SHAPE;
-  if (!elem_bytes(p->dtype)) return LA_ERR_UNSUPPORTED;
+  if (p->dtype == LA_Q8) {
+    if (!q8_shape_ok(p->shape)) return LA_ERR_UNSUPPORTED;
+    if (p->n_hp < 0 || p->n_hp % 2 || p->n_hp > p->shape.d_k / 4) return LA_ERR_SHAPE;
+    if (!p->hp_mask) return LA_ERR_NULL;
+    if (!aligned(p->hp_mask, 4)) return LA_ERR_ALIGN;
+  } else if (!elem_bytes(p->dtype)) {
+    return LA_ERR_UNSUPPORTED;
+  }
   if (!aligned(p->data, 16)) return LA_ERR_ALIGN;
   return LA_OK;
+}
+
+// Bytes of one slot of a (checked) pool.
+int64_t slot_bytes(const la_pool* p) {
+  const la_shape& s = p->shape;
+  if (p->dtype == LA_Q8) return (int64_t)s.n_v_heads * la::q8_tile_bytes(s.d_k, s.d_v, p->n_hp);
+  return (int64_t)s.n_v_heads * s.d_k * s.d_v * elem_bytes(p->dtype);
 }
 
 }  // namespace
@@ -106,16 +137,20 @@ int la_shape_supported(int32_t d_k, int32_t d_v) {
          (d_k == 128 && d_v == 128);
 }
 
-la_status la_state_step(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
-                        const int32_t* write_slot, int32_t B, const void* q, const void* k, const void* v,
-                        la_dtype io, const float* g, const float* beta, float scale, void* o, int32_t* err_word,
-                        void* stream) {
-  if (rule < LA_RULE_LINEAR || rule > LA_RULE_GATED_DELTA) return LA_ERR_UNSUPPORTED;
+// n_q_heads == 0: the default head direction; > 0: the query-group direction.  conv: the
+// short causal convolution ahead of the step (q, k, v are then its inputs), or NULL.
+static la_status step_impl(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
+                           const int32_t* write_slot, int32_t B, int32_t n_q_heads, const void* q, const void* k,
+                           const void* v, la_dtype io, const float* g, const float* beta, float scale, void* o,
+                           int32_t* err_word, void* stream, const la_conv* conv = nullptr) {
+  if (rule < LA_RULE_LINEAR || rule > LA_RULE_KDA) return LA_ERR_UNSUPPORTED;
   if (!err_word) return LA_ERR_NULL;
   if (B < 0) return LA_ERR_SHAPE;
   la_status st = check_pool(src);
   if (st != LA_OK) return st;
   if ((st = check_pool(dst)) != LA_OK) return st;
+  int32_t q_group = 1;
+  if (n_q_heads != 0 && (st = query_group(src->shape, n_q_heads, &q_group)) != LA_OK) return st;
   if (B == 0) return LA_OK;
   if (!q || !k || !v || !o) return LA_ERR_NULL;
   if (uses_gate(rule) && !g) return LA_ERR_NULL;
@@ -123,15 +158,35 @@ la_status la_state_step(la_rule rule, const la_pool* src, const int32_t* read_sl
   if (!same_shape(src->shape, dst->shape)) return LA_ERR_SHAPE;
   if (src->dtype != dst->dtype || !elem_bytes(io)) return LA_ERR_UNSUPPORTED;
   if (!la_shape_supported(src->shape.d_k, src->shape.d_v)) return LA_ERR_UNSUPPORTED;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, 4) ||
+  const bool q8 = src->dtype == LA_Q8;
+  if (q8 && n_q_heads != 0) return LA_ERR_UNSUPPORTED;
+  if (q8 && src->n_hp != dst->n_hp) return LA_ERR_SHAPE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, gate_align(rule)) ||
       !aligned(beta, 4) || !aligned(read_slot, 4) || !aligned(write_slot, 4) || !aligned(err_word, 4))
     return LA_ERR_ALIGN;
   if ((!read_slot && B > src->n_slots) || (!write_slot && B > dst->n_slots)) return LA_ERR_SHAPE;
   if ((int64_t)B * src->shape.n_v_heads > INT32_MAX) return LA_ERR_SHAPE;
 
   const la_shape& s = src->shape;
-  la::StepLaunchFn fn = (src->dtype == LA_F32) ? la::find_step_f32(rule, s.d_k, s.d_v, io)
-                                               : la::find_step_bf16(rule, s.d_k, s.d_v, io);
+  if (conv) {
+    if (q8) return LA_ERR_UNSUPPORTED;
+    if (conv->width < 2 || conv->width > la::kMaxConvWidth) return LA_ERR_UNSUPPORTED;
+    if (!conv->w_q || !conv->w_k || !conv->w_v || !conv->hist_src || !conv->hist_dst) return LA_ERR_NULL;
+    if (!aligned(conv->w_q, 4) || !aligned(conv->w_k, 4) || !aligned(conv->w_v, 4) || !aligned(conv->hist_src, 16) ||
+        !aligned(conv->hist_dst, 16))
+      return LA_ERR_ALIGN;
+  }
+  la::StepLaunchFn fn = nullptr;
+  if (conv)
+    fn = (src->dtype == LA_F32) ? la::find_step_conv_f32(rule, s.d_k, s.d_v, io)
+                                : la::find_step_conv_bf16(rule, s.d_k, s.d_v, io);
+  else if (q8)
+    fn = la::find_step_q8(rule, s.d_k, s.d_v, io);
+  else if (n_q_heads == 0)
+    fn = (src->dtype == LA_F32) ? la::find_step_f32(rule, s.d_k, s.d_v, io) : la::find_step_bf16(rule, s.d_k, s.d_v, io);
+  else
+    fn = (src->dtype == LA_F32) ? la::find_step_qgroups_f32(rule, s.d_k, s.d_v, io)
+                                : la::find_step_qgroups_bf16(rule, s.d_k, s.d_v, io);
   if (!fn) return LA_ERR_UNSUPPORTED;
   la::StepParams p;
   p.src = src->data;
@@ -143,6 +198,18 @@ la_status la_state_step(la_rule rule, const la_pool* src, const int32_t* read_sl
   p.B = B;
   p.n_qk_heads = s.n_qk_heads;
   p.n_v_heads = s.n_v_heads;
+  p.q_group = q_group;
+  p.n_hp = q8 ? src->n_hp : 0;
+  p.src_mask = q8 ? src->hp_mask : nullptr;
+  p.dst_mask = q8 ? dst->hp_mask : nullptr;
+  p.conv_w = conv ? conv->width : 0;
+  p.conv_act = conv ? conv->activation : 0;
+  p.conv_l2norm = conv ? conv->qk_l2norm : 0;
+  p.conv_wq = conv ? conv->w_q : nullptr;
+  p.conv_wk = conv ? conv->w_k : nullptr;
+  p.conv_wv = conv ? conv->w_v : nullptr;
+  p.conv_src = conv ? conv->hist_src : nullptr;
+  p.conv_dst = conv ? conv->hist_dst : nullptr;
   p.q = q;
   p.k = k;
   p.v = v;
@@ -154,17 +221,44 @@ la_status la_state_step(la_rule rule, const la_pool* src, const int32_t* read_sl
   return cuda_status(fn(p, static_cast<cudaStream_t>(stream)));
 }
 
+la_status la_state_step(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
+                        const int32_t* write_slot, int32_t B, const void* q, const void* k, const void* v,
+                        la_dtype io, const float* g, const float* beta, float scale, void* o, int32_t* err_word,
+                        void* stream) {
+  return step_impl(rule, src, read_slot, dst, write_slot, B, 0, q, k, v, io, g, beta, scale, o, err_word, stream);
+}
+
+la_status la_state_step_conv(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
+                             const int32_t* write_slot, int32_t B, const la_conv* conv, const void* xq,
+                             const void* xk, const void* xv, la_dtype io, const float* g, const float* beta,
+                             float scale, void* o, int32_t* err_word, void* stream) {
+  if (!conv) return LA_ERR_NULL;
+  return step_impl(rule, src, read_slot, dst, write_slot, B, 0, xq, xk, xv, io, g, beta, scale, o, err_word, stream,
+                   conv);
+}
+
+la_status la_state_step_qgroups(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
+                                const int32_t* write_slot, int32_t B, int32_t n_q_heads, const void* q, const void* k,
+                                const void* v, la_dtype io, const float* g, const float* beta, float scale, void* o,
+                                int32_t* err_word, void* stream) {
+  if (n_q_heads <= 0) return LA_ERR_SHAPE;
+  return step_impl(rule, src, read_slot, dst, write_slot, B, n_q_heads, q, k, v, io, g, beta, scale, o, err_word,
+                   stream);
+}
+
 static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
                            const int32_t* write_slot, int32_t n_seqs, const int32_t* cu_seqlens, int32_t total_tokens,
                            const int32_t* seq_order, const void* q, const void* k, const void* v, la_dtype io,
                            const float* g, const float* beta, float scale, void* o, int32_t ckpt_every,
                            const int32_t* ckpt_cu, const int32_t* ckpt_slots, int32_t* err_word, void* stream,
-                           bool chunked = false) {
-  if (rule < LA_RULE_LINEAR || rule > LA_RULE_GATED_DELTA) return LA_ERR_UNSUPPORTED;
+                           bool chunked = false, int32_t n_q_heads = 0) {
+  if (rule < LA_RULE_LINEAR || rule > LA_RULE_KDA) return LA_ERR_UNSUPPORTED;
   if (!err_word) return LA_ERR_NULL;
   if (n_seqs < 0 || total_tokens < 0) return LA_ERR_SHAPE;
   la_status st = check_pool(dst);
   if (st != LA_OK) return st;
+  int32_t q_group = 1;
+  if (n_q_heads != 0 && (st = query_group(dst->shape, n_q_heads, &q_group)) != LA_OK) return st;
   if (read_slot) {
     if ((st = check_pool(src)) != LA_OK) return st;
     if (!same_shape(src->shape, dst->shape)) return LA_ERR_SHAPE;
@@ -179,19 +273,24 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
   if (!elem_bytes(io)) return LA_ERR_UNSUPPORTED;
   const la_shape& s = dst->shape;
   if (!la_shape_supported(s.d_k, s.d_v)) return LA_ERR_UNSUPPORTED;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, 4) ||
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, gate_align(rule)) ||
       !aligned(beta, 4) || !aligned(read_slot, 4) || !aligned(write_slot, 4) || !aligned(cu_seqlens, 4) ||
       !aligned(seq_order, 4) || !aligned(err_word, 4))
     return LA_ERR_ALIGN;
   if (!write_slot && n_seqs > dst->n_slots) return LA_ERR_SHAPE;
   if ((int64_t)n_seqs * s.n_v_heads > INT32_MAX) return LA_ERR_SHAPE;
 
+  const bool q8 = dst->dtype == LA_Q8 || (read_slot && src->dtype == LA_Q8);
+  if (q8 && (chunked || n_q_heads != 0)) return LA_ERR_UNSUPPORTED;
   la::ScanLaunchFn fn = nullptr;
   if (chunked) {
     if (s.d_k != 128 || s.d_v != 128 || io != LA_BF16) return LA_ERR_UNSUPPORTED;
     fn = la::find_chunk_scan(rule);
-  } else {
+  } else if (n_q_heads == 0) {
     fn = (io == LA_F32) ? la::find_scan_f32io(rule, s.d_k, s.d_v) : la::find_scan_bf16io(rule, s.d_k, s.d_v);
+  } else {
+    fn = (io == LA_F32) ? la::find_scan_qgroups_f32io(rule, s.d_k, s.d_v)
+                        : la::find_scan_qgroups_bf16io(rule, s.d_k, s.d_v);
   }
   if (!fn) return LA_ERR_UNSUPPORTED;
   la::ScanParams p;
@@ -209,6 +308,11 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
   p.seq_order = seq_order;
   p.n_qk_heads = s.n_qk_heads;
   p.n_v_heads = s.n_v_heads;
+  p.q_group = q_group;
+  p.src_n_hp = read_slot && src->dtype == LA_Q8 ? src->n_hp : 0;
+  p.src_mask = read_slot && src->dtype == LA_Q8 ? src->hp_mask : nullptr;
+  p.dst_n_hp = dst->dtype == LA_Q8 ? dst->n_hp : 0;
+  p.dst_mask = dst->dtype == LA_Q8 ? dst->hp_mask : nullptr;
   p.q = q;
   p.k = k;
   p.v = v;
@@ -253,6 +357,16 @@ la_status la_state_scan_checkpointed(la_rule rule, const la_pool* src, const int
                    g, beta, scale, o, ckpt_every, ckpt_cu, ckpt_slots, err_word, stream);
 }
 
+la_status la_state_scan_qgroups(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
+                                const int32_t* write_slot, int32_t n_seqs, const int32_t* cu_seqlens,
+                                int32_t total_tokens, const int32_t* seq_order, int32_t n_q_heads, const void* q,
+                                const void* k, const void* v, la_dtype io, const float* g, const float* beta,
+                                float scale, void* o, int32_t* err_word, void* stream) {
+  if (n_q_heads <= 0) return LA_ERR_SHAPE;
+  return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, q, k, v, io,
+                   g, beta, scale, o, 0, nullptr, nullptr, err_word, stream, false, n_q_heads);
+}
+
 static la_status pool_op(const la_pool* pool, int32_t n, const int32_t* src_slots, const int32_t* dst_slots,
                          const void* src_dense, void* dst_dense, int zero, int32_t* err_word, void* stream) {
   if (!err_word) return LA_ERR_NULL;
@@ -264,7 +378,7 @@ static la_status pool_op(const la_pool* pool, int32_t n, const int32_t* src_slot
       !aligned(dst_dense, 16))
     return LA_ERR_ALIGN;
   la::PoolCopyParams p;
-  p.slot_bytes = (int64_t)la_state_bytes(&pool->shape, static_cast<la_dtype>(pool->dtype));
+  p.slot_bytes = slot_bytes(pool);
   p.n = n;
   p.zero = zero;
   p.err = err_word;
@@ -314,6 +428,47 @@ la_status la_state_pool_scatter(const la_pool* pool, int32_t n, const int32_t* s
 la_status la_state_pool_zero(const la_pool* pool, int32_t n, const int32_t* slots, int32_t* err_word, void* stream) {
   if (n > 0 && !slots) return LA_ERR_NULL;
   return pool_op(pool, n, nullptr, slots, nullptr, nullptr, 1, err_word, stream);
+}
+
+static la_status q8_codec(const la_pool* pool, int32_t n, const int32_t* slots, float* dense, int encode,
+                          int32_t* err_word, void* stream) {
+  if (!err_word) return LA_ERR_NULL;
+  if (n < 0) return LA_ERR_SHAPE;
+  la_status st = check_pool(pool);
+  if (st != LA_OK) return st;
+  if (pool->dtype != LA_Q8) return LA_ERR_UNSUPPORTED;
+  if (n == 0) return LA_OK;
+  if (!slots || !dense) return LA_ERR_NULL;
+  if (!aligned(slots, 4) || !aligned(dense, 16) || !aligned(err_word, 4)) return LA_ERR_ALIGN;
+  la::Q8CodecParams p;
+  p.pool = pool->data;
+  p.n_slots = pool->n_slots;
+  p.n_v_heads = pool->shape.n_v_heads;
+  p.d_k = pool->shape.d_k;
+  p.d_v = pool->shape.d_v;
+  p.n_hp = pool->n_hp;
+  p.mask = pool->hp_mask;
+  p.slots = slots;
+  p.n = n;
+  p.dense = dense;
+  p.encode = encode;
+  p.err = err_word;
+  return cuda_status(la::launch_q8_codec(p, static_cast<cudaStream_t>(stream)));
+}
+
+la_status la_state_pool_encode(const la_pool* pool, int32_t n, const int32_t* slots, const float* dense,
+                               int32_t* err_word, void* stream) {
+  return q8_codec(pool, n, slots, const_cast<float*>(dense), 1, err_word, stream);
+}
+
+la_status la_state_pool_decode(const la_pool* pool, int32_t n, const int32_t* slots, float* dense, int32_t* err_word,
+                               void* stream) {
+  return q8_codec(pool, n, slots, dense, 0, err_word, stream);
+}
+
+size_t la_pool_slot_bytes(const la_pool* pool) {
+  if (check_pool(pool) != LA_OK) return 0;
+  return (size_t)slot_bytes(pool);
 }
 
 la_status la_state_check_slots(int32_t B, const int32_t* read_slot_host, const int32_t* write_slot_host,

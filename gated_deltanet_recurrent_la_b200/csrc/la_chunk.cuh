@@ -39,23 +39,26 @@ constexpr int kThreads = kWarps * 32;
 // shared-memory layout (bytes)
 constexpr int kRow128 = kD * 2;                 // one BF16 row of 128
 constexpr int kRow64 = kC * 2;                  // one BF16 row of 64
-constexpr int kOffK = 0;                        // [64][128] bf16, swizzled
-constexpr int kOffQ = kOffK + kC * kRow128;
-constexpr int kOffV = kOffQ + kC * kRow128;
-constexpr int kOffS = kOffV + kC * kRow128;     // [128][128] bf16 state copy, swizzled
-constexpr int kOffL = kOffS + kD * kRow128;     // [64][64] fp32 (L, then reused for W)
-constexpr int kOffT = kOffL + kC * kC * 4;      // [64][64] fp32
+constexpr int kLs = kC + 4;                     // padded row stride of the FP32 L matrix
+constexpr int kInBytes = 3 * kC * kRow128;      // K, Q, V of one chunk
+constexpr int kOffIn = 0;                       // 2 x {K, Q, V} [64][128] bf16, swizzled
+constexpr int kOffS = kOffIn + 2 * kInBytes;    // [128][128] bf16 state copy, swizzled
+constexpr int kTs = kC + 8;                     // padded row stride of the FP32 T matrix
+constexpr int kXs = 24;                         // padded row stride of a 16 x 16 FP32 scratch block
+constexpr int kOffL = kOffS + kD * kRow128;     // [64][68] fp32 (L, then reused for W)
+constexpr int kOffT = kOffL + kC * kLs * 4;     // [64][72] fp32
 constexpr int kOffW = kOffL;                    // [64][128] bf16, swizzled (after T is formed)
-constexpr int kOffTw = kOffT + kC * kC * 4;     // [64][64] bf16, swizzled
+constexpr int kOffTw = kOffT + kC * kTs * 4;    // [64][64] bf16, swizzled
 constexpr int kOffTu = kOffTw + kC * kRow64;
 constexpr int kOffP = kOffTu + kC * kRow64;     // [64][64] bf16, swizzled (masked Q K^T)
 constexpr int kOffU = kOffP + kC * kRow64;      // [64][128] bf16, swizzled
 constexpr int kOffUs = kOffU + kC * kRow128;    // [64][128] bf16, swizzled (rows scaled)
-constexpr int kOffX = kOffUs + kC * kRow128;    // [3][16][16] fp32 (blocked inverse)
-constexpr int kOffG = kOffX + 3 * 256 * 4;      // per token: log|gamma|, sign, beta, gamma
-constexpr int kSmem = kOffG + 4 * kC * 4;
+constexpr int kOffX = kOffUs + kC * kRow128;    // [3][16][24] fp32 (per-warp scratch of the inverse)
+constexpr int kOffG = kOffX + 3 * 16 * kXs * 4; // per token: log|gamma|, sign, b, gamma, A, B
+constexpr int kOffGin = kOffG + 6 * kC * 4;     // 2 x {g, beta} [64] fp32 (staged gates)
+constexpr int kSmem = kOffGin + 2 * 2 * kC * 4;
 static_assert(kSmem <= 227 * 1024, "shared memory");
-static_assert(kOffW + kC * kRow128 <= kOffT + kC * kC * 4, "W reuses the L / T space");
+static_assert(kOffW + kC * kRow128 <= kOffT + kC * kTs * 4, "W reuses the L / T space");
 
 // byte offset of the 16-byte chunk `ch` of row `r` in a swizzled matrix with rows of `rowb` bytes
 __device__ __forceinline__ uint32_t swz(uint32_t base, int r, int ch, int rowb) {
@@ -81,6 +84,36 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D += A (16x8 tf32, row) * B (8x8 tf32, col), FP32 accumulate; operands are FP32 bit patterns
+__device__ __forceinline__ void mma1688_tf32(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// acc[2][4] (a 16 x 16 block as two 16 x 8 tiles) += A (16 x 16 at a, row stride lda) *
+// B (16 x 16 at b, row stride ldb), FP32 row-major operands in shared memory, TF32 MMA
+__device__ __forceinline__ void mma16x16x16_tf32(float (*acc)[4], const float* a, int lda, const float* b, int ldb,
+                                                 int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int ks = 0; ks < 16; ks += 8) {
+    uint32_t af[4];
+    af[0] = __float_as_uint(a[g * lda + ks + t]);
+    af[1] = __float_as_uint(a[(g + 8) * lda + ks + t]);
+    af[2] = __float_as_uint(a[g * lda + ks + t + 4]);
+    af[3] = __float_as_uint(a[(g + 8) * lda + ks + t + 4]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const uint32_t b0 = __float_as_uint(b[(ks + t) * ldb + 8 * nt + g]);
+      const uint32_t b1 = __float_as_uint(b[(ks + t + 4) * ldb + 8 * nt + g]);
+      mma1688_tf32(acc[nt], af, b0, b1);
+    }
+  }
 }
 
 // A fragment (rows m0..m0+15, k0..k0+15) of a row-major [m][k] matrix
@@ -121,6 +154,8 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
   float* sSg = sLg + kC;                                 // sign gamma_t
   float* sBt = sSg + kC;                                 // b_t
   float* sGm = sBt + kC;                                 // gamma_t
+  float* sFa = sGm + kC;                                 // gamma_t / e^m  (factored ratios)
+  float* sFb = sFa + kC;                                 // e^m / gamma_s
 
   constexpr bool kGate = Rule<RULE>::kUsesGate;
   constexpr bool kDelta = Rule<RULE>::kPredicts;
@@ -143,6 +178,17 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
   const int srow0 = 16 * warp;
   // this warp's block of U~ / U / O: token rows [16 mt, 16 mt + 16), columns [64 nh, 64 nh + 64)
   const int mt = warp & 3, nh = warp >> 2;
+
+  // the strictly upper 16 x 16 blocks of Tw and Tu are zero in every chunk
+  for (int idx = tid; idx < kC * kC / 2; idx += kThreads) {
+    const int r = idx >> 5, c = 2 * (idx & 31);
+    if ((c >> 4) > (r >> 4)) {
+      const uint32_t off = swz(kOffTw, r, c >> 3, kRow64) + 2 * (c & 7);
+      st_bf16x2(smem, off, 0.0f, 0.0f);
+      st_bf16x2(smem, off - kOffTw + kOffTu, 0.0f, 0.0f);
+    }
+  }
+  __syncthreads();
 
 #pragma unroll 1
   for (int64_t round = 0; round * G < units; ++round) {
@@ -191,72 +237,114 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
     }
 
     const int n_tok = t1 - t0;
+    const int n_chunks = (n_tok + kC - 1) / kC;
+    int* sFlag = reinterpret_cast<int*>(sX);  // [0]: 1 when this chunk uses factored gate ratios
+
+    // Stages chunk ci (K, Q, V rows and the gates) into input buffer ci & 1 with cp.async;
+    // rows beyond the sequence are zero and their gates are (1, 0).  Warp 0 stages the gates.
+    auto stage = [&](int ci) {
+      const int cc0 = ci * kC;
+      const int nn = (n_tok - cc0) < kC ? (n_tok - cc0) : kC;
+      unsigned char* in = smem + kOffIn + (ci & 1) * kInBytes;
+      for (int idx = tid; idx < kC * 16; idx += kThreads) {
+        const int r = idx >> 4, ch = idx & 15;
+        const uint32_t so = (uint32_t)(r * kRow128 + ((ch ^ (r & 7)) << 4));
+        if (r < nn) {
+          const int64_t tok = t0 + cc0 + r;
+          cp_async_16(in + so, kg + (tok * p.n_qk_heads + hq) * kD + ch * 8);
+          cp_async_16(in + kC * kRow128 + so, qg + (tok * p.n_qk_heads + hq) * kD + ch * 8);
+          cp_async_16(in + 2 * kC * kRow128 + so, vg + (tok * H + h) * kD + ch * 8);
+        } else {
+          *reinterpret_cast<uint4*>(in + so) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(in + kC * kRow128 + so) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(in + 2 * kC * kRow128 + so) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      if (warp == 0) {
+        float* gin = reinterpret_cast<float*>(smem + kOffGin) + (ci & 1) * 2 * kC;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 2 * lane + e;
+          if (t < nn) {
+            const int64_t gi = (int64_t)(t0 + cc0 + t) * H + h;
+            if (kGate) cp_async_4(gin + t, p.g + gi); else gin[t] = 1.0f;
+            if (Rule<RULE>::kUsesBeta) cp_async_4(gin + kC + t, p.beta + gi); else gin[kC + t] = 1.0f;
+          } else {
+            gin[t] = 1.0f;
+            gin[kC + t] = 0.0f;
+          }
+        }
+      }
+      cp_async_commit();
+    };
+
+    if (n_chunks > 0) stage(0);
 #pragma unroll 1
-    for (int c0 = 0; c0 < n_tok; c0 += kC) {
+    for (int ci = 0; ci < n_chunks; ++ci) {
+      const int c0 = ci * kC;
       const int n = (n_tok - c0) < kC ? (n_tok - c0) : kC;
+      const int kOffK = kOffIn + (ci & 1) * kInBytes;
+      const int kOffQ = kOffK + kC * kRow128;
+      const int kOffV = kOffQ + kC * kRow128;
       // ---- state copy (BF16) for this chunk's products
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         st_bf16x2(smem, swz(kOffS, srow0 + g8, j, kRow128) + 4 * t4, st[j][0], st[j][1]);
         st_bf16x2(smem, swz(kOffS, srow0 + g8 + 8, j, kRow128) + 4 * t4, st[j][2], st[j][3]);
       }
-      // ---- stage K, Q, V of the chunk (rows beyond n are zero)
-      for (int idx = tid; idx < kC * 16; idx += kThreads) {
-        const int r = idx >> 4, ch = idx & 15;
-        const uint32_t so = (uint32_t)(r * kRow128 + ((ch ^ (r & 7)) << 4));
-        if (r < n) {
-          const int64_t tok = t0 + c0 + r;
-          cp_async_16(smem + kOffK + so, kg + (tok * p.n_qk_heads + hq) * kD + ch * 8);
-          cp_async_16(smem + kOffQ + so, qg + (tok * p.n_qk_heads + hq) * kD + ch * 8);
-          cp_async_16(smem + kOffV + so, vg + (tok * H + h) * kD + ch * 8);
-        } else {
-          *reinterpret_cast<uint4*>(smem + kOffK + so) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(smem + kOffQ + so) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(smem + kOffV + so) = make_uint4(0, 0, 0, 0);
-        }
+      // ---- prefetch the next chunk, wait for this one
+      if (ci + 1 < n_chunks) {
+        stage(ci + 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
       }
-      cp_async_commit();
-      // ---- gates: log |gamma_t|, sign gamma_t (prefix over the chunk), b_t
+      // ---- gates: log |gamma_t|, sign gamma_t (prefix over the chunk), b_t, and the
+      //      factored ratios gamma_t / gamma_s = A_t B_s around the chunk's middle
       if (warp == 0) {
+        const float* gin = reinterpret_cast<const float*>(smem + kOffGin) + (ci & 1) * 2 * kC;
         float lg[2], sg[2];
+        bool big = false;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int t = 2 * lane + e;
-          float gt = 1.0f, bt = 1.0f;
-          if (t < n) {
-            const int64_t gi = (int64_t)(t0 + c0 + t) * H + h;
-            if (kGate) gt = __ldg(p.g + gi);
-            if (Rule<RULE>::kUsesBeta) bt = __ldg(p.beta + gi);
-          } else {
-            bt = 0.0f;
-          }
           float a, bc, cc;
-          Rule<RULE>::coeffs(gt, bt, a, bc, cc);
+          Rule<RULE>::coeffs(gin[t], gin[kC + t], a, bc, cc);
+          big |= fabsf(a) > 1.0f;
           lg[e] = __logf(fmaxf(fabsf(a), 1e-30f));
           sg[e] = a < 0.0f ? -1.0f : 1.0f;
           sBt[t] = bc;
         }
         // inclusive prefix (sum of logs, product of signs) over 64 tokens, 2 per lane
-        float l = lg[0] + lg[1], s = sg[0] * sg[1];
+        float l = lg[0] + lg[1], sgn = sg[0] * sg[1];
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
           const float lo = __shfl_up_sync(0xffffffffu, l, off);
-          const float so2 = __shfl_up_sync(0xffffffffu, s, off);
+          const float so2 = __shfl_up_sync(0xffffffffu, sgn, off);
           if (lane >= off) {
             l += lo;
-            s *= so2;
+            sgn *= so2;
           }
         }
-        const float lprev = l - (lg[0] + lg[1]), sprev = s * sg[0] * sg[1];  // exclusive (signs are +-1)
-        sLg[2 * lane] = lprev + lg[0];
-        sSg[2 * lane] = sprev * sg[0];
+        const float lprev = l - (lg[0] + lg[1]), sprev = sgn * sg[0] * sg[1];  // exclusive (signs are +-1)
+        const float l0 = lprev + lg[0], s0 = sprev * sg[0];
+        sLg[2 * lane] = l0;
+        sSg[2 * lane] = s0;
         sLg[2 * lane + 1] = l;
-        sSg[2 * lane + 1] = s;
-        sGm[2 * lane] = sprev * sg[0] * __expf(lprev + lg[0]);
-        sGm[2 * lane + 1] = s * __expf(l);
+        sSg[2 * lane + 1] = sgn;
+        sGm[2 * lane] = s0 * __expf(l0);
+        sGm[2 * lane + 1] = sgn * __expf(l);
+        const float lfirst = __shfl_sync(0xffffffffu, l0, 0), llast = __shfl_sync(0xffffffffu, l, 31);
+        const bool fact = !__any_sync(0xffffffffu, big) && (lfirst - llast) <= 80.0f;
+        const float m = 0.5f * (lfirst + llast);
+        sFa[2 * lane] = s0 * __expf(l0 - m);
+        sFb[2 * lane] = s0 * __expf(m - l0);
+        sFa[2 * lane + 1] = sgn * __expf(l - m);
+        sFb[2 * lane + 1] = sgn * __expf(m - l);
+        if (lane == 0) sFlag[0] = fact ? 1 : 0;
       }
-      cp_async_wait<0>();
       __syncthreads();
+      const bool fact = sFlag[0] != 0;
 
       // ---- step 1: K K^T (warps 0-3, delta rules) and Q K^T (warps 4-7), rows [16 mt, +16)
       if (kDelta || warp >= 4) {
@@ -287,73 +375,120 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
               const int s = 8 * j + 2 * t4 + f;
               v2[f] = 0.0f;
               if (s <= r) {  // gamma_r / gamma_s, only where it is used
-                const float ratio = sSg[r] * sSg[s] * __expf(sLg[r] - sLg[s]);
+                const float ratio = fact ? sFa[r] * sFb[s] : sSg[r] * sSg[s] * __expf(sLg[r] - sLg[s]);
                 if (warp < 4) {
                   if (s < r) v2[f] = sBt[r] * ratio * acc[j][e + f];
                 } else {
                   v2[f] = ratio * acc[j][e + f];
                 }
               }
-              if (warp < 4) sL[r * kC + s] = v2[f];
+              if (warp < 4) sL[r * kLs + s] = v2[f];
             }
             if (warp >= 4) st_bf16x2(smem, swz(kOffP, r, j, kRow64) + 4 * t4, v2[0], v2[1]);
+          }
+        }
+        // diagonal 16 x 16 block `warp` of T = (I + L)^-1, from this warp's own rows of L
+        // (overlapping the Q K^T of warps 4-7), in two levels of 8: lanes 0-7 / 8-15 solve
+        // the upper-left / lower-right 8 x 8 blocks by forward substitution (one column per
+        // lane), then lanes 0-7 form the lower-left block T21 = -T22 (L21 T11).  Tw =
+        // T diag(b gamma) and Tu = T diag(b) follow in BF16.
+        if (kDelta && warp < 4) {
+          __syncwarp();
+          const int b0 = 16 * warp;
+          const int c8 = lane & 7, o = b0 + 8 * ((lane >> 3) & 1);
+          float col[8];
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            float x = (r == c8) ? 1.0f : 0.0f;
+#pragma unroll
+            for (int j = 0; j < r; ++j) x -= sL[(o + r) * kLs + o + j] * col[j];
+            col[r] = (r < c8) ? 0.0f : x;
+          }
+          if (lane < 16) {
+#pragma unroll
+            for (int r = 0; r < 8; ++r) sT[(o + r) * kTs + o + c8] = col[r];
+          }
+          if (lane >= 8 && lane < 16) {
+#pragma unroll
+            for (int r = 0; r < 8; ++r) sT[(b0 + r) * kTs + b0 + 8 + c8] = 0.0f;
+          }
+          __syncwarp();
+          if (lane < 8) {
+            float xv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float a = 0.0f;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) a = fmaf(sL[(b0 + 8 + i) * kLs + b0 + k], col[k], a);
+              xv[i] = a;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float a = 0.0f;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) a = fmaf(sT[(b0 + 8 + i) * kTs + b0 + 8 + k], xv[k], a);
+              sT[(b0 + 8 + i) * kTs + b0 + c8] = -a;
+            }
+          }
+          __syncwarp();
+          const int c = lane & 15, sc = b0 + c;
+          const float fw = sBt[sc] * sGm[sc], fu = sBt[sc];
+#pragma unroll
+          for (int r = 0; r < 16; ++r) {
+            const float tv = sT[(b0 + r) * kTs + sc];
+            // pairs of columns (c, c + 1) into Tw / Tu
+            const float nw = __shfl_down_sync(0xffffffffu, tv * fw, 1);
+            const float nu = __shfl_down_sync(0xffffffffu, tv * fu, 1);
+            if (lane < 16 && (c & 1) == 0) {
+              const uint32_t off = swz(kOffTw, b0 + r, sc >> 3, kRow64) + 2 * (sc & 7);
+              st_bf16x2(smem, off, tv * fw, nw);
+              st_bf16x2(smem, off - kOffTw + kOffTu, tv * fu, nu);
+            }
           }
         }
       }
       __syncthreads();
 
-      // ---- step 2 (delta rules): T = (I + L)^-1 by 16 x 16 blocks, then Tw, Tu
+      // ---- step 2 (delta rules): the off-diagonal 16 x 16 blocks of T = (I + L)^-1 (the
+      //      diagonal ones came with step 1), written as FP32 (for the block recursion) and
+      //      as Tw = T diag(b gamma), Tu = T diag(b) (BF16, swizzled)
       if (kDelta) {
-        if (warp < 4 && lane < 16) {
-          const int b0 = 16 * warp, c = lane;
-          float col[16];
-#pragma unroll
-          for (int r = 0; r < 16; ++r) {
-            float x = (r == c) ? 1.0f : 0.0f;
-#pragma unroll
-            for (int j = 0; j < r; ++j) x -= sL[(b0 + r) * kC + b0 + j] * col[j];
-            col[r] = (r < c) ? 0.0f : x;
-          }
-#pragma unroll
-          for (int r = 0; r < 16; ++r) sT[(b0 + r) * kC + b0 + c] = col[r];
-        }
-        // zero the strictly upper blocks of T
-        for (int idx = tid; idx < kC * kC; idx += kThreads) {
-          const int r = idx >> 6, c = idx & 63;
-          if ((c >> 4) > (r >> 4)) sT[idx] = 0.0f;
-        }
-        __syncthreads();
+        // block row bi: T_{bi,j} = -T_{bi,bi} sum_{k=j}^{bi-1} L_{bi,k} T_{k,j}, warp j < bi
 #pragma unroll 1
         for (int bi = 1; bi < 4; ++bi) {
-          // X_ij = sum_{k=j}^{bi-1} L_ik T_kj  for j < bi
-          for (int idx = tid; idx < bi * 256; idx += kThreads) {
-            const int bj = idx >> 8, r = (idx >> 4) & 15, c = idx & 15;
-            float x = 0.0f;
+          if (warp < bi) {
+            const int bj = warp;
+            const int g = lane >> 2, t = lane & 3;
+            float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
             for (int bk = bj; bk < bi; ++bk)
+              mma16x16x16_tf32(x, sL + (16 * bi) * kLs + 16 * bk, kLs, sT + (16 * bk) * kTs + 16 * bj, kTs, lane);
+            float* xs = sX + warp * 16 * kXs;
 #pragma unroll
-              for (int m = 0; m < 16; ++m) x += sL[(16 * bi + r) * kC + 16 * bk + m] * sT[(16 * bk + m) * kC + 16 * bj + c];
-            sX[idx] = x;
-          }
-          __syncthreads();
-          // T_ij = -T_ii X_ij
-          for (int idx = tid; idx < bi * 256; idx += kThreads) {
-            const int bj = idx >> 8, r = (idx >> 4) & 15, c = idx & 15;
-            float x = 0.0f;
+            for (int nt = 0; nt < 2; ++nt) {
+              xs[g * kXs + 8 * nt + 2 * t] = x[nt][0];
+              xs[g * kXs + 8 * nt + 2 * t + 1] = x[nt][1];
+              xs[(g + 8) * kXs + 8 * nt + 2 * t] = x[nt][2];
+              xs[(g + 8) * kXs + 8 * nt + 2 * t + 1] = x[nt][3];
+            }
+            __syncwarp();
+            float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            mma16x16x16_tf32(y, sT + (16 * bi) * kTs + 16 * bi, kTs, xs, kXs, lane);
 #pragma unroll
-            for (int m = 0; m < 16; ++m) x += sT[(16 * bi + r) * kC + 16 * bi + m] * sX[(bj << 8) + m * 16 + c];
-            sT[(16 * bi + r) * kC + 16 * bj + c] = -x;
+            for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+              for (int hlf = 0; hlf < 2; ++hlf) {
+                const int r = 16 * bi + g + 8 * hlf, c = 16 * bj + 8 * nt + 2 * t;
+                const float v0 = -y[nt][2 * hlf], v1 = -y[nt][2 * hlf + 1];
+                sT[r * kTs + c] = v0;
+                sT[r * kTs + c + 1] = v1;
+                const uint32_t off = swz(kOffTw, r, c >> 3, kRow64) + 2 * (c & 7);
+                st_bf16x2(smem, off, v0 * sBt[c] * sGm[c], v1 * sBt[c + 1] * sGm[c + 1]);
+                st_bf16x2(smem, off - kOffTw + kOffTu, v0 * sBt[c], v1 * sBt[c + 1]);
+              }
+            }
           }
           __syncthreads();
         }
-        // Tw = T diag(b gamma), Tu = T diag(b)   (BF16, swizzled)
-        for (int idx = tid; idx < kC * kC / 2; idx += kThreads) {
-          const int r = idx >> 5, s = 2 * (idx & 31);
-          const float t0v = sT[r * kC + s], t1v = sT[r * kC + s + 1];
-          const uint32_t off = swz(kOffTw, r, s >> 3, kRow64) + 2 * (s & 7);
-          st_bf16x2(smem, off, t0v * sBt[s] * sGm[s], t1v * sBt[s + 1] * sGm[s + 1]);
-          st_bf16x2(smem, off - kOffTw + kOffTu, t0v * sBt[s], t1v * sBt[s + 1]);
-        }
-        __syncthreads();
       }
 
       // ---- step 3: this warp's U~ block (rows 16 mt, cols 64 nh) and -W block (K columns 64 nh)

@@ -217,6 +217,75 @@ struct StateVec<__nv_bfloat16> {
   }
 };
 
+// ---- mixed INT8 / BF16 state storage (LA_Q8) ----------------------------------------
+// Tile of d_k x d_v: INT8 codes [d_k - n_hp][d_v], FP32 scales [d_k - n_hp][d_v / 32],
+// BF16 rows [n_hp][d_v]; the rows whose bit is set in the head's mask (d_k / 32 words)
+// are the BF16 ones, each block in increasing row order.  A group of 32 columns of an
+// INT8 row with absmax a > 0 has scale s = a * fl(1/127) and inverse scale
+// inv = fl(1/a) * 127 (correctly rounded FP32 reciprocal and products); its codes are
+// rint(x * inv) clamped to +-127 (NaN -> 0), decoded as code * s; an all-zero group has
+// s = inv = 0.
+struct q8_t {};
+
+// Rows row0 .. row0 + n - 1 of a head (n <= 32, inside one 32-row word of the mask): each
+// row is BF16 (rank among the BF16 rows) or INT8 (rank among the INT8 rows).
+template <int DK>
+struct Q8Rows {
+  uint32_t word;  // the mask word holding the rows
+  int below;      // BF16 rows before that word
+  int row0;
+
+  __device__ __forceinline__ void init(const uint32_t* head_mask, int first_row) {
+    row0 = first_row;
+    below = 0;
+    word = 0u;
+#pragma unroll
+    for (int w = 0; w < DK / 32; ++w) {
+      const uint32_t m = __ldg(head_mask + w);
+      if (w < first_row / 32) below += __popc(m);
+      if (w == first_row / 32) word = m;
+    }
+  }
+  // row row0 + r: returns true for a BF16 row; idx = its rank in its block
+  __device__ __forceinline__ bool row(int r, int& idx) const {
+    const int i = row0 + r, b = i & 31;
+    const int pre = below + __popc(word & ((1u << b) - 1u));
+    const bool hp = (word >> b) & 1u;
+    idx = hp ? pre : i - pre;
+    return hp;
+  }
+};
+
+// scale and inverse scale of a group with absmax `amax` (both 0 for an all-zero group)
+__device__ __forceinline__ void q8_scales(float amax, float& s, float& inv) {
+  const bool nz = amax > 0.0f;
+  s = nz ? __fmul_rn(amax, 1.0f / 127.0f) : 0.0f;
+  inv = nz ? __fmul_rn(__frcp_rn(amax), 127.0f) : 0.0f;
+}
+
+__device__ __forceinline__ uint32_t q8_code(float x, float inv) {
+  const int c = __float2int_rn(__fmul_rn(x, inv));  // NaN -> 0
+  return (uint32_t)max(-127, min(127, c)) & 0xffu;
+}
+
+// N (4 or 8) consecutive values <-> codes packed little-endian into N bytes
+template <int N>
+__device__ __forceinline__ void q8_pack(const float* x, float inv, uint32_t* words) {
+#pragma unroll
+  for (int w = 0; w < N / 4; ++w)
+    words[w] = q8_code(x[4 * w], inv) | (q8_code(x[4 * w + 1], inv) << 8) | (q8_code(x[4 * w + 2], inv) << 16) |
+               (q8_code(x[4 * w + 3], inv) << 24);
+}
+
+template <int N>
+__device__ __forceinline__ void q8_unpack(const uint32_t* words, float s, float* x) {
+#pragma unroll
+  for (int w = 0; w < N / 4; ++w)
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      x[4 * w + b] = __fmul_rn((float)(int)(int8_t)((words[w] >> (8 * b)) & 0xffu), s);
+}
+
 // N consecutive io-type values -> FP32, with the widest aligned vector loads the byte
 // count allows (16 or 8 bytes; scalar otherwise).  `p` must be aligned to that width.
 template <typename IT, int N>
@@ -298,15 +367,20 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
 }
 
 // Coefficients (a, b, c) of a rule: S <- a S + k u^T, u = b (v - c S^T k).
+// kda (channel-wise gate): the decay is a per-row vector alpha applied to S before the
+// prediction, S <- Diag(alpha) S + k u^T with u = beta (v - (Diag(alpha) S)^T k); the
+// kernels fold alpha into the keys of the reductions, so its scalar coefficients are
+// a = 1 (the readout's S^T q already carries alpha), b = beta, c = 1.
 template <int RULE>
 struct Rule {
   static constexpr bool kUsesGate = (RULE == LA_RULE_GATED || RULE == LA_RULE_GATED_DELTA);
-  static constexpr bool kUsesBeta = (RULE == LA_RULE_DELTA || RULE == LA_RULE_GATED_DELTA);
+  static constexpr bool kChannelGate = (RULE == LA_RULE_KDA);
+  static constexpr bool kUsesBeta = (RULE == LA_RULE_DELTA || RULE == LA_RULE_GATED_DELTA || RULE == LA_RULE_KDA);
   static constexpr bool kPredicts = kUsesBeta;  // needs S^T k
   static __device__ __forceinline__ void coeffs(float g, float beta, float& a, float& b, float& c) {
     a = kUsesGate ? g : 1.0f;
     b = kUsesBeta ? beta : 1.0f;
-    c = (RULE == LA_RULE_DELTA) ? 1.0f : (RULE == LA_RULE_GATED_DELTA ? g : 0.0f);
+    c = (RULE == LA_RULE_DELTA || RULE == LA_RULE_KDA) ? 1.0f : (RULE == LA_RULE_GATED_DELTA ? g : 0.0f);
   }
 };
 

@@ -9,6 +9,12 @@
 
 namespace la {
 
+// Bytes of one (slot, head) tile of the mixed INT8 / BF16 (q8) storage: INT8 codes and
+// FP32 scales (one per 32 columns) of the d_k - n_hp INT8 rows, then n_hp BF16 rows.
+__host__ __device__ constexpr int64_t q8_tile_bytes(int dk, int dv, int n_hp) {
+  return (int64_t)(dk - n_hp) * dv + (int64_t)(dk - n_hp) * (dv / 32) * 4 + (int64_t)n_hp * dv * 2;
+}
+
 struct StepParams {
   const void* src;          // source pool data
   int32_t src_slots;
@@ -19,6 +25,19 @@ struct StepParams {
   int32_t B;
   int32_t n_qk_heads;
   int32_t n_v_heads;
+  int32_t q_group;          // queries per state head: 1, or up to 8 in the query-group direction
+  int32_t n_hp;             // q8 pools: BF16 key channels per head (same for source and destination)
+  const uint32_t* src_mask; // q8 pools: [H_v][d_k / 32] channel masks
+  const uint32_t* dst_mask;
+  // the short causal convolution ahead of the step (conv_w == 0: none)
+  int32_t conv_w;
+  int32_t conv_act;         // 1: SiLU
+  int32_t conv_l2norm;      // 1: q and k to unit length
+  const float* conv_wq;     // [H_qk][d_k][W]
+  const float* conv_wk;
+  const float* conv_wv;     // [H_v][d_v][W]
+  const void* conv_src;     // io dtype [src slots][H_v][2 d_k + d_v][W - 1]
+  void* conv_dst;
   const void* q;
   const void* k;
   const void* v;
@@ -44,6 +63,11 @@ struct ScanParams {
   const int32_t* seq_order;  // [n_seqs] or nullptr
   int32_t n_qk_heads;
   int32_t n_v_heads;
+  int32_t q_group;           // queries per state head: 1, or up to 8 in the query-group direction
+  int32_t src_n_hp;          // q8 pools: BF16 key channels per head and the channel masks
+  const uint32_t* src_mask;
+  int32_t dst_n_hp;
+  const uint32_t* dst_mask;
   const void* q;
   const void* k;
   const void* v;
@@ -80,10 +104,39 @@ StepLaunchFn find_step_bf16(int rule, int dk, int dv, int io);
 ScanLaunchFn find_scan_f32io(int rule, int dk, int dv);
 ScanLaunchFn find_scan_bf16io(int rule, int dk, int dv);
 
+// Decode step with the short causal convolution fused ahead (widths 2 .. kMaxConvWidth).
+constexpr int kMaxConvWidth = 4;
+StepLaunchFn find_step_conv_f32(int rule, int dk, int dv, int io);
+StepLaunchFn find_step_conv_bf16(int rule, int dk, int dv, int io);
+
+// The same in the query-group direction (k per state head, q_group <= kMaxQueryGroup
+// query heads reading each state head).
+constexpr int kMaxQueryGroup = 8;
+// q8 state storage (d_v a multiple of 32): (64,64), (128,64), (128,128)
+StepLaunchFn find_step_q8(int rule, int dk, int dv, int io);
+StepLaunchFn find_step_qgroups_f32(int rule, int dk, int dv, int io);
+StepLaunchFn find_step_qgroups_bf16(int rule, int dk, int dv, int io);
+ScanLaunchFn find_scan_qgroups_f32io(int rule, int dk, int dv);
+ScanLaunchFn find_scan_qgroups_bf16io(int rule, int dk, int dv);
+
 // Chunked tensor-core prefill (d_k = d_v = 128, BF16 io); nullptr for an unknown rule.
 ScanLaunchFn find_chunk_scan(int rule);
 
 cudaError_t launch_pool_copy(const PoolCopyParams& p, cudaStream_t stream);
+
+// FP32 dense tiles <-> q8 slots of a pool (n slots x H_v heads).
+struct Q8CodecParams {
+  void* pool;                // q8 pool data
+  int32_t n_slots;
+  int32_t n_v_heads, d_k, d_v, n_hp;
+  const uint32_t* mask;      // [H_v][d_k / 32]
+  const int32_t* slots;      // [n]
+  int32_t n;
+  float* dense;              // [n, H_v, d_k, d_v]
+  int32_t encode;            // 1: dense -> pool, 0: pool -> dense
+  int32_t* err;
+};
+cudaError_t launch_q8_codec(const Q8CodecParams& p, cudaStream_t stream);
 
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();

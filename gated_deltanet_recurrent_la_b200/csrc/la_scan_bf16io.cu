@@ -3,5 +3,5 @@
 #include "la_scan.cuh"
 
 namespace la {
-ScanLaunchFn find_scan_bf16io(int rule, int dk, int dv) { return find_scan_impl<__nv_bfloat16>(rule, dk, dv); }
+ScanLaunchFn find_scan_bf16io(int rule, int dk, int dv) { return find_scan_impl<__nv_bfloat16, false>(rule, dk, dv); }
 }  // namespace la

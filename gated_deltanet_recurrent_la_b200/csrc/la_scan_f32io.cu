@@ -3,5 +3,5 @@
 #include "la_scan.cuh"
 
 namespace la {
-ScanLaunchFn find_scan_f32io(int rule, int dk, int dv) { return find_scan_impl<float>(rule, dk, dv); }
+ScanLaunchFn find_scan_f32io(int rule, int dk, int dv) { return find_scan_impl<float, false>(rule, dk, dv); }
 }  // namespace la

@@ -1,0 +1,7 @@
+// la_scan_qg_f32io.cu -- scan kernels in the query-group direction with f32 q/k/v/o (all rules and tile
+// shapes); see la_scan.cuh.
+#include "la_scan.cuh"
+
+namespace la {
+ScanLaunchFn find_scan_qgroups_f32io(int rule, int dk, int dv) { return find_scan_impl<float, true>(rule, dk, dv); }
+}  // namespace la

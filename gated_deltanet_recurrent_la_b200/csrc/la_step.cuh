@@ -17,7 +17,7 @@
 //  * warp specialisation: one producer warp streams each whole d_k x d_v state tile (a
 //    contiguous 8-64 KiB block of the pool) plus q, k, v into a shared-memory stage
 //    with 1-D bulk copies on the TMA engine, signalling an mbarrier -- the
-//    "asynchronous state transfers" of the "Gated DeltaNet" page (How to read it) --
+//    asynchronous movement of the state named on the "Gated DeltaNet" page (How to read it) --
 //    so that several tiles are in flight per SM at all times;
 //  * every column of S evolves on its own, so each consumer warp owns a strip of up to
 //    32 columns of a tile for all d_k rows and needs nobody else: lanes split the strip
@@ -27,10 +27,14 @@
 //    Warps of different tiles run concurrently; there is no CTA-wide barrier.  Four
 //    consumer warps (plus the producer) keep every SM sub-partition at <= 2 warps so a
 //    thread may hold its 128 state values without spilling.
-//  * FP32 arithmetic in packed pairs (sm_100 FFMA2 / FMUL2).
+//  * the channel-wise gate of Kimi Delta Attention ("Seven Architectures ...", section
+//    "Kimi Linear") keeps every column independent: the d_k decays ride in the stage
+//    with the tile and scale the keys of the two reductions and the rows of the update.
+//  * FP32 arithmetic in pairs (packed FFMA2 / FMUL2 only where it measures faster).
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 
 #include "la_device.cuh"
 #include "la_internal.h"
@@ -45,8 +49,8 @@ struct StepMeta {
   float g;
   float beta;
   int32_t valid;
-  int32_t pad;
-  int64_t dst_off;  // element offset of the destination tile in the destination pool
+  int32_t ws;       // write slot (the convolution history goes there too)
+  int64_t dst_off;  // byte offset of the destination tile in the destination pool
   int64_t o_off;    // element offset of o[b, h, 0]
 };
 
@@ -65,10 +69,15 @@ struct StepMeta {
 #define LA_STEP_PDL 1
 #endif
 
-template <int DK, int DV, typename ST, typename IT>
+// CHG: the rule carries a channel-wise gate (kda), d_k FP32 decays staged with the tile.
+// QMAX: query rows a stage holds (1, or kMaxQueryGroup in the query-group direction).
+// CONV: the short causal convolution runs ahead of the step (the stage also holds the
+// tile's convolution history, and each consumer warp a scratch of post-convolution q, k, v).
+template <int DK, int DV, typename ST, typename IT, bool CHG = false, int QMAX = 1, bool CONV = false>
 struct StepCfg {
-  static constexpr int kSB = sizeof(ST);
-  static constexpr int kVec = StateVec<ST>::kElems;     // state elements per 16-byte chunk
+  static constexpr bool kQ8 = std::is_same<ST, q8_t>::value;
+  static constexpr int kSB = kQ8 ? 2 : (int)sizeof(ST);  // (q8: the BF16 rows' lane layout)
+  static constexpr int kVec = 16 / kSB;                  // state elements per lane and row
   static constexpr int kCW = DV < LA_STEP_STRIP_COLS ? DV : LA_STEP_STRIP_COLS;  // strip width
   static constexpr int kWPT = DV / kCW;                 // warps per tile
   static constexpr int kNCH = kCW / kVec;               // 16-byte chunks per strip row
@@ -77,26 +86,108 @@ struct StepCfg {
   static constexpr int kConsumerWarps = kWPT > LA_STEP_CONSUMER_WARPS ? kWPT : LA_STEP_CONSUMER_WARPS;
   static constexpr int kTeams = kConsumerWarps / kWPT;  // tiles in compute at once
   static constexpr int kThreads = (kConsumerWarps + 1) * 32;
-  static constexpr int kTileBytes = DK * DV * kSB;
+  // stage room for one tile; q8 tiles hold at most DK / 4 BF16 rows
+  static constexpr int kTileBytes = kQ8 ? (int)q8_tile_bytes(DK, DV, DK / 4) : DK * DV * kSB;
   static constexpr int kQKBytes = DK * (int)sizeof(IT);
   static constexpr int kVBytes = DV * (int)sizeof(IT);
-  static constexpr int kCopyBytes = kTileBytes + 2 * kQKBytes + kVBytes;
+  static constexpr int kGBytes = CHG ? DK * 4 : 0;
+  // stage layout: tile | QMAX query rows | key | v | decays (kda)
+  static constexpr int kOffK = kTileBytes + QMAX * kQKBytes;
+  static constexpr int kOffV = kOffK + kQKBytes;
+  static constexpr int kOffA = kOffV + kVBytes;
+  static constexpr int kOffHist = kOffA + kGBytes;
+  static constexpr int kHistBytes = CONV ? (2 * DK + DV) * (kMaxConvWidth - 1) * (int)sizeof(IT) : 0;
+  static constexpr int kCopyBytes = kOffHist + kHistBytes;  // with all QMAX query rows, widest history
   static constexpr int kStageBytes = round_up(kCopyBytes, 128);
   static constexpr int kStages = cmax(2, cmin(12, (204 * 1024) / kStageBytes));
   static constexpr int kOffMeta = kStages * kStageBytes;
   static constexpr int kOffBars = round_up(kOffMeta + kStages * (int)sizeof(StepMeta), 8);
-  static constexpr int kSmem = kOffBars + 2 * kStages * 8;
+  static constexpr int kOffScratch = round_up(kOffBars + 2 * kStages * 8, 16);
+  static constexpr int kScratchFloats = CONV ? 2 * DK + DV : 0;  // per consumer warp: q, k, v
+  static constexpr int kSmem = kOffScratch + kConsumerWarps * kScratchFloats * 4;
 
   static_assert(kNCH >= 1 && kNCH <= 32 && (32 % kNCH) == 0, "strip row must map onto a power-of-two lane group");
   static_assert(kRL >= 1 && DK % kRG == 0, "rows must split evenly over the row blocks");
   static_assert(kConsumerWarps % kWPT == 0, "whole tiles per team");
-  static_assert(kQKBytes % 16 == 0 && kVBytes % 16 == 0 && kTileBytes % 16 == 0, "bulk copies move 16-byte units");
+  static_assert(kQKBytes % 16 == 0 && kVBytes % 16 == 0 && kTileBytes % 16 == 0 && kGBytes % 16 == 0,
+                "bulk copies move 16-byte units");
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
-template <int RULE, int DK, int DV, typename ST, typename IT>
-__global__ void __launch_bounds__(StepCfg<DK, DV, ST, IT>::kThreads, 1) step_kernel(const StepParams p) {
-  using C = StepCfg<DK, DV, ST, IT>;
+// The short causal convolution ahead of the step, for one tile, by one consumer warp: the
+// post-convolution q, k (channels of the tile's q/k head) and v (the tile's head) go to the
+// warp's FP32 scratch [q | k | v]; channel c is y = sum_j w[c][j] x_{t-W+1+j} over the W - 1
+// staged history inputs and the current input, then SiLU when asked, then q and k scaled
+// to unit length when asked.  Warp `part` of the tile writes every kWPT-th 32-channel block
+// of the new history (the last W - 1 inputs) to write slot `ws` (skipped when ws < 0).
+template <int DK, int DV, typename IT, int WPT>
+__device__ __forceinline__ void conv_operands(const StepParams& p, const unsigned char* xq_s,
+                                              const unsigned char* xk_s, const unsigned char* xv_s,
+                                              const unsigned char* hist_s, int h, int H, int ws, int part, int lane,
+                                              float* scr) {
+  constexpr int CH = 2 * DK + DV;
+  const int W = p.conv_w;
+  const int hq = h / (H / p.n_qk_heads);
+  const IT* xq = reinterpret_cast<const IT*>(xq_s);
+  const IT* xk = reinterpret_cast<const IT*>(xk_s);
+  const IT* xv = reinterpret_cast<const IT*>(xv_s);
+  const IT* hist = reinterpret_cast<const IT*>(hist_s);
+  float sq = 0.0f, sk = 0.0f;
+  // all of a lane's channels at once (unrolled, widths padded to kMaxConvWidth) so the
+  // weight and history loads are in flight together
+#pragma unroll
+  for (int it = 0; it < (CH + 31) / 32; ++it) {
+    const int c = lane + 32 * it;
+    if (c < CH) {
+      const float* w = c < DK ? p.conv_wq + ((int64_t)hq * DK + c) * W
+                     : c < 2 * DK ? p.conv_wk + ((int64_t)hq * DK + (c - DK)) * W
+                                  : p.conv_wv + ((int64_t)h * DV + (c - 2 * DK)) * W;
+      const float x = io_load(c < DK ? xq + c : c < 2 * DK ? xk + (c - DK) : xv + (c - 2 * DK));
+      float y = __ldg(w + W - 1) * x;
+#pragma unroll
+      for (int j = 0; j < kMaxConvWidth - 1; ++j)
+        if (j < W - 1) y = fmaf(__ldg(w + j), io_load(hist + c * (W - 1) + j), y);
+      if (p.conv_act) y = y / (1.0f + __expf(-y));
+      scr[c] = y;
+      if (c < DK) sq = fmaf(y, y, sq);
+      else if (c < 2 * DK) sk = fmaf(y, y, sk);
+    }
+  }
+  if (p.conv_l2norm) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      sq += __shfl_xor_sync(0xffffffffu, sq, off);
+      sk += __shfl_xor_sync(0xffffffffu, sk, off);
+    }
+    const float rq = rsqrtf(sq + 1e-6f), rk = rsqrtf(sk + 1e-6f);
+    __syncwarp();
+#pragma unroll
+    for (int it = 0; it < (2 * DK + 31) / 32; ++it) {
+      const int c = lane + 32 * it;
+      if (c < 2 * DK) scr[c] *= c < DK ? rq : rk;
+    }
+  }
+  if (ws >= 0) {
+    IT* hd = static_cast<IT*>(p.conv_dst) + ((int64_t)ws * H + h) * CH * (W - 1);
+    for (int c = part * 32 + lane; c < CH; c += WPT * 32) {
+      for (int j = 0; j < W - 2; ++j) hd[c * (W - 1) + j] = hist[c * (W - 1) + j + 1];
+      hd[c * (W - 1) + W - 2] = c < DK ? xq[c] : c < 2 * DK ? xk[c - DK] : xv[c - 2 * DK];
+    }
+  }
+  __syncwarp();
+}
+
+// QGRP: the query-group direction of the ONNX operator -- k has one head per state head
+// and p.q_group query heads (consecutive) read each state head; every extra query costs
+// one more pass over the registers, the state is still read and written once.
+template <int RULE, int DK, int DV, typename ST, typename IT, bool QGRP, bool CONV>
+__global__ void __launch_bounds__(
+    StepCfg<DK, DV, ST, IT, Rule<RULE>::kChannelGate, QGRP ? kMaxQueryGroup : 1, CONV>::kThreads, 1)
+    step_kernel(const StepParams p) {
+  constexpr bool CHG = Rule<RULE>::kChannelGate;
+  using C = StepCfg<DK, DV, ST, IT, CHG, QGRP ? kMaxQueryGroup : 1, CONV>;
+  static_assert(!(CONV && QGRP), "the convolution runs in the default head direction");
+  const int qg = QGRP ? p.q_group : 1;
   extern __shared__ __align__(128) unsigned char smem[];
   StepMeta* meta = reinterpret_cast<StepMeta*>(smem + C::kOffMeta);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
@@ -128,7 +219,8 @@ __global__ void __launch_bounds__(StepCfg<DK, DV, ST, IT>::kThreads, 1) step_ker
     // ------------------------------------------------------------------ producer
     const uint64_t pol_stream = policy_evict_first();
     const int ratio = H / p.n_qk_heads;
-    const ST* src = static_cast<const ST*>(p.src);
+    const unsigned char* src = static_cast<const unsigned char*>(p.src);
+    const int tile_bytes = C::kQ8 ? (int)q8_tile_bytes(DK, DV, p.n_hp) : C::kTileBytes;
     const IT* q = static_cast<const IT*>(p.q);
     const IT* k = static_cast<const IT*>(p.k);
     const IT* v = static_cast<const IT*>(p.v);
@@ -166,24 +258,44 @@ __global__ void __launch_bounds__(StepCfg<DK, DV, ST, IT>::kThreads, 1) step_ker
             const int hq = h / ratio;
             const bool rs_ok = rs_j >= 0 && rs_j < p.src_slots;
             const bool ws_ok = ws_j >= 0 && ws_j < p.dst_slots;
+            bool mask_ok = true;
+            if constexpr (C::kQ8) {
+              // a head's masks must mark exactly n_hp rows, or the row ranks leave the tile
+              int cs = 0, cd = 0;
+#pragma unroll
+              for (int w = 0; w < DK / 32; ++w) {
+                cs += __popc(__ldg(p.src_mask + h * (DK / 32) + w));
+                cd += __popc(__ldg(p.dst_mask + h * (DK / 32) + w));
+              }
+              mask_ok = cs == p.n_hp && cd == p.n_hp;
+              if (!mask_ok) report(p.err, LA_DEVERR_Q8_MASK);
+            }
             StepMeta m;
             m.g = g_j;
             m.beta = b_j;
-            m.valid = rs_ok && ws_ok;
-            m.pad = 0;
-            m.dst_off = ((int64_t)ws_j * H + h) * (DK * DV);
-            m.o_off = t * DV;
+            m.valid = rs_ok && ws_ok && mask_ok;
+            m.ws = ws_j;
+            m.dst_off = ((int64_t)ws_j * H + h) * tile_bytes;
+            m.o_off = t * qg * DV;  // o row of the tile's first query
             meta[stage] = m;
             if (m.valid) {
               unsigned char* sb = smem + stage * C::kStageBytes;
-              mbar_arrive_expect_tx(&full[stage], C::kCopyBytes);
-              bulk_g2s_hint(sb, src + ((int64_t)rs_j * H + h) * (DK * DV), C::kTileBytes, &full[stage], pol_stream);
-              bulk_g2s(sb + C::kTileBytes, q + ((int64_t)b * p.n_qk_heads + hq) * DK, C::kQKBytes, &full[stage]);
-              bulk_g2s(sb + C::kTileBytes + C::kQKBytes, k + ((int64_t)b * p.n_qk_heads + hq) * DK, C::kQKBytes,
-                       &full[stage]);
-              bulk_g2s(sb + C::kTileBytes + 2 * C::kQKBytes, v + t * DV, C::kVBytes, &full[stage]);
+              // query rows: the tile's q/k head, or its qg consecutive query heads
+              const int64_t qrow = QGRP ? t * qg : (int64_t)b * p.n_qk_heads + hq;
+              const int hist_bytes = CONV ? (2 * DK + DV) * (p.conv_w - 1) * (int)sizeof(IT) : 0;
+              mbar_arrive_expect_tx(&full[stage],
+                                    C::kOffHist - C::kOffK + tile_bytes + qg * C::kQKBytes + hist_bytes);
+              bulk_g2s_hint(sb, src + ((int64_t)rs_j * H + h) * tile_bytes, tile_bytes, &full[stage], pol_stream);
+              bulk_g2s(sb + C::kTileBytes, q + qrow * DK, qg * C::kQKBytes, &full[stage]);
+              bulk_g2s(sb + C::kOffK, k + ((int64_t)b * p.n_qk_heads + hq) * DK, C::kQKBytes, &full[stage]);
+              bulk_g2s(sb + C::kOffV, v + t * DV, C::kVBytes, &full[stage]);
+              if (CHG) bulk_g2s(sb + C::kOffA, p.g + t * DK, C::kGBytes, &full[stage]);
+              if (CONV)
+                bulk_g2s(sb + C::kOffHist,
+                         static_cast<const unsigned char*>(p.conv_src) + ((int64_t)rs_j * H + h) * hist_bytes,
+                         hist_bytes, &full[stage]);
             } else {
-              report(p.err, (rs_ok ? 0u : LA_DEVERR_READ_SLOT) | (ws_ok ? 0u : LA_DEVERR_WRITE_SLOT));
+              if (!rs_ok || !ws_ok) report(p.err, (rs_ok ? 0u : LA_DEVERR_READ_SLOT) | (ws_ok ? 0u : LA_DEVERR_WRITE_SLOT));
               mbar_arrive(&full[stage]);
             }
           } else {
@@ -219,8 +331,11 @@ __global__ void __launch_bounds__(StepCfg<DK, DV, ST, IT>::kThreads, 1) step_ker
   const int rb = lane / C::kNCH;              // row block
   const int col0 = part * C::kCW + ch * V;    // first column held by this lane
   const int row0 = rb * RL;                   // first row held by this lane
-  ST* dst = static_cast<ST*>(p.dst);
+  unsigned char* dst = static_cast<unsigned char*>(p.dst);
   IT* out = static_cast<IT*>(p.o);
+  // q8: INT8 rows of the source / destination tiles (BF16 rows follow the codes and scales)
+  const int n8s = DK - p.n_hp, n8d = DK - p.n_hp;
+  constexpr int NG = DV / 32;
 
   for (int64_t it = team; it < n_my; it += C::kTeams) {
     const int stage = (int)(it % C::kStages);
@@ -232,20 +347,59 @@ __global__ void __launch_bounds__(StepCfg<DK, DV, ST, IT>::kThreads, 1) step_ker
     }
     const StepMeta m = meta[stage];
     const unsigned char* sb = smem + stage * C::kStageBytes;
-    const ST* tile = reinterpret_cast<const ST*>(sb);
-    const IT* qs = reinterpret_cast<const IT*>(sb + C::kTileBytes);
-    const IT* ks = reinterpret_cast<const IT*>(sb + C::kTileBytes + C::kQKBytes);
-    const IT* vs = reinterpret_cast<const IT*>(sb + C::kTileBytes + 2 * C::kQKBytes);
+    // q, k, v of the step: the staged rows, or (CONV) this warp's post-convolution scratch
+    using OT = std::conditional_t<CONV, float, IT>;
+    const OT* qs;
+    const OT* ks;
+    const OT* vs;
+    if constexpr (CONV) {
+      float* scr = reinterpret_cast<float*>(smem + C::kOffScratch) + warp * C::kScratchFloats;
+      conv_operands<DK, DV, IT, C::kWPT>(p, sb + C::kTileBytes, sb + C::kOffK, sb + C::kOffV, sb + C::kOffHist,
+                                         (int)((blockIdx.x + it * gridDim.x) % H), H, m.valid ? m.ws : -1, part,
+                                         lane, scr);
+      qs = scr;
+      ks = scr + DK;
+      vs = scr + 2 * DK;
+    } else {
+      qs = reinterpret_cast<const IT*>(sb + C::kTileBytes);
+      ks = reinterpret_cast<const IT*>(sb + C::kOffK);
+      vs = reinterpret_cast<const IT*>(sb + C::kOffV);
+    }
+    const float* as = reinterpret_cast<const float*>(sb + C::kOffA);
     float a, bcoef, c;
     Rule<RULE>::coeffs(m.g, m.beta, a, bcoef, c);
 
     float s[RL][V];
+    Q8Rows<DK> rows_src, rows_dst;  // (q8) this lane's rows in the source / destination masks
+    if constexpr (C::kQ8) {
+      // q8 tile: this lane's rows from the INT8 codes (with their group's scale; the strip
+      // is one 32-column group) or from the BF16 rows, as the head's mask says
+      const int h = (int)((blockIdx.x + it * gridDim.x) % H);
+      rows_src.init(p.src_mask + h * (DK / 32), row0);
+      rows_dst.init(p.dst_mask + h * (DK / 32), row0);
 #pragma unroll
-    for (int r = 0; r < RL; ++r)
-      StateVec<ST>::unpack(*reinterpret_cast<const uint4*>(tile + (row0 + r) * DV + col0), s[r]);
+      for (int r = 0; r < RL; ++r) {
+        int idx;
+        if (rows_src.row(r, idx)) {
+          const uint4 w = *reinterpret_cast<const uint4*>(sb + n8s * DV + n8s * NG * 4 + (idx * DV + col0) * 2);
+          StateVec<__nv_bfloat16>::unpack(w, s[r]);
+        } else {
+          const uint2 w = *reinterpret_cast<const uint2*>(sb + idx * DV + col0);
+          const float sc = *reinterpret_cast<const float*>(sb + n8s * DV + (idx * NG + part) * 4);
+          const uint32_t ww[2] = {w.x, w.y};
+          q8_unpack<8>(ww, sc, s[r]);
+        }
+      }
+    } else {
+      const ST* tile = reinterpret_cast<const ST*>(sb);
+#pragma unroll
+      for (int r = 0; r < RL; ++r)
+        StateVec<ST>::unpack(*reinterpret_cast<const uint4*>(tile + (row0 + r) * DV + col0), s[r]);
+    }
 
     // k.q, S^T k and S^T q over this lane's rows (k, q read from the stage in blocks of
-    // up to 8 rows), then across the row blocks
+    // up to 8 rows), then across the row blocks.  kda: the rows' decays scale the keys of
+    // both sums, (Diag(alpha) S)^T k and (Diag(alpha) S)^T q; k.q stays undecayed.
     constexpr int KB = RL < 8 ? RL : 8;
     float kq = 0.0f;
     float2 pp[V / 2], rr[V / 2];
@@ -253,14 +407,17 @@ __global__ void __launch_bounds__(StepCfg<DK, DV, ST, IT>::kThreads, 1) step_ker
     for (int j = 0; j < V / 2; ++j) pp[j] = rr[j] = f2(0.0f, 0.0f);
 #pragma unroll
     for (int r0 = 0; r0 < RL; r0 += KB) {
-      float kb[KB], qb[KB];
-      load_f32<IT, KB>(ks + row0 + r0, kb);
-      load_f32<IT, KB>(qs + row0 + r0, qb);
+      float kb[KB], qb[KB], ab[KB];
+      load_f32<OT, KB>(ks + row0 + r0, kb);
+      load_f32<OT, KB>(qs + row0 + r0, qb);
+      if (CHG) load_f32<float, KB>(as + row0 + r0, ab);
 #pragma unroll
       for (int r = 0; r < KB; ++r) {
         kq = fmaf(kb[r], qb[r], kq);
-        const float2 k2 = f2(kb[r], kb[r]);
-        const float2 q2 = f2(qb[r], qb[r]);
+        const float kr = CHG ? kb[r] * ab[r] : kb[r];
+        const float qr = CHG ? qb[r] * ab[r] : qb[r];
+        const float2 k2 = f2(kr, kr);
+        const float2 q2 = f2(qr, qr);
 #pragma unroll
         for (int j = 0; j < V / 2; ++j) {
           const float2 s2 = f2(s[r0 + r][2 * j], s[r0 + r][2 * j + 1]);
@@ -286,7 +443,7 @@ __global__ void __launch_bounds__(StepCfg<DK, DV, ST, IT>::kThreads, 1) step_ker
     if (m.valid) {
       // u = b (v - c p),  o = scale (a r + (k.q) u)
       float vv[V], u[V], o[V];
-      load_f32<IT, V>(vs + col0, vv);
+      load_f32<OT, V>(vs + col0, vv);
 #pragma unroll
       for (int j = 0; j < V / 2; ++j) {
         u[2 * j] = bcoef * (vv[2 * j] - c * pp[j].x);
@@ -296,25 +453,90 @@ __global__ void __launch_bounds__(StepCfg<DK, DV, ST, IT>::kThreads, 1) step_ker
       }
       if (rb == 0) store_f32<IT, V>(out + m.o_off + col0, o);
 
-      // S' = a S + k u^T, stored with 16-byte vectors
-      ST* dtile = dst + m.dst_off;
+      // the group's other queries read the same updated state: o = scale (a S^T q + (k.q) u)
+      if (QGRP) {
+#pragma unroll 1
+        for (int qi = 1; qi < qg; ++qi) {
+          float kqi = 0.0f;
+          float2 ri[V / 2];
+#pragma unroll
+          for (int j = 0; j < V / 2; ++j) ri[j] = f2(0.0f, 0.0f);
+#pragma unroll
+          for (int r0 = 0; r0 < RL; r0 += KB) {
+            float kb[KB], qb[KB], ab[KB];
+            load_f32<OT, KB>(ks + row0 + r0, kb);
+            load_f32<OT, KB>(qs + qi * DK + row0 + r0, qb);
+            if (CHG) load_f32<float, KB>(as + row0 + r0, ab);
+#pragma unroll
+            for (int r = 0; r < KB; ++r) {
+              kqi = fmaf(kb[r], qb[r], kqi);
+              const float qr = CHG ? qb[r] * ab[r] : qb[r];
+              const float2 q2 = f2(qr, qr);
+#pragma unroll
+              for (int j = 0; j < V / 2; ++j) ri[j] = fma2(f2(s[r0 + r][2 * j], s[r0 + r][2 * j + 1]), q2, ri[j]);
+            }
+          }
+#pragma unroll
+          for (int off = C::kNCH; off < 32; off <<= 1) {
+            kqi += __shfl_xor_sync(0xffffffffu, kqi, off);
+#pragma unroll
+            for (int j = 0; j < V / 2; ++j) {
+              ri[j].x += __shfl_xor_sync(0xffffffffu, ri[j].x, off);
+              ri[j].y += __shfl_xor_sync(0xffffffffu, ri[j].y, off);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < V / 2; ++j) {
+            o[2 * j] = p.scale * fmaf(a, ri[j].x, kqi * u[2 * j]);
+            o[2 * j + 1] = p.scale * fmaf(a, ri[j].y, kqi * u[2 * j + 1]);
+          }
+          if (rb == 0) store_f32<IT, V>(out + m.o_off + qi * DV + col0, o);
+        }
+      }
+
+      // S' = a S + k u^T, stored with 16-byte vectors (q8: 8 codes or 8 BF16 values)
+      unsigned char* dtile = dst + m.dst_off;
       const float2 a2 = f2(a, a);
 #pragma unroll
       for (int r0 = 0; r0 < RL; r0 += KB) {
-        float kb[KB];
-        load_f32<IT, KB>(ks + row0 + r0, kb);
+        float kb[KB], ab[KB];
+        load_f32<OT, KB>(ks + row0 + r0, kb);
+        if (CHG) load_f32<float, KB>(as + row0 + r0, ab);
 #pragma unroll
         for (int r = 0; r < KB; ++r) {
           const float2 k2 = f2(kb[r], kb[r]);
+          const float2 ar = CHG ? f2(ab[r], ab[r]) : a2;
           float y[V];
 #pragma unroll
           for (int j = 0; j < V / 2; ++j) {
             const float2 t =
-                fma2(k2, f2(u[2 * j], u[2 * j + 1]), mul2(a2, f2(s[r0 + r][2 * j], s[r0 + r][2 * j + 1])));
+                fma2(k2, f2(u[2 * j], u[2 * j + 1]), mul2(ar, f2(s[r0 + r][2 * j], s[r0 + r][2 * j + 1])));
             y[2 * j] = t.x;
             y[2 * j + 1] = t.y;
           }
-          *reinterpret_cast<uint4*>(dtile + (row0 + r0 + r) * DV + col0) = StateVec<ST>::pack(y);
+          if constexpr (C::kQ8) {
+            // group absmax over the 4 lanes holding this row of the strip
+            float amax = 0.0f;
+#pragma unroll
+            for (int e = 0; e < V; ++e) amax = fmaxf(amax, fabsf(y[e]));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            int idx;
+            if (rows_dst.row(r0 + r, idx)) {
+              *reinterpret_cast<uint4*>(dtile + n8d * DV + n8d * NG * 4 + (idx * DV + col0) * 2) =
+                  StateVec<__nv_bfloat16>::pack(y);
+            } else {
+              float sc, inv;
+              q8_scales(amax, sc, inv);
+              uint32_t w[2];
+              q8_pack<8>(y, inv, w);
+              *reinterpret_cast<uint2*>(dtile + idx * DV + col0) = make_uint2(w[0], w[1]);
+              if (ch == 0) *reinterpret_cast<float*>(dtile + n8d * DV + (idx * NG + part) * 4) = sc;
+            }
+          } else {
+            *reinterpret_cast<uint4*>(reinterpret_cast<ST*>(dtile) + (row0 + r0 + r) * DV + col0) =
+                StateVec<ST>::pack(y);
+          }
         }
       }
     }
@@ -323,10 +545,10 @@ __global__ void __launch_bounds__(StepCfg<DK, DV, ST, IT>::kThreads, 1) step_ker
   }
 }
 
-template <int RULE, int DK, int DV, typename ST, typename IT>
+template <int RULE, int DK, int DV, typename ST, typename IT, bool QGRP, bool CONV = false>
 cudaError_t launch_step(const StepParams& p, cudaStream_t stream) {
-  using C = StepCfg<DK, DV, ST, IT>;
-  const void* fn = reinterpret_cast<const void*>(&step_kernel<RULE, DK, DV, ST, IT>);
+  using C = StepCfg<DK, DV, ST, IT, Rule<RULE>::kChannelGate, QGRP ? kMaxQueryGroup : 1, CONV>;
+  const void* fn = reinterpret_cast<const void*>(&step_kernel<RULE, DK, DV, ST, IT, QGRP, CONV>);
   const int per_sm = prepare_kernel(fn, C::kThreads, C::kSmem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;
   const int64_t ntiles = (int64_t)p.B * p.n_v_heads;
@@ -343,27 +565,63 @@ cudaError_t launch_step(const StepParams& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, step_kernel<RULE, DK, DV, ST, IT>, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, step_kernel<RULE, DK, DV, ST, IT, QGRP, CONV>, p);
   if (e != cudaSuccess) return e;
 #else
-  step_kernel<RULE, DK, DV, ST, IT><<<grid, C::kThreads, C::kSmem, stream>>>(p);
+  step_kernel<RULE, DK, DV, ST, IT, QGRP, CONV><<<grid, C::kThreads, C::kSmem, stream>>>(p);
 #endif
   return cudaGetLastError();
 }
 
-// Launcher table for one state dtype: rule x (d_k, d_v) x io dtype.
-template <typename ST>
+// Launcher table for one state dtype and head direction: rule x (d_k, d_v) x io dtype.
+template <typename ST, bool QGRP>
 StepLaunchFn find_step_impl(int rule, int dk, int dv, int io) {
 #define LA_STEP_CASE(R, K, V)                                                                    \
   if (rule == R && dk == K && dv == V)                                                           \
-    return io == LA_F32 ? &launch_step<R, K, V, ST, float> : &launch_step<R, K, V, ST, __nv_bfloat16>;
+    return io == LA_F32 ? &launch_step<R, K, V, ST, float, QGRP> : &launch_step<R, K, V, ST, __nv_bfloat16, QGRP>;
 #define LA_STEP_SHAPES(R) LA_STEP_CASE(R, 16, 16) LA_STEP_CASE(R, 64, 64) LA_STEP_CASE(R, 128, 64) LA_STEP_CASE(R, 128, 128)
   LA_STEP_SHAPES(LA_RULE_LINEAR)
   LA_STEP_SHAPES(LA_RULE_GATED)
   LA_STEP_SHAPES(LA_RULE_DELTA)
   LA_STEP_SHAPES(LA_RULE_GATED_DELTA)
+  LA_STEP_SHAPES(LA_RULE_KDA)
 #undef LA_STEP_SHAPES
 #undef LA_STEP_CASE
+  return nullptr;
+}
+
+// Launcher table of the q8 state storage (d_v a multiple of the 32-column group).
+template <bool QGRP>
+StepLaunchFn find_step_q8_impl(int rule, int dk, int dv, int io) {
+#define LA_Q8_CASE(R, K, V)                                                                      \
+  if (rule == R && dk == K && dv == V)                                                           \
+    return io == LA_F32 ? &launch_step<R, K, V, q8_t, float, QGRP> : &launch_step<R, K, V, q8_t, __nv_bfloat16, QGRP>;
+#define LA_Q8_SHAPES(R) LA_Q8_CASE(R, 64, 64) LA_Q8_CASE(R, 128, 64) LA_Q8_CASE(R, 128, 128)
+  LA_Q8_SHAPES(LA_RULE_LINEAR)
+  LA_Q8_SHAPES(LA_RULE_GATED)
+  LA_Q8_SHAPES(LA_RULE_DELTA)
+  LA_Q8_SHAPES(LA_RULE_GATED_DELTA)
+  LA_Q8_SHAPES(LA_RULE_KDA)
+#undef LA_Q8_SHAPES
+#undef LA_Q8_CASE
+  return nullptr;
+}
+
+// Launcher table of the step with the convolution fused ahead (FP32 or BF16 state).
+template <typename ST>
+StepLaunchFn find_step_conv_impl(int rule, int dk, int dv, int io) {
+#define LA_CONV_CASE(R, K, V)                                                                    \
+  if (rule == R && dk == K && dv == V)                                                           \
+    return io == LA_F32 ? &launch_step<R, K, V, ST, float, false, true>                          \
+                        : &launch_step<R, K, V, ST, __nv_bfloat16, false, true>;
+#define LA_CONV_SHAPES(R) LA_CONV_CASE(R, 16, 16) LA_CONV_CASE(R, 64, 64) LA_CONV_CASE(R, 128, 64) LA_CONV_CASE(R, 128, 128)
+  LA_CONV_SHAPES(LA_RULE_LINEAR)
+  LA_CONV_SHAPES(LA_RULE_GATED)
+  LA_CONV_SHAPES(LA_RULE_DELTA)
+  LA_CONV_SHAPES(LA_RULE_GATED_DELTA)
+  LA_CONV_SHAPES(LA_RULE_KDA)
+#undef LA_CONV_SHAPES
+#undef LA_CONV_CASE
   return nullptr;
 }
 

@@ -3,5 +3,5 @@
 #include "la_step.cuh"
 
 namespace la {
-StepLaunchFn find_step_bf16(int rule, int dk, int dv, int io) { return find_step_impl<__nv_bfloat16>(rule, dk, dv, io); }
+StepLaunchFn find_step_bf16(int rule, int dk, int dv, int io) { return find_step_impl<__nv_bfloat16, false>(rule, dk, dv, io); }
 }  // namespace la

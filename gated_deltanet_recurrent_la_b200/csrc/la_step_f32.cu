@@ -3,5 +3,5 @@
 #include "la_step.cuh"
 
 namespace la {
-StepLaunchFn find_step_f32(int rule, int dk, int dv, int io) { return find_step_impl<float>(rule, dk, dv, io); }
+StepLaunchFn find_step_f32(int rule, int dk, int dv, int io) { return find_step_impl<float, false>(rule, dk, dv, io); }
 }  // namespace la

@@ -20,15 +20,16 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "liblastate.so")
 
-RULES = {"linear": 0, "gated": 1, "delta": 2, "gated_delta": 3}
-LA_F32, LA_BF16 = 0, 1
+RULES = {"linear": 0, "gated": 1, "delta": 2, "gated_delta": 3, "kda": 4}
+LA_F32, LA_BF16, LA_Q8 = 0, 1, 2
 STATUS = {0: "LA_OK", 1: "LA_ERR_NULL", 2: "LA_ERR_SHAPE", 3: "LA_ERR_UNSUPPORTED", 4: "LA_ERR_ALIGN",
           5: "LA_ERR_ALIAS", 6: "LA_ERR_CUDA"}
 LA_OK, LA_ERR_NULL, LA_ERR_SHAPE, LA_ERR_UNSUPPORTED, LA_ERR_ALIGN, LA_ERR_ALIAS, LA_ERR_CUDA = range(7)
-DEVERR_READ_SLOT, DEVERR_WRITE_SLOT, DEVERR_CU_SEQLENS, DEVERR_TIMEOUT = 1, 2, 4, 8
+DEVERR_READ_SLOT, DEVERR_WRITE_SLOT, DEVERR_CU_SEQLENS, DEVERR_TIMEOUT, DEVERR_Q8_MASK = 1, 2, 4, 8, 16
 
 EXPORTS = ("la_state_bytes", "la_shape_supported", "la_state_step", "la_state_scan", "la_state_scan_chunked",
-           "la_state_scan_checkpointed",
+           "la_state_scan_checkpointed", "la_state_step_qgroups", "la_state_scan_qgroups",
+           "la_pool_slot_bytes", "la_state_pool_encode", "la_state_pool_decode", "la_state_step_conv",
            "la_state_pool_copy",
            "la_state_pool_gather", "la_state_pool_scatter", "la_state_pool_zero", "la_state_check_slots",
            "la_status_str", "la_last_cuda_error", "la_abi_version")
@@ -50,7 +51,13 @@ class la_shape(ctypes.Structure):
 
 class la_pool(ctypes.Structure):
     _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("n_slots", ctypes.c_int32),
-                ("shape", la_shape)]
+                ("shape", la_shape), ("n_hp", ctypes.c_int32), ("hp_mask", ctypes.c_void_p)]
+
+
+class la_conv(ctypes.Structure):
+    _fields_ = [("width", ctypes.c_int32), ("activation", ctypes.c_int32), ("qk_l2norm", ctypes.c_int32),
+                ("w_q", ctypes.c_void_p), ("w_k", ctypes.c_void_p), ("w_v", ctypes.c_void_p),
+                ("hist_src", ctypes.c_void_p), ("hist_dst", ctypes.c_void_p)]
 
 
 _lib = None
@@ -78,12 +85,25 @@ def lib():
         L.la_state_scan_chunked.restype = I32
         L.la_state_scan_checkpointed.argtypes = L.la_state_scan.argtypes[:-2] + [I32, P, P, P, P]
         L.la_state_scan_checkpointed.restype = I32
+        L.la_state_step_qgroups.argtypes = L.la_state_step.argtypes[:6] + [I32] + L.la_state_step.argtypes[6:]
+        L.la_state_step_qgroups.restype = I32
+        L.la_state_scan_qgroups.argtypes = L.la_state_scan.argtypes[:9] + [I32] + L.la_state_scan.argtypes[9:]
+        L.la_state_scan_qgroups.restype = I32
         L.la_state_pool_copy.argtypes = [PP, I32, P, P, P, P]
         L.la_state_pool_gather.argtypes = [PP, I32, P, P, P, P]
         L.la_state_pool_scatter.argtypes = [PP, I32, P, P, P, P]
         L.la_state_pool_zero.argtypes = [PP, I32, P, P, P]
         for f in (L.la_state_pool_copy, L.la_state_pool_gather, L.la_state_pool_scatter, L.la_state_pool_zero):
             f.restype = I32
+        L.la_state_step_conv.argtypes = L.la_state_step.argtypes[:6] + [ctypes.POINTER(la_conv)] + \
+            L.la_state_step.argtypes[6:]
+        L.la_state_step_conv.restype = I32
+        L.la_pool_slot_bytes.argtypes = [PP]
+        L.la_pool_slot_bytes.restype = ctypes.c_size_t
+        L.la_state_pool_encode.argtypes = [PP, I32, P, P, P, P]
+        L.la_state_pool_encode.restype = I32
+        L.la_state_pool_decode.argtypes = [PP, I32, P, P, P, P]
+        L.la_state_pool_decode.restype = I32
         L.la_state_check_slots.argtypes = [I32, P, P, I32]
         L.la_state_check_slots.restype = I32
         L.la_status_str.argtypes = [I32]
@@ -126,15 +146,31 @@ def _stream(stream) -> ctypes.c_void_p:
 
 
 class Pool:
-    """A slot pool: tensor [n_slots, H_v, d_k, d_v] (float32 or bfloat16) plus H_qk."""
+    """A slot pool: tensor [n_slots, H_v, d_k, d_v] (float32 or bfloat16) plus H_qk; or, for
+    the mixed INT8 / BF16 storage, Pool.q8(...)."""
 
     def __init__(self, tensor: torch.Tensor, n_qk_heads: int):
         if tensor.dim() != 4:
             raise ValueError("pool tensor must be [n_slots, H_v, d_k, d_v]")
         self.tensor = tensor
+        self.mask = None
         n, hv, dk, dv = tensor.shape
         self.struct = la_pool(_ptr(tensor), dtype_code(tensor.dtype), n,
-                              la_shape(int(n_qk_heads), hv, dk, dv))
+                              la_shape(int(n_qk_heads), hv, dk, dv), 0, None)
+
+    @classmethod
+    def q8(cls, tensor: torch.Tensor, n_qk_heads: int, d_k: int, d_v: int, n_hp: int, mask: torch.Tensor):
+        """A q8 pool: tensor uint8 [n_slots, H_v, tile bytes], mask int32 [H_v, d_k / 32]
+        holding the uint32 channel-mask words (bit i set: channel i kept in BF16)."""
+        if tensor.dim() != 3 or tensor.dtype != torch.uint8:
+            raise ValueError("q8 pool tensor must be uint8 [n_slots, H_v, tile bytes]")
+        self = cls.__new__(cls)
+        self.tensor = tensor
+        self.mask = mask
+        n, hv, _ = tensor.shape
+        self.struct = la_pool(_ptr(tensor), LA_Q8, n, la_shape(int(n_qk_heads), hv, int(d_k), int(d_v)), int(n_hp),
+                              _ptr(mask, torch.int32))
+        return self
 
     @property
     def ref(self):
@@ -195,6 +231,74 @@ def la_state_scan_checkpointed(rule, src: Optional[Pool], read_slot, dst: Pool, 
         _ptr(v, q.dtype), io, _ptr(g, torch.float32), _ptr(beta, torch.float32), float(scale), _ptr(o, q.dtype),
         int(ckpt_every), _ptr(ckpt_cu, torch.int32), _ptr(ckpt_slots, torch.int32), _ptr(err_word, torch.int32),
         _stream(stream))
+
+
+class Conv:
+    """The short causal convolution ahead of the step: weights (float32 [heads, channels,
+    W] on the device) and the history pools (io dtype [n_slots, H_v, 2 d_k + d_v, W - 1])."""
+
+    def __init__(self, w_q, w_k, w_v, hist_src, hist_dst=None, activation=0, qk_l2norm=0):
+        self.keep = (w_q, w_k, w_v, hist_src, hist_dst)
+        hist_dst = hist_src if hist_dst is None else hist_dst
+        self.struct = la_conv(int(w_q.shape[2]), int(activation), int(qk_l2norm), _ptr(w_q, torch.float32),
+                              _ptr(w_k, torch.float32), _ptr(w_v, torch.float32), _ptr(hist_src), _ptr(hist_dst))
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+
+def la_state_step_conv(rule, src: Pool, read_slot, dst: Pool, write_slot, conv: Conv, xq, xk, xv, g, beta, scale, o,
+                       err_word, stream=None) -> int:
+    io = dtype_code(xq.dtype)
+    return lib().la_state_step_conv(RULES[rule] if isinstance(rule, str) else int(rule), src.ref,
+                                    _ptr(read_slot, torch.int32), dst.ref, _ptr(write_slot, torch.int32),
+                                    int(xq.shape[0]), conv.ref, _ptr(xq), _ptr(xk, xq.dtype), _ptr(xv, xq.dtype), io,
+                                    _ptr(g, torch.float32), _ptr(beta, torch.float32), float(scale),
+                                    _ptr(o, xq.dtype), _ptr(err_word, torch.int32), _stream(stream))
+
+
+def q8_tile_bytes(d_k: int, d_v: int, n_hp: int) -> int:
+    """Bytes of one (slot, head) tile of a q8 pool (the layout of la_state.h)."""
+    return (d_k - n_hp) * d_v + (d_k - n_hp) * (d_v // 32) * 4 + n_hp * d_v * 2
+
+
+def la_pool_slot_bytes(pool: Pool) -> int:
+    return lib().la_pool_slot_bytes(pool.ref)
+
+
+def la_state_pool_encode(pool: Pool, slots, dense, err_word, stream=None) -> int:
+    return lib().la_state_pool_encode(pool.ref, int(slots.numel()), _ptr(slots, torch.int32),
+                                      _ptr(dense, torch.float32), _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_state_pool_decode(pool: Pool, slots, dense, err_word, stream=None) -> int:
+    return lib().la_state_pool_decode(pool.ref, int(slots.numel()), _ptr(slots, torch.int32),
+                                      _ptr(dense, torch.float32), _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_state_step_qgroups(rule, src: Pool, read_slot, dst: Pool, write_slot, q, k, v, g, beta, scale, o, err_word,
+                          stream=None) -> int:
+    """Query-group direction: k [B, H_v, d_k], q [B, n_q_heads, d_k], o [B, n_q_heads, d_v]."""
+    io = dtype_code(q.dtype)
+    return lib().la_state_step_qgroups(RULES[rule] if isinstance(rule, str) else int(rule), src.ref,
+                                       _ptr(read_slot, torch.int32), dst.ref, _ptr(write_slot, torch.int32),
+                                       int(q.shape[0]), int(q.shape[1]), _ptr(q), _ptr(k, q.dtype), _ptr(v, q.dtype),
+                                       io, _ptr(g, torch.float32), _ptr(beta, torch.float32), float(scale),
+                                       _ptr(o, q.dtype), _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_state_scan_qgroups(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens, q, k, v, g, beta,
+                          scale, o, err_word, seq_order=None, stream=None) -> int:
+    """Query-group direction of la_state_scan: k [T, H_v, d_k], q [T, n_q_heads, d_k]."""
+    io = dtype_code(q.dtype)
+    return lib().la_state_scan_qgroups(RULES[rule] if isinstance(rule, str) else int(rule),
+                                       None if src is None else src.ref, _ptr(read_slot, torch.int32), dst.ref,
+                                       _ptr(write_slot, torch.int32), int(cu_seqlens.numel() - 1),
+                                       _ptr(cu_seqlens, torch.int32), int(q.shape[0]), _ptr(seq_order, torch.int32),
+                                       int(q.shape[1]), _ptr(q), _ptr(k, q.dtype), _ptr(v, q.dtype), io,
+                                       _ptr(g, torch.float32), _ptr(beta, torch.float32), float(scale),
+                                       _ptr(o, q.dtype), _ptr(err_word, torch.int32), _stream(stream))
 
 
 def la_state_pool_copy(pool: Pool, src_slots, dst_slots, err_word, stream=None) -> int:

@@ -21,6 +21,9 @@ Named workloads (sizes from the "SSM / linear-RNN decode" page, the ONNX section
   prefill32   32 packed sequences, lengths U_int[1024, 8192], 32 heads, 128 x 128 scan
   mamba2      B=256 gated decode, 128 heads x 64, d_state 128 (Nemotron-H-8B layer sizes)
   kda_decode64, kda_prefill32   the same shapes with the channel-wise (kda) gate
+  qgroup_decode256  B=256 decode, 16 state heads each read by 4 query heads (ONNX direction)
+  q8_decode64 decode64 on the mixed INT8 / BF16 state storage (1/8 of the key channels BF16)
+  conv_decode64  decode64 with the short causal convolution (width 4, SiLU, q/k norm) ahead
 """
 from __future__ import annotations
 
@@ -207,6 +210,55 @@ def kda_decode64(seed: int = 0) -> Inputs:
                        slot_map="perm", rule="kda")
 
 
+def qgroup_decode256(seed: int = 0) -> Inputs:
+    """Decode in the query-group direction of the ONNX operator: B=256, 16 KV (state) heads
+    each read by 4 query heads (64 query heads), 128 x 128 BF16 state, 1024-slot pool,
+    read = write = randperm(1024)[:256]."""
+    return step_inputs(B=256, n_qk_heads=16, n_v_heads=16, d_k=128, d_v=128, n_slots=1024, seed=seed,
+                       slot_map="perm", n_q_heads=64)
+
+
+def hp_masks(n_v_heads: int, d_k: int, n_hp: int, gen: torch.Generator) -> torch.Tensor:
+    """Channel masks of a q8 pool: for each head, n_hp key channels drawn at random (an
+    offline calibration would choose them; none is done here).  int32 [H_v, d_k / 32]
+    holding the uint32 mask words."""
+    words = torch.zeros(n_v_heads, d_k // 32, dtype=torch.int64)
+    for h in range(n_v_heads):
+        for i in torch.randperm(d_k, generator=gen)[:n_hp].tolist():
+            words[h, i // 32] |= 1 << (i % 32)
+    return ((words + 2 ** 31) % 2 ** 32 - 2 ** 31).to(torch.int32)
+
+
+def q8_decode64(seed: int = 0, n_hp: int = 16) -> Inputs:
+    """decode64 on a q8 pool (INT8 state with 1/8 of the key channels in BF16, 9.875 bits
+    per value): FP32 initial values N(0, 0.05) (encoded into the pool by the library),
+    channel masks drawn at random, the masks and n_hp in `extra`."""
+    inp = step_inputs(B=64, n_qk_heads=16, n_v_heads=32, d_k=128, d_v=128, n_slots=256, seed=seed,
+                      slot_map="perm", state_dtype=torch.float32)
+    inp.state_dtype = torch.uint8  # marks the q8 storage
+    inp.extra = {"n_hp": n_hp, "hp_mask": hp_masks(32, 128, n_hp, _gen(seed + 7))}
+    return inp
+
+
+def conv_decode64(seed: int = 0, width: int = 4) -> Inputs:
+    """decode64 with the short causal convolution ahead of the step: q, k, v are the
+    convolution's inputs (N(0, 1), not normalised), weights N(0, 1 / W) per channel, the
+    histories N(0, 1) in BF16 [256 slots, 32 heads, 2 * 128 + 128, W - 1]; SiLU and the q/k
+    normalisation on (`extra`)."""
+    inp = step_inputs(B=64, n_qk_heads=16, n_v_heads=32, d_k=128, d_v=128, n_slots=256, seed=seed,
+                      slot_map="perm", normalise_qk=False)
+    gen = _gen(seed + 11)
+    W = width
+    inp.extra = {
+        "width": W, "activation": 1, "qk_l2norm": 1,
+        "w_q": (torch.randn(16, 128, W, generator=gen) / W ** 0.5).contiguous(),
+        "w_k": (torch.randn(16, 128, W, generator=gen) / W ** 0.5).contiguous(),
+        "w_v": (torch.randn(32, 128, W, generator=gen) / W ** 0.5).contiguous(),
+        "hist": torch.randn(256, 32, 3 * 128, W - 1, generator=gen).to(torch.bfloat16).contiguous(),
+    }
+    return inp
+
+
 def decode512(seed: int = 0) -> Inputs:
     """Large decode: B=512, same heads, 1024-slot pool; half the requests read a
     checkpoint slot and write a distinct live slot, the rest update in place."""
@@ -259,4 +311,7 @@ WORKLOADS = {
     "mamba2": mamba2,
     "kda_decode64": kda_decode64,
     "kda_prefill32": kda_prefill32,
+    "qgroup_decode256": qgroup_decode256,
+    "q8_decode64": q8_decode64,
+    "conv_decode64": conv_decode64,
 }

@@ -10,10 +10,13 @@
  *   o = scale * S^T q                readout by the query, from the UPDATED state
  *
  *   rule         a   b     c       source
- *   linear       1   1     0       "basic additive"
- *   gated        g   1     0       "exponential decay"
- *   delta        1   beta  1       "delta rule without decay"
+ *   linear       1   1     0       plain additive update
+ *   gated        g   1     0       update decayed by a gate
+ *   delta        1   beta  1       delta correction without a gate
  *   gated_delta  g   beta  g       S <- g (I - beta k k^T) S + beta k v^T (the default)
+ *   kda          channel-wise gate: S <- (I - beta k k^T) Diag(alpha) S + beta k v^T,
+ *                i.e. u = beta (v - (Diag(alpha) S)^T k), S <- Diag(alpha) S + k u^T,
+ *                with alpha in R^{d_k} (one decay per key channel)
  *
  * The rule names, their one-line meanings and the default are those of the ONNX
  * LinearAttention operator described in "Seven Architectures Replacing KV Cache With
@@ -21,9 +24,11 @@
  * gated_delta recurrence is the one of the "Gated DeltaNet" glossary page (Technical
  * definition: decay by a gate, rank-one delta-rule correction, projection by the
  * query) and of the KDA formula in the "Kimi Linear" section of the same article,
- * read with a scalar gate.  The kernels compute the readout in the rearranged form of
- * the "Gated DeltaNet" page (Engineering details),
- *   o = scale * ( a * (S_old^T q) + (k . q) * u ),
+ * read with a scalar gate; kda is that formula with its channel-wise gate alpha_t
+ * (Kimi Delta Attention), the prediction taken from the decayed state.  The kernels
+ * compute the readout in the rearranged form of the "Gated DeltaNet" page
+ * (Engineering details),
+ *   o = scale * ( a * (S_old^T q) + (k . q) * u )   (kda: (Diag(alpha) S_old)^T q),
  * so that the update and the readout share one pass over S.  All arithmetic is FP32;
  * the state is stored in FP32 or BF16 (rounded to nearest even), as in the "Recurrent
  * state" glossary page (Why it matters: BF16 storage, FP32 compute).
@@ -34,6 +39,7 @@
  *   q, k         [B or T, H_qk, d_k]   io dtype  state head h reads q/k head h / (H_v/H_qk)
  *   v, o         [B or T, H_v,  d_v]   io dtype
  *   g, beta      [B or T, H_v]         float32
+ *   g (kda)      [B or T, H_v, d_k]    float32, 16-byte aligned
  * Supported (d_k, d_v): (16,16), (64,64), (128,64), (128,128).
  *
  * Slots.  A request reads its state from read_slot[b] of the source pool and writes
@@ -55,6 +61,9 @@
  *   - Preconditions (not checked on the device; la_state_check_slots checks them on the
  *     host): write slots are distinct, and no write slot equals another request's read
  *     slot.  Read slots may repeat; a request may read and write the same slot.
+ *   - LA_Q8 pools: la_state_step takes them as source and destination together (equal
+ *     n_hp; the masks may differ); the scans take them as source and / or destination;
+ *     la_state_scan_chunked and the query-group entry points return LA_ERR_UNSUPPORTED.
  *   - Pointers to the pool, q, k, v, o and dense buffers must be 16-byte aligned;
  *     g, beta and int32 arrays 4-byte aligned.
  */
@@ -68,16 +77,18 @@
 extern "C" {
 #endif
 
-#define LA_ABI_VERSION 1
+#define LA_ABI_VERSION 2
 
 typedef enum {
     LA_RULE_LINEAR = 0,
     LA_RULE_GATED = 1,
     LA_RULE_DELTA = 2,
-    LA_RULE_GATED_DELTA = 3
+    LA_RULE_GATED_DELTA = 3,
+    LA_RULE_KDA = 4 /* channel-wise gate (Kimi Delta Attention); g holds d_k decays per head */
 } la_rule;
 
-typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
+/* LA_Q8 (state pools only): the mixed INT8 / BF16 storage described at la_pool. */
+typedef enum { LA_F32 = 0, LA_BF16 = 1, LA_Q8 = 2 } la_dtype;
 
 typedef enum {
     LA_OK = 0,
@@ -94,6 +105,7 @@ typedef enum {
 #define LA_DEVERR_WRITE_SLOT 2u /* a write / destination slot index outside [0, n_slots) */
 #define LA_DEVERR_CU_SEQLENS 4u /* cu_seqlens not non-decreasing within [0, total_tokens], or a bad seq_order entry */
 #define LA_DEVERR_TIMEOUT 8u    /* an internal pipeline wait gave up (should never happen) */
+#define LA_DEVERR_Q8_MASK 16u   /* a q8 head's channel mask does not hold exactly n_hp rows */
 
 typedef struct {
     int32_t n_qk_heads; /* H_qk: heads of q and k */
@@ -102,15 +114,39 @@ typedef struct {
     int32_t d_v;
 } la_shape;
 
-/* A slot pool: n_slots states of `shape`, contiguous, [n_slots, H_v, d_k, d_v]. */
+/* A slot pool: n_slots states of `shape`, contiguous, [n_slots, H_v, d_k, d_v].
+ *
+ * LA_Q8 pools hold the state in the mixed precision of DAMP ("Seven Architectures ...",
+ * sections "ONNX LinearAttention / FlashInfer" and Practical Implications: the high-risk
+ * key channels in a higher precision, the rest in INT8, about 9.9 bits per value).  The
+ * pages fix no layout; this library's: per (slot, head) tile, the key channels (rows)
+ * whose bit is set in the head's mask are kept in BF16, every other row in INT8 codes
+ * with one FP32 scale per group of 32 columns:
+ *   s = absmax * fl(1/127),  inv = fl(1/absmax) * 127,  code = clamp(rint(x * inv), -127, 127),
+ *   x' = code * s
+ * (NaN codes to 0; s = inv = 0 and codes 0 for an all-zero group; every operation a
+ * correctly rounded FP32 one).  Tile
+ * bytes: codes [d_k - n_hp][d_v] int8, scales [d_k - n_hp][d_v / 32] float32, BF16 rows
+ * [n_hp][d_v], each block in increasing row order; n_hp = d_k / 8 gives 9.875 bits per
+ * value.  (d_k, d_v) in {(64,64), (128,64), (128,128)}; n_hp even, 0 <= n_hp <= d_k / 4.
+ * The mask (which channels are high-risk) comes from an offline calibration that is not
+ * part of this library. */
 typedef struct {
     void *data;     /* device pointer, 16-byte aligned */
     int32_t dtype;  /* la_dtype of the stored state */
     int32_t n_slots;
     la_shape shape;
+    int32_t n_hp;             /* LA_Q8: BF16 key channels per head; ignored otherwise */
+    const uint32_t *hp_mask;  /* LA_Q8: device uint32 [H_v][d_k / 32], bit i of head h's words
+                                 set for a BF16 channel (exactly n_hp per head); else NULL */
 } la_pool;
 
-/* Bytes of one slot (one request's state for one layer): H_v * d_k * d_v * sizeof(dtype).
+/* Bytes of one slot of `pool` for any dtype (q8 included); 0 for an invalid pool.  Pure
+ * host function. */
+size_t la_pool_slot_bytes(const la_pool *pool);
+
+/* Bytes of one slot (one request's state for one layer) of an LA_F32 or LA_BF16 pool:
+ * H_v * d_k * d_v * sizeof(dtype) (0 for LA_Q8: see la_pool_slot_bytes).
  * Pure host function; returns 0 for an invalid shape or dtype.  For 64 heads of 128 x 128
  * at 2 bytes this is 2 MiB, the per-request figure of the ONNX section of "Seven
  * Architectures ..."; for 128 heads of 128 x 64 at BF16 it is 2 MiB, the Nemotron-H-8B
@@ -125,7 +161,8 @@ int la_shape_supported(int32_t d_k, int32_t d_v);
  *   read_slot    device int32 [B] or NULL (request b reads src slot b)
  *   write_slot   device int32 [B] or NULL (request b writes dst slot b)
  *   q, k         [B, H_qk, d_k] io dtype;  v, o: [B, H_v, d_v] io dtype
- *   g            float32 [B, H_v]; required for gated / gated_delta, ignored otherwise
+ *   g            float32 [B, H_v]; required for gated / gated_delta, ignored otherwise;
+ *                kda: float32 [B, H_v, d_k] (16-byte aligned), required
  *   beta         float32 [B, H_v]; required for delta / gated_delta, ignored otherwise
  *   scale        multiplies the readout (1.0 for pre-normalised queries)
  *   err_word     device int32, required; bits LA_DEVERR_* are OR-ed in
@@ -151,6 +188,7 @@ la_status la_state_step(la_rule rule, const la_pool *src, const int32_t *read_sl
  *                   handed to the SMs (longest first balances the load best); each
  *                   sequence must appear exactly once.  NULL = 0, 1, 2, ...
  *   q, k            [T, H_qk, d_k];  v, o: [T, H_v, d_v];  g, beta: [T, H_v]
+ *                   (kda: g is [T, H_v, d_k], 16-byte aligned)
  * Empty sequences are allowed (their initial state is copied to the destination).
  * n_seqs == 0 is a no-op returning LA_OK. */
 la_status la_state_scan(la_rule rule, const la_pool *src, const int32_t *read_slot,
@@ -168,7 +206,8 @@ la_status la_state_scan(la_rule rule, const la_pool *src, const int32_t *read_sl
  * across the sequence.  Results agree with la_state_scan to BF16 precision (about 5e-3 of
  * the largest output over thousands of tokens), not bit for bit.
  * Arguments, outputs and errors as la_state_scan.  Supported: d_k = d_v = 128 with BF16
- * q/k/v/o (LA_ERR_UNSUPPORTED otherwise); any rule; gates of either sign. */
+ * q/k/v/o, the rules linear, gated, delta and gated_delta, gates of either sign
+ * (LA_ERR_UNSUPPORTED otherwise, kda included: use la_state_scan). */
 la_status la_state_scan_chunked(la_rule rule, const la_pool *src, const int32_t *read_slot,
                                 const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
                                 const int32_t *cu_seqlens, int32_t total_tokens, const int32_t *seq_order,
@@ -177,7 +216,7 @@ la_status la_state_scan_chunked(la_rule rule, const la_pool *src, const int32_t 
                                 int32_t *err_word, void *stream);
 
 /* The scan of la_state_scan that also stores intermediate states: the prefix-cache
- * checkpoints "aligned to KV block boundaries" of the "Gated DeltaNet" glossary page (Why
+ * checkpoints at KV-cache block boundaries of the "Gated DeltaNet" glossary page (Why
  * it matters), and state snapshots for speculative-decoding rollback ("Seven
  * Architectures ...", Limitations and Open Questions).
  *   ckpt_every  > 0; checkpoint j of sequence s is the state after the sequence's first
@@ -198,6 +237,61 @@ la_status la_state_scan_checkpointed(la_rule rule, const la_pool *src, const int
                                      float scale, void *o, int32_t ckpt_every, const int32_t *ckpt_cu,
                                      const int32_t *ckpt_slots, int32_t *err_word, void *stream);
 
+/* The short causal convolution fused ahead of the decode step ("Gated DeltaNet" glossary,
+ * Engineering details: Conv1D fused with the recurrence into one kernel).  The pages give
+ * no width, activation or normalisation; this library's reading: per channel c of the q,
+ * k and v projections, a depthwise causal convolution along time,
+ *   y_t[c] = sum_{j < W} w[c][j] x_{t-W+1+j}[c],
+ * optionally followed by SiLU (y / (1 + e^-y)), then q and k optionally scaled to unit
+ * length per head (y / sqrt(|y|^2 + 1e-6)); the results (FP32, not rounded) are the q, k, v
+ * of the step.  The W - 1 earlier inputs of every channel are kept per (slot, state head):
+ * head h holds its q/k head's 2 d_k channels and its own d_v channels (heads sharing a q/k
+ * head hold equal copies, so no two tiles ever write the same history). */
+typedef struct {
+    int32_t width;          /* W, 2 <= W <= 4 */
+    int32_t activation;     /* 0: none, 1: SiLU */
+    int32_t qk_l2norm;      /* 1: q and k scaled to unit length per head after the convolution */
+    const float *w_q;       /* device float32 [H_qk][d_k][W] (w[c][W - 1] multiplies the newest input) */
+    const float *w_k;       /* device float32 [H_qk][d_k][W] */
+    const float *w_v;       /* device float32 [H_v][d_v][W] */
+    const void *hist_src;   /* device, io dtype [src n_slots][H_v][2 d_k + d_v][W - 1] (q, k, v
+                               channels; oldest input first), read at read_slot; 16-byte aligned */
+    void *hist_dst;         /* same layout with dst n_slots, written at write_slot (may equal hist_src) */
+} la_conv;
+
+/* la_state_step with the convolution ahead of it: xq, xk, xv are the convolution's inputs
+ * (layouts of q, k, v); everything else as la_state_step.  FP32 or BF16 pools (not q8). */
+la_status la_state_step_conv(la_rule rule, const la_pool *src, const int32_t *read_slot,
+                             const la_pool *dst, const int32_t *write_slot, int32_t B,
+                             const la_conv *conv, const void *xq, const void *xk, const void *xv,
+                             la_dtype io, const float *g, const float *beta, float scale, void *o,
+                             int32_t *err_word, void *stream);
+
+/* The query-group direction of the ONNX LinearAttention operator ("Seven Architectures
+ * ...", section "ONNX LinearAttention / FlashInfer": each KV head and its recurrent state
+ * shared by a group of query heads, q_num_heads / kv_num_heads).  The state of head h is
+ * updated once per token with its own key k_h, value v_h and gates; query head i then
+ * reads the updated state of head i / (n_q_heads / H_v):
+ *   o_i = scale * S_h^T q_i        (rearranged in the kernels as for la_state_step)
+ *   pools     n_qk_heads == n_v_heads (the key has one head per state head)
+ *   q         [B or T, n_q_heads, d_k] io dtype;  k: [B or T, H_v, d_k];  v: [B or T, H_v, d_v]
+ *   o         [B or T, n_q_heads, d_v] io dtype;  g, beta as for la_state_step / la_state_scan
+ *   n_q_heads a multiple of H_v with n_q_heads / H_v <= 8 (LA_ERR_SHAPE when not a
+ *             multiple or when n_qk_heads != n_v_heads; LA_ERR_UNSUPPORTED above 8)
+ * Other arguments, supported shapes and errors as la_state_step / la_state_scan. */
+la_status la_state_step_qgroups(la_rule rule, const la_pool *src, const int32_t *read_slot,
+                                const la_pool *dst, const int32_t *write_slot, int32_t B,
+                                int32_t n_q_heads, const void *q, const void *k, const void *v,
+                                la_dtype io, const float *g, const float *beta, float scale,
+                                void *o, int32_t *err_word, void *stream);
+la_status la_state_scan_qgroups(la_rule rule, const la_pool *src, const int32_t *read_slot,
+                                const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
+                                const int32_t *cu_seqlens, int32_t total_tokens,
+                                const int32_t *seq_order, int32_t n_q_heads, const void *q,
+                                const void *k, const void *v, la_dtype io, const float *g,
+                                const float *beta, float scale, void *o, int32_t *err_word,
+                                void *stream);
+
 /* Slot-pool maintenance, bit-exact whole-slot copies ("Recurrent state" glossary: slot
  * allocation and prefix-cache checkpoints; "Seven Architectures ...", ONNX section:
  * snapshots saved and restored for speculative-decoding rollback, migrated between
@@ -215,6 +309,19 @@ la_status la_state_pool_scatter(const la_pool *pool, int32_t n, const int32_t *s
                                 const void *dense, int32_t *err_word, void *stream);
 la_status la_state_pool_zero(const la_pool *pool, int32_t n, const int32_t *slots,
                              int32_t *err_word, void *stream);
+
+/* Conversion between FP32 states and the slots of an LA_Q8 pool (for example, a prefill
+ * state handed to a quantised decode pool, or a quantised state read back):
+ *   encode   pool[slots[i]] <- q8(dense[i])      dense: float32 [n, H_v, d_k, d_v]
+ *   decode   dense[i] <- values of pool[slots[i]]
+ * A slot index outside the pool reports LA_DEVERR_WRITE_SLOT (encode) or
+ * LA_DEVERR_READ_SLOT (decode); a head whose mask does not hold n_hp rows reports
+ * LA_DEVERR_Q8_MASK; those tiles are skipped.  LA_ERR_UNSUPPORTED for a pool that is not
+ * LA_Q8. */
+la_status la_state_pool_encode(const la_pool *pool, int32_t n, const int32_t *slots,
+                               const float *dense, int32_t *err_word, void *stream);
+la_status la_state_pool_decode(const la_pool *pool, int32_t n, const int32_t *slots, float *dense,
+                               int32_t *err_word, void *stream);
 
 /* Host-side check of the slot preconditions of la_state_step / la_state_scan on HOST
  * copies of the slot arrays (either may be NULL = identity): every index in [0, n_slots),

@@ -124,3 +124,50 @@ def oracle_scan(inp, dst_dtype=None):
                        np64(inp.g), np64(inp.beta), inp.scale, src_pool=np64(inp.pool),
                        read_slot=None if inp.read_slot is None else inp.read_slot.numpy(),
                        dst_dtype=dname(dst_dtype), io_dtype=dname(inp.io_dtype))
+
+
+def gpu_step_qgroups(inp):
+    """la_state_step_qgroups on the device (query-group direction)."""
+    pool_t = dev(inp.pool)
+    pool = L.Pool(pool_t, inp.n_qk_heads)
+    B = inp.q.shape[0]
+    o = torch.full((B, inp.n_q_heads, inp.d_v), 7.0, dtype=inp.io_dtype, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = L.la_state_step_qgroups(inp.rule, pool, dev(inp.read_slot), pool, dev(inp.write_slot), dev(inp.q),
+                                 dev(inp.k), dev(inp.v), dev(inp.g), dev(inp.beta), inp.scale, o, err)
+    L.check(st)
+    torch.cuda.synchronize()
+    return pool_t.cpu(), o.cpu(), int(err.item())
+
+
+def oracle_step_qgroups(inp):
+    """Oracle decode step in the query-group direction on the whole pool (slots as given)."""
+    return oracle.step_qgroups(inp.rule, inp.n_q_heads, np64(inp.pool), np64(inp.q), np64(inp.k), np64(inp.v),
+                               np64(inp.g), np64(inp.beta), inp.scale, dst_dtype=dname(inp.state_dtype),
+                               io_dtype=dname(inp.io_dtype),
+                               read_slot=None if inp.read_slot is None else inp.read_slot.numpy(),
+                               write_slot=None if inp.write_slot is None else inp.write_slot.numpy())
+
+
+def gpu_scan_qgroups(inp, dst_dtype=None):
+    n_seqs = inp.cu_seqlens.numel() - 1
+    dst_dtype = inp.state_dtype if dst_dtype is None else dst_dtype
+    dst_t = torch.full((n_seqs, inp.n_v_heads, inp.d_k, inp.d_v), 3.0, dtype=dst_dtype, device="cuda")
+    src_t = dev(inp.pool)
+    src = None if src_t is None else L.Pool(src_t, inp.n_qk_heads)
+    o = torch.full((inp.q.shape[0], inp.n_q_heads, inp.d_v), 5.0, dtype=inp.io_dtype, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = L.la_state_scan_qgroups(inp.rule, src, dev(inp.read_slot), L.Pool(dst_t, inp.n_qk_heads), None,
+                                 dev(inp.cu_seqlens), dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.g), dev(inp.beta),
+                                 inp.scale, o, err)
+    L.check(st)
+    torch.cuda.synchronize()
+    return dst_t.cpu(), o.cpu(), int(err.item())
+
+
+def oracle_scan_qgroups(inp, dst_dtype=None):
+    dst_dtype = inp.state_dtype if dst_dtype is None else dst_dtype
+    return oracle.scan_qgroups(inp.rule, inp.n_q_heads, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k),
+                               np64(inp.v), np64(inp.g), np64(inp.beta), inp.scale, src_pool=np64(inp.pool),
+                               read_slot=None if inp.read_slot is None else inp.read_slot.numpy(),
+                               dst_dtype=dname(dst_dtype), io_dtype=dname(inp.io_dtype))

@@ -52,7 +52,8 @@ def test_library_exports_every_declared_symbol(lib):
     assert not missing, missing
     for f in declared_functions():
         assert hasattr(lib, f)
-    assert lib.la_abi_version() == 1
+    header = open(os.path.join(ROOT, "include", "la_state.h")).read()
+    assert lib.la_abi_version() == int(re.search(r"#define LA_ABI_VERSION (\d+)", header).group(1))
 
 
 def test_state_bytes_match_page_figures(lib):
@@ -125,6 +126,13 @@ def test_step_host_errors(lib):
     assert step(lib, src=pool(data=A + 4)) == L.LA_ERR_ALIGN
     assert step(lib, g=A + 2) == L.LA_ERR_ALIGN
     assert step(lib, B=9) == L.LA_ERR_SHAPE  # dense mode: B > n_slots
+    assert step(lib, rule=4, g=None) == L.LA_ERR_NULL      # kda needs its channel decays
+    assert step(lib, rule=4, beta=None) == L.LA_ERR_NULL
+    assert step(lib, rule=4, g=A + 4) == L.LA_ERR_ALIGN    # kda decays move in 16-byte pieces
+    # a scalar gate needs 4 bytes only: the call gets past the alignment checks and stops
+    # at the next one (nothing is launched on these fake addresses)
+    assert step(lib, rule=3, g=A + 4, B=9) == L.LA_ERR_SHAPE
+    assert step(lib, rule=5) == L.LA_ERR_UNSUPPORTED
 
 
 def scan(lib, rule=3, src=None, rs=None, dst=None, ws=None, n=2, cu=A, T=10, order=None, q=A, io=1, g=A, err=A):
@@ -148,15 +156,18 @@ def test_scan_host_errors(lib):
     assert scan(lib, cu=A + 2) == L.LA_ERR_ALIGN
     assert scan(lib, order=A + 1) == L.LA_ERR_ALIGN
     assert scan(lib, n=9) == L.LA_ERR_SHAPE
+    assert scan(lib, rule=4, g=None) == L.LA_ERR_NULL
+    assert scan(lib, rule=4, g=A + 8) == L.LA_ERR_ALIGN
 
 
 def test_chunked_scan_supported_set(lib):
     P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
 
-    def call(shape=(2, 4, 128, 128), io=1):
+    def call(shape=(2, 4, 128, 128), io=1, rule=3):
         dst = pool(shape=shape)
-        return lib.la_state_scan_chunked(3, None, None, ctypes.byref(dst), None, 2, P(A), 10, None, P(A), P(A), P(A),
-                                         io, P(A), P(A), 1.0, P(A), P(A), None)
+        return lib.la_state_scan_chunked(rule, None, None, ctypes.byref(dst), None, 2, P(A), 10, None, P(A), P(A),
+                                         P(A), io, P(A), P(A), 1.0, P(A), P(A), None)
+    assert call(rule=4) == L.LA_ERR_UNSUPPORTED  # kda: token-serial scan only
     assert call(shape=(2, 4, 64, 64)) == L.LA_ERR_UNSUPPORTED
     assert call(shape=(2, 4, 128, 64)) == L.LA_ERR_UNSUPPORTED
     assert call(io=0) == L.LA_ERR_UNSUPPORTED
@@ -185,6 +196,57 @@ def test_pool_host_errors(lib):
     assert lib.la_state_pool_zero(ctypes.byref(p), 1, P(A), None, None) == L.LA_ERR_NULL
     bad = pool(dtype=9)
     assert lib.la_state_pool_zero(ctypes.byref(bad), 1, P(A), P(A), None) == L.LA_ERR_UNSUPPORTED
+
+
+def test_q8_pools_host_side(lib):
+    """q8 pools: slot sizes of the layout (9.875 bits per value at 1/8 BF16 channels) and
+    the host-side errors of the entry points that take or refuse them."""
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+
+    def q8(shape=(2, 4, 128, 128), n_hp=16, mask=A, data=A, n=8):
+        return L.la_pool(ctypes.c_void_p(data), L.LA_Q8, n, L.la_shape(*shape), n_hp, P(mask))
+    assert lib.la_pool_slot_bytes(ctypes.byref(q8())) == 4 * (112 * 128 + 112 * 4 * 4 + 16 * 128 * 2)
+    assert lib.la_pool_slot_bytes(ctypes.byref(q8())) * 8 / (4 * 128 * 128) == 9.875
+    assert lib.la_pool_slot_bytes(ctypes.byref(q8(shape=(2, 4, 128, 64), n_hp=0))) == 4 * (128 * 64 + 128 * 2 * 4)
+    assert lib.la_pool_slot_bytes(ctypes.byref(pool(dtype=1))) == 4 * 128 * 128 * 2
+    assert lib.la_pool_slot_bytes(ctypes.byref(q8(shape=(2, 4, 16, 16)))) == 0     # no q8 tile of 16 x 16
+    assert lib.la_pool_slot_bytes(ctypes.byref(q8(n_hp=3))) == 0                   # odd
+    assert lib.la_pool_slot_bytes(ctypes.byref(q8(n_hp=34))) == 0                  # above d_k / 4
+    assert L.q8_tile_bytes(128, 128, 16) * 4 == lib.la_pool_slot_bytes(ctypes.byref(q8()))
+    assert step(lib, src=q8(mask=None), dst=q8(mask=None)) == L.LA_ERR_NULL
+    assert step(lib, src=q8(mask=A + 2), dst=q8(mask=A + 2)) == L.LA_ERR_ALIGN
+    assert step(lib, src=q8(shape=(2, 4, 16, 16)), dst=q8(shape=(2, 4, 16, 16))) == L.LA_ERR_UNSUPPORTED
+    assert step(lib, src=q8(n_hp=3), dst=q8(n_hp=3)) == L.LA_ERR_SHAPE
+    assert step(lib, src=q8(), dst=pool(dtype=1)) == L.LA_ERR_UNSUPPORTED        # formats differ
+    assert step(lib, src=q8(n_hp=16), dst=q8(n_hp=8)) == L.LA_ERR_SHAPE          # tile sizes differ
+    assert lib.la_state_step_qgroups(3, ctypes.byref(q8(shape=(4, 4, 128, 128))), None,
+                                     ctypes.byref(q8(shape=(4, 4, 128, 128))), None, 2, 8, P(A), P(A), P(A), 1,
+                                     P(A), P(A), 1.0, P(A), P(A), None) == L.LA_ERR_UNSUPPORTED
+    assert lib.la_state_scan_chunked(3, None, None, ctypes.byref(q8()), None, 2, P(A), 10, None, P(A), P(A), P(A), 1,
+                                     P(A), P(A), 1.0, P(A), P(A), None) == L.LA_ERR_UNSUPPORTED
+    assert lib.la_state_pool_encode(ctypes.byref(pool(dtype=1)), 2, P(A), P(A), P(A), None) == L.LA_ERR_UNSUPPORTED
+    assert lib.la_state_pool_decode(ctypes.byref(q8()), 2, None, P(A), P(A), None) == L.LA_ERR_NULL
+    assert lib.la_state_pool_decode(ctypes.byref(q8()), 2, P(A), P(A + 4), P(A), None) == L.LA_ERR_ALIGN
+    assert lib.la_state_pool_encode(ctypes.byref(q8()), 0, None, None, P(A), None) == L.LA_OK
+
+
+def test_conv_step_host_errors(lib):
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+
+    def call(width=4, wq=A, hist=A, src=None, B=4):
+        conv = L.la_conv(width, 1, 1, P(wq), P(A), P(A), P(hist), P(hist))
+        src = src or pool()
+        return lib.la_state_step_conv(3, ctypes.byref(src), None, ctypes.byref(src), None, B, ctypes.byref(conv),
+                                      P(A), P(A), P(A), 1, P(A), P(A), 1.0, P(A), P(A), None)
+    assert call(width=1) == L.LA_ERR_UNSUPPORTED
+    assert call(width=5) == L.LA_ERR_UNSUPPORTED
+    assert call(wq=None) == L.LA_ERR_NULL
+    assert call(hist=A + 8) == L.LA_ERR_ALIGN
+    assert call(B=0) == L.LA_OK
+    assert lib.la_state_step_conv(3, ctypes.byref(pool()), None, ctypes.byref(pool()), None, 4, None, P(A), P(A),
+                                  P(A), 1, P(A), P(A), 1.0, P(A), P(A), None) == L.LA_ERR_NULL
+    q8 = L.la_pool(ctypes.c_void_p(A), L.LA_Q8, 8, L.la_shape(2, 4, 128, 128), 16, P(A))
+    assert call(src=q8) == L.LA_ERR_UNSUPPORTED
 
 
 def test_check_slots(lib):

@@ -13,8 +13,9 @@ import torch
 import oracle
 from gated_deltanet_recurrent_la_b200 import lastate as L
 from gated_deltanet_recurrent_la_b200 import workloads as W
-from gpu_helpers import (BF16, F32, assert_close, check_step_against_oracle, dev, dname, gpu_scan, gpu_step,
-                         np64, oracle_scan, tolerances)
+from gpu_helpers import (BF16, F32, assert_close, check_step_against_oracle, dev, dname, gpu_scan, gpu_scan_qgroups,
+                         gpu_step, gpu_step_qgroups, np64, oracle_scan, oracle_scan_qgroups, oracle_step_qgroups,
+                         tolerances)
 
 pytestmark = pytest.mark.gpu
 
@@ -28,9 +29,9 @@ def _cuda():
     L.lib()
 
 
-# ---- the tiny workload: all four rules, as 64 decode steps and as one scan ------------
+# ---- the tiny workload: every rule, as 64 decode steps and as one scan ------------------
 
-@pytest.mark.parametrize("rule", W.RULES)
+@pytest.mark.parametrize("rule", W.ALL_RULES)
 def test_tiny_sequential_steps(rule):
     inp = W.tiny(rule)
     cu = inp.cu_seqlens.numpy()
@@ -49,7 +50,7 @@ def test_tiny_sequential_steps(rule):
         assert_close(np64(o), o_ref, 1e-4, f"{rule} o at step {t}")
 
 
-@pytest.mark.parametrize("rule", W.RULES)
+@pytest.mark.parametrize("rule", W.ALL_RULES)
 def test_tiny_scan(rule):
     inp = W.tiny(rule)
     S, o, err = gpu_scan(inp)
@@ -79,14 +80,9 @@ def test_mamba2_full():
 
 # ---- the full-size prefill workload, sampled ----------------------------------------------
 
-def test_prefill32_sampled():
-    inp = W.prefill32()
-    S, o, err = gpu_scan(inp)
-    assert err == 0
+def _check_sampled_units(inp, S, o, picks):
+    """(sequence, head) units of a full-size scan recomputed one by one by the oracle."""
     cu = inp.cu_seqlens.numpy()
-    lens = cu[1:] - cu[:-1]
-    order = np.argsort(lens)
-    picks = [(int(order[0]), 0), (int(order[0]), 31), (int(order[16]), 7), (int(order[-1]), 19)]
     tol_s, tol_o = tolerances(inp.state_dtype, inp.io_dtype)
     for s, h in picks:
         t0, t1 = int(cu[s]), int(cu[s + 1])
@@ -100,12 +96,22 @@ def test_prefill32_sampled():
     assert torch.isfinite(o.float()).all() and torch.isfinite(S.float()).all()
 
 
+def test_prefill32_sampled():
+    inp = W.prefill32()
+    S, o, err = gpu_scan(inp)
+    assert err == 0
+    cu = inp.cu_seqlens.numpy()
+    order = np.argsort(cu[1:] - cu[:-1])
+    _check_sampled_units(inp, S, o, [(int(order[0]), 0), (int(order[0]), 31), (int(order[16]), 7),
+                                     (int(order[-1]), 19)])
+
+
 # ---- every rule x tile shape x dtype, small batches -----------------------------------------
 
 @pytest.mark.parametrize("state", [F32, BF16], ids=["f32state", "bf16state"])
 @pytest.mark.parametrize("io", [F32, BF16], ids=["f32io", "bf16io"])
 @pytest.mark.parametrize("dk,dv", SHAPES, ids=[f"{a}x{b}" for a, b in SHAPES])
-@pytest.mark.parametrize("rule", W.RULES)
+@pytest.mark.parametrize("rule", W.ALL_RULES)
 def test_step_all_variants(rule, dk, dv, io, state):
     inp = W.step_inputs(B=5, n_qk_heads=2, n_v_heads=4, d_k=dk, d_v=dv, rule=rule, n_slots=11, state_dtype=state,
                         io_dtype=io, seed=dk + dv + len(rule), slot_map="perm", scale=0.9)
@@ -114,7 +120,7 @@ def test_step_all_variants(rule, dk, dv, io, state):
 
 @pytest.mark.parametrize("io", [F32, BF16], ids=["f32io", "bf16io"])
 @pytest.mark.parametrize("dk,dv", SHAPES, ids=[f"{a}x{b}" for a, b in SHAPES])
-@pytest.mark.parametrize("rule", W.RULES)
+@pytest.mark.parametrize("rule", W.ALL_RULES)
 def test_scan_all_variants(rule, dk, dv, io):
     inp = W.scan_inputs(lengths=[3, 37, 0, 1, 16, 17], n_qk_heads=2, n_v_heads=4, d_k=dk, d_v=dv, rule=rule,
                         state_dtype=BF16, io_dtype=io, seed=7 + dk, init="slots", init_dtype=F32, scale=1.1)
@@ -387,7 +393,7 @@ def _gpu_scan_ckpt(inp, every, ckpt_cu, ckpt_slots, n_dst, dst_dtype):
 
 
 @pytest.mark.parametrize("dst", [F32, BF16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("rule", W.RULES)
+@pytest.mark.parametrize("rule", W.ALL_RULES)
 def test_scan_checkpoints(rule, dst):
     lengths, every = [37, 8, 0, 64, 5, 16], 8
     inp = W.scan_inputs(lengths=lengths, n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128, rule=rule, io_dtype=BF16,
@@ -476,3 +482,139 @@ def test_chunked_prefill32_sampled():
         S_ref, o_ref, _ = oracle_scan(sub)
         assert_close(np64(S[s, h]), S_ref[0, 0], 2e-2, f"seq {s} head {h} final state")
         assert_close(np64(o[t0:t1, h]), o_ref[:, 0], 2e-2, f"seq {s} head {h} outputs")
+
+
+# ---- channel-wise gate (kda): the full-size workloads, special cases, the supported set ----
+
+def test_kda_decode64_full():
+    check_step_against_oracle(W.kda_decode64())
+
+
+def test_kda_prefill32_sampled():
+    inp = W.kda_prefill32()
+    S, o, err = gpu_scan(inp)
+    assert err == 0
+    cu = inp.cu_seqlens.numpy()
+    order = np.argsort(cu[1:] - cu[:-1])
+    _check_sampled_units(inp, S, o, [(int(order[0]), 5), (int(order[-1]), 30)])
+
+
+def test_kda_wide_gate_and_beta_ranges():
+    """alpha in [-1, 1] per channel and beta in [0, 2] are not clamped (decode and scan)."""
+    inp = W.step_inputs(B=7, n_qk_heads=1, n_v_heads=3, d_k=128, d_v=64, rule="kda", n_slots=7, state_dtype=F32,
+                        io_dtype=F32, g_mode="uniform_pm1", beta_mode="uniform_0_2", seed=51)
+    check_step_against_oracle(inp)
+    sc = W.scan_inputs(lengths=[60, 9], n_qk_heads=1, n_v_heads=3, d_k=64, d_v=64, rule="kda", state_dtype=F32,
+                       io_dtype=F32, g_mode="uniform_pm1", beta_mode="uniform_0_2", seed=52, init="slots",
+                       init_dtype=F32)
+    S, o, err = gpu_scan(sc)
+    S_ref, o_ref, _ = oracle_scan(sc)
+    assert err == 0
+    assert_close(np64(S), S_ref, 1e-4, "kda wide-range scan state")
+    assert_close(np64(o), o_ref, 1e-4, "kda wide-range scan outputs")
+
+
+def test_kda_equal_channels_matches_gated_delta():
+    """Every channel decaying by the same g: the kda kernels (decode and scan) agree with the
+    gated_delta kernels, a different code path, to FP32 precision."""
+    sc = W.scan_inputs(lengths=[33, 70], n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128, rule="gated_delta",
+                       state_dtype=F32, io_dtype=F32, seed=53, init="slots", init_dtype=F32)
+    kda = W.Inputs(**{**sc.__dict__, "rule": "kda", "g": sc.g[:, :, None].expand(-1, -1, 128).contiguous()})
+    S0, o0, e0 = gpu_scan(sc)
+    S1, o1, e1 = gpu_scan(kda)
+    assert e0 == e1 == 0
+    assert_close(np64(S1), np64(S0), 1e-4, "scan state")
+    assert_close(np64(o1), np64(o0), 1e-4, "scan outputs")
+    st = W.step_inputs(B=6, n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128, rule="gated_delta", n_slots=9,
+                       state_dtype=F32, io_dtype=F32, seed=54)
+    st_kda = W.Inputs(**{**st.__dict__, "rule": "kda", "g": st.g[:, :, None].expand(-1, -1, 128).contiguous()})
+    a0, p0, e0 = gpu_step(st)
+    a1, p1, e1 = gpu_step(st_kda)
+    assert e0 == e1 == 0
+    assert_close(np64(a1), np64(a0), 1e-4, "step state")
+    assert_close(np64(p1), np64(p0), 1e-4, "step outputs")
+
+
+def test_kda_checkpointed_scan_and_chunked_refusal():
+    lengths, every = [19, 40, 3], 8
+    inp = W.scan_inputs(lengths=lengths, n_qk_heads=1, n_v_heads=2, d_k=128, d_v=128, rule="kda", io_dtype=BF16,
+                        seed=55, init="slots", init_dtype=F32)
+    ckpt_cu, ckpt_slots = _ckpt_layout(lengths, every, len(lengths))
+    n_dst = len(lengths) + int(ckpt_cu[-1])
+    S, o, err = _gpu_scan_ckpt(inp, every, ckpt_cu, ckpt_slots, n_dst, F32)
+    assert err == 0
+    S_ref, o_ref, e = oracle.scan("kda", 1, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k), np64(inp.v),
+                                  np64(inp.g), np64(inp.beta), inp.scale, src_pool=np64(inp.pool),
+                                  read_slot=inp.read_slot.numpy(), dst_pool=np.zeros((n_dst, 2, 128, 128)),
+                                  dst_dtype="f32", io_dtype="bf16", ckpt_every=every, ckpt_cu=ckpt_cu,
+                                  ckpt_slots=ckpt_slots)
+    assert e == 0
+    assert_close(np64(S), S_ref, 1e-4, "kda checkpoints and final states")
+    assert_close(np64(o), o_ref, 2e-2, "kda outputs")
+    with pytest.raises(L.LAError):
+        _gpu_scan_chunked(inp, F32)
+
+
+# ---- query-group direction (ONNX: query heads sharing a KV head and its state) ---------------
+
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
+@pytest.mark.parametrize("state,io", [(F32, F32), (BF16, BF16), (BF16, F32)], ids=["f32", "bf16", "bf16state"])
+@pytest.mark.parametrize("dk,dv", [(16, 16), (128, 64), (128, 128)], ids=["16x16", "128x64", "128x128"])
+@pytest.mark.parametrize("rule", ["linear", "gated_delta", "kda"])
+def test_qgroups_step(rule, dk, dv, state, io, group):
+    inp = W.step_inputs(B=5, n_qk_heads=3, n_v_heads=3, d_k=dk, d_v=dv, rule=rule, n_slots=9, state_dtype=state,
+                        io_dtype=io, seed=60 + group, slot_map="perm", scale=0.9, n_q_heads=3 * group)
+    after, o, err = gpu_step_qgroups(inp)
+    assert err == 0
+    ref_pool, o_ref, e = oracle_step_qgroups(inp)
+    assert e == 0
+    tol_s, tol_o = tolerances(state, io)
+    assert_close(np64(after), ref_pool, tol_s, f"{rule} group {group}: pool after the step")
+    assert_close(np64(o), o_ref, tol_o, f"{rule} group {group}: outputs")
+
+
+@pytest.mark.parametrize("group", [2, 8])
+@pytest.mark.parametrize("io", [F32, BF16], ids=["f32io", "bf16io"])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128)], ids=["64x64", "128x128"])
+@pytest.mark.parametrize("rule", ["gated", "gated_delta", "kda"])
+def test_qgroups_scan(rule, dk, dv, io, group):
+    inp = W.scan_inputs(lengths=[3, 21, 0, 9], n_qk_heads=2, n_v_heads=2, d_k=dk, d_v=dv, rule=rule, state_dtype=BF16,
+                        io_dtype=io, seed=70 + group, init="slots", init_dtype=F32, scale=1.1, n_q_heads=2 * group)
+    for dst in (F32, BF16):
+        S, o, err = gpu_scan_qgroups(inp, dst)
+        assert err == 0
+        S_ref, o_ref, e = oracle_scan_qgroups(inp, dst)
+        assert e == 0
+        tol_s, tol_o = tolerances(dst, io)
+        assert_close(np64(S), S_ref, tol_s, f"{rule} group {group}: final states ({dst})")
+        assert_close(np64(o), o_ref, tol_o, f"{rule} group {group}: outputs")
+
+
+def test_qgroups_first_query_matches_default_direction_bitwise():
+    """With one query per state head the query-group kernels give the default kernels' bits."""
+    st = W.step_inputs(B=4, n_qk_heads=4, n_v_heads=4, d_k=128, d_v=128, seed=80, slot_map="perm", n_slots=6,
+                       n_q_heads=4)
+    a0, o0, e0 = gpu_step(st)
+    a1, o1, e1 = gpu_step_qgroups(st)
+    assert e0 == e1 == 0 and torch.equal(a0, a1) and torch.equal(o0, o1)
+    sc = W.scan_inputs(lengths=[40, 17], n_qk_heads=2, n_v_heads=2, d_k=128, d_v=128, seed=81, n_q_heads=2)
+    S0, o0, e0 = gpu_scan(sc)
+    S1, o1, e1 = gpu_scan_qgroups(sc)
+    assert e0 == e1 == 0 and torch.equal(S0, S1) and torch.equal(o0, o1)
+
+
+def test_qgroups_decode_full():
+    check = W.qgroup_decode256()
+    after, o, err = gpu_step_qgroups(check)
+    assert err == 0
+    rows = torch.arange(0, 256, 37)  # sampled requests recomputed by the oracle (dense, gathered tiles)
+    sub = W.Inputs(**{**check.__dict__, "q": check.q[rows], "k": check.k[rows], "v": check.v[rows],
+                      "g": check.g[rows], "beta": check.beta[rows], "pool": check.pool[check.read_slot[rows].long()],
+                      "read_slot": None, "write_slot": None})
+    ref_states, o_ref, e = oracle_step_qgroups(sub)
+    assert e == 0
+    ws = check.write_slot[rows].long()
+    assert_close(np64(after[ws]), ref_states, 2e-2, "sampled states")
+    assert_close(np64(o[rows]), o_ref, 2e-2, "sampled outputs")
+    untouched = np.setdiff1d(np.arange(check.pool.shape[0]), check.write_slot.numpy())
+    assert torch.equal(after[untouched].view(torch.int16), check.pool[untouched].view(torch.int16))
