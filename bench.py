@@ -121,6 +121,7 @@ def kernel_source_hash(files):
 KERNEL_SOURCES = {
     "step": ["la_step.cuh", "la_device.cuh"],
     "scan": ["la_scan.cuh", "la_device.cuh"],
+    "chunk": ["la_chunk.cuh", "la_device.cuh"],
     "pool": ["la_pool.cu"],
 }
 

@@ -172,7 +172,7 @@ static la_status step_impl(la_rule rule, const la_pool* src, const int32_t* read
     if (q8) return LA_ERR_UNSUPPORTED;
     if (conv->width < 2 || conv->width > la::kMaxConvWidth) return LA_ERR_UNSUPPORTED;
     if (!conv->w_q || !conv->w_k || !conv->w_v || !conv->hist_src || !conv->hist_dst) return LA_ERR_NULL;
-    if (!aligned(conv->w_q, 4) || !aligned(conv->w_k, 4) || !aligned(conv->w_v, 4) || !aligned(conv->hist_src, 16) ||
+    if (!aligned(conv->w_q, 16) || !aligned(conv->w_k, 16) || !aligned(conv->w_v, 16) || !aligned(conv->hist_src, 16) ||
         !aligned(conv->hist_dst, 16))
       return LA_ERR_ALIGN;
   }

@@ -387,72 +387,39 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
             if (warp >= 4) st_bf16x2(smem, swz(kOffP, r, j, kRow64) + 4 * t4, v2[0], v2[1]);
           }
         }
-        // diagonal 16 x 16 block `warp` of T = (I + L)^-1, from this warp's own rows of L
-        // (overlapping the Q K^T of warps 4-7), in two levels of 8: lanes 0-7 / 8-15 solve
-        // the upper-left / lower-right 8 x 8 blocks by forward substitution (one column per
-        // lane), then lanes 0-7 form the lower-left block T21 = -T22 (L21 T11).  Tw =
-        // T diag(b gamma) and Tu = T diag(b) follow in BF16.
-        if (kDelta && warp < 4) {
-          __syncwarp();
-          const int b0 = 16 * warp;
-          const int c8 = lane & 7, o = b0 + 8 * ((lane >> 3) & 1);
-          float col[8];
-#pragma unroll
-          for (int r = 0; r < 8; ++r) {
-            float x = (r == c8) ? 1.0f : 0.0f;
-#pragma unroll
-            for (int j = 0; j < r; ++j) x -= sL[(o + r) * kLs + o + j] * col[j];
-            col[r] = (r < c8) ? 0.0f : x;
-          }
-          if (lane < 16) {
-#pragma unroll
-            for (int r = 0; r < 8; ++r) sT[(o + r) * kTs + o + c8] = col[r];
-          }
-          if (lane >= 8 && lane < 16) {
-#pragma unroll
-            for (int r = 0; r < 8; ++r) sT[(b0 + r) * kTs + b0 + 8 + c8] = 0.0f;
-          }
-          __syncwarp();
-          if (lane < 8) {
-            float xv[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float a = 0.0f;
-#pragma unroll
-              for (int k = 0; k < 8; ++k) a = fmaf(sL[(b0 + 8 + i) * kLs + b0 + k], col[k], a);
-              xv[i] = a;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float a = 0.0f;
-#pragma unroll
-              for (int k = 0; k < 8; ++k) a = fmaf(sT[(b0 + 8 + i) * kTs + b0 + 8 + k], xv[k], a);
-              sT[(b0 + 8 + i) * kTs + b0 + c8] = -a;
-            }
-          }
-          __syncwarp();
-          const int c = lane & 15, sc = b0 + c;
-          const float fw = sBt[sc] * sGm[sc], fu = sBt[sc];
-#pragma unroll
-          for (int r = 0; r < 16; ++r) {
-            const float tv = sT[(b0 + r) * kTs + sc];
-            // pairs of columns (c, c + 1) into Tw / Tu
-            const float nw = __shfl_down_sync(0xffffffffu, tv * fw, 1);
-            const float nu = __shfl_down_sync(0xffffffffu, tv * fu, 1);
-            if (lane < 16 && (c & 1) == 0) {
-              const uint32_t off = swz(kOffTw, b0 + r, sc >> 3, kRow64) + 2 * (sc & 7);
-              st_bf16x2(smem, off, tv * fw, nw);
-              st_bf16x2(smem, off - kOffTw + kOffTu, tv * fu, nu);
-            }
-          }
-        }
       }
       __syncthreads();
 
-      // ---- step 2 (delta rules): the off-diagonal 16 x 16 blocks of T = (I + L)^-1 (the
-      //      diagonal ones came with step 1), written as FP32 (for the block recursion) and
-      //      as Tw = T diag(b gamma), Tu = T diag(b) (BF16, swizzled)
+      // ---- step 2 (delta rules): T = (I + L)^-1 by 16 x 16 blocks, written as FP32 (for the
+      //      block recursion) and as Tw = T diag(b gamma), Tu = T diag(b) (BF16, swizzled)
       if (kDelta) {
+        // diagonal blocks: forward substitution, lane c < 16 of warp b owns column c
+        if (warp < 4) {
+          const int b0 = 16 * warp, c = lane & 15;
+          float col[16];
+#pragma unroll
+          for (int r = 0; r < 16; ++r) {
+            float x = (r == c) ? 1.0f : 0.0f;
+#pragma unroll
+            for (int j = 0; j < r; ++j) x -= sL[(b0 + r) * kLs + b0 + j] * col[j];
+            col[r] = (r < c) ? 0.0f : x;
+          }
+          const int sc = b0 + c;
+          const float fw = sBt[sc] * sGm[sc], fu = sBt[sc];
+#pragma unroll
+          for (int r = 0; r < 16; ++r) {
+            if (lane < 16) sT[(b0 + r) * kTs + sc] = col[r];
+            // pairs of columns (c, c + 1) into Tw / Tu
+            const float nw = __shfl_down_sync(0xffffffffu, col[r] * fw, 1);
+            const float nu = __shfl_down_sync(0xffffffffu, col[r] * fu, 1);
+            if (lane < 16 && (c & 1) == 0) {
+              const uint32_t off = swz(kOffTw, b0 + r, sc >> 3, kRow64) + 2 * (sc & 7);
+              st_bf16x2(smem, off, col[r] * fw, nw);
+              st_bf16x2(smem, off - kOffTw + kOffTu, col[r] * fu, nu);
+            }
+          }
+        }
+        __syncthreads();
         // block row bi: T_{bi,j} = -T_{bi,bi} sum_{k=j}^{bi-1} L_{bi,k} T_{k,j}, warp j < bi
 #pragma unroll 1
         for (int bi = 1; bi < 4; ++bi) {

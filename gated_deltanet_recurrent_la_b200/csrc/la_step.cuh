@@ -97,14 +97,18 @@ struct StepCfg {
   static constexpr int kOffA = kOffV + kVBytes;
   static constexpr int kOffHist = kOffA + kGBytes;
   static constexpr int kHistBytes = CONV ? (2 * DK + DV) * (kMaxConvWidth - 1) * (int)sizeof(IT) : 0;
-  static constexpr int kCopyBytes = kOffHist + kHistBytes;  // with all QMAX query rows, widest history
+  static constexpr int kOffConvW = kOffHist + kHistBytes;   // the tile's weights [q | k | v channels][W]
+  static constexpr int kConvWBytes = CONV ? (2 * DK + DV) * kMaxConvWidth * 4 : 0;
+  static constexpr int kCopyBytes = kOffConvW + kConvWBytes;  // with all QMAX query rows, widest convolution
   static constexpr int kStageBytes = round_up(kCopyBytes, 128);
   static constexpr int kStages = cmax(2, cmin(12, (204 * 1024) / kStageBytes));
   static constexpr int kOffMeta = kStages * kStageBytes;
   static constexpr int kOffBars = round_up(kOffMeta + kStages * (int)sizeof(StepMeta), 8);
   static constexpr int kOffScratch = round_up(kOffBars + 2 * kStages * 8, 16);
-  static constexpr int kScratchFloats = CONV ? 2 * DK + DV : 0;  // per consumer warp: q, k, v
-  static constexpr int kSmem = kOffScratch + kConsumerWarps * kScratchFloats * 4;
+  // CONV, per team (the warps of one tile): post-convolution q | k | v, each warp's partial
+  // sums of q^2 and k^2, each warp's arrival flag
+  static constexpr int kScratchFloats = CONV ? 2 * DK + DV + 3 * kWPT : 0;
+  static constexpr int kSmem = kOffScratch + kTeams * kScratchFloats * 4;
 
   static_assert(kNCH >= 1 && kNCH <= 32 && (32 % kNCH) == 0, "strip row must map onto a power-of-two lane group");
   static_assert(kRL >= 1 && DK % kRG == 0, "rows must split evenly over the row blocks");
@@ -114,67 +118,75 @@ struct StepCfg {
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
-// The short causal convolution ahead of the step, for one tile, by one consumer warp: the
-// post-convolution q, k (channels of the tile's q/k head) and v (the tile's head) go to the
-// warp's FP32 scratch [q | k | v]; channel c is y = sum_j w[c][j] x_{t-W+1+j} over the W - 1
-// staged history inputs and the current input, then SiLU when asked, then q and k scaled
-// to unit length when asked.  Warp `part` of the tile writes every kWPT-th 32-channel block
-// of the new history (the last W - 1 inputs) to write slot `ws` (skipped when ws < 0).
+// The short causal convolution ahead of the step, for one tile, by the WPT warps of its
+// team, each taking every WPT-th 32-channel block: channel c is y = sum_j w[c][j]
+// x_{t-W+1+j} over the W - 1 staged history inputs and the current input (weights staged
+// with the tile), then SiLU when asked; q and k are then scaled to unit length when asked
+// (the team's partial sums of squares meet in shared memory).  The results land in the
+// team's FP32 scratch [q | k | v] for all of the team's warps.  Each warp writes its
+// channels' new histories (the last W - 1 inputs) to write slot `ws` (skipped when ws < 0).
+// Every warp of the team passes the team barrier (id bar) twice here.
 template <int DK, int DV, typename IT, int WPT>
 __device__ __forceinline__ void conv_operands(const StepParams& p, const unsigned char* xq_s,
                                               const unsigned char* xk_s, const unsigned char* xv_s,
-                                              const unsigned char* hist_s, int h, int H, int ws, int part, int lane,
-                                              float* scr) {
+                                              const unsigned char* hist_s, const float* w_s, int h, int H, int ws,
+                                              int part, int lane, float* scr, uint32_t bar) {
   constexpr int CH = 2 * DK + DV;
+  constexpr int kIters = (CH + 32 * WPT - 1) / (32 * WPT);
   const int W = p.conv_w;
-  const int hq = h / (H / p.n_qk_heads);
   const IT* xq = reinterpret_cast<const IT*>(xq_s);
   const IT* xk = reinterpret_cast<const IT*>(xk_s);
   const IT* xv = reinterpret_cast<const IT*>(xv_s);
   const IT* hist = reinterpret_cast<const IT*>(hist_s);
+  float* partial = scr + CH;  // [WPT][2]
   float sq = 0.0f, sk = 0.0f;
-  // all of a lane's channels at once (unrolled, widths padded to kMaxConvWidth) so the
-  // weight and history loads are in flight together
 #pragma unroll
-  for (int it = 0; it < (CH + 31) / 32; ++it) {
-    const int c = lane + 32 * it;
+  for (int it = 0; it < kIters; ++it) {
+    const int c = (part + WPT * it) * 32 + lane;
     if (c < CH) {
-      const float* w = c < DK ? p.conv_wq + ((int64_t)hq * DK + c) * W
-                     : c < 2 * DK ? p.conv_wk + ((int64_t)hq * DK + (c - DK)) * W
-                                  : p.conv_wv + ((int64_t)h * DV + (c - 2 * DK)) * W;
+      const float* w = w_s + c * W;  // staged weights: q channels, then k, then v
       const float x = io_load(c < DK ? xq + c : c < 2 * DK ? xk + (c - DK) : xv + (c - 2 * DK));
-      float y = __ldg(w + W - 1) * x;
+      float y = w[W - 1] * x;
 #pragma unroll
       for (int j = 0; j < kMaxConvWidth - 1; ++j)
-        if (j < W - 1) y = fmaf(__ldg(w + j), io_load(hist + c * (W - 1) + j), y);
-      if (p.conv_act) y = y / (1.0f + __expf(-y));
+        if (j < W - 1) y = fmaf(w[j], io_load(hist + c * (W - 1) + j), y);
+      if (p.conv_act) y = __fdividef(y, 1.0f + __expf(-y));
       scr[c] = y;
       if (c < DK) sq = fmaf(y, y, sq);
       else if (c < 2 * DK) sk = fmaf(y, y, sk);
+      if (ws >= 0) {
+        IT* hd = static_cast<IT*>(p.conv_dst) + ((int64_t)ws * H + h) * CH * (W - 1);
+        for (int j = 0; j < W - 2; ++j) hd[c * (W - 1) + j] = hist[c * (W - 1) + j + 1];
+        hd[c * (W - 1) + W - 2] = c < DK ? xq[c] : c < 2 * DK ? xk[c - DK] : xv[c - 2 * DK];
+      }
     }
   }
-  if (p.conv_l2norm) {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      sq += __shfl_xor_sync(0xffffffffu, sq, off);
-      sk += __shfl_xor_sync(0xffffffffu, sk, off);
+  for (int off = 16; off > 0; off >>= 1) {
+    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    sk += __shfl_xor_sync(0xffffffffu, sk, off);
+  }
+  if (lane == 0) {
+    partial[2 * part] = sq;
+    partial[2 * part + 1] = sk;
+  }
+  named_bar_sync(bar, WPT * 32);
+  if (p.conv_l2norm) {
+    sq = 0.0f;
+    sk = 0.0f;
+#pragma unroll
+    for (int w = 0; w < WPT; ++w) {
+      sq += partial[2 * w];
+      sk += partial[2 * w + 1];
     }
     const float rq = rsqrtf(sq + 1e-6f), rk = rsqrtf(sk + 1e-6f);
-    __syncwarp();
 #pragma unroll
-    for (int it = 0; it < (2 * DK + 31) / 32; ++it) {
-      const int c = lane + 32 * it;
+    for (int it = 0; it < kIters; ++it) {
+      const int c = (part + WPT * it) * 32 + lane;
       if (c < 2 * DK) scr[c] *= c < DK ? rq : rk;
     }
   }
-  if (ws >= 0) {
-    IT* hd = static_cast<IT*>(p.conv_dst) + ((int64_t)ws * H + h) * CH * (W - 1);
-    for (int c = part * 32 + lane; c < CH; c += WPT * 32) {
-      for (int j = 0; j < W - 2; ++j) hd[c * (W - 1) + j] = hist[c * (W - 1) + j + 1];
-      hd[c * (W - 1) + W - 2] = c < DK ? xq[c] : c < 2 * DK ? xk[c - DK] : xv[c - 2 * DK];
-    }
-  }
-  __syncwarp();
+  named_bar_sync(bar, WPT * 32);
 }
 
 // QGRP: the query-group direction of the ONNX operator -- k has one head per state head
@@ -283,17 +295,25 @@ __global__ void __launch_bounds__(
               // query rows: the tile's q/k head, or its qg consecutive query heads
               const int64_t qrow = QGRP ? t * qg : (int64_t)b * p.n_qk_heads + hq;
               const int hist_bytes = CONV ? (2 * DK + DV) * (p.conv_w - 1) * (int)sizeof(IT) : 0;
+              const int wbytes = CONV ? (2 * DK + DV) * p.conv_w * 4 : 0;
               mbar_arrive_expect_tx(&full[stage],
-                                    C::kOffHist - C::kOffK + tile_bytes + qg * C::kQKBytes + hist_bytes);
+                                    C::kOffHist - C::kOffK + tile_bytes + qg * C::kQKBytes + hist_bytes + wbytes);
               bulk_g2s_hint(sb, src + ((int64_t)rs_j * H + h) * tile_bytes, tile_bytes, &full[stage], pol_stream);
               bulk_g2s(sb + C::kTileBytes, q + qrow * DK, qg * C::kQKBytes, &full[stage]);
               bulk_g2s(sb + C::kOffK, k + ((int64_t)b * p.n_qk_heads + hq) * DK, C::kQKBytes, &full[stage]);
               bulk_g2s(sb + C::kOffV, v + t * DV, C::kVBytes, &full[stage]);
               if (CHG) bulk_g2s(sb + C::kOffA, p.g + t * DK, C::kGBytes, &full[stage]);
-              if (CONV)
+              if (CONV) {
                 bulk_g2s(sb + C::kOffHist,
                          static_cast<const unsigned char*>(p.conv_src) + ((int64_t)rs_j * H + h) * hist_bytes,
                          hist_bytes, &full[stage]);
+                // the weights of the tile's q/k head and head (the same for every request)
+                const int W = p.conv_w;
+                bulk_g2s(sb + C::kOffConvW, p.conv_wq + (int64_t)hq * DK * W, DK * W * 4, &full[stage]);
+                bulk_g2s(sb + C::kOffConvW + DK * W * 4, p.conv_wk + (int64_t)hq * DK * W, DK * W * 4, &full[stage]);
+                bulk_g2s(sb + C::kOffConvW + 2 * DK * W * 4, p.conv_wv + (int64_t)h * DV * W, DV * W * 4,
+                         &full[stage]);
+              }
             } else {
               if (!rs_ok || !ws_ok) report(p.err, (rs_ok ? 0u : LA_DEVERR_READ_SLOT) | (ws_ok ? 0u : LA_DEVERR_WRITE_SLOT));
               mbar_arrive(&full[stage]);
@@ -341,7 +361,20 @@ __global__ void __launch_bounds__(
     const int stage = (int)(it % C::kStages);
     const uint32_t round = (uint32_t)(it / C::kStages);
     const bool arrived = mbar_wait(&full[stage], round & 1u);
-    if (!__all_sync(0xffffffffu, arrived)) {
+    bool ok = __all_sync(0xffffffffu, arrived);
+    float* scr = nullptr;
+    if constexpr (CONV) {
+      // the team's warps meet at barriers inside the convolution, so they take the
+      // (bounded) arrival decision together: each posts its flag, all read all flags.
+      // This barrier also orders this tile's scratch writes after the previous tile's reads.
+      scr = reinterpret_cast<float*>(smem + C::kOffScratch) + team * C::kScratchFloats;
+      float* flags = scr + 2 * DK + DV + 2 * C::kWPT;
+      if (lane == 0) flags[part] = ok ? 1.0f : 0.0f;
+      named_bar_sync(1 + team, C::kWPT * 32);
+#pragma unroll
+      for (int w = 0; w < C::kWPT; ++w) ok = ok && flags[w] != 0.0f;
+    }
+    if (!ok) {
       if (lane == 0) report(p.err, LA_DEVERR_TIMEOUT);
       return;
     }
@@ -353,10 +386,10 @@ __global__ void __launch_bounds__(
     const OT* ks;
     const OT* vs;
     if constexpr (CONV) {
-      float* scr = reinterpret_cast<float*>(smem + C::kOffScratch) + warp * C::kScratchFloats;
       conv_operands<DK, DV, IT, C::kWPT>(p, sb + C::kTileBytes, sb + C::kOffK, sb + C::kOffV, sb + C::kOffHist,
+                                         reinterpret_cast<const float*>(sb + C::kOffConvW),
                                          (int)((blockIdx.x + it * gridDim.x) % H), H, m.valid ? m.ws : -1, part,
-                                         lane, scr);
+                                         lane, scr, 1 + team);
       qs = scr;
       ks = scr + DK;
       vs = scr + 2 * DK;

@@ -251,7 +251,8 @@ typedef struct {
     int32_t width;          /* W, 2 <= W <= 4 */
     int32_t activation;     /* 0: none, 1: SiLU */
     int32_t qk_l2norm;      /* 1: q and k scaled to unit length per head after the convolution */
-    const float *w_q;       /* device float32 [H_qk][d_k][W] (w[c][W - 1] multiplies the newest input) */
+    const float *w_q;       /* device float32 [H_qk][d_k][W] (w[c][W - 1] multiplies the newest
+                               input); 16-byte aligned, like w_k and w_v */
     const float *w_k;       /* device float32 [H_qk][d_k][W] */
     const float *w_v;       /* device float32 [H_v][d_v][W] */
     const void *hist_src;   /* device, io dtype [src n_slots][H_v][2 d_k + d_v][W - 1] (q, k, v
