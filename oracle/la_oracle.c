@@ -718,6 +718,52 @@ int lao_scan_qgroups(int rule, int n_q_heads, int n_v_heads, int dk, int dv,
                      g, beta, scale, o, 0, NULL, NULL, NULL);
 }
 
+/* Scan with the convolution ahead of every token: each (sequence, head) history starts
+ * from conv_src at read_slot[s] (zero when read_slot is NULL), runs through the sequence's
+ * tokens, and the history after its last token goes to conv_dst at write_slot[s] (slot s
+ * when NULL); an empty sequence passes its history through unchanged.  Histories have
+ * src_slots / dst_slots slots like the pools.  Then the scan of lao_scan with one q/k row
+ * per state head. */
+int lao_scan_conv(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+                  const double *src_pool, int src_slots, const int *read_slot,
+                  double *dst_pool, int dst_slots, int dst_dtype, const int *write_slot,
+                  int n_seqs, const int *cu_seqlens, int total_tokens,
+                  const double *xq, const double *xk, const double *xv, int io_dtype,
+                  const double *g, const double *beta, double scale, double *o,
+                  int W, int act, int l2norm, const double *wq, const double *wk, const double *wv,
+                  const double *conv_src, double *conv_dst)
+{
+    const size_t C = (size_t)(2 * dk + dv) * (W - 1);
+    const size_t cslot = (size_t)n_v_heads * C;
+    const size_t T = total_tokens > 0 ? (size_t)total_tokens : 1;
+    double *q = (double *)calloc(T * n_v_heads * dk, sizeof(double));
+    double *k = (double *)calloc(T * n_v_heads * dk, sizeof(double));
+    double *v = (double *)calloc(T * n_v_heads * dv, sizeof(double));
+    double *hist = (double *)calloc(cslot + 1, sizeof(double));
+    double *hout = (double *)calloc(cslot + 1, sizeof(double));
+    if (!q || !k || !v || !hist || !hout) { free(q); free(k); free(v); free(hist); free(hout); return -1; }
+    for (int s = 0; s < n_seqs; ++s) {
+        const int t0 = cu_seqlens[s], t1 = cu_seqlens[s + 1];
+        const int rs = read_slot ? read_slot[s] : 0, ws = write_slot ? write_slot[s] : s;
+        if (t0 < 0 || t1 < t0 || t1 > total_tokens) continue;             /* reported by the scan */
+        if ((read_slot && (rs < 0 || rs >= src_slots)) || ws < 0 || ws >= dst_slots) continue;
+        if (read_slot) memcpy(hist, conv_src + (size_t)rs * cslot, sizeof(double) * cslot);
+        else memset(hist, 0, sizeof(double) * cslot);
+        for (int t = t0; t < t1; ++t) {
+            lao_conv(n_qk_heads, n_v_heads, dk, dv, W, act, l2norm, 1, xq + (size_t)t * n_qk_heads * dk,
+                     xk + (size_t)t * n_qk_heads * dk, xv + (size_t)t * n_v_heads * dv, wq, wk, wv, hist, hout,
+                     q + (size_t)t * n_v_heads * dk, k + (size_t)t * n_v_heads * dk, v + (size_t)t * n_v_heads * dv);
+            memcpy(hist, hout, sizeof(double) * cslot);
+        }
+        memcpy(conv_dst + (size_t)ws * cslot, hist, sizeof(double) * cslot);
+    }
+    const int err = scan_impl(rule, n_v_heads, n_v_heads, 0, dk, dv, src_pool, src_slots, read_slot, dst_pool,
+                              dst_slots, dst_dtype, write_slot, n_seqs, cu_seqlens, total_tokens, q, k, v, io_dtype,
+                              g, beta, scale, o, 0, NULL, NULL, NULL);
+    free(q); free(k); free(v); free(hist); free(hout);
+    return err;
+}
+
 /* ---- slot pool: whole-slot byte copies ------------------------------------------ */
 /* Checkpoints and snapshots ("Recurrent state" glossary, Why it matters; "Seven
  * Architectures", ONNX section on saving and restoring state snapshots) are plain byte

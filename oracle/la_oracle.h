@@ -95,6 +95,15 @@ int lao_step_conv(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
                   int W, int act, int l2norm, const double *wq, const double *wk, const double *wv,
                   const double *conv_src, double *conv_dst);
 
+int lao_scan_conv(int rule, int n_qk_heads, int n_v_heads, int dk, int dv,
+                  const double *src_pool, int src_slots, const int *read_slot,
+                  double *dst_pool, int dst_slots, int dst_dtype, const int *write_slot,
+                  int n_seqs, const int *cu_seqlens, int total_tokens,
+                  const double *xq, const double *xk, const double *xv, int io_dtype,
+                  const double *g, const double *beta, double scale, double *o,
+                  int W, int act, int l2norm, const double *wq, const double *wk, const double *wv,
+                  const double *conv_src, double *conv_dst);
+
 int lao_pool_copy(unsigned char *pool, size_t slot_bytes, int n_slots, int n,
                   const int *src_slots, const int *dst_slots);
 int lao_pool_gather(const unsigned char *pool, size_t slot_bytes, int n_slots, int n,

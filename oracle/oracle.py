@@ -52,6 +52,8 @@ def lib():
         _lib.lao_step_conv.argtypes = [i, i, i, i, i, p, i, p, i, i, p, p, i, p, p, p, i, p, p, d, p,
                                        i, i, i, p, p, p, p, p]
         _lib.lao_step_conv.restype = i
+        _lib.lao_scan_conv.argtypes = _lib.lao_scan.argtypes + [i, i, i, p, p, p, p, p]
+        _lib.lao_scan_conv.restype = i
         _lib.lao_step_qgroups.argtypes = _lib.lao_step.argtypes
         _lib.lao_step_qgroups.restype = i
         _lib.lao_scan_qgroups.argtypes = _lib.lao_scan.argtypes
@@ -294,6 +296,36 @@ def step_conv(rule, n_qk_heads, src_pool, xq, xk, xv, g, beta, scale, wq, wk, wv
     return dst, cdst, o, err
 
 
+def scan_conv(rule, n_qk_heads, cu_seqlens, xq, xk, xv, g, beta, scale, wq, wk, wv, *, act=0, l2norm=0,
+              conv_src=None, src_pool=None, read_slot=None, dst_pool=None, conv_dst=None, write_slot=None,
+              dst_dtype="f64", io_dtype="f64"):
+    """Token-serial scan with the convolution ahead of every token (see la_oracle.c).
+    conv_src: histories [slots, H_v, 2 d_k + d_v, W - 1] read at read_slot (zeros when
+    read_slot is None).  Returns (dst_pool, conv_dst, o, err_bits)."""
+    cu = _i32(cu_seqlens)
+    n_seqs = cu.shape[0] - 1
+    xq, xk, xv, wq, wk, wv = (_f64(a) for a in (xq, xk, xv, wq, wk, wv))
+    T, _, dk = xq.shape
+    hv, dv = xv.shape[1], xv.shape[2]
+    W = wq.shape[2]
+    if dst_pool is None:
+        dst_pool = np.zeros((n_seqs, hv, dk, dv))
+    if conv_dst is None:
+        conv_dst = np.zeros((dst_pool.shape[0], hv, 2 * dk + dv, W - 1))
+    src = None if src_pool is None else _f64(src_pool)
+    csrc = np.zeros((1, hv, 2 * dk + dv, W - 1)) if conv_src is None else _f64(conv_src)
+    n_src = 0 if src is None else src.shape[0]
+    g = None if g is None else _f64(g)
+    beta = None if beta is None else _f64(beta)
+    o = np.zeros((T, hv, dv))
+    err = lib().lao_scan_conv(RULES[rule], n_qk_heads, hv, dk, dv, _ptr(src), n_src, _ptr(_i32(read_slot)),
+                              _ptr(dst_pool), dst_pool.shape[0], DTYPES[dst_dtype], _ptr(_i32(write_slot)), n_seqs,
+                              _ptr(cu), T, _ptr(xq), _ptr(xk), _ptr(xv), DTYPES[io_dtype], _ptr(g), _ptr(beta),
+                              float(scale), _ptr(o), W, int(act), int(l2norm), _ptr(wq), _ptr(wk), _ptr(wv),
+                              _ptr(csrc), _ptr(conv_dst))
+    return dst_pool, conv_dst, o, err
+
+
 def readout_rearranged(rule, n_qk_heads, state, q, k, v, g=None, beta=None, scale=1.0):
     """o of one decode step in the rearranged form; state [B, H_v, d_k, d_v] (dense)."""
     S = _f64(state)
@@ -383,7 +415,7 @@ def set_threads(n):
 __all__ = ["round_bf16", "round_to", "step", "readout_rearranged", "scan", "pool_copy",
            "pool_gather", "pool_scatter", "pool_zero", "num_threads", "set_threads", "RULES", "DTYPES",
            "step_qgroups", "scan_qgroups", "q8_tile_bytes", "q8_encode", "q8_decode", "step_q8", "scan_q8", "conv",
-           "step_conv"]
+           "step_conv", "scan_conv"]
 
 if os.environ.get("LAO_THREADS"):
     set_threads(int(os.environ["LAO_THREADS"]))

@@ -756,9 +756,42 @@ def pin_conv_fused_step(orc):
     assert np.array_equal(hnew[4], hists[4]) and np.array_equal(new[4], pool[4]), "read-only slot untouched"
 
 
+def pin_conv_scan(orc):
+    """The scan with the convolution ahead equals one fused decode step per token with the
+    history carried from step to step (sequences of unequal lengths, one empty, one shorter
+    than the window), from read-slot histories; the final histories (the last W - 1
+    inputs, the old history shifted in for short sequences) go to the write slots."""
+    rng = np.random.default_rng(50)
+    H, dk, dv, W = 2, 16, 8, 4
+    lens = [5, 0, 2, 9]
+    T = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    xq, xk, xv = rng.standard_normal((T, 1, dk)), rng.standard_normal((T, 1, dk)), rng.standard_normal((T, H, dv))
+    wq, wk, wv = rng.standard_normal((1, dk, W)), rng.standard_normal((1, dk, W)), rng.standard_normal((H, dv, W))
+    g, beta = rng.uniform(0.3, 1.0, (T, H)), rng.uniform(0.0, 1.0, (T, H))
+    pool = rng.standard_normal((6, H, dk, dv)) * 0.3
+    hists = rng.standard_normal((6, H, 2 * dk + dv, W - 1))
+    rs, ws = np.array([5, 2, 0, 3], np.int32), np.array([1, 4, 2, 0], np.int32)
+    S, hnew, o, err = orc.scan_conv("gated_delta", 1, cu, xq, xk, xv, g, beta, 0.8, wq, wk, wv, act=1, l2norm=1,
+                                    conv_src=hists, src_pool=pool, read_slot=rs, dst_pool=np.zeros((6, H, dk, dv)),
+                                    conv_dst=np.zeros_like(hists), write_slot=ws)
+    assert err == 0
+    for s_ in range(4):
+        st, hs = pool[rs[s_]][None].copy(), hists[rs[s_]][None].copy()
+        for t in range(cu[s_], cu[s_ + 1]):
+            st, hs2, ot, e = orc.step_conv("gated_delta", 1, st, xq[t:t + 1], xk[t:t + 1], xv[t:t + 1], g[t:t + 1],
+                                           beta[t:t + 1], 0.8, wq, wk, wv, hs, act=1, l2norm=1)
+            assert e == 0
+            hs = hs2
+            close(o[t], ot[0], 1e-12, f"seq {s_} token {t}")
+        close(S[ws[s_]], st[0], 1e-12, f"seq {s_} final state")
+        close(hnew[ws[s_]], hs[0], 1e-300, f"seq {s_} final history")
+
+
 ALL_PINS = [pin_bf16_rounding, pin_brute_force_all_rules, pin_gqa_grouping, pin_exact_rational,
             pin_linear_closed_form, pin_gated_closed_form, pin_beta0_g1_identity, pin_delta_stores_value,
             pin_rearranged_readout, pin_scan_structure, pin_wide_ranges_non_expansive,
             pin_long_sequence_bounded, pin_storage_rounding_points, pin_slots, pin_pool_ops,
             pin_scan_checkpoints, pin_kda_reductions, pin_kda_wide_ranges_non_expansive, pin_query_groups,
-            pin_q8_page_figures, pin_q8_codec, pin_q8_store_point, pin_conv_definition, pin_conv_fused_step]
+            pin_q8_page_figures, pin_q8_codec, pin_q8_store_point, pin_conv_definition, pin_conv_fused_step,
+            pin_conv_scan]
