@@ -423,9 +423,20 @@ class ScanRunner:
             self.dst_t = torch.empty(n_seqs + self.n_ckpt, inp.n_v_heads, inp.d_k, inp.d_v, dtype=inp.state_dtype,
                                      device="cuda")
             self.dst = L.Pool(self.dst_t, inp.n_qk_heads)
+        self.conv = None
+        if "width" in inp.extra:  # the short causal convolution ahead of every token (fresh prefill)
+            x = inp.extra
+            self.hist_t = torch.empty(n_seqs, inp.n_v_heads, 2 * inp.d_k + inp.d_v, x["width"] - 1,
+                                      dtype=inp.io_dtype, device="cuda")
+            self.conv = L.Conv(to_dev(x["w_q"]), to_dev(x["w_k"]), to_dev(x["w_v"]), self.hist_t, self.hist_t,
+                               activation=x["activation"], qk_l2norm=x["qk_l2norm"])
 
     def step(self, i=0, stream=None):
-        if self.chunked:
+        if self.conv is not None:
+            st = self.L.la_state_scan_conv(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu,
+                                           self.conv, self.q, self.k, self.v, self.g, self.beta, self.inp.scale,
+                                           self.o, self.err, seq_order=self.order, stream=stream)
+        elif self.chunked:
             st = self.L.la_state_scan_chunked(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu, self.q,
                                               self.k, self.v, self.g, self.beta, self.inp.scale, self.o, self.err,
                                               seq_order=self.order, stream=stream)
@@ -447,7 +458,13 @@ class ScanRunner:
                                     d_k=i.d_k, d_v=i.d_v, io_bytes=i.q.element_size(), rule=i.rule,
                                     final_state_bytes=self.dst_t.element_size(),
                                     init_state_bytes=0 if i.pool is None else i.pool.element_size())
-        return b + self.n_ckpt * i.n_v_heads * i.d_k * i.d_v * self.dst_t.element_size(), f
+        b += self.n_ckpt * i.n_v_heads * i.d_k * i.d_v * self.dst_t.element_size()
+        if self.conv is not None:  # the final histories and the weights
+            x = i.extra
+            b += self.n_seqs * i.n_v_heads * (2 * i.d_k + i.d_v) * (x["width"] - 1) * i.q.element_size()
+            b += 4 * x["width"] * (2 * i.n_qk_heads * i.d_k + i.n_v_heads * i.d_v)
+            f += 2 * self.T * i.n_v_heads * (2 * i.d_k + i.d_v) * x["width"]
+        return b, f
 
 
 class PoolRunner:
@@ -698,7 +715,7 @@ def cpu_baseline_decode(inp, budget_s=10.0):
 
 def build_runner(name, seed=0, prefill_seqs=32, ckpt_every=0, chunked=False):
     from gated_deltanet_recurrent_la_b200 import workloads as W
-    if name in ("prefill32", "kda_prefill32"):
+    if name in ("prefill32", "kda_prefill32", "conv_prefill32"):
         inp = W.WORKLOADS[name](seed, prefill_seqs)
     else:
         inp = W.WORKLOADS[name](seed)
@@ -772,7 +789,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode64",
                     choices=["decode64", "decode512", "mamba2", "prefill32", "kda_decode64", "kda_prefill32",
-                             "qgroup_decode256", "q8_decode64", "conv_decode64"])
+                             "qgroup_decode256", "q8_decode64", "conv_decode64", "conv_prefill32"])
     ap.add_argument("--rows", default="all", choices=["all", "none"])
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--scan-algo", default="serial", choices=["serial", "chunked"],
@@ -844,7 +861,7 @@ def main():
     if a.rows == "all":
         rows = {}
         for name in ("decode512", "mamba2", "prefill32", "kda_decode64", "kda_prefill32", "qgroup_decode256",
-                     "q8_decode64", "conv_decode64"):
+                     "q8_decode64", "conv_decode64", "conv_prefill32"):
             if name == a.workload:
                 continue
             k = a.steps if "prefill" not in name else max(3, min(a.steps, 20))

@@ -188,7 +188,7 @@ static la_status step_impl(la_rule rule, const la_pool* src, const int32_t* read
     fn = (src->dtype == LA_F32) ? la::find_step_qgroups_f32(rule, s.d_k, s.d_v, io)
                                 : la::find_step_qgroups_bf16(rule, s.d_k, s.d_v, io);
   if (!fn) return LA_ERR_UNSUPPORTED;
-  la::StepParams p;
+  la::StepParams p{};
   p.src = src->data;
   p.src_slots = src->n_slots;
   p.dst = dst->data;
@@ -251,7 +251,7 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
                            const int32_t* seq_order, const void* q, const void* k, const void* v, la_dtype io,
                            const float* g, const float* beta, float scale, void* o, int32_t ckpt_every,
                            const int32_t* ckpt_cu, const int32_t* ckpt_slots, int32_t* err_word, void* stream,
-                           bool chunked = false, int32_t n_q_heads = 0) {
+                           bool chunked = false, int32_t n_q_heads = 0, const la_conv* conv = nullptr) {
   if (rule < LA_RULE_LINEAR || rule > LA_RULE_KDA) return LA_ERR_UNSUPPORTED;
   if (!err_word) return LA_ERR_NULL;
   if (n_seqs < 0 || total_tokens < 0) return LA_ERR_SHAPE;
@@ -282,8 +282,19 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
 
   const bool q8 = dst->dtype == LA_Q8 || (read_slot && src->dtype == LA_Q8);
   if (q8 && (chunked || n_q_heads != 0)) return LA_ERR_UNSUPPORTED;
+  if (conv) {
+    if (q8 || chunked || n_q_heads != 0 || ckpt_every > 0) return LA_ERR_UNSUPPORTED;
+    if (conv->width < 2 || conv->width > la::kMaxConvWidth) return LA_ERR_UNSUPPORTED;
+    if (!conv->w_q || !conv->w_k || !conv->w_v || !conv->hist_dst || (read_slot && !conv->hist_src))
+      return LA_ERR_NULL;
+    if (!aligned(conv->w_q, 4) || !aligned(conv->w_k, 4) || !aligned(conv->w_v, 4) || !aligned(conv->hist_src, 16) ||
+        !aligned(conv->hist_dst, 16))
+      return LA_ERR_ALIGN;
+  }
   la::ScanLaunchFn fn = nullptr;
-  if (chunked) {
+  if (conv) {
+    fn = (io == LA_F32) ? la::find_scan_conv_f32io(rule, s.d_k, s.d_v) : la::find_scan_conv_bf16io(rule, s.d_k, s.d_v);
+  } else if (chunked) {
     if (s.d_k != 128 || s.d_v != 128 || io != LA_BF16) return LA_ERR_UNSUPPORTED;
     fn = la::find_chunk_scan(rule);
   } else if (n_q_heads == 0) {
@@ -293,7 +304,7 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
                         : la::find_scan_qgroups_bf16io(rule, s.d_k, s.d_v);
   }
   if (!fn) return LA_ERR_UNSUPPORTED;
-  la::ScanParams p;
+  la::ScanParams p{};
   p.src = read_slot ? src->data : nullptr;
   p.src_slots = read_slot ? src->n_slots : 0;
   p.src_dtype = read_slot ? src->dtype : dst->dtype;
@@ -324,6 +335,16 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
   p.ckpt_every = ckpt_every;
   p.ckpt_cu = ckpt_cu;
   p.ckpt_slots = ckpt_slots;
+  if (conv) {
+    p.conv_w = conv->width;
+    p.conv_act = conv->activation;
+    p.conv_l2norm = conv->qk_l2norm;
+    p.conv_wq = conv->w_q;
+    p.conv_wk = conv->w_k;
+    p.conv_wv = conv->w_v;
+    p.conv_src = conv->hist_src;
+    p.conv_dst = conv->hist_dst;
+  }
   return cuda_status(fn(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -355,6 +376,16 @@ la_status la_state_scan_checkpointed(la_rule rule, const la_pool* src, const int
   if (!aligned(ckpt_cu, 4) || !aligned(ckpt_slots, 4)) return LA_ERR_ALIGN;
   return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, q, k, v, io,
                    g, beta, scale, o, ckpt_every, ckpt_cu, ckpt_slots, err_word, stream);
+}
+
+la_status la_state_scan_conv(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
+                             const int32_t* write_slot, int32_t n_seqs, const int32_t* cu_seqlens,
+                             int32_t total_tokens, const int32_t* seq_order, const la_conv* conv, const void* xq,
+                             const void* xk, const void* xv, la_dtype io, const float* g, const float* beta,
+                             float scale, void* o, int32_t* err_word, void* stream) {
+  if (!conv) return LA_ERR_NULL;
+  return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, xq, xk, xv, io,
+                   g, beta, scale, o, 0, nullptr, nullptr, err_word, stream, false, 0, conv);
 }
 
 la_status la_state_scan_qgroups(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,

@@ -68,6 +68,15 @@ struct ScanParams {
   const uint32_t* src_mask;
   int32_t dst_n_hp;
   const uint32_t* dst_mask;
+  // the short causal convolution ahead of every token (conv_w == 0: none)
+  int32_t conv_w;
+  int32_t conv_act;
+  int32_t conv_l2norm;
+  const float* conv_wq;
+  const float* conv_wk;
+  const float* conv_wv;
+  const void* conv_src;     // io dtype [src slots][H_v][2 d_k + d_v][W - 1]
+  void* conv_dst;
   const void* q;
   const void* k;
   const void* v;
@@ -108,6 +117,8 @@ ScanLaunchFn find_scan_bf16io(int rule, int dk, int dv);
 constexpr int kMaxConvWidth = 4;
 StepLaunchFn find_step_conv_f32(int rule, int dk, int dv, int io);
 StepLaunchFn find_step_conv_bf16(int rule, int dk, int dv, int io);
+ScanLaunchFn find_scan_conv_f32io(int rule, int dk, int dv);
+ScanLaunchFn find_scan_conv_bf16io(int rule, int dk, int dv);
 
 // The same in the query-group direction (k per state head, q_group <= kMaxQueryGroup
 // query heads reading each state head).

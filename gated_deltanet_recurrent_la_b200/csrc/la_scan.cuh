@@ -53,7 +53,7 @@
 
 namespace la {
 
-template <int DK, int DV, typename IT, bool CHG = false, int QMAX = 1>
+template <int DK, int DV, typename IT, bool CHG = false, int QMAX = 1, bool CONV = false>
 struct ScanCfg {
   static constexpr int kLG = 4;                        // lanes sharing a column group (split d_k)
   static constexpr int kC = LA_SCAN_COLS;              // columns per lane
@@ -82,10 +82,15 @@ struct ScanCfg {
   static constexpr int kCvtKQ = kCvtQ + kTC * QMAX * kKP * 4;  // [kTC][QMAX]
   static constexpr int kCvtA = kCvtKQ + kTC * QMAX * 4;
   static constexpr int kCvtKt = kCvtA + (CHG ? kTC * kKP * 4 : 0);
-  static constexpr int kCvtBytes = kCvtKt + (CHG ? kTC * kKP * 4 : 0);
+  static constexpr int kCvtV = kCvtKt + (CHG ? kTC * kKP * 4 : 0);  // CONV: post-convolution v [kTC][DV]
+  static constexpr int kCvtBytes = kCvtV + (CONV ? kTC * DV * 4 : 0);
   static constexpr int kOffCvt = 2 * kRawBytes;
   static constexpr int kOffOnes = kOffCvt + 2 * kCvtBytes;  // kda: kKP ones (no pending decay)
-  static constexpr int kSmem = kOffOnes + (CHG ? kKP * 4 : 0);
+  // CONV: the unit's weights [2 DK + DV][W] and the last W - 1 raw inputs [W - 1][2 DK + DV]
+  static constexpr int kCH = 2 * DK + DV;
+  static constexpr int kOffConvW = kOffOnes + (CHG ? kKP * 4 : 0);
+  static constexpr int kOffCarry = kOffConvW + (CONV ? kCH * kMaxConvWidth * 4 : 0);
+  static constexpr int kSmem = kOffCarry + (CONV ? (kCH * (kMaxConvWidth - 1) * kIB + 15) / 16 * 16 : 0);
 
   static_assert(kC == 2 || kC == 4, "columns per lane");
   static_assert(DK % (4 * kLG) == 0, "rows per lane must be a multiple of 4");
@@ -95,17 +100,21 @@ struct ScanCfg {
   static_assert(kRawBytes % 16 == 0 && kCvtBytes % 16 == 0, "alignment of staging buffers");
 };
 
-template <int RULE, int DK, int DV, typename IT, int MIN_BLOCKS, bool CKPT, bool QGRP>
+template <int RULE, int DK, int DV, typename IT, int MIN_BLOCKS, bool CKPT, bool QGRP, bool CONV = false>
 __global__ void __launch_bounds__(
-    ScanCfg<DK, DV, IT, Rule<RULE>::kChannelGate, QGRP ? kMaxQueryGroup : 1>::kThreads, MIN_BLOCKS)
+    ScanCfg<DK, DV, IT, Rule<RULE>::kChannelGate, QGRP ? kMaxQueryGroup : 1, CONV>::kThreads, MIN_BLOCKS)
     scan_kernel(const ScanParams p) {
   constexpr bool CHG = Rule<RULE>::kChannelGate;
   constexpr int QM = QGRP ? kMaxQueryGroup : 1;
-  using C = ScanCfg<DK, DV, IT, CHG, QM>;
+  using C = ScanCfg<DK, DV, IT, CHG, QM, CONV>;
+  static_assert(!(CONV && (QGRP || CKPT)), "the convolution runs in the plain scan");
+  constexpr int CH = C::kCH;
   const int qg = QGRP ? p.q_group : 1;
   constexpr int R = C::kR;
   constexpr int KC = C::kC;
   extern __shared__ __align__(128) unsigned char smem[];
+  float* wconv = reinterpret_cast<float*>(smem + C::kOffConvW);  // CONV
+  IT* carry = reinterpret_cast<IT*>(smem + C::kOffCarry);          // CONV
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -222,6 +231,25 @@ __global__ void __launch_bounds__(
       for (int m = 0; m < R; ++m)
 #pragma unroll
         for (int c = 0; c < KC; ++c) S[m][c] = 0.0f;
+    }
+
+    // ---- convolution: the unit's weights and its history (the last W - 1 raw inputs of
+    //      every channel, oldest first: carry[j][c]) from the read slot, or zero
+    const int cw = CONV ? p.conv_w : 1;
+    if constexpr (CONV) {
+      for (int idx = tid; idx < CH * cw; idx += C::kThreads) {
+        const int c = idx / cw, j = idx % cw;
+        wconv[idx] = c < DK ? __ldg(p.conv_wq + ((int64_t)hq * DK + c) * cw + j)
+                   : c < 2 * DK ? __ldg(p.conv_wk + ((int64_t)hq * DK + (c - DK)) * cw + j)
+                                : __ldg(p.conv_wv + ((int64_t)h * DV + (c - 2 * DK)) * cw + j);
+      }
+      const IT* hs = static_cast<const IT*>(p.conv_src) + ((int64_t)rs * H + h) * CH * (cw - 1);
+      for (int idx = tid; idx < CH * (cw - 1); idx += C::kThreads) {
+        const int c = idx / (cw - 1), j = idx % (cw - 1);
+        if (p.read_slot) carry[j * CH + c] = hs[idx];
+        else io_store(carry + j * CH + c, 0.0f);
+      }
+      __syncthreads();
     }
 
     // ---- token loop
@@ -381,6 +409,80 @@ __global__ void __launch_bounds__(
 
       float* af = reinterpret_cast<float*>(cvt + C::kCvtA);
       float* ktf = reinterpret_cast<float*>(cvt + C::kCvtKt);
+      float* vf = reinterpret_cast<float*>(cvt + C::kCvtV);
+      if constexpr (CONV) {
+        // the convolution: a thread per channel walks the chunk's tokens with the window of
+        // its W - 1 previous inputs in registers (starting from the carried ones), and leaves
+        // the chunk's last W - 1 inputs as the new carried window of its channel
+        const IT* vraw_in = reinterpret_cast<const IT*>(raw + C::kRawV);
+        for (int c = tid; c < CH; c += C::kThreads) {
+          float w[kMaxConvWidth], win[kMaxConvWidth - 1];
+#pragma unroll
+          for (int j = 0; j < kMaxConvWidth; ++j) w[j] = j < cw ? wconv[c * cw + j] : 0.0f;
+          float wnew = 0.0f;  // the newest input's weight, w[cw - 1] (kept out of dynamic indexing)
+#pragma unroll
+          for (int j = 0; j < kMaxConvWidth; ++j)
+            if (j == cw - 1) wnew = w[j];
+#pragma unroll
+          for (int j = 0; j < kMaxConvWidth - 1; ++j) win[j] = j < cw - 1 ? io_load(carry + j * CH + c) : 0.0f;
+          const int i = c % DK;
+          const int prow = (i / R) * C::kRowStride + (i % R);
+          const IT* src = c < DK ? qraw + c : c < 2 * DK ? kraw + (c - DK) : vraw_in + (c - 2 * DK);
+          const int sstride = c < DK ? QM * DK : c < 2 * DK ? DK : DV;
+          float* dst = c < DK ? qf + prow : c < 2 * DK ? kf + prow : vf + (c - 2 * DK);
+          const int dstride = c < DK ? QM * C::kKP : c < 2 * DK ? C::kKP : DV;
+          for (int tt = 0; tt < n; ++tt) {
+            const float x = io_load(src + tt * sstride);
+            float y = wnew * x;
+#pragma unroll
+            for (int j = 0; j < kMaxConvWidth - 1; ++j)
+              if (j < cw - 1) y = fmaf(w[j], win[j], y);
+#pragma unroll
+            for (int j = 0; j < kMaxConvWidth - 1; ++j)
+              win[j] = j < cw - 2 ? win[j + 1] : (j == cw - 2 ? x : win[j]);
+            if (p.conv_act) y = __fdividef(y, 1.0f + __expf(-y));
+            dst[tt * dstride] = y;
+          }
+#pragma unroll
+          for (int j = 0; j < kMaxConvWidth - 1; ++j)
+            if (j < cw - 1) io_store(carry + j * CH + c, win[j]);
+        }
+        if (CHG) {
+          for (int idx = tid; idx < n * DK; idx += C::kThreads) {
+            const int tt = idx / DK, i = idx % DK;
+            af[tt * C::kKP + (i / R) * C::kRowStride + (i % R)] = reinterpret_cast<const float*>(raw + C::kRawA)[idx];
+          }
+        }
+        __syncthreads();
+        // per token: unit length for q and k (when asked), k.q, the decayed rows (kda)
+        for (int tt = warp; tt < n; tt += C::kWarps) {
+          float sq = 0.0f, sk = 0.0f, d = 0.0f;
+          for (int i = lane; i < DK; i += 32) {
+            const int pi = tt * C::kKP + (i / R) * C::kRowStride + (i % R);
+            const float qv = qf[tt * QM * C::kKP + (i / R) * C::kRowStride + (i % R)], kv = kf[pi];
+            sq = fmaf(qv, qv, sq);
+            sk = fmaf(kv, kv, sk);
+            d = fmaf(kv, qv, d);
+          }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            d += __shfl_xor_sync(0xffffffffu, d, off);
+          }
+          const float rq = p.conv_l2norm ? rsqrtf(sq + 1e-6f) : 1.0f;
+          const float rk = p.conv_l2norm ? rsqrtf(sk + 1e-6f) : 1.0f;
+          for (int i = lane; i < DK; i += 32) {
+            const int pi = tt * C::kKP + (i / R) * C::kRowStride + (i % R);
+            const int qi_ = tt * QM * C::kKP + (i / R) * C::kRowStride + (i % R);
+            const float kv = kf[pi] * rk;
+            kf[pi] = kv;
+            qf[qi_] = CHG ? qf[qi_] * rq * af[pi] : qf[qi_] * rq;
+            if (CHG) ktf[pi] = af[pi] * kv;
+          }
+          if (lane == 0) kqs[tt * QM] = d * rq * rk;
+        }
+      } else {
       // convert keys / queries to padded FP32, and k.q per token (kda: also the decays,
       // the decayed key and the decayed query)
       for (int idx = tid; idx < n * DK; idx += C::kThreads) {
@@ -409,6 +511,7 @@ __global__ void __launch_bounds__(
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
         if (lane == 0) kqs[tt * QM + qi] = d;
+      }
       }
       __syncthreads();
 
@@ -471,7 +574,10 @@ __global__ void __launch_bounds__(
         float vv[KC];
 #pragma unroll
         for (int c = 0; c < KC; ++c) vv[c] = 0.0f;
-        if (col_active) load_f32<IT, KC>(vraw + tt * DV + col0, vv);
+        if (col_active) {
+          if constexpr (CONV) load_f32<float, KC>(vf + tt * DV + col0, vv);
+          else load_f32<IT, KC>(vraw + tt * DV + col0, vv);
+        }
         // u = b (v - c S^T k),  o = scale (a S^T q + (k.q) u),  with S = gam St
         float uu[KC], oc[KC];
 #pragma unroll
@@ -565,17 +671,35 @@ __global__ void __launch_bounds__(
       __syncthreads();
     }
 
-    // ---- last pending update, store the final state
+    // ---- last pending update, store the final state (and the convolution history)
     if (kp) apply_pending();
     store_state(ws);
+    if constexpr (CONV) {
+      IT* hd = static_cast<IT*>(p.conv_dst) + ((int64_t)ws * H + h) * CH * (cw - 1);
+      for (int idx = tid; idx < CH * (cw - 1); idx += C::kThreads) {
+        const int c = idx / (cw - 1), j = idx % (cw - 1);
+        hd[idx] = carry[j * CH + c];
+      }
+    }
     // the next unit's staging must not overwrite what this unit still reads
     __syncthreads();
   }
 }
 
-template <int RULE, int DK, int DV, typename IT, bool QGRP>
+template <int RULE, int DK, int DV, typename IT, bool QGRP, bool CONV = false>
 cudaError_t launch_scan(const ScanParams& p, cudaStream_t stream) {
-  using C = ScanCfg<DK, DV, IT, Rule<RULE>::kChannelGate, QGRP ? kMaxQueryGroup : 1>;
+  using C = ScanCfg<DK, DV, IT, Rule<RULE>::kChannelGate, QGRP ? kMaxQueryGroup : 1, CONV>;
+  if constexpr (CONV) {
+    constexpr int kMinBlocks = 2;
+    const void* fn = reinterpret_cast<const void*>(&scan_kernel<RULE, DK, DV, IT, kMinBlocks, false, false, true>);
+    const int per_sm = prepare_kernel(fn, C::kThreads, C::kSmem);
+    if (per_sm <= 0) return cudaErrorInvalidConfiguration;
+    const int64_t units = (int64_t)p.n_seqs * p.n_v_heads;
+    const int64_t cap = (int64_t)device_sm_count() * per_sm;
+    const int grid = (int)(units < cap ? units : cap);
+    scan_kernel<RULE, DK, DV, IT, kMinBlocks, false, false, true><<<grid, C::kThreads, C::kSmem, stream>>>(p);
+    return cudaGetLastError();
+  }
   constexpr int kMinBlocks = 2;  // two CTAs (units) per SM
   // checkpoints are a separate instantiation so that the plain scan's loop carries no
   // checkpoint bookkeeping (the query-group direction has none)
@@ -606,6 +730,22 @@ ScanLaunchFn find_scan_impl(int rule, int dk, int dv) {
   LA_SCAN_SHAPES(LA_RULE_KDA)
 #undef LA_SCAN_SHAPES
 #undef LA_SCAN_CASE
+  return nullptr;
+}
+
+// Launcher table of the scan with the convolution ahead (io dtype IT).
+template <typename IT>
+ScanLaunchFn find_scan_conv_impl(int rule, int dk, int dv) {
+#define LA_SCONV_CASE(R, K, V) \
+  if (rule == R && dk == K && dv == V) return &launch_scan<R, K, V, IT, false, true>;
+#define LA_SCONV_SHAPES(R) LA_SCONV_CASE(R, 16, 16) LA_SCONV_CASE(R, 64, 64) LA_SCONV_CASE(R, 128, 64) LA_SCONV_CASE(R, 128, 128)
+  LA_SCONV_SHAPES(LA_RULE_LINEAR)
+  LA_SCONV_SHAPES(LA_RULE_GATED)
+  LA_SCONV_SHAPES(LA_RULE_DELTA)
+  LA_SCONV_SHAPES(LA_RULE_GATED_DELTA)
+  LA_SCONV_SHAPES(LA_RULE_KDA)
+#undef LA_SCONV_SHAPES
+#undef LA_SCONV_CASE
   return nullptr;
 }
 

@@ -30,6 +30,7 @@ DEVERR_READ_SLOT, DEVERR_WRITE_SLOT, DEVERR_CU_SEQLENS, DEVERR_TIMEOUT, DEVERR_Q
 EXPORTS = ("la_state_bytes", "la_shape_supported", "la_state_step", "la_state_scan", "la_state_scan_chunked",
            "la_state_scan_checkpointed", "la_state_step_qgroups", "la_state_scan_qgroups",
            "la_pool_slot_bytes", "la_state_pool_encode", "la_state_pool_decode", "la_state_step_conv",
+           "la_state_scan_conv",
            "la_state_pool_copy",
            "la_state_pool_gather", "la_state_pool_scatter", "la_state_pool_zero", "la_state_check_slots",
            "la_status_str", "la_last_cuda_error", "la_abi_version")
@@ -98,6 +99,9 @@ def lib():
         L.la_state_step_conv.argtypes = L.la_state_step.argtypes[:6] + [ctypes.POINTER(la_conv)] + \
             L.la_state_step.argtypes[6:]
         L.la_state_step_conv.restype = I32
+        L.la_state_scan_conv.argtypes = L.la_state_scan.argtypes[:9] + [ctypes.POINTER(la_conv)] + \
+            L.la_state_scan.argtypes[9:]
+        L.la_state_scan_conv.restype = I32
         L.la_pool_slot_bytes.argtypes = [PP]
         L.la_pool_slot_bytes.restype = ctypes.c_size_t
         L.la_state_pool_encode.argtypes = [PP, I32, P, P, P, P]
@@ -254,6 +258,18 @@ def la_state_step_conv(rule, src: Pool, read_slot, dst: Pool, write_slot, conv: 
     return lib().la_state_step_conv(RULES[rule] if isinstance(rule, str) else int(rule), src.ref,
                                     _ptr(read_slot, torch.int32), dst.ref, _ptr(write_slot, torch.int32),
                                     int(xq.shape[0]), conv.ref, _ptr(xq), _ptr(xk, xq.dtype), _ptr(xv, xq.dtype), io,
+                                    _ptr(g, torch.float32), _ptr(beta, torch.float32), float(scale),
+                                    _ptr(o, xq.dtype), _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_state_scan_conv(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens, conv: Conv, xq, xk,
+                       xv, g, beta, scale, o, err_word, seq_order=None, stream=None) -> int:
+    io = dtype_code(xq.dtype)
+    return lib().la_state_scan_conv(RULES[rule] if isinstance(rule, str) else int(rule),
+                                    None if src is None else src.ref, _ptr(read_slot, torch.int32), dst.ref,
+                                    _ptr(write_slot, torch.int32), int(cu_seqlens.numel() - 1),
+                                    _ptr(cu_seqlens, torch.int32), int(xq.shape[0]), _ptr(seq_order, torch.int32),
+                                    conv.ref, _ptr(xq), _ptr(xk, xq.dtype), _ptr(xv, xq.dtype), io,
                                     _ptr(g, torch.float32), _ptr(beta, torch.float32), float(scale),
                                     _ptr(o, xq.dtype), _ptr(err_word, torch.int32), _stream(stream))
 

@@ -24,6 +24,7 @@ Named workloads (sizes from the "SSM / linear-RNN decode" page, the ONNX section
   qgroup_decode256  B=256 decode, 16 state heads each read by 4 query heads (ONNX direction)
   q8_decode64 decode64 on the mixed INT8 / BF16 state storage (1/8 of the key channels BF16)
   conv_decode64  decode64 with the short causal convolution (width 4, SiLU, q/k norm) ahead
+  conv_prefill32 prefill32 with the same convolution ahead of every token (fresh prefill)
 """
 from __future__ import annotations
 
@@ -283,6 +284,22 @@ def kda_prefill32(seed: int = 0, n_seqs: int = 32) -> Inputs:
                        d_v=128, seed=seed + 1, rule="kda")
 
 
+def conv_prefill32(seed: int = 0, n_seqs: int = 32, width: int = 4) -> Inputs:
+    """prefill32 with the short causal convolution ahead of every token (fresh prefill:
+    zero histories): q, k, v are the convolution's inputs (N(0, 1), not normalised),
+    weights N(0, 1 / W), SiLU and the q/k normalisation on (`extra`)."""
+    inp = scan_inputs(lengths=prefill32_lengths(seed, n_seqs), n_qk_heads=32, n_v_heads=32, d_k=128, d_v=128,
+                      seed=seed + 1, normalise_qk=False)
+    gen = _gen(seed + 13)
+    inp.extra = {
+        "width": width, "activation": 1, "qk_l2norm": 1,
+        "w_q": (torch.randn(32, 128, width, generator=gen) / width ** 0.5).contiguous(),
+        "w_k": (torch.randn(32, 128, width, generator=gen) / width ** 0.5).contiguous(),
+        "w_v": (torch.randn(32, 128, width, generator=gen) / width ** 0.5).contiguous(),
+    }
+    return inp
+
+
 def mamba2(seed: int = 0, B: int = 256) -> Inputs:
     """Mamba-2-style gated decode read as the gated rule: d_inner 8192 = 128 heads x 64
     (d_v), d_state N = 128 (d_k), one B/C group (H_qk = 1).  k := B_t, q := C_t (both
@@ -314,4 +331,5 @@ WORKLOADS = {
     "qgroup_decode256": qgroup_decode256,
     "q8_decode64": q8_decode64,
     "conv_decode64": conv_decode64,
+    "conv_prefill32": conv_prefill32,
 }

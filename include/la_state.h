@@ -268,6 +268,22 @@ la_status la_state_step_conv(la_rule rule, const la_pool *src, const int32_t *re
                              la_dtype io, const float *g, const float *beta, float scale, void *o,
                              int32_t *err_word, void *stream);
 
+/* la_state_scan with the convolution ahead of every token: xq, xk, xv are the
+ * convolution's inputs (layouts of q, k, v).  Each (sequence, head) history is read from
+ * conv->hist_src at read_slot[s] (zero when read_slot is NULL: a fresh prefill), carried
+ * through the sequence, and the history after its last token is written to
+ * conv->hist_dst at write_slot[s] (an empty sequence passes its history through), ready
+ * for la_state_step_conv.  FP32 or BF16 pools, the default head direction, no
+ * checkpoints (LA_ERR_UNSUPPORTED otherwise).  Other arguments and errors as
+ * la_state_scan. */
+la_status la_state_scan_conv(la_rule rule, const la_pool *src, const int32_t *read_slot,
+                             const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
+                             const int32_t *cu_seqlens, int32_t total_tokens,
+                             const int32_t *seq_order, const la_conv *conv, const void *xq,
+                             const void *xk, const void *xv, la_dtype io, const float *g,
+                             const float *beta, float scale, void *o, int32_t *err_word,
+                             void *stream);
+
 /* The query-group direction of the ONNX LinearAttention operator ("Seven Architectures
  * ...", section "ONNX LinearAttention / FlashInfer": each KV head and its recurrent state
  * shared by a group of query heads, q_num_heads / kv_num_heads).  The state of head h is

@@ -249,6 +249,23 @@ def test_conv_step_host_errors(lib):
     assert call(src=q8) == L.LA_ERR_UNSUPPORTED
 
 
+def test_conv_scan_host_errors(lib):
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+
+    def call(width=4, rs=None, hist_src=A, dst=None):
+        conv = L.la_conv(width, 1, 1, P(A), P(A), P(A), P(hist_src), P(A))
+        dst = dst or pool()
+        return lib.la_state_scan_conv(3, ctypes.byref(pool()), P(rs), ctypes.byref(dst), None, 2, P(A), 10, None,
+                                      ctypes.byref(conv), P(A), P(A), P(A), 1, P(A), P(A), 1.0, P(A), P(A), None)
+    assert call(width=9) == L.LA_ERR_UNSUPPORTED
+    assert call(rs=A, hist_src=None) == L.LA_ERR_NULL
+    assert call(hist_src=A + 4) == L.LA_ERR_ALIGN
+    q8 = L.la_pool(ctypes.c_void_p(A), L.LA_Q8, 8, L.la_shape(2, 4, 128, 128), 16, P(A))
+    assert call(dst=q8) == L.LA_ERR_UNSUPPORTED
+    assert lib.la_state_scan_conv(3, None, None, ctypes.byref(pool()), None, 2, P(A), 10, None, None, P(A), P(A),
+                                  P(A), 1, P(A), P(A), 1.0, P(A), P(A), None) == L.LA_ERR_NULL
+
+
 def test_check_slots(lib):
     t = lambda x: torch.tensor(x, dtype=torch.int32)  # noqa: E731
     assert L.la_state_check_slots(t([0, 1, 2]), t([0, 1, 2]), 4) == L.LA_OK

@@ -93,3 +93,88 @@ def test_conv_decode64_full():
     assert_close(np64(after[ws]), ref, 2e-2, "sampled states")
     assert_close(np64(o.cpu()[rows]), o_ref, 2e-2, "sampled outputs")
     assert np.array_equal(np64(hist_t.cpu()[ws]), href), "sampled histories"
+
+
+def _conv_weights(nqk, H, dk, dv, width, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(nqk, dk, width, generator=g) / width ** 0.5,
+            torch.randn(nqk, dk, width, generator=g) / width ** 0.5,
+            torch.randn(H, dv, width, generator=g) / width ** 0.5)
+
+
+def run_scan_conv(inp, wq, wk, wv, width, act, l2, hist_src, n_dst, dst_dtype, read_slot=None, write_slot=None):
+    H, dk, dv = inp.n_v_heads, inp.d_k, inp.d_v
+    dst_t = torch.full((n_dst, H, dk, dv), 3.0, dtype=dst_dtype, device="cuda")
+    hist_dst = torch.full((n_dst, H, 2 * dk + dv, width - 1), 9.0, dtype=inp.io_dtype, device="cuda")
+    src = None if inp.pool is None else L.Pool(dev(inp.pool), inp.n_qk_heads)
+    hs = None if hist_src is None else dev(hist_src)
+    conv = L.Conv(dev(wq), dev(wk), dev(wv), hs if hs is not None else hist_dst, hist_dst, activation=act,
+                  qk_l2norm=l2)
+    o = torch.full((inp.q.shape[0], H, dv), 5.0, dtype=inp.io_dtype, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.check(L.la_state_scan_conv(inp.rule, src, dev(read_slot), L.Pool(dst_t, inp.n_qk_heads), dev(write_slot),
+                                 dev(inp.cu_seqlens), conv, dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.g),
+                                 dev(inp.beta), inp.scale, o, err))
+    torch.cuda.synchronize()
+    return dst_t.cpu(), hist_dst.cpu(), o.cpu(), int(err.item())
+
+
+@pytest.mark.parametrize("width", [2, 4])
+@pytest.mark.parametrize("act,l2", [(0, 0), (1, 1)], ids=["plain", "silu_norm"])
+@pytest.mark.parametrize("io", [F32, BF16], ids=["f32io", "bf16io"])
+@pytest.mark.parametrize("dk,dv", [(16, 16), (128, 64), (128, 128)], ids=["16x16", "128x64", "128x128"])
+@pytest.mark.parametrize("rule", ["gated_delta", "kda", "gated"])
+def test_scan_conv(rule, dk, dv, io, act, l2, width):
+    lengths = [5, 0, 2, 37, 17]
+    inp = W.scan_inputs(lengths=lengths, n_qk_heads=2, n_v_heads=4, d_k=dk, d_v=dv, rule=rule, state_dtype=F32,
+                        io_dtype=io, seed=110 + width + dk, init="slots", init_dtype=F32, normalise_qk=False,
+                        pool_std=0.3)
+    wq, wk, wv = _conv_weights(2, 4, dk, dv, width, 3 + width)
+    n = len(lengths)
+    hist = torch.randn(n, 4, 2 * dk + dv, width - 1, generator=torch.Generator().manual_seed(8)).to(io)
+    ws = torch.tensor([2, 0, 4, 1, 3], dtype=torch.int32)
+    S, hnew, o, err = run_scan_conv(inp, wq, wk, wv, width, act, l2, hist, n, F32, read_slot=inp.read_slot,
+                                    write_slot=ws)
+    assert err == 0
+    ref, href, o_ref, e = oracle.scan_conv(rule, 2, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k), np64(inp.v),
+                                           np64(inp.g), np64(inp.beta), inp.scale, wq.double().numpy(),
+                                           wk.double().numpy(), wv.double().numpy(), act=act, l2norm=l2,
+                                           conv_src=np64(hist), src_pool=np64(inp.pool),
+                                           read_slot=inp.read_slot.numpy(), dst_pool=np.zeros((n, 4, dk, dv)),
+                                           conv_dst=np.zeros((n, 4, 2 * dk + dv, width - 1)), write_slot=ws.numpy(),
+                                           dst_dtype="f32", io_dtype=dname(io))
+    assert e == 0
+    tol_s, tol_o = tolerances(F32, io)
+    assert_close(np64(S), ref, tol_s, f"{rule} W={width}: final states")
+    assert_close(np64(o), o_ref, tol_o, f"{rule} W={width}: outputs")
+    assert np.array_equal(np64(hnew), href), "final histories are exact copies of inputs"
+
+
+def test_scan_conv_then_step_conv_continues_the_sequence():
+    """A fresh prefill through the convolution, then one fused decode step from its slot,
+    equals the oracle scan over the whole sequence (state, last output, history)."""
+    width = 4
+    inp = W.scan_inputs(lengths=[30], n_qk_heads=1, n_v_heads=2, d_k=64, d_v=64, rule="gated_delta",
+                        state_dtype=F32, io_dtype=F32, seed=120, normalise_qk=False)
+    wq, wk, wv = _conv_weights(1, 2, 64, 64, width, 9)
+    pre = W.Inputs(**{**inp.__dict__, "q": inp.q[:29], "k": inp.k[:29], "v": inp.v[:29], "g": inp.g[:29],
+                      "beta": inp.beta[:29], "cu_seqlens": torch.tensor([0, 29], dtype=torch.int32)})
+    S, hist, o_pre, err = run_scan_conv(pre, wq, wk, wv, width, 1, 1, None, 1, F32)
+    assert err == 0
+    pool_t, hist_t = dev(S), dev(hist)
+    conv = L.Conv(dev(wq), dev(wk), dev(wv), hist_t, activation=1, qk_l2norm=1)
+    o = torch.empty(1, 2, 64, dtype=F32, device="cuda")
+    e = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.check(L.la_state_step_conv("gated_delta", L.Pool(pool_t, 1), None, L.Pool(pool_t, 1), None, conv,
+                                 dev(inp.q[29:]), dev(inp.k[29:]), dev(inp.v[29:]), dev(inp.g[29:]),
+                                 dev(inp.beta[29:]), 1.0, o, e))
+    torch.cuda.synchronize()
+    assert int(e.item()) == 0
+    ref, href, o_ref, er = oracle.scan_conv("gated_delta", 1, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k),
+                                            np64(inp.v), np64(inp.g), np64(inp.beta), 1.0, wq.double().numpy(),
+                                            wk.double().numpy(), wv.double().numpy(), act=1, l2norm=1)
+    assert er == 0
+    assert_close(np64(pool_t.cpu()), ref, 1e-4, "state after prefill + one step")
+    assert_close(np64(o.cpu())[0], o_ref[29], 1e-4, "the decode step's output")
+    assert_close(np64(o_pre), o_ref[:29], 1e-4, "prefill outputs")
+    assert np.array_equal(np64(hist_t.cpu()), href)
