@@ -423,6 +423,10 @@ class ScanRunner:
             self.dst_t = torch.empty(n_seqs + self.n_ckpt, inp.n_v_heads, inp.d_k, inp.d_v, dtype=inp.state_dtype,
                                      device="cuda")
             self.dst = L.Pool(self.dst_t, inp.n_qk_heads)
+        self.ws = None
+        if chunked == "ws":  # the two-launch form: the caller-owned workspace of the intra-chunk part
+            nb = L.la_scan_chunked_workspace_bytes(self.T, n_seqs, inp.n_v_heads)
+            self.ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
         self.conv = None
         if "width" in inp.extra:  # the short causal convolution ahead of every token (fresh prefill)
             x = inp.extra
@@ -436,6 +440,10 @@ class ScanRunner:
             st = self.L.la_state_scan_conv(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu,
                                            self.conv, self.q, self.k, self.v, self.g, self.beta, self.inp.scale,
                                            self.o, self.err, seq_order=self.order, stream=stream)
+        elif self.ws is not None:
+            st = self.L.la_state_scan_chunked_ws(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu,
+                                                 self.q, self.k, self.v, self.g, self.beta, self.inp.scale, self.o,
+                                                 self.ws, self.err, seq_order=self.order, stream=stream)
         elif self.chunked:
             st = self.L.la_state_scan_chunked(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu, self.q,
                                               self.k, self.v, self.g, self.beta, self.inp.scale, self.o, self.err,
@@ -767,7 +775,8 @@ def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_ev
             row["config"]["ckpt_every"] = ckpt_every
             row["config"]["checkpoints"] = run.n_ckpt
         if chunked:
-            row["config"]["algorithm"] = "chunked (64-token WY/UT form, BF16 tensor-core products)"
+            row["config"]["algorithm"] = "chunked (64-token WY/UT form, BF16 tensor-core products)" + \
+                ("; intra-chunk inverses as a separate parallel launch through a workspace" if chunked == "ws" else "")
             row["hbm"] = {"achieved_gb_s": row["gb_s"], "frac_of_measured": row["gb_s"] / peaks["hbm_gbs"]}
             row["token_serial_equivalent_tflops"] = tf  # 6 flops per state element per token, for comparison
             row["roofline"] = tensor_roofline(run, inp, ms, peaks)
@@ -792,8 +801,9 @@ def main():
                              "qgroup_decode256", "q8_decode64", "conv_decode64", "conv_prefill32"])
     ap.add_argument("--rows", default="all", choices=["all", "none"])
     ap.add_argument("--cpu-budget", type=float, default=10.0)
-    ap.add_argument("--scan-algo", default="serial", choices=["serial", "chunked"],
-                    help="prefill workload: token-serial scan or the chunked tensor-core form")
+    ap.add_argument("--scan-algo", default="serial", choices=["serial", "chunked", "chunked_ws"],
+                    help="prefill workload: token-serial scan, the chunked tensor-core form, or that form in "
+                         "two launches through a workspace")
     ap.add_argument("--prefill-seqs", type=int, default=32,
                     help="sequences of the prefill workload (fewer only to profile a smaller case)")
     a = ap.parse_args()
@@ -811,7 +821,8 @@ def main():
     sampler = ClockSampler(local)
     sampler.start()
 
-    run, inp = build_runner(a.workload, prefill_seqs=a.prefill_seqs, chunked=a.scan_algo == "chunked")
+    run, inp = build_runner(a.workload, prefill_seqs=a.prefill_seqs,
+                            chunked={"serial": False, "chunked": True, "chunked_ws": "ws"}[a.scan_algo])
     nbytes, flops = run.bytes_flops()
     ms = time_back_to_back(run, a.steps, a.warmup, world, sampler)
     sampler.stop()
@@ -839,7 +850,7 @@ def main():
         alu = fp32_alu_peak_tflops(sm_count, peaks["sm_max_mhz"])
         tf = flops / (ms * 1e-3) / 1e12
         out["tokens_per_s"] = world * run.T / (ms * 1e-3)
-        if a.scan_algo == "chunked":
+        if a.scan_algo != "serial":
             out["roofline"] = tensor_roofline(run, inp, ms, peaks)
         else:
             out["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
@@ -872,6 +883,9 @@ def main():
         torch.cuda.empty_cache()
         rows["prefill32_chunked"] = measure_row("prefill32", max(3, min(a.steps, 50)), a.warmup, world, peaks,
                                                 sm_count, None, chunked=True)
+        torch.cuda.empty_cache()
+        rows["prefill32_chunked_two_launch"] = measure_row("prefill32", max(3, min(a.steps, 50)), a.warmup, world,
+                                                           peaks, sm_count, None, chunked="ws")
         torch.cuda.empty_cache()
         pool_run = PoolRunner()
         pms = time_back_to_back(pool_run, min(a.steps, 500), a.warmup, world)

@@ -251,7 +251,8 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
                            const int32_t* seq_order, const void* q, const void* k, const void* v, la_dtype io,
                            const float* g, const float* beta, float scale, void* o, int32_t ckpt_every,
                            const int32_t* ckpt_cu, const int32_t* ckpt_slots, int32_t* err_word, void* stream,
-                           bool chunked = false, int32_t n_q_heads = 0, const la_conv* conv = nullptr) {
+                           bool chunked = false, int32_t n_q_heads = 0, const la_conv* conv = nullptr,
+                           void* workspace = nullptr, size_t workspace_bytes = 0) {
   if (rule < LA_RULE_LINEAR || rule > LA_RULE_KDA) return LA_ERR_UNSUPPORTED;
   if (!err_word) return LA_ERR_NULL;
   if (n_seqs < 0 || total_tokens < 0) return LA_ERR_SHAPE;
@@ -296,7 +297,13 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
     fn = (io == LA_F32) ? la::find_scan_conv_f32io(rule, s.d_k, s.d_v) : la::find_scan_conv_bf16io(rule, s.d_k, s.d_v);
   } else if (chunked) {
     if (s.d_k != 128 || s.d_v != 128 || io != LA_BF16) return LA_ERR_UNSUPPORTED;
-    fn = la::find_chunk_scan(rule);
+    if (workspace) {
+      if (!aligned(workspace, 16)) return LA_ERR_ALIGN;
+      if (workspace_bytes < la::chunk_workspace_bytes(total_tokens, n_seqs, s.n_v_heads)) return LA_ERR_SHAPE;
+      fn = la::find_chunk_scan_ws(rule);
+    } else {
+      fn = la::find_chunk_scan(rule);
+    }
   } else if (n_q_heads == 0) {
     fn = (io == LA_F32) ? la::find_scan_f32io(rule, s.d_k, s.d_v) : la::find_scan_bf16io(rule, s.d_k, s.d_v);
   } else {
@@ -335,6 +342,7 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
   p.ckpt_every = ckpt_every;
   p.ckpt_cu = ckpt_cu;
   p.ckpt_slots = ckpt_slots;
+  p.workspace = workspace;
   if (conv) {
     p.conv_w = conv->width;
     p.conv_act = conv->activation;
@@ -363,6 +371,22 @@ la_status la_state_scan_chunked(la_rule rule, const la_pool* src, const int32_t*
                                 int32_t* err_word, void* stream) {
   return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, q, k, v, io,
                    g, beta, scale, o, 0, nullptr, nullptr, err_word, stream, true);
+}
+
+size_t la_scan_chunked_workspace_bytes(int32_t total_tokens, int32_t n_seqs, int32_t n_v_heads) {
+  return la::chunk_workspace_bytes(total_tokens, n_seqs, n_v_heads);
+}
+
+la_status la_state_scan_chunked_ws(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
+                                   const int32_t* write_slot, int32_t n_seqs, const int32_t* cu_seqlens,
+                                   int32_t total_tokens, const int32_t* seq_order, const void* q, const void* k,
+                                   const void* v, la_dtype io, const float* g, const float* beta, float scale,
+                                   void* o, void* workspace, size_t workspace_bytes, int32_t* err_word,
+                                   void* stream) {
+  if (!workspace && n_seqs > 0) return LA_ERR_NULL;
+  return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, q, k, v, io,
+                   g, beta, scale, o, 0, nullptr, nullptr, err_word, stream, true, 0, nullptr, workspace,
+                   workspace_bytes);
 }
 
 la_status la_state_scan_checkpointed(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,

@@ -11,4 +11,19 @@ ScanLaunchFn find_chunk_scan(int rule) {
   }
   return nullptr;
 }
+size_t chunk_workspace_bytes(int64_t total_tokens, int64_t n_seqs, int64_t n_v_heads) {
+  if (total_tokens < 0 || n_seqs < 0 || n_v_heads <= 0) return 0;
+  const int64_t tiles = (total_tokens + chunk::kC - 1) / chunk::kC + n_seqs + 1;
+  return (size_t)(tiles * n_v_heads * chunk::kPrepTileBytes);
+}
+
+ScanLaunchFn find_chunk_scan_ws(int rule) {
+  switch (rule) {
+    case LA_RULE_LINEAR: return &launch_chunk_scan_ws<LA_RULE_LINEAR>;
+    case LA_RULE_GATED: return &launch_chunk_scan_ws<LA_RULE_GATED>;
+    case LA_RULE_DELTA: return &launch_chunk_scan_ws<LA_RULE_DELTA>;
+    case LA_RULE_GATED_DELTA: return &launch_chunk_scan_ws<LA_RULE_GATED_DELTA>;
+  }
+  return nullptr;
+}
 }  // namespace la

@@ -59,6 +59,10 @@ constexpr int kOffGin = kOffG + 6 * kC * 4;     // 2 x {g, beta} [64] fp32 (stag
 constexpr int kSmem = kOffGin + 2 * 2 * kC * 4;
 static_assert(kSmem <= 227 * 1024, "shared memory");
 static_assert(kOffW + kC * kRow128 <= kOffT + kC * kTs * 4, "W reuses the L / T space");
+// workspace tile of one (chunk, head): Tw then Tu, [64][64] BF16 each, in the swizzled layout
+constexpr int kPrepTileBytes = 2 * kC * kRow64;
+static_assert(kOffW + kC * kRow128 <= kOffT && kPrepTileBytes <= kC * kTs * 4,
+              "the second staged Tw / Tu buffer takes the T space, clear of W");
 
 // byte offset of the 16-byte chunk `ch` of row `r` in a swizzled matrix with rows of `rowb` bytes
 __device__ __forceinline__ uint32_t swz(uint32_t base, int r, int ch, int rowb) {
@@ -142,7 +146,9 @@ __device__ __forceinline__ void st_bf16x2(unsigned char* smem, uint32_t off, flo
 
 }  // namespace chunk
 
-template <int RULE>
+// PRE: Tw / Tu of every chunk come from the workspace that chunk_prep_kernel filled
+// (steps 1 and 2 shrink to Q K^T); otherwise everything happens here.
+template <int RULE, bool PRE = false>
 __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const ScanParams p) {
   using namespace chunk;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -180,7 +186,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
   const int mt = warp & 3, nh = warp >> 2;
 
   // the strictly upper 16 x 16 blocks of Tw and Tu are zero in every chunk
-  for (int idx = tid; idx < kC * kC / 2; idx += kThreads) {
+  for (int idx = tid; idx < (PRE ? 0 : kC * kC / 2); idx += kThreads) {
     const int r = idx >> 5, c = 2 * (idx & 31);
     if ((c >> 4) > (r >> 4)) {
       const uint32_t off = swz(kOffTw, r, c >> 3, kRow64) + 2 * (c & 7);
@@ -259,6 +265,13 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
           *reinterpret_cast<uint4*>(in + kC * kRow128 + so) = make_uint4(0, 0, 0, 0);
           *reinterpret_cast<uint4*>(in + 2 * kC * kRow128 + so) = make_uint4(0, 0, 0, 0);
         }
+      }
+      if (PRE && kDelta) {
+        // Tw and Tu (16 KB, already in the swizzled layout) into buffer ci & 1
+        const unsigned char* wsrc = static_cast<const unsigned char*>(p.workspace) +
+                                    (((int64_t)((t0 + cc0) / kC + seq)) * H + h) * kPrepTileBytes;
+        unsigned char* wdst = smem + ((ci & 1) ? kOffT : kOffTw);
+        for (int idx = tid; idx < kPrepTileBytes / 16; idx += kThreads) cp_async_16(wdst + idx * 16, wsrc + idx * 16);
       }
       if (warp == 0) {
         float* gin = reinterpret_cast<float*>(smem + kOffGin) + (ci & 1) * 2 * kC;
@@ -347,7 +360,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
       const bool fact = sFlag[0] != 0;
 
       // ---- step 1: K K^T (warps 0-3, delta rules) and Q K^T (warps 4-7), rows [16 mt, +16)
-      if (kDelta || warp >= 4) {
+      if ((kDelta && !PRE) || warp >= 4) {
         float acc[8][4];
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
@@ -392,16 +405,24 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
 
       // ---- step 2 (delta rules): T = (I + L)^-1 by 16 x 16 blocks, written as FP32 (for the
       //      block recursion) and as Tw = T diag(b gamma), Tu = T diag(b) (BF16, swizzled)
-      if (kDelta) {
+      if (kDelta && !PRE) {
         // diagonal blocks: forward substitution, lane c < 16 of warp b owns column c
         if (warp < 4) {
           const int b0 = 16 * warp, c = lane & 15;
           float col[16];
 #pragma unroll
           for (int r = 0; r < 16; ++r) {
+            // row r of the block's L in 16-byte pieces (issued ahead of the dependent chain)
+            const float4* lr = reinterpret_cast<const float4*>(sL + (b0 + r) * kLs + b0);
             float x = (r == c) ? 1.0f : 0.0f;
 #pragma unroll
-            for (int j = 0; j < r; ++j) x -= sL[(b0 + r) * kLs + b0 + j] * col[j];
+            for (int m = 0; m < (r + 3) / 4; ++m) {
+              const float4 l4 = lr[m];
+              const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (4 * m + e < r) x -= lv[e] * col[4 * m + e];
+            }
             col[r] = (r < c) ? 0.0f : x;
           }
           const int sc = b0 + c;
@@ -467,11 +488,13 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
           accu[j][0] = accu[j][1] = accu[j][2] = accu[j][3] = 0.0f;
           accw[j][0] = accw[j][1] = accw[j][2] = accw[j][3] = 0.0f;
         }
+        // Tw, Tu of this chunk (PRE: the staged copy in buffer ci & 1)
+        const uint32_t tw = sbase + ((PRE && (ci & 1)) ? kOffT : kOffTw), tu = tw + kC * kRow64;
 #pragma unroll
         for (int kk = 0; kk < kC; kk += 16) {
           uint32_t au[4], aw[4];
-          lda(au, sbase + kOffTu, kRow64, 16 * mt, kk, lane);
-          lda(aw, sbase + kOffTw, kRow64, 16 * mt, kk, lane);
+          lda(au, tu, kRow64, 16 * mt, kk, lane);
+          lda(aw, tw, kRow64, 16 * mt, kk, lane);
 #pragma unroll
           for (int np = 0; np < 4; ++np) {
             uint32_t b[4];
@@ -610,6 +633,257 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
   }
 }
 
+// ---- the intra-chunk part on its own: per (chunk, head), K K^T, the UT inverse and
+//      Tw = T diag(b gamma), Tu = T diag(b), written to the workspace for
+//      chunk_scan_kernel<RULE, true>.  Chunks are independent, so several CTAs share an SM
+//      and hide each other's latency.  Chunk c of sequence s goes to workspace tile
+//      (t0_s + 64 c) / 64 + s (distinct for every chunk; fewer than T / 64 + n_seqs + 1).
+namespace chunk {
+constexpr int kPOffK = 0;                           // [64][128] bf16, swizzled
+constexpr int kPOffL = kPOffK + kC * kRow128;       // [64][68] fp32
+constexpr int kPOffT = kPOffL + kC * kLs * 4;       // [64][72] fp32
+constexpr int kPOffTw = kPOffT + kC * kTs * 4;      // Tw, Tu [64][64] bf16, swizzled
+constexpr int kPOffX = kPOffTw + kPrepTileBytes;    // [3][16][24] fp32
+constexpr int kPOffG = kPOffX + 3 * 16 * kXs * 4;   // per token gate quantities [6][64]
+constexpr int kPOffGin = kPOffG + 6 * kC * 4;       // g, beta [2][64]
+constexpr int kPSmem = kPOffGin + 2 * kC * 4;
+}  // namespace chunk
+
+template <int RULE>
+__global__ void __launch_bounds__(chunk::kThreads, 2) chunk_prep_kernel(const ScanParams p) {
+  using namespace chunk;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const uint32_t sbase = smem_addr(smem);
+  float* sL = reinterpret_cast<float*>(smem + kPOffL);
+  float* sT = reinterpret_cast<float*>(smem + kPOffT);
+  float* sX = reinterpret_cast<float*>(smem + kPOffX);
+  float* sLg = reinterpret_cast<float*>(smem + kPOffG);
+  float* sSg = sLg + kC;
+  float* sBt = sSg + kC;
+  float* sGm = sBt + kC;
+  float* sFa = sGm + kC;
+  float* sFb = sFa + kC;
+  float* gin = reinterpret_cast<float*>(smem + kPOffGin);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g8 = lane >> 2, t4 = lane & 3;
+  const int H = p.n_v_heads;
+  const int ratio_h = H / p.n_qk_heads;
+  const int64_t units = (int64_t)p.n_seqs * H;
+  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(p.k);
+  const int kOffTw2 = kPOffTw, kOffTu2 = kPOffTw + kC * kRow64;
+
+  // the strictly upper 16 x 16 blocks of Tw and Tu are zero in every chunk
+  for (int idx = tid; idx < kC * kC / 2; idx += kThreads) {
+    const int r = idx >> 5, c = 2 * (idx & 31);
+    if ((c >> 4) > (r >> 4)) {
+      const uint32_t off = swz(kOffTw2, r, c >> 3, kRow64) + 2 * (c & 7);
+      st_bf16x2(smem, off, 0.0f, 0.0f);
+      st_bf16x2(smem, off - kOffTw2 + kOffTu2, 0.0f, 0.0f);
+    }
+  }
+  __syncthreads();
+
+#pragma unroll 1
+  for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+    const int seq = (int)(u / H), h = (int)(u % H), hq = h / ratio_h;
+    const int t0 = __ldg(p.cu_seqlens + seq), t1 = __ldg(p.cu_seqlens + seq + 1);
+    if (t0 < 0 || t1 < t0 || t1 > p.total_tokens) continue;  // reported by the main kernel
+    const int n_tok = t1 - t0;
+#pragma unroll 1
+    for (int c0 = 0; c0 < n_tok; c0 += kC) {
+      const int n = (n_tok - c0) < kC ? (n_tok - c0) : kC;
+      // stage K rows (zero beyond the sequence) and the gates ((1, 0) beyond it)
+      for (int idx = tid; idx < kC * 16; idx += kThreads) {
+        const int r = idx >> 4, ch = idx & 15;
+        const uint32_t so = (uint32_t)(kPOffK + r * kRow128 + ((ch ^ (r & 7)) << 4));
+        if (r < n) cp_async_16(smem + so, kg + ((int64_t)(t0 + c0 + r) * p.n_qk_heads + hq) * kD + ch * 8);
+        else *reinterpret_cast<uint4*>(smem + so) = make_uint4(0, 0, 0, 0);
+      }
+      if (warp == 0) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 2 * lane + e;
+          if (t < n) {
+            const int64_t gi = (int64_t)(t0 + c0 + t) * H + h;
+            if (Rule<RULE>::kUsesGate) cp_async_4(gin + t, p.g + gi); else gin[t] = 1.0f;
+            cp_async_4(gin + kC + t, p.beta + gi);
+          } else {
+            gin[t] = 1.0f;
+            gin[kC + t] = 0.0f;
+          }
+        }
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      __syncthreads();
+      // gates: b_t, gamma_t and the ratios gamma_t / gamma_s (as in chunk_scan_kernel)
+      bool fact_l = false;
+      if (warp == 0) {
+        float lg[2], sg[2];
+        bool big = false;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 2 * lane + e;
+          float a, bc, cc;
+          Rule<RULE>::coeffs(gin[t], gin[kC + t], a, bc, cc);
+          big |= fabsf(a) > 1.0f;
+          lg[e] = __logf(fmaxf(fabsf(a), 1e-30f));
+          sg[e] = a < 0.0f ? -1.0f : 1.0f;
+          sBt[t] = bc;
+        }
+        float l = lg[0] + lg[1], sgn = sg[0] * sg[1];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float lo = __shfl_up_sync(0xffffffffu, l, off);
+          const float so2 = __shfl_up_sync(0xffffffffu, sgn, off);
+          if (lane >= off) {
+            l += lo;
+            sgn *= so2;
+          }
+        }
+        const float lprev = l - (lg[0] + lg[1]), sprev = sgn * sg[0] * sg[1];
+        const float l0 = lprev + lg[0], s0 = sprev * sg[0];
+        sLg[2 * lane] = l0;
+        sSg[2 * lane] = s0;
+        sLg[2 * lane + 1] = l;
+        sSg[2 * lane + 1] = sgn;
+        sGm[2 * lane] = s0 * __expf(l0);
+        sGm[2 * lane + 1] = sgn * __expf(l);
+        const float lfirst = __shfl_sync(0xffffffffu, l0, 0), llast = __shfl_sync(0xffffffffu, l, 31);
+        fact_l = !__any_sync(0xffffffffu, big) && (lfirst - llast) <= 80.0f;
+        const float m = 0.5f * (lfirst + llast);
+        sFa[2 * lane] = s0 * __expf(l0 - m);
+        sFb[2 * lane] = s0 * __expf(m - l0);
+        sFa[2 * lane + 1] = sgn * __expf(l - m);
+        sFb[2 * lane + 1] = sgn * __expf(m - l);
+        if (lane == 0) sX[0] = fact_l ? 1.0f : 0.0f;  // (sX is scratch again only in the inverse)
+      }
+      __syncthreads();
+      const bool fact = sX[0] != 0.0f;
+      // L = strictly-lower(b_t gamma_t / gamma_s k_t . k_s): warp w, rows 16 (w & 3), columns 32 (w >> 2)
+      {
+        const int mt = warp & 3, nh2 = warp >> 2;
+        float acc[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+#pragma unroll
+        for (int kk = 0; kk < kD; kk += 16) {
+          uint32_t a[4];
+          lda(a, sbase + kPOffK, kRow128, 16 * mt, kk, lane);
+#pragma unroll
+          for (int np = 0; np < 2; ++np) {
+            uint32_t b[4];
+            ldb_nk(b, sbase + kPOffK, kRow128, 32 * nh2 + 16 * np, kk, lane);
+            mma16816(acc[2 * np], a, b[0], b[1]);
+            mma16816(acc[2 * np + 1], a, b[2], b[3]);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int r = 16 * mt + g8 + (e >> 1) * 8, s_ = 32 * nh2 + 8 * j + 2 * t4 + (e & 1);
+            float v = 0.0f;
+            if (s_ < r) {
+              const float ratio = fact ? sFa[r] * sFb[s_] : sSg[r] * sSg[s_] * __expf(sLg[r] - sLg[s_]);
+              v = sBt[r] * ratio * acc[j][e];
+            }
+            sL[r * kLs + s_] = v;
+          }
+        }
+      }
+      __syncthreads();
+      // diagonal blocks: forward substitution, lane c < 16 of warp b owns column c
+      if (warp < 4) {
+        const int b0 = 16 * warp, c = lane & 15;
+        float col[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const float4* lr = reinterpret_cast<const float4*>(sL + (b0 + r) * kLs + b0);
+          float x = (r == c) ? 1.0f : 0.0f;
+#pragma unroll
+          for (int m = 0; m < (r + 3) / 4; ++m) {
+            const float4 l4 = lr[m];
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (4 * m + e < r) x -= lv[e] * col[4 * m + e];
+          }
+          col[r] = (r < c) ? 0.0f : x;
+        }
+        const int sc = b0 + c;
+        const float fw = sBt[sc] * sGm[sc], fu = sBt[sc];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          if (lane < 16) sT[(b0 + r) * kTs + sc] = col[r];
+          const float nw = __shfl_down_sync(0xffffffffu, col[r] * fw, 1);
+          const float nu = __shfl_down_sync(0xffffffffu, col[r] * fu, 1);
+          if (lane < 16 && (c & 1) == 0) {
+            const uint32_t off = swz(kOffTw2, b0 + r, sc >> 3, kRow64) + 2 * (sc & 7);
+            st_bf16x2(smem, off, col[r] * fw, nw);
+            st_bf16x2(smem, off - kOffTw2 + kOffTu2, col[r] * fu, nu);
+          }
+        }
+      }
+      __syncthreads();
+      // block row bi: T_{bi,j} = -T_{bi,bi} sum_{k=j}^{bi-1} L_{bi,k} T_{k,j}, warp j < bi
+#pragma unroll 1
+      for (int bi = 1; bi < 4; ++bi) {
+        if (warp < bi) {
+          const int bj = warp;
+          const int g = lane >> 2, t = lane & 3;
+          float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+          for (int bk = bj; bk < bi; ++bk)
+            mma16x16x16_tf32(x, sL + (16 * bi) * kLs + 16 * bk, kLs, sT + (16 * bk) * kTs + 16 * bj, kTs, lane);
+          float* xs = sX + warp * 16 * kXs;  // per-warp scratch
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            xs[g * kXs + 8 * nt + 2 * t] = x[nt][0];
+            xs[g * kXs + 8 * nt + 2 * t + 1] = x[nt][1];
+            xs[(g + 8) * kXs + 8 * nt + 2 * t] = x[nt][2];
+            xs[(g + 8) * kXs + 8 * nt + 2 * t + 1] = x[nt][3];
+          }
+          __syncwarp();
+          float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+          mma16x16x16_tf32(y, sT + (16 * bi) * kTs + 16 * bi, kTs, xs, kXs, lane);
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+              const int r = 16 * bi + g + 8 * hlf, c = 16 * bj + 8 * nt + 2 * t;
+              const float v0 = -y[nt][2 * hlf], v1 = -y[nt][2 * hlf + 1];
+              sT[r * kTs + c] = v0;
+              sT[r * kTs + c + 1] = v1;
+              const uint32_t off = swz(kOffTw2, r, c >> 3, kRow64) + 2 * (c & 7);
+              st_bf16x2(smem, off, v0 * sBt[c] * sGm[c], v1 * sBt[c + 1] * sGm[c + 1]);
+              st_bf16x2(smem, off - kOffTw2 + kOffTu2, v0 * sBt[c], v1 * sBt[c + 1]);
+            }
+          }
+        }
+        __syncthreads();
+      }
+      // Tw, Tu to the workspace (16 KB, the swizzled layout as is)
+      uint4* dstw = reinterpret_cast<uint4*>(static_cast<unsigned char*>(const_cast<void*>(p.workspace)) +
+                                             (((int64_t)((t0 + c0) / kC + seq)) * H + h) * kPrepTileBytes);
+      const uint4* srcw = reinterpret_cast<const uint4*>(smem + kPOffTw);
+      for (int idx = tid; idx < kPrepTileBytes / 16; idx += kThreads) dstw[idx] = srcw[idx];
+      __syncthreads();
+    }
+  }
+}
+
+template <int RULE>
+cudaError_t launch_chunk_prep(const ScanParams& p, cudaStream_t stream) {
+  const void* fn = reinterpret_cast<const void*>(&chunk_prep_kernel<RULE>);
+  const int per_sm = prepare_kernel(fn, chunk::kThreads, chunk::kPSmem);
+  if (per_sm <= 0) return cudaErrorInvalidConfiguration;
+  const int64_t units = (int64_t)p.n_seqs * p.n_v_heads;
+  const int64_t cap = (int64_t)device_sm_count() * per_sm;
+  const int grid = (int)(units < cap ? units : cap);
+  chunk_prep_kernel<RULE><<<grid, chunk::kThreads, chunk::kPSmem, stream>>>(p);
+  return cudaGetLastError();
+}
+
 template <int RULE>
 cudaError_t launch_chunk_scan(const ScanParams& p, cudaStream_t stream) {
   const void* fn = reinterpret_cast<const void*>(&chunk_scan_kernel<RULE>);
@@ -621,5 +895,27 @@ cudaError_t launch_chunk_scan(const ScanParams& p, cudaStream_t stream) {
   chunk_scan_kernel<RULE><<<grid, chunk::kThreads, chunk::kSmem, stream>>>(p);
   return cudaGetLastError();
 }
+
+// The chunked prefill in two launches on the stream: the intra-chunk inverses of every
+// chunk (parallel), then the recurrence reading them.  Linear and gated rules have no
+// inverse and take the single fused kernel.
+template <int RULE>
+cudaError_t launch_chunk_scan_ws(const ScanParams& p, cudaStream_t stream) {
+  if constexpr (!Rule<RULE>::kPredicts) {
+    return launch_chunk_scan<RULE>(p, stream);
+  } else {
+    cudaError_t e = launch_chunk_prep<RULE>(p, stream);
+    if (e != cudaSuccess) return e;
+    const void* fn = reinterpret_cast<const void*>(&chunk_scan_kernel<RULE, true>);
+    const int per_sm = prepare_kernel(fn, chunk::kThreads, chunk::kSmem);
+    if (per_sm <= 0) return cudaErrorInvalidConfiguration;
+    const int64_t units = (int64_t)p.n_seqs * p.n_v_heads;
+    const int64_t cap = (int64_t)device_sm_count() * per_sm;
+    const int grid = (int)(units < cap ? units : cap);
+    chunk_scan_kernel<RULE, true><<<grid, chunk::kThreads, chunk::kSmem, stream>>>(p);
+    return cudaGetLastError();
+  }
+}
+
 
 }  // namespace la

@@ -77,6 +77,7 @@ struct ScanParams {
   const float* conv_wv;
   const void* conv_src;     // io dtype [src slots][H_v][2 d_k + d_v][W - 1]
   void* conv_dst;
+  const void* workspace;     // chunked prefill in two launches: the per-chunk Tw / Tu tiles
   const void* q;
   const void* k;
   const void* v;
@@ -131,7 +132,11 @@ ScanLaunchFn find_scan_qgroups_f32io(int rule, int dk, int dv);
 ScanLaunchFn find_scan_qgroups_bf16io(int rule, int dk, int dv);
 
 // Chunked tensor-core prefill (d_k = d_v = 128, BF16 io); nullptr for an unknown rule.
+// The _ws form runs the intra-chunk inverses as a separate launch through ScanParams::workspace.
 ScanLaunchFn find_chunk_scan(int rule);
+ScanLaunchFn find_chunk_scan_ws(int rule);
+// workspace of the _ws form: one 16 KiB tile per (chunk slot, head)
+size_t chunk_workspace_bytes(int64_t total_tokens, int64_t n_seqs, int64_t n_v_heads);
 
 cudaError_t launch_pool_copy(const PoolCopyParams& p, cudaStream_t stream);
 

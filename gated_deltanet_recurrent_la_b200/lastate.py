@@ -30,7 +30,7 @@ DEVERR_READ_SLOT, DEVERR_WRITE_SLOT, DEVERR_CU_SEQLENS, DEVERR_TIMEOUT, DEVERR_Q
 EXPORTS = ("la_state_bytes", "la_shape_supported", "la_state_step", "la_state_scan", "la_state_scan_chunked",
            "la_state_scan_checkpointed", "la_state_step_qgroups", "la_state_scan_qgroups",
            "la_pool_slot_bytes", "la_state_pool_encode", "la_state_pool_decode", "la_state_step_conv",
-           "la_state_scan_conv",
+           "la_state_scan_conv", "la_scan_chunked_workspace_bytes", "la_state_scan_chunked_ws",
            "la_state_pool_copy",
            "la_state_pool_gather", "la_state_pool_scatter", "la_state_pool_zero", "la_state_check_slots",
            "la_status_str", "la_last_cuda_error", "la_abi_version")
@@ -102,6 +102,10 @@ def lib():
         L.la_state_scan_conv.argtypes = L.la_state_scan.argtypes[:9] + [ctypes.POINTER(la_conv)] + \
             L.la_state_scan.argtypes[9:]
         L.la_state_scan_conv.restype = I32
+        L.la_scan_chunked_workspace_bytes.argtypes = [I32, I32, I32]
+        L.la_scan_chunked_workspace_bytes.restype = ctypes.c_size_t
+        L.la_state_scan_chunked_ws.argtypes = L.la_state_scan.argtypes[:-2] + [P, ctypes.c_size_t, P, P]
+        L.la_state_scan_chunked_ws.restype = I32
         L.la_pool_slot_bytes.argtypes = [PP]
         L.la_pool_slot_bytes.restype = ctypes.c_size_t
         L.la_state_pool_encode.argtypes = [PP, I32, P, P, P, P]
@@ -222,6 +226,24 @@ def la_state_scan_chunked(rule, src: Optional[Pool], read_slot, dst: Pool, write
                                        _ptr(q), _ptr(k, q.dtype), _ptr(v, q.dtype), io, _ptr(g, torch.float32),
                                        _ptr(beta, torch.float32), float(scale), _ptr(o, q.dtype),
                                        _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_scan_chunked_workspace_bytes(total_tokens: int, n_seqs: int, n_v_heads: int) -> int:
+    return lib().la_scan_chunked_workspace_bytes(int(total_tokens), int(n_seqs), int(n_v_heads))
+
+
+def la_state_scan_chunked_ws(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens, q, k, v, g,
+                             beta, scale, o, workspace, err_word, seq_order=None, stream=None) -> int:
+    """la_state_scan_chunked in two launches; workspace: a uint8 device tensor of at least
+    la_scan_chunked_workspace_bytes(...) bytes."""
+    io = dtype_code(q.dtype)
+    return lib().la_state_scan_chunked_ws(
+        RULES[rule] if isinstance(rule, str) else int(rule), None if src is None else src.ref,
+        _ptr(read_slot, torch.int32), dst.ref, _ptr(write_slot, torch.int32), int(cu_seqlens.numel() - 1),
+        _ptr(cu_seqlens, torch.int32), int(q.shape[0]), _ptr(seq_order, torch.int32), _ptr(q), _ptr(k, q.dtype),
+        _ptr(v, q.dtype), io, _ptr(g, torch.float32), _ptr(beta, torch.float32), float(scale), _ptr(o, q.dtype),
+        _ptr(workspace), int(workspace.numel() * workspace.element_size()), _ptr(err_word, torch.int32),
+        _stream(stream))
 
 
 def la_state_scan_checkpointed(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens, q, k, v, g,

@@ -215,6 +215,27 @@ la_status la_state_scan_chunked(la_rule rule, const la_pool *src, const int32_t 
                                 const float *g, const float *beta, float scale, void *o,
                                 int32_t *err_word, void *stream);
 
+/* la_state_scan_chunked in two launches: the intra-chunk part of every chunk (K K^T, the
+ * triangular inverse, Tw = T diag(beta gamma), Tu = T diag(beta)) as one parallel launch
+ * writing a caller-owned workspace, then the recurrence over the chunks reading it.  The
+ * chunks are independent in the first launch, so it fills the SMs (several CTAs each)
+ * instead of sitting on each sequence's critical path.  Same results as
+ * la_state_scan_chunked (the same arithmetic, bit for bit).
+ *   workspace        device, 16-byte aligned, at least
+ *                    la_scan_chunked_workspace_bytes(total_tokens, n_seqs, H_v) bytes;
+ *                    contents are scratch (overwritten, not read back by the caller)
+ * Other arguments, supported set and errors as la_state_scan_chunked; LA_ERR_SHAPE when
+ * workspace_bytes is too small, LA_ERR_NULL for a NULL workspace.  The linear and gated
+ * rules have no inverse and run the one-launch form (the workspace is not touched). */
+size_t la_scan_chunked_workspace_bytes(int32_t total_tokens, int32_t n_seqs, int32_t n_v_heads);
+la_status la_state_scan_chunked_ws(la_rule rule, const la_pool *src, const int32_t *read_slot,
+                                   const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
+                                   const int32_t *cu_seqlens, int32_t total_tokens,
+                                   const int32_t *seq_order, const void *q, const void *k,
+                                   const void *v, la_dtype io, const float *g, const float *beta,
+                                   float scale, void *o, void *workspace, size_t workspace_bytes,
+                                   int32_t *err_word, void *stream);
+
 /* The scan of la_state_scan that also stores intermediate states: the prefix-cache
  * checkpoints at KV-cache block boundaries of the "Gated DeltaNet" glossary page (Why
  * it matters), and state snapshots for speculative-decoding rollback ("Seven

@@ -468,6 +468,44 @@ def test_chunked_scan_wide_gate_and_beta_ranges():
     assert_close(np64(o), o_ref, 2e-2, "wide-range outputs")
 
 
+def _gpu_scan_chunked_ws(inp, dst_dtype):
+    n_seqs = inp.cu_seqlens.numel() - 1
+    dst_t = torch.full((n_seqs, inp.n_v_heads, inp.d_k, inp.d_v), 3.0, dtype=dst_dtype, device="cuda")
+    src = None if inp.pool is None else L.Pool(dev(inp.pool), inp.n_qk_heads)
+    o = torch.full((inp.q.shape[0], inp.n_v_heads, inp.d_v), 5.0, dtype=inp.io_dtype, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nbytes = L.la_scan_chunked_workspace_bytes(inp.q.shape[0], n_seqs, inp.n_v_heads)
+    ws = torch.full((nbytes,), 0xAB, dtype=torch.uint8, device="cuda")
+    st = L.la_state_scan_chunked_ws(inp.rule, src, dev(inp.read_slot), L.Pool(dst_t, inp.n_qk_heads), None,
+                                    dev(inp.cu_seqlens), dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.g),
+                                    dev(inp.beta), inp.scale, o, ws, err)
+    L.check(st)
+    torch.cuda.synchronize()
+    return dst_t.cpu(), o.cpu(), int(err.item())
+
+
+@pytest.mark.parametrize("rule", W.RULES)
+def test_chunked_two_launches_match_one_bitwise(rule):
+    """The two-launch form (intra-chunk inverses through the workspace) gives the fused
+    kernel's bits, and both match the oracle; the workspace size check is enforced."""
+    inp = W.scan_inputs(lengths=[100, 64, 1, 0, 200, 63, 129], n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128,
+                        rule=rule, io_dtype=BF16, seed=43, init="slots", init_dtype=F32, scale=0.8)
+    S1, o1, e1 = _gpu_scan_chunked(inp, F32)
+    S2, o2, e2 = _gpu_scan_chunked_ws(inp, F32)
+    assert e1 == e2 == 0
+    assert torch.equal(S1, S2) and torch.equal(o1, o2)
+    S_ref, o_ref, _ = oracle_scan(inp, dst_dtype=F32)
+    assert_close(np64(S2), S_ref, 2e-2, f"{rule}: final states")
+    assert_close(np64(o2), o_ref, 2e-2, f"{rule}: outputs")
+    small = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    dst_t = torch.zeros(7, 4, 128, 128, dtype=F32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = L.la_state_scan_chunked_ws(rule, None, None, L.Pool(dst_t, 2), None, dev(inp.cu_seqlens), dev(inp.q),
+                                    dev(inp.k), dev(inp.v), dev(inp.g), dev(inp.beta), 1.0,
+                                    torch.empty_like(dev(inp.v)), small, err)
+    assert st == L.LA_ERR_SHAPE
+
+
 def test_chunked_prefill32_sampled():
     inp = W.prefill32()
     S, o, err = _gpu_scan_chunked(inp, BF16)
