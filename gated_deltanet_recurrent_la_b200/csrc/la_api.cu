@@ -389,6 +389,18 @@ la_status la_state_scan_chunked_ws(la_rule rule, const la_pool* src, const int32
                    workspace_bytes);
 }
 
+la_status la_state_scan_chunked_noalloc(la_rule rule, const la_pool* src, const int32_t* read_slot,
+                                        const la_pool* dst, const int32_t* write_slot, int32_t n_seqs,
+                                        const int32_t* cu_seqlens, int32_t total_tokens, const int32_t* seq_order,
+                                        const void* q, const void* k, const void* v, la_dtype io, const float* g,
+                                        const float* beta, float scale, void* o, int32_t* err_word, void* stream) {
+  size_t bytes = 0;
+  void* ws = la::chunk_noalloc_workspace(&bytes);
+  if (!ws) return cuda_status(cudaGetLastError() != cudaSuccess ? cudaGetLastError() : cudaErrorUnknown);
+  return la_state_scan_chunked_ws(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order,
+                                  q, k, v, io, g, beta, scale, o, ws, bytes, err_word, stream);
+}
+
 la_status la_state_scan_checkpointed(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
                                      const int32_t* write_slot, int32_t n_seqs, const int32_t* cu_seqlens,
                                      int32_t total_tokens, const int32_t* seq_order, const void* q, const void* k,

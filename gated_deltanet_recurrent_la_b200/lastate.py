@@ -31,6 +31,7 @@ EXPORTS = ("la_state_bytes", "la_shape_supported", "la_state_step", "la_state_sc
            "la_state_scan_checkpointed", "la_state_step_qgroups", "la_state_scan_qgroups",
            "la_pool_slot_bytes", "la_state_pool_encode", "la_state_pool_decode", "la_state_step_conv",
            "la_state_scan_conv", "la_scan_chunked_workspace_bytes", "la_state_scan_chunked_ws",
+           "la_state_scan_chunked_noalloc",
            "la_state_pool_copy",
            "la_state_pool_gather", "la_state_pool_scatter", "la_state_pool_zero", "la_state_check_slots",
            "la_status_str", "la_last_cuda_error", "la_abi_version")
@@ -106,6 +107,8 @@ def lib():
         L.la_scan_chunked_workspace_bytes.restype = ctypes.c_size_t
         L.la_state_scan_chunked_ws.argtypes = L.la_state_scan.argtypes[:-2] + [P, ctypes.c_size_t, P, P]
         L.la_state_scan_chunked_ws.restype = I32
+        L.la_state_scan_chunked_noalloc.argtypes = L.la_state_scan.argtypes
+        L.la_state_scan_chunked_noalloc.restype = I32
         L.la_pool_slot_bytes.argtypes = [PP]
         L.la_pool_slot_bytes.restype = ctypes.c_size_t
         L.la_state_pool_encode.argtypes = [PP, I32, P, P, P, P]
@@ -244,6 +247,18 @@ def la_state_scan_chunked_ws(rule, src: Optional[Pool], read_slot, dst: Pool, wr
         _ptr(v, q.dtype), io, _ptr(g, torch.float32), _ptr(beta, torch.float32), float(scale), _ptr(o, q.dtype),
         _ptr(workspace), int(workspace.numel() * workspace.element_size()), _ptr(err_word, torch.int32),
         _stream(stream))
+
+
+def la_state_scan_chunked_noalloc(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens, q, k, v,
+                                  g, beta, scale, o, err_word, seq_order=None, stream=None) -> int:
+    """la_state_scan_chunked_ws with the library's own fixed workspace (no scratch argument)."""
+    io = dtype_code(q.dtype)
+    return lib().la_state_scan_chunked_noalloc(
+        RULES[rule] if isinstance(rule, str) else int(rule), None if src is None else src.ref,
+        _ptr(read_slot, torch.int32), dst.ref, _ptr(write_slot, torch.int32), int(cu_seqlens.numel() - 1),
+        _ptr(cu_seqlens, torch.int32), int(q.shape[0]), _ptr(seq_order, torch.int32), _ptr(q), _ptr(k, q.dtype),
+        _ptr(v, q.dtype), io, _ptr(g, torch.float32), _ptr(beta, torch.float32), float(scale), _ptr(o, q.dtype),
+        _ptr(err_word, torch.int32), _stream(stream))
 
 
 def la_state_scan_checkpointed(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens, q, k, v, g,

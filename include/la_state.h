@@ -236,6 +236,20 @@ la_status la_state_scan_chunked_ws(la_rule rule, const la_pool *src, const int32
                                    float scale, void *o, void *workspace, size_t workspace_bytes,
                                    int32_t *err_word, void *stream);
 
+/* la_state_scan_chunked_ws with the library's own workspace: a fixed 256 MiB device array
+ * of this library (one per device), so the caller passes no scratch buffer.  The array is
+ * shared by every call on a device: calls must not run concurrently on one device (the
+ * caller orders them, for example on one stream).  A call whose workspace would exceed
+ * the array (la_scan_chunked_workspace_bytes(total_tokens, n_seqs, H_v) > 256 MiB) returns
+ * LA_ERR_SHAPE before launching anything.  Other arguments and errors as
+ * la_state_scan_chunked. */
+la_status la_state_scan_chunked_noalloc(la_rule rule, const la_pool *src, const int32_t *read_slot,
+                                        const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
+                                        const int32_t *cu_seqlens, int32_t total_tokens,
+                                        const int32_t *seq_order, const void *q, const void *k,
+                                        const void *v, la_dtype io, const float *g, const float *beta,
+                                        float scale, void *o, int32_t *err_word, void *stream);
+
 /* The scan of la_state_scan that also stores intermediate states: the prefix-cache
  * checkpoints at KV-cache block boundaries of the "Gated DeltaNet" glossary page (Why
  * it matters), and state snapshots for speculative-decoding rollback ("Seven
