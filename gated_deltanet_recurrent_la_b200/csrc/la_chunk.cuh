@@ -359,8 +359,43 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
       __syncthreads();
       const bool fact = sFlag[0] != 0;
 
-      // ---- step 1: K K^T (warps 0-3, delta rules) and Q K^T (warps 4-7), rows [16 mt, +16)
-      if ((kDelta && !PRE) || warp >= 4) {
+      // ---- step 1: K K^T (warps 0-3, delta rules) and Q K^T (warps 4-7), rows [16 mt, +16).
+      //      PRE (no K K^T here): Q K^T over all 8 warps, rows 16 (warp & 3), columns
+      //      32 (warp >> 2), and no barrier before step 3, which does not read it
+      if constexpr (PRE) {
+        const int nh2 = warp >> 2;
+        float acc[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+#pragma unroll
+        for (int kk = 0; kk < kD; kk += 16) {
+          uint32_t a[4];
+          lda(a, sbase + kOffQ, kRow128, 16 * mt, kk, lane);
+#pragma unroll
+          for (int np = 0; np < 2; ++np) {
+            uint32_t b[4];
+            ldb_nk(b, sbase + kOffK, kRow128, 32 * nh2 + 16 * np, kk, lane);
+            mma16816(acc[2 * np], a, b[0], b[1]);
+            mma16816(acc[2 * np + 1], a, b[2], b[3]);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+          for (int e = 0; e < 4; e += 2) {
+            const int r = 16 * mt + g8 + (e >> 1) * 8;
+            float v2[2];
+#pragma unroll
+            for (int f = 0; f < 2; ++f) {
+              const int s_ = 32 * nh2 + 8 * j + 2 * t4 + f;
+              v2[f] = 0.0f;
+              if (s_ <= r)
+                v2[f] = (fact ? sFa[r] * sFb[s_] : sSg[r] * sSg[s_] * __expf(sLg[r] - sLg[s_])) * acc[j][e + f];
+            }
+            st_bf16x2(smem, swz(kOffP, r, 4 * nh2 + j, kRow64) + 4 * t4, v2[0], v2[1]);
+          }
+        }
+      } else if (kDelta || warp >= 4) {
         float acc[8][4];
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
@@ -401,7 +436,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
           }
         }
       }
-      __syncthreads();
+      if (!PRE) __syncthreads();
 
       // ---- step 2 (delta rules): T = (I + L)^-1 by 16 x 16 blocks, written as FP32 (for the
       //      block recursion) and as Tw = T diag(b gamma), Tu = T diag(b) (BF16, swizzled)
@@ -639,14 +674,14 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
 //      and hide each other's latency.  Chunk c of sequence s goes to workspace tile
 //      (t0_s + 64 c) / 64 + s (distinct for every chunk; fewer than T / 64 + n_seqs + 1).
 namespace chunk {
-constexpr int kPOffK = 0;                           // [64][128] bf16, swizzled
-constexpr int kPOffL = kPOffK + kC * kRow128;       // [64][68] fp32
+constexpr int kPOffK = 0;                           // 2 x [64][128] bf16, swizzled (double buffer)
+constexpr int kPOffL = kPOffK + 2 * kC * kRow128;   // [64][68] fp32
 constexpr int kPOffT = kPOffL + kC * kLs * 4;       // [64][72] fp32
 constexpr int kPOffTw = kPOffT + kC * kTs * 4;      // Tw, Tu [64][64] bf16, swizzled
 constexpr int kPOffX = kPOffTw + kPrepTileBytes;    // [3][16][24] fp32
 constexpr int kPOffG = kPOffX + 3 * 16 * kXs * 4;   // per token gate quantities [6][64]
-constexpr int kPOffGin = kPOffG + 6 * kC * 4;       // g, beta [2][64]
-constexpr int kPSmem = kPOffGin + 2 * kC * 4;
+constexpr int kPOffGin = kPOffG + 6 * kC * 4;       // 2 x g, beta [2][64] (double buffer)
+constexpr int kPSmem = kPOffGin + 2 * 2 * kC * 4;
 }  // namespace chunk
 
 template <int RULE>
@@ -689,33 +724,46 @@ __global__ void __launch_bounds__(chunk::kThreads, 2) chunk_prep_kernel(const Sc
     const int t0 = __ldg(p.cu_seqlens + seq), t1 = __ldg(p.cu_seqlens + seq + 1);
     if (t0 < 0 || t1 < t0 || t1 > p.total_tokens) continue;  // reported by the main kernel
     const int n_tok = t1 - t0;
-#pragma unroll 1
-    for (int c0 = 0; c0 < n_tok; c0 += kC) {
-      const int n = (n_tok - c0) < kC ? (n_tok - c0) : kC;
-      // stage K rows (zero beyond the sequence) and the gates ((1, 0) beyond it)
+    // stages the chunk at token c0s into buffer bs: K rows (zero beyond the sequence) and
+    // the gates ((1, 0) beyond it)
+    auto stage = [&](int c0s, int bs) {
+      const int ns = (n_tok - c0s) < kC ? (n_tok - c0s) : kC;
       for (int idx = tid; idx < kC * 16; idx += kThreads) {
         const int r = idx >> 4, ch = idx & 15;
-        const uint32_t so = (uint32_t)(kPOffK + r * kRow128 + ((ch ^ (r & 7)) << 4));
-        if (r < n) cp_async_16(smem + so, kg + ((int64_t)(t0 + c0 + r) * p.n_qk_heads + hq) * kD + ch * 8);
+        const uint32_t so = (uint32_t)(kPOffK + bs * kC * kRow128 + r * kRow128 + ((ch ^ (r & 7)) << 4));
+        if (r < ns) cp_async_16(smem + so, kg + ((int64_t)(t0 + c0s + r) * p.n_qk_heads + hq) * kD + ch * 8);
         else *reinterpret_cast<uint4*>(smem + so) = make_uint4(0, 0, 0, 0);
       }
       if (warp == 0) {
+        float* gs = gin + bs * 2 * kC;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int t = 2 * lane + e;
-          if (t < n) {
-            const int64_t gi = (int64_t)(t0 + c0 + t) * H + h;
-            if (Rule<RULE>::kUsesGate) cp_async_4(gin + t, p.g + gi); else gin[t] = 1.0f;
-            cp_async_4(gin + kC + t, p.beta + gi);
+          if (t < ns) {
+            const int64_t gi = (int64_t)(t0 + c0s + t) * H + h;
+            if (Rule<RULE>::kUsesGate) cp_async_4(gs + t, p.g + gi); else gs[t] = 1.0f;
+            cp_async_4(gs + kC + t, p.beta + gi);
           } else {
-            gin[t] = 1.0f;
-            gin[kC + t] = 0.0f;
+            gs[t] = 1.0f;
+            gs[kC + t] = 0.0f;
           }
         }
       }
       cp_async_commit();
-      cp_async_wait<0>();
+    };
+    if (n_tok > 0) stage(0, 0);
+#pragma unroll 1
+    for (int c0 = 0, it = 0; c0 < n_tok; c0 += kC, ++it) {
+      const int buf = it & 1;
+      if (c0 + kC < n_tok) {  // the next chunk's copies fly while this one is worked on
+        stage(c0 + kC, buf ^ 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
       __syncthreads();
+      const float* gb = gin + buf * 2 * kC;
+      const uint32_t kbase = sbase + kPOffK + buf * kC * kRow128;
       // gates: b_t, gamma_t and the ratios gamma_t / gamma_s (as in chunk_scan_kernel)
       bool fact_l = false;
       if (warp == 0) {
@@ -725,7 +773,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 2) chunk_prep_kernel(const Sc
         for (int e = 0; e < 2; ++e) {
           const int t = 2 * lane + e;
           float a, bc, cc;
-          Rule<RULE>::coeffs(gin[t], gin[kC + t], a, bc, cc);
+          Rule<RULE>::coeffs(gb[t], gb[kC + t], a, bc, cc);
           big |= fabsf(a) > 1.0f;
           lg[e] = __logf(fmaxf(fabsf(a), 1e-30f));
           sg[e] = a < 0.0f ? -1.0f : 1.0f;
@@ -769,11 +817,11 @@ __global__ void __launch_bounds__(chunk::kThreads, 2) chunk_prep_kernel(const Sc
 #pragma unroll
         for (int kk = 0; kk < kD; kk += 16) {
           uint32_t a[4];
-          lda(a, sbase + kPOffK, kRow128, 16 * mt, kk, lane);
+          lda(a, kbase, kRow128, 16 * mt, kk, lane);
 #pragma unroll
           for (int np = 0; np < 2; ++np) {
             uint32_t b[4];
-            ldb_nk(b, sbase + kPOffK, kRow128, 32 * nh2 + 16 * np, kk, lane);
+            ldb_nk(b, kbase, kRow128, 32 * nh2 + 16 * np, kk, lane);
             mma16816(acc[2 * np], a, b[0], b[1]);
             mma16816(acc[2 * np + 1], a, b[2], b[3]);
           }
