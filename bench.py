@@ -122,6 +122,7 @@ KERNEL_SOURCES = {
     "step": ["la_step.cuh", "la_device.cuh"],
     "scan": ["la_scan.cuh", "la_device.cuh"],
     "chunk": ["la_chunk.cuh", "la_device.cuh"],
+    "chunk_tc": ["la_chunk.cuh", "la_chunk_tc.cuh", "la_umma.cuh", "la_device.cuh"],
     "pool": ["la_pool.cu"],
 }
 
@@ -373,16 +374,24 @@ def chunk_mma_flops(lengths, n_v_heads, d_k, d_v, rule):
 
 
 def tensor_roofline(run, inp, ms, peaks):
-    """Roofline object of the chunked prefill: executed MMA flops against the measured dense
-    BF16 peak (a cuBLAS GEMM, tcgen05); this kernel issues mma.sync."""
+    """Roofline object of the chunked prefill: the chunked algorithm's MMA flops against the
+    measured dense BF16 peak (a cuBLAS GEMM on tcgen05).  The one-launch kernel issues
+    mma.sync; the two-launch form runs its recurrence on tcgen05 (delta rules)."""
     lens = (inp.cu_seqlens[1:] - inp.cu_seqlens[:-1]).tolist()
     tf = chunk_mma_flops(lens, inp.n_v_heads, inp.d_k, inp.d_v, inp.rule) / (ms * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)
-    return {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-            "traffic": recorded_traffic("chunk", "prefill32"),
-            "peak_note": "measured dense BF16 GEMM (MEASURED_PEAKS.json bf16_tflops); the kernel uses mma.sync "
-                         "BF16 m16n8k16, whose own ceiling on this part is about a third of that",
-            "hbm_gb_s": run.bytes_flops()[0] / (ms * 1e-3) / 1e9, "kernel": "la::chunk_scan_kernel"}
+    two = run.ws is not None and inp.rule in ("delta", "gated_delta")
+    out = {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+           "traffic": recorded_traffic("chunk_tc" if two else "chunk", "prefill32"),
+           "hbm_gb_s": run.bytes_flops()[0] / (ms * 1e-3) / 1e9}
+    if two:
+        out["kernel"] = "la::chunk_prep_kernel (mma.sync) + la::chunk_tc_kernel (tcgen05)"
+        out["peak_note"] = "measured dense BF16 GEMM (MEASURED_PEAKS.json bf16_tflops); both launches together"
+    else:
+        out["kernel"] = "la::chunk_scan_kernel"
+        out["peak_note"] = ("measured dense BF16 GEMM (MEASURED_PEAKS.json bf16_tflops); the kernel uses mma.sync "
+                            "BF16 m16n8k16, whose own ceiling on this part is about a third of that")
+    return out
 
 
 class ScanRunner:
@@ -776,7 +785,8 @@ def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_ev
             row["config"]["checkpoints"] = run.n_ckpt
         if chunked:
             row["config"]["algorithm"] = "chunked (64-token WY/UT form, BF16 tensor-core products)" + \
-                ("; intra-chunk inverses as a separate parallel launch through a workspace" if chunked == "ws" else "")
+                ("; intra-chunk inverses as a separate parallel launch through a workspace, the recurrence on "
+                 "tcgen05 with the state in tensor memory" if chunked == "ws" else "")
             row["hbm"] = {"achieved_gb_s": row["gb_s"], "frac_of_measured": row["gb_s"] / peaks["hbm_gbs"]}
             row["token_serial_equivalent_tflops"] = tf  # 6 flops per state element per token, for comparison
             row["roofline"] = tensor_roofline(run, inp, ms, peaks)

@@ -1,5 +1,6 @@
 // la_chunk.cu -- chunked tensor-core prefill kernels (all four rules); see la_chunk.cuh.
 #include "la_chunk.cuh"
+#include "la_chunk_tc.cuh"
 
 namespace la {
 ScanLaunchFn find_chunk_scan(int rule) {
@@ -17,12 +18,21 @@ size_t chunk_workspace_bytes(int64_t total_tokens, int64_t n_seqs, int64_t n_v_h
   return (size_t)(tiles * n_v_heads * chunk::kPrepTileBytes);
 }
 
+// The delta rules: the intra-chunk inverses of every chunk (parallel launch), then the
+// recurrence on the fifth-generation tensor cores reading them.
+template <int RULE>
+cudaError_t launch_chunk_scan_ws_tc(const ScanParams& p, cudaStream_t stream) {
+  cudaError_t e = launch_chunk_prep<RULE>(p, stream);
+  if (e != cudaSuccess) return e;
+  return launch_chunk_tc<RULE>(p, stream);
+}
+
 ScanLaunchFn find_chunk_scan_ws(int rule) {
   switch (rule) {
     case LA_RULE_LINEAR: return &launch_chunk_scan_ws<LA_RULE_LINEAR>;
     case LA_RULE_GATED: return &launch_chunk_scan_ws<LA_RULE_GATED>;
-    case LA_RULE_DELTA: return &launch_chunk_scan_ws<LA_RULE_DELTA>;
-    case LA_RULE_GATED_DELTA: return &launch_chunk_scan_ws<LA_RULE_GATED_DELTA>;
+    case LA_RULE_DELTA: return &launch_chunk_scan_ws_tc<LA_RULE_DELTA>;
+    case LA_RULE_GATED_DELTA: return &launch_chunk_scan_ws_tc<LA_RULE_GATED_DELTA>;
   }
   return nullptr;
 }

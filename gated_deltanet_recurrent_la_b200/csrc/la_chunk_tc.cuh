@@ -1,0 +1,490 @@
+// la_chunk_tc.cuh -- the recurrence of the two-launch chunked prefill on the
+// fifth-generation tensor cores (tcgen05), for the delta rules.
+//
+// Same algebra as la_chunk.cuh ("Seven Architectures Replacing KV Cache With Bounded
+// Mutable State": the "Kimi Linear" section's chunkwise-parallel kernel and the "Gated
+// DeltaNet-2" section's chunkwise WY algorithm).  chunk_prep_kernel has already written
+// Tw = T diag(b gamma) and Tu = T diag(b) of every 64-token chunk to the workspace; per
+// chunk this kernel forms
+//
+//   P   = (Q K^T) (.) M                         M_ts = gamma_t / gamma_s, s <= t
+//   U^T = V^T Tu^T - S0^T W^T,   W^T = K^T Tw^T
+//   O^T = scale ( S0^T Q^T diag(gamma) + U^T P^T )
+//   S^T = gamma_C S0^T + Us^T K,  Us = diag(gamma_C / gamma) U
+//
+// with every product an M = 128 tcgen05 MMA (M runs over d_v, d_k or the stacked rows of
+// Q and K), BF16 operands from shared memory and FP32 accumulators in tensor memory.  The
+// transposed forms put one d_v (or d_k) index in each tensor-memory lane, so the thread
+// that owns a lane writes whole operand rows back to shared memory.  The master state
+// S^T (d_v lanes x d_k columns, FP32) stays in tensor memory for the whole sequence.
+//
+// One CTA of 8 warps per SM; warp w reads tensor-memory lanes 32 (w % 4) .. + 31 and the
+// column half w / 4 of each accumulator.  Thread 0 issues the MMAs; three mbarriers signal
+// their completion, and every wait gives up after a time limit (LA_DEVERR_TIMEOUT).
+#pragma once
+
+#include <cstdint>
+
+#include "la_chunk.cuh"
+#include "la_umma.cuh"
+
+namespace la {
+namespace chunk_tc {
+
+constexpr int kC = 64;   // tokens per chunk
+constexpr int kD = 128;  // d_k = d_v
+constexpr int kThreads = 256;
+
+// shared memory (bytes from a 1024-byte aligned base); operands in 64-column panels
+constexpr int kBufBytes = 65536;             // one staged chunk:
+constexpr int kOffQK = 0;                    //   Q rows 0..63 and K rows 64..127, [128][128]
+constexpr int kOffV = 32768;                 //   V [64][128]
+constexpr int kOffTw = 49152;                //   Tw [64][64]
+constexpr int kOffTu = 57344;                //   Tu [64][64]
+constexpr int kOffS = 2 * kBufBytes;         // S0^T  [128 d_v][128 d_k] BF16
+constexpr int kOffW = kOffS + 32768;         // W^T   [128 d_k][64]
+constexpr int kOffP = kOffW + 16384;         // P     [64][64]
+constexpr int kOffU = kOffP + 8192;          // U^T   [128 d_v][64]
+constexpr int kOffUs = kOffU + 16384;        // Us^T  [128 d_v][64]
+constexpr int kOffG = kOffUs + 16384;        // per token: log|gamma|, sign, gamma, A, B, gamma_C/gamma
+constexpr int kOffGin = kOffG + 6 * kC * 4;  // 2 x {g, beta}[64] (staged gates)
+constexpr int kOffBar = kOffGin + 2 * 2 * kC * 4;
+constexpr int kOffMisc = kOffBar + 3 * 8;    // [0] tensor-memory base, [2] factored ratios
+constexpr int kSmem = kOffMisc + 16 + 1024;  // + slack for the 1024-byte alignment
+static_assert(kSmem <= 227 * 1024, "shared memory");
+static_assert(chunk::kPrepTileBytes == 16384 && kOffTu == kOffTw + 8192, "workspace tile = Tw then Tu");
+
+// tensor-memory columns (FP32 accumulators, 128 lanes each)
+constexpr uint32_t kTmemCols = 512;
+constexpr int kColS = 0;     // S^T   128 columns (d_k)
+constexpr int kColP = 128;   // [Q; K] K^T, 64 columns (lanes 0..63 are Q K^T)
+constexpr int kColW = 192;   // W^T   64
+constexpr int kColU = 256;   // U^T   64
+constexpr int kColO1 = 320;  // S0^T Q^T   64
+constexpr int kColO2 = 384;  // U^T P^T    64
+
+__device__ __forceinline__ uint4 pack8(const uint32_t* r) {
+  return make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                    pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                    pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                    pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+}
+
+}  // namespace chunk_tc
+
+template <int RULE>
+__global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const ScanParams p) {
+  using namespace chunk_tc;
+  static_assert(Rule<RULE>::kPredicts, "the delta rules only");
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  unsigned char* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t sb = smem_addr(smem);
+  float* sLg = reinterpret_cast<float*>(smem + kOffG);  // log |gamma_t|
+  float* sSg = sLg + kC;                                // sign gamma_t
+  float* sGm = sSg + kC;                                // gamma_t
+  float* sFa = sGm + kC;                                // gamma_t / e^m
+  float* sFb = sFa + kC;                                // e^m / gamma_t
+  float* sGu = sFb + kC;                                // gamma_C / gamma_t
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
+
+  constexpr bool kGate = Rule<RULE>::kUsesGate;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int q4 = warp & 3;         // tensor-memory lane quarter
+  const int hf = warp >> 2;        // column half
+  const int lrow = 32 * q4 + lane; // this thread's lane: a d_v (or d_k, or token) index
+  const int H = p.n_v_heads;
+  const int ratio_h = H / p.n_qk_heads;
+  const int64_t units = (int64_t)p.n_seqs * H;
+  const int64_t G = gridDim.x;
+  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
+  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(p.k);
+  const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(p.v);
+  __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.o);
+
+  if (warp == 0) umma::alloc(const_cast<uint32_t*>(misc), kTmemCols);
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    mbar_init(&bars[2], 1);
+    mbar_init_fence();
+  }
+  umma::fence_before();
+  __syncthreads();
+  umma::fence_after();
+  const uint32_t tmem = misc[0];
+  const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);  // this warp's lane quarter
+  uint32_t phase = 0;  // chunks completed by this CTA: the parity of all three barriers
+  bool abort = false;
+
+  // instruction descriptors
+  constexpr uint32_t kIdKK64 = umma::idesc_bf16(128, 64, false, false);
+  constexpr uint32_t kIdMK64 = umma::idesc_bf16(128, 64, true, false);
+  constexpr uint32_t kIdKM64n = umma::idesc_bf16(128, 64, false, true, true);
+  constexpr uint32_t kIdKM128 = umma::idesc_bf16(128, 128, false, true);
+
+#pragma unroll 1
+  for (int64_t round = 0; round * G < units; ++round) {
+    const int64_t u = round * G + ((round & 1) ? (G - 1 - blockIdx.x) : blockIdx.x);
+    if (u >= units) continue;
+    const int64_t si = u / H;
+    const int h = (int)(u % H);
+    const int hq = h / ratio_h;
+    const int seq = p.seq_order ? __ldg(p.seq_order + si) : (int)si;
+    if (seq < 0 || seq >= p.n_seqs) {
+      if (tid == 0) report(p.err, LA_DEVERR_CU_SEQLENS);
+      continue;
+    }
+    const int t0 = __ldg(p.cu_seqlens + seq);
+    const int t1 = __ldg(p.cu_seqlens + seq + 1);
+    if (seq == 0 && h == 0 && t0 != 0 && tid == 0) report(p.err, LA_DEVERR_CU_SEQLENS);
+    if (t0 < 0 || t1 < t0 || t1 > p.total_tokens) {
+      if (tid == 0) report(p.err, LA_DEVERR_CU_SEQLENS);
+      continue;
+    }
+    const int rs = p.read_slot ? __ldg(p.read_slot + seq) : 0;
+    const int ws = p.write_slot ? __ldg(p.write_slot + seq) : seq;
+    const bool rs_ok = !p.read_slot || (rs >= 0 && rs < p.src_slots);
+    const bool ws_ok = ws >= 0 && ws < p.dst_slots;
+    if (!rs_ok || !ws_ok) {
+      if (tid == 0) report(p.err, (rs_ok ? 0u : LA_DEVERR_READ_SLOT) | (ws_ok ? 0u : LA_DEVERR_WRITE_SLOT));
+      continue;
+    }
+
+    // ---- initial state S^T into tensor memory: lane = d_v index, columns = d_k (64 per half)
+    const int64_t sbase_src = ((int64_t)rs * H + h) * (kD * kD);
+#pragma unroll 1
+    for (int c16 = 0; c16 < 4; ++c16) {
+      uint32_t r[16];
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const int i = 64 * hf + 16 * c16 + x;
+        float s = 0.0f;
+        if (p.read_slot) {
+          const int64_t e = sbase_src + (int64_t)i * kD + lrow;
+          s = p.src_dtype == LA_F32 ? static_cast<const float*>(p.src)[e]
+                                    : __bfloat162float(static_cast<const __nv_bfloat16*>(p.src)[e]);
+        }
+        r[x] = __float_as_uint(s);
+      }
+      umma::st16(tq + kColS + 64 * hf + 16 * c16, r);
+    }
+    umma::wait_st();
+
+    const int n_tok = t1 - t0;
+    const int n_chunks = (n_tok + kC - 1) / kC;
+
+    // Stages chunk ci (Q, K, V rows, Tw / Tu from the workspace, gates) into buffer ci & 1;
+    // rows beyond the sequence are zero and their gates (1, 0).
+    auto stage = [&](int ci) {
+      const int cc0 = ci * kC;
+      const int nn = (n_tok - cc0) < kC ? (n_tok - cc0) : kC;
+      unsigned char* buf = smem + (ci & 1) * kBufBytes;
+      for (int idx = tid; idx < kC * 16; idx += kThreads) {
+        const int r = idx >> 4, ch = idx & 15;
+        unsigned char* dq = buf + kOffQK + umma::panel_piece(128, r, ch);
+        unsigned char* dk = buf + kOffQK + umma::panel_piece(128, r + kC, ch);
+        unsigned char* dv = buf + kOffV + umma::panel_piece(kC, r, ch);
+        if (r < nn) {
+          const int64_t tok = t0 + cc0 + r;
+          cp_async_16(dq, qg + (tok * p.n_qk_heads + hq) * kD + ch * 8);
+          cp_async_16(dk, kg + (tok * p.n_qk_heads + hq) * kD + ch * 8);
+          cp_async_16(dv, vg + (tok * H + h) * kD + ch * 8);
+        } else {
+          *reinterpret_cast<uint4*>(dq) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(dk) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(dv) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      const unsigned char* wsrc = static_cast<const unsigned char*>(p.workspace) +
+                                  (((int64_t)((t0 + cc0) / kC + seq)) * H + h) * chunk::kPrepTileBytes;
+      for (int idx = tid; idx < chunk::kPrepTileBytes / 16; idx += kThreads)
+        cp_async_16(buf + kOffTw + idx * 16, wsrc + idx * 16);
+      if (warp == 0) {
+        float* gin = reinterpret_cast<float*>(smem + kOffGin) + (ci & 1) * 2 * kC;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 2 * lane + e;
+          if (t < nn) {
+            const int64_t gi = (int64_t)(t0 + cc0 + t) * H + h;
+            if (kGate) cp_async_4(gin + t, p.g + gi); else gin[t] = 1.0f;
+            if (Rule<RULE>::kUsesBeta) cp_async_4(gin + kC + t, p.beta + gi); else gin[kC + t] = 1.0f;
+          } else {
+            gin[t] = 1.0f;
+            gin[kC + t] = 0.0f;
+          }
+        }
+      }
+      cp_async_commit();
+    };
+
+    if (n_chunks > 0) stage(0);
+#pragma unroll 1
+    for (int ci = 0; ci < n_chunks; ++ci) {
+      const int c0 = ci * kC;
+      const int n = (n_tok - c0) < kC ? (n_tok - c0) : kC;
+      const uint32_t bq = sb + (ci & 1) * kBufBytes + kOffQK;  // Q rows
+      const uint32_t bk = bq + kC * 128;                        // K rows (same panels)
+      const uint32_t bv = sb + (ci & 1) * kBufBytes + kOffV;
+      const uint32_t btw = sb + (ci & 1) * kBufBytes + kOffTw;
+      const uint32_t btu = sb + (ci & 1) * kBufBytes + kOffTu;
+      if (ci + 1 < n_chunks) {
+        stage(ci + 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      // ---- gates: prefix of log |a| and of the signs over the chunk (warp 0)
+      if (warp == 0) {
+        const float* gin = reinterpret_cast<const float*>(smem + kOffGin) + (ci & 1) * 2 * kC;
+        float lg[2], sg[2];
+        bool big = false;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 2 * lane + e;
+          float a, bc, cc;
+          Rule<RULE>::coeffs(gin[t], gin[kC + t], a, bc, cc);
+          big |= fabsf(a) > 1.0f;
+          lg[e] = __logf(fmaxf(fabsf(a), 1e-30f));
+          sg[e] = a < 0.0f ? -1.0f : 1.0f;
+        }
+        float l = lg[0] + lg[1], sgn = sg[0] * sg[1];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float lo = __shfl_up_sync(0xffffffffu, l, off);
+          const float so2 = __shfl_up_sync(0xffffffffu, sgn, off);
+          if (lane >= off) {
+            l += lo;
+            sgn *= so2;
+          }
+        }
+        const float lprev = l - (lg[0] + lg[1]), sprev = sgn * sg[0] * sg[1];
+        const float l0 = lprev + lg[0], s0 = sprev * sg[0];
+        sLg[2 * lane] = l0;
+        sSg[2 * lane] = s0;
+        sLg[2 * lane + 1] = l;
+        sSg[2 * lane + 1] = sgn;
+        sGm[2 * lane] = s0 * __expf(l0);
+        sGm[2 * lane + 1] = sgn * __expf(l);
+        const float lfirst = __shfl_sync(0xffffffffu, l0, 0), llast = __shfl_sync(0xffffffffu, l, 31);
+        const float slast = __shfl_sync(0xffffffffu, sgn, 31);
+        const bool fact = !__any_sync(0xffffffffu, big) && (lfirst - llast) <= 80.0f;
+        const float m = 0.5f * (lfirst + llast);
+        sFa[2 * lane] = s0 * __expf(l0 - m);
+        sFb[2 * lane] = s0 * __expf(m - l0);
+        sFa[2 * lane + 1] = sgn * __expf(l - m);
+        sFb[2 * lane + 1] = sgn * __expf(m - l);
+        sGu[2 * lane] = slast * s0 * __expf(llast - l0);
+        sGu[2 * lane + 1] = slast * sgn * __expf(llast - l);
+        if (lane == 0) misc[2] = fact ? 1u : 0u;
+      }
+      umma::fence_smem();  // staged operands -> tensor cores
+      __syncthreads();
+      const bool fact = misc[2] != 0;
+      const float gC = sGm[kC - 1];  // padded tokens have gate 1: the last real token's
+
+      // ---- S pass: BF16 copy of S0^T for this chunk's products, then S^T *= gamma_C
+#pragma unroll 1
+      for (int c16 = 0; c16 < 4; ++c16) {
+        uint32_t r[16];
+        umma::ld16(tq + kColS + 64 * hf + 16 * c16, r);
+        umma::wait_ld();
+#pragma unroll
+        for (int pc = 0; pc < 2; ++pc)
+          *reinterpret_cast<uint4*>(smem + kOffS + umma::panel_piece(128, lrow, 8 * hf + 2 * c16 + pc)) =
+              pack8(r + 8 * pc);
+        if (kGate) {
+#pragma unroll
+          for (int x = 0; x < 16; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * gC);
+          umma::st16(tq + kColS + 64 * hf + 16 * c16, r);
+        }
+      }
+      if (kGate) umma::wait_st();
+      umma::fence_smem();
+      umma::fence_before();
+      __syncthreads();
+
+      // ---- MMAs, group 1: P = [Q; K] K^T, W^T = K^T Tw^T, U^T = V^T Tu^T, O1^T = S0^T Q^T
+      if (tid == 0) {
+        umma::fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // K = d_k
+          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma::mma(tmem + kColP, umma::sdesc(bq + ko, 16, 1024), umma::sdesc(bk + ko, 16, 1024), kIdKK64, kk);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // K = tokens
+          umma::mma(tmem + kColW, umma::sdesc(bk + kk * 2048, 16384, 1024), umma::sdesc(btw + kk * 32, 16, 1024),
+                    kIdMK64, kk);
+          umma::mma(tmem + kColU, umma::sdesc(bv + kk * 2048, 8192, 1024), umma::sdesc(btu + kk * 32, 16, 1024),
+                    kIdMK64, kk);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // K = d_k
+          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma::mma(tmem + kColO1, umma::sdesc(sb + kOffS + ko, 16, 1024), umma::sdesc(bq + ko, 16, 1024), kIdKK64,
+                    kk);
+        }
+        umma::commit(&bars[0]);
+      }
+      bool ok = mbar_wait(&bars[0], phase & 1u);
+      umma::fence_after();
+      // W^T rows (lane = d_k index) -> shared memory, the B operand of the U update
+#pragma unroll
+      for (int c16 = 0; c16 < 2; ++c16) {
+        uint32_t r[16];
+        umma::ld16(tq + kColW + 32 * hf + 16 * c16, r);
+        umma::wait_ld();
+#pragma unroll
+        for (int pc = 0; pc < 2; ++pc)
+          *reinterpret_cast<uint4*>(smem + kOffW + umma::panel_piece(128, lrow, 4 * hf + 2 * c16 + pc)) =
+              pack8(r + 8 * pc);
+      }
+      // P rows (lanes 0..63 = token t): masked by the gate ratios
+      if (q4 < 2) {
+        const int t = lrow;
+#pragma unroll
+        for (int c16 = 0; c16 < 2; ++c16) {
+          uint32_t r[16];
+          umma::ld16(tq + kColP + 32 * hf + 16 * c16, r);
+          umma::wait_ld();
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const int s = 32 * hf + 16 * c16 + x;
+            float v = 0.0f;
+            if (s <= t)
+              v = (fact ? sFa[t] * sFb[s] : sSg[t] * sSg[s] * __expf(sLg[t] - sLg[s])) * __uint_as_float(r[x]);
+            r[x] = __float_as_uint(v);
+          }
+#pragma unroll
+          for (int pc = 0; pc < 2; ++pc)
+            *reinterpret_cast<uint4*>(smem + kOffP + umma::panel_piece(kC, t, 4 * hf + 2 * c16 + pc)) =
+                pack8(r + 8 * pc);
+        }
+      }
+      umma::fence_smem();
+      umma::fence_before();
+      if (__syncthreads_or(!ok)) {
+        abort = true;
+        break;
+      }
+
+      // ---- group 2: U^T -= S0^T W^T
+      if (tid == 0) {
+        umma::fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // K = d_k
+          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma::mma(tmem + kColU, umma::sdesc(sb + kOffS + ko, 16, 1024),
+                    umma::sdesc(sb + kOffW + kk * 2048, 16384, 1024), kIdKM64n, 1);
+        }
+        umma::commit(&bars[1]);
+      }
+      ok = mbar_wait(&bars[1], phase & 1u);
+      umma::fence_after();
+      // U^T rows (lane = d_v index) -> U and Us = U (gamma_C / gamma_t) per token column
+#pragma unroll
+      for (int c16 = 0; c16 < 2; ++c16) {
+        uint32_t r[16];
+        umma::ld16(tq + kColU + 32 * hf + 16 * c16, r);
+        umma::wait_ld();
+#pragma unroll
+        for (int pc = 0; pc < 2; ++pc)
+          *reinterpret_cast<uint4*>(smem + kOffU + umma::panel_piece(128, lrow, 4 * hf + 2 * c16 + pc)) =
+              pack8(r + 8 * pc);
+#pragma unroll
+        for (int x = 0; x < 16; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * sGu[32 * hf + 16 * c16 + x]);
+#pragma unroll
+        for (int pc = 0; pc < 2; ++pc)
+          *reinterpret_cast<uint4*>(smem + kOffUs + umma::panel_piece(128, lrow, 4 * hf + 2 * c16 + pc)) =
+              pack8(r + 8 * pc);
+      }
+      umma::fence_smem();
+      umma::fence_before();
+      if (__syncthreads_or(!ok)) {
+        abort = true;
+        break;
+      }
+
+      // ---- group 3: O2^T = U^T P^T ;  S^T += Us^T K
+      if (tid == 0) {
+        umma::fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // K = tokens
+          umma::mma(tmem + kColO2, umma::sdesc(sb + kOffU + kk * 32, 16, 1024),
+                    umma::sdesc(sb + kOffP + kk * 32, 16, 1024), kIdKK64, kk);
+          umma::mma(tmem + kColS, umma::sdesc(sb + kOffUs + kk * 32, 16, 1024),
+                    umma::sdesc(bk + kk * 2048, 16384, 1024), kIdKM128, 1);
+        }
+        umma::commit(&bars[2]);
+      }
+      ok = mbar_wait(&bars[2], phase & 1u);
+      umma::fence_after();
+      // O rows: o_t[j] = scale (gamma_t O1^T[j][t] + O2^T[j][t]), lane = j
+#pragma unroll
+      for (int c16 = 0; c16 < 2; ++c16) {
+        uint32_t r1[16], r2[16];
+        umma::ld16(tq + kColO1 + 32 * hf + 16 * c16, r1);
+        umma::ld16(tq + kColO2 + 32 * hf + 16 * c16, r2);
+        umma::wait_ld();
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const int t = 32 * hf + 16 * c16 + x;
+          if (t < n)
+            og[((int64_t)(t0 + c0 + t) * H + h) * kD + lrow] =
+                __float2bfloat16_rn(p.scale * (sGm[t] * __uint_as_float(r1[x]) + __uint_as_float(r2[x])));
+        }
+      }
+      umma::fence_before();
+      if (__syncthreads_or(!ok)) {
+        abort = true;
+        break;
+      }
+      ++phase;
+    }
+    if (abort) break;
+
+    // ---- final state: S[i][j] = S^T[j][i], lane j, columns i
+    const int64_t dbase = ((int64_t)ws * H + h) * (kD * kD);
+#pragma unroll 1
+    for (int c16 = 0; c16 < 4; ++c16) {
+      uint32_t r[16];
+      umma::ld16(tq + kColS + 64 * hf + 16 * c16, r);
+      umma::wait_ld();
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const int64_t e = dbase + (int64_t)(64 * hf + 16 * c16 + x) * kD + lrow;
+        if (p.dst_dtype == LA_F32)
+          static_cast<float*>(p.dst)[e] = __uint_as_float(r[x]);
+        else
+          static_cast<__nv_bfloat16*>(p.dst)[e] = __float2bfloat16_rn(__uint_as_float(r[x]));
+      }
+    }
+    umma::fence_before();
+    __syncthreads();
+  }
+
+  cp_async_wait<0>();
+  if (abort && tid == 0) report(p.err, LA_DEVERR_TIMEOUT);
+  umma::fence_before();
+  __syncthreads();
+  if (warp == 0) umma::dealloc(tmem, kTmemCols);
+}
+
+template <int RULE>
+cudaError_t launch_chunk_tc(const ScanParams& p, cudaStream_t stream) {
+  const void* fn = reinterpret_cast<const void*>(&chunk_tc_kernel<RULE>);
+  const int per_sm = prepare_kernel(fn, chunk_tc::kThreads, chunk_tc::kSmem);
+  // one CTA per SM: the kernel holds all of the SM's tensor memory
+  if (per_sm != 1) return cudaErrorInvalidConfiguration;
+  const int64_t units = (int64_t)p.n_seqs * p.n_v_heads;
+  const int64_t cap = device_sm_count();
+  const int grid = (int)(units < cap ? units : cap);
+  chunk_tc_kernel<RULE><<<grid, chunk_tc::kThreads, chunk_tc::kSmem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace la

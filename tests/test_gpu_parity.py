@@ -484,19 +484,22 @@ def _gpu_scan_chunked_ws(inp, dst_dtype):
     return dst_t.cpu(), o.cpu(), int(err.item())
 
 
+@pytest.mark.parametrize("dst", [F32, BF16], ids=["f32", "bf16"])
 @pytest.mark.parametrize("rule", W.RULES)
-def test_chunked_two_launches_match_one_bitwise(rule):
-    """The two-launch form (intra-chunk inverses through the workspace) gives the fused
-    kernel's bits, and both match the oracle; the workspace size check is enforced."""
+def test_chunked_two_launches_vs_oracle(rule, dst):
+    """The two-launch form (intra-chunk inverses through the workspace, then for the delta
+    rules the recurrence on tcgen05) against the oracle; the linear and gated rules take the
+    fused kernel there, bit for bit.  The workspace size check is enforced."""
     inp = W.scan_inputs(lengths=[100, 64, 1, 0, 200, 63, 129], n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128,
                         rule=rule, io_dtype=BF16, seed=43, init="slots", init_dtype=F32, scale=0.8)
-    S1, o1, e1 = _gpu_scan_chunked(inp, F32)
-    S2, o2, e2 = _gpu_scan_chunked_ws(inp, F32)
-    assert e1 == e2 == 0
-    assert torch.equal(S1, S2) and torch.equal(o1, o2)
-    S_ref, o_ref, _ = oracle_scan(inp, dst_dtype=F32)
+    S2, o2, e2 = _gpu_scan_chunked_ws(inp, dst)
+    assert e2 == 0
+    S_ref, o_ref, _ = oracle_scan(inp, dst_dtype=dst)
     assert_close(np64(S2), S_ref, 2e-2, f"{rule}: final states")
     assert_close(np64(o2), o_ref, 2e-2, f"{rule}: outputs")
+    if rule in ("linear", "gated"):
+        S1, o1, e1 = _gpu_scan_chunked(inp, dst)
+        assert e1 == 0 and torch.equal(S1, S2) and torch.equal(o1, o2)
     small = torch.zeros(16, dtype=torch.uint8, device="cuda")
     dst_t = torch.zeros(7, 4, 128, 128, dtype=F32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -504,6 +507,39 @@ def test_chunked_two_launches_match_one_bitwise(rule):
                                     dev(inp.k), dev(inp.v), dev(inp.g), dev(inp.beta), 1.0,
                                     torch.empty_like(dev(inp.v)), small, err)
     assert st == L.LA_ERR_SHAPE
+
+
+@pytest.mark.parametrize("rule", ["delta", "gated_delta"])
+def test_chunked_two_launches_special_ranges(rule):
+    """Gates in [-1, 1] (negative products, ratios outside the factored range) and beta in
+    [0, 2]; then beta = 0 with g = 1, which must leave the initial state as it is."""
+    inp = W.scan_inputs(lengths=[300, 70, 5], n_qk_heads=1, n_v_heads=2, d_k=128, d_v=128, rule=rule,
+                        io_dtype=BF16, seed=44, g_mode="uniform_pm1", beta_mode="uniform_0_2", init="slots",
+                        init_dtype=F32)
+    S, o, err = _gpu_scan_chunked_ws(inp, F32)
+    S_ref, o_ref, _ = oracle_scan(inp, dst_dtype=F32)
+    assert err == 0
+    assert_close(np64(S), S_ref, 2e-2, f"{rule}: wide-range final states")
+    assert_close(np64(o), o_ref, 2e-2, f"{rule}: wide-range outputs")
+    inp = W.scan_inputs(lengths=[130, 64], n_qk_heads=1, n_v_heads=2, d_k=128, d_v=128, rule=rule,
+                        io_dtype=BF16, seed=45, g_mode="one", beta_mode="zero", init="slots", init_dtype=F32)
+    S, o, err = _gpu_scan_chunked_ws(inp, F32)
+    assert err == 0
+    S0 = inp.pool[inp.read_slot.long()].float()
+    assert torch.equal(S, S0), "beta = 0, g = 1: the state passes through unchanged"
+    S_ref, o_ref, _ = oracle_scan(inp, dst_dtype=F32)
+    assert_close(np64(o), o_ref, 2e-2, f"{rule}: readout of the unchanged state")
+
+
+def test_chunked_two_launches_prefill32_sampled():
+    """The full prefill workload through the two-launch path, as the benchmark runs it:
+    the shortest and the longest sequence checked against the oracle on one head each."""
+    inp = W.prefill32()
+    S, o, err = _gpu_scan_chunked_ws(inp, BF16)
+    assert err == 0
+    cu = inp.cu_seqlens.numpy()
+    order = np.argsort(cu[1:] - cu[:-1])
+    _check_sampled_units(inp, S, o, [(int(order[0]), 7), (int(order[-1]), 21)])
 
 
 def test_chunked_prefill32_sampled():

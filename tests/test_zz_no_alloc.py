@@ -1,6 +1,6 @@
 """GPU check of la_state_scan_chunked_noalloc, the two-launch chunked prefill on the
-library's own fixed workspace: the same bits as the one-launch chunked prefill, parity with
-the oracle, and the size limit refused before any launch."""
+library's own fixed workspace: the same bits as the two-launch form on a caller's workspace,
+parity with the oracle, and the size limit refused before any launch."""
 import ctypes
 
 import numpy as np
@@ -33,11 +33,17 @@ def _run(fn, inp):
     return dst_t.cpu(), o.cpu(), int(err.item())
 
 
+def _chunked_ws(rule, src, read_slot, dst, write_slot, cu, q, k, v, g, beta, scale, o, err):
+    nbytes = L.la_scan_chunked_workspace_bytes(q.shape[0], cu.numel() - 1, v.shape[1])
+    ws = torch.empty((nbytes,), dtype=torch.uint8, device="cuda")
+    return L.la_state_scan_chunked_ws(rule, src, read_slot, dst, write_slot, cu, q, k, v, g, beta, scale, o, ws, err)
+
+
 @pytest.mark.parametrize("rule", ["delta", "gated_delta", "gated"])
 def test_noalloc_matches_the_chunked_prefill(rule):
     inp = W.scan_inputs(lengths=[130, 0, 64, 7, 300], n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128, rule=rule,
                         io_dtype=BF16, seed=61, init="slots", init_dtype=F32)
-    S1, o1, e1 = _run(L.la_state_scan_chunked, inp)
+    S1, o1, e1 = _run(_chunked_ws, inp)
     S2, o2, e2 = _run(L.la_state_scan_chunked_noalloc, inp)
     S3, o3, e3 = _run(L.la_state_scan_chunked_noalloc, inp)  # the fixed workspace is reused
     assert e1 == e2 == e3 == 0
