@@ -59,10 +59,13 @@ constexpr int kOffGin = kOffG + 6 * kC * 4;     // 2 x {g, beta} [64] fp32 (stag
 constexpr int kSmem = kOffGin + 2 * 2 * kC * 4;
 static_assert(kSmem <= 227 * 1024, "shared memory");
 static_assert(kOffW + kC * kRow128 <= kOffT + kC * kTs * 4, "W reuses the L / T space");
-// workspace tile of one (chunk, head): Tw then Tu, [64][64] BF16 each, in the swizzled layout
-constexpr int kPrepTileBytes = 2 * kC * kRow64;
-static_assert(kOffW + kC * kRow128 <= kOffT && kPrepTileBytes <= kC * kTs * 4,
-              "the second staged Tw / Tu buffer takes the T space, clear of W");
+// workspace tile of one (chunk, head): Tw then Tu, [64][64] BF16 each, rows 128 bytes
+// apart with the 16-byte piece c of row r at c ^ (r & 7); then the gate block, FP32
+// [6][64] = gamma_t, gamma_C / gamma_t, A_t = gamma_t / e^m, B_t = e^m / gamma_t,
+// log |gamma_t|, sign gamma_t, and one word that is 1 when gamma_t / gamma_s = A_t B_s
+// may be used (the chunk's gates are at most 1 in magnitude and span at most e^80)
+constexpr int kGateBlockBytes = (6 * kC + 4) * 4;
+constexpr int kPrepTileBytes = 2 * kC * kRow64 + kGateBlockBytes;
 
 // byte offset of the 16-byte chunk `ch` of row `r` in a swizzled matrix with rows of `rowb` bytes
 __device__ __forceinline__ uint32_t swz(uint32_t base, int r, int ch, int rowb) {
@@ -146,9 +149,7 @@ __device__ __forceinline__ void st_bf16x2(unsigned char* smem, uint32_t off, flo
 
 }  // namespace chunk
 
-// PRE: Tw / Tu of every chunk come from the workspace that chunk_prep_kernel filled
-// (steps 1 and 2 shrink to Q K^T); otherwise everything happens here.
-template <int RULE, bool PRE = false>
+template <int RULE>
 __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const ScanParams p) {
   using namespace chunk;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -186,7 +187,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
   const int mt = warp & 3, nh = warp >> 2;
 
   // the strictly upper 16 x 16 blocks of Tw and Tu are zero in every chunk
-  for (int idx = tid; idx < (PRE ? 0 : kC * kC / 2); idx += kThreads) {
+  for (int idx = tid; idx < kC * kC / 2; idx += kThreads) {
     const int r = idx >> 5, c = 2 * (idx & 31);
     if ((c >> 4) > (r >> 4)) {
       const uint32_t off = swz(kOffTw, r, c >> 3, kRow64) + 2 * (c & 7);
@@ -265,13 +266,6 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
           *reinterpret_cast<uint4*>(in + kC * kRow128 + so) = make_uint4(0, 0, 0, 0);
           *reinterpret_cast<uint4*>(in + 2 * kC * kRow128 + so) = make_uint4(0, 0, 0, 0);
         }
-      }
-      if (PRE && kDelta) {
-        // Tw and Tu (16 KB, already in the swizzled layout) into buffer ci & 1
-        const unsigned char* wsrc = static_cast<const unsigned char*>(p.workspace) +
-                                    (((int64_t)((t0 + cc0) / kC + seq)) * H + h) * kPrepTileBytes;
-        unsigned char* wdst = smem + ((ci & 1) ? kOffT : kOffTw);
-        for (int idx = tid; idx < kPrepTileBytes / 16; idx += kThreads) cp_async_16(wdst + idx * 16, wsrc + idx * 16);
       }
       if (warp == 0) {
         float* gin = reinterpret_cast<float*>(smem + kOffGin) + (ci & 1) * 2 * kC;
@@ -359,43 +353,8 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
       __syncthreads();
       const bool fact = sFlag[0] != 0;
 
-      // ---- step 1: K K^T (warps 0-3, delta rules) and Q K^T (warps 4-7), rows [16 mt, +16).
-      //      PRE (no K K^T here): Q K^T over all 8 warps, rows 16 (warp & 3), columns
-      //      32 (warp >> 2), and no barrier before step 3, which does not read it
-      if constexpr (PRE) {
-        const int nh2 = warp >> 2;
-        float acc[4][4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
-#pragma unroll
-        for (int kk = 0; kk < kD; kk += 16) {
-          uint32_t a[4];
-          lda(a, sbase + kOffQ, kRow128, 16 * mt, kk, lane);
-#pragma unroll
-          for (int np = 0; np < 2; ++np) {
-            uint32_t b[4];
-            ldb_nk(b, sbase + kOffK, kRow128, 32 * nh2 + 16 * np, kk, lane);
-            mma16816(acc[2 * np], a, b[0], b[1]);
-            mma16816(acc[2 * np + 1], a, b[2], b[3]);
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-#pragma unroll
-          for (int e = 0; e < 4; e += 2) {
-            const int r = 16 * mt + g8 + (e >> 1) * 8;
-            float v2[2];
-#pragma unroll
-            for (int f = 0; f < 2; ++f) {
-              const int s_ = 32 * nh2 + 8 * j + 2 * t4 + f;
-              v2[f] = 0.0f;
-              if (s_ <= r)
-                v2[f] = (fact ? sFa[r] * sFb[s_] : sSg[r] * sSg[s_] * __expf(sLg[r] - sLg[s_])) * acc[j][e + f];
-            }
-            st_bf16x2(smem, swz(kOffP, r, 4 * nh2 + j, kRow64) + 4 * t4, v2[0], v2[1]);
-          }
-        }
-      } else if (kDelta || warp >= 4) {
+      // ---- step 1: K K^T (warps 0-3, delta rules) and Q K^T (warps 4-7), rows [16 mt, +16)
+      if (kDelta || warp >= 4) {
         float acc[8][4];
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
@@ -436,11 +395,11 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
           }
         }
       }
-      if (!PRE) __syncthreads();
+      __syncthreads();
 
       // ---- step 2 (delta rules): T = (I + L)^-1 by 16 x 16 blocks, written as FP32 (for the
       //      block recursion) and as Tw = T diag(b gamma), Tu = T diag(b) (BF16, swizzled)
-      if (kDelta && !PRE) {
+      if (kDelta) {
         // diagonal blocks: forward substitution, lane c < 16 of warp b owns column c
         if (warp < 4) {
           const int b0 = 16 * warp, c = lane & 15;
@@ -523,8 +482,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
           accu[j][0] = accu[j][1] = accu[j][2] = accu[j][3] = 0.0f;
           accw[j][0] = accw[j][1] = accw[j][2] = accw[j][3] = 0.0f;
         }
-        // Tw, Tu of this chunk (PRE: the staged copy in buffer ci & 1)
-        const uint32_t tw = sbase + ((PRE && (ci & 1)) ? kOffT : kOffTw), tu = tw + kC * kRow64;
+        const uint32_t tw = sbase + kOffTw, tu = tw + kC * kRow64;
 #pragma unroll
         for (int kk = 0; kk < kC; kk += 16) {
           uint32_t au[4], aw[4];
@@ -670,7 +628,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
 
 // ---- the intra-chunk part on its own: per (chunk, head), K K^T, the UT inverse and
 //      Tw = T diag(b gamma), Tu = T diag(b), written to the workspace for
-//      chunk_scan_kernel<RULE, true>.  Chunks are independent, so several CTAs share an SM
+//      chunk_tc_kernel.  Chunks are independent, so several CTAs share an SM
 //      and hide each other's latency.  Chunk c of sequence s goes to workspace tile
 //      (t0_s + 64 c) / 64 + s (distinct for every chunk; fewer than T / 64 + n_seqs + 1).
 namespace chunk {
@@ -678,7 +636,8 @@ constexpr int kPOffK = 0;                           // 2 x [64][128] bf16, swizz
 constexpr int kPOffL = kPOffK + 2 * kC * kRow128;   // [64][68] fp32
 constexpr int kPOffT = kPOffL + kC * kLs * 4;       // [64][72] fp32
 constexpr int kPOffTw = kPOffT + kC * kTs * 4;      // Tw, Tu [64][64] bf16, swizzled
-constexpr int kPOffX = kPOffTw + kPrepTileBytes;    // [3][16][24] fp32
+constexpr int kPOffGB = kPOffTw + 2 * kC * kRow64;  // the gate block of the workspace tile
+constexpr int kPOffX = kPOffGB + kGateBlockBytes;   // [3][16][24] fp32
 constexpr int kPOffG = kPOffX + 3 * 16 * kXs * 4;   // per token gate quantities [6][64]
 constexpr int kPOffGin = kPOffG + 6 * kC * 4;       // 2 x g, beta [2][64] (double buffer)
 constexpr int kPSmem = kPOffGin + 2 * 2 * kC * 4;
@@ -805,6 +764,21 @@ __global__ void __launch_bounds__(chunk::kThreads, 2) chunk_prep_kernel(const Sc
         sFa[2 * lane + 1] = sgn * __expf(l - m);
         sFb[2 * lane + 1] = sgn * __expf(m - l);
         if (lane == 0) sX[0] = fact_l ? 1.0f : 0.0f;  // (sX is scratch again only in the inverse)
+        // the gate block for the recurrence launch
+        float* gbk = reinterpret_cast<float*>(smem + kPOffGB);
+        const float slast = __shfl_sync(0xffffffffu, sgn, 31);
+        const float lv[2] = {l0, l}, sv[2] = {s0, sgn};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 2 * lane + e;
+          gbk[t] = sGm[t];
+          gbk[kC + t] = slast * sv[e] * __expf(llast - lv[e]);
+          gbk[2 * kC + t] = sFa[t];
+          gbk[3 * kC + t] = sFb[t];
+          gbk[4 * kC + t] = lv[e];
+          gbk[5 * kC + t] = sv[e];
+        }
+        if (lane == 0) gbk[6 * kC] = fact_l ? 1.0f : 0.0f;
       }
       __syncthreads();
       const bool fact = sX[0] != 0.0f;
@@ -910,7 +884,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 2) chunk_prep_kernel(const Sc
         }
         __syncthreads();
       }
-      // Tw, Tu to the workspace (16 KB, the swizzled layout as is)
+      // Tw, Tu and the gate block to the workspace (the layout as is)
       uint4* dstw = reinterpret_cast<uint4*>(static_cast<unsigned char*>(const_cast<void*>(p.workspace)) +
                                              (((int64_t)((t0 + c0) / kC + seq)) * H + h) * kPrepTileBytes);
       const uint4* srcw = reinterpret_cast<const uint4*>(smem + kPOffTw);
@@ -944,26 +918,12 @@ cudaError_t launch_chunk_scan(const ScanParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// The chunked prefill in two launches on the stream: the intra-chunk inverses of every
-// chunk (parallel), then the recurrence reading them.  Linear and gated rules have no
-// inverse and take the single fused kernel.
+// The chunked prefill through the workspace for the linear and gated rules, which have no
+// intra-chunk inverse: the single fused kernel.
 template <int RULE>
 cudaError_t launch_chunk_scan_ws(const ScanParams& p, cudaStream_t stream) {
-  if constexpr (!Rule<RULE>::kPredicts) {
-    return launch_chunk_scan<RULE>(p, stream);
-  } else {
-    cudaError_t e = launch_chunk_prep<RULE>(p, stream);
-    if (e != cudaSuccess) return e;
-    const void* fn = reinterpret_cast<const void*>(&chunk_scan_kernel<RULE, true>);
-    const int per_sm = prepare_kernel(fn, chunk::kThreads, chunk::kSmem);
-    if (per_sm <= 0) return cudaErrorInvalidConfiguration;
-    const int64_t units = (int64_t)p.n_seqs * p.n_v_heads;
-    const int64_t cap = (int64_t)device_sm_count() * per_sm;
-    const int grid = (int)(units < cap ? units : cap);
-    chunk_scan_kernel<RULE, true><<<grid, chunk::kThreads, chunk::kSmem, stream>>>(p);
-    return cudaGetLastError();
-  }
+  static_assert(!Rule<RULE>::kPredicts, "the delta rules take chunk_prep_kernel + chunk_tc_kernel");
+  return launch_chunk_scan<RULE>(p, stream);
 }
-
 
 }  // namespace la

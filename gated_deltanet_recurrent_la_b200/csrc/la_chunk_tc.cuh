@@ -4,7 +4,8 @@
 // Same algebra as la_chunk.cuh ("Seven Architectures Replacing KV Cache With Bounded
 // Mutable State": the "Kimi Linear" section's chunkwise-parallel kernel and the "Gated
 // DeltaNet-2" section's chunkwise WY algorithm).  chunk_prep_kernel has already written
-// Tw = T diag(b gamma) and Tu = T diag(b) of every 64-token chunk to the workspace; per
+// Tw = T diag(b gamma), Tu = T diag(b) and the chunk's gate quantities (gamma_t,
+// gamma_C / gamma_t, the ratio factors) of every 64-token chunk to the workspace; per
 // chunk this kernel forms
 //
 //   P   = (Q K^T) (.) M                         M_ts = gamma_t / gamma_s, s <= t
@@ -36,23 +37,24 @@ constexpr int kD = 128;  // d_k = d_v
 constexpr int kThreads = 256;
 
 // shared memory (bytes from a 1024-byte aligned base); operands in 64-column panels
-constexpr int kBufBytes = 65536;             // one staged chunk:
+constexpr int kBufBytes = 67584;             // one staged chunk:
 constexpr int kOffQK = 0;                    //   Q rows 0..63 and K rows 64..127, [128][128]
 constexpr int kOffV = 32768;                 //   V [64][128]
-constexpr int kOffTw = 49152;                //   Tw [64][64]
-constexpr int kOffTu = 57344;                //   Tu [64][64]
+constexpr int kOffTw = 49152;                //   Tw [64][64]       } the workspace tile
+constexpr int kOffTu = 57344;                //   Tu [64][64]       }
+constexpr int kOffGB = 65536;                //   gate block        }
 constexpr int kOffS = 2 * kBufBytes;         // S0^T  [128 d_v][128 d_k] BF16
 constexpr int kOffW = kOffS + 32768;         // W^T   [128 d_k][64]
 constexpr int kOffP = kOffW + 16384;         // P     [64][64]
-constexpr int kOffU = kOffP + 8192;          // U^T   [128 d_v][64]
+constexpr int kOffU = kOffP + 8192;          // U^T   [128 d_v][64]; O [64][128] row-major at the end
 constexpr int kOffUs = kOffU + 16384;        // Us^T  [128 d_v][64]
-constexpr int kOffG = kOffUs + 16384;        // per token: log|gamma|, sign, gamma, A, B, gamma_C/gamma
-constexpr int kOffGin = kOffG + 6 * kC * 4;  // 2 x {g, beta}[64] (staged gates)
-constexpr int kOffBar = kOffGin + 2 * 2 * kC * 4;
-constexpr int kOffMisc = kOffBar + 3 * 8;    // [0] tensor-memory base, [2] factored ratios
+constexpr int kOffBar = kOffUs + 16384;
+constexpr int kOffMisc = kOffBar + 3 * 8;    // [0] tensor-memory base
 constexpr int kSmem = kOffMisc + 16 + 1024;  // + slack for the 1024-byte alignment
 static_assert(kSmem <= 227 * 1024, "shared memory");
-static_assert(chunk::kPrepTileBytes == 16384 && kOffTu == kOffTw + 8192, "workspace tile = Tw then Tu");
+static_assert(chunk::kPrepTileBytes == 16384 + chunk::kGateBlockBytes && kOffTu == kOffTw + 8192 &&
+                  kOffGB == kOffTu + 8192 && kOffGB + chunk::kGateBlockBytes <= kBufBytes && kBufBytes % 1024 == 0,
+              "workspace tile = Tw, Tu, gate block");
 
 // tensor-memory columns (FP32 accumulators, 128 lanes each)
 constexpr uint32_t kTmemCols = 512;
@@ -80,12 +82,6 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
   const uint32_t raw = smem_addr(smem_raw);
   unsigned char* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   const uint32_t sb = smem_addr(smem);
-  float* sLg = reinterpret_cast<float*>(smem + kOffG);  // log |gamma_t|
-  float* sSg = sLg + kC;                                // sign gamma_t
-  float* sGm = sSg + kC;                                // gamma_t
-  float* sFa = sGm + kC;                                // gamma_t / e^m
-  float* sFb = sFa + kC;                                // e^m / gamma_t
-  float* sGu = sFb + kC;                                // gamma_C / gamma_t
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
 
@@ -177,8 +173,8 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
     const int n_tok = t1 - t0;
     const int n_chunks = (n_tok + kC - 1) / kC;
 
-    // Stages chunk ci (Q, K, V rows, Tw / Tu from the workspace, gates) into buffer ci & 1;
-    // rows beyond the sequence are zero and their gates (1, 0).
+    // Stages chunk ci (Q, K, V rows; Tw, Tu and the gate block from the workspace) into
+    // buffer ci & 1; rows beyond the sequence are zero.
     auto stage = [&](int ci) {
       const int cc0 = ci * kC;
       const int nn = (n_tok - cc0) < kC ? (n_tok - cc0) : kC;
@@ -203,21 +199,6 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
                                   (((int64_t)((t0 + cc0) / kC + seq)) * H + h) * chunk::kPrepTileBytes;
       for (int idx = tid; idx < chunk::kPrepTileBytes / 16; idx += kThreads)
         cp_async_16(buf + kOffTw + idx * 16, wsrc + idx * 16);
-      if (warp == 0) {
-        float* gin = reinterpret_cast<float*>(smem + kOffGin) + (ci & 1) * 2 * kC;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = 2 * lane + e;
-          if (t < nn) {
-            const int64_t gi = (int64_t)(t0 + cc0 + t) * H + h;
-            if (kGate) cp_async_4(gin + t, p.g + gi); else gin[t] = 1.0f;
-            if (Rule<RULE>::kUsesBeta) cp_async_4(gin + kC + t, p.beta + gi); else gin[kC + t] = 1.0f;
-          } else {
-            gin[t] = 1.0f;
-            gin[kC + t] = 0.0f;
-          }
-        }
-      }
       cp_async_commit();
     };
 
@@ -230,60 +211,23 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       const uint32_t bk = bq + kC * 128;                        // K rows (same panels)
       const uint32_t bv = sb + (ci & 1) * kBufBytes + kOffV;
       const uint32_t btw = sb + (ci & 1) * kBufBytes + kOffTw;
-      const uint32_t btu = sb + (ci & 1) * kBufBytes + kOffTu;
       if (ci + 1 < n_chunks) {
         stage(ci + 1);
         cp_async_wait<1>();
       } else {
         cp_async_wait<0>();
       }
-      // ---- gates: prefix of log |a| and of the signs over the chunk (warp 0)
-      if (warp == 0) {
-        const float* gin = reinterpret_cast<const float*>(smem + kOffGin) + (ci & 1) * 2 * kC;
-        float lg[2], sg[2];
-        bool big = false;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = 2 * lane + e;
-          float a, bc, cc;
-          Rule<RULE>::coeffs(gin[t], gin[kC + t], a, bc, cc);
-          big |= fabsf(a) > 1.0f;
-          lg[e] = __logf(fmaxf(fabsf(a), 1e-30f));
-          sg[e] = a < 0.0f ? -1.0f : 1.0f;
-        }
-        float l = lg[0] + lg[1], sgn = sg[0] * sg[1];
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float lo = __shfl_up_sync(0xffffffffu, l, off);
-          const float so2 = __shfl_up_sync(0xffffffffu, sgn, off);
-          if (lane >= off) {
-            l += lo;
-            sgn *= so2;
-          }
-        }
-        const float lprev = l - (lg[0] + lg[1]), sprev = sgn * sg[0] * sg[1];
-        const float l0 = lprev + lg[0], s0 = sprev * sg[0];
-        sLg[2 * lane] = l0;
-        sSg[2 * lane] = s0;
-        sLg[2 * lane + 1] = l;
-        sSg[2 * lane + 1] = sgn;
-        sGm[2 * lane] = s0 * __expf(l0);
-        sGm[2 * lane + 1] = sgn * __expf(l);
-        const float lfirst = __shfl_sync(0xffffffffu, l0, 0), llast = __shfl_sync(0xffffffffu, l, 31);
-        const float slast = __shfl_sync(0xffffffffu, sgn, 31);
-        const bool fact = !__any_sync(0xffffffffu, big) && (lfirst - llast) <= 80.0f;
-        const float m = 0.5f * (lfirst + llast);
-        sFa[2 * lane] = s0 * __expf(l0 - m);
-        sFb[2 * lane] = s0 * __expf(m - l0);
-        sFa[2 * lane + 1] = sgn * __expf(l - m);
-        sFb[2 * lane + 1] = sgn * __expf(m - l);
-        sGu[2 * lane] = slast * s0 * __expf(llast - l0);
-        sGu[2 * lane + 1] = slast * sgn * __expf(llast - l);
-        if (lane == 0) misc[2] = fact ? 1u : 0u;
-      }
+      // ---- this chunk's gate quantities, from the workspace tile
+      const float* gbk = reinterpret_cast<const float*>(smem + (ci & 1) * kBufBytes + kOffGB);
+      const float* sGm = gbk;            // gamma_t
+      const float* sGu = gbk + kC;       // gamma_C / gamma_t
+      const float* sFa = gbk + 2 * kC;   // gamma_t / e^m
+      const float* sFb = gbk + 3 * kC;   // e^m / gamma_t
+      const float* sLg = gbk + 4 * kC;   // log |gamma_t|
+      const float* sSg = gbk + 5 * kC;   // sign gamma_t
       umma::fence_smem();  // staged operands -> tensor cores
       __syncthreads();
-      const bool fact = misc[2] != 0;
+      const bool fact = gbk[6 * kC] != 0.0f;
       const float gC = sGm[kC - 1];  // padded tokens have gate 1: the last real token's
 
       // ---- S pass: BF16 copy of S0^T for this chunk's products, then S^T *= gamma_C
@@ -308,25 +252,29 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       __syncthreads();
 
       // ---- MMAs, group 1: P = [Q; K] K^T, W^T = K^T Tw^T, U^T = V^T Tu^T, O1^T = S0^T Q^T
+      //      (descriptors: one per operand matrix, stepped by constant byte offsets)
+      const uint64_t dQK = umma::sdesc(bq, 16, 1024);     // [Q; K] rows, K-major
+      const uint64_t dKm = umma::sdesc(bk, 16384, 1024);  // K as an MN-major operand
+      const uint64_t dS = umma::sdesc(sb + kOffS, 16, 1024);
       if (tid == 0) {
         umma::fence_after();
+        const uint64_t dVm = umma::sdesc(bv, 8192, 1024);
+        const uint64_t dTw = umma::sdesc(btw, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // K = d_k
           const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma::mma(tmem + kColP, umma::sdesc(bq + ko, 16, 1024), umma::sdesc(bk + ko, 16, 1024), kIdKK64, kk);
+          umma::mma(tmem + kColP, umma::sdesc_add(dQK, ko), umma::sdesc_add(dQK, 8192 + ko), kIdKK64, kk);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {  // K = tokens
-          umma::mma(tmem + kColW, umma::sdesc(bk + kk * 2048, 16384, 1024), umma::sdesc(btw + kk * 32, 16, 1024),
-                    kIdMK64, kk);
-          umma::mma(tmem + kColU, umma::sdesc(bv + kk * 2048, 8192, 1024), umma::sdesc(btu + kk * 32, 16, 1024),
-                    kIdMK64, kk);
+          umma::mma(tmem + kColW, umma::sdesc_add(dKm, kk * 2048), umma::sdesc_add(dTw, kk * 32), kIdMK64, kk);
+          umma::mma(tmem + kColU, umma::sdesc_add(dVm, kk * 2048), umma::sdesc_add(dTw, 8192 + kk * 32), kIdMK64,
+                    kk);
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // K = d_k
           const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma::mma(tmem + kColO1, umma::sdesc(sb + kOffS + ko, 16, 1024), umma::sdesc(bq + ko, 16, 1024), kIdKK64,
-                    kk);
+          umma::mma(tmem + kColO1, umma::sdesc_add(dS, ko), umma::sdesc_add(dQK, ko), kIdKK64, kk);
         }
         umma::commit(&bars[0]);
       }
@@ -375,11 +323,11 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       // ---- group 2: U^T -= S0^T W^T
       if (tid == 0) {
         umma::fence_after();
+        const uint64_t dWm = umma::sdesc(sb + kOffW, 16384, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // K = d_k
           const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma::mma(tmem + kColU, umma::sdesc(sb + kOffS + ko, 16, 1024),
-                    umma::sdesc(sb + kOffW + kk * 2048, 16384, 1024), kIdKM64n, 1);
+          umma::mma(tmem + kColU, umma::sdesc_add(dS, ko), umma::sdesc_add(dWm, kk * 2048), kIdKM64n, 1);
         }
         umma::commit(&bars[1]);
       }
@@ -412,18 +360,21 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       // ---- group 3: O2^T = U^T P^T ;  S^T += Us^T K
       if (tid == 0) {
         umma::fence_after();
+        const uint64_t dP = umma::sdesc(sb + kOffP, 16, 1024);
+        const uint64_t dU = umma::sdesc(sb + kOffU, 16, 1024);
+        const uint64_t dUs = umma::sdesc(sb + kOffUs, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {  // K = tokens
-          umma::mma(tmem + kColO2, umma::sdesc(sb + kOffU + kk * 32, 16, 1024),
-                    umma::sdesc(sb + kOffP + kk * 32, 16, 1024), kIdKK64, kk);
-          umma::mma(tmem + kColS, umma::sdesc(sb + kOffUs + kk * 32, 16, 1024),
-                    umma::sdesc(bk + kk * 2048, 16384, 1024), kIdKM128, 1);
+          umma::mma(tmem + kColO2, umma::sdesc_add(dU, kk * 32), umma::sdesc_add(dP, kk * 32), kIdKK64, kk);
+          umma::mma(tmem + kColS, umma::sdesc_add(dUs, kk * 32), umma::sdesc_add(dKm, kk * 2048), kIdKM128, 1);
         }
         umma::commit(&bars[2]);
       }
       ok = mbar_wait(&bars[2], phase & 1u);
       umma::fence_after();
-      // O rows: o_t[j] = scale (gamma_t O1^T[j][t] + O2^T[j][t]), lane = j
+      // O rows: o_t[j] = scale (gamma_t O1^T[j][t] + O2^T[j][t]), lane = j, into the U
+      // space (free once group 3 is done) as a row-major [64][128] BF16 tile
+      __nv_bfloat16* sO = reinterpret_cast<__nv_bfloat16*>(smem + kOffU);
 #pragma unroll
       for (int c16 = 0; c16 < 2; ++c16) {
         uint32_t r1[16], r2[16];
@@ -433,15 +384,21 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
           const int t = 32 * hf + 16 * c16 + x;
-          if (t < n)
-            og[((int64_t)(t0 + c0 + t) * H + h) * kD + lrow] =
-                __float2bfloat16_rn(p.scale * (sGm[t] * __uint_as_float(r1[x]) + __uint_as_float(r2[x])));
+          sO[t * kD + lrow] =
+              __float2bfloat16_rn(p.scale * (sGm[t] * __uint_as_float(r1[x]) + __uint_as_float(r2[x])));
         }
       }
       umma::fence_before();
       if (__syncthreads_or(!ok)) {
         abort = true;
         break;
+      }
+      // the tile's rows to o (256 contiguous bytes per token)
+      for (int idx = tid; idx < kC * 16; idx += kThreads) {
+        const int t = idx >> 4, ch = idx & 15;
+        if (t < n)
+          *reinterpret_cast<uint4*>(og + ((int64_t)(t0 + c0 + t) * H + h) * kD + ch * 8) =
+              *reinterpret_cast<const uint4*>(sO + t * kD + ch * 8);
       }
       ++phase;
     }

@@ -216,11 +216,12 @@ la_status la_state_scan_chunked(la_rule rule, const la_pool *src, const int32_t 
                                 int32_t *err_word, void *stream);
 
 /* la_state_scan_chunked in two launches: the intra-chunk part of every chunk (K K^T, the
- * triangular inverse, Tw = T diag(beta gamma), Tu = T diag(beta)) as one parallel launch
- * writing a caller-owned workspace, then the recurrence over the chunks reading it.  The
+ * triangular inverse T, Tw = T diag(beta gamma), Tu = T diag(beta)) as one parallel launch
+ * writing a caller-owned workspace, then the recurrence over the chunks reading it, on the
+ * fifth-generation tensor cores (tcgen05 MMAs, the state in tensor memory).  The
  * chunks are independent in the first launch, so it fills the SMs (several CTAs each)
- * instead of sitting on each sequence's critical path.  Same results as
- * la_state_scan_chunked (the same arithmetic, bit for bit).
+ * instead of sitting on each sequence's critical path.  Same algorithm and precision as
+ * la_state_scan_chunked (BF16 products, FP32 accumulation and state), not bit for bit.
  *   workspace        device, 16-byte aligned, at least
  *                    la_scan_chunked_workspace_bytes(total_tokens, n_seqs, H_v) bytes;
  *                    contents are scratch (overwritten, not read back by the caller)
