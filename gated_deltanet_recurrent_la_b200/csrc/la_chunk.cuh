@@ -626,283 +626,240 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const Sc
   }
 }
 
-// ---- the intra-chunk part on its own: per (chunk, head), K K^T, the UT inverse and
-//      Tw = T diag(b gamma), Tu = T diag(b), written to the workspace for
-//      chunk_tc_kernel.  Chunks are independent, so several CTAs share an SM
-//      and hide each other's latency.  Chunk c of sequence s goes to workspace tile
+// ---- the intra-chunk part on its own, per (chunk, head) tile: K K^T, the UT inverse
+//      T = (I + L)^-1 by forward substitution in FP32 (one column of T per lane),
+//      Tw = T diag(b gamma), Tu = T diag(b) and the chunk's gate block, written to the
+//      workspace for chunk_tc_kernel.  Tiles are independent: a CTA of two warps takes one
+//      at a time and several CTAs share an SM.  Chunk c of sequence s is workspace tile
 //      (t0_s + 64 c) / 64 + s (distinct for every chunk; fewer than T / 64 + n_seqs + 1).
 namespace chunk {
-constexpr int kPOffK = 0;                           // 2 x [64][128] bf16, swizzled (double buffer)
-constexpr int kPOffL = kPOffK + 2 * kC * kRow128;   // [64][68] fp32
-constexpr int kPOffT = kPOffL + kC * kLs * 4;       // [64][72] fp32
-constexpr int kPOffTw = kPOffT + kC * kTs * 4;      // Tw, Tu [64][64] bf16, swizzled
-constexpr int kPOffGB = kPOffTw + 2 * kC * kRow64;  // the gate block of the workspace tile
-constexpr int kPOffX = kPOffGB + kGateBlockBytes;   // [3][16][24] fp32
-constexpr int kPOffG = kPOffX + 3 * 16 * kXs * 4;   // per token gate quantities [6][64]
-constexpr int kPOffGin = kPOffG + 6 * kC * 4;       // 2 x g, beta [2][64] (double buffer)
-constexpr int kPSmem = kPOffGin + 2 * 2 * kC * 4;
+constexpr int kPThreads = 64;
+constexpr int kPOffK = 0;                          // K [64][128] bf16, swizzled; then Tw, Tu [64][64]
+constexpr int kPOffGB = kPOffK + kC * kRow128;     // the gate block (Tw, Tu, gate block = the tile)
+constexpr int kPOffL = kPOffGB + kGateBlockBytes;  // L [64][68] fp32
+constexpr int kPOffB = kPOffL + kC * kLs * 4;      // b_t [64]
+constexpr int kPOffGin = kPOffB + kC * 4;          // g, beta [2][64]
+constexpr int kPSmem = kPOffGin + 2 * kC * 4;
+static_assert(2 * kC * kRow64 == kC * kRow128 && kPOffGB == 2 * kC * kRow64, "Tw, Tu take the K space");
+static_assert(kPOffL % 16 == 0, "L rows are read as float4");
 }  // namespace chunk
 
 template <int RULE>
-__global__ void __launch_bounds__(chunk::kThreads, 2) chunk_prep_kernel(const ScanParams p) {
+__global__ void __launch_bounds__(chunk::kPThreads) chunk_prep_kernel(const ScanParams p) {
   using namespace chunk;
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t sbase = smem_addr(smem);
   float* sL = reinterpret_cast<float*>(smem + kPOffL);
-  float* sT = reinterpret_cast<float*>(smem + kPOffT);
-  float* sX = reinterpret_cast<float*>(smem + kPOffX);
-  float* sLg = reinterpret_cast<float*>(smem + kPOffG);
-  float* sSg = sLg + kC;
-  float* sBt = sSg + kC;
-  float* sGm = sBt + kC;
-  float* sFa = sGm + kC;
-  float* sFb = sFa + kC;
+  float* gbk = reinterpret_cast<float*>(smem + kPOffGB);
+  float* sBt = reinterpret_cast<float*>(smem + kPOffB);
   float* gin = reinterpret_cast<float*>(smem + kPOffGin);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
   const int H = p.n_v_heads;
   const int ratio_h = H / p.n_qk_heads;
-  const int64_t units = (int64_t)p.n_seqs * H;
+  if (p.n_seqs <= 0) return;
+  const int64_t n_tiles = (int64_t)(p.total_tokens + kC - 1) / kC + p.n_seqs + 1;
+  const int64_t items = n_tiles * H;
   const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(p.k);
-  const int kOffTw2 = kPOffTw, kOffTu2 = kPOffTw + kC * kRow64;
 
-  // the strictly upper 16 x 16 blocks of Tw and Tu are zero in every chunk
-  for (int idx = tid; idx < kC * kC / 2; idx += kThreads) {
-    const int r = idx >> 5, c = 2 * (idx & 31);
-    if ((c >> 4) > (r >> 4)) {
-      const uint32_t off = swz(kOffTw2, r, c >> 3, kRow64) + 2 * (c & 7);
-      st_bf16x2(smem, off, 0.0f, 0.0f);
-      st_bf16x2(smem, off - kOffTw2 + kOffTu2, 0.0f, 0.0f);
+#pragma unroll 1
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+    const int gc = (int)(item / H), h = (int)(item % H), hq = h / ratio_h;
+    // the sequence of tile gc: the last s with cu[s] / 64 + s <= gc
+    int lo = 0, hi = p.n_seqs - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(p.cu_seqlens + mid) / kC + mid <= gc) lo = mid; else hi = mid - 1;
     }
-  }
-  __syncthreads();
-
-#pragma unroll 1
-  for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
-    const int seq = (int)(u / H), h = (int)(u % H), hq = h / ratio_h;
+    const int seq = lo;
     const int t0 = __ldg(p.cu_seqlens + seq), t1 = __ldg(p.cu_seqlens + seq + 1);
-    if (t0 < 0 || t1 < t0 || t1 > p.total_tokens) continue;  // reported by the main kernel
-    const int n_tok = t1 - t0;
-    // stages the chunk at token c0s into buffer bs: K rows (zero beyond the sequence) and
-    // the gates ((1, 0) beyond it)
-    auto stage = [&](int c0s, int bs) {
-      const int ns = (n_tok - c0s) < kC ? (n_tok - c0s) : kC;
-      for (int idx = tid; idx < kC * 16; idx += kThreads) {
-        const int r = idx >> 4, ch = idx & 15;
-        const uint32_t so = (uint32_t)(kPOffK + bs * kC * kRow128 + r * kRow128 + ((ch ^ (r & 7)) << 4));
-        if (r < ns) cp_async_16(smem + so, kg + ((int64_t)(t0 + c0s + r) * p.n_qk_heads + hq) * kD + ch * 8);
-        else *reinterpret_cast<uint4*>(smem + so) = make_uint4(0, 0, 0, 0);
-      }
-      if (warp == 0) {
-        float* gs = gin + bs * 2 * kC;
+    if (t0 < 0 || t1 < t0 || t1 > p.total_tokens) continue;  // reported by the recurrence launch
+    const int c0 = (gc - (t0 / kC + seq)) * kC;
+    if (c0 < 0 || c0 >= t1 - t0) continue;                   // a tile index no chunk uses
+    const int ns = (t1 - t0 - c0) < kC ? (t1 - t0 - c0) : kC;
+
+    // K rows (zero beyond the sequence) and the gates ((1, 0) beyond it)
+    for (int idx = tid; idx < kC * 16; idx += kPThreads) {
+      const int r = idx >> 4, ch = idx & 15;
+      unsigned char* d = smem + kPOffK + r * kRow128 + ((ch ^ (r & 7)) << 4);
+      if (r < ns) cp_async_16(d, kg + ((int64_t)(t0 + c0 + r) * p.n_qk_heads + hq) * kD + ch * 8);
+      else *reinterpret_cast<uint4*>(d) = make_uint4(0, 0, 0, 0);
+    }
+    if (warp == 0) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = 2 * lane + e;
-          if (t < ns) {
-            const int64_t gi = (int64_t)(t0 + c0s + t) * H + h;
-            if (Rule<RULE>::kUsesGate) cp_async_4(gs + t, p.g + gi); else gs[t] = 1.0f;
-            cp_async_4(gs + kC + t, p.beta + gi);
-          } else {
-            gs[t] = 1.0f;
-            gs[kC + t] = 0.0f;
-          }
+      for (int e = 0; e < 2; ++e) {
+        const int t = 2 * lane + e;
+        if (t < ns) {
+          const int64_t gi = (int64_t)(t0 + c0 + t) * H + h;
+          if (Rule<RULE>::kUsesGate) cp_async_4(gin + t, p.g + gi); else gin[t] = 1.0f;
+          cp_async_4(gin + kC + t, p.beta + gi);
+        } else {
+          gin[t] = 1.0f;
+          gin[kC + t] = 0.0f;
         }
       }
-      cp_async_commit();
-    };
-    if (n_tok > 0) stage(0, 0);
-#pragma unroll 1
-    for (int c0 = 0, it = 0; c0 < n_tok; c0 += kC, ++it) {
-      const int buf = it & 1;
-      if (c0 + kC < n_tok) {  // the next chunk's copies fly while this one is worked on
-        stage(c0 + kC, buf ^ 1);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+
+    // gates (warp 0): the gate block -- gamma_t, gamma_C / gamma_t, the factored ratios
+    // gamma_t / gamma_s = A_t B_s around the chunk's middle, log |gamma_t|, its sign -- and b_t
+    if (warp == 0) {
+      float lg[2], sg[2];
+      bool big = false;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int t = 2 * lane + e;
+        float a, bc, cc;
+        Rule<RULE>::coeffs(gin[t], gin[kC + t], a, bc, cc);
+        big |= fabsf(a) > 1.0f;
+        lg[e] = __logf(fmaxf(fabsf(a), 1e-30f));
+        sg[e] = a < 0.0f ? -1.0f : 1.0f;
+        sBt[t] = bc;
       }
-      __syncthreads();
-      const float* gb = gin + buf * 2 * kC;
-      const uint32_t kbase = sbase + kPOffK + buf * kC * kRow128;
-      // gates: b_t, gamma_t and the ratios gamma_t / gamma_s (as in chunk_scan_kernel)
-      bool fact_l = false;
-      if (warp == 0) {
-        float lg[2], sg[2];
-        bool big = false;
+      float l = lg[0] + lg[1], sgn = sg[0] * sg[1];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = 2 * lane + e;
-          float a, bc, cc;
-          Rule<RULE>::coeffs(gb[t], gb[kC + t], a, bc, cc);
-          big |= fabsf(a) > 1.0f;
-          lg[e] = __logf(fmaxf(fabsf(a), 1e-30f));
-          sg[e] = a < 0.0f ? -1.0f : 1.0f;
-          sBt[t] = bc;
+      for (int off = 1; off < 32; off <<= 1) {
+        const float lo2 = __shfl_up_sync(0xffffffffu, l, off);
+        const float so2 = __shfl_up_sync(0xffffffffu, sgn, off);
+        if (lane >= off) {
+          l += lo2;
+          sgn *= so2;
         }
-        float l = lg[0] + lg[1], sgn = sg[0] * sg[1];
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float lo = __shfl_up_sync(0xffffffffu, l, off);
-          const float so2 = __shfl_up_sync(0xffffffffu, sgn, off);
-          if (lane >= off) {
-            l += lo;
-            sgn *= so2;
-          }
-        }
-        const float lprev = l - (lg[0] + lg[1]), sprev = sgn * sg[0] * sg[1];
-        const float l0 = lprev + lg[0], s0 = sprev * sg[0];
-        sLg[2 * lane] = l0;
-        sSg[2 * lane] = s0;
-        sLg[2 * lane + 1] = l;
-        sSg[2 * lane + 1] = sgn;
-        sGm[2 * lane] = s0 * __expf(l0);
-        sGm[2 * lane + 1] = sgn * __expf(l);
-        const float lfirst = __shfl_sync(0xffffffffu, l0, 0), llast = __shfl_sync(0xffffffffu, l, 31);
-        fact_l = !__any_sync(0xffffffffu, big) && (lfirst - llast) <= 80.0f;
-        const float m = 0.5f * (lfirst + llast);
-        sFa[2 * lane] = s0 * __expf(l0 - m);
-        sFb[2 * lane] = s0 * __expf(m - l0);
-        sFa[2 * lane + 1] = sgn * __expf(l - m);
-        sFb[2 * lane + 1] = sgn * __expf(m - l);
-        if (lane == 0) sX[0] = fact_l ? 1.0f : 0.0f;  // (sX is scratch again only in the inverse)
-        // the gate block for the recurrence launch
-        float* gbk = reinterpret_cast<float*>(smem + kPOffGB);
-        const float slast = __shfl_sync(0xffffffffu, sgn, 31);
-        const float lv[2] = {l0, l}, sv[2] = {s0, sgn};
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = 2 * lane + e;
-          gbk[t] = sGm[t];
-          gbk[kC + t] = slast * sv[e] * __expf(llast - lv[e]);
-          gbk[2 * kC + t] = sFa[t];
-          gbk[3 * kC + t] = sFb[t];
-          gbk[4 * kC + t] = lv[e];
-          gbk[5 * kC + t] = sv[e];
-        }
-        if (lane == 0) gbk[6 * kC] = fact_l ? 1.0f : 0.0f;
       }
-      __syncthreads();
-      const bool fact = sX[0] != 0.0f;
-      // L = strictly-lower(b_t gamma_t / gamma_s k_t . k_s): warp w, rows 16 (w & 3), columns 32 (w >> 2)
-      {
-        const int mt = warp & 3, nh2 = warp >> 2;
-        float acc[4][4];
+      const float lprev = l - (lg[0] + lg[1]), sprev = sgn * sg[0] * sg[1];  // exclusive (signs are +-1)
+      const float lv[2] = {lprev + lg[0], l}, sv[2] = {sprev * sg[0], sgn};
+      const float lfirst = __shfl_sync(0xffffffffu, lv[0], 0), llast = __shfl_sync(0xffffffffu, l, 31);
+      const float slast = __shfl_sync(0xffffffffu, sgn, 31);
+      const bool fact = !__any_sync(0xffffffffu, big) && (lfirst - llast) <= 80.0f;
+      const float m = 0.5f * (lfirst + llast);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+      for (int e = 0; e < 2; ++e) {
+        const int t = 2 * lane + e;
+        gbk[t] = sv[e] * __expf(lv[e]);
+        gbk[kC + t] = slast * sv[e] * __expf(llast - lv[e]);
+        gbk[2 * kC + t] = sv[e] * __expf(lv[e] - m);
+        gbk[3 * kC + t] = sv[e] * __expf(m - lv[e]);
+        gbk[4 * kC + t] = lv[e];
+        gbk[5 * kC + t] = sv[e];
+      }
+      if (lane < 4) gbk[6 * kC + lane] = (lane == 0 && fact) ? 1.0f : 0.0f;
+    }
+    __syncthreads();
+    const bool fact = gbk[6 * kC] != 0.0f;
+    const float* sGm = gbk;
+    const float* sFa = gbk + 2 * kC;
+    const float* sFb = gbk + 3 * kC;
+    const float* sLg = gbk + 4 * kC;
+    const float* sSg = gbk + 5 * kC;
+
+    // L = strictly-lower(b_t gamma_t / gamma_s k_t . k_s): warp w, rows 32 w .. + 31
+    {
+      float acc[2][8][4];
 #pragma unroll
-        for (int kk = 0; kk < kD; kk += 16) {
-          uint32_t a[4];
-          lda(a, kbase, kRow128, 16 * mt, kk, lane);
+      for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
-          for (int np = 0; np < 2; ++np) {
-            uint32_t b[4];
-            ldb_nk(b, kbase, kRow128, 32 * nh2 + 16 * np, kk, lane);
-            mma16816(acc[2 * np], a, b[0], b[1]);
-            mma16816(acc[2 * np + 1], a, b[2], b[3]);
-          }
+        for (int j = 0; j < 8; ++j) acc[mi][j][0] = acc[mi][j][1] = acc[mi][j][2] = acc[mi][j][3] = 0.0f;
+#pragma unroll
+      for (int kk = 0; kk < kD; kk += 16) {
+        uint32_t a0[4], a1[4];
+        lda(a0, sbase + kPOffK, kRow128, 32 * warp, kk, lane);
+        lda(a1, sbase + kPOffK, kRow128, 32 * warp + 16, kk, lane);
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          uint32_t b[4];
+          ldb_nk(b, sbase + kPOffK, kRow128, 16 * np, kk, lane);
+          mma16816(acc[0][2 * np], a0, b[0], b[1]);
+          mma16816(acc[0][2 * np + 1], a0, b[2], b[3]);
+          mma16816(acc[1][2 * np], a1, b[0], b[1]);
+          mma16816(acc[1][2 * np + 1], a1, b[2], b[3]);
         }
+      }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+      for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int r = 16 * mt + g8 + (e >> 1) * 8, s_ = 32 * nh2 + 8 * j + 2 * t4 + (e & 1);
+            const int r = 32 * warp + 16 * mi + g8 + (e >> 1) * 8, s_ = 8 * j + 2 * t4 + (e & 1);
             float v = 0.0f;
             if (s_ < r) {
               const float ratio = fact ? sFa[r] * sFb[s_] : sSg[r] * sSg[s_] * __expf(sLg[r] - sLg[s_]);
-              v = sBt[r] * ratio * acc[j][e];
+              v = sBt[r] * ratio * acc[mi][j][e];
             }
             sL[r * kLs + s_] = v;
           }
-        }
-      }
-      __syncthreads();
-      // diagonal blocks: forward substitution, lane c < 16 of warp b owns column c
-      if (warp < 4) {
-        const int b0 = 16 * warp, c = lane & 15;
-        float col[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          const float4* lr = reinterpret_cast<const float4*>(sL + (b0 + r) * kLs + b0);
-          float x = (r == c) ? 1.0f : 0.0f;
-#pragma unroll
-          for (int m = 0; m < (r + 3) / 4; ++m) {
-            const float4 l4 = lr[m];
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (4 * m + e < r) x -= lv[e] * col[4 * m + e];
-          }
-          col[r] = (r < c) ? 0.0f : x;
-        }
-        const int sc = b0 + c;
-        const float fw = sBt[sc] * sGm[sc], fu = sBt[sc];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          if (lane < 16) sT[(b0 + r) * kTs + sc] = col[r];
-          const float nw = __shfl_down_sync(0xffffffffu, col[r] * fw, 1);
-          const float nu = __shfl_down_sync(0xffffffffu, col[r] * fu, 1);
-          if (lane < 16 && (c & 1) == 0) {
-            const uint32_t off = swz(kOffTw2, b0 + r, sc >> 3, kRow64) + 2 * (sc & 7);
-            st_bf16x2(smem, off, col[r] * fw, nw);
-            st_bf16x2(smem, off - kOffTw2 + kOffTu2, col[r] * fu, nu);
-          }
-        }
-      }
-      __syncthreads();
-      // block row bi: T_{bi,j} = -T_{bi,bi} sum_{k=j}^{bi-1} L_{bi,k} T_{k,j}, warp j < bi
-#pragma unroll 1
-      for (int bi = 1; bi < 4; ++bi) {
-        if (warp < bi) {
-          const int bj = warp;
-          const int g = lane >> 2, t = lane & 3;
-          float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-          for (int bk = bj; bk < bi; ++bk)
-            mma16x16x16_tf32(x, sL + (16 * bi) * kLs + 16 * bk, kLs, sT + (16 * bk) * kTs + 16 * bj, kTs, lane);
-          float* xs = sX + warp * 16 * kXs;  // per-warp scratch
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            xs[g * kXs + 8 * nt + 2 * t] = x[nt][0];
-            xs[g * kXs + 8 * nt + 2 * t + 1] = x[nt][1];
-            xs[(g + 8) * kXs + 8 * nt + 2 * t] = x[nt][2];
-            xs[(g + 8) * kXs + 8 * nt + 2 * t + 1] = x[nt][3];
-          }
-          __syncwarp();
-          float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-          mma16x16x16_tf32(y, sT + (16 * bi) * kTs + 16 * bi, kTs, xs, kXs, lane);
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-            for (int hlf = 0; hlf < 2; ++hlf) {
-              const int r = 16 * bi + g + 8 * hlf, c = 16 * bj + 8 * nt + 2 * t;
-              const float v0 = -y[nt][2 * hlf], v1 = -y[nt][2 * hlf + 1];
-              sT[r * kTs + c] = v0;
-              sT[r * kTs + c + 1] = v1;
-              const uint32_t off = swz(kOffTw2, r, c >> 3, kRow64) + 2 * (c & 7);
-              st_bf16x2(smem, off, v0 * sBt[c] * sGm[c], v1 * sBt[c + 1] * sGm[c + 1]);
-              st_bf16x2(smem, off - kOffTw2 + kOffTu2, v0 * sBt[c], v1 * sBt[c + 1]);
-            }
-          }
-        }
-        __syncthreads();
-      }
-      // Tw, Tu and the gate block to the workspace (the layout as is)
-      uint4* dstw = reinterpret_cast<uint4*>(static_cast<unsigned char*>(const_cast<void*>(p.workspace)) +
-                                             (((int64_t)((t0 + c0) / kC + seq)) * H + h) * kPrepTileBytes);
-      const uint4* srcw = reinterpret_cast<const uint4*>(smem + kPOffTw);
-      for (int idx = tid; idx < kPrepTileBytes / 16; idx += kThreads) dstw[idx] = srcw[idx];
-      __syncthreads();
     }
+    __syncthreads();  // L complete; the K space is free for Tw, Tu
+
+    // T = (I + L)^-1, column c = 32 w + lane: x_r = [r == c] - sum_{s < r} L_rs x_s.  Rows
+    // above c stay zero, so warp 1 (c >= 32) starts at row 32.
+    {
+      const int c = 32 * warp + lane;
+      float x[kC];
+#pragma unroll
+      for (int r = 0; r < kC; ++r) x[r] = (r == c) ? 1.0f : 0.0f;
+      if (warp == 0) {
+#pragma unroll
+        for (int r = 1; r < kC; ++r) {
+          float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+          for (int s4 = 0; s4 < r; s4 += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(sL + r * kLs + s4);
+            float& a = ((s4 >> 2) & 1) ? a1 : a0;
+            a = fmaf(l4.x, x[s4], a);
+            if (s4 + 1 < r) a = fmaf(l4.y, x[s4 + 1], a);
+            if (s4 + 2 < r) a = fmaf(l4.z, x[s4 + 2], a);
+            if (s4 + 3 < r) a = fmaf(l4.w, x[s4 + 3], a);
+          }
+          x[r] -= a0 + a1;
+        }
+      } else {
+#pragma unroll
+        for (int r = 33; r < kC; ++r) {
+          float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+          for (int s4 = 32; s4 < r; s4 += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(sL + r * kLs + s4);
+            float& a = ((s4 >> 2) & 1) ? a1 : a0;
+            a = fmaf(l4.x, x[s4], a);
+            if (s4 + 1 < r) a = fmaf(l4.y, x[s4 + 1], a);
+            if (s4 + 2 < r) a = fmaf(l4.z, x[s4 + 2], a);
+            if (s4 + 3 < r) a = fmaf(l4.w, x[s4 + 3], a);
+          }
+          x[r] -= a0 + a1;
+        }
+      }
+      // Tw = T diag(b gamma), Tu = T diag(b) (BF16, rows 128 bytes apart, piece ^ (row & 7))
+      const float fw = sBt[c] * sGm[c], fu = sBt[c];
+#pragma unroll
+      for (int r = 0; r < kC; ++r) {
+        const uint32_t off = kPOffK + r * kRow64 + (((c >> 3) ^ (r & 7)) << 4) + 2 * (c & 7);
+        *reinterpret_cast<__nv_bfloat16*>(smem + off) = __float2bfloat16_rn(x[r] * fw);
+        *reinterpret_cast<__nv_bfloat16*>(smem + off + kC * kRow64) = __float2bfloat16_rn(x[r] * fu);
+      }
+    }
+    __syncthreads();
+    // Tw, Tu and the gate block to the workspace (contiguous in shared memory as in the tile)
+    uint4* dstw = reinterpret_cast<uint4*>(static_cast<unsigned char*>(const_cast<void*>(p.workspace)) +
+                                           ((int64_t)gc * H + h) * kPrepTileBytes);
+    const uint4* srcw = reinterpret_cast<const uint4*>(smem + kPOffK);
+    for (int idx = tid; idx < kPrepTileBytes / 16; idx += kPThreads) dstw[idx] = srcw[idx];
+    __syncthreads();
   }
 }
 
 template <int RULE>
 cudaError_t launch_chunk_prep(const ScanParams& p, cudaStream_t stream) {
   const void* fn = reinterpret_cast<const void*>(&chunk_prep_kernel<RULE>);
-  const int per_sm = prepare_kernel(fn, chunk::kThreads, chunk::kPSmem);
+  const int per_sm = prepare_kernel(fn, chunk::kPThreads, chunk::kPSmem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;
-  const int64_t units = (int64_t)p.n_seqs * p.n_v_heads;
+  const int64_t items = ((int64_t)(p.total_tokens + chunk::kC - 1) / chunk::kC + p.n_seqs + 1) * p.n_v_heads;
   const int64_t cap = (int64_t)device_sm_count() * per_sm;
-  const int grid = (int)(units < cap ? units : cap);
-  chunk_prep_kernel<RULE><<<grid, chunk::kThreads, chunk::kPSmem, stream>>>(p);
+  const int grid = (int)(items < cap ? items : cap);
+  if (grid <= 0) return cudaSuccess;
+  chunk_prep_kernel<RULE><<<grid, chunk::kPThreads, chunk::kPSmem, stream>>>(p);
   return cudaGetLastError();
 }
 
