@@ -793,52 +793,71 @@ __global__ void __launch_bounds__(chunk::kPThreads) chunk_prep_kernel(const Scan
     }
     __syncthreads();  // L complete; the K space is free for Tw, Tu
 
-    // T = (I + L)^-1, column c = 32 w + lane: x_r = [r == c] - sum_{s < r} L_rs x_s.  Rows
-    // above c stay zero, so warp 1 (c >= 32) starts at row 32.
+    // T = (I + L)^-1 by 32 x 32 blocks, L = [L00 0; L10 L11]:  T = [A 0; C D] with
+    // A = (I + L00)^-1 (warp 0) and D = (I + L11)^-1 (warp 1) by forward substitution in
+    // FP32, one column per lane (x_r = [r == c] - sum_{s < r} L_rs x_s, four partial sums),
+    // then C = -D (L10 A) by both warps.  A, D and M = L10 A pass through the K space.
     {
-      const int c = 32 * warp + lane;
-      float x[kC];
+      float* sA = reinterpret_cast<float*>(smem + kPOffK);  // [32][33] fp32
+      float* sD = sA + 32 * 33;
+      float* sM = sD + 32 * 33;
+      const int r0 = 32 * warp;
+      float x[32];
 #pragma unroll
-      for (int r = 0; r < kC; ++r) x[r] = (r == c) ? 1.0f : 0.0f;
-      if (warp == 0) {
+      for (int r = 0; r < 32; ++r) x[r] = (r == lane) ? 1.0f : 0.0f;
 #pragma unroll
-        for (int r = 1; r < kC; ++r) {
-          float a0 = 0.0f, a1 = 0.0f;
+      for (int r = 1; r < 32; ++r) {
+        float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
 #pragma unroll
-          for (int s4 = 0; s4 < r; s4 += 4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(sL + r * kLs + s4);
-            float& a = ((s4 >> 2) & 1) ? a1 : a0;
-            a = fmaf(l4.x, x[s4], a);
-            if (s4 + 1 < r) a = fmaf(l4.y, x[s4 + 1], a);
-            if (s4 + 2 < r) a = fmaf(l4.z, x[s4 + 2], a);
-            if (s4 + 3 < r) a = fmaf(l4.w, x[s4 + 3], a);
-          }
-          x[r] -= a0 + a1;
+        for (int s4 = 0; s4 < r; s4 += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(sL + (r0 + r) * kLs + r0 + s4);
+          a0 = fmaf(l4.x, x[s4], a0);
+          if (s4 + 1 < r) a1 = fmaf(l4.y, x[s4 + 1], a1);
+          if (s4 + 2 < r) a2 = fmaf(l4.z, x[s4 + 2], a2);
+          if (s4 + 3 < r) a3 = fmaf(l4.w, x[s4 + 3], a3);
         }
-      } else {
-#pragma unroll
-        for (int r = 33; r < kC; ++r) {
-          float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-          for (int s4 = 32; s4 < r; s4 += 4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(sL + r * kLs + s4);
-            float& a = ((s4 >> 2) & 1) ? a1 : a0;
-            a = fmaf(l4.x, x[s4], a);
-            if (s4 + 1 < r) a = fmaf(l4.y, x[s4 + 1], a);
-            if (s4 + 2 < r) a = fmaf(l4.z, x[s4 + 2], a);
-            if (s4 + 3 < r) a = fmaf(l4.w, x[s4 + 3], a);
-          }
-          x[r] -= a0 + a1;
-        }
+        x[r] -= (a0 + a1) + (a2 + a3);
       }
+      float* sBlk = warp == 0 ? sA : sD;
+#pragma unroll
+      for (int r = 0; r < 32; ++r) sBlk[r * 33 + lane] = x[r];
+      __syncthreads();
+      // M = L10 A: column lane, rows 16 warp .. + 15
+      float acc[16];
+#pragma unroll
+      for (int i2 = 0; i2 < 16; ++i2) acc[i2] = 0.0f;
+#pragma unroll 4
+      for (int k = 0; k < 32; ++k) {
+        const float a = sA[k * 33 + lane];
+#pragma unroll
+        for (int i2 = 0; i2 < 16; ++i2) acc[i2] = fmaf(sL[(32 + 16 * warp + i2) * kLs + k], a, acc[i2]);
+      }
+#pragma unroll
+      for (int i2 = 0; i2 < 16; ++i2) sM[(16 * warp + i2) * 33 + lane] = acc[i2];
+      __syncthreads();
+      // C = -D M: column lane, rows 16 warp .. + 15
+#pragma unroll
+      for (int i2 = 0; i2 < 16; ++i2) acc[i2] = 0.0f;
+#pragma unroll 4
+      for (int k = 0; k < 32; ++k) {
+        const float mv = sM[k * 33 + lane];
+#pragma unroll
+        for (int i2 = 0; i2 < 16; ++i2) acc[i2] = fmaf(sD[(16 * warp + i2) * 33 + k], mv, acc[i2]);
+      }
+      __syncthreads();  // A, D and M are read: the K space takes Tw, Tu
       // Tw = T diag(b gamma), Tu = T diag(b) (BF16, rows 128 bytes apart, piece ^ (row & 7))
-      const float fw = sBt[c] * sGm[c], fu = sBt[c];
-#pragma unroll
-      for (int r = 0; r < kC; ++r) {
+      auto put = [&](int r, int c, float v) {
         const uint32_t off = kPOffK + r * kRow64 + (((c >> 3) ^ (r & 7)) << 4) + 2 * (c & 7);
-        *reinterpret_cast<__nv_bfloat16*>(smem + off) = __float2bfloat16_rn(x[r] * fw);
-        *reinterpret_cast<__nv_bfloat16*>(smem + off + kC * kRow64) = __float2bfloat16_rn(x[r] * fu);
+        *reinterpret_cast<__nv_bfloat16*>(smem + off) = __float2bfloat16_rn(v * sBt[c] * sGm[c]);
+        *reinterpret_cast<__nv_bfloat16*>(smem + off + kC * kRow64) = __float2bfloat16_rn(v * sBt[c]);
+      };
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        put(r0 + r, r0 + lane, x[r]);           // A or D
+        if (warp == 1) put(r, 32 + lane, 0.0f);  // the zero block above D
       }
+#pragma unroll
+      for (int i2 = 0; i2 < 16; ++i2) put(32 + 16 * warp + i2, lane, -acc[i2]);  // C
     }
     __syncthreads();
     // Tw, Tu and the gate block to the workspace (contiguous in shared memory as in the tile)

@@ -62,8 +62,8 @@ constexpr int kColS = 0;     // S^T   128 columns (d_k)
 constexpr int kColP = 128;   // [Q; K] K^T, 64 columns (lanes 0..63 are Q K^T)
 constexpr int kColW = 192;   // W^T   64
 constexpr int kColU = 256;   // U^T   64
-constexpr int kColO1 = 320;  // S0^T Q^T   64
-constexpr int kColO2 = 384;  // U^T P^T    64
+constexpr int kColO1 = 320;  // S0^T Q^T   2 x 64 (chunk parity: read back during the next chunk)
+constexpr int kColO2 = 448;  // U^T P^T    64
 
 __device__ __forceinline__ uint4 pack8(const uint32_t* r) {
   return make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
@@ -202,24 +202,48 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       cp_async_commit();
     };
 
+    // The outputs of chunk cj: o_t[j] = scale (gamma_t O1^T[j][t] + O2^T[j][t]), lane = j,
+    // into the U space as a row-major [64][128] BF16 tile (o_tile), then its rows to o,
+    // 256 contiguous bytes per token (o_rows).  Both run one chunk late, beside the next
+    // chunk's first two MMA groups on the tensor cores.
+    __nv_bfloat16* sO = reinterpret_cast<__nv_bfloat16*>(smem + kOffU);
+    auto o_tile = [&](int cj) {
+      const float* gm = reinterpret_cast<const float*>(smem + (cj & 1) * kBufBytes + kOffGB);
+#pragma unroll
+      for (int c16 = 0; c16 < 2; ++c16) {
+        uint32_t r1[16], r2[16];
+        umma::ld16(tq + kColO1 + 64 * (cj & 1) + 32 * hf + 16 * c16, r1);
+        umma::ld16(tq + kColO2 + 32 * hf + 16 * c16, r2);
+        umma::wait_ld();
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const int t = 32 * hf + 16 * c16 + x;
+          sO[t * kD + lrow] =
+              __float2bfloat16_rn(p.scale * (gm[t] * __uint_as_float(r1[x]) + __uint_as_float(r2[x])));
+        }
+      }
+    };
+    auto o_rows = [&](int cj) {
+      const int cc0 = cj * kC;
+      const int nn = (n_tok - cc0) < kC ? (n_tok - cc0) : kC;
+      for (int idx = tid; idx < kC * 16; idx += kThreads) {
+        const int t = idx >> 4, ch = idx & 15;
+        if (t < nn)
+          *reinterpret_cast<uint4*>(og + ((int64_t)(t0 + cc0 + t) * H + h) * kD + ch * 8) =
+              *reinterpret_cast<const uint4*>(sO + t * kD + ch * 8);
+      }
+    };
+
     if (n_chunks > 0) stage(0);
 #pragma unroll 1
     for (int ci = 0; ci < n_chunks; ++ci) {
-      const int c0 = ci * kC;
-      const int n = (n_tok - c0) < kC ? (n_tok - c0) : kC;
       const uint32_t bq = sb + (ci & 1) * kBufBytes + kOffQK;  // Q rows
       const uint32_t bk = bq + kC * 128;                        // K rows (same panels)
       const uint32_t bv = sb + (ci & 1) * kBufBytes + kOffV;
       const uint32_t btw = sb + (ci & 1) * kBufBytes + kOffTw;
-      if (ci + 1 < n_chunks) {
-        stage(ci + 1);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
+      cp_async_wait<0>();  // chunk ci (staged during chunk ci - 1)
       // ---- this chunk's gate quantities, from the workspace tile
       const float* gbk = reinterpret_cast<const float*>(smem + (ci & 1) * kBufBytes + kOffGB);
-      const float* sGm = gbk;            // gamma_t
       const float* sGu = gbk + kC;       // gamma_C / gamma_t
       const float* sFa = gbk + 2 * kC;   // gamma_t / e^m
       const float* sFb = gbk + 3 * kC;   // e^m / gamma_t
@@ -228,7 +252,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       umma::fence_smem();  // staged operands -> tensor cores
       __syncthreads();
       const bool fact = gbk[6 * kC] != 0.0f;
-      const float gC = sGm[kC - 1];  // padded tokens have gate 1: the last real token's
+      const float gC = gbk[kC - 1];  // gamma_C (padded tokens have gate 1: the last real token's)
 
       // ---- S pass: BF16 copy of S0^T for this chunk's products, then S^T *= gamma_C
 #pragma unroll 1
@@ -274,10 +298,11 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // K = d_k
           const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma::mma(tmem + kColO1, umma::sdesc_add(dS, ko), umma::sdesc_add(dQK, ko), kIdKK64, kk);
+          umma::mma(tmem + kColO1 + 64 * (ci & 1), umma::sdesc_add(dS, ko), umma::sdesc_add(dQK, ko), kIdKK64, kk);
         }
         umma::commit(&bars[0]);
       }
+      if (ci > 0) o_tile(ci - 1);  // beside group 1
       bool ok = mbar_wait(&bars[0], phase & 1u);
       umma::fence_after();
       // W^T rows (lane = d_k index) -> shared memory, the B operand of the U update
@@ -320,6 +345,10 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
         break;
       }
 
+      // the next chunk into buffer (ci + 1) & 1, whose operands and gates chunk ci - 1 no
+      // longer needs
+      if (ci + 1 < n_chunks) stage(ci + 1);
+
       // ---- group 2: U^T -= S0^T W^T
       if (tid == 0) {
         umma::fence_after();
@@ -331,6 +360,8 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
         }
         umma::commit(&bars[1]);
       }
+      if (ci > 0) o_rows(ci - 1);  // beside group 2
+      __syncthreads();              // the U space is rewritten below
       ok = mbar_wait(&bars[1], phase & 1u);
       umma::fence_after();
       // U^T rows (lane = d_v index) -> U and Us = U (gamma_C / gamma_t) per token column
@@ -372,37 +403,19 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       }
       ok = mbar_wait(&bars[2], phase & 1u);
       umma::fence_after();
-      // O rows: o_t[j] = scale (gamma_t O1^T[j][t] + O2^T[j][t]), lane = j, into the U
-      // space (free once group 3 is done) as a row-major [64][128] BF16 tile
-      __nv_bfloat16* sO = reinterpret_cast<__nv_bfloat16*>(smem + kOffU);
-#pragma unroll
-      for (int c16 = 0; c16 < 2; ++c16) {
-        uint32_t r1[16], r2[16];
-        umma::ld16(tq + kColO1 + 32 * hf + 16 * c16, r1);
-        umma::ld16(tq + kColO2 + 32 * hf + 16 * c16, r2);
-        umma::wait_ld();
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const int t = 32 * hf + 16 * c16 + x;
-          sO[t * kD + lrow] =
-              __float2bfloat16_rn(p.scale * (sGm[t] * __uint_as_float(r1[x]) + __uint_as_float(r2[x])));
-        }
-      }
       umma::fence_before();
       if (__syncthreads_or(!ok)) {
         abort = true;
         break;
       }
-      // the tile's rows to o (256 contiguous bytes per token)
-      for (int idx = tid; idx < kC * 16; idx += kThreads) {
-        const int t = idx >> 4, ch = idx & 15;
-        if (t < n)
-          *reinterpret_cast<uint4*>(og + ((int64_t)(t0 + c0 + t) * H + h) * kD + ch * 8) =
-              *reinterpret_cast<const uint4*>(sO + t * kD + ch * 8);
-      }
       ++phase;
     }
     if (abort) break;
+    if (n_chunks > 0) {
+      o_tile(n_chunks - 1);
+      __syncthreads();
+      o_rows(n_chunks - 1);
+    }
 
     // ---- final state: S[i][j] = S^T[j][i], lane j, columns i
     const int64_t dbase = ((int64_t)ws * H + h) * (kD * kD);
