@@ -19,9 +19,10 @@
 // that owns a lane writes whole operand rows back to shared memory.  The master state
 // S^T (d_v lanes x d_k columns, FP32) stays in tensor memory for the whole sequence.
 //
-// One CTA of 8 warps per SM; warp w reads tensor-memory lanes 32 (w % 4) .. + 31 and the
-// column half w / 4 of each accumulator.  Thread 0 issues the MMAs; three mbarriers signal
-// their completion, and every wait gives up after a time limit (LA_DEVERR_TIMEOUT).
+// One CTA of 9 warps per SM: worker warp w < 8 reads tensor-memory lanes 32 (w % 4) .. + 31
+// and the column half w / 4 of each accumulator; lane 0 of warp 8 only issues the MMAs, so
+// issuing never holds up an epilogue.  Three mbarriers signal the completion of each MMA
+// group, and every wait gives up after a time limit (LA_DEVERR_TIMEOUT).
 #pragma once
 
 #include <cstdint>
@@ -34,7 +35,8 @@ namespace chunk_tc {
 
 constexpr int kC = 64;   // tokens per chunk
 constexpr int kD = 128;  // d_k = d_v
-constexpr int kThreads = 256;
+constexpr int kWorkers = 256;             // 8 warps: tensor-memory epilogues, staging
+constexpr int kThreads = kWorkers + 32;   // + 1 warp whose lane 0 issues the MMAs
 
 // shared memory (bytes from a 1024-byte aligned base); operands in 64-column panels
 constexpr int kBufBytes = 67584;             // one staged chunk:
@@ -89,8 +91,9 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  const bool worker = warp < 8;
   const int q4 = warp & 3;         // tensor-memory lane quarter
-  const int hf = warp >> 2;        // column half
+  const int hf = (warp >> 2) & 1;  // column half
   const int lrow = 32 * q4 + lane; // this thread's lane: a d_v (or d_k, or token) index
   const int H = p.n_v_heads;
   const int ratio_h = H / p.n_qk_heads;
@@ -153,7 +156,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
     // ---- initial state S^T into tensor memory: lane = d_v index, columns = d_k (64 per half)
     const int64_t sbase_src = ((int64_t)rs * H + h) * (kD * kD);
 #pragma unroll 1
-    for (int c16 = 0; c16 < 4; ++c16) {
+    for (int c16 = 0; c16 < (worker ? 4 : 0); ++c16) {
       uint32_t r[16];
 #pragma unroll
       for (int x = 0; x < 16; ++x) {
@@ -168,7 +171,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       }
       umma::st16(tq + kColS + 64 * hf + 16 * c16, r);
     }
-    umma::wait_st();
+    if (worker) umma::wait_st();
 
     const int n_tok = t1 - t0;
     const int n_chunks = (n_tok + kC - 1) / kC;
@@ -208,6 +211,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
     // chunk's first two MMA groups on the tensor cores.
     __nv_bfloat16* sO = reinterpret_cast<__nv_bfloat16*>(smem + kOffU);
     auto o_tile = [&](int cj) {
+      if (!worker) return;
       const float* gm = reinterpret_cast<const float*>(smem + (cj & 1) * kBufBytes + kOffGB);
 #pragma unroll
       for (int c16 = 0; c16 < 2; ++c16) {
@@ -256,7 +260,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
 
       // ---- S pass: BF16 copy of S0^T for this chunk's products, then S^T *= gamma_C
 #pragma unroll 1
-      for (int c16 = 0; c16 < 4; ++c16) {
+      for (int c16 = 0; c16 < (worker ? 4 : 0); ++c16) {
         uint32_t r[16];
         umma::ld16(tq + kColS + 64 * hf + 16 * c16, r);
         umma::wait_ld();
@@ -270,7 +274,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
           umma::st16(tq + kColS + 64 * hf + 16 * c16, r);
         }
       }
-      if (kGate) umma::wait_st();
+      if (kGate && worker) umma::wait_st();
       umma::fence_smem();
       umma::fence_before();
       __syncthreads();
@@ -280,7 +284,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       const uint64_t dQK = umma::sdesc(bq, 16, 1024);     // [Q; K] rows, K-major
       const uint64_t dKm = umma::sdesc(bk, 16384, 1024);  // K as an MN-major operand
       const uint64_t dS = umma::sdesc(sb + kOffS, 16, 1024);
-      if (tid == 0) {
+      if (tid == kWorkers) {
         umma::fence_after();
         const uint64_t dVm = umma::sdesc(bv, 8192, 1024);
         const uint64_t dTw = umma::sdesc(btw, 16, 1024);
@@ -307,7 +311,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       umma::fence_after();
       // W^T rows (lane = d_k index) -> shared memory, the B operand of the U update
 #pragma unroll
-      for (int c16 = 0; c16 < 2; ++c16) {
+      for (int c16 = 0; c16 < (worker ? 2 : 0); ++c16) {
         uint32_t r[16];
         umma::ld16(tq + kColW + 32 * hf + 16 * c16, r);
         umma::wait_ld();
@@ -317,7 +321,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
               pack8(r + 8 * pc);
       }
       // P rows (lanes 0..63 = token t): masked by the gate ratios
-      if (q4 < 2) {
+      if (worker && q4 < 2) {
         const int t = lrow;
 #pragma unroll
         for (int c16 = 0; c16 < 2; ++c16) {
@@ -350,7 +354,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       if (ci + 1 < n_chunks) stage(ci + 1);
 
       // ---- group 2: U^T -= S0^T W^T
-      if (tid == 0) {
+      if (tid == kWorkers) {
         umma::fence_after();
         const uint64_t dWm = umma::sdesc(sb + kOffW, 16384, 1024);
 #pragma unroll
@@ -366,7 +370,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       umma::fence_after();
       // U^T rows (lane = d_v index) -> U and Us = U (gamma_C / gamma_t) per token column
 #pragma unroll
-      for (int c16 = 0; c16 < 2; ++c16) {
+      for (int c16 = 0; c16 < (worker ? 2 : 0); ++c16) {
         uint32_t r[16];
         umma::ld16(tq + kColU + 32 * hf + 16 * c16, r);
         umma::wait_ld();
@@ -389,7 +393,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       }
 
       // ---- group 3: O2^T = U^T P^T ;  S^T += Us^T K
-      if (tid == 0) {
+      if (tid == kWorkers) {
         umma::fence_after();
         const uint64_t dP = umma::sdesc(sb + kOffP, 16, 1024);
         const uint64_t dU = umma::sdesc(sb + kOffU, 16, 1024);
@@ -420,7 +424,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
     // ---- final state: S[i][j] = S^T[j][i], lane j, columns i
     const int64_t dbase = ((int64_t)ws * H + h) * (kD * kD);
 #pragma unroll 1
-    for (int c16 = 0; c16 < 4; ++c16) {
+    for (int c16 = 0; c16 < (worker ? 4 : 0); ++c16) {
       uint32_t r[16];
       umma::ld16(tq + kColS + 64 * hf + 16 * c16, r);
       umma::wait_ld();
