@@ -50,8 +50,8 @@ constexpr int kOffW = kOffS + 32768;         // W^T   [128 d_k][64]
 constexpr int kOffP = kOffW + 16384;         // P     [64][64]
 constexpr int kOffU = kOffP + 8192;          // U^T   [128 d_v][64]; O [64][128] row-major at the end
 constexpr int kOffUs = kOffU + 16384;        // Us^T  [128 d_v][64]
-constexpr int kOffBar = kOffUs + 16384;
-constexpr int kOffMisc = kOffBar + 3 * 8;    // [0] tensor-memory base
+constexpr int kOffBar = kOffUs + 16384;      // MMA groups 1-3, then the two staging buffers
+constexpr int kOffMisc = kOffBar + 5 * 8;    // [0] tensor-memory base
 constexpr int kSmem = kOffMisc + 16 + 1024;  // + slack for the 1024-byte alignment
 static_assert(kSmem <= 227 * 1024, "shared memory");
 static_assert(chunk::kPrepTileBytes == 16384 + chunk::kGateBlockBytes && kOffTu == kOffTw + 8192 &&
@@ -74,10 +74,21 @@ __device__ __forceinline__ uint4 pack8(const uint32_t* r) {
                     pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
 }
 
+// bytes that land in a staging buffer per chunk: Q, K, V (two 64 x 64 panels each) and
+// the workspace tile
+constexpr uint32_t kStageBytes = 6 * kC * 128 + chunk::kPrepTileBytes;
+
 }  // namespace chunk_tc
 
+// Tensor maps of q, k and v, each [tokens][heads][128] BF16 viewed as the 3-D array
+// {128, heads, tokens}; box {64, 1, 64} with the 128-byte swizzle, i.e. one 64 x 64 panel.
+struct TcMaps {
+  CUtensorMap q, k, v;
+};
+
 template <int RULE>
-__global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const ScanParams p) {
+__global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const ScanParams p,
+                                                                         const __grid_constant__ TcMaps maps) {
   using namespace chunk_tc;
   static_assert(Rule<RULE>::kPredicts, "the delta rules only");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -99,9 +110,6 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
   const int ratio_h = H / p.n_qk_heads;
   const int64_t units = (int64_t)p.n_seqs * H;
   const int64_t G = gridDim.x;
-  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
-  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(p.k);
-  const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(p.v);
   __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.o);
 
   if (warp == 0) umma::alloc(const_cast<uint32_t*>(misc), kTmemCols);
@@ -109,6 +117,8 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
     mbar_init(&bars[2], 1);
+    mbar_init(&bars[3], 1);
+    mbar_init(&bars[4], 1);
     mbar_init_fence();
   }
   umma::fence_before();
@@ -116,7 +126,9 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
   umma::fence_after();
   const uint32_t tmem = misc[0];
   const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);  // this warp's lane quarter
-  uint32_t phase = 0;  // chunks completed by this CTA: the parity of all three barriers
+  uint32_t phase = 0;   // chunks completed by this CTA: the parity of the MMA-group barriers
+  uint32_t lpar = 0;    // bit b: the parity of staging buffer b's next completion
+  uint32_t pending = 0; // bit b: staging buffer b has copies in flight (issuer lane)
   bool abort = false;
 
   // instruction descriptors
@@ -176,33 +188,27 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
     const int n_tok = t1 - t0;
     const int n_chunks = (n_tok + kC - 1) / kC;
 
-    // Stages chunk ci (Q, K, V rows; Tw, Tu and the gate block from the workspace) into
-    // buffer ci & 1; rows beyond the sequence are zero.
+    // Stages chunk ci into buffer ci & 1 with the TMA engine (the issuer lane): the Q, K and
+    // V panels by tensor maps (rows beyond the last token read as zero) and the workspace
+    // tile (Tw, Tu, gate block) as one bulk copy; all of it completes on bars[3 + (ci & 1)].
     auto stage = [&](int ci) {
-      const int cc0 = ci * kC;
-      const int nn = (n_tok - cc0) < kC ? (n_tok - cc0) : kC;
-      unsigned char* buf = smem + (ci & 1) * kBufBytes;
-      for (int idx = tid; idx < kC * 16; idx += kThreads) {
-        const int r = idx >> 4, ch = idx & 15;
-        unsigned char* dq = buf + kOffQK + umma::panel_piece(128, r, ch);
-        unsigned char* dk = buf + kOffQK + umma::panel_piece(128, r + kC, ch);
-        unsigned char* dv = buf + kOffV + umma::panel_piece(kC, r, ch);
-        if (r < nn) {
-          const int64_t tok = t0 + cc0 + r;
-          cp_async_16(dq, qg + (tok * p.n_qk_heads + hq) * kD + ch * 8);
-          cp_async_16(dk, kg + (tok * p.n_qk_heads + hq) * kD + ch * 8);
-          cp_async_16(dv, vg + (tok * H + h) * kD + ch * 8);
-        } else {
-          *reinterpret_cast<uint4*>(dq) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(dk) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(dv) = make_uint4(0, 0, 0, 0);
-        }
+      if (tid != kWorkers) return;
+      const int b = ci & 1;
+      unsigned char* buf = smem + b * kBufBytes;
+      const int tok0 = t0 + ci * kC;
+      uint64_t* full = &bars[3 + b];
+      mbar_arrive_expect_tx(full, kStageBytes);
+#pragma unroll
+      for (int pnl = 0; pnl < 2; ++pnl) {
+        umma::tma_load_3d(buf + kOffQK + pnl * 16384, &maps.q, 64 * pnl, hq, tok0, full);
+        umma::tma_load_3d(buf + kOffQK + pnl * 16384 + kC * 128, &maps.k, 64 * pnl, hq, tok0, full);
+        umma::tma_load_3d(buf + kOffV + pnl * 8192, &maps.v, 64 * pnl, h, tok0, full);
       }
-      const unsigned char* wsrc = static_cast<const unsigned char*>(p.workspace) +
-                                  (((int64_t)((t0 + cc0) / kC + seq)) * H + h) * chunk::kPrepTileBytes;
-      for (int idx = tid; idx < chunk::kPrepTileBytes / 16; idx += kThreads)
-        cp_async_16(buf + kOffTw + idx * 16, wsrc + idx * 16);
-      cp_async_commit();
+      bulk_g2s(buf + kOffTw,
+               static_cast<const unsigned char*>(p.workspace) +
+                   (((int64_t)(tok0 / kC + seq)) * H + h) * chunk::kPrepTileBytes,
+               chunk::kPrepTileBytes, full);
+      pending |= 1u << b;
     };
 
     // The outputs of chunk cj: o_t[j] = scale (gamma_t O1^T[j][t] + O2^T[j][t]), lane = j,
@@ -245,7 +251,21 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       const uint32_t bk = bq + kC * 128;                        // K rows (same panels)
       const uint32_t bv = sb + (ci & 1) * kBufBytes + kOffV;
       const uint32_t btw = sb + (ci & 1) * kBufBytes + kOffTw;
-      cp_async_wait<0>();  // chunk ci (staged during chunk ci - 1)
+      // chunk ci (staged during chunk ci - 1)
+      const bool okl = mbar_wait(&bars[3 + (ci & 1)], (lpar >> (ci & 1)) & 1u);
+      lpar ^= 1u << (ci & 1);
+      pending &= ~(1u << (ci & 1));
+      // rows past the end of the sequence: zero (they hold the next tokens of the array)
+      const int nrow = (n_tok - ci * kC) < kC ? (n_tok - ci * kC) : kC;
+      if (nrow < kC && worker) {
+        unsigned char* buf = smem + (ci & 1) * kBufBytes;
+        for (int idx = tid; idx < (kC - nrow) * 16; idx += kWorkers) {
+          const int r = nrow + (idx >> 4), ch = idx & 15;
+          *reinterpret_cast<uint4*>(buf + kOffQK + umma::panel_piece(128, r, ch)) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(buf + kOffQK + umma::panel_piece(128, r + kC, ch)) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(buf + kOffV + umma::panel_piece(kC, r, ch)) = make_uint4(0, 0, 0, 0);
+        }
+      }
       // ---- this chunk's gate quantities, from the workspace tile
       const float* gbk = reinterpret_cast<const float*>(smem + (ci & 1) * kBufBytes + kOffGB);
       const float* sGu = gbk + kC;       // gamma_C / gamma_t
@@ -253,8 +273,11 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       const float* sFb = gbk + 3 * kC;   // e^m / gamma_t
       const float* sLg = gbk + 4 * kC;   // log |gamma_t|
       const float* sSg = gbk + 5 * kC;   // sign gamma_t
-      umma::fence_smem();  // staged operands -> tensor cores
-      __syncthreads();
+      umma::fence_smem();  // zeroed rows -> tensor cores
+      if (__syncthreads_or(!okl)) {
+        abort = true;
+        break;
+      }
       const bool fact = gbk[6 * kC] != 0.0f;
       const float gC = gbk[kC - 1];  // gamma_C (padded tokens have gate 1: the last real token's)
 
@@ -437,15 +460,50 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
           static_cast<__nv_bfloat16*>(p.dst)[e] = __float2bfloat16_rn(__uint_as_float(r[x]));
       }
     }
+    umma::fence_smem();  // this unit's reads of the staging buffers precede the next unit's copies
     umma::fence_before();
     __syncthreads();
   }
 
-  cp_async_wait<0>();
+  // copies still in flight (only after a wait gave up): let them land, within the limit
+  if (tid == kWorkers) {
+    for (int b = 0; b < 2; ++b)
+      if (pending & (1u << b)) mbar_wait(&bars[3 + b], (lpar >> b) & 1u);
+  }
   if (abort && tid == 0) report(p.err, LA_DEVERR_TIMEOUT);
   umma::fence_before();
   __syncthreads();
   if (warp == 0) umma::dealloc(tmem, kTmemCols);
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+inline EncodeTiledFn encode_tiled_fn() {
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// [tokens][heads][128] BF16 rows as the 3-D array {128, heads, tokens}: 64 x 64 panels
+// with the 128-byte swizzle; reads past the last token return zero.
+inline bool encode_rows_map(CUtensorMap* m, const void* base, int heads, int64_t tokens) {
+  const EncodeTiledFn fn = encode_tiled_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {128, (cuuint64_t)heads, (cuuint64_t)(tokens > 0 ? tokens : 1)};
+  const cuuint64_t strides[2] = {256, (cuuint64_t)heads * 256};
+  const cuuint32_t box[3] = {64, 1, 64};
+  const cuuint32_t elem[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, elem,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int RULE>
@@ -454,10 +512,15 @@ cudaError_t launch_chunk_tc(const ScanParams& p, cudaStream_t stream) {
   const int per_sm = prepare_kernel(fn, chunk_tc::kThreads, chunk_tc::kSmem);
   // one CTA per SM: the kernel holds all of the SM's tensor memory
   if (per_sm != 1) return cudaErrorInvalidConfiguration;
+  TcMaps maps;
+  if (!encode_rows_map(&maps.q, p.q, p.n_qk_heads, p.total_tokens) ||
+      !encode_rows_map(&maps.k, p.k, p.n_qk_heads, p.total_tokens) ||
+      !encode_rows_map(&maps.v, p.v, p.n_v_heads, p.total_tokens))
+    return cudaErrorInvalidValue;
   const int64_t units = (int64_t)p.n_seqs * p.n_v_heads;
   const int64_t cap = device_sm_count();
   const int grid = (int)(units < cap ? units : cap);
-  chunk_tc_kernel<RULE><<<grid, chunk_tc::kThreads, chunk_tc::kSmem, stream>>>(p);
+  chunk_tc_kernel<RULE><<<grid, chunk_tc::kThreads, chunk_tc::kSmem, stream>>>(p, maps);
   return cudaGetLastError();
 }
 

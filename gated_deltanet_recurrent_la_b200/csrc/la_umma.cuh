@@ -9,6 +9,8 @@
 // as an MN-major operand (M or N along the 64 columns, K along the rows).
 #pragma once
 
+#include <cuda.h>
+
 #include <cstdint>
 
 #include "la_device.cuh"
@@ -94,6 +96,18 @@ __device__ __forceinline__ void st16(uint32_t taddr, const uint32_t* r) {
 }
 __device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Tiled TMA load of a 3-D box (coordinates in elements, innermost first) into shared
+// memory, completing its bytes on `bar`.  The innermost coordinate times the element size
+// is a multiple of 16 bytes at every call site (0 or 64 BF16 elements).
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_addr(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
+      : "memory");
+}
 
 // tensor-memory address of (lane, column)
 __device__ __forceinline__ uint32_t taddr(uint32_t base, int lane, int col) {
