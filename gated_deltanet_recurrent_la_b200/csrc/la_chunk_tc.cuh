@@ -50,7 +50,8 @@ constexpr int kOffW = kOffS + 32768;         // W^T   [128 d_k][64]
 constexpr int kOffP = kOffW + 16384;         // P     [64][64]
 constexpr int kOffU = kOffP + 8192;          // U^T   [128 d_v][64]; O [64][128] row-major at the end
 constexpr int kOffUs = kOffU + 16384;        // Us^T  [128 d_v][64]
-constexpr int kOffBar = kOffUs + 16384;      // MMA groups 1-3, then the two staging buffers
+constexpr int kOffGo = kOffUs + 16384;       // gamma_t of the last two chunks [2][64] fp32 (outputs)
+constexpr int kOffBar = kOffGo + 2 * kC * 4; // MMA groups 1-3, then the two staging buffers
 constexpr int kOffMisc = kOffBar + 5 * 8;    // [0] tensor-memory base
 constexpr int kSmem = kOffMisc + 16 + 1024;  // + slack for the 1024-byte alignment
 static_assert(kSmem <= 227 * 1024, "shared memory");
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
     __nv_bfloat16* sO = reinterpret_cast<__nv_bfloat16*>(smem + kOffU);
     auto o_tile = [&](int cj) {
       if (!worker) return;
-      const float* gm = reinterpret_cast<const float*>(smem + (cj & 1) * kBufBytes + kOffGB);
+      const float* gm = reinterpret_cast<const float*>(smem + kOffGo) + (cj & 1) * kC;
 #pragma unroll
       for (int c16 = 0; c16 < 2; ++c16) {
         uint32_t r1[16], r2[16];
@@ -251,7 +252,8 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       const uint32_t bk = bq + kC * 128;                        // K rows (same panels)
       const uint32_t bv = sb + (ci & 1) * kBufBytes + kOffV;
       const uint32_t btw = sb + (ci & 1) * kBufBytes + kOffTw;
-      // chunk ci (staged during chunk ci - 1)
+      // the next chunk into the other buffer (chunk ci - 1 is done with it), then chunk ci
+      if (ci + 1 < n_chunks) stage(ci + 1);
       const bool okl = mbar_wait(&bars[3 + (ci & 1)], (lpar >> (ci & 1)) & 1u);
       lpar ^= 1u << (ci & 1);
       pending &= ~(1u << (ci & 1));
@@ -266,8 +268,10 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
           *reinterpret_cast<uint4*>(buf + kOffV + umma::panel_piece(kC, r, ch)) = make_uint4(0, 0, 0, 0);
         }
       }
-      // ---- this chunk's gate quantities, from the workspace tile
+      // ---- this chunk's gate quantities, from the workspace tile; gamma_t also kept for the
+      //      output epilogue, which runs during the next chunk
       const float* gbk = reinterpret_cast<const float*>(smem + (ci & 1) * kBufBytes + kOffGB);
+      if (tid < kC) reinterpret_cast<float*>(smem + kOffGo)[(ci & 1) * kC + tid] = gbk[tid];
       const float* sGu = gbk + kC;       // gamma_C / gamma_t
       const float* sFa = gbk + 2 * kC;   // gamma_t / e^m
       const float* sFb = gbk + 3 * kC;   // e^m / gamma_t
@@ -372,10 +376,6 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
         break;
       }
 
-      // the next chunk into buffer (ci + 1) & 1, whose operands and gates chunk ci - 1 no
-      // longer needs
-      if (ci + 1 < n_chunks) stage(ci + 1);
-
       // ---- group 2: U^T -= S0^T W^T
       if (tid == kWorkers) {
         umma::fence_after();
@@ -430,6 +430,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       }
       ok = mbar_wait(&bars[2], phase & 1u);
       umma::fence_after();
+      umma::fence_smem();  // this chunk's reads of its staging buffer precede the copies into it
       umma::fence_before();
       if (__syncthreads_or(!ok)) {
         abort = true;
