@@ -792,7 +792,8 @@ def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_ev
             row["roofline"] = tensor_roofline(run, inp, ms, peaks)
         else:
             row["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
-                               "traffic": recorded_traffic("scan", name), "hbm_gb_s": row["gb_s"],
+                               "traffic": recorded_traffic("scan", name + (f"_ckpt{ckpt_every}" if ckpt_every else "")),
+                               "hbm_gb_s": row["gb_s"],
                                "effective_state_gb_s": run.T * inp.n_v_heads * 2 * inp.d_k * inp.d_v * 4 /
                                (ms * 1e-3) / 1e9,
                                "peak_note": "SMs x 128 FP32 lanes x 2 x max SM clock"}
