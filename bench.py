@@ -578,8 +578,8 @@ def time_e2e(run: DecodeRunner, steps, warmup, world):
     import torch
     inp = run.inp
     L = run.L
-    parts = [inp.q, inp.k, inp.v, inp.g, inp.beta]
-    sizes = [p.numel() * p.element_size() for p in parts] + [run.B * 4, run.B * 4]
+    parts = [inp.q, inp.k, inp.v, inp.g, inp.beta]  # g / beta are None for rules that ignore them
+    sizes = [0 if p is None else p.numel() * p.element_size() for p in parts] + [run.B * 4, run.B * 4]
     offs, total = [], 0
     for sz in sizes:
         offs.append(total)
@@ -589,7 +589,8 @@ def time_e2e(run: DecodeRunner, steps, warmup, world):
     for r, w in run.sets:
         hb = torch.zeros(total, dtype=torch.uint8, pin_memory=True)
         for p, off in zip(parts, offs):
-            hb[off:off + p.numel() * p.element_size()].copy_(p.contiguous().view(-1).view(torch.uint8))
+            if p is not None:
+                hb[off:off + p.numel() * p.element_size()].copy_(p.contiguous().view(-1).view(torch.uint8))
         if r is not None:
             hb[offs[5]:offs[5] + run.B * 4].copy_(r.cpu().view(torch.uint8))
             hb[offs[6]:offs[6] + run.B * 4].copy_(w.cpu().view(torch.uint8))
@@ -606,7 +607,8 @@ def time_e2e(run: DecodeRunner, steps, warmup, world):
                 n *= x
             return dev[offs[i]:offs[i] + n * torch.empty(0, dtype=dtype).element_size()].view(dtype).view(shape)
         return (v(0, inp.q.dtype, inp.q.shape), v(1, inp.k.dtype, inp.k.shape), v(2, inp.v.dtype, inp.v.shape),
-                v(3, torch.float32, inp.g.shape), v(4, torch.float32, inp.beta.shape),
+                v(3, torch.float32, inp.g.shape) if inp.g is not None else None,
+                v(4, torch.float32, inp.beta.shape) if inp.beta is not None else None,
                 v(5, torch.int32, (run.B,)) if inp.read_slot is not None else None,
                 v(6, torch.int32, (run.B,)) if inp.read_slot is not None else None)
     vs = [views(d) for d in devs]
