@@ -321,17 +321,20 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
           umma::mma(tmem + kColP, umma::sdesc_add(dQK, ko), umma::sdesc_add(dQK, 8192 + ko), kIdKK64, kk);
         }
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // K = tokens
+        for (int kk = 0; kk < 4; ++kk)  // K = tokens
           umma::mma(tmem + kColW, umma::sdesc_add(dKm, kk * 2048), umma::sdesc_add(dTw, kk * 32), kIdMK64, kk);
+        // P and W^T are all the first epilogue needs: it starts while U~ and O1 still run
+        // (group 2's commit covers those, the tensor core keeps issue order)
+        umma::commit(&bars[0]);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // K = tokens
           umma::mma(tmem + kColU, umma::sdesc_add(dVm, kk * 2048), umma::sdesc_add(dTw, 8192 + kk * 32), kIdMK64,
                     kk);
-        }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // K = d_k
           const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
           umma::mma(tmem + kColO1 + 64 * (ci & 1), umma::sdesc_add(dS, ko), umma::sdesc_add(dQK, ko), kIdKK64, kk);
         }
-        umma::commit(&bars[0]);
       }
       if (ci > 0) o_tile(ci - 1);  // beside group 1
       bool ok = mbar_wait(&bars[0], phase & 1u);
