@@ -51,8 +51,8 @@ constexpr int kOffP = kOffW + 16384;         // P     [64][64]
 constexpr int kOffU = kOffP + 8192;          // U^T   [128 d_v][64]; O [64][128] row-major at the end
 constexpr int kOffUs = kOffU + 16384;        // Us^T  [128 d_v][64]
 constexpr int kOffGo = kOffUs + 16384;       // gamma_t of the last two chunks [2][64] fp32 (outputs)
-constexpr int kOffBar = kOffGo + 2 * kC * 4; // MMA groups 1-3, then the two staging buffers
-constexpr int kOffMisc = kOffBar + 5 * 8;    // [0] tensor-memory base
+constexpr int kOffBar = kOffGo + 2 * kC * 4; // MMA groups 1-3, the two staging buffers, O2
+constexpr int kOffMisc = kOffBar + 6 * 8;    // [0] tensor-memory base
 constexpr int kSmem = kOffMisc + 16 + 1024;  // + slack for the 1024-byte alignment
 static_assert(kSmem <= 227 * 1024, "shared memory");
 static_assert(chunk::kPrepTileBytes == 16384 + chunk::kGateBlockBytes && kOffTu == kOffTw + 8192 &&
@@ -120,6 +120,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
     mbar_init(&bars[2], 1);
     mbar_init(&bars[3], 1);
     mbar_init(&bars[4], 1);
+    mbar_init(&bars[5], 1);
     mbar_init_fence();
   }
   umma::fence_before();
@@ -217,8 +218,11 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
     // 256 contiguous bytes per token (o_rows).  Both run one chunk late, beside the next
     // chunk's first two MMA groups on the tensor cores.
     __nv_bfloat16* sO = reinterpret_cast<__nv_bfloat16*>(smem + kOffU);
-    auto o_tile = [&](int cj) {
-      if (!worker) return;
+    auto o_tile = [&](int cj) -> bool {
+      if (!worker) return true;
+      // O2 of chunk cj (committed at the end of chunk cj, the CTA's chunk number phase - 1)
+      const bool okw = mbar_wait(&bars[5], (phase - 1u) & 1u);
+      umma::fence_after();
       const float* gm = reinterpret_cast<const float*>(smem + kOffGo) + (cj & 1) * kC;
 #pragma unroll
       for (int c16 = 0; c16 < 2; ++c16) {
@@ -233,6 +237,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
               __float2bfloat16_rn(p.scale * (gm[t] * __uint_as_float(r1[x]) + __uint_as_float(r2[x])));
         }
       }
+      return okw;
     };
     auto o_rows = [&](int cj) {
       const int cc0 = cj * kC;
@@ -285,6 +290,33 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       const bool fact = gbk[6 * kC] != 0.0f;
       const float gC = gbk[kC - 1];  // gamma_C (padded tokens have gate 1: the last real token's)
 
+      // ---- MMAs, group 1 (descriptors: one per operand matrix, stepped by constant byte
+      //      offsets).  P = [Q; K] K^T, W^T = K^T Tw^T and U^T = V^T Tu^T need no state:
+      //      they go first and run beside the S pass; P and W^T are all the first epilogue
+      //      needs, so their commit comes before U~ (group 2's commit covers the rest: the
+      //      tensor core keeps issue order).  O1^T = S0^T Q^T follows the S pass.
+      const uint64_t dQK = umma::sdesc(bq, 16, 1024);     // [Q; K] rows, K-major
+      const uint64_t dKm = umma::sdesc(bk, 16384, 1024);  // K as an MN-major operand
+      const uint64_t dS = umma::sdesc(sb + kOffS, 16, 1024);
+      if (tid == kWorkers) {
+        umma::fence_after();
+        const uint64_t dVm = umma::sdesc(bv, 8192, 1024);
+        const uint64_t dTw = umma::sdesc(btw, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // K = d_k
+          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma::mma(tmem + kColP, umma::sdesc_add(dQK, ko), umma::sdesc_add(dQK, 8192 + ko), kIdKK64, kk);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // K = tokens
+          umma::mma(tmem + kColW, umma::sdesc_add(dKm, kk * 2048), umma::sdesc_add(dTw, kk * 32), kIdMK64, kk);
+        umma::commit(&bars[0]);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // K = tokens
+          umma::mma(tmem + kColU, umma::sdesc_add(dVm, kk * 2048), umma::sdesc_add(dTw, 8192 + kk * 32), kIdMK64,
+                    kk);
+      }
+
       // ---- S pass: BF16 copy of S0^T for this chunk's products, then S^T *= gamma_C
 #pragma unroll 1
       for (int c16 = 0; c16 < (worker ? 4 : 0); ++c16) {
@@ -302,41 +334,21 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
         }
       }
       if (kGate && worker) umma::wait_st();
+      const bool okt = ci > 0 ? o_tile(ci - 1) : true;  // beside group 1
       umma::fence_smem();
       umma::fence_before();
-      __syncthreads();
-
-      // ---- MMAs, group 1: P = [Q; K] K^T, W^T = K^T Tw^T, U^T = V^T Tu^T, O1^T = S0^T Q^T
-      //      (descriptors: one per operand matrix, stepped by constant byte offsets)
-      const uint64_t dQK = umma::sdesc(bq, 16, 1024);     // [Q; K] rows, K-major
-      const uint64_t dKm = umma::sdesc(bk, 16384, 1024);  // K as an MN-major operand
-      const uint64_t dS = umma::sdesc(sb + kOffS, 16, 1024);
+      if (__syncthreads_or(!okt)) {
+        abort = true;
+        break;
+      }
       if (tid == kWorkers) {
         umma::fence_after();
-        const uint64_t dVm = umma::sdesc(bv, 8192, 1024);
-        const uint64_t dTw = umma::sdesc(btw, 16, 1024);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // K = d_k
-          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma::mma(tmem + kColP, umma::sdesc_add(dQK, ko), umma::sdesc_add(dQK, 8192 + ko), kIdKK64, kk);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // K = tokens
-          umma::mma(tmem + kColW, umma::sdesc_add(dKm, kk * 2048), umma::sdesc_add(dTw, kk * 32), kIdMK64, kk);
-        // P and W^T are all the first epilogue needs: it starts while U~ and O1 still run
-        // (group 2's commit covers those, the tensor core keeps issue order)
-        umma::commit(&bars[0]);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // K = tokens
-          umma::mma(tmem + kColU, umma::sdesc_add(dVm, kk * 2048), umma::sdesc_add(dTw, 8192 + kk * 32), kIdMK64,
-                    kk);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // K = d_k
           const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
           umma::mma(tmem + kColO1 + 64 * (ci & 1), umma::sdesc_add(dS, ko), umma::sdesc_add(dQK, ko), kIdKK64, kk);
         }
       }
-      if (ci > 0) o_tile(ci - 1);  // beside group 1
       bool ok = mbar_wait(&bars[0], phase & 1u);
       umma::fence_after();
       // W^T rows (lane = d_k index) -> shared memory, the B operand of the U update
@@ -425,11 +437,13 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
         const uint64_t dU = umma::sdesc(sb + kOffU, 16, 1024);
         const uint64_t dUs = umma::sdesc(sb + kOffUs, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // K = tokens
-          umma::mma(tmem + kColO2, umma::sdesc_add(dU, kk * 32), umma::sdesc_add(dP, kk * 32), kIdKK64, kk);
+        for (int kk = 0; kk < 4; ++kk)  // K = tokens
           umma::mma(tmem + kColS, umma::sdesc_add(dUs, kk * 32), umma::sdesc_add(dKm, kk * 2048), kIdKM128, 1);
-        }
-        umma::commit(&bars[2]);
+        umma::commit(&bars[2]);  // the state: the next chunk's S pass waits for this
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // K = tokens
+          umma::mma(tmem + kColO2, umma::sdesc_add(dU, kk * 32), umma::sdesc_add(dP, kk * 32), kIdKK64, kk);
+        umma::commit(&bars[5]);  // O2: the output epilogue, one chunk later, waits for this
       }
       ok = mbar_wait(&bars[2], phase & 1u);
       umma::fence_after();
@@ -443,8 +457,11 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
     }
     if (abort) break;
     if (n_chunks > 0) {
-      o_tile(n_chunks - 1);
-      __syncthreads();
+      const bool okt = o_tile(n_chunks - 1);
+      if (__syncthreads_or(!okt)) {
+        abort = true;
+        break;
+      }
       o_rows(n_chunks - 1);
     }
 
