@@ -15,7 +15,7 @@ ScanLaunchFn find_chunk_scan(int rule) {
 size_t chunk_workspace_bytes(int64_t total_tokens, int64_t n_seqs, int64_t n_v_heads) {
   if (total_tokens < 0 || n_seqs < 0 || n_v_heads <= 0) return 0;
   const int64_t tiles = (total_tokens + chunk::kC - 1) / chunk::kC + n_seqs + 1;
-  return (size_t)(tiles * n_v_heads * chunk::kPrepTileBytes);
+  return (size_t)(chunk::kWsHeadBytes + tiles * n_v_heads * chunk::kPrepTileBytes);
 }
 
 // The delta rules: the intra-chunk inverses of every chunk (parallel launch), then the

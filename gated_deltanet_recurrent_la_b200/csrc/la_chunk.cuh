@@ -66,6 +66,9 @@ static_assert(kOffW + kC * kRow128 <= kOffT + kC * kTs * 4, "W reuses the L / T 
 // may be used (the chunk's gates are at most 1 in magnitude and span at most e^80)
 constexpr int kGateBlockBytes = (6 * kC + 4) * 4;
 constexpr int kPrepTileBytes = 2 * kC * kRow64 + kGateBlockBytes;
+// the workspace starts with a 256-byte header: word 0 counts the (sequence, head) units the
+// recurrence launch has handed out (the prep launch zeroes it); the tiles follow
+constexpr int kWsHeadBytes = 256;
 
 // byte offset of the 16-byte chunk `ch` of row `r` in a swizzled matrix with rows of `rowb` bytes
 __device__ __forceinline__ uint32_t swz(uint32_t base, int r, int ch, int rowb) {
@@ -657,6 +660,7 @@ __global__ void __launch_bounds__(chunk::kPThreads) chunk_prep_kernel(const Scan
   const int g8 = lane >> 2, t4 = lane & 3;
   const int H = p.n_v_heads;
   const int ratio_h = H / p.n_qk_heads;
+  if (blockIdx.x == 0 && tid == 0) *static_cast<unsigned int*>(const_cast<void*>(p.workspace)) = 0u;
   if (p.n_seqs <= 0) return;
   const int64_t n_tiles = (int64_t)(p.total_tokens + kC - 1) / kC + p.n_seqs + 1;
   const int64_t items = n_tiles * H;
@@ -861,7 +865,7 @@ __global__ void __launch_bounds__(chunk::kPThreads) chunk_prep_kernel(const Scan
     }
     __syncthreads();
     // Tw, Tu and the gate block to the workspace (contiguous in shared memory as in the tile)
-    uint4* dstw = reinterpret_cast<uint4*>(static_cast<unsigned char*>(const_cast<void*>(p.workspace)) +
+    uint4* dstw = reinterpret_cast<uint4*>(static_cast<unsigned char*>(const_cast<void*>(p.workspace)) + kWsHeadBytes +
                                            ((int64_t)gc * H + h) * kPrepTileBytes);
     const uint4* srcw = reinterpret_cast<const uint4*>(smem + kPOffK);
     for (int idx = tid; idx < kPrepTileBytes / 16; idx += kPThreads) dstw[idx] = srcw[idx];

@@ -52,7 +52,7 @@ constexpr int kOffU = kOffP + 8192;          // U^T   [128 d_v][64]; O [64][128]
 constexpr int kOffUs = kOffU + 16384;        // Us^T  [128 d_v][64]
 constexpr int kOffGo = kOffUs + 16384;       // gamma_t of the last two chunks [2][64] fp32 (outputs)
 constexpr int kOffBar = kOffGo + 2 * kC * 4; // MMA groups 1-3, the two staging buffers, O2
-constexpr int kOffMisc = kOffBar + 6 * 8;    // [0] tensor-memory base
+constexpr int kOffMisc = kOffBar + 6 * 8;    // [0] tensor-memory base, [3] the next unit
 constexpr int kSmem = kOffMisc + 16 + 1024;  // + slack for the 1024-byte alignment
 static_assert(kSmem <= 227 * 1024, "shared memory");
 static_assert(chunk::kPrepTileBytes == 16384 + chunk::kGateBlockBytes && kOffTu == kOffTw + 8192 &&
@@ -110,7 +110,6 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
   const int H = p.n_v_heads;
   const int ratio_h = H / p.n_qk_heads;
   const int64_t units = (int64_t)p.n_seqs * H;
-  const int64_t G = gridDim.x;
   __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.o);
 
   if (warp == 0) umma::alloc(const_cast<uint32_t*>(misc), kTmemCols);
@@ -139,10 +138,17 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
   constexpr uint32_t kIdKM64n = umma::idesc_bf16(128, 64, false, true, true);
   constexpr uint32_t kIdKM128 = umma::idesc_bf16(128, 128, false, true);
 
+  // units are handed out one at a time from the workspace's counter (zeroed by the prep
+  // launch), in seq_order order: longest sequences first, each CTA taking the next unit
+  // when it finishes one
+  unsigned int* next_unit = static_cast<unsigned int*>(const_cast<void*>(p.workspace));
 #pragma unroll 1
-  for (int64_t round = 0; round * G < units; ++round) {
-    const int64_t u = round * G + ((round & 1) ? (G - 1 - blockIdx.x) : blockIdx.x);
-    if (u >= units) continue;
+  for (;;) {
+    if (tid == 0) misc[3] = atomicAdd(next_unit, 1u);
+    __syncthreads();
+    const int64_t u = misc[3];
+    __syncthreads();  // (misc[3] is rewritten at the next unit)
+    if (u >= units) break;
     const int64_t si = u / H;
     const int h = (int)(u % H);
     const int hq = h / ratio_h;
@@ -208,7 +214,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
       }
       bulk_g2s(buf + kOffTw,
                static_cast<const unsigned char*>(p.workspace) +
-                   (((int64_t)(tok0 / kC + seq)) * H + h) * chunk::kPrepTileBytes,
+                   chunk::kWsHeadBytes + (((int64_t)(tok0 / kC + seq)) * H + h) * chunk::kPrepTileBytes,
                chunk::kPrepTileBytes, full);
       pending |= 1u << b;
     };

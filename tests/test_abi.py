@@ -173,6 +173,20 @@ def test_chunked_scan_supported_set(lib):
     assert call(io=0) == L.LA_ERR_UNSUPPORTED
 
 
+def test_chunked_workspace_size(lib):
+    """The two-launch prefill's workspace: a fixed header plus one tile per (chunk, head),
+    chunks counted per sequence (a ragged tail is a whole tile); every tile starts on a
+    16-byte boundary, as the bulk copies that read it require."""
+    b = L.la_scan_chunked_workspace_bytes
+    head = b(0, 1, 1) - (b(0, 1, 2) - b(0, 1, 1))  # size = head + tiles * H * tile
+    tile = (b(0, 1, 2) - b(0, 1, 1)) // 2               # (0 tokens, 1 sequence: 2 tiles per head)
+    assert head >= 16 and head % 16 == 0 and tile % 16 == 0 and tile > 2 * 64 * 64 * 2
+    for T, n, H in [(1, 1, 1), (64, 1, 32), (65, 2, 4), (172058, 32, 32), (1 << 20, 1, 32)]:
+        tiles = (T + 63) // 64 + n + 1
+        assert b(T, n, H) == head + tiles * H * tile
+    assert b(10, 0, 4) == head + 2 * 4 * tile and b(-1, 1, 1) == 0
+
+
 def test_checkpointed_scan_host_errors(lib):
     dst = pool()
     P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
