@@ -111,10 +111,16 @@ def fp32_alu_peak_tflops(sm_count, mhz):
 
 
 def kernel_source_hash(files):
+    """Hash of the kernel's source code with comments and blank lines dropped, so that a
+    recorded capture stays attached to the code it measured and not to its comments."""
+    import re
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "gated_deltanet_recurrent_la_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "gated_deltanet_recurrent_la_b200", "csrc", f), "r", encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update("\n".join(l.rstrip() for l in text.splitlines() if l.strip()).encode())
     return h.hexdigest()[:16]
 
 

@@ -20,9 +20,13 @@
 // S^T (d_v lanes x d_k columns, FP32) stays in tensor memory for the whole sequence.
 //
 // One CTA of 9 warps per SM: worker warp w < 8 reads tensor-memory lanes 32 (w % 4) .. + 31
-// and the column half w / 4 of each accumulator; lane 0 of warp 8 only issues the MMAs, so
-// issuing never holds up an epilogue.  Three mbarriers signal the completion of each MMA
-// group, and every wait gives up after a time limit (LA_DEVERR_TIMEOUT).
+// and the column half w / 4 of each accumulator; lane 0 of warp 8 only issues the MMAs and
+// the TMA copies, so issuing never holds up an epilogue.  Per chunk the state-free
+// products (P, W^T, U~) are issued as soon as the chunk has landed and run beside the S
+// pass; O1 follows it; the U update, then the state update and O2.  Four mbarriers signal
+// MMA completion (P and W^T; U; the state; O2) and two the staged chunks; every wait gives
+// up after a time limit (LA_DEVERR_TIMEOUT).  A chunk's outputs are assembled during the
+// next chunk.  (Sequence, head) units come from a counter in the workspace header.
 #pragma once
 
 #include <cstdint>
