@@ -41,6 +41,18 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(la_[a-z_]+)\s*\(", text)))
 
 
+def test_header_is_plain_c():
+    """The boundary header compiles as C99 and as C++11 on its own (no torch or CUDA types)."""
+    import shutil
+    hdr = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "la_state.h")
+    for cc, std, lang in (("gcc", "-std=c99", "c"), ("g++", "-std=c++11", "c++")):
+        if shutil.which(cc) is None:
+            pytest.skip(f"{cc} not installed")
+        r = subprocess.run([cc, std, "-fsyntax-only", "-Wall", "-Werror", "-x", lang, hdr], capture_output=True,
+                           text=True)
+        assert r.returncode == 0, r.stderr
+
+
 def test_header_declares_the_binding_exports():
     assert declared_functions() == sorted(L.EXPORTS)
 
