@@ -30,6 +30,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cstring>
 
 #include "la_chunk.cuh"
 #include "la_umma.cuh"
@@ -544,9 +545,11 @@ cudaError_t launch_chunk_tc(const ScanParams& p, cudaStream_t stream) {
   // one CTA per SM: the kernel holds all of the SM's tensor memory
   if (per_sm != 1) return cudaErrorInvalidConfiguration;
   TcMaps maps;
-  if (!encode_rows_map(&maps.q, p.q, p.n_qk_heads, p.total_tokens) ||
-      !encode_rows_map(&maps.k, p.k, p.n_qk_heads, p.total_tokens) ||
-      !encode_rows_map(&maps.v, p.v, p.n_v_heads, p.total_tokens))
+  memset(&maps, 0, sizeof(maps));  // no tokens: nothing is staged, the maps are never read
+  if (p.total_tokens > 0 &&
+      (!encode_rows_map(&maps.q, p.q, p.n_qk_heads, p.total_tokens) ||
+       !encode_rows_map(&maps.k, p.k, p.n_qk_heads, p.total_tokens) ||
+       !encode_rows_map(&maps.v, p.v, p.n_v_heads, p.total_tokens)))
     return cudaErrorInvalidValue;
   const int64_t units = (int64_t)p.n_seqs * p.n_v_heads;
   const int64_t cap = device_sm_count();

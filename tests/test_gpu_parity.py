@@ -531,6 +531,17 @@ def test_chunked_two_launches_special_ranges(rule):
     assert_close(np64(o), o_ref, 2e-2, f"{rule}: readout of the unchanged state")
 
 
+@pytest.mark.parametrize("rule", ["delta", "gated_delta"])
+def test_chunked_two_launches_all_sequences_empty(rule):
+    """No tokens at all: every sequence stores its initial state (the tensor maps of the
+    empty q / k / v are never used)."""
+    inp = W.scan_inputs(lengths=[0, 0, 0], n_qk_heads=1, n_v_heads=2, d_k=128, d_v=128, rule=rule,
+                        io_dtype=BF16, seed=46, init="slots", init_dtype=F32)
+    S, o, err = _gpu_scan_chunked_ws(inp, F32)
+    assert err == 0 and o.numel() == 0
+    assert torch.equal(S, inp.pool[inp.read_slot.long()].float())
+
+
 def test_chunked_two_launches_prefill32_sampled():
     """The full prefill workload through the two-launch path, as the benchmark runs it:
     the shortest and the longest sequence checked against the oracle on one head each."""
