@@ -542,6 +542,33 @@ def test_chunked_two_launches_all_sequences_empty(rule):
     assert torch.equal(S, inp.pool[inp.read_slot.long()].float())
 
 
+def test_chunked_two_launches_pool_slots_and_order():
+    """Write slots into a larger pool (other slots untouched), a seq_order that reverses the
+    sequences, BF16 final states: the pool semantics of the two-launch path."""
+    inp = W.scan_inputs(lengths=[90, 200, 3, 64], n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128, io_dtype=BF16,
+                        seed=47, init="slots", init_dtype=F32)
+    n_seqs = 4
+    dst_t = torch.full((9, 4, 128, 128), 3.0, dtype=BF16, device="cuda")
+    write = torch.tensor([7, 2, 5, 0], dtype=torch.int32)
+    o = torch.full((inp.q.shape[0], 4, 128), 5.0, dtype=BF16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(L.la_scan_chunked_workspace_bytes(inp.q.shape[0], n_seqs, 4), dtype=torch.uint8, device="cuda")
+    st = L.la_state_scan_chunked_ws(inp.rule, L.Pool(dev(inp.pool), 2), dev(inp.read_slot), L.Pool(dst_t, 2),
+                                    dev(write), dev(inp.cu_seqlens), dev(inp.q), dev(inp.k), dev(inp.v),
+                                    dev(inp.g), dev(inp.beta), inp.scale, o, ws, err,
+                                    seq_order=torch.tensor([3, 2, 1, 0], dtype=torch.int32, device="cuda"))
+    L.check(st)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    S_ref, o_ref, _ = oracle_scan(inp, dst_dtype=BF16)
+    got = dst_t.cpu()
+    for s in range(n_seqs):
+        assert_close(np64(got[int(write[s])]), S_ref[s], 2e-2, f"sequence {s} state in slot {int(write[s])}")
+    untouched = [i for i in range(9) if i not in write.tolist()]
+    assert torch.all(got[untouched] == 3.0)
+    assert_close(np64(o.cpu()), o_ref, 2e-2, "outputs")
+
+
 def test_chunked_two_launches_prefill32_sampled():
     """The full prefill workload through the two-launch path, as the benchmark runs it:
     the shortest and the longest sequence checked against the oracle on one head each."""
