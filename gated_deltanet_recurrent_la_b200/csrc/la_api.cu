@@ -83,6 +83,8 @@ la_status cuda_status(cudaError_t e) {
 
 bool uses_gate(la_rule r) { return r == LA_RULE_GATED || r == LA_RULE_GATED_DELTA || r == LA_RULE_KDA; }
 bool uses_beta(la_rule r) { return r == LA_RULE_DELTA || r == LA_RULE_GATED_DELTA || r == LA_RULE_KDA; }
+// the rules whose chunked prefill solves intra-chunk corrections (the two-launch form's workspace)
+bool chunk_inverse(la_rule r) { return r == LA_RULE_DELTA || r == LA_RULE_GATED_DELTA; }
 // the gate array's alignment: kda's per-channel decays are moved in 16-byte pieces
 size_t gate_align(la_rule r) { return r == LA_RULE_KDA ? 16 : 4; }
 
@@ -297,7 +299,7 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
     fn = (io == LA_F32) ? la::find_scan_conv_f32io(rule, s.d_k, s.d_v) : la::find_scan_conv_bf16io(rule, s.d_k, s.d_v);
   } else if (chunked) {
     if (s.d_k != 128 || s.d_v != 128 || io != LA_BF16) return LA_ERR_UNSUPPORTED;
-    if (workspace) {
+    if (workspace && chunk_inverse(rule)) {
       if (!aligned(workspace, 16)) return LA_ERR_ALIGN;
       if (workspace_bytes < la::chunk_workspace_bytes(total_tokens, n_seqs, s.n_v_heads)) return LA_ERR_SHAPE;
       fn = la::find_chunk_scan_ws(rule);
@@ -383,7 +385,7 @@ la_status la_state_scan_chunked_ws(la_rule rule, const la_pool* src, const int32
                                    const void* v, la_dtype io, const float* g, const float* beta, float scale,
                                    void* o, void* workspace, size_t workspace_bytes, int32_t* err_word,
                                    void* stream) {
-  if (!workspace && n_seqs > 0) return LA_ERR_NULL;
+  if (!workspace && n_seqs > 0 && chunk_inverse(rule)) return LA_ERR_NULL;
   return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, q, k, v, io,
                    g, beta, scale, o, 0, nullptr, nullptr, err_word, stream, true, 0, nullptr, workspace,
                    workspace_bytes);
@@ -395,8 +397,9 @@ la_status la_state_scan_chunked_noalloc(la_rule rule, const la_pool* src, const 
                                         const void* q, const void* k, const void* v, la_dtype io, const float* g,
                                         const float* beta, float scale, void* o, int32_t* err_word, void* stream) {
   size_t bytes = 0;
-  void* ws = la::chunk_noalloc_workspace(&bytes);
-  if (!ws) return cuda_status(cudaGetLastError() != cudaSuccess ? cudaGetLastError() : cudaErrorUnknown);
+  void* ws = nullptr;
+  const cudaError_t e = la::chunk_noalloc_workspace(&ws, &bytes);
+  if (e != cudaSuccess) return cuda_status(e);
   return la_state_scan_chunked_ws(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order,
                                   q, k, v, io, g, beta, scale, o, ws, bytes, err_word, stream);
 }

@@ -137,8 +137,9 @@ ScanLaunchFn find_chunk_scan(int rule);
 ScanLaunchFn find_chunk_scan_ws(int rule);
 // workspace of the _ws form: one 16 KiB tile per (chunk slot, head)
 size_t chunk_workspace_bytes(int64_t total_tokens, int64_t n_seqs, int64_t n_v_heads);
-// the library's own fixed workspace on the current device (nullptr on failure); *bytes = its size
-void* chunk_noalloc_workspace(size_t* bytes);
+// the library's own fixed workspace on the current device: *addr = its device address,
+// *bytes = its size; the error of the device query or the symbol lookup otherwise
+cudaError_t chunk_noalloc_workspace(void** addr, size_t* bytes);
 
 cudaError_t launch_pool_copy(const PoolCopyParams& p, cudaStream_t stream);
 

@@ -225,9 +225,10 @@ la_status la_state_scan_chunked(la_rule rule, const la_pool *src, const int32_t 
  *   workspace        device, 16-byte aligned, at least
  *                    la_scan_chunked_workspace_bytes(total_tokens, n_seqs, H_v) bytes;
  *                    contents are scratch (overwritten, not read back by the caller)
- * Other arguments, supported set and errors as la_state_scan_chunked; LA_ERR_SHAPE when
- * workspace_bytes is too small, LA_ERR_NULL for a NULL workspace.  The linear and gated
- * rules have no inverse and run the one-launch form (the workspace is not touched). */
+ * Other arguments, supported set and errors as la_state_scan_chunked; for the delta rules
+ * LA_ERR_SHAPE when workspace_bytes is too small and LA_ERR_NULL for a NULL workspace.  The
+ * linear and gated rules have no inverse and run the one-launch form: the workspace and
+ * its size are ignored (NULL allowed, never touched). */
 size_t la_scan_chunked_workspace_bytes(int32_t total_tokens, int32_t n_seqs, int32_t n_v_heads);
 la_status la_state_scan_chunked_ws(la_rule rule, const la_pool *src, const int32_t *read_slot,
                                    const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
@@ -239,11 +240,18 @@ la_status la_state_scan_chunked_ws(la_rule rule, const la_pool *src, const int32
 
 /* la_state_scan_chunked_ws with the library's own workspace: a fixed 256 MiB device array
  * of this library (one per device), so the caller passes no scratch buffer.  The array is
+ * a file-scope __device__ variable of the library's device code: it is reserved on a
+ * device when the module holding it is loaded there, which under the CUDA runtime's lazy
+ * module loading (the default) is this entry point's first call on that device, and under
+ * CUDA_MODULE_LOADING=EAGER is context creation -- then every process that loads the
+ * library pays the 256 MiB per device, callers of the other entry points included.  It
+ * stays reserved until the process exits (or the device is reset).  The array is
  * shared by every call on a device: calls must not run concurrently on one device (the
- * caller orders them, for example on one stream).  A call whose workspace would exceed
- * the array (la_scan_chunked_workspace_bytes(total_tokens, n_seqs, H_v) > 256 MiB) returns
- * LA_ERR_SHAPE before launching anything.  Other arguments and errors as
- * la_state_scan_chunked. */
+ * caller orders them, for example on one stream).  A call of a delta rule whose workspace
+ * would exceed the array (la_scan_chunked_workspace_bytes(total_tokens, n_seqs, H_v) >
+ * 256 MiB) returns LA_ERR_SHAPE before launching anything; the linear and gated rules do
+ * not use the array and have no such limit.  A failed device query or symbol lookup
+ * returns LA_ERR_CUDA.  Other arguments and errors as la_state_scan_chunked. */
 la_status la_state_scan_chunked_noalloc(la_rule rule, const la_pool *src, const int32_t *read_slot,
                                         const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
                                         const int32_t *cu_seqlens, int32_t total_tokens,

@@ -199,6 +199,40 @@ def test_chunked_workspace_size(lib):
     assert b(10, 0, 4) == head + 2 * 4 * tile and b(-1, 1, 1) == 0
 
 
+def test_noalloc_lookup_failure_is_an_error(lib):
+    """The no-alloc prefill looks up the address of the library's own workspace before
+    anything else; where that lookup fails (here: no CUDA device at all), the call reports
+    LA_ERR_CUDA with the runtime's error code -- never LA_OK with nothing launched."""
+    if torch.cuda.is_available():
+        pytest.skip("the lookup succeeds on a GPU host")
+    dst = pool()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    st = lib.la_state_scan_chunked_noalloc(3, None, None, ctypes.byref(dst), None, 2, P(A), 10, None, P(A), P(A),
+                                           P(A), 1, P(A), P(A), 1.0, P(A), P(A), None)
+    assert st == L.LA_ERR_CUDA
+    assert lib.la_last_cuda_error() != 0
+    # a second call fails the same way (nothing half-initialised is cached)
+    assert lib.la_state_scan_chunked_noalloc(3, None, None, ctypes.byref(dst), None, 2, P(A), 10, None, P(A), P(A),
+                                             P(A), 1, P(A), P(A), 1.0, P(A), P(A), None) == L.LA_ERR_CUDA
+
+
+def test_chunked_ws_linear_and_gated_ignore_the_workspace(lib):
+    """The linear and gated rules have no intra-chunk inverse: the two-launch entry point
+    neither needs nor checks a workspace for them (a NULL workspace of size 0 passes the
+    host checks, which end here at an unsupported io type before any launch), while the
+    delta rules still require one."""
+    dst = pool()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+
+    def call(rule, ws, nbytes, io=0):
+        return lib.la_state_scan_chunked_ws(rule, None, None, ctypes.byref(dst), None, 2, P(A), 10, None, P(A),
+                                            P(A), P(A), io, P(A), P(A), 1.0, P(A), P(ws), nbytes, P(A), None)
+    assert call(0, None, 0) == L.LA_ERR_UNSUPPORTED       # linear: no workspace needed
+    assert call(1, None, 0) == L.LA_ERR_UNSUPPORTED       # gated
+    assert call(3, None, 0) == L.LA_ERR_NULL              # gated_delta: required
+    assert call(3, A, 16, io=1) == L.LA_ERR_SHAPE         # and sized
+
+
 def test_checkpointed_scan_host_errors(lib):
     dst = pool()
     P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
