@@ -1,14 +1,17 @@
-// la_chunk.cu -- chunked tensor-core prefill kernels (all four rules); see la_chunk.cuh.
+// la_chunk.cu -- chunked tensor-core prefill kernels: the fused one-launch form (all four
+// rules, la_chunk_fused.cuh) and the two-launch form of the delta rules (la_chunk.cuh prep +
+// la_chunk_tc.cuh recurrence).
 #include "la_chunk.cuh"
+#include "la_chunk_fused.cuh"
 #include "la_chunk_tc.cuh"
 
 namespace la {
 ScanLaunchFn find_chunk_scan(int rule) {
   switch (rule) {
-    case LA_RULE_LINEAR: return &launch_chunk_scan<LA_RULE_LINEAR>;
-    case LA_RULE_GATED: return &launch_chunk_scan<LA_RULE_GATED>;
-    case LA_RULE_DELTA: return &launch_chunk_scan<LA_RULE_DELTA>;
-    case LA_RULE_GATED_DELTA: return &launch_chunk_scan<LA_RULE_GATED_DELTA>;
+    case LA_RULE_LINEAR: return &launch_chunk_fused<LA_RULE_LINEAR>;
+    case LA_RULE_GATED: return &launch_chunk_fused<LA_RULE_GATED>;
+    case LA_RULE_DELTA: return &launch_chunk_fused<LA_RULE_DELTA>;
+    case LA_RULE_GATED_DELTA: return &launch_chunk_fused<LA_RULE_GATED_DELTA>;
   }
   return nullptr;
 }
@@ -29,8 +32,8 @@ cudaError_t launch_chunk_scan_ws_tc(const ScanParams& p, cudaStream_t stream) {
 
 ScanLaunchFn find_chunk_scan_ws(int rule) {
   switch (rule) {
-    case LA_RULE_LINEAR: return &launch_chunk_scan_ws<LA_RULE_LINEAR>;
-    case LA_RULE_GATED: return &launch_chunk_scan_ws<LA_RULE_GATED>;
+    case LA_RULE_LINEAR: return &launch_chunk_fused<LA_RULE_LINEAR>;  // no inverse, no workspace
+    case LA_RULE_GATED: return &launch_chunk_fused<LA_RULE_GATED>;
     case LA_RULE_DELTA: return &launch_chunk_scan_ws_tc<LA_RULE_DELTA>;
     case LA_RULE_GATED_DELTA: return &launch_chunk_scan_ws_tc<LA_RULE_GATED_DELTA>;
   }

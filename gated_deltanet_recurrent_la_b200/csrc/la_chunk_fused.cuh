@@ -1,0 +1,939 @@
+// la_chunk_fused.cuh -- the chunked (WY / UT) prefill in one launch on the fifth-generation
+// tensor cores, with every intra-chunk quantity kept on chip.
+//
+// Algebra ("Seven Architectures Replacing KV Cache With Bounded Mutable State": the "Kimi
+// Linear" section's chunkwise-parallel kernel, the "Gated DeltaNet-2" section's chunkwise
+// WY algorithm).  Per (sequence, head) and chunk of C = 64 tokens, with S0 the state at the
+// chunk start, gamma_t the product of the chunk's decays up to token t and b_t the write
+// strength of the rule:
+//
+//   L  = strictly-lower( b_t (gamma_t / gamma_s) k_t . k_s ),   T = (I + L)^-1
+//   W  = T diag(b gamma) K,    U~ = T diag(b) V,    U = U~ - W S0      (delta rules; else U = V)
+//   O  = scale ( Q~ S0 + P U ),   Q~ = diag(gamma) Q,   P = (Q K^T) (.) M,  M_ts = gamma_t / gamma_s (s <= t)
+//   S  = gamma_C S0 + K~^T U,     K~ = diag(gamma_C / gamma) K
+//
+// which unrolls the token recurrence u_t = b (v_t - c S_{t-1}^T k_t), S_t = a S_{t-1} + k_t u_t^T
+// exactly.  Every product is an M = 128 tcgen05 MMA with BF16 operands and an FP32
+// accumulator in tensor memory; the transposed forms (U^T, O^T, S^T: one d_v index per
+// tensor-memory lane) let the state, its BF16 copy S0^T and the BF16 copy of U^T feed the
+// next products straight from tensor memory as the A operand.
+//
+// One CTA of 14 warps per SM, each role a pipeline stage joined by mbarriers:
+//   warp 0       loads: Q, K, V of a chunk by TMA tensor maps into one of three stages,
+//                the chunk's gates by its lanes
+//   warp 1       lane 0 issues every MMA (and owns the tensor-memory allocation)
+//   warps 2-5    intra-chunk work, up to two chunks ahead of the state: gate prefixes,
+//                P and L from [Q; K] K^T, Q~ and K~ in place, T = (I + L)^-1 (16 x 16
+//                diagonal blocks by FP32 substitution, off-diagonal blocks by TF32 MMA),
+//                Tw = T diag(b gamma), Tu = T diag(b)
+//   warps 6-9    the state: S0^T -> BF16 copy and S^T *= gamma_C per chunk, U^T -> BF16,
+//                initial and final states
+//   warps 10-13  W^T -> shared memory, outputs to global memory
+// Per chunk j the issuer runs: W_j and U~_j (after the intra-chunk work of chunk j),
+// U_j -= S0^T W^T, O_j = S0^T Q~^T, then S^T += U^T K~ and O_j += U^T P^T, then [Q; K] K^T of
+// chunk j + 2; only the S pass -> U -> U epilogue -> state update chain is serial across
+// chunks.  Every wait has a time limit and a CTA-wide abort flag: a wait that gives up
+// stops every role, the issuer drains its MMAs, the loader its copies, and the kernel
+// reports LA_DEVERR_TIMEOUT.  Units (sequence, head) are dealt to the CTAs in a fixed
+// boustrophedon order over seq_order (longest first balances the load).
+#pragma once
+
+#include <cstdint>
+#include <cstring>
+
+#include "la_chunk.cuh"
+#include "la_chunk_tc.cuh"
+#include "la_umma.cuh"
+
+namespace la {
+namespace fused {
+
+constexpr int kC = 64;   // tokens per chunk
+constexpr int kD = 128;  // d_k = d_v
+constexpr int kStages = 3;
+
+// warp roles
+constexpr int kWarpLoad = 0;
+constexpr int kWarpMma = 1;
+constexpr int kWarpPrep = 2;   // warps 2..5
+constexpr int kWarpState = 6;  // warps 6..9
+constexpr int kWarpOut = 10;   // warps 10..13
+constexpr int kThreads = 14 * 32;
+// named barriers of the warp groups (0 is __syncthreads)
+constexpr uint32_t kNbPrep = 1, kNbState = 2, kNbOut = 3;
+
+// shared memory (bytes from a 1024-byte aligned base); BF16 operands in 64-column panels
+constexpr int kStageBytes = 49152;
+constexpr int kOffQK = 0;      // in a stage: two panels of 128 rows, Q rows 0..63, K rows 64..127
+constexpr int kOffV = 32768;   //             two panels of 64 rows
+constexpr int kOffWt = kStages * kStageBytes;  // W^T [128 d_k][64 t]
+constexpr int kOffP = kOffWt + 16384;          // P [2][64 t][64 s] (chunk parity)
+constexpr int kOffTw = kOffP + 2 * 8192;       // Tw [64 t][64 s]
+constexpr int kOffTu = kOffTw + 8192;          // Tu [64 t][64 s]
+constexpr int kLs = kC + 4;                    // padded row stride of L / T (fp32)
+constexpr int kOffL = kOffTu + 8192;           // L, then T in place [64][68] fp32
+constexpr int kXs = 24;
+constexpr int kOffX = kOffL + kC * kLs * 4;    // [3][16][24] fp32, scratch of the block recursion
+constexpr int kOffGin = kOffX + 3 * 16 * kXs * 4;        // [kStages][2][64] fp32: g, beta as given
+constexpr int kGB = 8 * kC;                              // floats per gate block
+constexpr int kOffGB = kOffGin + kStages * 2 * kC * 4;   // [2][kGB] fp32 (chunk parity)
+// gate block: [0, 64) gamma_t, [64, 128) gamma_C / gamma_t, [128, 192) A_t = gamma_t / e^m,
+// [192, 256) B_t = e^m / gamma_t, [256, 320) log |gamma_t|, [320, 384) sign gamma_t,
+// [384, 448) b_t, [448] 1 when gamma_t / gamma_s = A_t B_s may be used
+constexpr int kOffBar = kOffGB + 2 * kGB * 4;
+enum Bar {
+  kFull = 0,        // [3] stage loaded (TMA bytes + 32 lane arrivals of the gates)
+  kEmpty = 3,       // [3] stage free (MMA commit)
+  kG1Full = 6,      // [Q; K] K^T of a chunk in tensor memory (MMA commit)
+  kG1Free,          // the intra-chunk group has read it
+  kPrepDone,        // Tw, Tu, P, Q~ (and K~ for the rules without inverse) ready
+  kWFull,           // W^T and U~^T in tensor memory (MMA commit)
+  kWFree,           // W^T is in shared memory
+  kSPass,           // S0^T copied to BF16 and S^T scaled by gamma_C
+  kUFull,           // U^T in tensor memory (MMA commit)
+  kUDone,           // U^T copied to BF16
+  kKt,              // K~ ready (delta rules)
+  kSFull,           // state update done (MMA commit)
+  kOFull,           // outputs of a chunk in tensor memory (MMA commit)
+  kOFree,           // outputs read
+  kDrain,           // every MMA issued has completed
+  kNumBars
+};
+constexpr int kOffMisc = kOffBar + kNumBars * 8;  // [0] tensor-memory base, [1] abort, [2] gate blocks done
+constexpr int kSmem = kOffMisc + 16 + 1024;       // + slack for the 1024-byte alignment
+static_assert(kSmem <= 227 * 1024, "shared memory");
+static_assert(kOffWt % 1024 == 0 && kOffP % 1024 == 0 && kOffTw % 1024 == 0 && kOffL % 16 == 0, "alignment");
+
+// bytes the TMA engine writes into a stage per chunk: Q, K, V (two 64 x 64 panels each)
+constexpr uint32_t kTmaBytes = 6 * kC * 128;
+
+// tensor-memory columns (FP32 accumulators unless noted; 128 lanes each)
+constexpr uint32_t kTmemCols = 512;
+constexpr int kColS = 0;     // S^T        [d_v][d_k]     128
+constexpr int kColSb = 128;  // S0^T BF16  [d_v][d_k / 2]  64 (A operand)
+constexpr int kColG1 = 192;  // [Q; K] K^T [128][64]       64
+constexpr int kColW = 256;   // W^T        [d_k][64]       64
+constexpr int kColU = 320;   // U^T        [d_v][64]       64
+constexpr int kColUb = 384;  // U^T BF16   [d_v][32]       32 (A operand)
+constexpr int kColO = 448;   // O^T        [d_v][64]       64
+
+// D (tensor memory) = A (tensor memory, BF16 packed two per column) B (shared memory)
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+// A pipeline wait with a time limit and the CTA's abort flag: false when it gave up (the
+// flag is then set) or another role gave up first.
+__device__ __forceinline__ bool fwait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t polls = 1;; ++polls) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((polls & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (polls >= kWaitMaxPolls || global_timer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1u;
+        return false;
+      }
+    }
+  }
+}
+
+// One (sequence, head) unit: its tokens, slots and whether it can be processed.
+struct Unit {
+  int seq, h, hq, t0, n_tok, rs, ws;
+  uint32_t err;  // bits to report (also for some processed units: cu_seqlens[0] != 0)
+  bool valid;
+};
+
+__device__ __forceinline__ Unit unit_info(const ScanParams& p, int64_t u) {
+  Unit x;
+  const int H = p.n_v_heads;
+  const int64_t si = u / H;
+  x.h = (int)(u % H);
+  x.hq = x.h / (H / p.n_qk_heads);
+  x.seq = p.seq_order ? __ldg(p.seq_order + si) : (int)si;
+  x.err = 0u;
+  x.valid = false;
+  x.t0 = x.n_tok = x.rs = x.ws = 0;
+  if (x.seq < 0 || x.seq >= p.n_seqs) {
+    x.err = LA_DEVERR_CU_SEQLENS;
+    return x;
+  }
+  const int t0 = __ldg(p.cu_seqlens + x.seq), t1 = __ldg(p.cu_seqlens + x.seq + 1);
+  if (x.seq == 0 && x.h == 0 && t0 != 0) x.err |= LA_DEVERR_CU_SEQLENS;
+  if (t0 < 0 || t1 < t0 || t1 > p.total_tokens) {
+    x.err |= LA_DEVERR_CU_SEQLENS;
+    return x;
+  }
+  x.rs = p.read_slot ? __ldg(p.read_slot + x.seq) : 0;
+  x.ws = p.write_slot ? __ldg(p.write_slot + x.seq) : x.seq;
+  const bool rs_ok = !p.read_slot || (x.rs >= 0 && x.rs < p.src_slots);
+  const bool ws_ok = x.ws >= 0 && x.ws < p.dst_slots;
+  if (!rs_ok || !ws_ok) {
+    x.err |= (rs_ok ? 0u : LA_DEVERR_READ_SLOT) | (ws_ok ? 0u : LA_DEVERR_WRITE_SLOT);
+    return x;
+  }
+  x.t0 = t0;
+  x.n_tok = t1 - t0;
+  x.valid = true;
+  return x;
+}
+
+// the unit of round r for CTA b: boustrophedon over the grid
+__device__ __forceinline__ int64_t unit_of(int64_t r, int64_t G, int64_t b) {
+  return r * G + ((r & 1) ? (G - 1 - b) : b);
+}
+
+__device__ __forceinline__ uint32_t pack2(uint32_t lo, uint32_t hi) {
+  return pack_bf16x2(__uint_as_float(lo), __uint_as_float(hi));
+}
+
+}  // namespace fused
+
+template <int RULE>
+__global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const ScanParams p,
+                                                                         const __grid_constant__ TcMaps maps) {
+  using namespace fused;
+  constexpr bool kDelta = Rule<RULE>::kPredicts;
+  constexpr bool kGate = Rule<RULE>::kUsesGate;
+  static_assert(!Rule<RULE>::kChannelGate, "scalar gates only");
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  unsigned char* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t sb = smem_addr(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
+  volatile uint32_t* abort_flag = misc + 1;
+  volatile uint32_t* gates_done = misc + 2;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int H = p.n_v_heads;
+  const int64_t units = (int64_t)p.n_seqs * H;
+  const int64_t G = gridDim.x;
+
+  if (warp == kWarpMma) umma::alloc(const_cast<uint32_t*>(misc), kTmemCols);
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars[kFull + s], 33);
+      mbar_init(&bars[kEmpty + s], 1);
+    }
+    for (int b = kG1Full; b < kNumBars; ++b) mbar_init(&bars[b], 1);
+    misc[1] = 0u;
+    misc[2] = 0u;
+    mbar_init_fence();
+  }
+  // the strictly upper 16 x 16 blocks of Tw and Tu stay zero in every chunk
+  if (kDelta && warp >= kWarpPrep && warp < kWarpState) {
+    for (int idx = tid - kWarpPrep * 32; idx < kC * kC / 2; idx += 128) {
+      const int r = idx >> 5, c = 2 * (idx & 31);
+      if ((c >> 4) > (r >> 4)) {
+        const uint32_t off = umma::panel_off(kC, r, c);
+        *reinterpret_cast<uint32_t*>(smem + kOffTw + off) = 0u;
+        *reinterpret_cast<uint32_t*>(smem + kOffTu + off) = 0u;
+      }
+    }
+  }
+  umma::fence_before();
+  __syncthreads();
+  umma::fence_after();
+  const uint32_t tmem = misc[0];
+
+  // chunks this CTA processes (every role walks the same units in the same order)
+  int64_t n_total = 0;
+  for (int64_t r = 0; r * G < units; ++r) {
+    const int64_t u = unit_of(r, G, blockIdx.x);
+    if (u >= units) continue;
+    const Unit x = unit_info(p, u);
+    if (x.valid) n_total += (x.n_tok + kC - 1) / kC;
+  }
+
+  if (warp == kWarpLoad) {
+    // ------------------------------------------------------------------ loader
+    int64_t j = 0;
+    bool ok = true;
+    for (int64_t r = 0; ok && r * G < units; ++r) {
+      const int64_t u = unit_of(r, G, blockIdx.x);
+      if (u >= units) continue;
+      const Unit x = unit_info(p, u);
+      if (!x.valid) continue;
+      const int nch = (x.n_tok + kC - 1) / kC;
+      for (int c = 0; c < nch; ++c, ++j) {
+        const int s = (int)(j % kStages);
+        const int tok0 = x.t0 + c * kC;
+        const int nv = min(kC, x.n_tok - c * kC);
+        // the chunk's gates (raw g and beta; padded tokens: no decay, no write)
+        float ga = 1.0f, gb = 1.0f, ba = 0.0f, bb = 0.0f;
+        if (lane < nv) {
+          const int64_t gi = (int64_t)(tok0 + lane) * H + x.h;
+          ga = kGate ? __ldg(p.g + gi) : 1.0f;
+          ba = Rule<RULE>::kUsesBeta ? __ldg(p.beta + gi) : 1.0f;
+        }
+        if (lane + 32 < nv) {
+          const int64_t gi = (int64_t)(tok0 + lane + 32) * H + x.h;
+          gb = kGate ? __ldg(p.g + gi) : 1.0f;
+          bb = Rule<RULE>::kUsesBeta ? __ldg(p.beta + gi) : 1.0f;
+        }
+        if (j >= kStages && lane == 0) ok = fwait(&bars[kEmpty + s], (uint32_t)((j / kStages) + 1) & 1u, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        unsigned char* st = smem + s * kStageBytes;
+        if (lane == 0) {
+          uint64_t* full = &bars[kFull + s];
+          mbar_arrive_expect_tx(full, kTmaBytes);
+#pragma unroll
+          for (int pnl = 0; pnl < 2; ++pnl) {
+            umma::tma_load_3d(st + kOffQK + pnl * 16384, &maps.q, 64 * pnl, x.hq, tok0, full);
+            umma::tma_load_3d(st + kOffQK + pnl * 16384 + kC * 128, &maps.k, 64 * pnl, x.hq, tok0, full);
+            umma::tma_load_3d(st + kOffV + pnl * 8192, &maps.v, 64 * pnl, x.h, tok0, full);
+          }
+        }
+        float* gin = reinterpret_cast<float*>(smem + kOffGin) + s * 2 * kC;
+        gin[lane] = ga;
+        gin[lane + 32] = gb;
+        gin[kC + lane] = ba;
+        gin[kC + lane + 32] = bb;
+        mbar_arrive(&bars[kFull + s]);
+      }
+    }
+    // copies still in flight (after an abort): let them land, within the limit
+    if (lane == 0) {
+      for (int64_t jj = (j > kStages ? j - kStages : 0); jj < j; ++jj)
+        mbar_wait(&bars[kFull + (int)(jj % kStages)], (uint32_t)(jj / kStages) & 1u);
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdKK64 = umma::idesc_bf16(128, 64, false, false);      // A, B K-major
+      constexpr uint32_t kIdMK64 = umma::idesc_bf16(128, 64, true, false);       // A MN-major
+      constexpr uint32_t kIdTM64n = umma::idesc_bf16(128, 64, false, true, true);  // A tmem, B MN, -A
+      constexpr uint32_t kIdTK64 = umma::idesc_bf16(128, 64, false, false);      // A tmem, B K-major
+      constexpr uint32_t kIdTM128 = umma::idesc_bf16(128, 128, false, true);     // A tmem, B MN-major
+      constexpr uint32_t kIdMM128 = umma::idesc_bf16(128, 128, true, true);      // A, B MN-major
+      const uint64_t dTw = umma::sdesc(sb + kOffTw, 16, 1024);
+      const uint64_t dTu = umma::sdesc(sb + kOffTu, 16, 1024);
+      const uint64_t dWm = umma::sdesc(sb + kOffWt, 16384, 1024);
+      auto W = [&](int b, int64_t ph) { return fwait(&bars[b], (uint32_t)ph & 1u, abort_flag); };
+      // [Q; K] K^T of chunk jj (its stage has landed)
+      auto g1 = [&](int64_t jj) {
+        const uint32_t st = sb + (uint32_t)(jj % kStages) * kStageBytes;
+        const uint64_t dQK = umma::sdesc(st + kOffQK, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // K = d_k
+          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma::mma(tmem + kColG1, umma::sdesc_add(dQK, ko), umma::sdesc_add(dQK, 8192 + ko), kIdKK64, kk);
+        }
+        umma::commit(&bars[kG1Full]);
+      };
+      bool ok = true;
+      if (n_total > 0 && (ok = W(kFull + 0, 0))) {
+        umma::fence_after();
+        g1(0);
+      }
+      if (ok && n_total > 1 && (ok = W(kFull + 1, 0) && W(kG1Free, 0))) {
+        umma::fence_after();
+        g1(1);
+      }
+      for (int64_t j = 0; ok && j < n_total; ++j) {
+        const uint32_t st = sb + (uint32_t)(j % kStages) * kStageBytes;
+        const uint64_t dQK = umma::sdesc(st + kOffQK, 16, 1024);       // [Q~; K] rows, K-major
+        const uint64_t dKm = umma::sdesc(st + kOffQK + 8192, 16384, 1024);  // K (K~) as MN-major
+        const uint64_t dVm = umma::sdesc(st + kOffV, 8192, 1024);      // V as MN-major
+        const uint64_t dP = umma::sdesc(sb + kOffP + (uint32_t)(j & 1) * 8192, 16, 1024);
+        if (kDelta) {
+          if (!(ok = W(kPrepDone, j))) break;
+          umma::fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // W^T = K^T Tw^T (K = tokens)
+            umma::mma(tmem + kColW, umma::sdesc_add(dKm, kk * 2048), umma::sdesc_add(dTw, kk * 32), kIdMK64, kk);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // U^T = V^T Tu^T
+            umma::mma(tmem + kColU, umma::sdesc_add(dVm, kk * 2048), umma::sdesc_add(dTu, kk * 32), kIdMK64, kk);
+          umma::commit(&bars[kWFull]);
+          if (!(ok = W(kWFree, j) && W(kSPass, j))) break;
+          umma::fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // U^T -= S0^T W^T (K = d_k)
+            mma_ts(tmem + kColU, tmem + kColSb + 8 * kk, umma::sdesc_add(dWm, kk * 2048), kIdTM64n, 1);
+          umma::commit(&bars[kUFull]);
+        } else {
+          if (!(ok = W(kPrepDone, j) && W(kSPass, j))) break;
+          umma::fence_after();
+        }
+        if (j > 0 && !(ok = W(kOFree, j - 1))) break;
+        umma::fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // O^T = S0^T Q~^T (K = d_k)
+          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ts(tmem + kColO, tmem + kColSb + 8 * kk, umma::sdesc_add(dQK, ko), kIdTK64, kk);
+        }
+        if (kDelta) {
+          if (!(ok = W(kUDone, j) && W(kKt, j))) break;
+          umma::fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // S^T += U^T K~ (K = tokens)
+            mma_ts(tmem + kColS, tmem + kColUb + 8 * kk, umma::sdesc_add(dKm, kk * 2048), kIdTM128, 1);
+          umma::commit(&bars[kSFull]);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // O^T += U^T P^T
+            mma_ts(tmem + kColO, tmem + kColUb + 8 * kk, umma::sdesc_add(dP, kk * 32), kIdTK64, 1);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // S^T += V^T K~
+            umma::mma(tmem + kColS, umma::sdesc_add(dVm, kk * 2048), umma::sdesc_add(dKm, kk * 2048), kIdMM128, 1);
+          umma::commit(&bars[kSFull]);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // O^T += V^T P^T
+            umma::mma(tmem + kColO, umma::sdesc_add(dVm, kk * 2048), umma::sdesc_add(dP, kk * 32), kIdMK64, 1);
+        }
+        umma::commit(&bars[kOFull]);
+        umma::commit(&bars[kEmpty + (int)(j % kStages)]);
+        if (j + 2 < n_total) {
+          if (!(ok = W(kFull + (int)((j + 2) % kStages), (j + 2) / kStages) && W(kG1Free, j + 1))) break;
+          umma::fence_after();
+          g1(j + 2);
+        }
+      }
+      // every MMA issued completes before the tensor memory is released
+      umma::commit(&bars[kDrain]);
+      mbar_wait(&bars[kDrain], 0);
+    }
+  } else if (warp < kWarpState) {
+    // ------------------------------------------------------------------ intra-chunk group
+    const int wi = warp - kWarpPrep;               // 0..3 within the group
+    const int tp = tid - kWarpPrep * 32;           // 0..127
+    const int q4 = warp & 3;
+    const int r = 32 * q4 + lane;                  // this thread's tensor-memory lane
+    const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
+    float* sL = reinterpret_cast<float*>(smem + kOffL);
+    float* sX = reinterpret_cast<float*>(smem + kOffX);
+    int64_t j = 0;
+    int prev_nv = 0;
+    bool ok = true;
+
+    // K~ = diag(gamma_C / gamma) K in place (rows beyond the chunk's tokens zeroed)
+    auto ktilde = [&](int64_t jj, int nv) {
+      unsigned char* st = smem + (uint32_t)(jj % kStages) * kStageBytes + kOffQK;
+      const float* gcg = reinterpret_cast<const float*>(smem + kOffGB) + (jj & 1) * kGB + kC;
+#pragma unroll 2
+      for (int i = 0; i < 8; ++i) {
+        const int idx = tp + 128 * i;
+        const int t = idx >> 4, ch = idx & 15;
+        uint4* ptr = reinterpret_cast<uint4*>(st + umma::panel_piece(128, kC + t, ch));
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (t < nv) {
+          const uint4 v = *ptr;
+          const float f = gcg[t];
+          w.x = pack_bf16x2(bf16_lo(v.x) * f, bf16_hi(v.x) * f);
+          w.y = pack_bf16x2(bf16_lo(v.y) * f, bf16_hi(v.y) * f);
+          w.z = pack_bf16x2(bf16_lo(v.z) * f, bf16_hi(v.z) * f);
+          w.w = pack_bf16x2(bf16_lo(v.w) * f, bf16_hi(v.w) * f);
+        }
+        *ptr = w;
+      }
+    };
+
+    for (int64_t ru = 0; ok && ru * G < units; ++ru) {
+      const int64_t u = unit_of(ru, G, blockIdx.x);
+      if (u >= units) continue;
+      const Unit x = unit_info(p, u);
+      if (!x.valid) continue;
+      const int nch = (x.n_tok + kC - 1) / kC;
+      for (int c = 0; c < nch; ++c, ++j) {
+        const int s = (int)(j % kStages);
+        const int nv = min(kC, x.n_tok - c * kC);
+        float* gbk = reinterpret_cast<float*>(smem + kOffGB) + (j & 1) * kGB;
+        if (j > 0) {
+          // delta rules: K~ of the previous chunk once W_{j-1} (and U~_{j-1}) have read K
+          // and Tw, Tu; the other rules: the previous state update has been issued
+          ok = fwait(&bars[kDelta ? kWFull : kSFull], (uint32_t)(j - 1) & 1u, abort_flag);
+          if (named_bar_or(kNbPrep, 128, !ok)) {
+            ok = false;
+            break;
+          }
+          if (kDelta) {
+            ktilde(j - 1, prev_nv);
+            umma::fence_smem();
+            named_bar_sync(kNbPrep, 128);
+            if (tp == 0) mbar_arrive(&bars[kKt]);
+          }
+        }
+        ok = fwait(&bars[kFull + s], (uint32_t)(j / kStages) & 1u, abort_flag);
+        if (named_bar_or(kNbPrep, 128, !ok)) {
+          ok = false;
+          break;
+        }
+        // gate block (warp wi == 0): prefixes of log |a| and of the sign over the chunk
+        if (wi == 0) {
+          const float* gin = reinterpret_cast<const float*>(smem + kOffGin) + s * 2 * kC;
+          float lg[2], sg[2];
+          bool big = false;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int t = 2 * lane + e;
+            float a, bc, cc;
+            Rule<RULE>::coeffs(gin[t], gin[kC + t], a, bc, cc);
+            if (t >= nv) bc = 0.0f;  // padded tokens write nothing
+            big |= fabsf(a) > 1.0f;
+            lg[e] = __logf(fmaxf(fabsf(a), 1e-30f));
+            sg[e] = a < 0.0f ? -1.0f : 1.0f;
+            gbk[6 * kC + t] = bc;
+          }
+          float l = lg[0] + lg[1], sgn = sg[0] * sg[1];
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const float lo2 = __shfl_up_sync(0xffffffffu, l, off);
+            const float so2 = __shfl_up_sync(0xffffffffu, sgn, off);
+            if (lane >= off) {
+              l += lo2;
+              sgn *= so2;
+            }
+          }
+          const float lprev = l - (lg[0] + lg[1]), sprev = sgn * sg[0] * sg[1];
+          const float lv[2] = {lprev + lg[0], l}, sv[2] = {sprev * sg[0], sgn};
+          const float lfirst = __shfl_sync(0xffffffffu, lv[0], 0), llast = __shfl_sync(0xffffffffu, l, 31);
+          const float slast = __shfl_sync(0xffffffffu, sgn, 31);
+          const bool fact = !__any_sync(0xffffffffu, big) && (lfirst - llast) <= 80.0f;
+          const float m = 0.5f * (lfirst + llast);
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int t = 2 * lane + e;
+            gbk[t] = sv[e] * __expf(lv[e]);
+            gbk[kC + t] = slast * sv[e] * __expf(llast - lv[e]);
+            gbk[2 * kC + t] = sv[e] * __expf(lv[e] - m);
+            gbk[3 * kC + t] = sv[e] * __expf(m - lv[e]);
+            gbk[4 * kC + t] = lv[e];
+            gbk[5 * kC + t] = sv[e];
+          }
+          if (lane == 0) gbk[7 * kC] = fact ? 1.0f : 0.0f;
+          __threadfence_block();
+        }
+        named_bar_sync(kNbPrep, 128);
+        if (tp == 0) *gates_done = (uint32_t)(j + 1);  // the state group reads gamma_C from here
+        const bool fact = gbk[7 * kC] != 0.0f;
+        const float* sFa = gbk + 2 * kC;
+        const float* sFb = gbk + 3 * kC;
+        const float* sLg = gbk + 4 * kC;
+        const float* sSg = gbk + 5 * kC;
+        const float* sBt = gbk + 6 * kC;
+
+        // P = (Q K^T) (.) M (lanes 0..63) and L (lanes 64..127, delta rules) from tensor memory
+        ok = fwait(&bars[kG1Full], (uint32_t)j & 1u, abort_flag);
+        if (named_bar_or(kNbPrep, 128, !ok)) {
+          ok = false;
+          break;
+        }
+        umma::fence_after();
+        if (r < kC) {
+          const int t = r;
+          unsigned char* sP = smem + kOffP + (j & 1) * 8192;
+#pragma unroll
+          for (int c16 = 0; c16 < 4; ++c16) {
+            uint32_t v[16];
+            umma::ld16(tq + kColG1 + 16 * c16, v);
+            umma::wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int s_ = 16 * c16 + e;
+              float y = 0.0f;
+              if (s_ <= t)
+                y = (fact ? sFa[t] * sFb[s_] : sSg[t] * sSg[s_] * __expf(sLg[t] - sLg[s_])) * __uint_as_float(v[e]);
+              v[e] = __float_as_uint(y);
+            }
+#pragma unroll
+            for (int pc = 0; pc < 2; ++pc)
+              *reinterpret_cast<uint4*>(sP + umma::panel_piece(kC, t, 2 * c16 + pc)) =
+                  make_uint4(pack2(v[8 * pc], v[8 * pc + 1]), pack2(v[8 * pc + 2], v[8 * pc + 3]),
+                             pack2(v[8 * pc + 4], v[8 * pc + 5]), pack2(v[8 * pc + 6], v[8 * pc + 7]));
+          }
+        } else if (kDelta) {
+          const int t = r - kC;
+#pragma unroll
+          for (int c16 = 0; c16 < 4; ++c16) {
+            uint32_t v[16];
+            umma::ld16(tq + kColG1 + 16 * c16, v);
+            umma::wait_ld();
+            float y[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int s_ = 16 * c16 + e;
+              y[e] = 0.0f;
+              if (s_ < t)
+                y[e] = sBt[t] * (fact ? sFa[t] * sFb[s_] : sSg[t] * sSg[s_] * __expf(sLg[t] - sLg[s_])) *
+                       __uint_as_float(v[e]);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<float4*>(sL + t * kLs + 16 * c16 + 4 * q) =
+                  make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+          }
+        }
+        umma::fence_before();
+        named_bar_sync(kNbPrep, 128);
+        if (tp == 0) mbar_arrive(&bars[kG1Free]);
+
+        // Q~ = diag(gamma) Q in place
+        {
+          unsigned char* st = smem + s * kStageBytes + kOffQK;
+#pragma unroll 2
+          for (int i = 0; i < 8; ++i) {
+            const int idx = tp + 128 * i;
+            const int t = idx >> 4, ch = idx & 15;
+            uint4* ptr = reinterpret_cast<uint4*>(st + umma::panel_piece(128, t, ch));
+            const uint4 v = *ptr;
+            const float f = gbk[t];
+            *ptr = make_uint4(pack_bf16x2(bf16_lo(v.x) * f, bf16_hi(v.x) * f),
+                              pack_bf16x2(bf16_lo(v.y) * f, bf16_hi(v.y) * f),
+                              pack_bf16x2(bf16_lo(v.z) * f, bf16_hi(v.z) * f),
+                              pack_bf16x2(bf16_lo(v.w) * f, bf16_hi(v.w) * f));
+          }
+        }
+
+        if (kDelta) {
+          // T = (I + L)^-1 in place of L, by 16 x 16 blocks; Tw = T diag(b gamma), Tu = T diag(b)
+          const float* sGm = gbk;
+          auto put2 = [&](int row, int col, float v0, float v1) {
+            const uint32_t off = umma::panel_off(kC, row, col);
+            *reinterpret_cast<uint32_t*>(smem + kOffTw + off) =
+                pack_bf16x2(v0 * sBt[col] * sGm[col], v1 * sBt[col + 1] * sGm[col + 1]);
+            *reinterpret_cast<uint32_t*>(smem + kOffTu + off) = pack_bf16x2(v0 * sBt[col], v1 * sBt[col + 1]);
+          };
+          {
+            // diagonal block wi by forward substitution: lane c < 16 owns column c
+            const int b0 = 16 * wi, cc = lane & 15;
+            float col[16];
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+              const float4* lr = reinterpret_cast<const float4*>(sL + (b0 + rr) * kLs + b0);
+              float xv = (rr == cc) ? 1.0f : 0.0f;
+#pragma unroll
+              for (int m4 = 0; m4 < (rr + 3) / 4; ++m4) {
+                const float4 l4 = lr[m4];
+                const float lv4[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (4 * m4 + e < rr) xv -= lv4[e] * col[4 * m4 + e];
+              }
+              col[rr] = (rr < cc) ? 0.0f : xv;
+            }
+            __syncwarp();
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+              if (lane < 16) sL[(b0 + rr) * kLs + b0 + cc] = col[rr];
+              const float nxt = __shfl_down_sync(0xffffffffu, col[rr], 1);
+              if (lane < 16 && (cc & 1) == 0) put2(b0 + rr, b0 + cc, col[rr], nxt);
+            }
+          }
+          named_bar_sync(kNbPrep, 128);
+          // block row bi: T_{bi,bj} = -D_bi sum_{bk=bj}^{bi-1} L_{bi,bk} T_{bk,bj}, warp bj < bi
+#pragma unroll 1
+          for (int bi = 1; bi < 4; ++bi) {
+            float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            if (wi < bi) {
+              const int bj = wi;
+              const int g8 = lane >> 2, t4 = lane & 3;
+              float xs[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+              for (int bk = bj; bk < bi; ++bk)
+                chunk::mma16x16x16_tf32(xs, sL + (16 * bi) * kLs + 16 * bk, kLs, sL + (16 * bk) * kLs + 16 * bj,
+                                        kLs, lane);
+              float* xw = sX + wi * 16 * kXs;
+#pragma unroll
+              for (int nt = 0; nt < 2; ++nt) {
+                xw[g8 * kXs + 8 * nt + 2 * t4] = xs[nt][0];
+                xw[g8 * kXs + 8 * nt + 2 * t4 + 1] = xs[nt][1];
+                xw[(g8 + 8) * kXs + 8 * nt + 2 * t4] = xs[nt][2];
+                xw[(g8 + 8) * kXs + 8 * nt + 2 * t4 + 1] = xs[nt][3];
+              }
+              __syncwarp();
+              chunk::mma16x16x16_tf32(y, sL + (16 * bi) * kLs + 16 * bi, kLs, xw, kXs, lane);
+            }
+            named_bar_sync(kNbPrep, 128);  // row bi of L is read: its blocks may now take T
+            if (wi < bi) {
+              const int bj = wi;
+              const int g8 = lane >> 2, t4 = lane & 3;
+#pragma unroll
+              for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+                for (int hlf = 0; hlf < 2; ++hlf) {
+                  const int row = 16 * bi + g8 + 8 * hlf, col = 16 * bj + 8 * nt + 2 * t4;
+                  const float v0 = -y[nt][2 * hlf], v1 = -y[nt][2 * hlf + 1];
+                  sL[row * kLs + col] = v0;
+                  sL[row * kLs + col + 1] = v1;
+                  put2(row, col, v0, v1);
+                }
+              }
+            }
+            named_bar_sync(kNbPrep, 128);
+          }
+        } else {
+          ktilde(j, nv);  // G1 of this chunk has read K
+        }
+        umma::fence_smem();  // P, Q~, Tw, Tu (K~) -> tensor cores
+        named_bar_sync(kNbPrep, 128);
+        if (tp == 0) mbar_arrive(&bars[kPrepDone]);
+        prev_nv = nv;
+      }
+    }
+    if (kDelta && ok && j > 0) {
+      // K~ of the last chunk
+      ok = fwait(&bars[kWFull], (uint32_t)(j - 1) & 1u, abort_flag);
+      if (!named_bar_or(kNbPrep, 128, !ok)) {
+        ktilde(j - 1, prev_nv);
+        umma::fence_smem();
+        named_bar_sync(kNbPrep, 128);
+        if (tp == 0) mbar_arrive(&bars[kKt]);
+      }
+    }
+  } else if (warp < kWarpOut) {
+    // ------------------------------------------------------------------ state group
+    const int tp = tid - kWarpState * 32;
+    const int q4 = warp & 3;
+    const int r = 32 * q4 + lane;  // d_v index
+    const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
+    int64_t j = 0;
+    bool ok = true;
+    for (int64_t ru = 0; ok && ru * G < units; ++ru) {
+      const int64_t u = unit_of(ru, G, blockIdx.x);
+      if (u >= units) continue;
+      const Unit x = unit_info(p, u);
+      if (x.err && tp == 0) report(p.err, x.err);
+      if (!x.valid) continue;
+      const int nch = (x.n_tok + kC - 1) / kC;
+      const int64_t sbase_src = ((int64_t)x.rs * H + x.h) * (kD * kD);
+      const int64_t dbase = ((int64_t)x.ws * H + x.h) * (kD * kD);
+      if (nch == 0) {
+        // empty sequence: the initial state (or zero) goes to the destination
+        for (int i = 0; i < kD; ++i) {
+          float v = 0.0f;
+          if (p.read_slot)
+            v = p.src_dtype == LA_F32 ? static_cast<const float*>(p.src)[sbase_src + i * kD + r]
+                                      : __bfloat162float(static_cast<const __nv_bfloat16*>(p.src)[sbase_src + i * kD + r]);
+          if (p.dst_dtype == LA_F32)
+            static_cast<float*>(p.dst)[dbase + i * kD + r] = v;
+          else
+            static_cast<__nv_bfloat16*>(p.dst)[dbase + i * kD + r] = __float2bfloat16_rn(v);
+        }
+        continue;
+      }
+      // initial state S^T: lane = d_v index r, columns = d_k
+#pragma unroll 1
+      for (int c16 = 0; c16 < 8; ++c16) {
+        uint32_t v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int i = 16 * c16 + e;
+          float sv = 0.0f;
+          if (p.read_slot) {
+            const int64_t el = sbase_src + (int64_t)i * kD + r;
+            sv = p.src_dtype == LA_F32 ? static_cast<const float*>(p.src)[el]
+                                       : __bfloat162float(static_cast<const __nv_bfloat16*>(p.src)[el]);
+          }
+          v[e] = __float_as_uint(sv);
+        }
+        umma::st16(tq + kColS + 16 * c16, v);
+      }
+      umma::wait_st();
+      for (int c = 0; c < nch; ++c, ++j) {
+        if (c > 0) ok = fwait(&bars[kSFull], (uint32_t)(j - 1) & 1u, abort_flag);
+        // the chunk's gate block (gamma_C), published by the intra-chunk group
+        if (ok) {
+          const uint64_t t0 = global_timer_ns();
+          uint32_t polls = 0;
+          while (*gates_done <= (uint32_t)j) {
+            if ((++polls & 15u) == 0 && (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs)) {
+              *abort_flag = 1u;
+              ok = false;
+              break;
+            }
+          }
+          __threadfence_block();
+        }
+        if (named_bar_or(kNbState, 128, !ok)) {
+          ok = false;
+          break;
+        }
+        umma::fence_after();
+        const float gC = (reinterpret_cast<const float*>(smem + kOffGB) + (j & 1) * kGB)[kC - 1];
+        // S pass: S0^T -> BF16 (the A operand of this chunk's products), S^T *= gamma_C
+#pragma unroll 1
+        for (int c32 = 0; c32 < 4; ++c32) {
+          uint32_t a[16], b[16], w[16];
+          umma::ld16(tq + kColS + 32 * c32, a);
+          umma::ld16(tq + kColS + 32 * c32 + 16, b);
+          umma::wait_ld();
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            w[e] = pack2(a[2 * e], a[2 * e + 1]);
+            w[8 + e] = pack2(b[2 * e], b[2 * e + 1]);
+          }
+          umma::st16(tq + kColSb + 16 * c32, w);
+          if (kGate) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              a[e] = __float_as_uint(__uint_as_float(a[e]) * gC);
+              b[e] = __float_as_uint(__uint_as_float(b[e]) * gC);
+            }
+            umma::st16(tq + kColS + 32 * c32, a);
+            umma::st16(tq + kColS + 32 * c32 + 16, b);
+          }
+        }
+        umma::wait_st();
+        umma::fence_before();
+        named_bar_sync(kNbState, 128);
+        if (tp == 0) mbar_arrive(&bars[kSPass]);
+        if (kDelta) {
+          ok = fwait(&bars[kUFull], (uint32_t)j & 1u, abort_flag);
+          if (named_bar_or(kNbState, 128, !ok)) {
+            ok = false;
+            break;
+          }
+          umma::fence_after();
+#pragma unroll
+          for (int c32 = 0; c32 < 2; ++c32) {
+            uint32_t a[16], b[16], w[16];
+            umma::ld16(tq + kColU + 32 * c32, a);
+            umma::ld16(tq + kColU + 32 * c32 + 16, b);
+            umma::wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              w[e] = pack2(a[2 * e], a[2 * e + 1]);
+              w[8 + e] = pack2(b[2 * e], b[2 * e + 1]);
+            }
+            umma::st16(tq + kColUb + 16 * c32, w);
+          }
+          umma::wait_st();
+          umma::fence_before();
+          named_bar_sync(kNbState, 128);
+          if (tp == 0) mbar_arrive(&bars[kUDone]);
+        }
+      }
+      if (!ok) break;
+      // final state S[i][r] = S^T[r][i]
+      ok = fwait(&bars[kSFull], (uint32_t)(j - 1) & 1u, abort_flag);
+      if (named_bar_or(kNbState, 128, !ok)) {
+        ok = false;
+        break;
+      }
+      umma::fence_after();
+#pragma unroll 1
+      for (int c16 = 0; c16 < 8; ++c16) {
+        uint32_t v[16];
+        umma::ld16(tq + kColS + 16 * c16, v);
+        umma::wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int64_t el = dbase + (int64_t)(16 * c16 + e) * kD + r;
+          if (p.dst_dtype == LA_F32)
+            static_cast<float*>(p.dst)[el] = __uint_as_float(v[e]);
+          else
+            static_cast<__nv_bfloat16*>(p.dst)[el] = __float2bfloat16_rn(__uint_as_float(v[e]));
+        }
+      }
+      umma::fence_before();
+    }
+  } else {
+    // ------------------------------------------------------------------ output group
+    const int tp = tid - kWarpOut * 32;
+    const int q4 = warp & 3;
+    const int r = 32 * q4 + lane;  // d_k index (W^T) / d_v index (O^T)
+    const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
+    __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.o);
+    int64_t j = 0;
+    bool ok = true;
+    for (int64_t ru = 0; ok && ru * G < units; ++ru) {
+      const int64_t u = unit_of(ru, G, blockIdx.x);
+      if (u >= units) continue;
+      const Unit x = unit_info(p, u);
+      if (!x.valid) continue;
+      const int nch = (x.n_tok + kC - 1) / kC;
+      for (int c = 0; c < nch; ++c, ++j) {
+        if (kDelta) {
+          // W^T rows (lane = d_k index) -> shared memory, the B operand of the U update
+          ok = fwait(&bars[kWFull], (uint32_t)j & 1u, abort_flag);
+          if (named_bar_or(kNbOut, 128, !ok)) {
+            ok = false;
+            break;
+          }
+          umma::fence_after();
+#pragma unroll
+          for (int c16 = 0; c16 < 4; ++c16) {
+            uint32_t v[16];
+            umma::ld16(tq + kColW + 16 * c16, v);
+            umma::wait_ld();
+#pragma unroll
+            for (int pc = 0; pc < 2; ++pc)
+              *reinterpret_cast<uint4*>(smem + kOffWt + umma::panel_piece(128, r, 2 * c16 + pc)) =
+                  make_uint4(pack2(v[8 * pc], v[8 * pc + 1]), pack2(v[8 * pc + 2], v[8 * pc + 3]),
+                             pack2(v[8 * pc + 4], v[8 * pc + 5]), pack2(v[8 * pc + 6], v[8 * pc + 7]));
+          }
+          umma::fence_smem();
+          umma::fence_before();
+          named_bar_sync(kNbOut, 128);
+          if (tp == 0) mbar_arrive(&bars[kWFree]);
+        }
+        // outputs o_t[r] = scale O^T[r][t] for the chunk's tokens
+        ok = fwait(&bars[kOFull], (uint32_t)j & 1u, abort_flag);
+        if (named_bar_or(kNbOut, 128, !ok)) {
+          ok = false;
+          break;
+        }
+        umma::fence_after();
+        const int tok0 = x.t0 + c * kC;
+        const int nv = min(kC, x.n_tok - c * kC);
+        __nv_bfloat16* orow = og + ((int64_t)tok0 * H + x.h) * kD + r;
+#pragma unroll
+        for (int c16 = 0; c16 < 4; ++c16) {
+          uint32_t v[16];
+          umma::ld16(tq + kColO + 16 * c16, v);
+          umma::wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int t = 16 * c16 + e;
+            if (t < nv) orow[(int64_t)t * H * kD] = __float2bfloat16_rn(p.scale * __uint_as_float(v[e]));
+          }
+        }
+        umma::fence_before();
+        named_bar_sync(kNbOut, 128);
+        if (tp == 0) mbar_arrive(&bars[kOFree]);
+      }
+    }
+  }
+
+  if (tid == 0 && *abort_flag) report(p.err, LA_DEVERR_TIMEOUT);
+  umma::fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    umma::fence_after();
+    umma::dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int RULE>
+cudaError_t launch_chunk_fused(const ScanParams& p, cudaStream_t stream) {
+  const void* fn = reinterpret_cast<const void*>(&chunk_fused_kernel<RULE>);
+  const int per_sm = prepare_kernel(fn, fused::kThreads, fused::kSmem);
+  // one CTA per SM: the kernel holds all of the SM's tensor memory
+  if (per_sm != 1) return cudaErrorInvalidConfiguration;
+  TcMaps maps;
+  memset(&maps, 0, sizeof(maps));  // no tokens: nothing is staged, the maps are never read
+  if (p.total_tokens > 0 &&
+      (!encode_rows_map(&maps.q, p.q, p.n_qk_heads, p.total_tokens) ||
+       !encode_rows_map(&maps.k, p.k, p.n_qk_heads, p.total_tokens) ||
+       !encode_rows_map(&maps.v, p.v, p.n_v_heads, p.total_tokens)))
+    return cudaErrorInvalidValue;
+  const int64_t units = (int64_t)p.n_seqs * p.n_v_heads;
+  const int64_t cap = device_sm_count();
+  const int grid = (int)(units < cap ? units : cap);
+  if (grid <= 0) return cudaSuccess;
+  chunk_fused_kernel<RULE><<<grid, fused::kThreads, fused::kSmem, stream>>>(p, maps);
+  return cudaGetLastError();
+}
+
+}  // namespace la
