@@ -1,23 +1,25 @@
 """Benchmark of the recurrent-state step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode64|decode512|mamba2|prefill32] [--rows all|none]
+                    [--workload decode512|decode64|mamba2|prefill32|...] [--rows all|none]
 
-Prints ONE JSON line.  The headline workload is the batched decode step the metric is
-quoted on (decode64: B=64 requests, 16 q/k heads shared by 32 state heads, 128 x 128
-BF16 state in a 256-slot pool, gated_delta).  One step = one call of la_state_step over
-the batch (slot gather, load, S^T k / S^T q reductions, delta vector, update, readout,
-store: every row of the decode path).  `value` = algorithmic state-update bytes of all
-ranks / device time of one step (max over ranks), in GB/s; `e2e` is the same metric
-measured through the same C-ABI call with the step's inputs copied from pinned host
-memory and its output copied back inside the timed region.
+Prints ONE JSON line.  The headline workload is the largest single-GPU configuration of the
+batched decode step the metric is quoted on (decode512: B=512 requests, 16 q/k heads shared
+by 32 state heads, 128 x 128 BF16 state in a 1024-slot pool, half the requests reading a
+prefix-cache checkpoint slot and writing a distinct live slot, gated_delta).  One step = one
+call of la_state_step over the batch (slot gather, load, S^T k / S^T q reductions, delta
+vector, update, readout, store: every row of the decode path).  `value` = algorithmic
+state-update bytes of all ranks / device time of one step (max over ranks), in GB/s; `e2e`
+is the same metric measured through the same C-ABI call with the step's inputs copied from
+pinned host memory and its output copied back inside the timed region.
 
 Timing: W untimed warm-up steps, then K steps back to back between CUDA events on the
-launching stream, bracketed by a barrier and a device synchronize.  The decode64 pool
-(256 MiB) is larger than L2 (126 MB): step i uses slot set i mod 4 of four disjoint
-sets of 64 slots, so each step's state was last touched three steps (384 MiB of
-traffic) earlier.  A second figure with an L2 flush (a 256 MiB write) before every step
-is reported beside it.
+launching stream, bracketed by a barrier and a device synchronize.  decode512 moves 1 GiB of
+state per step through a 1 GiB pool (the 126 MB L2 holds an eighth of one step's traffic); a
+second figure with an L2 flush (a 256 MiB write) before every step is reported beside it.
+The other workloads (decode64, mamba2, the token-serial and chunked prefills, the kda /
+query-group / q8 / convolution variants, the pool copy) are measured under `rows`, and a
+compact summary of every row closes the line (`rows_summary`).
 
 With --gpus N (launched by torchrun) every rank runs its own replica of the workload
 on its own GPU: the step has no exchange between GPUs (every (request, head) tile is
@@ -129,6 +131,7 @@ KERNEL_SOURCES = {
     "scan": ["la_scan.cuh", "la_device.cuh"],
     "chunk": ["la_chunk.cuh", "la_device.cuh"],
     "chunk_tc": ["la_chunk.cuh", "la_chunk_tc.cuh", "la_umma.cuh", "la_device.cuh"],
+    "chunk_fused": ["la_chunk.cuh", "la_chunk_fused.cuh", "la_chunk_tc.cuh", "la_umma.cuh", "la_device.cuh"],
     "pool": ["la_pool.cu"],
 }
 
@@ -379,24 +382,27 @@ def chunk_mma_flops(lengths, n_v_heads, d_k, d_v, rule):
     return chunks * n_v_heads * per
 
 
-def tensor_roofline(run, inp, ms, peaks):
-    """Roofline object of the chunked prefill: the chunked algorithm's MMA flops against the
-    measured dense BF16 peak (a cuBLAS GEMM on tcgen05).  The one-launch kernel issues
-    mma.sync; the two-launch form runs its recurrence on tcgen05 (delta rules)."""
+def chunk_roofline(run, inp, ms, peaks):
+    """Roofline object of the chunked prefill.  Its tensor-core work is a dense contraction
+    that finishes below the HBM time, so the bound is HBM: the method's algorithmic bytes
+    (q, k, v, o, gates of every token, the final state; no re-reads) over the device time,
+    against the measured copy bandwidth.  The tensor rate is reported beside it twice: the
+    method's own 6 flops per state element and token, and the chunked algorithm's MMA flops
+    (which the measured dense BF16 GEMM peak bounds)."""
     lens = (inp.cu_seqlens[1:] - inp.cu_seqlens[:-1]).tolist()
-    tf = chunk_mma_flops(lens, inp.n_v_heads, inp.d_k, inp.d_v, inp.rule) / (ms * 1e-3) / 1e12
-    peak = peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)
+    nbytes, flops = run.bytes_flops()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    mma_tf = chunk_mma_flops(lens, inp.n_v_heads, inp.d_k, inp.d_v, inp.rule) / (ms * 1e-3) / 1e12
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)
     two = run.ws is not None and inp.rule in ("delta", "gated_delta")
-    out = {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-           "traffic": recorded_traffic("chunk_tc" if two else "chunk", "prefill32"),
-           "hbm_gb_s": run.bytes_flops()[0] / (ms * 1e-3) / 1e9}
-    if two:
-        out["kernel"] = "la::chunk_prep_kernel (mma.sync) + la::chunk_tc_kernel (tcgen05)"
-        out["peak_note"] = "measured dense BF16 GEMM (MEASURED_PEAKS.json bf16_tflops); both launches together"
-    else:
-        out["kernel"] = "la::chunk_scan_kernel"
-        out["peak_note"] = ("measured dense BF16 GEMM (MEASURED_PEAKS.json bf16_tflops); the kernel uses mma.sync "
-                            "BF16 m16n8k16, whose own ceiling on this part is about a third of that")
+    out = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+           "traffic": recorded_traffic("chunk_tc" if two else "chunk_fused", "prefill32"),
+           "algorithmic_bytes_per_launch": nbytes,
+           "method_tflops": flops / (ms * 1e-3) / 1e12,
+           "mma_tflops": mma_tf, "mma_frac_of_bf16_peak": mma_tf / peak_tf,
+           "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs; bf16_tflops for mma_frac)"}
+    out["kernel"] = ("la::chunk_prep_kernel (mma.sync) + la::chunk_tc_kernel (tcgen05)" if two
+                     else "la::chunk_fused_kernel (tcgen05)")
     return out
 
 
@@ -735,6 +741,53 @@ def cpu_baseline_decode(inp, budget_s=10.0):
     return 1e3 * statistics.median(times), oracle.num_threads(), f"{len(times)} whole decode steps of the workload"
 
 
+def cpu_baseline_scan(inp, n_sub=4, budget_s=10.0, max_tokens=None):
+    """The CPU oracle as it stands on a prefill workload, on a fixed subset: the first
+    n_sub sequences (all heads; with max_tokens, only that many leading tokens of the first
+    sequence), repeated until about budget_s; the rate is scaled to the whole workload by
+    bytes and tokens (the oracle's cost is linear in tokens).  Returns (GB/s, tokens/s,
+    threads, sample description) or None."""
+    import oracle
+    import numpy as np
+    cu = inp.cu_seqlens.numpy()
+    n = min(n_sub, len(cu) - 1)
+    if max_tokens is not None:
+        n = 1
+        cu = np.array([0, min(int(cu[1]), int(max_tokens))], dtype=np.int64)
+    t1 = int(cu[n])
+    if t1 <= 0:
+        return None
+    sub = lambda t: None if t is None else t[:t1].double().numpy()  # noqa: E731
+    st = "bf16" if inp.state_dtype.itemsize == 2 else "f32"
+    io = "bf16" if inp.io_dtype.itemsize == 2 else "f32"
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while time.perf_counter() < t_end or not times:
+        t0 = time.perf_counter()
+        oracle.scan(inp.rule, inp.n_qk_heads, cu[:n + 1].astype(np.int32), sub(inp.q), sub(inp.k), sub(inp.v),
+                    sub(inp.g), sub(inp.beta), inp.scale, dst_dtype=st, io_dtype=io)
+        times.append(time.perf_counter() - t0)
+    sec = statistics.median(times)
+    b, _ = scan_bytes_and_flops(T=t1, n_seqs=n, n_qk_heads=inp.n_qk_heads, n_v_heads=inp.n_v_heads, d_k=inp.d_k,
+                                d_v=inp.d_v, io_bytes=inp.q.element_size(), rule=inp.rule,
+                                final_state_bytes=inp.state_dtype.itemsize)
+    return (b / sec / 1e9, t1 / sec, oracle.num_threads(),
+            (f"the first {t1} tokens of sequence 0" if max_tokens is not None else f"sequences 0..{n - 1}") +
+            f" of the workload ({t1} tokens, all {inp.n_v_heads} heads), median of {len(times)} runs; rates "
+            f"scaled to the whole workload by bytes and tokens")
+
+
+def cpu_single_thread(fn, *args, **kw):
+    """Runs a CPU baseline with the oracle held to one thread (restored afterwards)."""
+    import oracle
+    n = oracle.num_threads()
+    oracle.set_threads(1)
+    try:
+        return fn(*args, **kw)
+    finally:
+        oracle.set_threads(n)
+
+
 # --------------------------------------------------------------------------------------
 
 
@@ -792,12 +845,11 @@ def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_ev
             row["config"]["ckpt_every"] = ckpt_every
             row["config"]["checkpoints"] = run.n_ckpt
         if chunked:
-            row["config"]["algorithm"] = "chunked (64-token WY/UT form, BF16 tensor-core products)" + \
-                ("; intra-chunk inverses as a separate parallel launch through a workspace, the recurrence on "
-                 "tcgen05 with the state in tensor memory" if chunked == "ws" else "")
-            row["hbm"] = {"achieved_gb_s": row["gb_s"], "frac_of_measured": row["gb_s"] / peaks["hbm_gbs"]}
-            row["token_serial_equivalent_tflops"] = tf  # 6 flops per state element per token, for comparison
-            row["roofline"] = tensor_roofline(run, inp, ms, peaks)
+            row["config"]["algorithm"] = "chunked (64-token WY/UT form, BF16 tcgen05 products, FP32 state)" + \
+                ("; intra-chunk inverses as a separate parallel launch through a workspace, then the recurrence "
+                 "with the state in tensor memory" if chunked == "ws" else
+                 "; one launch, the intra-chunk inverses computed on chip beside the recurrence")
+            row["roofline"] = chunk_roofline(run, inp, ms, peaks)
         else:
             row["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
                                "traffic": recorded_traffic("scan", name + (f"_ckpt{ckpt_every}" if ckpt_every else "")),
@@ -809,13 +861,33 @@ def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_ev
     return row
 
 
+def build_runner_inputs(name, seed=0):
+    """The host inputs of a workload (no device buffers)."""
+    from gated_deltanet_recurrent_la_b200 import workloads as W
+    return W.WORKLOADS[name](seed)
+
+
+def rows_summary(rows):
+    """One short entry per row (time, achieved rate, roofline fraction), so that every
+    row's figures sit at the end of the printed line."""
+    out = {}
+    for name, r in rows.items():
+        rf = r.get("roofline", {})
+        e = {"ms": round(r.get("ms_per_step", r.get("ms_per_call", float("nan"))), 5)}
+        if rf:
+            e.update(bound=rf.get("bound"), achieved=round(rf.get("achieved", 0.0), 1), unit=rf.get("unit"),
+                     frac=round(rf.get("frac", 0.0), 4))
+        out[name] = e
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode64",
+    ap.add_argument("--workload", default="decode512",
                     choices=["decode64", "decode512", "mamba2", "prefill32", "kda_decode64", "kda_prefill32",
                              "qgroup_decode256", "q8_decode64", "conv_decode64", "conv_prefill32"])
     ap.add_argument("--rows", default="all", choices=["all", "none"])
@@ -854,7 +926,8 @@ def main():
            "data": "synthetic (seeded host generator; no dataset)",
            "config": dict(describe(a.workload, inp), parallelism=f"replicas x{world}",
                           l2="inputs larger than L2: 4 disjoint 64-slot sets of the 256 MiB pool rotated step to step"
-                          if a.workload == "decode64" else "inputs larger than L2")}
+                          if a.workload == "decode64" else "inputs larger than L2 (1 GiB of state per step)"
+                          if a.workload == "decode512" else "inputs larger than L2")}
     if inp.kind == "step":
         out["pct_of_peak"] = 100 * per_gpu / peaks["hbm_gbs"]
         out["pct_of_spec_8000"] = 100 * per_gpu / SPEC_HBM_GBS
@@ -870,7 +943,7 @@ def main():
         tf = flops / (ms * 1e-3) / 1e12
         out["tokens_per_s"] = world * run.T / (ms * 1e-3)
         if a.scan_algo != "serial":
-            out["roofline"] = tensor_roofline(run, inp, ms, peaks)
+            out["roofline"] = chunk_roofline(run, inp, ms, peaks)
         else:
             out["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
                                "traffic": recorded_traffic("scan", a.workload), "kernel": "la::scan_kernel"}
@@ -890,8 +963,8 @@ def main():
 
     if a.rows == "all":
         rows = {}
-        for name in ("decode512", "mamba2", "prefill32", "kda_decode64", "kda_prefill32", "qgroup_decode256",
-                     "q8_decode64", "conv_decode64", "conv_prefill32"):
+        for name in ("decode512", "decode64", "mamba2", "prefill32", "kda_decode64", "kda_prefill32",
+                     "qgroup_decode256", "q8_decode64", "conv_decode64", "conv_prefill32"):
             if name == a.workload:
                 continue
             k = a.steps if "prefill" not in name else max(3, min(a.steps, 20))
@@ -920,10 +993,34 @@ def main():
 
     if rank == 0:
         if world == 1:
-            cms, cores, sample = cpu_baseline_decode(inp, a.cpu_budget) if inp.kind == "step" else (None, None, None)
-            if cms is not None:
+            if inp.kind == "step":
+                cms, cores, sample = cpu_baseline_decode(inp, a.cpu_budget)
                 out["cpu_baseline"] = {"value": nbytes / (cms * 1e-3) / 1e9, "unit": "GB/s", "cores": cores,
                                        "kind": "oracle", "sample": sample, "ms_per_step": cms}
+                c1, _, s1 = cpu_single_thread(cpu_baseline_decode, inp, min(a.cpu_budget, 5.0))
+                out["cpu_baseline"]["single_thread"] = {"value": nbytes / (c1 * 1e-3) / 1e9, "unit": "GB/s",
+                                                        "cores": 1, "sample": s1, "ms_per_step": c1}
+            else:
+                cb = cpu_baseline_scan(inp, budget_s=a.cpu_budget)
+                if cb is not None:
+                    out["cpu_baseline"] = {"value": cb[0], "unit": "GB/s", "cores": cb[2], "kind": "oracle",
+                                           "sample": cb[3], "tokens_per_s": cb[1], "scaled": True}
+            if "rows" in out and "prefill32" in out["rows"]:
+                # the prefill workload (all its forms share it): a fixed 4-sequence subset on all
+                # host cores and a 1024-token prefix on one core, both scaled by tokens
+                pin = build_runner_inputs("prefill32")
+                cb = cpu_baseline_scan(pin, budget_s=a.cpu_budget)
+                c1 = cpu_single_thread(cpu_baseline_scan, pin, budget_s=0.0, max_tokens=1024)
+                if cb is not None and c1 is not None:
+                    base = {"value": cb[0], "unit": "GB/s", "cores": cb[2], "kind": "oracle", "sample": cb[3],
+                            "tokens_per_s": cb[1], "scaled": True,
+                            "single_thread": {"value": c1[0], "unit": "GB/s", "cores": 1, "sample": c1[3],
+                                              "tokens_per_s": c1[1], "scaled": True}}
+                    for name in ("prefill32", "prefill32_chunked", "prefill32_chunked_two_launch"):
+                        if name in out["rows"]:
+                            out["rows"][name]["cpu_baseline"] = base
+        if "rows" in out:
+            out["rows_summary"] = rows_summary(out["rows"])
         print(json.dumps(out), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -10,29 +10,35 @@
 //   L  = strictly-lower( b_t (gamma_t / gamma_s) k_t . k_s ),   T = (I + L)^-1
 //   W  = T diag(b gamma) K,    U~ = T diag(b) V,    U = U~ - W S0      (delta rules; else U = V)
 //   O  = scale ( Q~ S0 + P U ),   Q~ = diag(gamma) Q,   P = (Q K^T) (.) M,  M_ts = gamma_t / gamma_s (s <= t)
-//   S  = gamma_C S0 + K~^T U,     K~ = diag(gamma_C / gamma) K
+//   S  = gamma_C S0 + K^T Us,     Us = diag(gamma_C / gamma) U     (rules without inverse: K~^T V,
+//                                                                    K~ = diag(gamma_C / gamma) K)
 //
 // which unrolls the token recurrence u_t = b (v_t - c S_{t-1}^T k_t), S_t = a S_{t-1} + k_t u_t^T
 // exactly.  Every product is an M = 128 tcgen05 MMA with BF16 operands and an FP32
 // accumulator in tensor memory; the transposed forms (U^T, O^T, S^T: one d_v index per
-// tensor-memory lane) let the state, its BF16 copy S0^T and the BF16 copy of U^T feed the
-// next products straight from tensor memory as the A operand.
+// tensor-memory lane) let the state, its BF16 copy S0^T and the BF16 copies of U^T and Us^T
+// feed the next products straight from tensor memory as the A operand.
 //
 // One CTA of 14 warps per SM, each role a pipeline stage joined by mbarriers:
-//   warp 0       loads: Q, K, V of a chunk by TMA tensor maps into one of three stages,
-//                the chunk's gates by its lanes
+//   warp 0       loads: Q, K, V of a chunk by TMA tensor maps into one of three stages;
+//                its lanes read the chunk's gates and write the stage's gate block
+//                (prefix products of the decays, their factored ratios, b_t)
 //   warp 1       lane 0 issues every MMA (and owns the tensor-memory allocation)
-//   warps 2-5    intra-chunk work, up to two chunks ahead of the state: gate prefixes,
-//                P and L from [Q; K] K^T, Q~ and K~ in place, T = (I + L)^-1 (16 x 16
-//                diagonal blocks by FP32 substitution, off-diagonal blocks by TF32 MMA),
-//                Tw = T diag(b gamma), Tu = T diag(b)
-//   warps 6-9    the state: S0^T -> BF16 copy and S^T *= gamma_C per chunk, U^T -> BF16,
-//                initial and final states
-//   warps 10-13  W^T -> shared memory, outputs to global memory
+//   warps 2-5    intra-chunk work, ahead of the state: P and L from [Q; K] K^T,
+//                T = (I + L)^-1 (16 x 16 diagonal blocks by FP32 substitution, off-diagonal
+//                blocks by TF32 MMA), then Tw = T diag(b gamma), Tu = T diag(b) in one pass;
+//                for the rules without inverse Q~ and K~ in place
+//   warps 6-9    the state: S0^T -> BF16 copy and S^T *= gamma_C per chunk, U^T -> BF16
+//                U^T and Us^T, initial and final states
+//   warps 10-13  W^T -> shared memory and Q~ in place (delta rules), outputs (staged in
+//                shared memory, written as 16-byte pieces of whole rows)
+// The per-iteration code of every role is kept compact (rolled loops): the four roles share
+// each SM sub-partition's instruction cache, and unrolled epilogues thrashed it.  A group
+// waits on an mbarrier through one polling thread; the others sleep on the group's named
+// barrier.
 // Per chunk j the issuer runs: W_j and U~_j (after the intra-chunk work of chunk j),
-// U_j -= S0^T W^T, O_j = S0^T Q~^T, then S^T += U^T K~ and O_j += U^T P^T, then [Q; K] K^T of
-// chunk j + 2; only the S pass -> U -> U epilogue -> state update chain is serial across
-// chunks.  Every wait has a time limit and a CTA-wide abort flag: a wait that gives up
+// U_j -= S0^T W^T, O_j = S0^T Q~^T, then S^T += Us^T K and O_j += U^T P^T, then [Q; K] K^T of
+// chunk j + 2.  Every wait has a time limit and a CTA-wide abort flag: a wait that gives up
 // stops every role, the issuer drains its MMAs, the loader its copies, and the kernel
 // reports LA_DEVERR_TIMEOUT.  Units (sequence, head) are dealt to the CTAs in a fixed
 // boustrophedon order over seq_order (longest first balances the load).
@@ -66,7 +72,7 @@ constexpr uint32_t kNbPrep = 1, kNbState = 2, kNbOut = 3;
 constexpr int kStageBytes = 49152;
 constexpr int kOffQK = 0;      // in a stage: two panels of 128 rows, Q rows 0..63, K rows 64..127
 constexpr int kOffV = 32768;   //             two panels of 64 rows
-constexpr int kOffWt = kStages * kStageBytes;  // W^T [128 d_k][64 t]
+constexpr int kOffWt = kStages * kStageBytes;  // W^T [128 d_k][64 t]; the outputs' staging tile
 constexpr int kOffP = kOffWt + 16384;          // P [2][64 t][64 s] (chunk parity)
 constexpr int kOffTw = kOffP + 2 * 8192;       // Tw [64 t][64 s]
 constexpr int kOffTu = kOffTw + 8192;          // Tu [64 t][64 s]
@@ -74,48 +80,50 @@ constexpr int kLs = kC + 4;                    // padded row stride of L / T (fp
 constexpr int kOffL = kOffTu + 8192;           // L, then T in place [64][68] fp32
 constexpr int kXs = 24;
 constexpr int kOffX = kOffL + kC * kLs * 4;    // [3][16][24] fp32, scratch of the block recursion
-constexpr int kOffGin = kOffX + 3 * 16 * kXs * 4;        // [kStages][2][64] fp32: g, beta as given
-constexpr int kGB = 8 * kC;                              // floats per gate block
-constexpr int kOffGB = kOffGin + kStages * 2 * kC * 4;   // [2][kGB] fp32 (chunk parity)
-// gate block: [0, 64) gamma_t, [64, 128) gamma_C / gamma_t, [128, 192) A_t = gamma_t / e^m,
-// [192, 256) B_t = e^m / gamma_t, [256, 320) log |gamma_t|, [320, 384) sign gamma_t,
-// [384, 448) b_t, [448] 1 when gamma_t / gamma_s = A_t B_s may be used
-constexpr int kOffBar = kOffGB + 2 * kGB * 4;
+// gate block of a stage (written by the loader): [0, 64) gamma_t, [64, 128) gamma_C / gamma_t,
+// [128, 192) A_t = gamma_t / e^m, [192, 256) B_t = e^m / gamma_t, [256, 320) log |gamma_t|,
+// [320, 384) sign gamma_t, [384, 448) b_t, [448] 1 when gamma_t / gamma_s = A_t B_s may be used
+constexpr int kGB = 7 * kC + 4;                         // floats per gate block
+constexpr int kOffGB = kOffX + 3 * 16 * kXs * 4;        // [kStages][kGB] fp32
+constexpr int kOffBar = kOffGB + kStages * kGB * 4;
 enum Bar {
-  kFull = 0,        // [3] stage loaded (TMA bytes + 32 lane arrivals of the gates)
+  kFull = 0,        // [3] stage loaded (TMA bytes + 32 lane arrivals of the gate block)
   kEmpty = 3,       // [3] stage free (MMA commit)
   kG1Full = 6,      // [Q; K] K^T of a chunk in tensor memory (MMA commit)
   kG1Free,          // the intra-chunk group has read it
-  kPrepDone,        // Tw, Tu, P, Q~ (and K~ for the rules without inverse) ready
+  kPrepDone,        // Tw, Tu and P ready (rules without inverse: P, Q~ and K~)
   kWFull,           // W^T and U~^T in tensor memory (MMA commit)
   kWFree,           // W^T is in shared memory
+  kQt,              // Q~ ready (delta rules)
   kSPass,           // S0^T copied to BF16 and S^T scaled by gamma_C
   kUFull,           // U^T in tensor memory (MMA commit)
-  kUDone,           // U^T copied to BF16
-  kKt,              // K~ ready (delta rules)
+  kUDone,           // U^T and Us^T copied to BF16
   kSFull,           // state update done (MMA commit)
   kOFull,           // outputs of a chunk in tensor memory (MMA commit)
   kOFree,           // outputs read
   kDrain,           // every MMA issued has completed
   kNumBars
 };
-constexpr int kOffMisc = kOffBar + kNumBars * 8;  // [0] tensor-memory base, [1] abort, [2] gate blocks done
+constexpr int kOffMisc = kOffBar + kNumBars * 8;  // [0] tensor-memory base, [1] abort
 constexpr int kSmem = kOffMisc + 16 + 1024;       // + slack for the 1024-byte alignment
 static_assert(kSmem <= 227 * 1024, "shared memory");
-static_assert(kOffWt % 1024 == 0 && kOffP % 1024 == 0 && kOffTw % 1024 == 0 && kOffL % 16 == 0, "alignment");
+static_assert(kOffWt % 1024 == 0 && kOffP % 1024 == 0 && kOffTw % 1024 == 0 && kOffL % 16 == 0 &&
+                  kOffGB % 16 == 0 && (kGB * 4) % 16 == 0 && kOffBar % 8 == 0,
+              "alignment");
 
 // bytes the TMA engine writes into a stage per chunk: Q, K, V (two 64 x 64 panels each)
 constexpr uint32_t kTmaBytes = 6 * kC * 128;
 
 // tensor-memory columns (FP32 accumulators unless noted; 128 lanes each)
 constexpr uint32_t kTmemCols = 512;
-constexpr int kColS = 0;     // S^T        [d_v][d_k]     128
-constexpr int kColSb = 128;  // S0^T BF16  [d_v][d_k / 2]  64 (A operand)
-constexpr int kColG1 = 192;  // [Q; K] K^T [128][64]       64
-constexpr int kColW = 256;   // W^T        [d_k][64]       64
-constexpr int kColU = 320;   // U^T        [d_v][64]       64
-constexpr int kColUb = 384;  // U^T BF16   [d_v][32]       32 (A operand)
-constexpr int kColO = 448;   // O^T        [d_v][64]       64
+constexpr int kColS = 0;      // S^T        [d_v][d_k]     128
+constexpr int kColSb = 128;   // S0^T BF16  [d_v][d_k / 2]  64 (A operand)
+constexpr int kColG1 = 192;   // [Q; K] K^T [128][64]       64
+constexpr int kColW = 256;    // W^T        [d_k][64]       64
+constexpr int kColU = 320;    // U^T        [d_v][64]       64
+constexpr int kColUb = 384;   // U^T BF16   [d_v][32]       32 (A operand)
+constexpr int kColUsb = 416;  // Us^T BF16  [d_v][32]       32 (A operand)
+constexpr int kColO = 448;    // O^T        [d_v][64]       64
 
 // D (tensor memory) = A (tensor memory, BF16 packed two per column) B (shared memory)
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
@@ -127,21 +135,43 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// mbarrier phase test that lets the hardware suspend the thread (up to about `hint_ns`)
+// until the phase completes, instead of returning at once
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return done != 0;
+}
+
 // A pipeline wait with a time limit and the CTA's abort flag: false when it gave up (the
-// flag is then set) or another role gave up first.
+// flag is then set) or another role gave up first.  Called by ONE thread of a group: the
+// others wait on the group's named barrier (gwait), which costs no shared-memory traffic.
 __device__ __forceinline__ bool fwait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t polls = 1;; ++polls) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((polls & 15u) == 0) {
-      if (*abort_flag) return false;
-      if (polls >= kWaitMaxPolls || global_timer_ns() - t0 > kWaitLimitNs) {
-        *abort_flag = 1u;
-        return false;
-      }
+    if (mbar_try_wait_hint(bar, parity, 200000u)) return true;
+    if (*abort_flag) return false;
+    if (polls >= kWaitMaxPolls || global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1u;
+      return false;
     }
   }
+}
+
+// The same for a warp group of 128 threads: thread 0 of the group polls, every thread leaves
+// with the same answer (true: the phase completed; false: abort).
+__device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag, int tp,
+                                      uint32_t nb) {
+  bool ok = true;
+  if (tp == 0) ok = fwait(bar, parity, abort_flag);
+  return !named_bar_or(nb, 128, !ok);
 }
 
 // One (sequence, head) unit: its tokens, slots and whether it can be processed.
@@ -194,6 +224,27 @@ __device__ __forceinline__ uint32_t pack2(uint32_t lo, uint32_t hi) {
   return pack_bf16x2(__uint_as_float(lo), __uint_as_float(hi));
 }
 
+// rows [row0, row0 + 64) of a stage's [Q; K] panel pair scaled in place, row t by f[t] (rows
+// at or past nv zeroed when zero_tail), by the 128 threads of a group (tp = 0..127):
+// Q~ = diag(gamma) Q, K~ = diag(gamma_C / gamma) K
+__device__ __forceinline__ void scale_rows(unsigned char* st, int row0, const float* f, int nv, bool zero_tail,
+                                           int tp) {
+#pragma unroll 4
+  for (int i = 0; i < 8; ++i) {
+    const int idx = tp + 128 * i;
+    const int t = idx >> 4, ch = idx & 15;
+    uint4* ptr = reinterpret_cast<uint4*>(st + umma::panel_piece(128, row0 + t, ch));
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (!zero_tail || t < nv) {
+      const uint4 v = *ptr;
+      const float ft = f[t];
+      w = make_uint4(pack_bf16x2(bf16_lo(v.x) * ft, bf16_hi(v.x) * ft), pack_bf16x2(bf16_lo(v.y) * ft, bf16_hi(v.y) * ft),
+                     pack_bf16x2(bf16_lo(v.z) * ft, bf16_hi(v.z) * ft), pack_bf16x2(bf16_lo(v.w) * ft, bf16_hi(v.w) * ft));
+    }
+    *ptr = w;
+  }
+}
+
 }  // namespace fused
 
 template <int RULE>
@@ -210,7 +261,6 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
   volatile uint32_t* abort_flag = misc + 1;
-  volatile uint32_t* gates_done = misc + 2;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -227,7 +277,6 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
     }
     for (int b = kG1Full; b < kNumBars; ++b) mbar_init(&bars[b], 1);
     misc[1] = 0u;
-    misc[2] = 0u;
     mbar_init_fence();
   }
   // the strictly upper 16 x 16 blocks of Tw and Tu stay zero in every chunk
@@ -269,17 +318,16 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
         const int s = (int)(j % kStages);
         const int tok0 = x.t0 + c * kC;
         const int nv = min(kC, x.n_tok - c * kC);
-        // the chunk's gates (raw g and beta; padded tokens: no decay, no write)
-        float ga = 1.0f, gb = 1.0f, ba = 0.0f, bb = 0.0f;
-        if (lane < nv) {
-          const int64_t gi = (int64_t)(tok0 + lane) * H + x.h;
-          ga = kGate ? __ldg(p.g + gi) : 1.0f;
-          ba = Rule<RULE>::kUsesBeta ? __ldg(p.beta + gi) : 1.0f;
-        }
-        if (lane + 32 < nv) {
-          const int64_t gi = (int64_t)(tok0 + lane + 32) * H + x.h;
-          gb = kGate ? __ldg(p.g + gi) : 1.0f;
-          bb = Rule<RULE>::kUsesBeta ? __ldg(p.beta + gi) : 1.0f;
+        // the chunk's gates: tokens 2 lane and 2 lane + 1 (padded tokens: no decay, no write)
+        float gi[2] = {1.0f, 1.0f}, bi[2] = {0.0f, 0.0f};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 2 * lane + e;
+          if (t < nv) {
+            const int64_t ix = (int64_t)(tok0 + t) * H + x.h;
+            gi[e] = kGate ? __ldg(p.g + ix) : 1.0f;
+            bi[e] = Rule<RULE>::kUsesBeta ? __ldg(p.beta + ix) : 1.0f;
+          }
         }
         if (j >= kStages && lane == 0) ok = fwait(&bars[kEmpty + s], (uint32_t)((j / kStages) + 1) & 1u, abort_flag);
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -295,12 +343,51 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
             umma::tma_load_3d(st + kOffV + pnl * 8192, &maps.v, 64 * pnl, x.h, tok0, full);
           }
         }
-        float* gin = reinterpret_cast<float*>(smem + kOffGin) + s * 2 * kC;
-        gin[lane] = ga;
-        gin[lane + 32] = gb;
-        gin[kC + lane] = ba;
-        gin[kC + lane + 32] = bb;
-        mbar_arrive(&bars[kFull + s]);
+        // gate block: prefixes of log |a| and of the sign over the chunk, the factored
+        // ratios gamma_t / gamma_s = A_t B_s around the chunk's middle (when the chunk's
+        // gates are at most 1 in magnitude and span at most e^80), b_t
+        float* gbk = reinterpret_cast<float*>(smem + kOffGB) + s * kGB;
+        float lg[2], sg[2];
+        bool big = false;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 2 * lane + e;
+          float a, bc, cc;
+          Rule<RULE>::coeffs(gi[e], bi[e], a, bc, cc);
+          if (t >= nv) bc = 0.0f;  // padded tokens write nothing
+          big |= fabsf(a) > 1.0f;
+          lg[e] = __logf(fmaxf(fabsf(a), 1e-30f));
+          sg[e] = a < 0.0f ? -1.0f : 1.0f;
+          gbk[6 * kC + t] = bc;
+        }
+        float l = lg[0] + lg[1], sgn = sg[0] * sg[1];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float lo2 = __shfl_up_sync(0xffffffffu, l, off);
+          const float so2 = __shfl_up_sync(0xffffffffu, sgn, off);
+          if (lane >= off) {
+            l += lo2;
+            sgn *= so2;
+          }
+        }
+        const float lprev = l - (lg[0] + lg[1]), sprev = sgn * sg[0] * sg[1];
+        const float lv[2] = {lprev + lg[0], l}, sv[2] = {sprev * sg[0], sgn};
+        const float lfirst = __shfl_sync(0xffffffffu, lv[0], 0), llast = __shfl_sync(0xffffffffu, l, 31);
+        const float slast = __shfl_sync(0xffffffffu, sgn, 31);
+        const bool fact = !__any_sync(0xffffffffu, big) && (lfirst - llast) <= 80.0f;
+        const float m = 0.5f * (lfirst + llast);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 2 * lane + e;
+          gbk[t] = sv[e] * __expf(lv[e]);
+          gbk[kC + t] = slast * sv[e] * __expf(llast - lv[e]);
+          gbk[2 * kC + t] = sv[e] * __expf(lv[e] - m);
+          gbk[3 * kC + t] = sv[e] * __expf(m - lv[e]);
+          gbk[4 * kC + t] = lv[e];
+          gbk[5 * kC + t] = sv[e];
+        }
+        if (lane == 0) gbk[7 * kC] = fact ? 1.0f : 0.0f;
+        mbar_arrive(&bars[kFull + s]);  // release: this lane's gate-block writes
       }
     }
     // copies still in flight (after an abort): let them land, within the limit
@@ -311,12 +398,12 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdKK64 = umma::idesc_bf16(128, 64, false, false);      // A, B K-major
-      constexpr uint32_t kIdMK64 = umma::idesc_bf16(128, 64, true, false);       // A MN-major
+      constexpr uint32_t kIdKK64 = umma::idesc_bf16(128, 64, false, false);        // A, B K-major
+      constexpr uint32_t kIdMK64 = umma::idesc_bf16(128, 64, true, false);         // A MN-major
       constexpr uint32_t kIdTM64n = umma::idesc_bf16(128, 64, false, true, true);  // A tmem, B MN, -A
-      constexpr uint32_t kIdTK64 = umma::idesc_bf16(128, 64, false, false);      // A tmem, B K-major
-      constexpr uint32_t kIdTM128 = umma::idesc_bf16(128, 128, false, true);     // A tmem, B MN-major
-      constexpr uint32_t kIdMM128 = umma::idesc_bf16(128, 128, true, true);      // A, B MN-major
+      constexpr uint32_t kIdTK64 = umma::idesc_bf16(128, 64, false, false);        // A tmem, B K-major
+      constexpr uint32_t kIdTM128 = umma::idesc_bf16(128, 128, false, true);       // A tmem, B MN-major
+      constexpr uint32_t kIdMM128 = umma::idesc_bf16(128, 128, true, true);        // A, B MN-major
       const uint64_t dTw = umma::sdesc(sb + kOffTw, 16, 1024);
       const uint64_t dTu = umma::sdesc(sb + kOffTu, 16, 1024);
       const uint64_t dWm = umma::sdesc(sb + kOffWt, 16384, 1024);
@@ -343,9 +430,9 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
       }
       for (int64_t j = 0; ok && j < n_total; ++j) {
         const uint32_t st = sb + (uint32_t)(j % kStages) * kStageBytes;
-        const uint64_t dQK = umma::sdesc(st + kOffQK, 16, 1024);       // [Q~; K] rows, K-major
-        const uint64_t dKm = umma::sdesc(st + kOffQK + 8192, 16384, 1024);  // K (K~) as MN-major
-        const uint64_t dVm = umma::sdesc(st + kOffV, 8192, 1024);      // V as MN-major
+        const uint64_t dQK = umma::sdesc(st + kOffQK, 16, 1024);            // [Q~; K] rows, K-major
+        const uint64_t dKm = umma::sdesc(st + kOffQK + 8192, 16384, 1024);  // K (or K~) as MN-major
+        const uint64_t dVm = umma::sdesc(st + kOffV, 8192, 1024);           // V as MN-major
         const uint64_t dP = umma::sdesc(sb + kOffP + (uint32_t)(j & 1) * 8192, 16, 1024);
         if (kDelta) {
           if (!(ok = W(kPrepDone, j))) break;
@@ -363,9 +450,9 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
           for (int kk = 0; kk < 8; ++kk)  // U^T -= S0^T W^T (K = d_k)
             mma_ts(tmem + kColU, tmem + kColSb + 8 * kk, umma::sdesc_add(dWm, kk * 2048), kIdTM64n, 1);
           umma::commit(&bars[kUFull]);
+          if (!(ok = W(kQt, j))) break;
         } else {
           if (!(ok = W(kPrepDone, j) && W(kSPass, j))) break;
-          umma::fence_after();
         }
         if (j > 0 && !(ok = W(kOFree, j - 1))) break;
         umma::fence_after();
@@ -375,11 +462,11 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
           mma_ts(tmem + kColO, tmem + kColSb + 8 * kk, umma::sdesc_add(dQK, ko), kIdTK64, kk);
         }
         if (kDelta) {
-          if (!(ok = W(kUDone, j) && W(kKt, j))) break;
+          if (!(ok = W(kUDone, j))) break;
           umma::fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // S^T += U^T K~ (K = tokens)
-            mma_ts(tmem + kColS, tmem + kColUb + 8 * kk, umma::sdesc_add(dKm, kk * 2048), kIdTM128, 1);
+          for (int kk = 0; kk < 4; ++kk)  // S^T += Us^T K (K = tokens)
+            mma_ts(tmem + kColS, tmem + kColUsb + 8 * kk, umma::sdesc_add(dKm, kk * 2048), kIdTM128, 1);
           umma::commit(&bars[kSFull]);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)  // O^T += U^T P^T
@@ -407,39 +494,15 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
     }
   } else if (warp < kWarpState) {
     // ------------------------------------------------------------------ intra-chunk group
-    const int wi = warp - kWarpPrep;               // 0..3 within the group
-    const int tp = tid - kWarpPrep * 32;           // 0..127
+    const int wi = warp - kWarpPrep;      // 0..3 within the group
+    const int tp = tid - kWarpPrep * 32;  // 0..127
     const int q4 = warp & 3;
-    const int r = 32 * q4 + lane;                  // this thread's tensor-memory lane
+    const int r = 32 * q4 + lane;         // this thread's tensor-memory lane
     const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
     float* sL = reinterpret_cast<float*>(smem + kOffL);
     float* sX = reinterpret_cast<float*>(smem + kOffX);
     int64_t j = 0;
-    int prev_nv = 0;
     bool ok = true;
-
-    // K~ = diag(gamma_C / gamma) K in place (rows beyond the chunk's tokens zeroed)
-    auto ktilde = [&](int64_t jj, int nv) {
-      unsigned char* st = smem + (uint32_t)(jj % kStages) * kStageBytes + kOffQK;
-      const float* gcg = reinterpret_cast<const float*>(smem + kOffGB) + (jj & 1) * kGB + kC;
-#pragma unroll 2
-      for (int i = 0; i < 8; ++i) {
-        const int idx = tp + 128 * i;
-        const int t = idx >> 4, ch = idx & 15;
-        uint4* ptr = reinterpret_cast<uint4*>(st + umma::panel_piece(128, kC + t, ch));
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (t < nv) {
-          const uint4 v = *ptr;
-          const float f = gcg[t];
-          w.x = pack_bf16x2(bf16_lo(v.x) * f, bf16_hi(v.x) * f);
-          w.y = pack_bf16x2(bf16_lo(v.y) * f, bf16_hi(v.y) * f);
-          w.z = pack_bf16x2(bf16_lo(v.z) * f, bf16_hi(v.z) * f);
-          w.w = pack_bf16x2(bf16_lo(v.w) * f, bf16_hi(v.w) * f);
-        }
-        *ptr = w;
-      }
-    };
-
     for (int64_t ru = 0; ok && ru * G < units; ++ru) {
       const int64_t u = unit_of(ru, G, blockIdx.x);
       if (u >= units) continue;
@@ -449,74 +512,14 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
       for (int c = 0; c < nch; ++c, ++j) {
         const int s = (int)(j % kStages);
         const int nv = min(kC, x.n_tok - c * kC);
-        float* gbk = reinterpret_cast<float*>(smem + kOffGB) + (j & 1) * kGB;
-        if (j > 0) {
-          // delta rules: K~ of the previous chunk once W_{j-1} (and U~_{j-1}) have read K
-          // and Tw, Tu; the other rules: the previous state update has been issued
-          ok = fwait(&bars[kDelta ? kWFull : kSFull], (uint32_t)(j - 1) & 1u, abort_flag);
-          if (named_bar_or(kNbPrep, 128, !ok)) {
-            ok = false;
-            break;
-          }
-          if (kDelta) {
-            ktilde(j - 1, prev_nv);
-            umma::fence_smem();
-            named_bar_sync(kNbPrep, 128);
-            if (tp == 0) mbar_arrive(&bars[kKt]);
-          }
-        }
-        ok = fwait(&bars[kFull + s], (uint32_t)(j / kStages) & 1u, abort_flag);
-        if (named_bar_or(kNbPrep, 128, !ok)) {
-          ok = false;
-          break;
-        }
-        // gate block (warp wi == 0): prefixes of log |a| and of the sign over the chunk
-        if (wi == 0) {
-          const float* gin = reinterpret_cast<const float*>(smem + kOffGin) + s * 2 * kC;
-          float lg[2], sg[2];
-          bool big = false;
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int t = 2 * lane + e;
-            float a, bc, cc;
-            Rule<RULE>::coeffs(gin[t], gin[kC + t], a, bc, cc);
-            if (t >= nv) bc = 0.0f;  // padded tokens write nothing
-            big |= fabsf(a) > 1.0f;
-            lg[e] = __logf(fmaxf(fabsf(a), 1e-30f));
-            sg[e] = a < 0.0f ? -1.0f : 1.0f;
-            gbk[6 * kC + t] = bc;
-          }
-          float l = lg[0] + lg[1], sgn = sg[0] * sg[1];
-#pragma unroll
-          for (int off = 1; off < 32; off <<= 1) {
-            const float lo2 = __shfl_up_sync(0xffffffffu, l, off);
-            const float so2 = __shfl_up_sync(0xffffffffu, sgn, off);
-            if (lane >= off) {
-              l += lo2;
-              sgn *= so2;
-            }
-          }
-          const float lprev = l - (lg[0] + lg[1]), sprev = sgn * sg[0] * sg[1];
-          const float lv[2] = {lprev + lg[0], l}, sv[2] = {sprev * sg[0], sgn};
-          const float lfirst = __shfl_sync(0xffffffffu, lv[0], 0), llast = __shfl_sync(0xffffffffu, l, 31);
-          const float slast = __shfl_sync(0xffffffffu, sgn, 31);
-          const bool fact = !__any_sync(0xffffffffu, big) && (lfirst - llast) <= 80.0f;
-          const float m = 0.5f * (lfirst + llast);
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int t = 2 * lane + e;
-            gbk[t] = sv[e] * __expf(lv[e]);
-            gbk[kC + t] = slast * sv[e] * __expf(llast - lv[e]);
-            gbk[2 * kC + t] = sv[e] * __expf(lv[e] - m);
-            gbk[3 * kC + t] = sv[e] * __expf(m - lv[e]);
-            gbk[4 * kC + t] = lv[e];
-            gbk[5 * kC + t] = sv[e];
-          }
-          if (lane == 0) gbk[7 * kC] = fact ? 1.0f : 0.0f;
-          __threadfence_block();
-        }
-        named_bar_sync(kNbPrep, 128);
-        if (tp == 0) *gates_done = (uint32_t)(j + 1);  // the state group reads gamma_C from here
+        unsigned char* st = smem + s * kStageBytes + kOffQK;
+        const float* gbk = reinterpret_cast<const float*>(smem + kOffGB) + s * kGB;
+        // rules without inverse: stay behind the state update of chunk j - 1 (the MMA issuer
+        // then never falls two phases behind this group's completions)
+        if (!kDelta && j > 0 && !(ok = gwait(&bars[kSFull], (uint32_t)(j - 1) & 1u, abort_flag, tp, kNbPrep))) break;
+        // the stage (and its gate block), then [Q; K] K^T of the chunk
+        if (!(ok = gwait(&bars[kFull + s], (uint32_t)(j / kStages) & 1u, abort_flag, tp, kNbPrep))) break;
+        if (!(ok = gwait(&bars[kG1Full], (uint32_t)j & 1u, abort_flag, tp, kNbPrep))) break;
         const bool fact = gbk[7 * kC] != 0.0f;
         const float* sFa = gbk + 2 * kC;
         const float* sFb = gbk + 3 * kC;
@@ -525,110 +528,100 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
         const float* sBt = gbk + 6 * kC;
 
         // P = (Q K^T) (.) M (lanes 0..63) and L (lanes 64..127, delta rules) from tensor memory
-        ok = fwait(&bars[kG1Full], (uint32_t)j & 1u, abort_flag);
-        if (named_bar_or(kNbPrep, 128, !ok)) {
-          ok = false;
-          break;
-        }
         umma::fence_after();
-        if (r < kC) {
-          const int t = r;
+        if (r < kC || kDelta) {
+          // row t of P (lanes 0..63: masked by gamma_t / gamma_s, s <= t) or of L (lanes
+          // 64..127: b_t gamma_t / gamma_s k_t . k_s, s < t), 32 columns at a time
+          const bool is_p = r < kC;
+          const int t = is_p ? r : r - kC;
+          const float bt = is_p ? 1.0f : sBt[t];
+          const float fa = sFa[t] * bt, sgt = sSg[t] * bt, lgt = sLg[t];
           unsigned char* sP = smem + kOffP + (j & 1) * 8192;
+#pragma unroll 1
+          for (int c32 = 0; c32 < 2; ++c32) {
+            uint32_t v[32];
+            umma::ld16(tq + kColG1 + 32 * c32, v);
+            umma::ld16(tq + kColG1 + 32 * c32 + 16, v + 16);
+            float rt[32];  // the ratios b_t gamma_t / gamma_s of the 32 columns
+            if (fact) {
 #pragma unroll
-          for (int c16 = 0; c16 < 4; ++c16) {
-            uint32_t v[16];
-            umma::ld16(tq + kColG1 + 16 * c16, v);
-            umma::wait_ld();
+              for (int q = 0; q < 8; ++q) {
+                const float4 fb = *reinterpret_cast<const float4*>(sFb + 32 * c32 + 4 * q);
+                rt[4 * q] = fa * fb.x;
+                rt[4 * q + 1] = fa * fb.y;
+                rt[4 * q + 2] = fa * fb.z;
+                rt[4 * q + 3] = fa * fb.w;
+              }
+            } else {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int s_ = 16 * c16 + e;
-              float y = 0.0f;
-              if (s_ <= t)
-                y = (fact ? sFa[t] * sFb[s_] : sSg[t] * sSg[s_] * __expf(sLg[t] - sLg[s_])) * __uint_as_float(v[e]);
-              v[e] = __float_as_uint(y);
+              for (int q = 0; q < 8; ++q) {
+                const float4 lg4 = *reinterpret_cast<const float4*>(sLg + 32 * c32 + 4 * q);
+                const float4 sg4 = *reinterpret_cast<const float4*>(sSg + 32 * c32 + 4 * q);
+                rt[4 * q] = sgt * sg4.x * __expf(lgt - lg4.x);
+                rt[4 * q + 1] = sgt * sg4.y * __expf(lgt - lg4.y);
+                rt[4 * q + 2] = sgt * sg4.z * __expf(lgt - lg4.z);
+                rt[4 * q + 3] = sgt * sg4.w * __expf(lgt - lg4.w);
+              }
             }
-#pragma unroll
-            for (int pc = 0; pc < 2; ++pc)
-              *reinterpret_cast<uint4*>(sP + umma::panel_piece(kC, t, 2 * c16 + pc)) =
-                  make_uint4(pack2(v[8 * pc], v[8 * pc + 1]), pack2(v[8 * pc + 2], v[8 * pc + 3]),
-                             pack2(v[8 * pc + 4], v[8 * pc + 5]), pack2(v[8 * pc + 6], v[8 * pc + 7]));
-          }
-        } else if (kDelta) {
-          const int t = r - kC;
-#pragma unroll
-          for (int c16 = 0; c16 < 4; ++c16) {
-            uint32_t v[16];
-            umma::ld16(tq + kColG1 + 16 * c16, v);
             umma::wait_ld();
-            float y[16];
+            // the masked entries: s <= t for P, s < t for L
+            const int lim = is_p ? t - 32 * c32 : t - 32 * c32 - 1;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int s_ = 16 * c16 + e;
-              y[e] = 0.0f;
-              if (s_ < t)
-                y[e] = sBt[t] * (fact ? sFa[t] * sFb[s_] : sSg[t] * sSg[s_] * __expf(sLg[t] - sLg[s_])) *
-                       __uint_as_float(v[e]);
+            for (int e = 0; e < 32; ++e) rt[e] = e <= lim ? rt[e] * __uint_as_float(v[e]) : 0.0f;
+            if (is_p) {
+#pragma unroll
+              for (int pc = 0; pc < 4; ++pc)
+                *reinterpret_cast<uint4*>(sP + umma::panel_piece(kC, t, 4 * c32 + pc)) =
+                    make_uint4(pack_bf16x2(rt[8 * pc], rt[8 * pc + 1]), pack_bf16x2(rt[8 * pc + 2], rt[8 * pc + 3]),
+                               pack_bf16x2(rt[8 * pc + 4], rt[8 * pc + 5]),
+                               pack_bf16x2(rt[8 * pc + 6], rt[8 * pc + 7]));
+            } else {
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<float4*>(sL + t * kLs + 32 * c32 + 4 * q) =
+                    make_float4(rt[4 * q], rt[4 * q + 1], rt[4 * q + 2], rt[4 * q + 3]);
             }
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              *reinterpret_cast<float4*>(sL + t * kLs + 16 * c16 + 4 * q) =
-                  make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
           }
         }
         umma::fence_before();
         named_bar_sync(kNbPrep, 128);
         if (tp == 0) mbar_arrive(&bars[kG1Free]);
 
-        // Q~ = diag(gamma) Q in place
-        {
-          unsigned char* st = smem + s * kStageBytes + kOffQK;
-#pragma unroll 2
-          for (int i = 0; i < 8; ++i) {
-            const int idx = tp + 128 * i;
-            const int t = idx >> 4, ch = idx & 15;
-            uint4* ptr = reinterpret_cast<uint4*>(st + umma::panel_piece(128, t, ch));
-            const uint4 v = *ptr;
-            const float f = gbk[t];
-            *ptr = make_uint4(pack_bf16x2(bf16_lo(v.x) * f, bf16_hi(v.x) * f),
-                              pack_bf16x2(bf16_lo(v.y) * f, bf16_hi(v.y) * f),
-                              pack_bf16x2(bf16_lo(v.z) * f, bf16_hi(v.z) * f),
-                              pack_bf16x2(bf16_lo(v.w) * f, bf16_hi(v.w) * f));
-          }
-        }
-
-        if (kDelta) {
-          // T = (I + L)^-1 in place of L, by 16 x 16 blocks; Tw = T diag(b gamma), Tu = T diag(b)
-          const float* sGm = gbk;
-          auto put2 = [&](int row, int col, float v0, float v1) {
-            const uint32_t off = umma::panel_off(kC, row, col);
-            *reinterpret_cast<uint32_t*>(smem + kOffTw + off) =
-                pack_bf16x2(v0 * sBt[col] * sGm[col], v1 * sBt[col + 1] * sGm[col + 1]);
-            *reinterpret_cast<uint32_t*>(smem + kOffTu + off) = pack_bf16x2(v0 * sBt[col], v1 * sBt[col + 1]);
-          };
+        if (!kDelta) {
+          scale_rows(st, 0, gbk, nv, false, tp);        // Q~ = diag(gamma) Q
+          scale_rows(st, kC, gbk + kC, nv, true, tp);   // K~ (its only reader left is the state update)
+        } else {
+          // T = (I + L)^-1 in place of L, by 16 x 16 blocks.  Diagonal block wi by forward
+          // substitution, lane c (and c + 16) owning column c; L's upper triangle is zero and
+          // the column starts at zero, so full 16-term rows are exact.
           {
-            // diagonal block wi by forward substitution: lane c < 16 owns column c
             const int b0 = 16 * wi, cc = lane & 15;
-            float col[16];
+            float xc[16];
 #pragma unroll
+            for (int q = 0; q < 16; ++q) xc[q] = 0.0f;
+            const float4* lr = reinterpret_cast<const float4*>(sL + b0 * kLs + b0);
+            float4 l0 = lr[0], l1 = lr[1], l2 = lr[2], l3 = lr[3];
+#pragma unroll 1
             for (int rr = 0; rr < 16; ++rr) {
-              const float4* lr = reinterpret_cast<const float4*>(sL + (b0 + rr) * kLs + b0);
-              float xv = (rr == cc) ? 1.0f : 0.0f;
+              // the next row's L while this row's sums run
+              const float4* ln = reinterpret_cast<const float4*>(sL + (b0 + (rr < 15 ? rr + 1 : rr)) * kLs + b0);
+              const float4 n0 = ln[0], n1 = ln[1], n2 = ln[2], n3 = ln[3];
+              const float a0 = fmaf(l0.x, xc[0], fmaf(l0.y, xc[1], fmaf(l0.z, xc[2], l0.w * xc[3])));
+              const float a1 = fmaf(l1.x, xc[4], fmaf(l1.y, xc[5], fmaf(l1.z, xc[6], l1.w * xc[7])));
+              const float a2 = fmaf(l2.x, xc[8], fmaf(l2.y, xc[9], fmaf(l2.z, xc[10], l2.w * xc[11])));
+              const float a3 = fmaf(l3.x, xc[12], fmaf(l3.y, xc[13], fmaf(l3.z, xc[14], l3.w * xc[15])));
+              const float xv = (rr == cc ? 1.0f : 0.0f) - ((a0 + a1) + (a2 + a3));
 #pragma unroll
-              for (int m4 = 0; m4 < (rr + 3) / 4; ++m4) {
-                const float4 l4 = lr[m4];
-                const float lv4[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  if (4 * m4 + e < rr) xv -= lv4[e] * col[4 * m4 + e];
-              }
-              col[rr] = (rr < cc) ? 0.0f : xv;
+              for (int q = 0; q < 16; ++q) xc[q] = (q == rr) ? xv : xc[q];
+              l0 = n0;
+              l1 = n1;
+              l2 = n2;
+              l3 = n3;
             }
             __syncwarp();
+            if (lane < 16) {
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) {
-              if (lane < 16) sL[(b0 + rr) * kLs + b0 + cc] = col[rr];
-              const float nxt = __shfl_down_sync(0xffffffffu, col[rr], 1);
-              if (lane < 16 && (cc & 1) == 0) put2(b0 + rr, b0 + cc, col[rr], nxt);
+              for (int rr = 0; rr < 16; ++rr) sL[(b0 + rr) * kLs + b0 + cc] = xc[rr];
             }
           }
           named_bar_sync(kNbPrep, 128);
@@ -640,16 +633,15 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
               const int bj = wi;
               const int g8 = lane >> 2, t4 = lane & 3;
               float xs[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll 1
               for (int bk = bj; bk < bi; ++bk)
                 chunk::mma16x16x16_tf32(xs, sL + (16 * bi) * kLs + 16 * bk, kLs, sL + (16 * bk) * kLs + 16 * bj,
                                         kLs, lane);
               float* xw = sX + wi * 16 * kXs;
 #pragma unroll
               for (int nt = 0; nt < 2; ++nt) {
-                xw[g8 * kXs + 8 * nt + 2 * t4] = xs[nt][0];
-                xw[g8 * kXs + 8 * nt + 2 * t4 + 1] = xs[nt][1];
-                xw[(g8 + 8) * kXs + 8 * nt + 2 * t4] = xs[nt][2];
-                xw[(g8 + 8) * kXs + 8 * nt + 2 * t4 + 1] = xs[nt][3];
+                *reinterpret_cast<float2*>(xw + g8 * kXs + 8 * nt + 2 * t4) = make_float2(xs[nt][0], xs[nt][1]);
+                *reinterpret_cast<float2*>(xw + (g8 + 8) * kXs + 8 * nt + 2 * t4) = make_float2(xs[nt][2], xs[nt][3]);
               }
               __syncwarp();
               chunk::mma16x16x16_tf32(y, sL + (16 * bi) * kLs + 16 * bi, kLs, xw, kXs, lane);
@@ -660,35 +652,35 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
               const int g8 = lane >> 2, t4 = lane & 3;
 #pragma unroll
               for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-                for (int hlf = 0; hlf < 2; ++hlf) {
-                  const int row = 16 * bi + g8 + 8 * hlf, col = 16 * bj + 8 * nt + 2 * t4;
-                  const float v0 = -y[nt][2 * hlf], v1 = -y[nt][2 * hlf + 1];
-                  sL[row * kLs + col] = v0;
-                  sL[row * kLs + col + 1] = v1;
-                  put2(row, col, v0, v1);
-                }
+                const int col = 16 * bj + 8 * nt + 2 * t4;
+                *reinterpret_cast<float2*>(sL + (16 * bi + g8) * kLs + col) = make_float2(-y[nt][0], -y[nt][1]);
+                *reinterpret_cast<float2*>(sL + (16 * bi + g8 + 8) * kLs + col) = make_float2(-y[nt][2], -y[nt][3]);
               }
             }
             named_bar_sync(kNbPrep, 128);
           }
-        } else {
-          ktilde(j, nv);  // G1 of this chunk has read K
+          // Tw and Tu of chunk j - 1 must have been read (W_{j-1} and U~_{j-1} complete)
+          if (j > 0 && !(ok = gwait(&bars[kWFull], (uint32_t)(j - 1) & 1u, abort_flag, tp, kNbPrep))) break;
+          // Tw = T diag(b gamma), Tu = T diag(b) (BF16), the ten lower 16 x 16 blocks: block i
+          // of (0,0) (1,0) (1,1) (2,0) ... (3,3), thread tp -> row tp / 8, columns 2 (tp % 8) + {0, 1}
+          const float* sGm = gbk;
+          const int rb = tp >> 3, cp = 2 * (tp & 7);
+#pragma unroll 2
+          for (int i = 0; i < 10; ++i) {
+            const int bi = i >= 6 ? 3 : i >= 3 ? 2 : i >= 1 ? 1 : 0;
+            const int bj = i - (bi * (bi + 1)) / 2;
+            const int row = 16 * bi + rb, col = 16 * bj + cp;
+            const float2 tv = *reinterpret_cast<const float2*>(sL + row * kLs + col);
+            const float b0 = sBt[col], b1 = sBt[col + 1];
+            const uint32_t off = umma::panel_off(kC, row, col);
+            *reinterpret_cast<uint32_t*>(smem + kOffTw + off) =
+                pack_bf16x2(tv.x * b0 * sGm[col], tv.y * b1 * sGm[col + 1]);
+            *reinterpret_cast<uint32_t*>(smem + kOffTu + off) = pack_bf16x2(tv.x * b0, tv.y * b1);
+          }
         }
-        umma::fence_smem();  // P, Q~, Tw, Tu (K~) -> tensor cores
+        umma::fence_smem();  // P, Tw, Tu (Q~, K~) -> tensor cores
         named_bar_sync(kNbPrep, 128);
         if (tp == 0) mbar_arrive(&bars[kPrepDone]);
-        prev_nv = nv;
-      }
-    }
-    if (kDelta && ok && j > 0) {
-      // K~ of the last chunk
-      ok = fwait(&bars[kWFull], (uint32_t)(j - 1) & 1u, abort_flag);
-      if (!named_bar_or(kNbPrep, 128, !ok)) {
-        ktilde(j - 1, prev_nv);
-        umma::fence_smem();
-        named_bar_sync(kNbPrep, 128);
-        if (tp == 0) mbar_arrive(&bars[kKt]);
       }
     }
   } else if (warp < kWarpOut) {
@@ -741,26 +733,20 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
       }
       umma::wait_st();
       for (int c = 0; c < nch; ++c, ++j) {
-        if (c > 0) ok = fwait(&bars[kSFull], (uint32_t)(j - 1) & 1u, abort_flag);
-        // the chunk's gate block (gamma_C), published by the intra-chunk group
-        if (ok) {
-          const uint64_t t0 = global_timer_ns();
-          uint32_t polls = 0;
-          while (*gates_done <= (uint32_t)j) {
-            if ((++polls & 15u) == 0 && (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs)) {
-              *abort_flag = 1u;
-              ok = false;
-              break;
-            }
-          }
-          __threadfence_block();
+        const int s = (int)(j % kStages);
+        const float* gbk = reinterpret_cast<const float*>(smem + kOffGB) + s * kGB;
+        // the previous chunk's state update and this chunk's gate block (the stage is not
+        // reloaded before this chunk's last MMA, which waits for this group)
+        if (tp == 0) {
+          if (c > 0) ok = fwait(&bars[kSFull], (uint32_t)(j - 1) & 1u, abort_flag);
+          if (ok) ok = fwait(&bars[kFull + s], (uint32_t)(j / kStages) & 1u, abort_flag);
         }
         if (named_bar_or(kNbState, 128, !ok)) {
           ok = false;
           break;
         }
         umma::fence_after();
-        const float gC = (reinterpret_cast<const float*>(smem + kOffGB) + (j & 1) * kGB)[kC - 1];
+        const float gC = gbk[kC - 1];  // gamma_C (padded tokens have gate 1: the last real token's)
         // S pass: S0^T -> BF16 (the A operand of this chunk's products), S^T *= gamma_C
 #pragma unroll 1
         for (int c32 = 0; c32 < 4; ++c32) {
@@ -789,13 +775,11 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
         named_bar_sync(kNbState, 128);
         if (tp == 0) mbar_arrive(&bars[kSPass]);
         if (kDelta) {
-          ok = fwait(&bars[kUFull], (uint32_t)j & 1u, abort_flag);
-          if (named_bar_or(kNbState, 128, !ok)) {
-            ok = false;
-            break;
-          }
+          if (!(ok = gwait(&bars[kUFull], (uint32_t)j & 1u, abort_flag, tp, kNbState))) break;
           umma::fence_after();
-#pragma unroll
+          // U^T -> BF16 (the A operand of O += U^T P^T) and Us^T = U^T diag(gamma_C / gamma) (the
+          // A operand of the state update)
+#pragma unroll 1
           for (int c32 = 0; c32 < 2; ++c32) {
             uint32_t a[16], b[16], w[16];
             umma::ld16(tq + kColU + 32 * c32, a);
@@ -807,6 +791,14 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
               w[8 + e] = pack2(b[2 * e], b[2 * e + 1]);
             }
             umma::st16(tq + kColUb + 16 * c32, w);
+            const float* gcg = gbk + kC + 32 * c32;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              w[e] = pack_bf16x2(__uint_as_float(a[2 * e]) * gcg[2 * e], __uint_as_float(a[2 * e + 1]) * gcg[2 * e + 1]);
+              w[8 + e] = pack_bf16x2(__uint_as_float(b[2 * e]) * gcg[16 + 2 * e],
+                                     __uint_as_float(b[2 * e + 1]) * gcg[16 + 2 * e + 1]);
+            }
+            umma::st16(tq + kColUsb + 16 * c32, w);
           }
           umma::wait_st();
           umma::fence_before();
@@ -816,11 +808,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
       }
       if (!ok) break;
       // final state S[i][r] = S^T[r][i]
-      ok = fwait(&bars[kSFull], (uint32_t)(j - 1) & 1u, abort_flag);
-      if (named_bar_or(kNbState, 128, !ok)) {
-        ok = false;
-        break;
-      }
+      if (!(ok = gwait(&bars[kSFull], (uint32_t)(j - 1) & 1u, abort_flag, tp, kNbState))) break;
       umma::fence_after();
 #pragma unroll 1
       for (int c16 = 0; c16 < 8; ++c16) {
@@ -845,6 +833,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
     const int r = 32 * q4 + lane;  // d_k index (W^T) / d_v index (O^T)
     const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
     __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.o);
+    __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(smem + kOffWt);
     int64_t j = 0;
     bool ok = true;
     for (int64_t ru = 0; ok && ru * G < units; ++ru) {
@@ -854,22 +843,20 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
       if (!x.valid) continue;
       const int nch = (x.n_tok + kC - 1) / kC;
       for (int c = 0; c < nch; ++c, ++j) {
+        const int s = (int)(j % kStages);
         if (kDelta) {
           // W^T rows (lane = d_k index) -> shared memory, the B operand of the U update
-          ok = fwait(&bars[kWFull], (uint32_t)j & 1u, abort_flag);
-          if (named_bar_or(kNbOut, 128, !ok)) {
-            ok = false;
-            break;
-          }
+          if (!(ok = gwait(&bars[kWFull], (uint32_t)j & 1u, abort_flag, tp, kNbOut))) break;
           umma::fence_after();
-#pragma unroll
-          for (int c16 = 0; c16 < 4; ++c16) {
-            uint32_t v[16];
-            umma::ld16(tq + kColW + 16 * c16, v);
+#pragma unroll 1
+          for (int c32 = 0; c32 < 2; ++c32) {
+            uint32_t v[32];
+            umma::ld16(tq + kColW + 32 * c32, v);
+            umma::ld16(tq + kColW + 32 * c32 + 16, v + 16);
             umma::wait_ld();
 #pragma unroll
-            for (int pc = 0; pc < 2; ++pc)
-              *reinterpret_cast<uint4*>(smem + kOffWt + umma::panel_piece(128, r, 2 * c16 + pc)) =
+            for (int pc = 0; pc < 4; ++pc)
+              *reinterpret_cast<uint4*>(smem + kOffWt + umma::panel_piece(128, r, 4 * c32 + pc)) =
                   make_uint4(pack2(v[8 * pc], v[8 * pc + 1]), pack2(v[8 * pc + 2], v[8 * pc + 3]),
                              pack2(v[8 * pc + 4], v[8 * pc + 5]), pack2(v[8 * pc + 6], v[8 * pc + 7]));
           }
@@ -877,31 +864,44 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
           umma::fence_before();
           named_bar_sync(kNbOut, 128);
           if (tp == 0) mbar_arrive(&bars[kWFree]);
+          // Q~ = diag(gamma) Q in place: [Q; K] K^T, the last reader of Q, completed before W
+          // (the gate block of the stage landed with it)
+          if (!(ok = gwait(&bars[kFull + s], (uint32_t)(j / kStages) & 1u, abort_flag, tp, kNbOut))) break;
+          scale_rows(smem + s * kStageBytes + kOffQK, 0, reinterpret_cast<const float*>(smem + kOffGB) + s * kGB,
+                     kC, false, tp);
+          umma::fence_smem();
+          named_bar_sync(kNbOut, 128);
+          if (tp == 0) mbar_arrive(&bars[kQt]);
         }
-        // outputs o_t[r] = scale O^T[r][t] for the chunk's tokens
-        ok = fwait(&bars[kOFull], (uint32_t)j & 1u, abort_flag);
-        if (named_bar_or(kNbOut, 128, !ok)) {
-          ok = false;
-          break;
-        }
+        // outputs o_t[r] = scale O^T[r][t] for the chunk's tokens: staged as a row-major
+        // [64][128] BF16 tile in the W^T buffer (free: U_j, its reader, has completed), then
+        // written as 16-byte pieces of whole 256-byte rows
+        if (!(ok = gwait(&bars[kOFull], (uint32_t)j & 1u, abort_flag, tp, kNbOut))) break;
         umma::fence_after();
-        const int tok0 = x.t0 + c * kC;
-        const int nv = min(kC, x.n_tok - c * kC);
-        __nv_bfloat16* orow = og + ((int64_t)tok0 * H + x.h) * kD + r;
-#pragma unroll
+#pragma unroll 1
         for (int c16 = 0; c16 < 4; ++c16) {
           uint32_t v[16];
           umma::ld16(tq + kColO + 16 * c16, v);
           umma::wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int t = 16 * c16 + e;
-            if (t < nv) orow[(int64_t)t * H * kD] = __float2bfloat16_rn(p.scale * __uint_as_float(v[e]));
-          }
+          for (int e = 0; e < 16; ++e) so[(16 * c16 + e) * kD + r] = __float2bfloat16_rn(p.scale * __uint_as_float(v[e]));
         }
         umma::fence_before();
         named_bar_sync(kNbOut, 128);
         if (tp == 0) mbar_arrive(&bars[kOFree]);
+        {
+          const int tok0 = x.t0 + c * kC;
+          const int nv = min(kC, x.n_tok - c * kC);
+#pragma unroll 2
+          for (int i = 0; i < 8; ++i) {
+            const int idx = tp + 128 * i;
+            const int t = idx >> 4, ch = idx & 15;
+            if (t < nv)
+              *reinterpret_cast<uint4*>(og + ((int64_t)(tok0 + t) * H + x.h) * kD + ch * 8) =
+                  *reinterpret_cast<const uint4*>(so + t * kD + ch * 8);
+          }
+        }
+        named_bar_sync(kNbOut, 128);  // the staging tile is read before the next W^T lands there
       }
     }
   }
@@ -910,6 +910,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
   umma::fence_before();
   __syncthreads();
   if (warp == kWarpMma) {
+    __syncwarp();
     umma::fence_after();
     umma::dealloc(tmem, kTmemCols);
   }
