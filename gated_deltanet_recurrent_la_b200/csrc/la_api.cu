@@ -12,12 +12,17 @@
 
 #include "la_internal.h"
 #include "la_state.h"
+#include "la_device.cuh"
 
 namespace la {
 
 namespace {
 
 thread_local int32_t g_last_cuda_error = 0;
+// failure-path test hooks (la_debug_*): the wait limit of the decode step's pipeline waits,
+// and a one-shot request to withhold one tile's arrival in the next decode step of the thread
+thread_local uint64_t g_wait_ns = 0;       // 0: the default limit
+thread_local int64_t g_withhold_tile = -1;
 
 constexpr int kMaxDevices = 128;
 int g_sm_count[kMaxDevices] = {0};
@@ -220,6 +225,9 @@ static la_status step_impl(la_rule rule, const la_pool* src, const int32_t* read
   p.scale = scale;
   p.o = o;
   p.err = err_word;
+  p.wait_ns = la::g_wait_ns ? la::g_wait_ns : la::kWaitLimitNs;
+  p.withhold = la::g_withhold_tile;
+  la::g_withhold_tile = -1;  // one-shot
   return cuda_status(fn(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -299,6 +307,8 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
     fn = (io == LA_F32) ? la::find_scan_conv_f32io(rule, s.d_k, s.d_v) : la::find_scan_conv_bf16io(rule, s.d_k, s.d_v);
   } else if (chunked) {
     if (s.d_k != 128 || s.d_v != 128 || io != LA_BF16) return LA_ERR_UNSUPPORTED;
+    // checkpoints fall on chunk boundaries, in the one-launch form
+    if (ckpt_every > 0 && (ckpt_every % 64 != 0 || workspace)) return LA_ERR_UNSUPPORTED;
     if (workspace && chunk_inverse(rule)) {
       if (!aligned(workspace, 16)) return LA_ERR_ALIGN;
       if (workspace_bytes < la::chunk_workspace_bytes(total_tokens, n_seqs, s.n_v_heads)) return LA_ERR_SHAPE;
@@ -415,6 +425,20 @@ la_status la_state_scan_checkpointed(la_rule rule, const la_pool* src, const int
   if (!aligned(ckpt_cu, 4) || !aligned(ckpt_slots, 4)) return LA_ERR_ALIGN;
   return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, q, k, v, io,
                    g, beta, scale, o, ckpt_every, ckpt_cu, ckpt_slots, err_word, stream);
+}
+
+la_status la_state_scan_chunked_checkpointed(la_rule rule, const la_pool* src, const int32_t* read_slot,
+                                             const la_pool* dst, const int32_t* write_slot, int32_t n_seqs,
+                                             const int32_t* cu_seqlens, int32_t total_tokens,
+                                             const int32_t* seq_order, const void* q, const void* k, const void* v,
+                                             la_dtype io, const float* g, const float* beta, float scale, void* o,
+                                             int32_t ckpt_every, const int32_t* ckpt_cu, const int32_t* ckpt_slots,
+                                             int32_t* err_word, void* stream) {
+  if (ckpt_every <= 0) return LA_ERR_SHAPE;
+  if (n_seqs > 0 && (!ckpt_cu || !ckpt_slots)) return LA_ERR_NULL;
+  if (!aligned(ckpt_cu, 4) || !aligned(ckpt_slots, 4)) return LA_ERR_ALIGN;
+  return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, q, k, v, io,
+                   g, beta, scale, o, ckpt_every, ckpt_cu, ckpt_slots, err_word, stream, true);
 }
 
 la_status la_state_scan_conv(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,
@@ -573,6 +597,10 @@ const char* la_status_str(la_status status) {
 }
 
 int32_t la_last_cuda_error(void) { return la::g_last_cuda_error; }
+
+void la_debug_set_wait_limit_us(uint32_t us) { la::g_wait_ns = (uint64_t)us * 1000u; }
+
+void la_debug_withhold_step_tile(int32_t tile) { la::g_withhold_tile = tile < 0 ? -1 : tile; }
 
 int32_t la_abi_version(void) { return LA_ABI_VERSION; }
 

@@ -700,6 +700,41 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
       const int nch = (x.n_tok + kC - 1) / kC;
       const int64_t sbase_src = ((int64_t)x.rs * H + x.h) * (kD * kD);
       const int64_t dbase = ((int64_t)x.ws * H + x.h) * (kD * kD);
+      // checkpoints (ckpt_every a multiple of the chunk): checkpoint k is the state after the
+      // first (k + 1) ckpt_every tokens, k < n_ck, to dst slot ckpt_slots[ckpt_cu[seq] + k]
+      int n_ck = 0, ck_base = 0;
+      if (p.ckpt_every > 0) {
+        ck_base = __ldg(p.ckpt_cu + x.seq);
+        n_ck = __ldg(p.ckpt_cu + x.seq + 1) - ck_base;
+        const int fit = x.n_tok / p.ckpt_every;
+        if (n_ck < 0 || n_ck > fit) {
+          if (tp == 0) report(p.err, LA_DEVERR_CU_SEQLENS);
+          n_ck = n_ck < 0 ? 0 : fit;
+        }
+      }
+      // the destination of the state after the first `tok` tokens: its checkpoint slot's
+      // base element, or -1 (no checkpoint there, or a bad slot, which is reported)
+      auto ckpt_base = [&](int tok) -> int64_t {
+        if (p.ckpt_every <= 0 || tok == 0 || tok % p.ckpt_every) return -1;
+        const int k = tok / p.ckpt_every - 1;
+        if (k >= n_ck) return -1;
+        const int cs = __ldg(p.ckpt_slots + ck_base + k);
+        if (cs < 0 || cs >= p.dst_slots) {
+          if (tp == 0) report(p.err, LA_DEVERR_WRITE_SLOT);
+          return -1;
+        }
+        return ((int64_t)cs * H + x.h) * (kD * kD);
+      };
+      auto store_col = [&](int64_t base, int i0, const uint32_t* v) {  // S[i0 + e][r] = v[e], e < 16
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int64_t el = base + (int64_t)(i0 + e) * kD + r;
+          if (p.dst_dtype == LA_F32)
+            static_cast<float*>(p.dst)[el] = __uint_as_float(v[e]);
+          else
+            static_cast<__nv_bfloat16*>(p.dst)[el] = __float2bfloat16_rn(__uint_as_float(v[e]));
+        }
+      };
       if (nch == 0) {
         // empty sequence: the initial state (or zero) goes to the destination
         for (int i = 0; i < kD; ++i) {
@@ -747,6 +782,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
         }
         umma::fence_after();
         const float gC = gbk[kC - 1];  // gamma_C (padded tokens have gate 1: the last real token's)
+        const int64_t ckb = ckpt_base(c * kC);  // a checkpoint at this chunk boundary
         // S pass: S0^T -> BF16 (the A operand of this chunk's products), S^T *= gamma_C
 #pragma unroll 1
         for (int c32 = 0; c32 < 4; ++c32) {
@@ -754,6 +790,10 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
           umma::ld16(tq + kColS + 32 * c32, a);
           umma::ld16(tq + kColS + 32 * c32 + 16, b);
           umma::wait_ld();
+          if (ckb >= 0) {
+            store_col(ckb, 32 * c32, a);
+            store_col(ckb, 32 * c32 + 16, b);
+          }
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             w[e] = pack2(a[2 * e], a[2 * e + 1]);
@@ -807,22 +847,17 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
         }
       }
       if (!ok) break;
-      // final state S[i][r] = S^T[r][i]
+      // final state S[i][r] = S^T[r][i] (and the last checkpoint when it falls on the end)
       if (!(ok = gwait(&bars[kSFull], (uint32_t)(j - 1) & 1u, abort_flag, tp, kNbState))) break;
       umma::fence_after();
+      const int64_t ckf = ckpt_base(x.n_tok);
 #pragma unroll 1
       for (int c16 = 0; c16 < 8; ++c16) {
         uint32_t v[16];
         umma::ld16(tq + kColS + 16 * c16, v);
         umma::wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int64_t el = dbase + (int64_t)(16 * c16 + e) * kD + r;
-          if (p.dst_dtype == LA_F32)
-            static_cast<float*>(p.dst)[el] = __uint_as_float(v[e]);
-          else
-            static_cast<__nv_bfloat16*>(p.dst)[el] = __float2bfloat16_rn(__uint_as_float(v[e]));
-        }
+        store_col(dbase, 16 * c16, v);
+        if (ckf >= 0) store_col(ckf, 16 * c16, v);
       }
       umma::fence_before();
     }

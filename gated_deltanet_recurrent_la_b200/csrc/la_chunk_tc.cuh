@@ -56,8 +56,8 @@ constexpr int kOffP = kOffW + 16384;         // P     [64][64]
 constexpr int kOffU = kOffP + 8192;          // U^T   [128 d_v][64]; O [64][128] row-major at the end
 constexpr int kOffUs = kOffU + 16384;        // Us^T  [128 d_v][64]
 constexpr int kOffGo = kOffUs + 16384;       // gamma_t of the last two chunks [2][64] fp32 (outputs)
-constexpr int kOffBar = kOffGo + 2 * kC * 4; // MMA groups 1-3, the two staging buffers, O2
-constexpr int kOffMisc = kOffBar + 6 * 8;    // [0] tensor-memory base, [3] the next unit
+constexpr int kOffBar = kOffGo + 2 * kC * 4; // MMA groups 1-3, the two staging buffers, O2, drain
+constexpr int kOffMisc = kOffBar + 7 * 8;    // [0] tensor-memory base, [3] the next unit
 constexpr int kSmem = kOffMisc + 16 + 1024;  // + slack for the 1024-byte alignment
 static_assert(kSmem <= 227 * 1024, "shared memory");
 static_assert(chunk::kPrepTileBytes == 16384 + chunk::kGateBlockBytes && kOffTu == kOffTw + 8192 &&
@@ -125,6 +125,7 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
     mbar_init(&bars[3], 1);
     mbar_init(&bars[4], 1);
     mbar_init(&bars[5], 1);
+    mbar_init(&bars[6], 1);
     mbar_init_fence();
   }
   umma::fence_before();
@@ -497,10 +498,13 @@ __global__ void __launch_bounds__(chunk_tc::kThreads, 1) chunk_tc_kernel(const S
     __syncthreads();
   }
 
-  // copies still in flight (only after a wait gave up): let them land, within the limit
+  // copies still in flight (only after a wait gave up): let them land, within the limit;
+  // and every MMA issued completes before the tensor memory is released
   if (tid == kWorkers) {
     for (int b = 0; b < 2; ++b)
       if (pending & (1u << b)) mbar_wait(&bars[3 + b], (lpar >> b) & 1u);
+    umma::commit(&bars[6]);
+    mbar_wait(&bars[6], 0);
   }
   if (abort && tid == 0) report(p.err, LA_DEVERR_TIMEOUT);
   umma::fence_before();

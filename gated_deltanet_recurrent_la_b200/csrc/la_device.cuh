@@ -66,13 +66,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits until the phase of `bar` with the given parity has completed.  Returns false
-// (without reporting) if the time limit or the poll cap is reached first.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// (without reporting) if the time limit (nanoseconds) or the poll cap is reached first.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t polls = 1; polls < kWaitMaxPolls; ++polls) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((polls & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if ((polls & 63u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
   }
   return false;
 }

@@ -46,6 +46,10 @@ struct StepParams {
   float scale;
   void* o;
   int32_t* err;
+  // failure-path test hooks: the time limit of every pipeline wait (ns), and a tile whose
+  // arrival the producer of CTA 0 withholds (-1: none) so that its consumers' waits expire
+  uint64_t wait_ns;
+  int64_t withhold;
 };
 
 struct ScanParams {

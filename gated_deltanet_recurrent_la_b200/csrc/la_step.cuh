@@ -262,8 +262,12 @@ __global__ void __launch_bounds__(
         const uint32_t round = (uint32_t)(it / C::kStages);
         bool ok = true;
         if (lane == 0) {
-          ok = mbar_wait(&empty[stage], (round & 1u) ^ 1u);
-          if (ok) {
+          ok = mbar_wait(&empty[stage], (round & 1u) ^ 1u, p.wait_ns);
+          if (ok && blockIdx.x == 0 && it == p.withhold) {
+            // test hook: this tile's copies are never issued and its arrival never comes (its
+            // consumers' waits run out); nothing of it is in flight, and the rest is abandoned
+            ok = false;
+          } else if (ok) {
             const int64_t t = blockIdx.x + it * gridDim.x;
             const int b = (int)(t / H);
             const int h = (int)(t % H);
@@ -335,7 +339,8 @@ __global__ void __launch_bounds__(
       for (int s = 0; s < C::kStages; ++s) {
         if (issued > s) {
           const int64_t last = issued - 1 - ((issued - 1 - s) % C::kStages);
-          if (!mbar_wait(&full[s], (uint32_t)(last / C::kStages) & 1u)) report(p.err, LA_DEVERR_TIMEOUT);
+          if (blockIdx.x == 0 && last == p.withhold) continue;  // withheld: nothing issued
+          if (!mbar_wait(&full[s], (uint32_t)(last / C::kStages) & 1u, p.wait_ns)) report(p.err, LA_DEVERR_TIMEOUT);
         }
       }
     }
@@ -360,7 +365,7 @@ __global__ void __launch_bounds__(
   for (int64_t it = team; it < n_my; it += C::kTeams) {
     const int stage = (int)(it % C::kStages);
     const uint32_t round = (uint32_t)(it / C::kStages);
-    const bool arrived = mbar_wait(&full[stage], round & 1u);
+    const bool arrived = mbar_wait(&full[stage], round & 1u, p.wait_ns);
     bool ok = __all_sync(0xffffffffu, arrived);
     float* scr = nullptr;
     if constexpr (CONV) {

@@ -28,13 +28,15 @@ LA_OK, LA_ERR_NULL, LA_ERR_SHAPE, LA_ERR_UNSUPPORTED, LA_ERR_ALIGN, LA_ERR_ALIAS
 DEVERR_READ_SLOT, DEVERR_WRITE_SLOT, DEVERR_CU_SEQLENS, DEVERR_TIMEOUT, DEVERR_Q8_MASK = 1, 2, 4, 8, 16
 
 EXPORTS = ("la_state_bytes", "la_shape_supported", "la_state_step", "la_state_scan", "la_state_scan_chunked",
-           "la_state_scan_checkpointed", "la_state_step_qgroups", "la_state_scan_qgroups",
+           "la_state_scan_checkpointed", "la_state_scan_chunked_checkpointed", "la_state_step_qgroups",
+           "la_state_scan_qgroups",
            "la_pool_slot_bytes", "la_state_pool_encode", "la_state_pool_decode", "la_state_step_conv",
            "la_state_scan_conv", "la_scan_chunked_workspace_bytes", "la_state_scan_chunked_ws",
            "la_state_scan_chunked_noalloc",
            "la_state_pool_copy",
            "la_state_pool_gather", "la_state_pool_scatter", "la_state_pool_zero", "la_state_check_slots",
-           "la_status_str", "la_last_cuda_error", "la_abi_version")
+           "la_status_str", "la_last_cuda_error", "la_abi_version", "la_debug_set_wait_limit_us",
+           "la_debug_withhold_step_tile")
 
 
 class LAError(RuntimeError):
@@ -87,6 +89,8 @@ def lib():
         L.la_state_scan_chunked.restype = I32
         L.la_state_scan_checkpointed.argtypes = L.la_state_scan.argtypes[:-2] + [I32, P, P, P, P]
         L.la_state_scan_checkpointed.restype = I32
+        L.la_state_scan_chunked_checkpointed.argtypes = L.la_state_scan_checkpointed.argtypes
+        L.la_state_scan_chunked_checkpointed.restype = I32
         L.la_state_step_qgroups.argtypes = L.la_state_step.argtypes[:6] + [I32] + L.la_state_step.argtypes[6:]
         L.la_state_step_qgroups.restype = I32
         L.la_state_scan_qgroups.argtypes = L.la_state_scan.argtypes[:9] + [I32] + L.la_state_scan.argtypes[9:]
@@ -121,6 +125,10 @@ def lib():
         L.la_status_str.restype = ctypes.c_char_p
         L.la_last_cuda_error.restype = I32
         L.la_abi_version.restype = I32
+        L.la_debug_set_wait_limit_us.argtypes = [ctypes.c_uint32]
+        L.la_debug_set_wait_limit_us.restype = None
+        L.la_debug_withhold_step_tile.argtypes = [I32]
+        L.la_debug_withhold_step_tile.restype = None
         _lib = L
     return _lib
 
@@ -274,6 +282,20 @@ def la_state_scan_checkpointed(rule, src: Optional[Pool], read_slot, dst: Pool, 
         _stream(stream))
 
 
+def la_state_scan_chunked_checkpointed(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens, q, k,
+                                       v, g, beta, scale, o, ckpt_every, ckpt_cu, ckpt_slots, err_word,
+                                       seq_order=None, stream=None) -> int:
+    """la_state_scan_checkpointed by the one-launch chunked prefill (ckpt_every a multiple of 64)."""
+    io = dtype_code(q.dtype)
+    return lib().la_state_scan_chunked_checkpointed(
+        RULES[rule] if isinstance(rule, str) else int(rule), None if src is None else src.ref,
+        _ptr(read_slot, torch.int32), dst.ref, _ptr(write_slot, torch.int32), int(cu_seqlens.numel() - 1),
+        _ptr(cu_seqlens, torch.int32), int(q.shape[0]), _ptr(seq_order, torch.int32), _ptr(q), _ptr(k, q.dtype),
+        _ptr(v, q.dtype), io, _ptr(g, torch.float32), _ptr(beta, torch.float32), float(scale), _ptr(o, q.dtype),
+        int(ckpt_every), _ptr(ckpt_cu, torch.int32), _ptr(ckpt_slots, torch.int32), _ptr(err_word, torch.int32),
+        _stream(stream))
+
+
 class Conv:
     """The short causal convolution ahead of the step: weights (float32 [heads, channels,
     W] on the device) and the history pools (io dtype [n_slots, H_v, 2 d_k + d_v, W - 1])."""
@@ -390,3 +412,14 @@ def la_state_check_slots(read_slot_host, write_slot_host, n_slots: int, B: Optio
 
 def la_abi_version() -> int:
     return lib().la_abi_version()
+
+
+def la_debug_set_wait_limit_us(us: int) -> None:
+    """Test hook: the decode step's pipeline wait limit on this thread (0: the default 1 s)."""
+    lib().la_debug_set_wait_limit_us(int(us))
+
+
+def la_debug_withhold_step_tile(tile: int) -> None:
+    """Test hook: the next decode step on this thread withholds one tile's arrival, so its
+    waits run out and LA_DEVERR_TIMEOUT is reported (nothing is left in flight)."""
+    lib().la_debug_withhold_step_tile(int(tile))

@@ -77,7 +77,7 @@
 extern "C" {
 #endif
 
-#define LA_ABI_VERSION 2
+#define LA_ABI_VERSION 3
 
 typedef enum {
     LA_RULE_LINEAR = 0,
@@ -281,6 +281,20 @@ la_status la_state_scan_checkpointed(la_rule rule, const la_pool *src, const int
                                      float scale, void *o, int32_t ckpt_every, const int32_t *ckpt_cu,
                                      const int32_t *ckpt_slots, int32_t *err_word, void *stream);
 
+/* la_state_scan_checkpointed evaluated by la_state_scan_chunked (one launch): the checkpoints
+ * fall on chunk boundaries, so ckpt_every must be a multiple of 64 (the chunk length); each
+ * checkpoint is the FP32 state the chunked recurrence holds at that boundary, stored in the dst
+ * dtype.  Arguments, checkpoint semantics and errors as la_state_scan_checkpointed; supported
+ * set as la_state_scan_chunked; LA_ERR_UNSUPPORTED when ckpt_every is not a multiple of 64. */
+la_status la_state_scan_chunked_checkpointed(la_rule rule, const la_pool *src, const int32_t *read_slot,
+                                             const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
+                                             const int32_t *cu_seqlens, int32_t total_tokens,
+                                             const int32_t *seq_order, const void *q, const void *k,
+                                             const void *v, la_dtype io, const float *g, const float *beta,
+                                             float scale, void *o, int32_t ckpt_every,
+                                             const int32_t *ckpt_cu, const int32_t *ckpt_slots,
+                                             int32_t *err_word, void *stream);
+
 /* The short causal convolution fused ahead of the decode step ("Gated DeltaNet" glossary,
  * Engineering details: Conv1D fused with the recurrence into one kernel).  The pages give
  * no width, activation or normalisation; this library's reading: per channel c of the q,
@@ -399,6 +413,21 @@ int32_t la_last_cuda_error(void);
 
 /* LA_ABI_VERSION of the loaded library. */
 int32_t la_abi_version(void);
+
+/* Failure-path test hooks.  Every pipeline wait inside the kernels has a time limit after
+ * which the kernel stops, reports LA_DEVERR_TIMEOUT through the error word and returns, so
+ * the CUDA context stays usable.  These two calls let a test exercise that path without any
+ * fault: they change nothing else, and results are unaffected while they are unused.
+ *   la_debug_set_wait_limit_us  the limit of the decode step's (la_state_step and its
+ *                               variants) waits on the calling thread, in microseconds;
+ *                               0 restores the default of one second
+ *   la_debug_withhold_step_tile the next decode step on the calling thread withholds the
+ *                               given tile (its index in the first CTA's order, 0 = first):
+ *                               the producer issues no copy for it and signals nothing, so
+ *                               the consumers' waits run out (nothing is left in flight); one
+ *                               call only affects one step; a negative tile cancels it */
+void la_debug_set_wait_limit_us(uint32_t us);
+void la_debug_withhold_step_tile(int32_t tile);
 
 #ifdef __cplusplus
 }

@@ -233,6 +233,32 @@ def test_chunked_ws_linear_and_gated_ignore_the_workspace(lib):
     assert call(3, A, 16, io=1) == L.LA_ERR_SHAPE         # and sized
 
 
+def test_failure_hooks_are_plain_host_calls(lib):
+    """The failure-path test hooks only set host state (no device work): callable here."""
+    L.la_debug_set_wait_limit_us(1500)
+    L.la_debug_withhold_step_tile(3)
+    L.la_debug_withhold_step_tile(-1)
+    L.la_debug_set_wait_limit_us(0)
+
+
+def test_chunked_checkpointed_host_errors(lib):
+    """The chunked checkpointed prefill: checkpoints on the 64-token chunk grid only, and the
+    checkpointed scan's own host checks."""
+    dst = pool()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+
+    def call(every=128, ccu=A, cs=A, n=2, rule=3):
+        return lib.la_state_scan_chunked_checkpointed(rule, None, None, ctypes.byref(dst), None, n, P(A), 10, None,
+                                                      P(A), P(A), P(A), 1, P(A), P(A), 1.0, P(A), every, P(ccu),
+                                                      P(cs), P(A), None)
+    assert call(every=0) == L.LA_ERR_SHAPE
+    assert call(ccu=None) == L.LA_ERR_NULL
+    assert call(cs=A + 2) == L.LA_ERR_ALIGN
+    assert call(every=100) == L.LA_ERR_UNSUPPORTED
+    assert call(rule=4) == L.LA_ERR_UNSUPPORTED  # kda
+    assert call(n=0) == L.LA_OK
+
+
 def test_checkpointed_scan_host_errors(lib):
     dst = pool()
     P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
