@@ -9,7 +9,7 @@ import torch
 import oracle
 from gated_deltanet_recurrent_la_b200 import lastate as L
 from gated_deltanet_recurrent_la_b200 import workloads as W
-from gpu_helpers import BF16, F32, assert_close, dev, dname, np64, tolerances
+from gpu_helpers import BF16, F32, assert_close, dev, dname, np64, prefill_picks, scan_unit_inputs, tolerances
 
 pytestmark = pytest.mark.gpu
 
@@ -178,3 +178,34 @@ def test_scan_conv_then_step_conv_continues_the_sequence():
     assert_close(np64(o.cpu())[0], o_ref[29], 1e-4, "the decode step's output")
     assert_close(np64(o_pre), o_ref[:29], 1e-4, "prefill outputs")
     assert np.array_equal(np64(hist_t.cpu()), href)
+
+
+def test_conv_prefill32_units():
+    """The full prefill workload with the convolution ahead of every token (fresh prefill):
+    every sequence on two heads and the longest on all 32 against the oracle's convolved scan,
+    including the final histories (exact copies of the last raw inputs)."""
+    inp = W.conv_prefill32()
+    x = inp.extra
+    width, n = x["width"], inp.cu_seqlens.numel() - 1
+    S, hnew, o, err = run_scan_conv(inp, x["w_q"], x["w_k"], x["w_v"], width, x["activation"], x["qk_l2norm"], None,
+                                    n, inp.state_dtype)
+    assert err == 0
+    cu = inp.cu_seqlens.numpy()
+    tol_s, tol_o = tolerances(inp.state_dtype, inp.io_dtype)
+    by_head = {}
+    for s_, h in prefill_picks(inp):
+        by_head.setdefault(h, []).append(s_)
+    for h, seqs in sorted(by_head.items()):
+        sub = scan_unit_inputs(inp, [(s_, h) for s_ in seqs])
+        ref, href, o_ref, e = oracle.scan_conv(
+            inp.rule, 1, sub.cu_seqlens.numpy(), np64(sub.q), np64(sub.k), np64(sub.v), np64(sub.g), np64(sub.beta),
+            inp.scale, x["w_q"][h:h + 1].double().numpy(), x["w_k"][h:h + 1].double().numpy(),
+            x["w_v"][h:h + 1].double().numpy(), act=x["activation"], l2norm=x["qk_l2norm"],
+            dst_dtype=dname(inp.state_dtype), io_dtype=dname(inp.io_dtype))
+        assert e == 0
+        ucu = sub.cu_seqlens.numpy()
+        for i, s_ in enumerate(seqs):
+            t0, t1 = int(cu[s_]), int(cu[s_ + 1])
+            assert_close(np64(S[s_, h]), ref[i, 0], tol_s, f"seq {s_} head {h} final state")
+            assert_close(np64(o[t0:t1, h]), o_ref[int(ucu[i]):int(ucu[i + 1]), 0], tol_o, f"seq {s_} head {h} outputs")
+            assert np.array_equal(np64(hnew[s_, h]), href[i, 0]), f"seq {s_} head {h} final history"

@@ -13,9 +13,9 @@ import torch
 import oracle
 from gated_deltanet_recurrent_la_b200 import lastate as L
 from gated_deltanet_recurrent_la_b200 import workloads as W
-from gpu_helpers import (BF16, F32, assert_close, check_step_against_oracle, dev, dname, gpu_scan, gpu_scan_qgroups,
-                         gpu_step, gpu_step_qgroups, np64, oracle_scan, oracle_scan_qgroups, oracle_step_qgroups,
-                         tolerances)
+from gpu_helpers import (BF16, F32, assert_close, check_scan_units, check_step_against_oracle, dev, dname, gpu_scan,
+                         gpu_scan_qgroups, gpu_step, gpu_step_qgroups, np64, oracle_scan, oracle_scan_qgroups,
+                         oracle_step_qgroups, prefill_picks, tolerances)
 
 pytestmark = pytest.mark.gpu
 
@@ -64,46 +64,30 @@ def test_tiny_scan(rule):
 # ---- the full-size decode workloads ----------------------------------------------------
 
 def test_decode64_full():
-    check_step_against_oracle(W.decode64())
+    check_step_against_oracle(W.decode64(), ulps=True)
 
 
 def test_decode512_full_with_checkpoints():
     inp = W.decode512()
     rs, ws = inp.read_slot.numpy(), inp.write_slot.numpy()
     assert (rs != ws).sum() == 256 and len(set(ws)) == 512
-    check_step_against_oracle(inp)  # also proves every checkpoint slot is bit-identical afterwards
+    check_step_against_oracle(inp, ulps=True)  # also proves every checkpoint slot is bit-identical afterwards
 
 
 def test_mamba2_full():
-    check_step_against_oracle(W.mamba2())
+    check_step_against_oracle(W.mamba2(), ulps=True)
 
 
-# ---- the full-size prefill workload, sampled ----------------------------------------------
+# ---- the full-size prefill workload ------------------------------------------------------
 
-def _check_sampled_units(inp, S, o, picks):
-    """(sequence, head) units of a full-size scan recomputed one by one by the oracle."""
-    cu = inp.cu_seqlens.numpy()
-    tol_s, tol_o = tolerances(inp.state_dtype, inp.io_dtype)
-    for s, h in picks:
-        t0, t1 = int(cu[s]), int(cu[s + 1])
-        sub = W.Inputs("scan", inp.rule, 1, 1, 128, 128, inp.state_dtype, inp.io_dtype, inp.q[t0:t1, h:h + 1],
-                       inp.k[t0:t1, h:h + 1], inp.v[t0:t1, h:h + 1], inp.g[t0:t1, h:h + 1],
-                       inp.beta[t0:t1, h:h + 1], 1.0, None, None, None, torch.tensor([0, t1 - t0], dtype=torch.int32))
-        S_ref, o_ref, e = oracle_scan(sub)
-        assert e == 0
-        assert_close(np64(S[s, h]), S_ref[0, 0], tol_s, f"seq {s} head {h} final state")
-        assert_close(np64(o[t0:t1, h]), o_ref[:, 0], tol_o, f"seq {s} head {h} outputs")
-    assert torch.isfinite(o.float()).all() and torch.isfinite(S.float()).all()
-
-
-def test_prefill32_sampled():
+def test_prefill32_units():
+    """The full prefill workload: every sequence on two heads and the longest on all 32
+    against the oracle (94 (sequence, head) units)."""
     inp = W.prefill32()
     S, o, err = gpu_scan(inp)
     assert err == 0
-    cu = inp.cu_seqlens.numpy()
-    order = np.argsort(cu[1:] - cu[:-1])
-    _check_sampled_units(inp, S, o, [(int(order[0]), 0), (int(order[0]), 31), (int(order[16]), 7),
-                                     (int(order[-1]), 19)])
+    tol_s, tol_o = tolerances(inp.state_dtype, inp.io_dtype)
+    check_scan_units(inp, S, o, prefill_picks(inp), tol_s, tol_o)
 
 
 # ---- every rule x tile shape x dtype, small batches -----------------------------------------
@@ -376,13 +360,14 @@ def _ckpt_layout(lengths, every, extra_slot_base):
     return cu, slots
 
 
-def _gpu_scan_ckpt(inp, every, ckpt_cu, ckpt_slots, n_dst, dst_dtype):
+def _gpu_scan_ckpt(inp, every, ckpt_cu, ckpt_slots, n_dst, dst_dtype, chunked=False):
     n_seqs = inp.cu_seqlens.numel() - 1
     dst_t = torch.full((n_dst, inp.n_v_heads, inp.d_k, inp.d_v), 3.0, dtype=dst_dtype, device="cuda")
     src = None if inp.pool is None else L.Pool(dev(inp.pool), inp.n_qk_heads)
     o = torch.full((inp.q.shape[0], inp.n_v_heads, inp.d_v), 5.0, dtype=inp.io_dtype, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    st = L.la_state_scan_checkpointed(inp.rule, src, dev(inp.read_slot), L.Pool(dst_t, inp.n_qk_heads), None,
+    fn = L.la_state_scan_chunked_checkpointed if chunked else L.la_state_scan_checkpointed
+    st = fn(inp.rule, src, dev(inp.read_slot), L.Pool(dst_t, inp.n_qk_heads), None,
                                       dev(inp.cu_seqlens), dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.g),
                                       dev(inp.beta), inp.scale, o, every, dev(torch.as_tensor(ckpt_cu)),
                                       dev(torch.as_tensor(ckpt_slots)), err)
@@ -573,31 +558,67 @@ def test_chunked_two_launches_pool_slots_and_order():
     assert_close(np64(o.cpu()), o_ref, 2e-2, "outputs")
 
 
-def test_chunked_two_launches_prefill32_sampled():
+def test_chunked_two_launches_prefill32_units():
     """The full prefill workload through the two-launch path, as the benchmark runs it:
-    the shortest and the longest sequence checked against the oracle on one head each."""
+    every sequence on two heads and the longest on all 32 against the oracle."""
     inp = W.prefill32()
     S, o, err = _gpu_scan_chunked_ws(inp, BF16)
     assert err == 0
-    cu = inp.cu_seqlens.numpy()
-    order = np.argsort(cu[1:] - cu[:-1])
-    _check_sampled_units(inp, S, o, [(int(order[0]), 7), (int(order[-1]), 21)])
+    check_scan_units(inp, S, o, prefill_picks(inp), 2e-2, 2e-2)
 
 
-def test_chunked_prefill32_sampled():
+def test_chunked_prefill32_units():
+    """The full prefill workload through the one-launch chunked prefill: every sequence on
+    two heads and the longest on all 32 against the oracle."""
     inp = W.prefill32()
     S, o, err = _gpu_scan_chunked(inp, BF16)
     assert err == 0
-    cu = inp.cu_seqlens.numpy()
-    order = np.argsort(cu[1:] - cu[:-1])
-    for s, h in [(int(order[0]), 3), (int(order[-1]), 29)]:
-        t0, t1 = int(cu[s]), int(cu[s + 1])
-        sub = W.Inputs("scan", inp.rule, 1, 1, 128, 128, BF16, BF16, inp.q[t0:t1, h:h + 1], inp.k[t0:t1, h:h + 1],
-                       inp.v[t0:t1, h:h + 1], inp.g[t0:t1, h:h + 1], inp.beta[t0:t1, h:h + 1], 1.0, None, None, None,
-                       torch.tensor([0, t1 - t0], dtype=torch.int32))
-        S_ref, o_ref, _ = oracle_scan(sub)
-        assert_close(np64(S[s, h]), S_ref[0, 0], 2e-2, f"seq {s} head {h} final state")
-        assert_close(np64(o[t0:t1, h]), o_ref[:, 0], 2e-2, f"seq {s} head {h} outputs")
+    check_scan_units(inp, S, o, prefill_picks(inp), 2e-2, 2e-2)
+
+
+@pytest.mark.parametrize("dst", [F32, BF16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("rule", W.RULES)
+def test_chunked_checkpoints(rule, dst):
+    """Prefix-cache checkpoints from the one-launch chunked prefill, every 128 tokens (chunk
+    boundaries): every checkpoint and final state against the oracle's checkpointed scan at
+    the BF16-operand tolerance; the outputs and final states are those of the plain chunked
+    call, bit for bit (a checkpoint is a store of the state the recurrence already holds)."""
+    lengths, every = [300, 64, 0, 129, 256, 5, 640], 128
+    inp = W.scan_inputs(lengths=lengths, n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128, rule=rule, io_dtype=BF16,
+                        seed=33, init="slots", init_dtype=F32, scale=0.8)
+    ckpt_cu, ckpt_slots = _ckpt_layout(lengths, every, len(lengths))
+    n_dst = len(lengths) + int(ckpt_cu[-1])
+    S, o, err = _gpu_scan_ckpt(inp, every, ckpt_cu, ckpt_slots, n_dst, dst, chunked=True)
+    assert err == 0
+    S_ref, o_ref, e = oracle.scan(rule, 2, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k), np64(inp.v),
+                                  np64(inp.g), np64(inp.beta), inp.scale, src_pool=np64(inp.pool),
+                                  read_slot=inp.read_slot.numpy(), dst_pool=np.zeros((n_dst, 4, 128, 128)),
+                                  dst_dtype=dname(dst), io_dtype="bf16", ckpt_every=every, ckpt_cu=ckpt_cu,
+                                  ckpt_slots=ckpt_slots)
+    assert e == 0
+    assert_close(np64(S), S_ref, 2e-2, f"{rule}: final states and checkpoints")
+    assert_close(np64(o), o_ref, 2e-2, f"{rule}: outputs")
+    S1, o1, e1 = _gpu_scan_chunked(inp, dst)
+    assert e1 == 0 and torch.equal(o, o1) and torch.equal(S[:len(lengths)], S1)
+
+
+def test_chunked_checkpoints_supported_set_and_errors():
+    """ckpt_every off the chunk grid is refused on the host; too many checkpoints for a
+    sequence and a slot outside the pool are reported on the device, the others written."""
+    lengths = [256, 130]
+    inp = W.scan_inputs(lengths=lengths, n_qk_heads=1, n_v_heads=2, d_k=128, d_v=128, io_dtype=BF16, seed=34)
+    with pytest.raises(L.LAError) as ei:
+        _gpu_scan_ckpt(inp, 100, np.array([0, 2, 3], np.int32), np.array([2, 3, 4], np.int32), 5, BF16, chunked=True)
+    assert ei.value.status == L.LA_ERR_UNSUPPORTED
+    cu = np.array([0, 3, 4], dtype=np.int32)            # sequence 0 fits only 2 checkpoints of 128
+    slots = np.array([2, 3, 4, 99], dtype=np.int32)      # slot 99 is outside the pool
+    S, o, err = _gpu_scan_ckpt(inp, 128, cu, slots, 5, BF16, chunked=True)
+    assert err == (L.DEVERR_CU_SEQLENS | L.DEVERR_WRITE_SLOT)
+    S_ref, _, _ = oracle.scan("gated_delta", 1, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k), np64(inp.v),
+                              np64(inp.g), np64(inp.beta), dst_pool=np.zeros((5, 2, 128, 128)), dst_dtype="bf16",
+                              io_dtype="bf16", ckpt_every=128, ckpt_cu=np.array([0, 2, 3], dtype=np.int32),
+                              ckpt_slots=np.array([2, 3, 4], dtype=np.int32))
+    assert_close(np64(S[:4]), S_ref[:4], 2e-2, "checkpoints that fit are written")
 
 
 # ---- channel-wise gate (kda): the full-size workloads, special cases, the supported set ----
@@ -606,13 +627,12 @@ def test_kda_decode64_full():
     check_step_against_oracle(W.kda_decode64())
 
 
-def test_kda_prefill32_sampled():
+def test_kda_prefill32_units():
     inp = W.kda_prefill32()
     S, o, err = gpu_scan(inp)
     assert err == 0
-    cu = inp.cu_seqlens.numpy()
-    order = np.argsort(cu[1:] - cu[:-1])
-    _check_sampled_units(inp, S, o, [(int(order[0]), 5), (int(order[-1]), 30)])
+    tol_s, tol_o = tolerances(inp.state_dtype, inp.io_dtype)
+    check_scan_units(inp, S, o, prefill_picks(inp), tol_s, tol_o)
 
 
 def test_kda_wide_gate_and_beta_ranges():
