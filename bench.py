@@ -396,7 +396,8 @@ def chunk_roofline(run, inp, ms, peaks):
     peak_tf = peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)
     two = run.ws is not None and inp.rule in ("delta", "gated_delta")
     out = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
-           "traffic": recorded_traffic("chunk_tc" if two else "chunk_fused", "prefill32"),
+           "traffic": recorded_traffic("chunk_tc" if two else "chunk_fused",
+                                       "prefill32" + (f"_ckpt{run.ckpt_every}" if run.ckpt_every else "")),
            "algorithmic_bytes_per_launch": nbytes,
            "method_tflops": flops / (ms * 1e-3) / 1e12,
            "mma_tflops": mma_tf, "mma_frac_of_bf16_peak": mma_tf / peak_tf,
@@ -465,6 +466,12 @@ class ScanRunner:
             st = self.L.la_state_scan_chunked_ws(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu,
                                                  self.q, self.k, self.v, self.g, self.beta, self.inp.scale, self.o,
                                                  self.ws, self.err, seq_order=self.order, stream=stream)
+        elif self.chunked and self.ckpt_every > 0:
+            st = self.L.la_state_scan_chunked_checkpointed(self.inp.rule, self.src, self.read_slot, self.dst, None,
+                                                           self.cu, self.q, self.k, self.v, self.g, self.beta,
+                                                           self.inp.scale, self.o, self.ckpt_every, self.ckpt_cu,
+                                                           self.ckpt_slots, self.err, seq_order=self.order,
+                                                           stream=stream)
         elif self.chunked:
             st = self.L.la_state_scan_chunked(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu, self.q,
                                               self.k, self.v, self.g, self.beta, self.inp.scale, self.o, self.err,
@@ -978,6 +985,9 @@ def main():
         torch.cuda.empty_cache()
         rows["prefill32_chunked_two_launch"] = measure_row("prefill32", max(3, min(a.steps, 50)), a.warmup, world,
                                                            peaks, sm_count, None, chunked="ws")
+        torch.cuda.empty_cache()
+        rows["prefill32_chunked_ckpt256"] = measure_row("prefill32", max(3, min(a.steps, 50)), a.warmup, world,
+                                                        peaks, sm_count, None, ckpt_every=256, chunked=True)
         torch.cuda.empty_cache()
         pool_run = PoolRunner()
         pms = time_back_to_back(pool_run, min(a.steps, 500), a.warmup, world)
