@@ -17,10 +17,12 @@
 // which unrolls u_t = b (v_t - c S_{t-1}^T k_t), S_t = a S_{t-1} + k_t u_t^T exactly (the
 // linear and gated rules have U = V).  Gate ratios use log|g| and a sign product, so
 // negative gates are allowed.  Products take BF16 operands with FP32 accumulation; the
-// FP32 state lives in the accumulators of the state update across the whole sequence.
+// FP32 state stays on chip (in tensor memory) across the whole sequence.
 //
-// This kernel: d_k = d_v = 128, BF16 q/k/v/o, one CTA of 8 warps per (sequence, head),
-// warp-level tensor-core MMA (m16n8k16) fed by ldmatrix from XOR-swizzled shared memory.
+// This file: the definitions shared by the chunked kernels (d_k = d_v = 128, BF16
+// q/k/v/o) and the intra-chunk launch of the two-launch form (chunk_prep_kernel).  The
+// one-launch form is la_chunk_fused.cuh, the recurrence of the two-launch form
+// la_chunk_tc.cuh.
 #pragma once
 
 #include <cstdint>
@@ -33,32 +35,11 @@ namespace chunk {
 
 constexpr int kC = 64;         // tokens per chunk
 constexpr int kD = 128;        // d_k = d_v
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
 
 // shared-memory layout (bytes)
 constexpr int kRow128 = kD * 2;                 // one BF16 row of 128
 constexpr int kRow64 = kC * 2;                  // one BF16 row of 64
 constexpr int kLs = kC + 4;                     // padded row stride of the FP32 L matrix
-constexpr int kInBytes = 3 * kC * kRow128;      // K, Q, V of one chunk
-constexpr int kOffIn = 0;                       // 2 x {K, Q, V} [64][128] bf16, swizzled
-constexpr int kOffS = kOffIn + 2 * kInBytes;    // [128][128] bf16 state copy, swizzled
-constexpr int kTs = kC + 8;                     // padded row stride of the FP32 T matrix
-constexpr int kXs = 24;                         // padded row stride of a 16 x 16 FP32 scratch block
-constexpr int kOffL = kOffS + kD * kRow128;     // [64][68] fp32 (L, then reused for W)
-constexpr int kOffT = kOffL + kC * kLs * 4;     // [64][72] fp32
-constexpr int kOffW = kOffL;                    // [64][128] bf16, swizzled (after T is formed)
-constexpr int kOffTw = kOffT + kC * kTs * 4;    // [64][64] bf16, swizzled
-constexpr int kOffTu = kOffTw + kC * kRow64;
-constexpr int kOffP = kOffTu + kC * kRow64;     // [64][64] bf16, swizzled (masked Q K^T)
-constexpr int kOffU = kOffP + kC * kRow64;      // [64][128] bf16, swizzled
-constexpr int kOffUs = kOffU + kC * kRow128;    // [64][128] bf16, swizzled (rows scaled)
-constexpr int kOffX = kOffUs + kC * kRow128;    // [3][16][24] fp32 (per-warp scratch of the inverse)
-constexpr int kOffG = kOffX + 3 * 16 * kXs * 4; // per token: log|gamma|, sign, b, gamma, A, B
-constexpr int kOffGin = kOffG + 6 * kC * 4;     // 2 x {g, beta} [64] fp32 (staged gates)
-constexpr int kSmem = kOffGin + 2 * 2 * kC * 4;
-static_assert(kSmem <= 227 * 1024, "shared memory");
-static_assert(kOffW + kC * kRow128 <= kOffT + kC * kTs * 4, "W reuses the L / T space");
 // workspace tile of one (chunk, head): Tw then Tu, [64][64] BF16 each, rows 128 bytes
 // apart with the 16-byte piece c of row r at c ^ (r & 7); then the gate block, FP32
 // [6][64] = gamma_t, gamma_C / gamma_t, A_t = gamma_t / e^m, B_t = e^m / gamma_t,
@@ -77,12 +58,6 @@ __device__ __forceinline__ uint32_t swz(uint32_t base, int r, int ch, int rowb) 
 
 __device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm4t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
 }
@@ -130,504 +105,12 @@ __device__ __forceinline__ void mma16x16x16_tf32(float (*acc)[4], const float* a
 __device__ __forceinline__ void lda(uint32_t* a, uint32_t base, int rowb, int m0, int k0, int lane) {
   ldsm4(swz(base, m0 + (lane & 15), (k0 >> 3) + (lane >> 4), rowb), a[0], a[1], a[2], a[3]);
 }
-// A fragment (rows m0.., k0..) of A = X^T where X is a row-major [k][m] matrix
-__device__ __forceinline__ void lda_t(uint32_t* a, uint32_t base, int rowb, int m0, int k0, int lane) {
-  ldsm4t(swz(base, k0 + (lane & 7) + ((lane >> 4) << 3), (m0 >> 3) + ((lane >> 3) & 1), rowb), a[0], a[1], a[2],
-         a[3]);
-}
 // B fragments of two n-tiles (n0..n0+15, k0..k0+15) where B[k][n] = X[n][k], X row-major [n][k]
 __device__ __forceinline__ void ldb_nk(uint32_t* b, uint32_t base, int rowb, int n0, int k0, int lane) {
   ldsm4(swz(base, n0 + (lane & 7) + ((lane >> 4) << 3), (k0 >> 3) + ((lane >> 3) & 1), rowb), b[0], b[1], b[2],
         b[3]);
 }
-// B fragments of two n-tiles (n0..n0+15, k0..k0+15) of a row-major [k][n] matrix
-__device__ __forceinline__ void ldb_kn(uint32_t* b, uint32_t base, int rowb, int n0, int k0, int lane) {
-  ldsm4t(swz(base, k0 + (lane & 7) + (((lane >> 3) & 1) << 3), (n0 >> 3) + (lane >> 4), rowb), b[0], b[1], b[2],
-         b[3]);
-}
-
-__device__ __forceinline__ void st_bf16x2(unsigned char* smem, uint32_t off, float x, float y) {
-  *reinterpret_cast<uint32_t*>(smem + off) = pack_bf16x2(x, y);
-}
-
 }  // namespace chunk
-
-template <int RULE>
-__global__ void __launch_bounds__(chunk::kThreads, 1) chunk_scan_kernel(const ScanParams p) {
-  using namespace chunk;
-  extern __shared__ __align__(1024) unsigned char smem[];
-  const uint32_t sbase = smem_addr(smem);
-  float* sL = reinterpret_cast<float*>(smem + kOffL);
-  float* sT = reinterpret_cast<float*>(smem + kOffT);
-  float* sX = reinterpret_cast<float*>(smem + kOffX);
-  float* sLg = reinterpret_cast<float*>(smem + kOffG);  // log |gamma_t|
-  float* sSg = sLg + kC;                                 // sign gamma_t
-  float* sBt = sSg + kC;                                 // b_t
-  float* sGm = sBt + kC;                                 // gamma_t
-  float* sFa = sGm + kC;                                 // gamma_t / e^m  (factored ratios)
-  float* sFb = sFa + kC;                                 // e^m / gamma_s
-
-  constexpr bool kGate = Rule<RULE>::kUsesGate;
-  constexpr bool kDelta = Rule<RULE>::kPredicts;
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int lane = tid & 31;
-  const int g8 = lane >> 2;  // fragment row within 8
-  const int t4 = lane & 3;   // fragment column pair
-  const int H = p.n_v_heads;
-  const int ratio_h = H / p.n_qk_heads;
-  const int64_t units = (int64_t)p.n_seqs * H;
-  const int64_t G = gridDim.x;
-  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
-  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(p.k);
-  const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(p.v);
-  __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.o);
-
-  // this warp's block of the master state: rows [16 warp, 16 warp + 16), all 128 columns,
-  // as 16 accumulator tiles of 16 x 8 (mma C layout)
-  const int srow0 = 16 * warp;
-  // this warp's block of U~ / U / O: token rows [16 mt, 16 mt + 16), columns [64 nh, 64 nh + 64)
-  const int mt = warp & 3, nh = warp >> 2;
-
-  // the strictly upper 16 x 16 blocks of Tw and Tu are zero in every chunk
-  for (int idx = tid; idx < kC * kC / 2; idx += kThreads) {
-    const int r = idx >> 5, c = 2 * (idx & 31);
-    if ((c >> 4) > (r >> 4)) {
-      const uint32_t off = swz(kOffTw, r, c >> 3, kRow64) + 2 * (c & 7);
-      st_bf16x2(smem, off, 0.0f, 0.0f);
-      st_bf16x2(smem, off - kOffTw + kOffTu, 0.0f, 0.0f);
-    }
-  }
-  __syncthreads();
-
-#pragma unroll 1
-  for (int64_t round = 0; round * G < units; ++round) {
-    const int64_t u = round * G + ((round & 1) ? (G - 1 - blockIdx.x) : blockIdx.x);
-    if (u >= units) continue;
-    const int64_t si = u / H;
-    const int h = (int)(u % H);
-    const int hq = h / ratio_h;
-    const int seq = p.seq_order ? __ldg(p.seq_order + si) : (int)si;
-    if (seq < 0 || seq >= p.n_seqs) {
-      if (tid == 0) report(p.err, LA_DEVERR_CU_SEQLENS);
-      continue;
-    }
-    const int t0 = __ldg(p.cu_seqlens + seq);
-    const int t1 = __ldg(p.cu_seqlens + seq + 1);
-    if (seq == 0 && h == 0 && t0 != 0 && tid == 0) report(p.err, LA_DEVERR_CU_SEQLENS);
-    if (t0 < 0 || t1 < t0 || t1 > p.total_tokens) {
-      if (tid == 0) report(p.err, LA_DEVERR_CU_SEQLENS);
-      continue;
-    }
-    const int rs = p.read_slot ? __ldg(p.read_slot + seq) : 0;
-    const int ws = p.write_slot ? __ldg(p.write_slot + seq) : seq;
-    const bool rs_ok = !p.read_slot || (rs >= 0 && rs < p.src_slots);
-    const bool ws_ok = ws >= 0 && ws < p.dst_slots;
-    if (!rs_ok || !ws_ok) {
-      if (tid == 0) report(p.err, (rs_ok ? 0u : LA_DEVERR_READ_SLOT) | (ws_ok ? 0u : LA_DEVERR_WRITE_SLOT));
-      continue;
-    }
-
-    // ---- initial state into the accumulators: st[j][0..1] = row g8, cols 8j + 2 t4 (+1);
-    //      st[j][2..3] = row g8 + 8
-    float st[16][4];
-    const int64_t sbase_src = ((int64_t)rs * H + h) * (kD * kD);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = srow0 + g8 + (e >> 1) * 8, c = 8 * j + 2 * t4 + (e & 1);
-        float x = 0.0f;
-        if (p.read_slot) {
-          x = p.src_dtype == LA_F32 ? static_cast<const float*>(p.src)[sbase_src + r * kD + c]
-                                    : __bfloat162float(static_cast<const __nv_bfloat16*>(p.src)[sbase_src + r * kD + c]);
-        }
-        st[j][e] = x;
-      }
-    }
-
-    const int n_tok = t1 - t0;
-    const int n_chunks = (n_tok + kC - 1) / kC;
-    int* sFlag = reinterpret_cast<int*>(sX);  // [0]: 1 when this chunk uses factored gate ratios
-
-    // Stages chunk ci (K, Q, V rows and the gates) into input buffer ci & 1 with cp.async;
-    // rows beyond the sequence are zero and their gates are (1, 0).  Warp 0 stages the gates.
-    auto stage = [&](int ci) {
-      const int cc0 = ci * kC;
-      const int nn = (n_tok - cc0) < kC ? (n_tok - cc0) : kC;
-      unsigned char* in = smem + kOffIn + (ci & 1) * kInBytes;
-      for (int idx = tid; idx < kC * 16; idx += kThreads) {
-        const int r = idx >> 4, ch = idx & 15;
-        const uint32_t so = (uint32_t)(r * kRow128 + ((ch ^ (r & 7)) << 4));
-        if (r < nn) {
-          const int64_t tok = t0 + cc0 + r;
-          cp_async_16(in + so, kg + (tok * p.n_qk_heads + hq) * kD + ch * 8);
-          cp_async_16(in + kC * kRow128 + so, qg + (tok * p.n_qk_heads + hq) * kD + ch * 8);
-          cp_async_16(in + 2 * kC * kRow128 + so, vg + (tok * H + h) * kD + ch * 8);
-        } else {
-          *reinterpret_cast<uint4*>(in + so) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(in + kC * kRow128 + so) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(in + 2 * kC * kRow128 + so) = make_uint4(0, 0, 0, 0);
-        }
-      }
-      if (warp == 0) {
-        float* gin = reinterpret_cast<float*>(smem + kOffGin) + (ci & 1) * 2 * kC;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = 2 * lane + e;
-          if (t < nn) {
-            const int64_t gi = (int64_t)(t0 + cc0 + t) * H + h;
-            if (kGate) cp_async_4(gin + t, p.g + gi); else gin[t] = 1.0f;
-            if (Rule<RULE>::kUsesBeta) cp_async_4(gin + kC + t, p.beta + gi); else gin[kC + t] = 1.0f;
-          } else {
-            gin[t] = 1.0f;
-            gin[kC + t] = 0.0f;
-          }
-        }
-      }
-      cp_async_commit();
-    };
-
-    if (n_chunks > 0) stage(0);
-#pragma unroll 1
-    for (int ci = 0; ci < n_chunks; ++ci) {
-      const int c0 = ci * kC;
-      const int n = (n_tok - c0) < kC ? (n_tok - c0) : kC;
-      const int kOffK = kOffIn + (ci & 1) * kInBytes;
-      const int kOffQ = kOffK + kC * kRow128;
-      const int kOffV = kOffQ + kC * kRow128;
-      // ---- state copy (BF16) for this chunk's products
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        st_bf16x2(smem, swz(kOffS, srow0 + g8, j, kRow128) + 4 * t4, st[j][0], st[j][1]);
-        st_bf16x2(smem, swz(kOffS, srow0 + g8 + 8, j, kRow128) + 4 * t4, st[j][2], st[j][3]);
-      }
-      // ---- prefetch the next chunk, wait for this one
-      if (ci + 1 < n_chunks) {
-        stage(ci + 1);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
-      // ---- gates: log |gamma_t|, sign gamma_t (prefix over the chunk), b_t, and the
-      //      factored ratios gamma_t / gamma_s = A_t B_s around the chunk's middle
-      if (warp == 0) {
-        const float* gin = reinterpret_cast<const float*>(smem + kOffGin) + (ci & 1) * 2 * kC;
-        float lg[2], sg[2];
-        bool big = false;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = 2 * lane + e;
-          float a, bc, cc;
-          Rule<RULE>::coeffs(gin[t], gin[kC + t], a, bc, cc);
-          big |= fabsf(a) > 1.0f;
-          lg[e] = __logf(fmaxf(fabsf(a), 1e-30f));
-          sg[e] = a < 0.0f ? -1.0f : 1.0f;
-          sBt[t] = bc;
-        }
-        // inclusive prefix (sum of logs, product of signs) over 64 tokens, 2 per lane
-        float l = lg[0] + lg[1], sgn = sg[0] * sg[1];
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float lo = __shfl_up_sync(0xffffffffu, l, off);
-          const float so2 = __shfl_up_sync(0xffffffffu, sgn, off);
-          if (lane >= off) {
-            l += lo;
-            sgn *= so2;
-          }
-        }
-        const float lprev = l - (lg[0] + lg[1]), sprev = sgn * sg[0] * sg[1];  // exclusive (signs are +-1)
-        const float l0 = lprev + lg[0], s0 = sprev * sg[0];
-        sLg[2 * lane] = l0;
-        sSg[2 * lane] = s0;
-        sLg[2 * lane + 1] = l;
-        sSg[2 * lane + 1] = sgn;
-        sGm[2 * lane] = s0 * __expf(l0);
-        sGm[2 * lane + 1] = sgn * __expf(l);
-        const float lfirst = __shfl_sync(0xffffffffu, l0, 0), llast = __shfl_sync(0xffffffffu, l, 31);
-        const bool fact = !__any_sync(0xffffffffu, big) && (lfirst - llast) <= 80.0f;
-        const float m = 0.5f * (lfirst + llast);
-        sFa[2 * lane] = s0 * __expf(l0 - m);
-        sFb[2 * lane] = s0 * __expf(m - l0);
-        sFa[2 * lane + 1] = sgn * __expf(l - m);
-        sFb[2 * lane + 1] = sgn * __expf(m - l);
-        if (lane == 0) sFlag[0] = fact ? 1 : 0;
-      }
-      __syncthreads();
-      const bool fact = sFlag[0] != 0;
-
-      // ---- step 1: K K^T (warps 0-3, delta rules) and Q K^T (warps 4-7), rows [16 mt, +16)
-      if (kDelta || warp >= 4) {
-        float acc[8][4];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
-        const uint32_t abase = sbase + (warp < 4 ? kOffK : kOffQ);
-#pragma unroll
-        for (int kk = 0; kk < kD; kk += 16) {
-          uint32_t a[4];
-          lda(a, abase, kRow128, 16 * mt, kk, lane);
-#pragma unroll
-          for (int np = 0; np < 4; ++np) {
-            uint32_t b[4];
-            ldb_nk(b, sbase + kOffK, kRow128, 16 * np, kk, lane);
-            mma16816(acc[2 * np], a, b[0], b[1]);
-            mma16816(acc[2 * np + 1], a, b[2], b[3]);
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-#pragma unroll
-          for (int e = 0; e < 4; e += 2) {
-            const int r = 16 * mt + g8 + (e >> 1) * 8;
-            float v2[2];
-#pragma unroll
-            for (int f = 0; f < 2; ++f) {
-              const int s = 8 * j + 2 * t4 + f;
-              v2[f] = 0.0f;
-              if (s <= r) {  // gamma_r / gamma_s, only where it is used
-                const float ratio = fact ? sFa[r] * sFb[s] : sSg[r] * sSg[s] * __expf(sLg[r] - sLg[s]);
-                if (warp < 4) {
-                  if (s < r) v2[f] = sBt[r] * ratio * acc[j][e + f];
-                } else {
-                  v2[f] = ratio * acc[j][e + f];
-                }
-              }
-              if (warp < 4) sL[r * kLs + s] = v2[f];
-            }
-            if (warp >= 4) st_bf16x2(smem, swz(kOffP, r, j, kRow64) + 4 * t4, v2[0], v2[1]);
-          }
-        }
-      }
-      __syncthreads();
-
-      // ---- step 2 (delta rules): T = (I + L)^-1 by 16 x 16 blocks, written as FP32 (for the
-      //      block recursion) and as Tw = T diag(b gamma), Tu = T diag(b) (BF16, swizzled)
-      if (kDelta) {
-        // diagonal blocks: forward substitution, lane c < 16 of warp b owns column c
-        if (warp < 4) {
-          const int b0 = 16 * warp, c = lane & 15;
-          float col[16];
-#pragma unroll
-          for (int r = 0; r < 16; ++r) {
-            // row r of the block's L in 16-byte pieces (issued ahead of the dependent chain)
-            const float4* lr = reinterpret_cast<const float4*>(sL + (b0 + r) * kLs + b0);
-            float x = (r == c) ? 1.0f : 0.0f;
-#pragma unroll
-            for (int m = 0; m < (r + 3) / 4; ++m) {
-              const float4 l4 = lr[m];
-              const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (4 * m + e < r) x -= lv[e] * col[4 * m + e];
-            }
-            col[r] = (r < c) ? 0.0f : x;
-          }
-          const int sc = b0 + c;
-          const float fw = sBt[sc] * sGm[sc], fu = sBt[sc];
-#pragma unroll
-          for (int r = 0; r < 16; ++r) {
-            if (lane < 16) sT[(b0 + r) * kTs + sc] = col[r];
-            // pairs of columns (c, c + 1) into Tw / Tu
-            const float nw = __shfl_down_sync(0xffffffffu, col[r] * fw, 1);
-            const float nu = __shfl_down_sync(0xffffffffu, col[r] * fu, 1);
-            if (lane < 16 && (c & 1) == 0) {
-              const uint32_t off = swz(kOffTw, b0 + r, sc >> 3, kRow64) + 2 * (sc & 7);
-              st_bf16x2(smem, off, col[r] * fw, nw);
-              st_bf16x2(smem, off - kOffTw + kOffTu, col[r] * fu, nu);
-            }
-          }
-        }
-        __syncthreads();
-        // block row bi: T_{bi,j} = -T_{bi,bi} sum_{k=j}^{bi-1} L_{bi,k} T_{k,j}, warp j < bi
-#pragma unroll 1
-        for (int bi = 1; bi < 4; ++bi) {
-          if (warp < bi) {
-            const int bj = warp;
-            const int g = lane >> 2, t = lane & 3;
-            float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            for (int bk = bj; bk < bi; ++bk)
-              mma16x16x16_tf32(x, sL + (16 * bi) * kLs + 16 * bk, kLs, sT + (16 * bk) * kTs + 16 * bj, kTs, lane);
-            float* xs = sX + warp * 16 * kXs;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-              xs[g * kXs + 8 * nt + 2 * t] = x[nt][0];
-              xs[g * kXs + 8 * nt + 2 * t + 1] = x[nt][1];
-              xs[(g + 8) * kXs + 8 * nt + 2 * t] = x[nt][2];
-              xs[(g + 8) * kXs + 8 * nt + 2 * t + 1] = x[nt][3];
-            }
-            __syncwarp();
-            float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            mma16x16x16_tf32(y, sT + (16 * bi) * kTs + 16 * bi, kTs, xs, kXs, lane);
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-              for (int hlf = 0; hlf < 2; ++hlf) {
-                const int r = 16 * bi + g + 8 * hlf, c = 16 * bj + 8 * nt + 2 * t;
-                const float v0 = -y[nt][2 * hlf], v1 = -y[nt][2 * hlf + 1];
-                sT[r * kTs + c] = v0;
-                sT[r * kTs + c + 1] = v1;
-                const uint32_t off = swz(kOffTw, r, c >> 3, kRow64) + 2 * (c & 7);
-                st_bf16x2(smem, off, v0 * sBt[c] * sGm[c], v1 * sBt[c + 1] * sGm[c + 1]);
-                st_bf16x2(smem, off - kOffTw + kOffTu, v0 * sBt[c], v1 * sBt[c + 1]);
-              }
-            }
-          }
-          __syncthreads();
-        }
-      }
-
-      // ---- step 3: this warp's U~ block (rows 16 mt, cols 64 nh) and -W block (K columns 64 nh)
-      float accu[8][4];
-      if (kDelta) {
-        float accw[8][4];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          accu[j][0] = accu[j][1] = accu[j][2] = accu[j][3] = 0.0f;
-          accw[j][0] = accw[j][1] = accw[j][2] = accw[j][3] = 0.0f;
-        }
-        const uint32_t tw = sbase + kOffTw, tu = tw + kC * kRow64;
-#pragma unroll
-        for (int kk = 0; kk < kC; kk += 16) {
-          uint32_t au[4], aw[4];
-          lda(au, tu, kRow64, 16 * mt, kk, lane);
-          lda(aw, tw, kRow64, 16 * mt, kk, lane);
-#pragma unroll
-          for (int np = 0; np < 4; ++np) {
-            uint32_t b[4];
-            ldb_kn(b, sbase + kOffV, kRow128, 64 * nh + 16 * np, kk, lane);
-            mma16816(accu[2 * np], au, b[0], b[1]);
-            mma16816(accu[2 * np + 1], au, b[2], b[3]);
-            ldb_kn(b, sbase + kOffK, kRow128, 64 * nh + 16 * np, kk, lane);
-            mma16816(accw[2 * np], aw, b[0], b[1]);
-            mma16816(accw[2 * np + 1], aw, b[2], b[3]);
-          }
-        }
-        // -W into shared memory (the L / T space is free once Tw, Tu exist)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = 64 * nh + 8 * j;
-          st_bf16x2(smem, swz(kOffW, 16 * mt + g8, col >> 3, kRow128) + 4 * t4, -accw[j][0], -accw[j][1]);
-          st_bf16x2(smem, swz(kOffW, 16 * mt + g8 + 8, col >> 3, kRow128) + 4 * t4, -accw[j][2], -accw[j][3]);
-        }
-      } else {
-        // linear / gated: u_t = v_t
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = 64 * nh + 8 * j + 2 * t4;
-#pragma unroll
-          for (int e = 0; e < 4; e += 2) {
-            const int r = 16 * mt + g8 + (e >> 1) * 8;
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(smem + swz(kOffV, r, col >> 3, kRow128) + 2 * (col & 7));
-            accu[j][e] = bf16_lo(w);
-            accu[j][e + 1] = bf16_hi(w);
-          }
-        }
-      }
-      __syncthreads();
-
-      // ---- step 4: U = U~ - W S0 ;  O = gamma (.) Q S0  (rows 16 mt, cols 64 nh)
-      float acco[8][4];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acco[j][0] = acco[j][1] = acco[j][2] = acco[j][3] = 0.0f;
-#pragma unroll
-      for (int kk = 0; kk < kD; kk += 16) {
-        uint32_t aq[4], aw[4];
-        lda(aq, sbase + kOffQ, kRow128, 16 * mt, kk, lane);
-        if (kDelta) lda(aw, sbase + kOffW, kRow128, 16 * mt, kk, lane);
-#pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          uint32_t b[4];
-          ldb_kn(b, sbase + kOffS, kRow128, 64 * nh + 16 * np, kk, lane);
-          mma16816(acco[2 * np], aq, b[0], b[1]);
-          mma16816(acco[2 * np + 1], aq, b[2], b[3]);
-          if (kDelta) {
-            mma16816(accu[2 * np], aw, b[0], b[1]);
-            mma16816(accu[2 * np + 1], aw, b[2], b[3]);
-          }
-        }
-      }
-      const int rlo = 16 * mt + g8, rhi = rlo + 8;
-      const float glo = sGm[rlo], ghi = sGm[rhi];
-      const float gC = sGm[kC - 1];  // padded tokens have gate 1, so this is the last real token's
-      // gamma_C / gamma_t from the log difference (no 0 / 0 when gamma underflows)
-      const float slo = sSg[kC - 1] * sSg[rlo] * __expf(sLg[kC - 1] - sLg[rlo]);
-      const float shi = sSg[kC - 1] * sSg[rhi] * __expf(sLg[kC - 1] - sLg[rhi]);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        acco[j][0] *= glo;
-        acco[j][1] *= glo;
-        acco[j][2] *= ghi;
-        acco[j][3] *= ghi;
-        const int col = 64 * nh + 8 * j;
-        st_bf16x2(smem, swz(kOffU, rlo, col >> 3, kRow128) + 4 * t4, accu[j][0], accu[j][1]);
-        st_bf16x2(smem, swz(kOffU, rhi, col >> 3, kRow128) + 4 * t4, accu[j][2], accu[j][3]);
-        st_bf16x2(smem, swz(kOffUs, rlo, col >> 3, kRow128) + 4 * t4, accu[j][0] * slo, accu[j][1] * slo);
-        st_bf16x2(smem, swz(kOffUs, rhi, col >> 3, kRow128) + 4 * t4, accu[j][2] * shi, accu[j][3] * shi);
-      }
-      __syncthreads();
-
-      // ---- step 5: O += (Q K^T (.) M) U ; store O.   S = gamma_C S + K^T Us.
-#pragma unroll
-      for (int kk = 0; kk < kC; kk += 16) {
-        uint32_t a[4];
-        lda(a, sbase + kOffP, kRow64, 16 * mt, kk, lane);
-#pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          uint32_t b[4];
-          ldb_kn(b, sbase + kOffU, kRow128, 64 * nh + 16 * np, kk, lane);
-          mma16816(acco[2 * np], a, b[0], b[1]);
-          mma16816(acco[2 * np + 1], a, b[2], b[3]);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int col = 64 * nh + 8 * j + 2 * t4;
-        if (rlo < n) {
-          *reinterpret_cast<uint32_t*>(og + ((int64_t)(t0 + c0 + rlo) * H + h) * kD + col) =
-              pack_bf16x2(p.scale * acco[j][0], p.scale * acco[j][1]);
-        }
-        if (rhi < n) {
-          *reinterpret_cast<uint32_t*>(og + ((int64_t)(t0 + c0 + rhi) * H + h) * kD + col) =
-              pack_bf16x2(p.scale * acco[j][2], p.scale * acco[j][3]);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) st[j][e] *= gC;
-#pragma unroll
-      for (int kk = 0; kk < kC; kk += 16) {
-        uint32_t a[4];
-        lda_t(a, sbase + kOffK, kRow128, srow0, kk, lane);
-#pragma unroll
-        for (int np = 0; np < 8; ++np) {
-          uint32_t b[4];
-          ldb_kn(b, sbase + kOffUs, kRow128, 16 * np, kk, lane);
-          mma16816(st[2 * np], a, b[0], b[1]);
-          mma16816(st[2 * np + 1], a, b[2], b[3]);
-        }
-      }
-      __syncthreads();  // the next chunk overwrites K, Q, V, S, U
-    }
-
-    // ---- final state
-    const int64_t dbase = ((int64_t)ws * H + h) * (kD * kD);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-#pragma unroll
-      for (int e = 0; e < 4; e += 2) {
-        const int r = srow0 + g8 + (e >> 1) * 8, c = 8 * j + 2 * t4;
-        if (p.dst_dtype == LA_F32) {
-          *reinterpret_cast<float2*>(static_cast<float*>(p.dst) + dbase + r * kD + c) = make_float2(st[j][e], st[j][e + 1]);
-        } else {
-          *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.dst) + dbase + r * kD + c) =
-              pack_bf16x2(st[j][e], st[j][e + 1]);
-        }
-      }
-    }
-    __syncthreads();
-  }
-}
 
 // ---- the intra-chunk part on its own, per (chunk, head) tile: K K^T, the UT inverse
 //      T = (I + L)^-1 by forward substitution in FP32 (one column of T per lane),
@@ -884,26 +367,6 @@ cudaError_t launch_chunk_prep(const ScanParams& p, cudaStream_t stream) {
   if (grid <= 0) return cudaSuccess;
   chunk_prep_kernel<RULE><<<grid, chunk::kPThreads, chunk::kPSmem, stream>>>(p);
   return cudaGetLastError();
-}
-
-template <int RULE>
-cudaError_t launch_chunk_scan(const ScanParams& p, cudaStream_t stream) {
-  const void* fn = reinterpret_cast<const void*>(&chunk_scan_kernel<RULE>);
-  const int per_sm = prepare_kernel(fn, chunk::kThreads, chunk::kSmem);
-  if (per_sm <= 0) return cudaErrorInvalidConfiguration;
-  const int64_t units = (int64_t)p.n_seqs * p.n_v_heads;
-  const int64_t cap = (int64_t)device_sm_count() * per_sm;
-  const int grid = (int)(units < cap ? units : cap);
-  chunk_scan_kernel<RULE><<<grid, chunk::kThreads, chunk::kSmem, stream>>>(p);
-  return cudaGetLastError();
-}
-
-// The chunked prefill through the workspace for the linear and gated rules, which have no
-// intra-chunk inverse: the single fused kernel.
-template <int RULE>
-cudaError_t launch_chunk_scan_ws(const ScanParams& p, cudaStream_t stream) {
-  static_assert(!Rule<RULE>::kPredicts, "the delta rules take chunk_prep_kernel + chunk_tc_kernel");
-  return launch_chunk_scan<RULE>(p, stream);
 }
 
 }  // namespace la
