@@ -414,7 +414,13 @@ def test_scan_checkpoint_errors_reported():
     assert_close(np64(S[:4]), S_ref[:4], 2e-2, "checkpoints that fit are written")
 
 
-# ---- chunked tensor-core prefill (BF16 operands: compared at the BF16 tolerance) ----------
+# ---- chunked tensor-core prefill (BF16 operands) -------------------------------------------
+# Within a chunk the products take BF16 operands, so the chunked prefill agrees with the
+# oracle to BF16 precision, not to the FP32 1e-4: over sequences of up to a few hundred
+# tokens (every rule, gates and beta at the wide ranges too) its largest deviation stays
+# under 1e-2 of the largest value, half the general BF16 bound of 2e-2, which the full-size
+# prefill comparisons keep.
+CHUNK_TOL = 1e-2
 
 def _gpu_scan_chunked(inp, dst_dtype):
     n_seqs = inp.cu_seqlens.numel() - 1
@@ -439,8 +445,8 @@ def test_chunked_scan_vs_oracle(rule, dst):
     assert err == 0
     S_ref, o_ref, e = oracle_scan(inp, dst_dtype=dst)
     assert e == 0
-    assert_close(np64(S), S_ref, 2e-2, f"{rule}: final states")
-    assert_close(np64(o), o_ref, 2e-2, f"{rule}: outputs")
+    assert_close(np64(S), S_ref, CHUNK_TOL, f"{rule}: final states")
+    assert_close(np64(o), o_ref, CHUNK_TOL, f"{rule}: outputs")
 
 
 def test_chunked_scan_wide_gate_and_beta_ranges():
@@ -449,8 +455,8 @@ def test_chunked_scan_wide_gate_and_beta_ranges():
     S, o, err = _gpu_scan_chunked(inp, F32)
     S_ref, o_ref, _ = oracle_scan(inp, dst_dtype=F32)
     assert err == 0
-    assert_close(np64(S), S_ref, 2e-2, "wide-range final states")
-    assert_close(np64(o), o_ref, 2e-2, "wide-range outputs")
+    assert_close(np64(S), S_ref, CHUNK_TOL, "wide-range final states")
+    assert_close(np64(o), o_ref, CHUNK_TOL, "wide-range outputs")
 
 
 def _gpu_scan_chunked_ws(inp, dst_dtype):
@@ -481,8 +487,8 @@ def test_chunked_two_launches_vs_oracle(rule, dst):
     S2, o2, e2 = _gpu_scan_chunked_ws(inp, dst)
     assert e2 == 0
     S_ref, o_ref, _ = oracle_scan(inp, dst_dtype=dst)
-    assert_close(np64(S2), S_ref, 2e-2, f"{rule}: final states")
-    assert_close(np64(o2), o_ref, 2e-2, f"{rule}: outputs")
+    assert_close(np64(S2), S_ref, CHUNK_TOL, f"{rule}: final states")
+    assert_close(np64(o2), o_ref, CHUNK_TOL, f"{rule}: outputs")
     if rule in ("linear", "gated"):
         S1, o1, e1 = _gpu_scan_chunked(inp, dst)
         assert e1 == 0 and torch.equal(S1, S2) and torch.equal(o1, o2)
@@ -508,8 +514,8 @@ def test_chunked_two_launches_special_ranges(rule):
     S, o, err = _gpu_scan_chunked_ws(inp, F32)
     S_ref, o_ref, _ = oracle_scan(inp, dst_dtype=F32)
     assert err == 0
-    assert_close(np64(S), S_ref, 2e-2, f"{rule}: wide-range final states")
-    assert_close(np64(o), o_ref, 2e-2, f"{rule}: wide-range outputs")
+    assert_close(np64(S), S_ref, CHUNK_TOL, f"{rule}: wide-range final states")
+    assert_close(np64(o), o_ref, CHUNK_TOL, f"{rule}: wide-range outputs")
     inp = W.scan_inputs(lengths=[130, 64], n_qk_heads=1, n_v_heads=2, d_k=128, d_v=128, rule=rule,
                         io_dtype=BF16, seed=45, g_mode="one", beta_mode="zero", init="slots", init_dtype=F32)
     S, o, err = _gpu_scan_chunked_ws(inp, F32)
@@ -517,7 +523,7 @@ def test_chunked_two_launches_special_ranges(rule):
     S0 = inp.pool[inp.read_slot.long()].float()
     assert torch.equal(S, S0), "beta = 0, g = 1: the state passes through unchanged"
     S_ref, o_ref, _ = oracle_scan(inp, dst_dtype=F32)
-    assert_close(np64(o), o_ref, 2e-2, f"{rule}: readout of the unchanged state")
+    assert_close(np64(o), o_ref, CHUNK_TOL, f"{rule}: readout of the unchanged state")
 
 
 @pytest.mark.parametrize("rule", ["delta", "gated_delta"])
@@ -552,10 +558,10 @@ def test_chunked_two_launches_pool_slots_and_order():
     S_ref, o_ref, _ = oracle_scan(inp, dst_dtype=BF16)
     got = dst_t.cpu()
     for s in range(n_seqs):
-        assert_close(np64(got[int(write[s])]), S_ref[s], 2e-2, f"sequence {s} state in slot {int(write[s])}")
+        assert_close(np64(got[int(write[s])]), S_ref[s], CHUNK_TOL, f"sequence {s} state in slot {int(write[s])}")
     untouched = [i for i in range(9) if i not in write.tolist()]
     assert torch.all(got[untouched] == 3.0)
-    assert_close(np64(o.cpu()), o_ref, 2e-2, "outputs")
+    assert_close(np64(o.cpu()), o_ref, CHUNK_TOL, "outputs")
 
 
 def test_chunked_two_launches_prefill32_units():
@@ -596,8 +602,8 @@ def test_chunked_checkpoints(rule, dst):
                                   dst_dtype=dname(dst), io_dtype="bf16", ckpt_every=every, ckpt_cu=ckpt_cu,
                                   ckpt_slots=ckpt_slots)
     assert e == 0
-    assert_close(np64(S), S_ref, 2e-2, f"{rule}: final states and checkpoints")
-    assert_close(np64(o), o_ref, 2e-2, f"{rule}: outputs")
+    assert_close(np64(S), S_ref, CHUNK_TOL, f"{rule}: final states and checkpoints")
+    assert_close(np64(o), o_ref, CHUNK_TOL, f"{rule}: outputs")
     S1, o1, e1 = _gpu_scan_chunked(inp, dst)
     assert e1 == 0 and torch.equal(o, o1) and torch.equal(S[:len(lengths)], S1)
 
