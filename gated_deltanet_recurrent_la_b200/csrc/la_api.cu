@@ -88,8 +88,13 @@ la_status cuda_status(cudaError_t e) {
 
 bool uses_gate(la_rule r) { return r == LA_RULE_GATED || r == LA_RULE_GATED_DELTA || r == LA_RULE_KDA; }
 bool uses_beta(la_rule r) { return r == LA_RULE_DELTA || r == LA_RULE_GATED_DELTA || r == LA_RULE_KDA; }
-// the rules whose chunked prefill solves intra-chunk corrections (the two-launch form's workspace)
-bool chunk_inverse(la_rule r) { return r == LA_RULE_DELTA || r == LA_RULE_GATED_DELTA; }
+// the rules whose chunked prefill has an intra-chunk launch (the two-launch form's workspace):
+// the delta corrections of the delta rules, and kda's decay-scaled operands
+bool chunk_inverse(la_rule r) { return r == LA_RULE_DELTA || r == LA_RULE_GATED_DELTA || r == LA_RULE_KDA; }
+size_t chunk_ws_bytes(la_rule r, int64_t total_tokens, int64_t n_seqs, int64_t n_v_heads) {
+  if (r == LA_RULE_KDA) return la::chunk_kda_workspace_bytes(total_tokens, n_seqs, n_v_heads);
+  return chunk_inverse(r) ? la::chunk_workspace_bytes(total_tokens, n_seqs, n_v_heads) : 0;
+}
 // the gate array's alignment: kda's per-channel decays are moved in 16-byte pieces
 size_t gate_align(la_rule r) { return r == LA_RULE_KDA ? 16 : 4; }
 
@@ -311,7 +316,7 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
     if (ckpt_every > 0 && (ckpt_every % 64 != 0 || workspace)) return LA_ERR_UNSUPPORTED;
     if (workspace && chunk_inverse(rule)) {
       if (!aligned(workspace, 16)) return LA_ERR_ALIGN;
-      if (workspace_bytes < la::chunk_workspace_bytes(total_tokens, n_seqs, s.n_v_heads)) return LA_ERR_SHAPE;
+      if (workspace_bytes < chunk_ws_bytes(rule, total_tokens, n_seqs, s.n_v_heads)) return LA_ERR_SHAPE;
       fn = la::find_chunk_scan_ws(rule);
     } else {
       fn = la::find_chunk_scan(rule);
@@ -387,6 +392,12 @@ la_status la_state_scan_chunked(la_rule rule, const la_pool* src, const int32_t*
 
 size_t la_scan_chunked_workspace_bytes(int32_t total_tokens, int32_t n_seqs, int32_t n_v_heads) {
   return la::chunk_workspace_bytes(total_tokens, n_seqs, n_v_heads);
+}
+
+size_t la_scan_chunked_workspace_bytes_rule(la_rule rule, int32_t total_tokens, int32_t n_seqs,
+                                            int32_t n_v_heads) {
+  if (rule < LA_RULE_LINEAR || rule > LA_RULE_KDA) return 0;
+  return chunk_ws_bytes(rule, total_tokens, n_seqs, n_v_heads);
 }
 
 la_status la_state_scan_chunked_ws(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,

@@ -1,8 +1,10 @@
-// la_chunk.cu -- chunked tensor-core prefill kernels: the fused one-launch form (all four
-// rules, la_chunk_fused.cuh) and the two-launch form of the delta rules (la_chunk.cuh prep +
-// la_chunk_tc.cuh recurrence).
+// la_chunk.cu -- chunked tensor-core prefill kernels: the fused one-launch form (the four
+// scalar-gate rules, la_chunk_fused.cuh), the two-launch form of the delta rules
+// (la_chunk.cuh prep + la_chunk_tc.cuh recurrence) and the two-launch form of the
+// channel-wise gate (la_chunk_kda.cuh).
 #include "la_chunk.cuh"
 #include "la_chunk_fused.cuh"
+#include "la_chunk_kda.cuh"
 #include "la_chunk_tc.cuh"
 
 namespace la {
@@ -36,7 +38,11 @@ ScanLaunchFn find_chunk_scan_ws(int rule) {
     case LA_RULE_GATED: return &launch_chunk_fused<LA_RULE_GATED>;
     case LA_RULE_DELTA: return &launch_chunk_scan_ws_tc<LA_RULE_DELTA>;
     case LA_RULE_GATED_DELTA: return &launch_chunk_scan_ws_tc<LA_RULE_GATED_DELTA>;
+    case LA_RULE_KDA: return &launch_chunk_kda;
   }
   return nullptr;
+}
+size_t chunk_kda_workspace_bytes(int64_t total_tokens, int64_t n_seqs, int64_t n_v_heads) {
+  return kda_workspace_bytes(total_tokens, n_seqs, n_v_heads);
 }
 }  // namespace la

@@ -78,7 +78,7 @@ constexpr int kOffTw = kOffP + 2 * 8192;       // Tw [64 t][64 s]
 constexpr int kOffTu = kOffTw + 8192;          // Tu [64 t][64 s]
 constexpr int kLs = kC + 4;                    // padded row stride of L / T (fp32)
 constexpr int kOffL = kOffTu + 8192;           // L, then T in place [64][68] fp32
-constexpr int kXs = 24;
+constexpr int kXs = chunk::kXs;
 constexpr int kOffX = kOffL + kC * kLs * 4;    // [3][16][24] fp32, scratch of the block recursion
 // gate block of a stage (written by the loader): [0, 64) gamma_t, [64, 128) gamma_C / gamma_t,
 // [128, 192) A_t = gamma_t / e^m, [192, 256) B_t = e^m / gamma_t, [256, 320) log |gamma_t|,
@@ -591,74 +591,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
           scale_rows(st, 0, gbk, nv, false, tp);        // Q~ = diag(gamma) Q
           scale_rows(st, kC, gbk + kC, nv, true, tp);   // K~ (its only reader left is the state update)
         } else {
-          // T = (I + L)^-1 in place of L, by 16 x 16 blocks.  Diagonal block wi by forward
-          // substitution, lane c (and c + 16) owning column c; L's upper triangle is zero and
-          // the column starts at zero, so full 16-term rows are exact.
-          {
-            const int b0 = 16 * wi, cc = lane & 15;
-            float xc[16];
-#pragma unroll
-            for (int q = 0; q < 16; ++q) xc[q] = 0.0f;
-            const float4* lr = reinterpret_cast<const float4*>(sL + b0 * kLs + b0);
-            float4 l0 = lr[0], l1 = lr[1], l2 = lr[2], l3 = lr[3];
-#pragma unroll 1
-            for (int rr = 0; rr < 16; ++rr) {
-              // the next row's L while this row's sums run
-              const float4* ln = reinterpret_cast<const float4*>(sL + (b0 + (rr < 15 ? rr + 1 : rr)) * kLs + b0);
-              const float4 n0 = ln[0], n1 = ln[1], n2 = ln[2], n3 = ln[3];
-              const float a0 = fmaf(l0.x, xc[0], fmaf(l0.y, xc[1], fmaf(l0.z, xc[2], l0.w * xc[3])));
-              const float a1 = fmaf(l1.x, xc[4], fmaf(l1.y, xc[5], fmaf(l1.z, xc[6], l1.w * xc[7])));
-              const float a2 = fmaf(l2.x, xc[8], fmaf(l2.y, xc[9], fmaf(l2.z, xc[10], l2.w * xc[11])));
-              const float a3 = fmaf(l3.x, xc[12], fmaf(l3.y, xc[13], fmaf(l3.z, xc[14], l3.w * xc[15])));
-              const float xv = (rr == cc ? 1.0f : 0.0f) - ((a0 + a1) + (a2 + a3));
-#pragma unroll
-              for (int q = 0; q < 16; ++q) xc[q] = (q == rr) ? xv : xc[q];
-              l0 = n0;
-              l1 = n1;
-              l2 = n2;
-              l3 = n3;
-            }
-            __syncwarp();
-            if (lane < 16) {
-#pragma unroll
-              for (int rr = 0; rr < 16; ++rr) sL[(b0 + rr) * kLs + b0 + cc] = xc[rr];
-            }
-          }
-          named_bar_sync(kNbPrep, 128);
-          // block row bi: T_{bi,bj} = -D_bi sum_{bk=bj}^{bi-1} L_{bi,bk} T_{bk,bj}, warp bj < bi
-#pragma unroll 1
-          for (int bi = 1; bi < 4; ++bi) {
-            float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            if (wi < bi) {
-              const int bj = wi;
-              const int g8 = lane >> 2, t4 = lane & 3;
-              float xs[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll 1
-              for (int bk = bj; bk < bi; ++bk)
-                chunk::mma16x16x16_tf32(xs, sL + (16 * bi) * kLs + 16 * bk, kLs, sL + (16 * bk) * kLs + 16 * bj,
-                                        kLs, lane);
-              float* xw = sX + wi * 16 * kXs;
-#pragma unroll
-              for (int nt = 0; nt < 2; ++nt) {
-                *reinterpret_cast<float2*>(xw + g8 * kXs + 8 * nt + 2 * t4) = make_float2(xs[nt][0], xs[nt][1]);
-                *reinterpret_cast<float2*>(xw + (g8 + 8) * kXs + 8 * nt + 2 * t4) = make_float2(xs[nt][2], xs[nt][3]);
-              }
-              __syncwarp();
-              chunk::mma16x16x16_tf32(y, sL + (16 * bi) * kLs + 16 * bi, kLs, xw, kXs, lane);
-            }
-            named_bar_sync(kNbPrep, 128);  // row bi of L is read: its blocks may now take T
-            if (wi < bi) {
-              const int bj = wi;
-              const int g8 = lane >> 2, t4 = lane & 3;
-#pragma unroll
-              for (int nt = 0; nt < 2; ++nt) {
-                const int col = 16 * bj + 8 * nt + 2 * t4;
-                *reinterpret_cast<float2*>(sL + (16 * bi + g8) * kLs + col) = make_float2(-y[nt][0], -y[nt][1]);
-                *reinterpret_cast<float2*>(sL + (16 * bi + g8 + 8) * kLs + col) = make_float2(-y[nt][2], -y[nt][3]);
-              }
-            }
-            named_bar_sync(kNbPrep, 128);
-          }
+          chunk::ut_inverse64(sL, sX, wi, lane, kNbPrep);
           // Tw and Tu of chunk j - 1 must have been read (W_{j-1} and U~_{j-1} complete)
           if (j > 0 && !(ok = gwait(&bars[kWFull], (uint32_t)(j - 1) & 1u, abort_flag, tp, kNbPrep))) break;
           // Tw = T diag(b gamma), Tu = T diag(b) (BF16), the ten lower 16 x 16 blocks: block i

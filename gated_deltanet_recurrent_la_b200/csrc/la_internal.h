@@ -135,12 +135,15 @@ StepLaunchFn find_step_qgroups_bf16(int rule, int dk, int dv, int io);
 ScanLaunchFn find_scan_qgroups_f32io(int rule, int dk, int dv);
 ScanLaunchFn find_scan_qgroups_bf16io(int rule, int dk, int dv);
 
-// Chunked tensor-core prefill (d_k = d_v = 128, BF16 io); nullptr for an unknown rule.
-// The _ws form runs the intra-chunk inverses as a separate launch through ScanParams::workspace.
+// Chunked tensor-core prefill (d_k = d_v = 128, BF16 io); nullptr for a rule without it.
+// The _ws form runs the intra-chunk part as a separate launch through ScanParams::workspace
+// (the delta rules and kda; kda has only this form).
 ScanLaunchFn find_chunk_scan(int rule);
 ScanLaunchFn find_chunk_scan_ws(int rule);
-// workspace of the _ws form: one 16 KiB tile per (chunk slot, head)
+// workspace of the _ws form: one tile per (chunk slot, head), 17.9 KB for the delta rules,
+// 65 KB for kda
 size_t chunk_workspace_bytes(int64_t total_tokens, int64_t n_seqs, int64_t n_v_heads);
+size_t chunk_kda_workspace_bytes(int64_t total_tokens, int64_t n_seqs, int64_t n_v_heads);
 // the library's own fixed workspace on the current device: *addr = its device address,
 // *bytes = its size; the error of the device query or the symbol lookup otherwise
 cudaError_t chunk_noalloc_workspace(void** addr, size_t* bytes);

@@ -31,7 +31,8 @@ EXPORTS = ("la_state_bytes", "la_shape_supported", "la_state_step", "la_state_sc
            "la_state_scan_checkpointed", "la_state_scan_chunked_checkpointed", "la_state_step_qgroups",
            "la_state_scan_qgroups",
            "la_pool_slot_bytes", "la_state_pool_encode", "la_state_pool_decode", "la_state_step_conv",
-           "la_state_scan_conv", "la_scan_chunked_workspace_bytes", "la_state_scan_chunked_ws",
+           "la_state_scan_conv", "la_scan_chunked_workspace_bytes", "la_scan_chunked_workspace_bytes_rule",
+           "la_state_scan_chunked_ws",
            "la_state_scan_chunked_noalloc",
            "la_state_pool_copy",
            "la_state_pool_gather", "la_state_pool_scatter", "la_state_pool_zero", "la_state_check_slots",
@@ -109,6 +110,8 @@ def lib():
         L.la_state_scan_conv.restype = I32
         L.la_scan_chunked_workspace_bytes.argtypes = [I32, I32, I32]
         L.la_scan_chunked_workspace_bytes.restype = ctypes.c_size_t
+        L.la_scan_chunked_workspace_bytes_rule.argtypes = [ctypes.c_int, I32, I32, I32]
+        L.la_scan_chunked_workspace_bytes_rule.restype = ctypes.c_size_t
         L.la_state_scan_chunked_ws.argtypes = L.la_state_scan.argtypes[:-2] + [P, ctypes.c_size_t, P, P]
         L.la_state_scan_chunked_ws.restype = I32
         L.la_state_scan_chunked_noalloc.argtypes = L.la_state_scan.argtypes
@@ -243,10 +246,15 @@ def la_scan_chunked_workspace_bytes(total_tokens: int, n_seqs: int, n_v_heads: i
     return lib().la_scan_chunked_workspace_bytes(int(total_tokens), int(n_seqs), int(n_v_heads))
 
 
+def la_scan_chunked_workspace_bytes_rule(rule, total_tokens: int, n_seqs: int, n_v_heads: int) -> int:
+    return lib().la_scan_chunked_workspace_bytes_rule(RULES[rule] if isinstance(rule, str) else int(rule),
+                                                      int(total_tokens), int(n_seqs), int(n_v_heads))
+
+
 def la_state_scan_chunked_ws(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens, q, k, v, g,
                              beta, scale, o, workspace, err_word, seq_order=None, stream=None) -> int:
     """la_state_scan_chunked in two launches; workspace: a uint8 device tensor of at least
-    la_scan_chunked_workspace_bytes(...) bytes."""
+    la_scan_chunked_workspace_bytes_rule(rule, ...) bytes."""
     io = dtype_code(q.dtype)
     return lib().la_state_scan_chunked_ws(
         RULES[rule] if isinstance(rule, str) else int(rule), None if src is None else src.ref,

@@ -77,7 +77,7 @@
 extern "C" {
 #endif
 
-#define LA_ABI_VERSION 3
+#define LA_ABI_VERSION 4
 
 typedef enum {
     LA_RULE_LINEAR = 0,
@@ -208,7 +208,7 @@ la_status la_state_scan(la_rule rule, const la_pool *src, const int32_t *read_sl
  * sequences of 2,000 tokens, every rule, gates in [-1, 1] and beta in [0, 2] included).
  * Arguments, outputs and errors as la_state_scan.  Supported: d_k = d_v = 128 with BF16
  * q/k/v/o, the rules linear, gated, delta and gated_delta, gates of either sign
- * (LA_ERR_UNSUPPORTED otherwise, kda included: use la_state_scan). */
+ * (LA_ERR_UNSUPPORTED otherwise; kda has the two-launch form la_state_scan_chunked_ws). */
 la_status la_state_scan_chunked(la_rule rule, const la_pool *src, const int32_t *read_slot,
                                 const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
                                 const int32_t *cu_seqlens, int32_t total_tokens, const int32_t *seq_order,
@@ -216,21 +216,36 @@ la_status la_state_scan_chunked(la_rule rule, const la_pool *src, const int32_t 
                                 const float *g, const float *beta, float scale, void *o,
                                 int32_t *err_word, void *stream);
 
-/* la_state_scan_chunked in two launches: the intra-chunk part of every chunk (K K^T, the
- * triangular inverse T, Tw = T diag(beta gamma), Tu = T diag(beta)) as one parallel launch
- * writing a caller-owned workspace, then the recurrence over the chunks reading it, on the
- * fifth-generation tensor cores (tcgen05 MMAs, the state in tensor memory).  The
+/* la_state_scan_chunked in two launches: the intra-chunk part of every chunk as one parallel
+ * launch writing a caller-owned workspace, then the recurrence over the chunks reading it,
+ * on the fifth-generation tensor cores (tcgen05 MMAs, the state in tensor memory).  The
  * chunks are independent in the first launch, so it fills the SMs (several CTAs each)
- * instead of sitting on each sequence's critical path.  Same algorithm and precision as
+ * instead of sitting on each sequence's critical path.  Same precision as
  * la_state_scan_chunked (BF16 products, FP32 accumulation and state), not bit for bit.
+ *   delta rules      the first launch forms K K^T, the triangular inverse T,
+ *                    Tw = T diag(beta gamma) and Tu = T diag(beta) (17.9 KB per chunk and head)
+ *   kda              the channel-wise gate ("Kimi Linear": S <- (I - beta k k^T) Diag(alpha) S
+ *                    + beta k v^T): the chunk's decay products Gamma_t (d_k vectors) are
+ *                    absorbed into the operands, Q (.) Gamma, K (.) Gamma and
+ *                    K (.) Gamma_C / Gamma, and into the intra-chunk products [Q; K] K^T, whose
+ *                    ratios Gamma_t / Gamma_s are factored around the middle of each 16-token
+ *                    block; the first launch writes those operands, P, Tw = T diag(beta) and
+ *                    Gamma_C (65 KB per chunk and head).  Each token's decay magnitude is
+ *                    taken within [e^-8, e^8]: magnitudes below e^-8, zero included, act as
+ *                    e^-8 (sign kept), a change of at most e^-8 (3.4e-4) of a decayed state
+ *                    row; within 1e-2 of la_state_scan for decays in [-1, 1] and beta in [0, 2].
  *   workspace        device, 16-byte aligned, at least
- *                    la_scan_chunked_workspace_bytes(total_tokens, n_seqs, H_v) bytes;
+ *                    la_scan_chunked_workspace_bytes_rule(rule, total_tokens, n_seqs, H_v)
+ *                    bytes (la_scan_chunked_workspace_bytes: the same for the delta rules);
  *                    contents are scratch (overwritten, not read back by the caller)
- * Other arguments, supported set and errors as la_state_scan_chunked; for the delta rules
- * LA_ERR_SHAPE when workspace_bytes is too small and LA_ERR_NULL for a NULL workspace.  The
- * linear and gated rules have no inverse and run the one-launch form: the workspace and
- * its size are ignored (NULL allowed, never touched). */
+ * Other arguments, supported set and errors as la_state_scan_chunked (kda added); for the
+ * delta rules and kda LA_ERR_SHAPE when workspace_bytes is too small and LA_ERR_NULL for a
+ * NULL workspace.  The linear and gated rules have no intra-chunk launch and run the
+ * one-launch form: the workspace and its size are ignored (NULL allowed, never touched), and
+ * la_scan_chunked_workspace_bytes_rule returns 0 for them (and for an unknown rule). */
 size_t la_scan_chunked_workspace_bytes(int32_t total_tokens, int32_t n_seqs, int32_t n_v_heads);
+size_t la_scan_chunked_workspace_bytes_rule(la_rule rule, int32_t total_tokens, int32_t n_seqs,
+                                            int32_t n_v_heads);
 la_status la_state_scan_chunked_ws(la_rule rule, const la_pool *src, const int32_t *read_slot,
                                    const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
                                    const int32_t *cu_seqlens, int32_t total_tokens,
@@ -248,10 +263,10 @@ la_status la_state_scan_chunked_ws(la_rule rule, const la_pool *src, const int32
  * library pays the 256 MiB per device, callers of the other entry points included.  It
  * stays reserved until the process exits (or the device is reset).  The array is
  * shared by every call on a device: calls must not run concurrently on one device (the
- * caller orders them, for example on one stream).  A call of a delta rule whose workspace
- * would exceed the array (la_scan_chunked_workspace_bytes(total_tokens, n_seqs, H_v) >
- * 256 MiB) returns LA_ERR_SHAPE before launching anything; the linear and gated rules do
- * not use the array and have no such limit.  A failed device query or symbol lookup
+ * caller orders them, for example on one stream).  A call of a delta rule or kda whose
+ * workspace would exceed the array (la_scan_chunked_workspace_bytes_rule(rule,
+ * total_tokens, n_seqs, H_v) > 256 MiB) returns LA_ERR_SHAPE before launching anything;
+ * the linear and gated rules do not use the array and have no such limit.  A failed device query or symbol lookup
  * returns LA_ERR_CUDA.  Other arguments and errors as la_state_scan_chunked. */
 la_status la_state_scan_chunked_noalloc(la_rule rule, const la_pool *src, const int32_t *read_slot,
                                         const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,

@@ -179,7 +179,7 @@ def test_chunked_scan_supported_set(lib):
         dst = pool(shape=shape)
         return lib.la_state_scan_chunked(rule, None, None, ctypes.byref(dst), None, 2, P(A), 10, None, P(A), P(A),
                                          P(A), io, P(A), P(A), 1.0, P(A), P(A), None)
-    assert call(rule=4) == L.LA_ERR_UNSUPPORTED  # kda: token-serial scan only
+    assert call(rule=4) == L.LA_ERR_UNSUPPORTED  # kda: the two-launch form only
     assert call(shape=(2, 4, 64, 64)) == L.LA_ERR_UNSUPPORTED
     assert call(shape=(2, 4, 128, 64)) == L.LA_ERR_UNSUPPORTED
     assert call(io=0) == L.LA_ERR_UNSUPPORTED
@@ -197,6 +197,46 @@ def test_chunked_workspace_size(lib):
         tiles = (T + 63) // 64 + n + 1
         assert b(T, n, H) == head + tiles * H * tile
     assert b(10, 0, 4) == head + 2 * 4 * tile and b(-1, 1, 1) == 0
+
+
+def test_chunked_workspace_size_per_rule(lib):
+    """The workspace of the two-launch prefill per rule: the delta rules' tiles as above,
+    kda's 65 KB tiles (the decay-scaled Q, K twice, K, P, Tw and Gamma_C of one chunk and
+    head, 1024 bytes apart), none for the linear and gated rules or an unknown rule."""
+    b = L.la_scan_chunked_workspace_bytes
+    r = L.la_scan_chunked_workspace_bytes_rule
+    for T, n, H in [(1, 1, 1), (65, 2, 4), (172058, 32, 32)]:
+        assert r("delta", T, n, H) == r("gated_delta", T, n, H) == b(T, n, H)
+        assert r("linear", T, n, H) == r("gated", T, n, H) == 0
+        assert r(7, T, n, H) == 0 and r(-1, T, n, H) == 0
+    head = r("kda", 0, 1, 1) - (r("kda", 0, 1, 2) - r("kda", 0, 1, 1))
+    tile = (r("kda", 0, 1, 2) - r("kda", 0, 1, 1)) // 2
+    assert head >= 16 and head % 16 == 0 and tile % 1024 == 0
+    assert tile >= 3 * 64 * 128 * 2 + 2 * 64 * 64 * 2 + 128 * 4
+    for T, n, H in [(1, 1, 1), (64, 1, 32), (65, 2, 4), (172058, 32, 32)]:
+        assert r("kda", T, n, H) == head + ((T + 63) // 64 + n + 1) * H * tile
+    assert r("kda", -1, 1, 1) == 0
+
+
+def test_chunked_kda_host_errors(lib):
+    """kda on the chunked path: the two-launch entry point requires a workspace of kda's
+    size; the one-launch and checkpointed chunked entry points have no kda form."""
+    dst = pool()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    need = L.la_scan_chunked_workspace_bytes_rule("kda", 10, 2, 4)
+
+    def ws_call(ws, nbytes):
+        return lib.la_state_scan_chunked_ws(4, None, None, ctypes.byref(dst), None, 2, P(A), 10, None, P(A), P(A),
+                                            P(A), 1, P(A), P(A), 1.0, P(A), P(ws), nbytes, P(A), None)
+    assert ws_call(None, 0) == L.LA_ERR_NULL
+    assert ws_call(A, need - 1) == L.LA_ERR_SHAPE
+    assert ws_call(A, L.la_scan_chunked_workspace_bytes(10, 2, 4)) == L.LA_ERR_SHAPE  # the delta size is too small
+    assert lib.la_state_scan_chunked(4, None, None, ctypes.byref(dst), None, 2, P(A), 10, None, P(A), P(A), P(A), 1,
+                                     P(A), P(A), 1.0, P(A), P(A), None) == L.LA_ERR_UNSUPPORTED
+    ck = (ctypes.c_int32 * 3)(0, 0, 0)
+    assert lib.la_state_scan_chunked_checkpointed(4, None, None, ctypes.byref(dst), None, 2, P(A), 10, None, P(A),
+                                                  P(A), P(A), 1, P(A), P(A), 1.0, P(A), 64, ck, ck, P(A),
+                                                  None) == L.LA_ERR_UNSUPPORTED
 
 
 def test_noalloc_lookup_failure_is_an_error(lib):

@@ -465,7 +465,7 @@ def _gpu_scan_chunked_ws(inp, dst_dtype):
     src = None if inp.pool is None else L.Pool(dev(inp.pool), inp.n_qk_heads)
     o = torch.full((inp.q.shape[0], inp.n_v_heads, inp.d_v), 5.0, dtype=inp.io_dtype, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    nbytes = L.la_scan_chunked_workspace_bytes(inp.q.shape[0], n_seqs, inp.n_v_heads)
+    nbytes = max(16, L.la_scan_chunked_workspace_bytes_rule(inp.rule, inp.q.shape[0], n_seqs, inp.n_v_heads))
     ws = torch.full((nbytes,), 0xAB, dtype=torch.uint8, device="cuda")
     st = L.la_state_scan_chunked_ws(inp.rule, src, dev(inp.read_slot), L.Pool(dst_t, inp.n_qk_heads), None,
                                     dev(inp.cu_seqlens), dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.g),
