@@ -132,6 +132,8 @@ KERNEL_SOURCES = {
     "chunk": ["la_chunk.cuh", "la_device.cuh"],
     "chunk_tc": ["la_chunk.cuh", "la_chunk_tc.cuh", "la_umma.cuh", "la_device.cuh"],
     "chunk_fused": ["la_chunk.cuh", "la_chunk_fused.cuh", "la_chunk_tc.cuh", "la_umma.cuh", "la_device.cuh"],
+    "chunk_kda": ["la_chunk.cuh", "la_chunk_kda.cuh", "la_chunk_fused.cuh", "la_chunk_tc.cuh", "la_umma.cuh",
+                  "la_device.cuh"],
     "pool": ["la_pool.cu"],
 }
 
@@ -378,6 +380,11 @@ def chunk_mma_flops(lengths, n_v_heads, d_k, d_v, rule):
     per = 2 * C * C * d_k + 2 * C * C * d_v + 4 * C * d_k * d_v
     if rule in ("delta", "gated_delta"):
         per += 4 * C * C * d_k + 2 * C * C * d_v + 2 * C * d_k * d_v
+    elif rule == "kda":
+        # [Q; K] against the decay-scaled keys by the ten 16 x 16 blocks on and below the
+        # diagonal, in place of Q K^T; then W = Tw K+, U~ = Tw V and W S0
+        per += 2 * (10 * 32 * 16) * d_k - 2 * C * C * d_k
+        per += 2 * C * C * d_k + 2 * C * C * d_v + 2 * C * d_k * d_v
     chunks = sum((int(n) + C - 1) // C for n in lengths)
     return chunks * n_v_heads * per
 
@@ -395,14 +402,17 @@ def chunk_roofline(run, inp, ms, peaks):
     mma_tf = chunk_mma_flops(lens, inp.n_v_heads, inp.d_k, inp.d_v, inp.rule) / (ms * 1e-3) / 1e12
     peak_tf = peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)
     two = run.ws is not None and inp.rule in ("delta", "gated_delta")
+    kda = inp.rule == "kda"
+    kernel = "chunk_kda" if kda else ("chunk_tc" if two else "chunk_fused")
     out = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
-           "traffic": recorded_traffic("chunk_tc" if two else "chunk_fused",
-                                       "prefill32" + (f"_ckpt{run.ckpt_every}" if run.ckpt_every else "")),
+           "traffic": recorded_traffic(kernel, ("kda_prefill32" if kda else "prefill32") +
+                                       (f"_ckpt{run.ckpt_every}" if run.ckpt_every else "")),
            "algorithmic_bytes_per_launch": nbytes,
            "method_tflops": flops / (ms * 1e-3) / 1e12,
            "mma_tflops": mma_tf, "mma_frac_of_bf16_peak": mma_tf / peak_tf,
            "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs; bf16_tflops for mma_frac)"}
-    out["kernel"] = ("la::chunk_prep_kernel (mma.sync) + la::chunk_tc_kernel (tcgen05)" if two
+    out["kernel"] = ("la::chunk_kda_prep_kernel (mma.sync) + la::chunk_kda_kernel (tcgen05)" if kda else
+                     "la::chunk_prep_kernel (mma.sync) + la::chunk_tc_kernel (tcgen05)" if two
                      else "la::chunk_fused_kernel (tcgen05)")
     return out
 
@@ -447,7 +457,7 @@ class ScanRunner:
             self.dst = L.Pool(self.dst_t, inp.n_qk_heads)
         self.ws = None
         if chunked == "ws":  # the two-launch form: the caller-owned workspace of the intra-chunk part
-            nb = L.la_scan_chunked_workspace_bytes(self.T, n_seqs, inp.n_v_heads)
+            nb = L.la_scan_chunked_workspace_bytes_rule(inp.rule, self.T, n_seqs, inp.n_v_heads)
             self.ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
         self.conv = None
         if "width" in inp.extra:  # the short causal convolution ahead of every token (fresh prefill)
@@ -853,7 +863,10 @@ def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_ev
             row["config"]["checkpoints"] = run.n_ckpt
         if chunked:
             row["config"]["algorithm"] = "chunked (64-token WY/UT form, BF16 tcgen05 products, FP32 state)" + \
-                ("; intra-chunk inverses as a separate parallel launch through a workspace, then the recurrence "
+                ("; the decay-scaled operands and intra-chunk products as a separate parallel launch through a "
+                 "workspace, then the recurrence with the state in tensor memory" if chunked == "ws" and
+                 inp.rule == "kda" else
+                 "; intra-chunk inverses as a separate parallel launch through a workspace, then the recurrence "
                  "with the state in tensor memory" if chunked == "ws" else
                  "; one launch, the intra-chunk inverses computed on chip beside the recurrence")
             row["roofline"] = chunk_roofline(run, inp, ms, peaks)
@@ -988,6 +1001,9 @@ def main():
         torch.cuda.empty_cache()
         rows["prefill32_chunked_ckpt256"] = measure_row("prefill32", max(3, min(a.steps, 50)), a.warmup, world,
                                                         peaks, sm_count, None, ckpt_every=256, chunked=True)
+        torch.cuda.empty_cache()
+        rows["kda_prefill32_chunked"] = measure_row("kda_prefill32", max(3, min(a.steps, 50)), a.warmup, world,
+                                                    peaks, sm_count, None, chunked="ws")
         torch.cuda.empty_cache()
         pool_run = PoolRunner()
         pms = time_back_to_back(pool_run, min(a.steps, 500), a.warmup, world)
