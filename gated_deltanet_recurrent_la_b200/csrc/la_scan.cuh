@@ -50,6 +50,18 @@
 #ifndef LA_SCAN_COLS
 #define LA_SCAN_COLS 4
 #endif
+// resident units (CTAs) per SM that the scan's register budget is held to: three for the
+// plain scan (168 registers, no spills: twelve warps per SM hide more of the FMA and
+// shuffle latencies), two with checkpoints (whose bookkeeping would spill at three)
+#ifndef LA_SCAN_MIN_BLOCKS
+#define LA_SCAN_MIN_BLOCKS 3
+#endif
+#ifndef LA_SCAN_MIN_BLOCKS_CKPT
+#define LA_SCAN_MIN_BLOCKS_CKPT 2
+#endif
+#ifndef LA_SCAN_MIN_BLOCKS_CONV
+#define LA_SCAN_MIN_BLOCKS_CONV 2
+#endif
 
 namespace la {
 
@@ -690,7 +702,7 @@ template <int RULE, int DK, int DV, typename IT, bool QGRP, bool CONV = false>
 cudaError_t launch_scan(const ScanParams& p, cudaStream_t stream) {
   using C = ScanCfg<DK, DV, IT, Rule<RULE>::kChannelGate, QGRP ? kMaxQueryGroup : 1, CONV>;
   if constexpr (CONV) {
-    constexpr int kMinBlocks = 2;
+    constexpr int kMinBlocks = LA_SCAN_MIN_BLOCKS_CONV;
     const void* fn = reinterpret_cast<const void*>(&scan_kernel<RULE, DK, DV, IT, kMinBlocks, false, false, true>);
     const int per_sm = prepare_kernel(fn, C::kThreads, C::kSmem);
     if (per_sm <= 0) return cudaErrorInvalidConfiguration;
@@ -700,11 +712,12 @@ cudaError_t launch_scan(const ScanParams& p, cudaStream_t stream) {
     scan_kernel<RULE, DK, DV, IT, kMinBlocks, false, false, true><<<grid, C::kThreads, C::kSmem, stream>>>(p);
     return cudaGetLastError();
   }
-  constexpr int kMinBlocks = 2;  // two CTAs (units) per SM
+  constexpr int kMinBlocks = LA_SCAN_MIN_BLOCKS;
+  constexpr int kMinBlocksCk = LA_SCAN_MIN_BLOCKS_CKPT;
   // checkpoints are a separate instantiation so that the plain scan's loop carries no
   // checkpoint bookkeeping (the query-group direction has none)
   const bool ck = !QGRP && p.ckpt_every > 0;
-  const void* fn = ck ? reinterpret_cast<const void*>(&scan_kernel<RULE, DK, DV, IT, kMinBlocks, !QGRP, QGRP>)
+  const void* fn = ck ? reinterpret_cast<const void*>(&scan_kernel<RULE, DK, DV, IT, kMinBlocksCk, !QGRP, QGRP>)
                       : reinterpret_cast<const void*>(&scan_kernel<RULE, DK, DV, IT, kMinBlocks, false, QGRP>);
   const int per_sm = prepare_kernel(fn, C::kThreads, C::kSmem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;
@@ -712,7 +725,7 @@ cudaError_t launch_scan(const ScanParams& p, cudaStream_t stream) {
   const int64_t cap = (int64_t)device_sm_count() * per_sm;
   const int grid = (int)(units < cap ? units : cap);
   if (ck)
-    scan_kernel<RULE, DK, DV, IT, kMinBlocks, !QGRP, QGRP><<<grid, C::kThreads, C::kSmem, stream>>>(p);
+    scan_kernel<RULE, DK, DV, IT, kMinBlocksCk, !QGRP, QGRP><<<grid, C::kThreads, C::kSmem, stream>>>(p);
   else
     scan_kernel<RULE, DK, DV, IT, kMinBlocks, false, QGRP><<<grid, C::kThreads, C::kSmem, stream>>>(p);
   return cudaGetLastError();
