@@ -17,6 +17,15 @@ ScanLaunchFn find_chunk_scan(int rule) {
   }
   return nullptr;
 }
+ScanLaunchFn find_chunk_scan_conv(int rule) {
+  switch (rule) {
+    case LA_RULE_LINEAR: return &launch_chunk_fused<LA_RULE_LINEAR, true>;
+    case LA_RULE_GATED: return &launch_chunk_fused<LA_RULE_GATED, true>;
+    case LA_RULE_DELTA: return &launch_chunk_fused<LA_RULE_DELTA, true>;
+    case LA_RULE_GATED_DELTA: return &launch_chunk_fused<LA_RULE_GATED_DELTA, true>;
+  }
+  return nullptr;
+}
 size_t chunk_workspace_bytes(int64_t total_tokens, int64_t n_seqs, int64_t n_v_heads) {
   if (total_tokens < 0 || n_seqs < 0 || n_v_heads <= 0) return 0;
   const int64_t tiles = (total_tokens + chunk::kC - 1) / chunk::kC + n_seqs + 1;

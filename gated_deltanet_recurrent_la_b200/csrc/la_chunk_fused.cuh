@@ -102,6 +102,7 @@ enum Bar {
   kOFull,           // outputs of a chunk in tensor memory (MMA commit)
   kOFree,           // outputs read
   kDrain,           // every MMA issued has completed
+  kConvDone,        // the convolution of a chunk's q, k, v is in its stage (with the convolution)
   kNumBars
 };
 constexpr int kOffMisc = kOffBar + kNumBars * 8;  // [0] tensor-memory base, [1] abort
@@ -247,7 +248,13 @@ __device__ __forceinline__ void scale_rows(unsigned char* st, int row0, const fl
 
 }  // namespace fused
 
-template <int RULE>
+// CONV: the short causal convolution (and SiLU, q/k unit length) runs on the raw q, k, v of
+// each staged chunk, in place, by the output group, two chunks ahead of its outputs: thread
+// tp owns channel tp of q, k and v for a whole unit, with its weights and the window of its
+// last W - 1 raw inputs in registers (read from the history at the read slot when the unit
+// starts, written to the history at the write slot when it ends).  The issuer forms a
+// chunk's [Q; K] K^T only once its convolution is done.
+template <int RULE, bool CONV = false>
 __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const ScanParams p,
                                                                          const __grid_constant__ TcMaps maps) {
   using namespace fused;
@@ -420,11 +427,11 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
         umma::commit(&bars[kG1Full]);
       };
       bool ok = true;
-      if (n_total > 0 && (ok = W(kFull + 0, 0))) {
+      if (n_total > 0 && (ok = W(kFull + 0, 0) && (!CONV || W(kConvDone, 0)))) {
         umma::fence_after();
         g1(0);
       }
-      if (ok && n_total > 1 && (ok = W(kFull + 1, 0) && W(kG1Free, 0))) {
+      if (ok && n_total > 1 && (ok = W(kFull + 1, 0) && W(kG1Free, 0) && (!CONV || W(kConvDone, 1)))) {
         umma::fence_after();
         g1(1);
       }
@@ -483,7 +490,9 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
         umma::commit(&bars[kOFull]);
         umma::commit(&bars[kEmpty + (int)(j % kStages)]);
         if (j + 2 < n_total) {
-          if (!(ok = W(kFull + (int)((j + 2) % kStages), (j + 2) / kStages) && W(kG1Free, j + 1))) break;
+          if (!(ok = W(kFull + (int)((j + 2) % kStages), (j + 2) / kStages) && W(kG1Free, j + 1) &&
+                     (!CONV || W(kConvDone, j + 2))))
+            break;
           umma::fence_after();
           g1(j + 2);
         }
@@ -669,6 +678,12 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
         }
       };
       if (nch == 0) {
+        if (CONV) {  // its convolution history passes through (zero without a read slot)
+          const int wm1 = p.conv_w - 1;
+          const __nv_bfloat16* hs = static_cast<const __nv_bfloat16*>(p.conv_src) + ((int64_t)x.rs * H + x.h) * 384 * wm1;
+          __nv_bfloat16* hd = static_cast<__nv_bfloat16*>(p.conv_dst) + ((int64_t)x.ws * H + x.h) * 384 * wm1;
+          for (int idx = tp; idx < 384 * wm1; idx += 128) hd[idx] = p.read_slot ? hs[idx] : __float2bfloat16_rn(0.0f);
+        }
         // empty sequence: the initial state (or zero) goes to the destination
         for (int i = 0; i < kD; ++i) {
           float v = 0.0f;
@@ -804,6 +819,113 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
     __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(smem + kOffWt);
     int64_t j = 0;
     bool ok = true;
+    // CONV: the chunks to convolve, two ahead of the outputs (unit round cr, its chunk cc of
+    // cn, global chunk jc), and the current unit's weights and windows of channel tp of q, k, v
+    int64_t cr = -1, jc = 0;
+    int cc = 0, cn = 0;
+    Unit cx{};
+    float cwt[3][kMaxConvWidth], cwin[3][kMaxConvWidth - 1];
+    const int cwid = CONV ? p.conv_w : 2;
+    // the next unit with tokens: its weights and windows (the history at its read slot, or zero)
+    auto conv_unit = [&]() {
+      for (;;) {
+        ++cr;
+        if (cr * G >= units) return;
+        const int64_t u = unit_of(cr, G, blockIdx.x);
+        if (u >= units) continue;
+        cx = unit_info(p, u);
+        if (cx.valid && cx.n_tok > 0) break;
+      }
+      cc = 0;
+      cn = (cx.n_tok + kC - 1) / kC;
+      const __nv_bfloat16* hs =
+          static_cast<const __nv_bfloat16*>(p.conv_src) + ((int64_t)cx.rs * H + cx.h) * 384 * (cwid - 1);
+#pragma unroll
+      for (int m = 0; m < 3; ++m) {
+        const float* wsrc = (m == 0 ? p.conv_wq : m == 1 ? p.conv_wk : p.conv_wv) +
+                            ((int64_t)(m == 2 ? cx.h : cx.hq) * kD + tp) * cwid;
+#pragma unroll
+        for (int jj = 0; jj < kMaxConvWidth; ++jj) cwt[m][jj] = jj < cwid ? __ldg(wsrc + jj) : 0.0f;
+#pragma unroll
+        for (int jj = 0; jj < kMaxConvWidth - 1; ++jj)
+          cwin[m][jj] = (jj < cwid - 1 && p.read_slot) ? __bfloat162float(hs[(m * kD + tp) * (cwid - 1) + jj]) : 0.0f;
+      }
+    };
+    // y_t = sum_j w[j] x_{t-W+1+j} of the chunk's real tokens, in place (then SiLU, then q_t and
+    // k_t to unit length); the window after the unit's last chunk is its new history
+    auto conv_chunk = [&]() -> bool {
+      const int s = (int)(jc % kStages);
+      if (!gwait(&bars[kFull + s], (uint32_t)(jc / kStages) & 1u, abort_flag, tp, kNbOut)) return false;
+      unsigned char* st = smem + s * kStageBytes;
+      const int nv = min(kC, cx.n_tok - cc * kC);
+      float wnew[3];
+#pragma unroll
+      for (int m = 0; m < 3; ++m) {
+        wnew[m] = 0.0f;
+#pragma unroll
+        for (int jj = 0; jj < kMaxConvWidth; ++jj)
+          if (jj == cwid - 1) wnew[m] = cwt[m][jj];
+      }
+#pragma unroll 1
+      for (int t = 0; t < nv; ++t) {
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+          __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(
+              st + (m == 2 ? kOffV + umma::panel_off(kC, t, tp) : kOffQK + umma::panel_off(128, m * kC + t, tp)));
+          const float xin = __bfloat162float(*e);
+          float y = wnew[m] * xin;
+#pragma unroll
+          for (int jj = 0; jj < kMaxConvWidth - 1; ++jj)
+            if (jj < cwid - 1) y = fmaf(cwt[m][jj], cwin[m][jj], y);
+#pragma unroll
+          for (int jj = 0; jj < kMaxConvWidth - 1; ++jj)
+            cwin[m][jj] = jj < cwid - 2 ? cwin[m][jj + 1] : (jj == cwid - 2 ? xin : cwin[m][jj]);
+          if (p.conv_act) y = __fdividef(y, 1.0f + __expf(-y));
+          *e = __float2bfloat16_rn(y);
+        }
+      }
+      named_bar_sync(kNbOut, 128);  // every channel of the chunk is convolved
+      if (p.conv_l2norm) {
+        // q_t (rows 0..63) and k_t (rows 64..127) to unit length: thread tp takes row tp
+        if ((tp & (kC - 1)) < nv) {
+          float ss = 0.0f;
+#pragma unroll 4
+          for (int ch = 0; ch < 16; ++ch) {
+            const uint4 w = *reinterpret_cast<const uint4*>(st + kOffQK + umma::panel_piece(128, tp, ch));
+            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) ss = fmaf(bf16_lo(wv[e2]), bf16_lo(wv[e2]), fmaf(bf16_hi(wv[e2]), bf16_hi(wv[e2]), ss));
+          }
+          const float rs = rsqrtf(ss + 1e-6f);
+#pragma unroll 4
+          for (int ch = 0; ch < 16; ++ch) {
+            uint4* ptr = reinterpret_cast<uint4*>(st + kOffQK + umma::panel_piece(128, tp, ch));
+            const uint4 w = *ptr;
+            *ptr = make_uint4(pack_bf16x2(bf16_lo(w.x) * rs, bf16_hi(w.x) * rs), pack_bf16x2(bf16_lo(w.y) * rs, bf16_hi(w.y) * rs),
+                              pack_bf16x2(bf16_lo(w.z) * rs, bf16_hi(w.z) * rs), pack_bf16x2(bf16_lo(w.w) * rs, bf16_hi(w.w) * rs));
+          }
+        }
+        named_bar_sync(kNbOut, 128);
+      }
+      if (++cc == cn) {
+        __nv_bfloat16* hd = static_cast<__nv_bfloat16*>(p.conv_dst) + ((int64_t)cx.ws * H + cx.h) * 384 * (cwid - 1);
+#pragma unroll
+        for (int m = 0; m < 3; ++m)
+#pragma unroll
+          for (int jj = 0; jj < kMaxConvWidth - 1; ++jj)
+            if (jj < cwid - 1) hd[(m * kD + tp) * (cwid - 1) + jj] = __float2bfloat16_rn(cwin[m][jj]);
+        conv_unit();
+      }
+      umma::fence_smem();  // the convolved rows -> tensor cores
+      named_bar_sync(kNbOut, 128);
+      if (tp == 0) mbar_arrive(&bars[kConvDone]);
+      ++jc;
+      return true;
+    };
+    if (CONV) {
+      conv_unit();
+      for (int i = 0; ok && i < 2 && jc < n_total; ++i) ok = conv_chunk();
+    }
     for (int64_t ru = 0; ok && ru * G < units; ++ru) {
       const int64_t u = unit_of(ru, G, blockIdx.x);
       if (u >= units) continue;
@@ -870,6 +992,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
           }
         }
         named_bar_sync(kNbOut, 128);  // the staging tile is read before the next W^T lands there
+        if (CONV && jc < n_total && !(ok = conv_chunk())) break;
       }
     }
   }
@@ -884,9 +1007,9 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
   }
 }
 
-template <int RULE>
+template <int RULE, bool CONV = false>
 cudaError_t launch_chunk_fused(const ScanParams& p, cudaStream_t stream) {
-  const void* fn = reinterpret_cast<const void*>(&chunk_fused_kernel<RULE>);
+  const void* fn = reinterpret_cast<const void*>(&chunk_fused_kernel<RULE, CONV>);
   const int per_sm = prepare_kernel(fn, fused::kThreads, fused::kSmem);
   // one CTA per SM: the kernel holds all of the SM's tensor memory
   if (per_sm != 1) return cudaErrorInvalidConfiguration;
@@ -901,7 +1024,7 @@ cudaError_t launch_chunk_fused(const ScanParams& p, cudaStream_t stream) {
   const int64_t cap = device_sm_count();
   const int grid = (int)(units < cap ? units : cap);
   if (grid <= 0) return cudaSuccess;
-  chunk_fused_kernel<RULE><<<grid, fused::kThreads, fused::kSmem, stream>>>(p, maps);
+  chunk_fused_kernel<RULE, CONV><<<grid, fused::kThreads, fused::kSmem, stream>>>(p, maps);
   return cudaGetLastError();
 }
 

@@ -31,7 +31,7 @@ EXPORTS = ("la_state_bytes", "la_shape_supported", "la_state_step", "la_state_sc
            "la_state_scan_checkpointed", "la_state_scan_chunked_checkpointed", "la_state_step_qgroups",
            "la_state_scan_qgroups",
            "la_pool_slot_bytes", "la_state_pool_encode", "la_state_pool_decode", "la_state_step_conv",
-           "la_state_scan_conv", "la_scan_chunked_workspace_bytes", "la_scan_chunked_workspace_bytes_rule",
+           "la_state_scan_conv", "la_state_scan_chunked_conv", "la_scan_chunked_workspace_bytes", "la_scan_chunked_workspace_bytes_rule",
            "la_state_scan_chunked_ws",
            "la_state_scan_chunked_noalloc",
            "la_state_pool_copy",
@@ -108,6 +108,8 @@ def lib():
         L.la_state_scan_conv.argtypes = L.la_state_scan.argtypes[:9] + [ctypes.POINTER(la_conv)] + \
             L.la_state_scan.argtypes[9:]
         L.la_state_scan_conv.restype = I32
+        L.la_state_scan_chunked_conv.argtypes = L.la_state_scan_conv.argtypes
+        L.la_state_scan_chunked_conv.restype = I32
         L.la_scan_chunked_workspace_bytes.argtypes = [I32, I32, I32]
         L.la_scan_chunked_workspace_bytes.restype = ctypes.c_size_t
         L.la_scan_chunked_workspace_bytes_rule.argtypes = [ctypes.c_int, I32, I32, I32]
@@ -339,6 +341,19 @@ def la_state_scan_conv(rule, src: Optional[Pool], read_slot, dst: Pool, write_sl
                                     conv.ref, _ptr(xq), _ptr(xk, xq.dtype), _ptr(xv, xq.dtype), io,
                                     _ptr(g, torch.float32), _ptr(beta, torch.float32), float(scale),
                                     _ptr(o, xq.dtype), _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_state_scan_chunked_conv(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens, conv: Conv,
+                               xq, xk, xv, g, beta, scale, o, err_word, seq_order=None, stream=None) -> int:
+    io = dtype_code(xq.dtype)
+    return lib().la_state_scan_chunked_conv(RULES[rule] if isinstance(rule, str) else int(rule),
+                                            None if src is None else src.ref, _ptr(read_slot, torch.int32), dst.ref,
+                                            _ptr(write_slot, torch.int32), int(cu_seqlens.numel() - 1),
+                                            _ptr(cu_seqlens, torch.int32), int(xq.shape[0]),
+                                            _ptr(seq_order, torch.int32), conv.ref, _ptr(xq), _ptr(xk, xq.dtype),
+                                            _ptr(xv, xq.dtype), io, _ptr(g, torch.float32),
+                                            _ptr(beta, torch.float32), float(scale), _ptr(o, xq.dtype),
+                                            _ptr(err_word, torch.int32), _stream(stream))
 
 
 def q8_tile_bytes(d_k: int, d_v: int, n_hp: int) -> int:

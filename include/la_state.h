@@ -358,6 +358,25 @@ la_status la_state_scan_conv(la_rule rule, const la_pool *src, const int32_t *re
                              const float *beta, float scale, void *o, int32_t *err_word,
                              void *stream);
 
+/* la_state_scan_chunked with the convolution of la_state_scan_conv ahead of every token, in
+ * the same launch ("Gated DeltaNet" glossary, Engineering details: the convolution fused
+ * with the recurrence): each chunk's raw xq, xk, xv are convolved (then SiLU, then q and k
+ * to unit length, as conv asks) in place in shared memory after they are staged, two chunks
+ * ahead of the chunk's products; each (sequence, head) carries the window of its last
+ * W - 1 raw inputs from chunk to chunk, starting from conv->hist_src at read_slot[s] (zero
+ * when read_slot is NULL) and leaving it in conv->hist_dst at write_slot[s] (an empty
+ * sequence passes its history through).  The convolved q, k, v are rounded to BF16 before
+ * the products (q and k normalised from the rounded values).  Supported: the scalar-gate
+ * rules, d_k = d_v = 128, BF16 io and histories (LA_ERR_UNSUPPORTED otherwise, kda
+ * included).  Other arguments and errors as la_state_scan_conv. */
+la_status la_state_scan_chunked_conv(la_rule rule, const la_pool *src, const int32_t *read_slot,
+                                     const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
+                                     const int32_t *cu_seqlens, int32_t total_tokens,
+                                     const int32_t *seq_order, const la_conv *conv, const void *xq,
+                                     const void *xk, const void *xv, la_dtype io, const float *g,
+                                     const float *beta, float scale, void *o, int32_t *err_word,
+                                     void *stream);
+
 /* The query-group direction of the ONNX LinearAttention operator ("Seven Architectures
  * ...", section "ONNX LinearAttention / FlashInfer": each KV head and its recurrent state
  * shared by a group of query heads, q_num_heads / kv_num_heads).  The state of head h is

@@ -239,6 +239,23 @@ def test_chunked_kda_host_errors(lib):
                                                   None) == L.LA_ERR_UNSUPPORTED
 
 
+def test_chunked_conv_host_errors(lib):
+    """The convolution on the chunked path: a conv description is required, kda and FP32 io
+    are not supported there, and a bad width is refused before any launch."""
+    dst = pool()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    conv = L.la_conv(4, 1, 1, A, A, A, A, A)
+
+    def call(rule=3, io=1, c=conv):
+        return lib.la_state_scan_chunked_conv(rule, None, None, ctypes.byref(dst), None, 2, P(A), 10, None,
+                                              None if c is None else ctypes.byref(c), P(A), P(A), P(A), io, P(A),
+                                              P(A), 1.0, P(A), P(A), None)
+    assert call(c=None) == L.LA_ERR_NULL
+    assert call(rule=4) == L.LA_ERR_UNSUPPORTED
+    assert call(io=0) == L.LA_ERR_UNSUPPORTED
+    assert call(c=L.la_conv(5, 1, 1, A, A, A, A, A)) == L.LA_ERR_UNSUPPORTED
+
+
 def test_noalloc_lookup_failure_is_an_error(lib):
     """The no-alloc prefill looks up the address of the library's own workspace before
     anything else; where that lookup fails (here: no CUDA device at all), the call reports

@@ -209,3 +209,127 @@ def test_conv_prefill32_units():
             assert_close(np64(S[s_, h]), ref[i, 0], tol_s, f"seq {s_} head {h} final state")
             assert_close(np64(o[t0:t1, h]), o_ref[int(ucu[i]):int(ucu[i + 1]), 0], tol_o, f"seq {s_} head {h} outputs")
             assert np.array_equal(np64(hnew[s_, h]), href[i, 0]), f"seq {s_} head {h} final history"
+
+
+# ---- the convolution inside the one-launch chunked prefill ------------------------------
+# The chunked prefill rounds its operands to BF16 (the convolved q, k, v included), so its
+# states and outputs are compared at the chunked tolerance (1e-2 of the largest value on
+# these sizes); the histories are exact copies of raw inputs on both sides.
+CHUNK_TOL = 1e-2
+
+
+def run_chunked_conv(inp, wq, wk, wv, width, act, l2, hist_src, n_dst, dst_dtype, read_slot=None, write_slot=None,
+                     seq_order=None):
+    H, dk, dv = inp.n_v_heads, inp.d_k, inp.d_v
+    dst_t = torch.full((n_dst, H, dk, dv), 3.0, dtype=dst_dtype, device="cuda")
+    hist_dst = torch.full((n_dst, H, 2 * dk + dv, width - 1), 9.0, dtype=inp.io_dtype, device="cuda")
+    src = None if inp.pool is None else L.Pool(dev(inp.pool), inp.n_qk_heads)
+    hs = None if hist_src is None else dev(hist_src)
+    conv = L.Conv(dev(wq), dev(wk), dev(wv), hs if hs is not None else hist_dst, hist_dst, activation=act,
+                  qk_l2norm=l2)
+    o = torch.full((inp.q.shape[0], H, dv), 5.0, dtype=inp.io_dtype, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.check(L.la_state_scan_chunked_conv(inp.rule, src, dev(read_slot), L.Pool(dst_t, inp.n_qk_heads),
+                                         dev(write_slot), dev(inp.cu_seqlens), conv, dev(inp.q), dev(inp.k),
+                                         dev(inp.v), dev(inp.g), dev(inp.beta), inp.scale, o, err,
+                                         seq_order=None if seq_order is None else dev(seq_order)))
+    torch.cuda.synchronize()
+    return dst_t.cpu(), hist_dst.cpu(), o.cpu(), int(err.item())
+
+
+@pytest.mark.parametrize("width", [2, 3, 4])
+@pytest.mark.parametrize("rule,act,l2", [("linear", 0, 0), ("linear", 1, 1), ("gated", 0, 0), ("gated", 1, 1),
+                                         ("delta", 0, 1), ("delta", 1, 1), ("gated_delta", 0, 1),
+                                         ("gated_delta", 1, 1)])
+def test_chunked_scan_conv(rule, act, l2, width):
+    """Sequences shorter than the window, empty, across chunk boundaries (64, 65, 130
+    tokens), two state heads per q/k head, histories read at permuted read slots and
+    written at other write slots, against the oracle's convolved scan.  The delta rules
+    take unit-length keys (their recurrence with raw convolution outputs, |k|^2 ~ d_k,
+    diverges within a hundred tokens on both sides)."""
+    lengths = [5, 0, 2, 130, 37, 64, 65]
+    n = len(lengths)
+    inp = W.scan_inputs(lengths=lengths, n_qk_heads=2, n_v_heads=4, d_k=128, d_v=128, rule=rule, state_dtype=F32,
+                        io_dtype=BF16, seed=130 + width + 3 * act, init="slots", init_dtype=F32, normalise_qk=False,
+                        pool_std=0.3)
+    wq, wk, wv = _conv_weights(2, 4, 128, 128, width, 13 + width)
+    hist = torch.randn(n, 4, 384, width - 1, generator=torch.Generator().manual_seed(18)).to(BF16)
+    ws = torch.tensor([2, 0, 4, 1, 3, 6, 5], dtype=torch.int32)
+    S, hnew, o, err = run_chunked_conv(inp, wq, wk, wv, width, act, l2, hist, n, F32, read_slot=inp.read_slot,
+                                       write_slot=ws)
+    assert err == 0
+    ref, href, o_ref, e = oracle.scan_conv(rule, 2, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k), np64(inp.v),
+                                           np64(inp.g), np64(inp.beta), inp.scale, wq.double().numpy(),
+                                           wk.double().numpy(), wv.double().numpy(), act=act, l2norm=l2,
+                                           conv_src=np64(hist), src_pool=np64(inp.pool),
+                                           read_slot=inp.read_slot.numpy(), dst_pool=np.zeros((n, 4, 128, 128)),
+                                           conv_dst=np.zeros((n, 4, 384, width - 1)), write_slot=ws.numpy(),
+                                           dst_dtype="f32", io_dtype="bf16")
+    assert e == 0
+    assert_close(np64(S), ref, CHUNK_TOL, f"{rule} W={width}: final states")
+    assert_close(np64(o), o_ref, CHUNK_TOL, f"{rule} W={width}: outputs")
+    assert np.array_equal(np64(hnew), href), "final histories are exact copies of inputs"
+
+
+def test_chunked_scan_conv_fresh_prefill_and_order():
+    """No read slots (zero histories, zero initial states), the sequences dealt longest
+    first, BF16 final states."""
+    lengths = [300, 3, 64, 129]
+    inp = W.scan_inputs(lengths=lengths, n_qk_heads=1, n_v_heads=2, d_k=128, d_v=128, rule="gated_delta",
+                        io_dtype=BF16, seed=141, normalise_qk=False)
+    wq, wk, wv = _conv_weights(1, 2, 128, 128, 4, 19)
+    order = torch.tensor([0, 3, 2, 1], dtype=torch.int32)
+    S, hnew, o, err = run_chunked_conv(inp, wq, wk, wv, 4, 1, 1, None, 4, BF16, seq_order=order)
+    assert err == 0
+    ref, href, o_ref, e = oracle.scan_conv("gated_delta", 1, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k),
+                                           np64(inp.v), np64(inp.g), np64(inp.beta), inp.scale, wq.double().numpy(),
+                                           wk.double().numpy(), wv.double().numpy(), act=1, l2norm=1,
+                                           dst_dtype="bf16", io_dtype="bf16")
+    assert e == 0
+    assert_close(np64(S), ref, CHUNK_TOL, "final states")
+    assert_close(np64(o), o_ref, CHUNK_TOL, "outputs")
+    assert np.array_equal(np64(hnew), href)
+
+
+def test_chunked_scan_conv_unsupported():
+    inp = W.scan_inputs(lengths=[10], n_qk_heads=1, n_v_heads=2, d_k=128, d_v=128, rule="kda", io_dtype=BF16,
+                        seed=142, normalise_qk=False)
+    wq, wk, wv = _conv_weights(1, 2, 128, 128, 4, 20)
+    dst_t = torch.zeros(1, 2, 128, 128, dtype=F32, device="cuda")
+    hist = torch.zeros(1, 2, 384, 3, dtype=BF16, device="cuda")
+    conv = L.Conv(dev(wq), dev(wk), dev(wv), hist, hist, activation=1, qk_l2norm=1)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o = torch.empty(10, 2, 128, dtype=BF16, device="cuda")
+    st = L.la_state_scan_chunked_conv("kda", None, None, L.Pool(dst_t, 1), None, dev(inp.cu_seqlens), conv,
+                                      dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.g), dev(inp.beta), 1.0, o, err)
+    assert st == L.LA_ERR_UNSUPPORTED
+
+
+def test_conv_prefill32_chunked_units():
+    """The full prefill workload with the convolution, through the chunked prefill with the
+    convolution in the same launch: every sequence on two heads and the longest on all 32
+    against the oracle's convolved scan, final histories exact."""
+    inp = W.conv_prefill32()
+    x = inp.extra
+    width, n = x["width"], inp.cu_seqlens.numel() - 1
+    S, hnew, o, err = run_chunked_conv(inp, x["w_q"], x["w_k"], x["w_v"], width, x["activation"], x["qk_l2norm"],
+                                       None, n, inp.state_dtype)
+    assert err == 0
+    cu = inp.cu_seqlens.numpy()
+    by_head = {}
+    for s_, h in prefill_picks(inp):
+        by_head.setdefault(h, []).append(s_)
+    for h, seqs in sorted(by_head.items()):
+        sub = scan_unit_inputs(inp, [(s_, h) for s_ in seqs])
+        ref, href, o_ref, e = oracle.scan_conv(
+            inp.rule, 1, sub.cu_seqlens.numpy(), np64(sub.q), np64(sub.k), np64(sub.v), np64(sub.g), np64(sub.beta),
+            inp.scale, x["w_q"][h:h + 1].double().numpy(), x["w_k"][h:h + 1].double().numpy(),
+            x["w_v"][h:h + 1].double().numpy(), act=x["activation"], l2norm=x["qk_l2norm"],
+            dst_dtype=dname(inp.state_dtype), io_dtype=dname(inp.io_dtype))
+        assert e == 0
+        ucu = sub.cu_seqlens.numpy()
+        for i, s_ in enumerate(seqs):
+            t0, t1 = int(cu[s_]), int(cu[s_ + 1])
+            assert_close(np64(S[s_, h]), ref[i, 0], 2e-2, f"seq {s_} head {h} final state")
+            assert_close(np64(o[t0:t1, h]), o_ref[int(ucu[i]):int(ucu[i + 1]), 0], 2e-2, f"seq {s_} head {h} outputs")
+            assert np.array_equal(np64(hnew[s_, h]), href[i, 0]), f"seq {s_} head {h} final history"
