@@ -403,9 +403,10 @@ def chunk_roofline(run, inp, ms, peaks):
     peak_tf = peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)
     two = run.ws is not None and inp.rule in ("delta", "gated_delta")
     kda = inp.rule == "kda"
+    conv = run.conv is not None
     kernel = "chunk_kda" if kda else ("chunk_tc" if two else "chunk_fused")
     out = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
-           "traffic": recorded_traffic(kernel, ("kda_prefill32" if kda else "prefill32") +
+           "traffic": recorded_traffic(kernel, ("kda_prefill32" if kda else "conv_prefill32" if conv else "prefill32") +
                                        (f"_ckpt{run.ckpt_every}" if run.ckpt_every else "")),
            "algorithmic_bytes_per_launch": nbytes,
            "method_tflops": flops / (ms * 1e-3) / 1e12,
@@ -413,7 +414,7 @@ def chunk_roofline(run, inp, ms, peaks):
            "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs; bf16_tflops for mma_frac)"}
     out["kernel"] = ("la::chunk_kda_prep_kernel (mma.sync) + la::chunk_kda_kernel (tcgen05)" if kda else
                      "la::chunk_prep_kernel (mma.sync) + la::chunk_tc_kernel (tcgen05)" if two
-                     else "la::chunk_fused_kernel (tcgen05)")
+                     else "la::chunk_fused_kernel (tcgen05)" + (", the convolution in the same launch" if conv else ""))
     return out
 
 
@@ -468,7 +469,12 @@ class ScanRunner:
                                activation=x["activation"], qk_l2norm=x["qk_l2norm"])
 
     def step(self, i=0, stream=None):
-        if self.conv is not None:
+        if self.conv is not None and self.chunked:
+            st = self.L.la_state_scan_chunked_conv(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu,
+                                                   self.conv, self.q, self.k, self.v, self.g, self.beta,
+                                                   self.inp.scale, self.o, self.err, seq_order=self.order,
+                                                   stream=stream)
+        elif self.conv is not None:
             st = self.L.la_state_scan_conv(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu,
                                            self.conv, self.q, self.k, self.v, self.g, self.beta, self.inp.scale,
                                            self.o, self.err, seq_order=self.order, stream=stream)
@@ -868,7 +874,8 @@ def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_ev
                  inp.rule == "kda" else
                  "; intra-chunk inverses as a separate parallel launch through a workspace, then the recurrence "
                  "with the state in tensor memory" if chunked == "ws" else
-                 "; one launch, the intra-chunk inverses computed on chip beside the recurrence")
+                 "; one launch, the intra-chunk inverses computed on chip beside the recurrence") + \
+                ("; the convolution of every staged chunk in the same launch" if run.conv is not None else "")
             row["roofline"] = chunk_roofline(run, inp, ms, peaks)
         else:
             row["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
@@ -1004,6 +1011,9 @@ def main():
         torch.cuda.empty_cache()
         rows["kda_prefill32_chunked"] = measure_row("kda_prefill32", max(3, min(a.steps, 50)), a.warmup, world,
                                                     peaks, sm_count, None, chunked="ws")
+        torch.cuda.empty_cache()
+        rows["conv_prefill32_chunked"] = measure_row("conv_prefill32", max(3, min(a.steps, 50)), a.warmup, world,
+                                                     peaks, sm_count, None, chunked=True)
         torch.cuda.empty_cache()
         pool_run = PoolRunner()
         pms = time_back_to_back(pool_run, min(a.steps, 500), a.warmup, world)

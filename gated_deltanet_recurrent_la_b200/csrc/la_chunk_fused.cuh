@@ -64,9 +64,11 @@ constexpr int kWarpMma = 1;
 constexpr int kWarpPrep = 2;   // warps 2..5
 constexpr int kWarpState = 6;  // warps 6..9
 constexpr int kWarpOut = 10;   // warps 10..13
+constexpr int kWarpConv = 14;  // warps 14, 15 (with the convolution)
 constexpr int kThreads = 14 * 32;
+constexpr int kThreadsConv = 16 * 32;
 // named barriers of the warp groups (0 is __syncthreads)
-constexpr uint32_t kNbPrep = 1, kNbState = 2, kNbOut = 3;
+constexpr uint32_t kNbPrep = 1, kNbState = 2, kNbOut = 3, kNbConv = 4;
 
 // shared memory (bytes from a 1024-byte aligned base); BF16 operands in 64-column panels
 constexpr int kStageBytes = 49152;
@@ -249,13 +251,14 @@ __device__ __forceinline__ void scale_rows(unsigned char* st, int row0, const fl
 }  // namespace fused
 
 // CONV: the short causal convolution (and SiLU, q/k unit length) runs on the raw q, k, v of
-// each staged chunk, in place, by the output group, two chunks ahead of its outputs: thread
-// tp owns channel tp of q, k and v for a whole unit, with its weights and the window of its
-// last W - 1 raw inputs in registers (read from the history at the read slot when the unit
-// starts, written to the history at the write slot when it ends).  The issuer forms a
-// chunk's [Q; K] K^T only once its convolution is done.
+// each staged chunk, in place, in a group of two more warps (14, 15) as soon as the chunk has
+// landed: thread tc owns the channel pair (2 tc, 2 tc + 1) of q, k and v for a whole unit,
+// with its weights and the window of its last W - 1 raw inputs in registers (read from the
+// history at the read slot when the unit starts, written to the history at the write slot
+// when it ends).  The issuer forms a chunk's [Q; K] K^T only once its convolution is done.
 template <int RULE, bool CONV = false>
-__global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const ScanParams p,
+__global__ void __launch_bounds__(CONV ? fused::kThreadsConv : fused::kThreads, 1)
+    chunk_fused_kernel(const ScanParams p,
                                                                          const __grid_constant__ TcMaps maps) {
   using namespace fused;
   constexpr bool kDelta = Rule<RULE>::kPredicts;
@@ -809,7 +812,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
       }
       umma::fence_before();
     }
-  } else {
+  } else if (warp < kWarpConv) {
     // ------------------------------------------------------------------ output group
     const int tp = tid - kWarpOut * 32;
     const int q4 = warp & 3;
@@ -819,113 +822,6 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
     __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(smem + kOffWt);
     int64_t j = 0;
     bool ok = true;
-    // CONV: the chunks to convolve, two ahead of the outputs (unit round cr, its chunk cc of
-    // cn, global chunk jc), and the current unit's weights and windows of channel tp of q, k, v
-    int64_t cr = -1, jc = 0;
-    int cc = 0, cn = 0;
-    Unit cx{};
-    float cwt[3][kMaxConvWidth], cwin[3][kMaxConvWidth - 1];
-    const int cwid = CONV ? p.conv_w : 2;
-    // the next unit with tokens: its weights and windows (the history at its read slot, or zero)
-    auto conv_unit = [&]() {
-      for (;;) {
-        ++cr;
-        if (cr * G >= units) return;
-        const int64_t u = unit_of(cr, G, blockIdx.x);
-        if (u >= units) continue;
-        cx = unit_info(p, u);
-        if (cx.valid && cx.n_tok > 0) break;
-      }
-      cc = 0;
-      cn = (cx.n_tok + kC - 1) / kC;
-      const __nv_bfloat16* hs =
-          static_cast<const __nv_bfloat16*>(p.conv_src) + ((int64_t)cx.rs * H + cx.h) * 384 * (cwid - 1);
-#pragma unroll
-      for (int m = 0; m < 3; ++m) {
-        const float* wsrc = (m == 0 ? p.conv_wq : m == 1 ? p.conv_wk : p.conv_wv) +
-                            ((int64_t)(m == 2 ? cx.h : cx.hq) * kD + tp) * cwid;
-#pragma unroll
-        for (int jj = 0; jj < kMaxConvWidth; ++jj) cwt[m][jj] = jj < cwid ? __ldg(wsrc + jj) : 0.0f;
-#pragma unroll
-        for (int jj = 0; jj < kMaxConvWidth - 1; ++jj)
-          cwin[m][jj] = (jj < cwid - 1 && p.read_slot) ? __bfloat162float(hs[(m * kD + tp) * (cwid - 1) + jj]) : 0.0f;
-      }
-    };
-    // y_t = sum_j w[j] x_{t-W+1+j} of the chunk's real tokens, in place (then SiLU, then q_t and
-    // k_t to unit length); the window after the unit's last chunk is its new history
-    auto conv_chunk = [&]() -> bool {
-      const int s = (int)(jc % kStages);
-      if (!gwait(&bars[kFull + s], (uint32_t)(jc / kStages) & 1u, abort_flag, tp, kNbOut)) return false;
-      unsigned char* st = smem + s * kStageBytes;
-      const int nv = min(kC, cx.n_tok - cc * kC);
-      float wnew[3];
-#pragma unroll
-      for (int m = 0; m < 3; ++m) {
-        wnew[m] = 0.0f;
-#pragma unroll
-        for (int jj = 0; jj < kMaxConvWidth; ++jj)
-          if (jj == cwid - 1) wnew[m] = cwt[m][jj];
-      }
-#pragma unroll 1
-      for (int t = 0; t < nv; ++t) {
-#pragma unroll
-        for (int m = 0; m < 3; ++m) {
-          __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(
-              st + (m == 2 ? kOffV + umma::panel_off(kC, t, tp) : kOffQK + umma::panel_off(128, m * kC + t, tp)));
-          const float xin = __bfloat162float(*e);
-          float y = wnew[m] * xin;
-#pragma unroll
-          for (int jj = 0; jj < kMaxConvWidth - 1; ++jj)
-            if (jj < cwid - 1) y = fmaf(cwt[m][jj], cwin[m][jj], y);
-#pragma unroll
-          for (int jj = 0; jj < kMaxConvWidth - 1; ++jj)
-            cwin[m][jj] = jj < cwid - 2 ? cwin[m][jj + 1] : (jj == cwid - 2 ? xin : cwin[m][jj]);
-          if (p.conv_act) y = __fdividef(y, 1.0f + __expf(-y));
-          *e = __float2bfloat16_rn(y);
-        }
-      }
-      named_bar_sync(kNbOut, 128);  // every channel of the chunk is convolved
-      if (p.conv_l2norm) {
-        // q_t (rows 0..63) and k_t (rows 64..127) to unit length: thread tp takes row tp
-        if ((tp & (kC - 1)) < nv) {
-          float ss = 0.0f;
-#pragma unroll 4
-          for (int ch = 0; ch < 16; ++ch) {
-            const uint4 w = *reinterpret_cast<const uint4*>(st + kOffQK + umma::panel_piece(128, tp, ch));
-            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int e2 = 0; e2 < 4; ++e2) ss = fmaf(bf16_lo(wv[e2]), bf16_lo(wv[e2]), fmaf(bf16_hi(wv[e2]), bf16_hi(wv[e2]), ss));
-          }
-          const float rs = rsqrtf(ss + 1e-6f);
-#pragma unroll 4
-          for (int ch = 0; ch < 16; ++ch) {
-            uint4* ptr = reinterpret_cast<uint4*>(st + kOffQK + umma::panel_piece(128, tp, ch));
-            const uint4 w = *ptr;
-            *ptr = make_uint4(pack_bf16x2(bf16_lo(w.x) * rs, bf16_hi(w.x) * rs), pack_bf16x2(bf16_lo(w.y) * rs, bf16_hi(w.y) * rs),
-                              pack_bf16x2(bf16_lo(w.z) * rs, bf16_hi(w.z) * rs), pack_bf16x2(bf16_lo(w.w) * rs, bf16_hi(w.w) * rs));
-          }
-        }
-        named_bar_sync(kNbOut, 128);
-      }
-      if (++cc == cn) {
-        __nv_bfloat16* hd = static_cast<__nv_bfloat16*>(p.conv_dst) + ((int64_t)cx.ws * H + cx.h) * 384 * (cwid - 1);
-#pragma unroll
-        for (int m = 0; m < 3; ++m)
-#pragma unroll
-          for (int jj = 0; jj < kMaxConvWidth - 1; ++jj)
-            if (jj < cwid - 1) hd[(m * kD + tp) * (cwid - 1) + jj] = __float2bfloat16_rn(cwin[m][jj]);
-        conv_unit();
-      }
-      umma::fence_smem();  // the convolved rows -> tensor cores
-      named_bar_sync(kNbOut, 128);
-      if (tp == 0) mbar_arrive(&bars[kConvDone]);
-      ++jc;
-      return true;
-    };
-    if (CONV) {
-      conv_unit();
-      for (int i = 0; ok && i < 2 && jc < n_total; ++i) ok = conv_chunk();
-    }
     for (int64_t ru = 0; ok && ru * G < units; ++ru) {
       const int64_t u = unit_of(ru, G, blockIdx.x);
       if (u >= units) continue;
@@ -992,8 +888,161 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
           }
         }
         named_bar_sync(kNbOut, 128);  // the staging tile is read before the next W^T lands there
-        if (CONV && jc < n_total && !(ok = conv_chunk())) break;
       }
+    }
+  } else if (CONV) {
+    // ------------------------------------------------------------------ convolution group
+    const int tc = tid - kWarpConv * 32;  // channel pair (2 tc, 2 tc + 1) of q, k and v
+    const int wid = p.conv_w;
+    const uint32_t piece = (uint32_t)(((2 * tc) & 63) >> 3);
+    const uint32_t pair_off[3] = {kOffQK + umma::panel_off(128, 0, 2 * tc), kOffQK + umma::panel_off(128, kC, 2 * tc),
+                                  kOffV + umma::panel_off(kC, 0, 2 * tc)};
+    // four taps over the window of the last three raw inputs and the current one (a narrower
+    // convolution's weights sit in the last taps, the others are zero)
+    float w[3][2][4], win[3][2][3];
+    int64_t jj = 0;
+    bool ok = true;
+    for (int64_t ru = 0; ok && ru * G < units; ++ru) {
+      const int64_t u = unit_of(ru, G, blockIdx.x);
+      if (u >= units) continue;
+      const Unit x = unit_info(p, u);
+      if (!x.valid || x.n_tok == 0) continue;  // an empty sequence's history: the state group
+      const int nch = (x.n_tok + kC - 1) / kC;
+      const __nv_bfloat16* hs =
+          static_cast<const __nv_bfloat16*>(p.conv_src) + ((int64_t)x.rs * H + x.h) * 384 * (wid - 1);
+#pragma unroll
+      for (int m = 0; m < 3; ++m) {
+        const float* wsrc = (m == 0 ? p.conv_wq : m == 1 ? p.conv_wk : p.conv_wv) +
+                            ((int64_t)(m == 2 ? x.h : x.hq) * kD + 2 * tc) * wid;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+#pragma unroll
+          for (int tap = 0; tap < 4; ++tap) {
+            const int src = tap - (4 - wid);  // tap multiplies x_{t-3+tap}
+            w[m][e][tap] = src >= 0 ? __ldg(wsrc + e * wid + src) : 0.0f;
+          }
+#pragma unroll
+          for (int sl = 0; sl < 3; ++sl) {
+            const int src = sl - (4 - wid);  // slot sl holds x_{t-3+sl}: history entry src
+            win[m][e][sl] =
+                (src >= 0 && p.read_slot) ? __bfloat162float(hs[(m * kD + 2 * tc + e) * (wid - 1) + src]) : 0.0f;
+          }
+        }
+      }
+      for (int c = 0; c < nch; ++c, ++jj) {
+        const int s = (int)(jj % kStages);
+        bool okc = true;
+        if (tc == 0) okc = fwait(&bars[kFull + s], (uint32_t)(jj / kStages) & 1u, abort_flag);
+        if (named_bar_or(kNbConv, 64, !okc)) {
+          ok = false;
+          break;
+        }
+        unsigned char* st = smem + s * kStageBytes;
+        const int nv = min(kC, x.n_tok - c * kC);
+        // blocks of 8 tokens: the row swizzle of a panel repeats every 8 rows, so the addresses
+        // within a block are constant offsets; tokens at or past nv are left as they are
+#pragma unroll 1
+        for (int t0 = 0; t0 < nv; t0 += 8) {
+          const int nr = min(8, nv - t0);  // real tokens of the block
+#pragma unroll
+          for (int m = 0; m < 3; ++m) {
+            const uint32_t base = pair_off[m] + t0 * 128 - (piece << 4);
+            uint32_t xr[8];
+#pragma unroll
+            for (int v8 = 0; v8 < 8; ++v8) xr[v8] = *reinterpret_cast<const uint32_t*>(st + base + v8 * 128 + ((piece ^ v8) << 4));
+            float y[2][8];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              // the inputs x_{t0-3} .. x_{t0+7}: the window, then the block's 8 rows
+              float xs[11];
+#pragma unroll
+              for (int i = 0; i < 3; ++i) xs[i] = win[m][e][i];
+#pragma unroll
+              for (int v8 = 0; v8 < 8; ++v8) xs[3 + v8] = e ? bf16_hi(xr[v8]) : bf16_lo(xr[v8]);
+#pragma unroll
+              for (int v8 = 0; v8 < 8; ++v8)
+                y[e][v8] = fmaf(w[m][e][3], xs[v8 + 3],
+                                fmaf(w[m][e][2], xs[v8 + 2], fmaf(w[m][e][1], xs[v8 + 1], w[m][e][0] * xs[v8])));
+              // the window after the block's real tokens: the last three of x_{t0-3} .. x_{t0+nr-1}
+              if (nr == 8) {
+#pragma unroll
+                for (int i = 0; i < 3; ++i) win[m][e][i] = xs[8 + i];
+              } else {
+#pragma unroll
+                for (int i = 0; i < 3; ++i) {
+                  float nw = xs[i];
+#pragma unroll
+                  for (int k = 1; k < 8; ++k)
+                    if (nr == k) nw = xs[k + i];
+                  win[m][e][i] = nw;
+                }
+              }
+            }
+            if (p.conv_act) {
+#pragma unroll
+              for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int v8 = 0; v8 < 8; ++v8) y[e][v8] = __fdividef(y[e][v8], 1.0f + __expf(-y[e][v8]));
+            }
+#pragma unroll
+            for (int v8 = 0; v8 < 8; ++v8)
+              if (v8 < nr)
+                *reinterpret_cast<uint32_t*>(st + base + v8 * 128 + ((piece ^ v8) << 4)) = pack_bf16x2(y[0][v8], y[1][v8]);
+          }
+        }
+        named_bar_sync(kNbConv, 64);  // every channel of the chunk is convolved
+        if (p.conv_l2norm) {
+          // q_t (rows 0..63) and k_t (rows 64..127) to unit length: thread tc takes rows tc, 64 + tc
+#pragma unroll 1
+          for (int rr = tc; rr < 128; rr += 64) {
+            if ((rr & (kC - 1)) >= nv) continue;
+            float ss = 0.0f;
+#pragma unroll 4
+            for (int ch = 0; ch < 16; ++ch) {
+              const uint4 q4 = *reinterpret_cast<const uint4*>(st + kOffQK + umma::panel_piece(128, rr, ch));
+              const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+              for (int e2 = 0; e2 < 4; ++e2)
+                ss = fmaf(bf16_lo(qw[e2]), bf16_lo(qw[e2]), fmaf(bf16_hi(qw[e2]), bf16_hi(qw[e2]), ss));
+            }
+            const float rs = rsqrtf(ss + 1e-6f);
+#pragma unroll 4
+            for (int ch = 0; ch < 16; ++ch) {
+              uint4* ptr = reinterpret_cast<uint4*>(st + kOffQK + umma::panel_piece(128, rr, ch));
+              const uint4 q4 = *ptr;
+              *ptr = make_uint4(pack_bf16x2(bf16_lo(q4.x) * rs, bf16_hi(q4.x) * rs),
+                                pack_bf16x2(bf16_lo(q4.y) * rs, bf16_hi(q4.y) * rs),
+                                pack_bf16x2(bf16_lo(q4.z) * rs, bf16_hi(q4.z) * rs),
+                                pack_bf16x2(bf16_lo(q4.w) * rs, bf16_hi(q4.w) * rs));
+            }
+          }
+          named_bar_sync(kNbConv, 64);
+        }
+        umma::fence_smem();  // the convolved rows -> tensor cores
+        named_bar_sync(kNbConv, 64);
+        // announced once the issuer has taken the previous chunk's convolution (its [Q; K] K^T
+        // completed), so that the barrier's phases never run two ahead of the issuer
+        if (tc == 0) {
+          if (jj > 0) okc = fwait(&bars[kG1Full], (uint32_t)(jj - 1) & 1u, abort_flag);
+          if (okc) mbar_arrive(&bars[kConvDone]);
+        }
+        if (named_bar_or(kNbConv, 64, !okc)) {
+          ok = false;
+          break;
+        }
+      }
+      if (!ok) break;
+      // the window after the unit's last token: its history at the write slot
+      __nv_bfloat16* hd = static_cast<__nv_bfloat16*>(p.conv_dst) + ((int64_t)x.ws * H + x.h) * 384 * (wid - 1);
+#pragma unroll
+      for (int m = 0; m < 3; ++m)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+          for (int sl = 0; sl < 3; ++sl) {
+            const int dst = sl - (4 - wid);
+            if (dst >= 0) hd[(m * kD + 2 * tc + e) * (wid - 1) + dst] = __float2bfloat16_rn(win[m][e][sl]);
+          }
     }
   }
 
@@ -1010,7 +1059,8 @@ __global__ void __launch_bounds__(fused::kThreads, 1) chunk_fused_kernel(const S
 template <int RULE, bool CONV = false>
 cudaError_t launch_chunk_fused(const ScanParams& p, cudaStream_t stream) {
   const void* fn = reinterpret_cast<const void*>(&chunk_fused_kernel<RULE, CONV>);
-  const int per_sm = prepare_kernel(fn, fused::kThreads, fused::kSmem);
+  constexpr int threads = CONV ? fused::kThreadsConv : fused::kThreads;
+  const int per_sm = prepare_kernel(fn, threads, fused::kSmem);
   // one CTA per SM: the kernel holds all of the SM's tensor memory
   if (per_sm != 1) return cudaErrorInvalidConfiguration;
   TcMaps maps;
@@ -1024,7 +1074,7 @@ cudaError_t launch_chunk_fused(const ScanParams& p, cudaStream_t stream) {
   const int64_t cap = device_sm_count();
   const int grid = (int)(units < cap ? units : cap);
   if (grid <= 0) return cudaSuccess;
-  chunk_fused_kernel<RULE, CONV><<<grid, fused::kThreads, fused::kSmem, stream>>>(p, maps);
+  chunk_fused_kernel<RULE, CONV><<<grid, threads, fused::kSmem, stream>>>(p, maps);
   return cudaGetLastError();
 }
 
