@@ -401,9 +401,9 @@ def chunk_roofline(run, inp, ms, peaks):
     gbs = nbytes / (ms * 1e-3) / 1e9
     mma_tf = chunk_mma_flops(lens, inp.n_v_heads, inp.d_k, inp.d_v, inp.rule) / (ms * 1e-3) / 1e12
     peak_tf = peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)
-    two = run.ws is not None and inp.rule in ("delta", "gated_delta")
-    kda = inp.rule == "kda"
     conv = run.conv is not None
+    two = run.ws is not None and inp.rule in ("delta", "gated_delta") and not conv
+    kda = inp.rule == "kda"
     kernel = "chunk_kda" if kda else ("chunk_tc" if two else "chunk_fused")
     out = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
            "traffic": recorded_traffic(kernel, ("kda_prefill32" if kda else "conv_prefill32" if conv else "prefill32") +
@@ -414,6 +414,7 @@ def chunk_roofline(run, inp, ms, peaks):
            "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs; bf16_tflops for mma_frac)"}
     out["kernel"] = ("la::chunk_kda_prep_kernel (mma.sync) + la::chunk_kda_kernel (tcgen05)" if kda else
                      "la::chunk_prep_kernel (mma.sync) + la::chunk_tc_kernel (tcgen05)" if two
+                     else "la::chunk_conv_kernel + la::chunk_fused_kernel (tcgen05)" if conv and run.ws is not None
                      else "la::chunk_fused_kernel (tcgen05)" + (", the convolution in the same launch" if conv else ""))
     return out
 
@@ -458,7 +459,8 @@ class ScanRunner:
             self.dst = L.Pool(self.dst_t, inp.n_qk_heads)
         self.ws = None
         if chunked == "ws":  # the two-launch form: the caller-owned workspace of the intra-chunk part
-            nb = L.la_scan_chunked_workspace_bytes_rule(inp.rule, self.T, n_seqs, inp.n_v_heads)
+            nb = (L.la_scan_chunked_conv_workspace_bytes(self.T, inp.n_v_heads) if "width" in inp.extra else
+                  L.la_scan_chunked_workspace_bytes_rule(inp.rule, self.T, n_seqs, inp.n_v_heads))
             self.ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
         self.conv = None
         if "width" in inp.extra:  # the short causal convolution ahead of every token (fresh prefill)
@@ -469,7 +471,12 @@ class ScanRunner:
                                activation=x["activation"], qk_l2norm=x["qk_l2norm"])
 
     def step(self, i=0, stream=None):
-        if self.conv is not None and self.chunked:
+        if self.conv is not None and self.ws is not None:
+            st = self.L.la_state_scan_chunked_conv_ws(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu,
+                                                      self.conv, self.q, self.k, self.v, self.g, self.beta,
+                                                      self.inp.scale, self.o, self.ws, self.err, seq_order=self.order,
+                                                      stream=stream)
+        elif self.conv is not None and self.chunked:
             st = self.L.la_state_scan_chunked_conv(self.inp.rule, self.src, self.read_slot, self.dst, None, self.cu,
                                                    self.conv, self.q, self.k, self.v, self.g, self.beta,
                                                    self.inp.scale, self.o, self.err, seq_order=self.order,
@@ -875,7 +882,9 @@ def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_ev
                  "; intra-chunk inverses as a separate parallel launch through a workspace, then the recurrence "
                  "with the state in tensor memory" if chunked == "ws" else
                  "; one launch, the intra-chunk inverses computed on chip beside the recurrence") + \
-                ("; the convolution of every staged chunk in the same launch" if run.conv is not None else "")
+                ("; the convolution as a launch of its own, its output through a workspace" if run.conv is not None
+                 and chunked == "ws" else
+                 "; the convolution of every staged chunk in the same launch" if run.conv is not None else "")
             row["roofline"] = chunk_roofline(run, inp, ms, peaks)
         else:
             row["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu, "unit": "TFLOP/s", "frac": tf / alu,
@@ -1014,6 +1023,9 @@ def main():
         torch.cuda.empty_cache()
         rows["conv_prefill32_chunked"] = measure_row("conv_prefill32", max(3, min(a.steps, 50)), a.warmup, world,
                                                      peaks, sm_count, None, chunked=True)
+        torch.cuda.empty_cache()
+        rows["conv_prefill32_chunked_two_launch"] = measure_row("conv_prefill32", max(3, min(a.steps, 50)), a.warmup,
+                                                                world, peaks, sm_count, None, chunked="ws")
         torch.cuda.empty_cache()
         pool_run = PoolRunner()
         pms = time_back_to_back(pool_run, min(a.steps, 500), a.warmup, world)

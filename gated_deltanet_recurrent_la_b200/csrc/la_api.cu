@@ -299,7 +299,7 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
   const bool q8 = dst->dtype == LA_Q8 || (read_slot && src->dtype == LA_Q8);
   if (q8 && (chunked || n_q_heads != 0)) return LA_ERR_UNSUPPORTED;
   if (conv) {
-    if (q8 || (chunked && workspace) || n_q_heads != 0 || ckpt_every > 0) return LA_ERR_UNSUPPORTED;
+    if (q8 || n_q_heads != 0 || ckpt_every > 0) return LA_ERR_UNSUPPORTED;
     if (conv->width < 2 || conv->width > la::kMaxConvWidth) return LA_ERR_UNSUPPORTED;
     if (!conv->w_q || !conv->w_k || !conv->w_v || !conv->hist_dst || (read_slot && !conv->hist_src))
       return LA_ERR_NULL;
@@ -310,7 +310,13 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
   la::ScanLaunchFn fn = nullptr;
   if (conv && chunked) {
     if (s.d_k != 128 || s.d_v != 128 || io != LA_BF16) return LA_ERR_UNSUPPORTED;
-    fn = la::find_chunk_scan_conv(rule);
+    if (workspace) {
+      if (!aligned(workspace, 16)) return LA_ERR_ALIGN;
+      if (workspace_bytes < la::chunk_conv_workspace_bytes(total_tokens, s.n_v_heads)) return LA_ERR_SHAPE;
+      fn = la::find_chunk_scan_conv_ws(rule);
+    } else {
+      fn = la::find_chunk_scan_conv(rule);
+    }
   } else if (conv) {
     fn = (io == LA_F32) ? la::find_scan_conv_f32io(rule, s.d_k, s.d_v) : la::find_scan_conv_bf16io(rule, s.d_k, s.d_v);
   } else if (chunked) {
@@ -473,6 +479,23 @@ la_status la_state_scan_chunked_conv(la_rule rule, const la_pool* src, const int
   if (!conv) return LA_ERR_NULL;
   return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, xq, xk, xv, io,
                    g, beta, scale, o, 0, nullptr, nullptr, err_word, stream, true, 0, conv);
+}
+
+size_t la_scan_chunked_conv_workspace_bytes(int32_t total_tokens, int32_t n_v_heads) {
+  return la::chunk_conv_workspace_bytes(total_tokens, n_v_heads);
+}
+
+la_status la_state_scan_chunked_conv_ws(la_rule rule, const la_pool* src, const int32_t* read_slot,
+                                        const la_pool* dst, const int32_t* write_slot, int32_t n_seqs,
+                                        const int32_t* cu_seqlens, int32_t total_tokens, const int32_t* seq_order,
+                                        const la_conv* conv, const void* xq, const void* xk, const void* xv,
+                                        la_dtype io, const float* g, const float* beta, float scale, void* o,
+                                        void* workspace, size_t workspace_bytes, int32_t* err_word, void* stream) {
+  if (!conv) return LA_ERR_NULL;
+  if (!workspace && n_seqs > 0) return LA_ERR_NULL;
+  return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, xq, xk, xv, io,
+                   g, beta, scale, o, 0, nullptr, nullptr, err_word, stream, true, 0, conv, workspace,
+                   workspace_bytes);
 }
 
 la_status la_state_scan_qgroups(la_rule rule, const la_pool* src, const int32_t* read_slot, const la_pool* dst,

@@ -140,8 +140,12 @@ ScanLaunchFn find_scan_qgroups_bf16io(int rule, int dk, int dv);
 // (the delta rules and kda; kda has only this form).
 ScanLaunchFn find_chunk_scan(int rule);
 ScanLaunchFn find_chunk_scan_ws(int rule);
-// the one-launch form with the short causal convolution ahead (scalar-gate rules)
+// the one-launch form with the short causal convolution ahead (scalar-gate rules), and the
+// two-launch form (the convolution's output through a workspace of
+// chunk_conv_workspace_bytes(T, H_v) bytes)
 ScanLaunchFn find_chunk_scan_conv(int rule);
+ScanLaunchFn find_chunk_scan_conv_ws(int rule);
+size_t chunk_conv_workspace_bytes(int64_t total_tokens, int64_t n_v_heads);
 // workspace of the _ws form: one tile per (chunk slot, head), 17.9 KB for the delta rules,
 // 65 KB for kda
 size_t chunk_workspace_bytes(int64_t total_tokens, int64_t n_seqs, int64_t n_v_heads);

@@ -31,7 +31,8 @@ EXPORTS = ("la_state_bytes", "la_shape_supported", "la_state_step", "la_state_sc
            "la_state_scan_checkpointed", "la_state_scan_chunked_checkpointed", "la_state_step_qgroups",
            "la_state_scan_qgroups",
            "la_pool_slot_bytes", "la_state_pool_encode", "la_state_pool_decode", "la_state_step_conv",
-           "la_state_scan_conv", "la_state_scan_chunked_conv", "la_scan_chunked_workspace_bytes", "la_scan_chunked_workspace_bytes_rule",
+           "la_state_scan_conv", "la_state_scan_chunked_conv", "la_state_scan_chunked_conv_ws",
+           "la_scan_chunked_conv_workspace_bytes", "la_scan_chunked_workspace_bytes", "la_scan_chunked_workspace_bytes_rule",
            "la_state_scan_chunked_ws",
            "la_state_scan_chunked_noalloc",
            "la_state_pool_copy",
@@ -110,6 +111,11 @@ def lib():
         L.la_state_scan_conv.restype = I32
         L.la_state_scan_chunked_conv.argtypes = L.la_state_scan_conv.argtypes
         L.la_state_scan_chunked_conv.restype = I32
+        L.la_state_scan_chunked_conv_ws.argtypes = L.la_state_scan_conv.argtypes[:-2] + [ctypes.c_void_p, ctypes.c_size_t] + \
+            L.la_state_scan_conv.argtypes[-2:]
+        L.la_state_scan_chunked_conv_ws.restype = I32
+        L.la_scan_chunked_conv_workspace_bytes.argtypes = [I32, I32]
+        L.la_scan_chunked_conv_workspace_bytes.restype = ctypes.c_size_t
         L.la_scan_chunked_workspace_bytes.argtypes = [I32, I32, I32]
         L.la_scan_chunked_workspace_bytes.restype = ctypes.c_size_t
         L.la_scan_chunked_workspace_bytes_rule.argtypes = [ctypes.c_int, I32, I32, I32]
@@ -354,6 +360,27 @@ def la_state_scan_chunked_conv(rule, src: Optional[Pool], read_slot, dst: Pool, 
                                             _ptr(xv, xq.dtype), io, _ptr(g, torch.float32),
                                             _ptr(beta, torch.float32), float(scale), _ptr(o, xq.dtype),
                                             _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_scan_chunked_conv_workspace_bytes(total_tokens: int, n_v_heads: int) -> int:
+    return lib().la_scan_chunked_conv_workspace_bytes(int(total_tokens), int(n_v_heads))
+
+
+def la_state_scan_chunked_conv_ws(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens,
+                                  conv: Conv, xq, xk, xv, g, beta, scale, o, workspace, err_word, seq_order=None,
+                                  stream=None) -> int:
+    """la_state_scan_chunked_conv in two launches; workspace: a uint8 device tensor of at
+    least la_scan_chunked_conv_workspace_bytes(...) bytes."""
+    io = dtype_code(xq.dtype)
+    return lib().la_state_scan_chunked_conv_ws(RULES[rule] if isinstance(rule, str) else int(rule),
+                                               None if src is None else src.ref, _ptr(read_slot, torch.int32),
+                                               dst.ref, _ptr(write_slot, torch.int32), int(cu_seqlens.numel() - 1),
+                                               _ptr(cu_seqlens, torch.int32), int(xq.shape[0]),
+                                               _ptr(seq_order, torch.int32), conv.ref, _ptr(xq), _ptr(xk, xq.dtype),
+                                               _ptr(xv, xq.dtype), io, _ptr(g, torch.float32),
+                                               _ptr(beta, torch.float32), float(scale), _ptr(o, xq.dtype),
+                                               _ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                                               _ptr(err_word, torch.int32), _stream(stream))
 
 
 def q8_tile_bytes(d_k: int, d_v: int, n_hp: int) -> int:

@@ -377,6 +377,25 @@ la_status la_state_scan_chunked_conv(la_rule rule, const la_pool *src, const int
                                      const float *beta, float scale, void *o, int32_t *err_word,
                                      void *stream);
 
+/* la_state_scan_chunked_conv in two launches: the convolution of every (chunk, state head)
+ * as a launch of its own (each chunk reads the raw rows before it, or the history at the
+ * read slot, so every chunk is independent), writing the convolved q, k, v of every state
+ * head to a caller-owned workspace, then the chunked prefill reading them.  Same results as
+ * la_state_scan_chunked_conv up to the order of the products (histories identical).
+ *   workspace        device, 16-byte aligned, at least
+ *                    la_scan_chunked_conv_workspace_bytes(total_tokens, H_v) bytes (a header
+ *                    and 3 T H_v 128 BF16 values); contents are scratch
+ * LA_ERR_NULL for a NULL workspace, LA_ERR_SHAPE when it is too small; other arguments,
+ * supported set and errors as la_state_scan_chunked_conv. */
+size_t la_scan_chunked_conv_workspace_bytes(int32_t total_tokens, int32_t n_v_heads);
+la_status la_state_scan_chunked_conv_ws(la_rule rule, const la_pool *src, const int32_t *read_slot,
+                                        const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
+                                        const int32_t *cu_seqlens, int32_t total_tokens,
+                                        const int32_t *seq_order, const la_conv *conv, const void *xq,
+                                        const void *xk, const void *xv, la_dtype io, const float *g,
+                                        const float *beta, float scale, void *o, void *workspace,
+                                        size_t workspace_bytes, int32_t *err_word, void *stream);
+
 /* The query-group direction of the ONNX LinearAttention operator ("Seven Architectures
  * ...", section "ONNX LinearAttention / FlashInfer": each KV head and its recurrent state
  * shared by a group of query heads, q_num_heads / kv_num_heads).  The state of head h is

@@ -254,6 +254,19 @@ def test_chunked_conv_host_errors(lib):
     assert call(rule=4) == L.LA_ERR_UNSUPPORTED
     assert call(io=0) == L.LA_ERR_UNSUPPORTED
     assert call(c=L.la_conv(5, 1, 1, A, A, A, A, A)) == L.LA_ERR_UNSUPPORTED
+    # the two-launch form: a workspace of the convolved q, k, v (header + 3 T H_v 128 BF16)
+    need = L.la_scan_chunked_conv_workspace_bytes(10, 4)
+    assert need == L.la_scan_chunked_conv_workspace_bytes(0, 4) + 3 * 10 * 4 * 128 * 2
+    assert L.la_scan_chunked_conv_workspace_bytes(-1, 4) == 0
+
+    def ws_call(ws, nbytes, rule=3):
+        return lib.la_state_scan_chunked_conv_ws(rule, None, None, ctypes.byref(dst), None, 2, P(A), 10, None,
+                                                 ctypes.byref(conv), P(A), P(A), P(A), 1, P(A), P(A), 1.0, P(A),
+                                                 P(ws), nbytes, P(A), None)
+    assert ws_call(None, 0) == L.LA_ERR_NULL
+    assert ws_call(A, need - 16) == L.LA_ERR_SHAPE
+    assert ws_call(A + 8, need) == L.LA_ERR_ALIGN
+    assert ws_call(A, need, rule=4) == L.LA_ERR_UNSUPPORTED
 
 
 def test_noalloc_lookup_failure_is_an_error(lib):

@@ -219,7 +219,10 @@ CHUNK_TOL = 1e-2
 
 
 def run_chunked_conv(inp, wq, wk, wv, width, act, l2, hist_src, n_dst, dst_dtype, read_slot=None, write_slot=None,
-                     seq_order=None):
+                     seq_order=None, form="one"):
+    """form "one": la_state_scan_chunked_conv (the convolution in the chunked kernel);
+    "ws": la_state_scan_chunked_conv_ws (the convolution as its own launch, its output
+    through a workspace filled with NaN bytes beforehand)."""
     H, dk, dv = inp.n_v_heads, inp.d_k, inp.d_v
     dst_t = torch.full((n_dst, H, dk, dv), 3.0, dtype=dst_dtype, device="cuda")
     hist_dst = torch.full((n_dst, H, 2 * dk + dv, width - 1), 9.0, dtype=inp.io_dtype, device="cuda")
@@ -229,19 +232,28 @@ def run_chunked_conv(inp, wq, wk, wv, width, act, l2, hist_src, n_dst, dst_dtype
                   qk_l2norm=l2)
     o = torch.full((inp.q.shape[0], H, dv), 5.0, dtype=inp.io_dtype, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    L.check(L.la_state_scan_chunked_conv(inp.rule, src, dev(read_slot), L.Pool(dst_t, inp.n_qk_heads),
-                                         dev(write_slot), dev(inp.cu_seqlens), conv, dev(inp.q), dev(inp.k),
-                                         dev(inp.v), dev(inp.g), dev(inp.beta), inp.scale, o, err,
-                                         seq_order=None if seq_order is None else dev(seq_order)))
+    order = None if seq_order is None else dev(seq_order)
+    if form == "ws":
+        nbytes = L.la_scan_chunked_conv_workspace_bytes(inp.q.shape[0], H)
+        ws = torch.full((nbytes,), 0xFF, dtype=torch.uint8, device="cuda")
+        L.check(L.la_state_scan_chunked_conv_ws(inp.rule, src, dev(read_slot), L.Pool(dst_t, inp.n_qk_heads),
+                                                dev(write_slot), dev(inp.cu_seqlens), conv, dev(inp.q), dev(inp.k),
+                                                dev(inp.v), dev(inp.g), dev(inp.beta), inp.scale, o, ws, err,
+                                                seq_order=order))
+    else:
+        L.check(L.la_state_scan_chunked_conv(inp.rule, src, dev(read_slot), L.Pool(dst_t, inp.n_qk_heads),
+                                             dev(write_slot), dev(inp.cu_seqlens), conv, dev(inp.q), dev(inp.k),
+                                             dev(inp.v), dev(inp.g), dev(inp.beta), inp.scale, o, err, seq_order=order))
     torch.cuda.synchronize()
     return dst_t.cpu(), hist_dst.cpu(), o.cpu(), int(err.item())
 
 
+@pytest.mark.parametrize("form", ["one", "ws"])
 @pytest.mark.parametrize("width", [2, 3, 4])
 @pytest.mark.parametrize("rule,act,l2", [("linear", 0, 0), ("linear", 1, 1), ("gated", 0, 0), ("gated", 1, 1),
                                          ("delta", 0, 1), ("delta", 1, 1), ("gated_delta", 0, 1),
                                          ("gated_delta", 1, 1)])
-def test_chunked_scan_conv(rule, act, l2, width):
+def test_chunked_scan_conv(rule, act, l2, width, form):
     """Sequences shorter than the window, empty, across chunk boundaries (64, 65, 130
     tokens), two state heads per q/k head, histories read at permuted read slots and
     written at other write slots, against the oracle's convolved scan.  The delta rules
@@ -256,7 +268,7 @@ def test_chunked_scan_conv(rule, act, l2, width):
     hist = torch.randn(n, 4, 384, width - 1, generator=torch.Generator().manual_seed(18)).to(BF16)
     ws = torch.tensor([2, 0, 4, 1, 3, 6, 5], dtype=torch.int32)
     S, hnew, o, err = run_chunked_conv(inp, wq, wk, wv, width, act, l2, hist, n, F32, read_slot=inp.read_slot,
-                                       write_slot=ws)
+                                       write_slot=ws, form=form)
     assert err == 0
     ref, href, o_ref, e = oracle.scan_conv(rule, 2, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k), np64(inp.v),
                                            np64(inp.g), np64(inp.beta), inp.scale, wq.double().numpy(),
@@ -271,7 +283,8 @@ def test_chunked_scan_conv(rule, act, l2, width):
     assert np.array_equal(np64(hnew), href), "final histories are exact copies of inputs"
 
 
-def test_chunked_scan_conv_fresh_prefill_and_order():
+@pytest.mark.parametrize("form", ["one", "ws"])
+def test_chunked_scan_conv_fresh_prefill_and_order(form):
     """No read slots (zero histories, zero initial states), the sequences dealt longest
     first, BF16 final states."""
     lengths = [300, 3, 64, 129]
@@ -279,7 +292,7 @@ def test_chunked_scan_conv_fresh_prefill_and_order():
                         io_dtype=BF16, seed=141, normalise_qk=False)
     wq, wk, wv = _conv_weights(1, 2, 128, 128, 4, 19)
     order = torch.tensor([0, 3, 2, 1], dtype=torch.int32)
-    S, hnew, o, err = run_chunked_conv(inp, wq, wk, wv, 4, 1, 1, None, 4, BF16, seq_order=order)
+    S, hnew, o, err = run_chunked_conv(inp, wq, wk, wv, 4, 1, 1, None, 4, BF16, seq_order=order, form=form)
     assert err == 0
     ref, href, o_ref, e = oracle.scan_conv("gated_delta", 1, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k),
                                            np64(inp.v), np64(inp.g), np64(inp.beta), inp.scale, wq.double().numpy(),
@@ -305,7 +318,8 @@ def test_chunked_scan_conv_unsupported():
     assert st == L.LA_ERR_UNSUPPORTED
 
 
-def test_conv_prefill32_chunked_units():
+@pytest.mark.parametrize("form", ["one", "ws"])
+def test_conv_prefill32_chunked_units(form):
     """The full prefill workload with the convolution, through the chunked prefill with the
     convolution in the same launch: every sequence on two heads and the longest on all 32
     against the oracle's convolved scan, final histories exact."""
@@ -313,7 +327,7 @@ def test_conv_prefill32_chunked_units():
     x = inp.extra
     width, n = x["width"], inp.cu_seqlens.numel() - 1
     S, hnew, o, err = run_chunked_conv(inp, x["w_q"], x["w_k"], x["w_v"], width, x["activation"], x["qk_l2norm"],
-                                       None, n, inp.state_dtype)
+                                       None, n, inp.state_dtype, form=form)
     assert err == 0
     cu = inp.cu_seqlens.numpy()
     by_head = {}
