@@ -134,6 +134,8 @@ KERNEL_SOURCES = {
     "chunk_fused": ["la_chunk.cuh", "la_chunk_fused.cuh", "la_chunk_tc.cuh", "la_umma.cuh", "la_device.cuh"],
     "chunk_kda": ["la_chunk.cuh", "la_chunk_kda.cuh", "la_chunk_fused.cuh", "la_chunk_tc.cuh", "la_umma.cuh",
                   "la_device.cuh"],
+    "chunk_conv": ["la_chunk_conv.cuh", "la_chunk.cuh", "la_chunk_fused.cuh", "la_chunk_tc.cuh", "la_umma.cuh",
+                   "la_device.cuh"],
     "pool": ["la_pool.cu"],
 }
 
@@ -404,7 +406,7 @@ def chunk_roofline(run, inp, ms, peaks):
     conv = run.conv is not None
     two = run.ws is not None and inp.rule in ("delta", "gated_delta") and not conv
     kda = inp.rule == "kda"
-    kernel = "chunk_kda" if kda else ("chunk_tc" if two else "chunk_fused")
+    kernel = "chunk_kda" if kda else "chunk_conv" if conv and run.ws is not None else ("chunk_tc" if two else "chunk_fused")
     out = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
            "traffic": recorded_traffic(kernel, ("kda_prefill32" if kda else "conv_prefill32" if conv else "prefill32") +
                                        (f"_ckpt{run.ckpt_every}" if run.ckpt_every else "")),
