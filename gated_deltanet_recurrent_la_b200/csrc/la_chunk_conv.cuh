@@ -40,7 +40,7 @@ inline size_t chunk_conv_workspace_bytes_impl(int64_t total_tokens, int64_t n_v_
 
 __global__ void __launch_bounds__(cconv::kThreads) chunk_conv_kernel(const ScanParams p) {
   using namespace cconv;
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(1024) unsigned char smem[];
   float* rnorm = reinterpret_cast<float*>(smem + kOffNorm);
   const int tid = threadIdx.x;
   const int m = tid / 64, pr = tid % 64;  // q, k or v; channel pair
