@@ -297,7 +297,8 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
   if ((int64_t)n_seqs * s.n_v_heads > INT32_MAX) return LA_ERR_SHAPE;
 
   const bool q8 = dst->dtype == LA_Q8 || (read_slot && src->dtype == LA_Q8);
-  if (q8 && (chunked || n_q_heads != 0)) return LA_ERR_UNSUPPORTED;
+  // q8 pools on the chunked path: the one-launch form of the scalar-gate rules
+  if (q8 && (n_q_heads != 0 || (chunked && (workspace || conv || rule == LA_RULE_KDA)))) return LA_ERR_UNSUPPORTED;
   if (conv) {
     if (q8 || n_q_heads != 0 || ckpt_every > 0) return LA_ERR_UNSUPPORTED;
     if (conv->width < 2 || conv->width > la::kMaxConvWidth) return LA_ERR_UNSUPPORTED;

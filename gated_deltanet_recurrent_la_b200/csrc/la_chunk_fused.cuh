@@ -177,6 +177,51 @@ __device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, volatile u
   return !named_bar_or(nb, 128, !ok);
 }
 
+// q8 pools (d_k = d_v = 128): row i of a head is BF16 (idx = its rank among the BF16 rows)
+// or INT8 (idx = its rank among the INT8 rows), as the head's mask says
+__device__ __forceinline__ bool q8_row(const uint32_t* mask, int h, int i, int& idx) {
+  int below = 0;
+  uint32_t word = 0u;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const uint32_t m = __ldg(mask + h * 4 + w);
+    if (w < (i >> 5)) below += __popc(m);
+    if (w == (i >> 5)) word = m;
+  }
+  const int b = i & 31;
+  const int pre = below + __popc(word & ((1u << b) - 1u));
+  const bool hp = (word >> b) & 1u;
+  idx = hp ? pre : i - pre;
+  return hp;
+}
+
+// S[i][r] of a q8 tile `tl` (n8 INT8 rows) -- kept out of line, with scalar arguments, so that
+// the state group's loop stays compact for the instruction cache
+__device__ __noinline__ float q8_load_elem(const unsigned char* tl, int n8, const uint32_t* mask, int h, int i, int r) {
+  int idx;
+  if (q8_row(mask, h, i, idx))
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(tl + n8 * 128 + n8 * 16)[idx * 128 + r]);
+  return __fmul_rn((float)(int)(int8_t)tl[idx * 128 + r],
+                   *reinterpret_cast<const float*>(tl + n8 * 128 + (idx * 4 + (r >> 5)) * 4));
+}
+
+// S[i][r] = y into a q8 tile: the warp's 32 lanes hold row i's 32-column group r / 32, whose
+// absmax sets its scale (called by whole warps, all with the same i)
+__device__ __noinline__ void q8_store_elem(unsigned char* tl, int n8, const uint32_t* mask, int h, int i, int r, float y) {
+  int idx;
+  if (q8_row(mask, h, i, idx)) {
+    reinterpret_cast<__nv_bfloat16*>(tl + n8 * 128 + n8 * 16)[idx * 128 + r] = __float2bfloat16_rn(y);
+    return;
+  }
+  float amax = fabsf(y);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  float sc, inv;
+  q8_scales(amax, sc, inv);
+  tl[idx * 128 + r] = (unsigned char)q8_code(y, inv);
+  if ((r & 31) == 0) *reinterpret_cast<float*>(tl + n8 * 128 + (idx * 4 + (r >> 5)) * 4) = sc;
+}
+
 // One (sequence, head) unit: its tokens, slots and whether it can be processed.
 struct Unit {
   int seq, h, hq, t0, n_tok, rs, ws;
@@ -211,6 +256,18 @@ __device__ __forceinline__ Unit unit_info(const ScanParams& p, int64_t u) {
   if (!rs_ok || !ws_ok) {
     x.err |= (rs_ok ? 0u : LA_DEVERR_READ_SLOT) | (ws_ok ? 0u : LA_DEVERR_WRITE_SLOT);
     return x;
+  }
+  // q8 pools: the head's masks must mark exactly n_hp rows, or the row ranks leave the tile
+  if ((p.read_slot && p.src_dtype == LA_Q8) || p.dst_dtype == LA_Q8) {
+    int cs = p.src_n_hp, cd = p.dst_n_hp;
+    for (int w = 0; w < 4; ++w) {
+      if (p.read_slot && p.src_dtype == LA_Q8) cs -= __popc(__ldg(p.src_mask + x.h * 4 + w));
+      if (p.dst_dtype == LA_Q8) cd -= __popc(__ldg(p.dst_mask + x.h * 4 + w));
+    }
+    if (cs != 0 || cd != 0) {
+      x.err |= LA_DEVERR_Q8_MASK;
+      return x;
+    }
   }
   x.t0 = t0;
   x.n_tok = t1 - t0;
@@ -643,8 +700,6 @@ __global__ void __launch_bounds__(CONV ? fused::kThreadsConv : fused::kThreads, 
       if (x.err && tp == 0) report(p.err, x.err);
       if (!x.valid) continue;
       const int nch = (x.n_tok + kC - 1) / kC;
-      const int64_t sbase_src = ((int64_t)x.rs * H + x.h) * (kD * kD);
-      const int64_t dbase = ((int64_t)x.ws * H + x.h) * (kD * kD);
       // checkpoints (ckpt_every a multiple of the chunk): checkpoint k is the state after the
       // first (k + 1) ckpt_every tokens, k < n_ck, to dst slot ckpt_slots[ckpt_cu[seq] + k]
       int n_ck = 0, ck_base = 0;
@@ -657,9 +712,9 @@ __global__ void __launch_bounds__(CONV ? fused::kThreadsConv : fused::kThreads, 
           n_ck = n_ck < 0 ? 0 : fit;
         }
       }
-      // the destination of the state after the first `tok` tokens: its checkpoint slot's
-      // base element, or -1 (no checkpoint there, or a bad slot, which is reported)
-      auto ckpt_base = [&](int tok) -> int64_t {
+      // the checkpoint slot of the state after the first `tok` tokens, or -1 (no checkpoint
+      // there, or a bad slot, which is reported)
+      auto ckpt_slot = [&](int tok) -> int {
         if (p.ckpt_every <= 0 || tok == 0 || tok % p.ckpt_every) return -1;
         const int k = tok / p.ckpt_every - 1;
         if (k >= n_ck) return -1;
@@ -668,9 +723,40 @@ __global__ void __launch_bounds__(CONV ? fused::kThreadsConv : fused::kThreads, 
           if (tp == 0) report(p.err, LA_DEVERR_WRITE_SLOT);
           return -1;
         }
-        return ((int64_t)cs * H + x.h) * (kD * kD);
+        return cs;
       };
-      auto store_col = [&](int64_t base, int i0, const uint32_t* v) {  // S[i0 + e][r] = v[e], e < 16
+      // S[i0 + e][r] of the initial state (zero without a read slot), e < 16
+      auto load_col = [&](int i0, uint32_t* v) {
+        if (p.read_slot && p.src_dtype == LA_Q8) {
+          const unsigned char* tl = static_cast<const unsigned char*>(p.src) +
+                                    ((int64_t)x.rs * H + x.h) * q8_tile_bytes(kD, kD, p.src_n_hp);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            v[e] = __float_as_uint(q8_load_elem(tl, kD - p.src_n_hp, p.src_mask, x.h, i0 + e, r));
+          return;
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float sv = 0.0f;
+          if (p.read_slot) {
+            const int64_t el = ((int64_t)x.rs * H + x.h) * (kD * kD) + (int64_t)(i0 + e) * kD + r;
+            sv = p.src_dtype == LA_F32 ? static_cast<const float*>(p.src)[el]
+                                       : __bfloat162float(static_cast<const __nv_bfloat16*>(p.src)[el]);
+          }
+          v[e] = __float_as_uint(sv);
+        }
+      };
+      // S[i0 + e][r] = v[e] (e < 16) into slot `slot` of the destination
+      auto store_col = [&](int slot, int i0, const uint32_t* v) {
+        if (p.dst_dtype == LA_Q8) {
+          unsigned char* tl =
+              static_cast<unsigned char*>(p.dst) + ((int64_t)slot * H + x.h) * q8_tile_bytes(kD, kD, p.dst_n_hp);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            q8_store_elem(tl, kD - p.dst_n_hp, p.dst_mask, x.h, i0 + e, r, __uint_as_float(v[e]));
+          return;
+        }
+        const int64_t base = ((int64_t)slot * H + x.h) * (kD * kD);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int64_t el = base + (int64_t)(i0 + e) * kD + r;
@@ -688,15 +774,11 @@ __global__ void __launch_bounds__(CONV ? fused::kThreadsConv : fused::kThreads, 
           for (int idx = tp; idx < 384 * wm1; idx += 128) hd[idx] = p.read_slot ? hs[idx] : __float2bfloat16_rn(0.0f);
         }
         // empty sequence: the initial state (or zero) goes to the destination
-        for (int i = 0; i < kD; ++i) {
-          float v = 0.0f;
-          if (p.read_slot)
-            v = p.src_dtype == LA_F32 ? static_cast<const float*>(p.src)[sbase_src + i * kD + r]
-                                      : __bfloat162float(static_cast<const __nv_bfloat16*>(p.src)[sbase_src + i * kD + r]);
-          if (p.dst_dtype == LA_F32)
-            static_cast<float*>(p.dst)[dbase + i * kD + r] = v;
-          else
-            static_cast<__nv_bfloat16*>(p.dst)[dbase + i * kD + r] = __float2bfloat16_rn(v);
+#pragma unroll 1
+        for (int c16 = 0; c16 < 8; ++c16) {
+          uint32_t v[16];
+          load_col(16 * c16, v);
+          store_col(x.ws, 16 * c16, v);
         }
         continue;
       }
@@ -704,17 +786,7 @@ __global__ void __launch_bounds__(CONV ? fused::kThreadsConv : fused::kThreads, 
 #pragma unroll 1
       for (int c16 = 0; c16 < 8; ++c16) {
         uint32_t v[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int i = 16 * c16 + e;
-          float sv = 0.0f;
-          if (p.read_slot) {
-            const int64_t el = sbase_src + (int64_t)i * kD + r;
-            sv = p.src_dtype == LA_F32 ? static_cast<const float*>(p.src)[el]
-                                       : __bfloat162float(static_cast<const __nv_bfloat16*>(p.src)[el]);
-          }
-          v[e] = __float_as_uint(sv);
-        }
+        load_col(16 * c16, v);
         umma::st16(tq + kColS + 16 * c16, v);
       }
       umma::wait_st();
@@ -733,7 +805,7 @@ __global__ void __launch_bounds__(CONV ? fused::kThreadsConv : fused::kThreads, 
         }
         umma::fence_after();
         const float gC = gbk[kC - 1];  // gamma_C (padded tokens have gate 1: the last real token's)
-        const int64_t ckb = ckpt_base(c * kC);  // a checkpoint at this chunk boundary
+        const int ckb = ckpt_slot(c * kC);  // a checkpoint at this chunk boundary
         // S pass: S0^T -> BF16 (the A operand of this chunk's products), S^T *= gamma_C
 #pragma unroll 1
         for (int c32 = 0; c32 < 4; ++c32) {
@@ -801,13 +873,13 @@ __global__ void __launch_bounds__(CONV ? fused::kThreadsConv : fused::kThreads, 
       // final state S[i][r] = S^T[r][i] (and the last checkpoint when it falls on the end)
       if (!(ok = gwait(&bars[kSFull], (uint32_t)(j - 1) & 1u, abort_flag, tp, kNbState))) break;
       umma::fence_after();
-      const int64_t ckf = ckpt_base(x.n_tok);
+      const int ckf = ckpt_slot(x.n_tok);
 #pragma unroll 1
       for (int c16 = 0; c16 < 8; ++c16) {
         uint32_t v[16];
         umma::ld16(tq + kColS + 16 * c16, v);
         umma::wait_ld();
-        store_col(dbase, 16 * c16, v);
+        store_col(x.ws, 16 * c16, v);
         if (ckf >= 0) store_col(ckf, 16 * c16, v);
       }
       umma::fence_before();

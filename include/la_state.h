@@ -207,8 +207,9 @@ la_status la_state_scan(la_rule rule, const la_pool *src, const int32_t *read_sl
  * bit: within 1e-2 of the largest output or state value (up to 7e-3 measured over
  * sequences of 2,000 tokens, every rule, gates in [-1, 1] and beta in [0, 2] included).
  * Arguments, outputs and errors as la_state_scan.  Supported: d_k = d_v = 128 with BF16
- * q/k/v/o, the rules linear, gated, delta and gated_delta, gates of either sign
- * (LA_ERR_UNSUPPORTED otherwise; kda has the two-launch form la_state_scan_chunked_ws). */
+ * q/k/v/o, the rules linear, gated, delta and gated_delta, gates of either sign, FP32, BF16
+ * or q8 pools (LA_ERR_UNSUPPORTED otherwise; kda has the two-launch form
+ * la_state_scan_chunked_ws, which takes FP32 or BF16 pools). */
 la_status la_state_scan_chunked(la_rule rule, const la_pool *src, const int32_t *read_slot,
                                 const la_pool *dst, const int32_t *write_slot, int32_t n_seqs,
                                 const int32_t *cu_seqlens, int32_t total_tokens, const int32_t *seq_order,

@@ -378,8 +378,13 @@ def test_q8_pools_host_side(lib):
     assert lib.la_state_step_qgroups(3, ctypes.byref(q8(shape=(4, 4, 128, 128))), None,
                                      ctypes.byref(q8(shape=(4, 4, 128, 128))), None, 2, 8, P(A), P(A), P(A), 1,
                                      P(A), P(A), 1.0, P(A), P(A), None) == L.LA_ERR_UNSUPPORTED
-    assert lib.la_state_scan_chunked(3, None, None, ctypes.byref(q8()), None, 2, P(A), 10, None, P(A), P(A), P(A), 1,
-                                     P(A), P(A), 1.0, P(A), P(A), None) == L.LA_ERR_UNSUPPORTED
+    # the chunked path takes q8 pools in its one-launch form only (not through a workspace)
+    assert lib.la_state_scan_chunked_ws(3, None, None, ctypes.byref(q8()), None, 2, P(A), 10, None, P(A), P(A),
+                                        P(A), 1, P(A), P(A), 1.0, P(A), P(A), 1 << 30, P(A),
+                                        None) == L.LA_ERR_UNSUPPORTED
+    assert lib.la_state_scan_chunked_ws(4, None, None, ctypes.byref(q8()), None, 2, P(A), 10, None, P(A), P(A),
+                                        P(A), 1, P(A), P(A), 1.0, P(A), P(A), 1 << 30, P(A),
+                                        None) == L.LA_ERR_UNSUPPORTED
     assert lib.la_state_pool_encode(ctypes.byref(pool(dtype=1)), 2, P(A), P(A), P(A), None) == L.LA_ERR_UNSUPPORTED
     assert lib.la_state_pool_decode(ctypes.byref(q8()), 2, None, P(A), P(A), None) == L.LA_ERR_NULL
     assert lib.la_state_pool_decode(ctypes.byref(q8()), 2, P(A), P(A + 4), P(A), None) == L.LA_ERR_ALIGN

@@ -203,3 +203,92 @@ def test_q8_decode64_full():
     assert_close(np64(o.cpu()[sl]), o_ref, 2e-2, "sampled outputs")
     untouched = np.setdiff1d(np.arange(256), inp.write_slot.numpy())
     assert torch.equal(after[untouched], before[untouched])
+
+
+# ---- q8 pools on the chunked prefill (one launch; BF16 operands inside the chunks, so the
+#      states are compared at the chunked prefill's tolerance) ---------------------------
+
+@pytest.mark.parametrize("src_kind,dst_kind", [("q8", "q8"), ("f32", "q8"), ("q8", "bf16"), ("q8", "f32")])
+@pytest.mark.parametrize("rule", ["linear", "gated_delta"])
+def test_chunked_scan_q8(rule, src_kind, dst_kind):
+    dk, dv, n_hp = 128, 128, 16
+    lengths = [37, 0, 130, 64]
+    inp = W.scan_inputs(lengths=lengths, n_qk_heads=2, n_v_heads=2, d_k=dk, d_v=dv, rule=rule, state_dtype=BF16,
+                        io_dtype=BF16, seed=96, init="slots", init_dtype=F32, pool_std=0.3)
+    mask = masks_of(2, dk, n_hp, 6)
+    if src_kind == "q8":
+        src, st = q8_pool(inp.pool, 2, n_hp, mask)
+        src_vals = _values_of(st, dk, dv, n_hp, mask)
+    else:
+        src = L.Pool(dev(inp.pool), 2)
+        src_vals = np64(inp.pool)
+    n = len(lengths)
+    if dst_kind == "q8":
+        dt = torch.zeros(n, 2, L.q8_tile_bytes(dk, dv, n_hp), dtype=torch.uint8, device="cuda")
+        dst = L.Pool.q8(dt, 2, dk, dv, n_hp, mask.cuda())
+    else:
+        dt = torch.zeros(n, 2, dk, dv, dtype=BF16 if dst_kind == "bf16" else F32, device="cuda")
+        dst = L.Pool(dt, 2)
+    o = torch.empty(inp.q.shape[0], 2, dv, dtype=BF16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.check(L.la_state_scan_chunked(rule, src, dev(inp.read_slot), dst, None, dev(inp.cu_seqlens), dev(inp.q),
+                                    dev(inp.k), dev(inp.v), dev(inp.g), dev(inp.beta), inp.scale, o, err))
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    args = (rule, 2, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k), np64(inp.v), np64(inp.g), np64(inp.beta),
+            inp.scale)
+    kw = dict(src_pool=src_vals, read_slot=inp.read_slot.numpy(), io_dtype="bf16")
+    if dst_kind == "q8":
+        ref, o_ref, e = oracle.scan_q8(*args, masks=u32(mask), **kw)
+        got = _values_of(dt, dk, dv, n_hp, mask)
+    else:
+        ref, o_ref, e = oracle.scan(*args, dst_dtype=dst_kind, **kw)
+        got = np64(dt.cpu())
+    assert e == 0
+    assert_close(got, ref, 1e-2, f"chunked {rule} {src_kind}->{dst_kind}: final states")
+    assert_close(np64(o.cpu()), o_ref, 1e-2, f"chunked {rule} {src_kind}->{dst_kind}: outputs")
+    # the empty sequence (index 1) stores its initial state through the destination's format
+    assert_close(got[1], ref[1], 1e-5, f"chunked {rule} {src_kind}->{dst_kind}: empty sequence")
+
+
+def test_chunked_scan_q8_checkpoints_and_bad_mask():
+    """Checkpoints every 64 tokens into a q8 pool (the chunked checkpointed entry point),
+    against the oracle's checkpointed scan decoded through the same codec; then a mask with
+    the wrong number of BF16 rows: that head is skipped and reported."""
+    dk, dv, n_hp = 128, 128, 16
+    lengths, every = [130, 64, 5], 64
+    inp = W.scan_inputs(lengths=lengths, n_qk_heads=1, n_v_heads=2, d_k=dk, d_v=dv, rule="gated_delta",
+                        state_dtype=BF16, io_dtype=BF16, seed=98, init="slots", init_dtype=F32, pool_std=0.3)
+    mask = masks_of(2, dk, n_hp, 7)
+    src, st = q8_pool(inp.pool, 1, n_hp, mask)
+    src_vals = _values_of(st, dk, dv, n_hp, mask)
+    n_ck = [l // every for l in lengths]
+    ckpt_cu = np.concatenate([[0], np.cumsum(n_ck)]).astype(np.int32)
+    n_dst = len(lengths) + int(ckpt_cu[-1])
+    ckpt_slots = np.arange(len(lengths), n_dst, dtype=np.int32)
+    dt = torch.zeros(n_dst, 2, L.q8_tile_bytes(dk, dv, n_hp), dtype=torch.uint8, device="cuda")
+    dst = L.Pool.q8(dt, 1, dk, dv, n_hp, mask.cuda())
+    o = torch.empty(inp.q.shape[0], 2, dv, dtype=BF16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.check(L.la_state_scan_chunked_checkpointed("gated_delta", src, dev(inp.read_slot), dst, None,
+                                                 dev(inp.cu_seqlens), dev(inp.q), dev(inp.k), dev(inp.v),
+                                                 dev(inp.g), dev(inp.beta), inp.scale, o, every,
+                                                 dev(torch.from_numpy(ckpt_cu)), dev(torch.from_numpy(ckpt_slots)),
+                                                 err))
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ref, o_ref, e = oracle.scan_q8("gated_delta", 1, inp.cu_seqlens.numpy(), np64(inp.q), np64(inp.k), np64(inp.v),
+                                   np64(inp.g), np64(inp.beta), inp.scale, masks=u32(mask), src_pool=src_vals,
+                                   read_slot=inp.read_slot.numpy(), io_dtype="bf16",
+                                   dst_pool=np.zeros((n_dst, 2, dk, dv)), ckpt_every=every,
+                                   ckpt_cu=ckpt_cu, ckpt_slots=ckpt_slots)
+    assert e == 0
+    assert_close(_values_of(dt, dk, dv, n_hp, mask), ref, 1e-2, "q8 checkpoints and final states")
+    bad = mask.clone()
+    bad[1, 0] = 0 if int(bad[1, 0]) != 0 else 1
+    dst_bad = L.Pool.q8(dt, 1, dk, dv, n_hp, bad.cuda())
+    err.zero_()
+    L.check(L.la_state_scan_chunked("gated_delta", src, dev(inp.read_slot), dst_bad, None, dev(inp.cu_seqlens),
+                                    dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.g), dev(inp.beta), inp.scale, o, err))
+    torch.cuda.synchronize()
+    assert int(err.item()) & L.DEVERR_Q8_MASK
