@@ -297,8 +297,10 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
   if ((int64_t)n_seqs * s.n_v_heads > INT32_MAX) return LA_ERR_SHAPE;
 
   const bool q8 = dst->dtype == LA_Q8 || (read_slot && src->dtype == LA_Q8);
-  // q8 pools on the chunked path: the one-launch form of the scalar-gate rules
-  if (q8 && (n_q_heads != 0 || (chunked && (workspace || conv || rule == LA_RULE_KDA)))) return LA_ERR_UNSUPPORTED;
+  // q8 pools on the chunked path: the one-launch form of the scalar-gate rules (query groups
+  // included); on the token-serial scan not in the query-group direction
+  if (q8 && ((n_q_heads != 0 && !chunked) || (chunked && (workspace || conv || rule == LA_RULE_KDA))))
+    return LA_ERR_UNSUPPORTED;
   if (conv) {
     if (q8 || n_q_heads != 0 || ckpt_every > 0) return LA_ERR_UNSUPPORTED;
     if (conv->width < 2 || conv->width > la::kMaxConvWidth) return LA_ERR_UNSUPPORTED;
@@ -320,6 +322,11 @@ static la_status scan_impl(la_rule rule, const la_pool* src, const int32_t* read
     }
   } else if (conv) {
     fn = (io == LA_F32) ? la::find_scan_conv_f32io(rule, s.d_k, s.d_v) : la::find_scan_conv_bf16io(rule, s.d_k, s.d_v);
+  } else if (chunked && n_q_heads != 0) {
+    // the query-group direction: the one-launch form of the scalar-gate rules, once per query
+    if (s.d_k != 128 || s.d_v != 128 || io != LA_BF16) return LA_ERR_UNSUPPORTED;
+    if (ckpt_every > 0 || workspace) return LA_ERR_UNSUPPORTED;
+    fn = la::find_chunk_scan_qgroups(rule);
   } else if (chunked) {
     if (s.d_k != 128 || s.d_v != 128 || io != LA_BF16) return LA_ERR_UNSUPPORTED;
     // checkpoints fall on chunk boundaries, in the one-launch form
@@ -507,6 +514,17 @@ la_status la_state_scan_qgroups(la_rule rule, const la_pool* src, const int32_t*
   if (n_q_heads <= 0) return LA_ERR_SHAPE;
   return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, q, k, v, io,
                    g, beta, scale, o, 0, nullptr, nullptr, err_word, stream, false, n_q_heads);
+}
+
+la_status la_state_scan_chunked_qgroups(la_rule rule, const la_pool* src, const int32_t* read_slot,
+                                        const la_pool* dst, const int32_t* write_slot, int32_t n_seqs,
+                                        const int32_t* cu_seqlens, int32_t total_tokens, const int32_t* seq_order,
+                                        int32_t n_q_heads, const void* q, const void* k, const void* v, la_dtype io,
+                                        const float* g, const float* beta, float scale, void* o, int32_t* err_word,
+                                        void* stream) {
+  if (n_q_heads <= 0) return LA_ERR_SHAPE;
+  return scan_impl(rule, src, read_slot, dst, write_slot, n_seqs, cu_seqlens, total_tokens, seq_order, q, k, v, io,
+                   g, beta, scale, o, 0, nullptr, nullptr, err_word, stream, true, n_q_heads);
 }
 
 static la_status pool_op(const la_pool* pool, int32_t n, const int32_t* src_slots, const int32_t* dst_slots,

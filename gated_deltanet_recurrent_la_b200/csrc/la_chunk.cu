@@ -18,6 +18,28 @@ ScanLaunchFn find_chunk_scan(int rule) {
   }
   return nullptr;
 }
+// The query-group direction: the one-launch form once per query of the group, each launch
+// writing its query head's outputs; the state (the same in every launch) is written by the
+// launch of query 0, which runs last (a read slot may be the write slot).
+template <int RULE>
+cudaError_t launch_chunk_qgroups(const ScanParams& p, cudaStream_t stream) {
+  for (int qi = p.q_group - 1; qi >= 0; --qi) {
+    ScanParams f = p;
+    f.q_index = qi;
+    const cudaError_t e = launch_chunk_fused<RULE, false>(f, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+ScanLaunchFn find_chunk_scan_qgroups(int rule) {
+  switch (rule) {
+    case LA_RULE_LINEAR: return &launch_chunk_qgroups<LA_RULE_LINEAR>;
+    case LA_RULE_GATED: return &launch_chunk_qgroups<LA_RULE_GATED>;
+    case LA_RULE_DELTA: return &launch_chunk_qgroups<LA_RULE_DELTA>;
+    case LA_RULE_GATED_DELTA: return &launch_chunk_qgroups<LA_RULE_GATED_DELTA>;
+  }
+  return nullptr;
+}
 ScanLaunchFn find_chunk_scan_conv(int rule) {
   switch (rule) {
     case LA_RULE_LINEAR: return &launch_chunk_fused<LA_RULE_LINEAR, true>;

@@ -381,6 +381,8 @@ __global__ void __launch_bounds__(CONV ? fused::kThreadsConv : fused::kThreads, 
       const Unit x = unit_info(p, u);
       if (!x.valid) continue;
       const int nch = (x.n_tok + kC - 1) / kC;
+      // the query head: of the q/k head, or query q_index of the state head's group
+      const int qhead = p.q_group > 1 ? x.h * p.q_group + p.q_index : x.hq;
       for (int c = 0; c < nch; ++c, ++j) {
         const int s = (int)(j % kStages);
         const int tok0 = x.t0 + c * kC;
@@ -405,7 +407,7 @@ __global__ void __launch_bounds__(CONV ? fused::kThreadsConv : fused::kThreads, 
           mbar_arrive_expect_tx(full, kTmaBytes);
 #pragma unroll
           for (int pnl = 0; pnl < 2; ++pnl) {
-            umma::tma_load_3d(st + kOffQK + pnl * 16384, &maps.q, 64 * pnl, x.hq, tok0, full);
+            umma::tma_load_3d(st + kOffQK + pnl * 16384, &maps.q, 64 * pnl, qhead, tok0, full);
             umma::tma_load_3d(st + kOffQK + pnl * 16384 + kC * 128, &maps.k, 64 * pnl, x.hq, tok0, full);
             umma::tma_load_3d(st + kOffV + pnl * 8192, &maps.v, 64 * pnl, x.h, tok0, full);
           }
@@ -746,8 +748,10 @@ __global__ void __launch_bounds__(CONV ? fused::kThreadsConv : fused::kThreads, 
           v[e] = __float_as_uint(sv);
         }
       };
-      // S[i0 + e][r] = v[e] (e < 16) into slot `slot` of the destination
+      // S[i0 + e][r] = v[e] (e < 16) into slot `slot` of the destination (in the query-group
+      // direction by the launch of query 0 alone)
       auto store_col = [&](int slot, int i0, const uint32_t* v) {
+        if (p.q_index != 0) return;
         if (p.dst_dtype == LA_Q8) {
           unsigned char* tl =
               static_cast<unsigned char*>(p.dst) + ((int64_t)slot * H + x.h) * q8_tile_bytes(kD, kD, p.dst_n_hp);
@@ -955,7 +959,7 @@ __global__ void __launch_bounds__(CONV ? fused::kThreadsConv : fused::kThreads, 
             const int idx = tp + 128 * i;
             const int t = idx >> 4, ch = idx & 15;
             if (t < nv)
-              *reinterpret_cast<uint4*>(og + ((int64_t)(tok0 + t) * H + x.h) * kD + ch * 8) =
+              *reinterpret_cast<uint4*>(og + ((int64_t)(tok0 + t) * H * p.q_group + x.h * p.q_group + p.q_index) * kD + ch * 8) =
                   *reinterpret_cast<const uint4*>(so + t * kD + ch * 8);
           }
         }
@@ -1138,7 +1142,7 @@ cudaError_t launch_chunk_fused(const ScanParams& p, cudaStream_t stream) {
   TcMaps maps;
   memset(&maps, 0, sizeof(maps));  // no tokens: nothing is staged, the maps are never read
   if (p.total_tokens > 0 &&
-      (!encode_rows_map(&maps.q, p.q, p.n_qk_heads, p.total_tokens) ||
+      (!encode_rows_map(&maps.q, p.q, p.n_qk_heads * p.q_group, p.total_tokens) ||
        !encode_rows_map(&maps.k, p.k, p.n_qk_heads, p.total_tokens) ||
        !encode_rows_map(&maps.v, p.v, p.n_v_heads, p.total_tokens)))
     return cudaErrorInvalidValue;

@@ -68,6 +68,8 @@ struct ScanParams {
   int32_t n_qk_heads;
   int32_t n_v_heads;
   int32_t q_group;           // queries per state head: 1, or up to 8 in the query-group direction
+  int32_t q_index;           // chunked prefill in the query-group direction: the query of the group
+                             // this launch reads (the state is written by query 0 alone)
   int32_t src_n_hp;          // q8 pools: BF16 key channels per head and the channel masks
   const uint32_t* src_mask;
   int32_t dst_n_hp;
@@ -140,6 +142,8 @@ ScanLaunchFn find_scan_qgroups_bf16io(int rule, int dk, int dv);
 // (the delta rules and kda; kda has only this form).
 ScanLaunchFn find_chunk_scan(int rule);
 ScanLaunchFn find_chunk_scan_ws(int rule);
+// the one-launch form in the query-group direction (scalar-gate rules)
+ScanLaunchFn find_chunk_scan_qgroups(int rule);
 // the one-launch form with the short causal convolution ahead (scalar-gate rules), and the
 // two-launch form (the convolution's output through a workspace of
 // chunk_conv_workspace_bytes(T, H_v) bytes)

@@ -29,7 +29,7 @@ DEVERR_READ_SLOT, DEVERR_WRITE_SLOT, DEVERR_CU_SEQLENS, DEVERR_TIMEOUT, DEVERR_Q
 
 EXPORTS = ("la_state_bytes", "la_shape_supported", "la_state_step", "la_state_scan", "la_state_scan_chunked",
            "la_state_scan_checkpointed", "la_state_scan_chunked_checkpointed", "la_state_step_qgroups",
-           "la_state_scan_qgroups",
+           "la_state_scan_qgroups", "la_state_scan_chunked_qgroups",
            "la_pool_slot_bytes", "la_state_pool_encode", "la_state_pool_decode", "la_state_step_conv",
            "la_state_scan_conv", "la_state_scan_chunked_conv", "la_state_scan_chunked_conv_ws",
            "la_scan_chunked_conv_workspace_bytes", "la_scan_chunked_workspace_bytes", "la_scan_chunked_workspace_bytes_rule",
@@ -97,6 +97,8 @@ def lib():
         L.la_state_step_qgroups.restype = I32
         L.la_state_scan_qgroups.argtypes = L.la_state_scan.argtypes[:9] + [I32] + L.la_state_scan.argtypes[9:]
         L.la_state_scan_qgroups.restype = I32
+        L.la_state_scan_chunked_qgroups.argtypes = L.la_state_scan_qgroups.argtypes
+        L.la_state_scan_chunked_qgroups.restype = I32
         L.la_state_pool_copy.argtypes = [PP, I32, P, P, P, P]
         L.la_state_pool_gather.argtypes = [PP, I32, P, P, P, P]
         L.la_state_pool_scatter.argtypes = [PP, I32, P, P, P, P]
@@ -424,6 +426,20 @@ def la_state_scan_qgroups(rule, src: Optional[Pool], read_slot, dst: Pool, write
                                        int(q.shape[1]), _ptr(q), _ptr(k, q.dtype), _ptr(v, q.dtype), io,
                                        _ptr(g, torch.float32), _ptr(beta, torch.float32), float(scale),
                                        _ptr(o, q.dtype), _ptr(err_word, torch.int32), _stream(stream))
+
+
+def la_state_scan_chunked_qgroups(rule, src: Optional[Pool], read_slot, dst: Pool, write_slot, cu_seqlens, q, k, v, g,
+                                  beta, scale, o, err_word, seq_order=None, stream=None) -> int:
+    """Query-group direction of la_state_scan_chunked: k [T, H_v, 128], q [T, n_q_heads, 128]."""
+    io = dtype_code(q.dtype)
+    return lib().la_state_scan_chunked_qgroups(RULES[rule] if isinstance(rule, str) else int(rule),
+                                               None if src is None else src.ref, _ptr(read_slot, torch.int32),
+                                               dst.ref, _ptr(write_slot, torch.int32), int(cu_seqlens.numel() - 1),
+                                               _ptr(cu_seqlens, torch.int32), int(q.shape[0]),
+                                               _ptr(seq_order, torch.int32), int(q.shape[1]), _ptr(q),
+                                               _ptr(k, q.dtype), _ptr(v, q.dtype), io, _ptr(g, torch.float32),
+                                               _ptr(beta, torch.float32), float(scale), _ptr(o, q.dtype),
+                                               _ptr(err_word, torch.int32), _stream(stream))
 
 
 def la_state_pool_copy(pool: Pool, src_slots, dst_slots, err_word, stream=None) -> int:

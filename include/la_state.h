@@ -421,6 +421,19 @@ la_status la_state_scan_qgroups(la_rule rule, const la_pool *src, const int32_t 
                                 const void *k, const void *v, la_dtype io, const float *g,
                                 const float *beta, float scale, void *o, int32_t *err_word,
                                 void *stream);
+/* The same on the chunked (WY/UT) form of la_state_scan_chunked, its precision claim and
+ * supported shapes (d_k = d_v = 128, BF16 io, rules other than kda, FP32/BF16/q8 pools).
+ * The one-launch chunked pass runs once per query of the group, each writing its query
+ * head's outputs; the state is the same in every pass and is written by the last, so a
+ * request may read and write one slot. */
+la_status la_state_scan_chunked_qgroups(la_rule rule, const la_pool *src,
+                                        const int32_t *read_slot, const la_pool *dst,
+                                        const int32_t *write_slot, int32_t n_seqs,
+                                        const int32_t *cu_seqlens, int32_t total_tokens,
+                                        const int32_t *seq_order, int32_t n_q_heads,
+                                        const void *q, const void *k, const void *v, la_dtype io,
+                                        const float *g, const float *beta, float scale, void *o,
+                                        int32_t *err_word, void *stream);
 
 /* Slot-pool maintenance, bit-exact whole-slot copies ("Recurrent state" glossary: slot
  * allocation and prefix-cache checkpoints; "Seven Architectures ...", ONNX section:

@@ -269,6 +269,26 @@ def test_chunked_conv_host_errors(lib):
     assert ws_call(A, need, rule=4) == L.LA_ERR_UNSUPPORTED
 
 
+def test_chunked_qgroups_host_errors(lib):
+    """The chunked prefill in the query-group direction: the one-launch form of the
+    scalar-gate rules at d_k = d_v = 128 with BF16 io; the group as for the token-serial
+    scan (a multiple of H_v, at most 8 queries per state head, n_qk_heads == n_v_heads)."""
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+
+    def call(rule=3, nq=16, io=1, shape=(4, 4, 128, 128), dst=None):
+        d = dst or pool(shape=shape)
+        return lib.la_state_scan_chunked_qgroups(rule, None, None, ctypes.byref(d), None, 2, P(A), 10, None, nq,
+                                                 P(A), P(A), P(A), io, P(A), P(A), 1.0, P(A), P(A), None)
+    assert call(nq=0) == L.LA_ERR_SHAPE
+    assert call(nq=6) == L.LA_ERR_SHAPE                                  # not a multiple of H_v
+    assert call(shape=(2, 4, 128, 128)) == L.LA_ERR_SHAPE                # n_qk_heads != n_v_heads
+    assert call(nq=36) == L.LA_ERR_UNSUPPORTED                           # 9 queries per state head
+    assert call(rule=4) == L.LA_ERR_UNSUPPORTED                          # kda
+    assert call(io=0) == L.LA_ERR_UNSUPPORTED                            # FP32 io
+    assert call(shape=(4, 4, 64, 64)) == L.LA_ERR_UNSUPPORTED
+    assert call(dst=pool(shape=(4, 4, 128, 128), data=0)) == L.LA_ERR_NULL
+
+
 def test_noalloc_lookup_failure_is_an_error(lib):
     """The no-alloc prefill looks up the address of the library's own workspace before
     anything else; where that lookup fails (here: no CUDA device at all), the call reports

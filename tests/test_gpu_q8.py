@@ -251,6 +251,41 @@ def test_chunked_scan_q8(rule, src_kind, dst_kind):
     assert_close(got[1], ref[1], 1e-5, f"chunked {rule} {src_kind}->{dst_kind}: empty sequence")
 
 
+def test_chunked_scan_qgroups_q8():
+    """The chunked prefill in the query-group direction from and to q8 pools: the state
+    against the oracle's q8 scan, the outputs (taken before the state is encoded) against
+    its query-group scan from the decoded initial states."""
+    dk, dv, n_hp, H, group = 128, 128, 16, 2, 3
+    lengths = [70, 0, 129]
+    inp = W.scan_inputs(lengths=lengths, n_qk_heads=H, n_v_heads=H, d_k=dk, d_v=dv, rule="gated_delta",
+                        state_dtype=BF16, io_dtype=BF16, seed=99, init="slots", init_dtype=F32, pool_std=0.3,
+                        n_q_heads=H * group)
+    mask = masks_of(H, dk, n_hp, 8)
+    src, st = q8_pool(inp.pool, H, n_hp, mask)
+    src_vals = _values_of(st, dk, dv, n_hp, mask)
+    dt = torch.zeros(len(lengths), H, L.q8_tile_bytes(dk, dv, n_hp), dtype=torch.uint8, device="cuda")
+    dst = L.Pool.q8(dt, H, dk, dv, n_hp, mask.cuda())
+    o = torch.empty(inp.q.shape[0], H * group, dv, dtype=BF16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.check(L.la_state_scan_chunked_qgroups("gated_delta", src, dev(inp.read_slot), dst, None, dev(inp.cu_seqlens),
+                                            dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.g), dev(inp.beta),
+                                            inp.scale, o, err))
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    cu = inp.cu_seqlens.numpy()
+    q0 = np64(inp.q).reshape(-1, H, group, dk)[:, :, 0]
+    ref, _, e = oracle.scan_q8("gated_delta", H, cu, q0, np64(inp.k), np64(inp.v), np64(inp.g), np64(inp.beta),
+                               inp.scale, masks=u32(mask), src_pool=src_vals, read_slot=inp.read_slot.numpy(),
+                               io_dtype="bf16")
+    assert e == 0
+    _, o_ref, e = oracle.scan_qgroups("gated_delta", H * group, cu, np64(inp.q), np64(inp.k), np64(inp.v),
+                                      np64(inp.g), np64(inp.beta), inp.scale, src_pool=src_vals,
+                                      read_slot=inp.read_slot.numpy(), dst_dtype="f32", io_dtype="bf16")
+    assert e == 0
+    assert_close(_values_of(dt, dk, dv, n_hp, mask), ref, 1e-2, "chunked query groups q8: final states")
+    assert_close(np64(o.cpu()), o_ref, 1e-2, "chunked query groups q8: outputs")
+
+
 def test_chunked_scan_q8_checkpoints_and_bad_mask():
     """Checkpoints every 64 tokens into a q8 pool (the chunked checkpointed entry point),
     against the oracle's checkpointed scan decoded through the same codec; then a mask with
