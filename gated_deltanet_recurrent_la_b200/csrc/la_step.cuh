@@ -189,6 +189,135 @@ __device__ __forceinline__ void conv_operands(const StepParams& p, const unsigne
   named_bar_sync(bar, WPT * 32);
 }
 
+// The producer warp of a step CTA (whose stage layout is C): its lanes fetch the slot ids
+// and gates of the next 32 of the CTA's tiles; lane 0 checks each tile (slots in range,
+// q8 masks marking n_hp rows), writes its meta, and issues its bulk copies into the next
+// free stage (the state tile with an evict-first policy), or arrives without data for a
+// tile that is skipped.  A wait that runs out reports LA_DEVERR_TIMEOUT and ends the
+// issue; the warp never retires with copies in flight.
+template <int RULE, int DK, int DV, typename ST, typename IT, bool QGRP, bool CONV, typename C>
+__device__ __forceinline__ void step_producer(const StepParams& p, unsigned char* smem, StepMeta* meta,
+                                              uint64_t* full, uint64_t* empty, int64_t n_my, int lane) {
+  constexpr bool CHG = Rule<RULE>::kChannelGate;
+  const int H = p.n_v_heads;
+  const int qg = QGRP ? p.q_group : 1;
+  const uint64_t pol_stream = policy_evict_first();
+  const int ratio = H / p.n_qk_heads;
+  const unsigned char* src = static_cast<const unsigned char*>(p.src);
+  const int tile_bytes = C::kQ8 ? (int)q8_tile_bytes(DK, DV, p.n_hp) : C::kTileBytes;
+  const IT* q = static_cast<const IT*>(p.q);
+  const IT* k = static_cast<const IT*>(p.k);
+  const IT* v = static_cast<const IT*>(p.v);
+  bool abort = false;
+  int64_t issued = 0;
+  for (int64_t i0 = 0; i0 < n_my && !abort; i0 += 32) {
+    // lanes fetch the slot ids and gates of the next 32 tiles
+    const int64_t ii = i0 + lane;
+    int32_t rs = -1, ws = -1;
+    float gg = 1.0f, bb = 1.0f;
+    if (ii < n_my) {
+      const int64_t t = blockIdx.x + ii * gridDim.x;
+      const int b = (int)(t / H);
+      rs = p.read_slot ? __ldg(p.read_slot + b) : b;
+      ws = p.write_slot ? __ldg(p.write_slot + b) : b;
+      if (Rule<RULE>::kUsesGate) gg = __ldg(p.g + t);
+      if (Rule<RULE>::kUsesBeta) bb = __ldg(p.beta + t);
+    }
+    const int cnt = (int)((n_my - i0) < 32 ? (n_my - i0) : 32);
+    for (int j = 0; j < cnt; ++j) {
+      const int32_t rs_j = __shfl_sync(0xffffffffu, rs, j);
+      const int32_t ws_j = __shfl_sync(0xffffffffu, ws, j);
+      const float g_j = __shfl_sync(0xffffffffu, gg, j);
+      const float b_j = __shfl_sync(0xffffffffu, bb, j);
+      const int64_t it = i0 + j;
+      const int stage = (int)(it % C::kStages);
+      const uint32_t round = (uint32_t)(it / C::kStages);
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait(&empty[stage], (round & 1u) ^ 1u, p.wait_ns);
+        if (ok && blockIdx.x == 0 && it == p.withhold) {
+          // test hook: this tile's copies are never issued and its arrival never comes (its
+          // consumers' waits run out); nothing of it is in flight, and the rest is abandoned
+          ok = false;
+        } else if (ok) {
+          const int64_t t = blockIdx.x + it * gridDim.x;
+          const int b = (int)(t / H);
+          const int h = (int)(t % H);
+          const int hq = h / ratio;
+          const bool rs_ok = rs_j >= 0 && rs_j < p.src_slots;
+          const bool ws_ok = ws_j >= 0 && ws_j < p.dst_slots;
+          bool mask_ok = true;
+          if constexpr (C::kQ8) {
+            // a head's masks must mark exactly n_hp rows, or the row ranks leave the tile
+            int cs = 0, cd = 0;
+#pragma unroll
+            for (int w = 0; w < DK / 32; ++w) {
+              cs += __popc(__ldg(p.src_mask + h * (DK / 32) + w));
+              cd += __popc(__ldg(p.dst_mask + h * (DK / 32) + w));
+            }
+            mask_ok = cs == p.n_hp && cd == p.n_hp;
+            if (!mask_ok) report(p.err, LA_DEVERR_Q8_MASK);
+          }
+          StepMeta m;
+          m.g = g_j;
+          m.beta = b_j;
+          m.valid = rs_ok && ws_ok && mask_ok;
+          m.ws = ws_j;
+          m.dst_off = ((int64_t)ws_j * H + h) * tile_bytes;
+          m.o_off = t * qg * DV;  // o row of the tile's first query
+          meta[stage] = m;
+          if (m.valid) {
+            unsigned char* sb = smem + stage * C::kStageBytes;
+            // query rows: the tile's q/k head, or its qg consecutive query heads
+            const int64_t qrow = QGRP ? t * qg : (int64_t)b * p.n_qk_heads + hq;
+            const int hist_bytes = CONV ? (2 * DK + DV) * (p.conv_w - 1) * (int)sizeof(IT) : 0;
+            const int wbytes = CONV ? (2 * DK + DV) * p.conv_w * 4 : 0;
+            mbar_arrive_expect_tx(&full[stage],
+                                  C::kOffHist - C::kOffK + tile_bytes + qg * C::kQKBytes + hist_bytes + wbytes);
+            bulk_g2s_hint(sb, src + ((int64_t)rs_j * H + h) * tile_bytes, tile_bytes, &full[stage], pol_stream);
+            bulk_g2s(sb + C::kTileBytes, q + qrow * DK, qg * C::kQKBytes, &full[stage]);
+            bulk_g2s(sb + C::kOffK, k + ((int64_t)b * p.n_qk_heads + hq) * DK, C::kQKBytes, &full[stage]);
+            bulk_g2s(sb + C::kOffV, v + t * DV, C::kVBytes, &full[stage]);
+            if (CHG) bulk_g2s(sb + C::kOffA, p.g + t * DK, C::kGBytes, &full[stage]);
+            if (CONV) {
+              bulk_g2s(sb + C::kOffHist,
+                       static_cast<const unsigned char*>(p.conv_src) + ((int64_t)rs_j * H + h) * hist_bytes,
+                       hist_bytes, &full[stage]);
+              // the weights of the tile's q/k head and head (the same for every request)
+              const int W = p.conv_w;
+              bulk_g2s(sb + C::kOffConvW, p.conv_wq + (int64_t)hq * DK * W, DK * W * 4, &full[stage]);
+              bulk_g2s(sb + C::kOffConvW + DK * W * 4, p.conv_wk + (int64_t)hq * DK * W, DK * W * 4, &full[stage]);
+              bulk_g2s(sb + C::kOffConvW + 2 * DK * W * 4, p.conv_wv + (int64_t)h * DV * W, DV * W * 4,
+                       &full[stage]);
+            }
+          } else {
+            if (!rs_ok || !ws_ok) report(p.err, (rs_ok ? 0u : LA_DEVERR_READ_SLOT) | (ws_ok ? 0u : LA_DEVERR_WRITE_SLOT));
+            mbar_arrive(&full[stage]);
+          }
+        } else {
+          report(p.err, LA_DEVERR_TIMEOUT);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        abort = true;
+        break;
+      }
+      ++issued;
+    }
+  }
+  // Never retire with copies in flight: wait for the last phase issued on each stage.
+  if (lane == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      if (issued > s) {
+        const int64_t last = issued - 1 - ((issued - 1 - s) % C::kStages);
+        if (blockIdx.x == 0 && last == p.withhold) continue;  // withheld: nothing issued
+        if (!mbar_wait(&full[s], (uint32_t)(last / C::kStages) & 1u, p.wait_ns)) report(p.err, LA_DEVERR_TIMEOUT);
+      }
+    }
+  }
+}
+
 // QGRP: the query-group direction of the ONNX operator -- k has one head per state head
 // and p.q_group query heads (consecutive) read each state head; every extra query costs
 // one more pass over the registers, the state is still read and written once.
@@ -228,122 +357,7 @@ __global__ void __launch_bounds__(
   const int lane = threadIdx.x & 31;
 
   if (warp == C::kConsumerWarps) {
-    // ------------------------------------------------------------------ producer
-    const uint64_t pol_stream = policy_evict_first();
-    const int ratio = H / p.n_qk_heads;
-    const unsigned char* src = static_cast<const unsigned char*>(p.src);
-    const int tile_bytes = C::kQ8 ? (int)q8_tile_bytes(DK, DV, p.n_hp) : C::kTileBytes;
-    const IT* q = static_cast<const IT*>(p.q);
-    const IT* k = static_cast<const IT*>(p.k);
-    const IT* v = static_cast<const IT*>(p.v);
-    bool abort = false;
-    int64_t issued = 0;
-    for (int64_t i0 = 0; i0 < n_my && !abort; i0 += 32) {
-      // lanes fetch the slot ids and gates of the next 32 tiles
-      const int64_t ii = i0 + lane;
-      int32_t rs = -1, ws = -1;
-      float gg = 1.0f, bb = 1.0f;
-      if (ii < n_my) {
-        const int64_t t = blockIdx.x + ii * gridDim.x;
-        const int b = (int)(t / H);
-        rs = p.read_slot ? __ldg(p.read_slot + b) : b;
-        ws = p.write_slot ? __ldg(p.write_slot + b) : b;
-        if (Rule<RULE>::kUsesGate) gg = __ldg(p.g + t);
-        if (Rule<RULE>::kUsesBeta) bb = __ldg(p.beta + t);
-      }
-      const int cnt = (int)((n_my - i0) < 32 ? (n_my - i0) : 32);
-      for (int j = 0; j < cnt; ++j) {
-        const int32_t rs_j = __shfl_sync(0xffffffffu, rs, j);
-        const int32_t ws_j = __shfl_sync(0xffffffffu, ws, j);
-        const float g_j = __shfl_sync(0xffffffffu, gg, j);
-        const float b_j = __shfl_sync(0xffffffffu, bb, j);
-        const int64_t it = i0 + j;
-        const int stage = (int)(it % C::kStages);
-        const uint32_t round = (uint32_t)(it / C::kStages);
-        bool ok = true;
-        if (lane == 0) {
-          ok = mbar_wait(&empty[stage], (round & 1u) ^ 1u, p.wait_ns);
-          if (ok && blockIdx.x == 0 && it == p.withhold) {
-            // test hook: this tile's copies are never issued and its arrival never comes (its
-            // consumers' waits run out); nothing of it is in flight, and the rest is abandoned
-            ok = false;
-          } else if (ok) {
-            const int64_t t = blockIdx.x + it * gridDim.x;
-            const int b = (int)(t / H);
-            const int h = (int)(t % H);
-            const int hq = h / ratio;
-            const bool rs_ok = rs_j >= 0 && rs_j < p.src_slots;
-            const bool ws_ok = ws_j >= 0 && ws_j < p.dst_slots;
-            bool mask_ok = true;
-            if constexpr (C::kQ8) {
-              // a head's masks must mark exactly n_hp rows, or the row ranks leave the tile
-              int cs = 0, cd = 0;
-#pragma unroll
-              for (int w = 0; w < DK / 32; ++w) {
-                cs += __popc(__ldg(p.src_mask + h * (DK / 32) + w));
-                cd += __popc(__ldg(p.dst_mask + h * (DK / 32) + w));
-              }
-              mask_ok = cs == p.n_hp && cd == p.n_hp;
-              if (!mask_ok) report(p.err, LA_DEVERR_Q8_MASK);
-            }
-            StepMeta m;
-            m.g = g_j;
-            m.beta = b_j;
-            m.valid = rs_ok && ws_ok && mask_ok;
-            m.ws = ws_j;
-            m.dst_off = ((int64_t)ws_j * H + h) * tile_bytes;
-            m.o_off = t * qg * DV;  // o row of the tile's first query
-            meta[stage] = m;
-            if (m.valid) {
-              unsigned char* sb = smem + stage * C::kStageBytes;
-              // query rows: the tile's q/k head, or its qg consecutive query heads
-              const int64_t qrow = QGRP ? t * qg : (int64_t)b * p.n_qk_heads + hq;
-              const int hist_bytes = CONV ? (2 * DK + DV) * (p.conv_w - 1) * (int)sizeof(IT) : 0;
-              const int wbytes = CONV ? (2 * DK + DV) * p.conv_w * 4 : 0;
-              mbar_arrive_expect_tx(&full[stage],
-                                    C::kOffHist - C::kOffK + tile_bytes + qg * C::kQKBytes + hist_bytes + wbytes);
-              bulk_g2s_hint(sb, src + ((int64_t)rs_j * H + h) * tile_bytes, tile_bytes, &full[stage], pol_stream);
-              bulk_g2s(sb + C::kTileBytes, q + qrow * DK, qg * C::kQKBytes, &full[stage]);
-              bulk_g2s(sb + C::kOffK, k + ((int64_t)b * p.n_qk_heads + hq) * DK, C::kQKBytes, &full[stage]);
-              bulk_g2s(sb + C::kOffV, v + t * DV, C::kVBytes, &full[stage]);
-              if (CHG) bulk_g2s(sb + C::kOffA, p.g + t * DK, C::kGBytes, &full[stage]);
-              if (CONV) {
-                bulk_g2s(sb + C::kOffHist,
-                         static_cast<const unsigned char*>(p.conv_src) + ((int64_t)rs_j * H + h) * hist_bytes,
-                         hist_bytes, &full[stage]);
-                // the weights of the tile's q/k head and head (the same for every request)
-                const int W = p.conv_w;
-                bulk_g2s(sb + C::kOffConvW, p.conv_wq + (int64_t)hq * DK * W, DK * W * 4, &full[stage]);
-                bulk_g2s(sb + C::kOffConvW + DK * W * 4, p.conv_wk + (int64_t)hq * DK * W, DK * W * 4, &full[stage]);
-                bulk_g2s(sb + C::kOffConvW + 2 * DK * W * 4, p.conv_wv + (int64_t)h * DV * W, DV * W * 4,
-                         &full[stage]);
-              }
-            } else {
-              if (!rs_ok || !ws_ok) report(p.err, (rs_ok ? 0u : LA_DEVERR_READ_SLOT) | (ws_ok ? 0u : LA_DEVERR_WRITE_SLOT));
-              mbar_arrive(&full[stage]);
-            }
-          } else {
-            report(p.err, LA_DEVERR_TIMEOUT);
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) {
-          abort = true;
-          break;
-        }
-        ++issued;
-      }
-    }
-    // Never retire with copies in flight: wait for the last phase issued on each stage.
-    if (lane == 0) {
-      for (int s = 0; s < C::kStages; ++s) {
-        if (issued > s) {
-          const int64_t last = issued - 1 - ((issued - 1 - s) % C::kStages);
-          if (blockIdx.x == 0 && last == p.withhold) continue;  // withheld: nothing issued
-          if (!mbar_wait(&full[s], (uint32_t)(last / C::kStages) & 1u, p.wait_ns)) report(p.err, LA_DEVERR_TIMEOUT);
-        }
-      }
-    }
+    step_producer<RULE, DK, DV, ST, IT, QGRP, CONV, C>(p, smem, meta, full, empty, n_my, lane);
     return;
   }
 

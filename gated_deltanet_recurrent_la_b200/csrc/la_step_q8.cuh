@@ -1,0 +1,373 @@
+// la_step_q8.cuh -- the decode step on q8 state pools whose source and destination share
+// one channel mask (the in-place decode of a serving pool: the same pool, or pools with
+// the same mask array).
+//
+// The q8 format (DAMP-style mixed storage, "Seven Architectures Replacing KV Cache With
+// Bounded Mutable State", sections "ONNX LinearAttention / FlashInfer" and Practical
+// Implications) stores a tile's rows in two blocks: the INT8 rows (codes, then one FP32
+// scale per 32 columns) and the BF16 rows, each block in increasing key channel.  With one
+// mask for both tiles a row has the same place in the source and the destination, so the
+// lanes here walk the rows in that storage order: lane block rb takes storage rows
+// 8 r + rb (r = 0 .. d_k / 8 - 1), the INT8 rows first.  At each r all lanes then see the
+// same kind of row (when the number of INT8 rows is a multiple of 8; otherwise one r is
+// mixed), so the warp does not diverge, and the key channel of a row only matters for its
+// key, query and decay, which each warp gathers once per tile into row order.
+//
+// Arithmetic (same update and readout as the other step kernels, FP32):
+//  * an INT8 row is held as its exact integer codes and the group scale s; the sums take
+//    sum_i code_ij (s_i k_i), the update a S + k u^T takes code (a s) + k u;
+//  * codes become floats without the conversion unit: the byte, offset by 128, placed in
+//    the mantissa of 2^23 and 2^23 + 128 subtracted (exact);
+//  * new codes are rint(y * inv) as the codec rounds them: the product rounded to FP32, then
+//    added to 1.5 * 2^23, whose low byte is then the two's-complement code (exact for
+//    |y * inv| < 2^22, and |y * inv| <= 127.00002 here);  a row group holding a non-finite
+//    value (rare) takes the codec's own conversion, which sends NaN to 0;
+//  * the pairwise products run as packed FP32 pairs (FFMA2 / FMUL2 / FADD2: the same
+//    correctly rounded results as two scalar operations, half the instructions);
+//  * two passes over the staged tile (sums, then update and store) instead of holding the
+//    tile in registers: a thread needs few registers, so three tiles are in compute per SM
+//    (twelve consumer warps) to hide the latencies of one warp per tile strip.
+#pragma once
+
+#include "la_step.cuh"
+
+namespace la {
+
+#ifndef LA_Q8S_CONSUMER_WARPS
+#define LA_Q8S_CONSUMER_WARPS 12
+#endif
+
+// Stage layout of the generic step (StepCfg) with NCW consumer warps, each with its own
+// row-ordered key / query / decay vectors after the stages.
+template <int DK, int DV, typename IT, bool CHG, int NCW>
+struct Q8sCfg : StepCfg<DK, DV, q8_t, IT, CHG> {
+  using Base = StepCfg<DK, DV, q8_t, IT, CHG>;
+  static constexpr int kConsumerWarps = NCW;
+  static constexpr int kTeams = NCW / Base::kWPT;
+  static constexpr int kThreads = (NCW + 1) * 32;
+  static constexpr int kPermFloats = 3 * DK;  // k | q | alpha, in lane-major row order
+  static constexpr int kFixed = NCW * kPermFloats * 4 + 12 * ((int)sizeof(StepMeta) + 16) + 64;
+  static constexpr int kStages = cmax(2, cmin(12, (227 * 1024 - kFixed) / Base::kStageBytes));
+  static constexpr int kOffMeta = kStages * Base::kStageBytes;
+  static constexpr int kOffBars = round_up(kOffMeta + kStages * (int)sizeof(StepMeta), 8);
+  static constexpr int kOffPerm = round_up(kOffBars + 2 * kStages * 8, 16);
+  static constexpr int kSmem = kOffPerm + NCW * kPermFloats * 4;
+  static_assert(NCW % Base::kWPT == 0, "whole tiles per team");
+  static_assert(Base::kVec == 8 && Base::kNCH == 4 && Base::kRG == 8, "lanes: 4 x 8 columns by 8 row blocks");
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+};
+
+// max that keeps a NaN (so that one compare tells a row group holding a non-finite value)
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// 8 signed codes (little-endian bytes) -> their exact values as floats
+__device__ __forceinline__ void q8s_codes(uint2 w, float* c) {
+  const uint32_t x[2] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u};
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      c[4 * i + b] = __uint_as_float(__byte_perm(x[i], 0x4B000000u, 0x7540u | b));
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    const float2 r = __fadd2_rn(make_float2(c[e], c[e + 1]), make_float2(-8388736.0f, -8388736.0f));
+    c[e] = r.x; c[e + 1] = r.y;
+  }
+}
+
+// codes rint(y * inv) of 8 finite values with |y| <= the group's absmax, packed into 8 bytes
+__device__ __forceinline__ void q8s_pack(const float* y, float inv, uint32_t* w) {
+  uint32_t b[8];
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    const float2 r = __fadd2_rn(__fmul2_rn(make_float2(y[e], y[e + 1]), make_float2(inv, inv)),
+                                make_float2(12582912.0f, 12582912.0f));
+    b[e] = __float_as_uint(r.x); b[e + 1] = __float_as_uint(r.y);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    w[i] = __byte_perm(__byte_perm(b[4 * i], b[4 * i + 1], 0x0040u), __byte_perm(b[4 * i + 2], b[4 * i + 3], 0x0040u),
+                       0x5410u);
+}
+
+// Registers per thread: each SM sub-partition holds a quarter of the register file, and the
+// sub-partition with the most warps (the producer's) must fit all of its warps.
+constexpr int q8s_max_regs(int ncw) { return (65536 / 4) / (((ncw + 1 + 3) / 4) * 32) / 8 * 8; }
+
+template <int RULE, int DK, int DV, typename IT, int NCW>
+__global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, NCW>::kThreads)
+    __maxnreg__(q8s_max_regs(NCW) > 255 ? 255 : q8s_max_regs(NCW)) step_q8s_kernel(const StepParams p) {
+  constexpr bool CHG = Rule<RULE>::kChannelGate;
+  using C = Q8sCfg<DK, DV, IT, CHG, NCW>;
+  constexpr int RL = DK / 8;   // rows per lane
+  constexpr int NG = DV / 32;  // 32-column groups per row
+  extern __shared__ __align__(128) unsigned char smem[];
+  StepMeta* meta = reinterpret_cast<StepMeta*>(smem + C::kOffMeta);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
+  uint64_t* empty = full + C::kStages;
+
+  const int H = p.n_v_heads;
+  const int64_t ntiles = (int64_t)p.B * H;
+  const int64_t n_my = (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], C::kWPT);
+    }
+    mbar_init_fence();
+  }
+  __syncthreads();
+#if LA_STEP_PDL
+  griddep_wait();
+  griddep_launch_dependents();
+#endif
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp == NCW) {
+    step_producer<RULE, DK, DV, q8_t, IT, false, false, C>(p, smem, meta, full, empty, n_my, lane);
+    return;
+  }
+
+  const int team = warp / C::kWPT;
+  const int part = warp % C::kWPT;
+  const int ch = lane & 3;   // 8-column chunk of the warp's 32-column strip (one group)
+  const int rb = lane >> 2;  // row block: storage rows 8 r + rb
+  const int col0 = part * 32 + ch * 8;
+  const int n8 = DK - p.n_hp;
+  float* kp = reinterpret_cast<float*>(smem + C::kOffPerm) + warp * C::kPermFloats;
+  float* qp = kp + DK;
+  float* ap = qp + DK;
+  unsigned char* dst = static_cast<unsigned char*>(p.dst);
+  IT* out = static_cast<IT*>(p.o);
+  const unsigned char* sc8 = nullptr;  // (per tile) the INT8 block's scales
+  const unsigned char* hp = nullptr;   // (per tile) the BF16 rows
+
+  for (int64_t it = team; it < n_my; it += C::kTeams) {
+    const int stage = (int)(it % C::kStages);
+    const uint32_t round = (uint32_t)(it / C::kStages);
+    const bool arrived = mbar_wait(&full[stage], round & 1u, p.wait_ns);
+    if (!__all_sync(0xffffffffu, arrived)) {
+      if (lane == 0) report(p.err, LA_DEVERR_TIMEOUT);
+      return;
+    }
+    const StepMeta m = meta[stage];
+    if (m.valid) {  // (the same for the whole warp)
+      const unsigned char* sb = smem + stage * C::kStageBytes;
+      sc8 = sb + n8 * DV;
+      hp = sc8 + n8 * NG * 4;
+      const IT* qs = reinterpret_cast<const IT*>(sb + C::kTileBytes);
+      const IT* ks = reinterpret_cast<const IT*>(sb + C::kOffK);
+      const IT* vs = reinterpret_cast<const IT*>(sb + C::kOffV);
+      const float* as = reinterpret_cast<const float*>(sb + C::kOffA);
+      float a, bcoef, c;
+      Rule<RULE>::coeffs(m.g, m.beta, a, bcoef, c);
+
+      // key, query (and decay) of each storage row, stored lane-major: row 8 r + rb at
+      // rb * RL + r.  Lane j places key channels j, j + 32, ...; the producer has checked
+      // that the mask marks exactly n_hp rows, so every place is inside the vectors.
+      {
+        const int h = (int)((blockIdx.x + it * gridDim.x) % H);
+        const uint32_t* mk = p.src_mask + h * (DK / 32);
+        int below = 0;
+#pragma unroll
+        for (int w = 0; w < DK / 32; ++w) {
+          const uint32_t mw = __ldg(mk + w);
+          const int cix = 32 * w + lane;
+          const int pre = below + __popc(mw & ((1u << lane) - 1u));
+          below += __popc(mw);
+          const int vr = ((mw >> lane) & 1u) ? n8 + pre : cix - pre;
+          const int pos = (vr & 7) * RL + (vr >> 3);
+          kp[pos] = io_load(ks + cix);
+          qp[pos] = io_load(qs + cix);
+          if (CHG) ap[pos] = as[cix];
+        }
+        __syncwarp();
+      }
+
+      // a storage row of the warp's strip: its 8 values as code, scale (s = 1 for BF16 rows)
+      auto load_row = [&](int vr, float* cv, float& s) {
+        if (vr < n8) {
+          q8s_codes(*reinterpret_cast<const uint2*>(sb + vr * DV + col0), cv);
+          s = *reinterpret_cast<const float*>(sc8 + (vr * NG + part) * 4);
+        } else {
+          StateVec<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(hp + ((vr - n8) * DV + col0) * 2), cv);
+          s = 1.0f;
+        }
+      };
+
+      // pass 1: k.q, S^T k and S^T q (kda: the rows' decays scale the keys of both sums)
+      float kq = 0.0f, pp[8], rr[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) pp[j] = rr[j] = 0.0f;
+#pragma unroll
+      for (int r0 = 0; r0 < RL; r0 += 4) {
+        const float4 k4 = *reinterpret_cast<const float4*>(kp + rb * RL + r0);
+        const float4 q4 = *reinterpret_cast<const float4*>(qp + rb * RL + r0);
+        float4 a4 = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+        if (CHG) a4 = *reinterpret_cast<const float4*>(ap + rb * RL + r0);
+        const float kk4[4] = {k4.x, k4.y, k4.z, k4.w}, qq4[4] = {q4.x, q4.y, q4.z, q4.w};
+        const float aa4[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          float cv[8], s;
+          load_row((r0 + r) * 8 + rb, cv, s);
+          kq = fmaf(kk4[r], qq4[r], kq);
+          const float k1 = s * (CHG ? kk4[r] * aa4[r] : kk4[r]);
+          const float q1 = s * (CHG ? qq4[r] * aa4[r] : qq4[r]);
+#pragma unroll
+          for (int j = 0; j < 8; j += 2) {
+            const float2 c2 = make_float2(cv[j], cv[j + 1]);
+            if (Rule<RULE>::kPredicts) {
+              const float2 r2 = __ffma2_rn(c2, make_float2(k1, k1), make_float2(pp[j], pp[j + 1]));
+              pp[j] = r2.x; pp[j + 1] = r2.y;
+            }
+            const float2 r3 = __ffma2_rn(c2, make_float2(q1, q1), make_float2(rr[j], rr[j + 1]));
+            rr[j] = r3.x; rr[j + 1] = r3.y;
+          }
+        }
+      }
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        kq += __shfl_xor_sync(0xffffffffu, kq, off);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (Rule<RULE>::kPredicts) pp[j] += __shfl_xor_sync(0xffffffffu, pp[j], off);
+          rr[j] += __shfl_xor_sync(0xffffffffu, rr[j], off);
+        }
+      }
+
+      // u = b (v - c p),  o = scale (a r + (k.q) u)
+      float u[8];
+      {
+        float vv[8], o[8];
+        load_f32<IT, 8>(vs + col0, vv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          u[j] = bcoef * (vv[j] - c * pp[j]);
+          o[j] = p.scale * fmaf(a, rr[j], kq * u[j]);
+        }
+        if (rb == 0) store_f32<IT, 8>(out + m.o_off + col0, o);
+      }
+
+      // pass 2: S' = a S + k u^T, stored in the tile's format at the same storage rows
+      unsigned char* dtile = dst + m.dst_off;
+      unsigned char* dsc8 = dtile + n8 * DV;
+      unsigned char* dhp = dsc8 + n8 * NG * 4;
+#pragma unroll
+      for (int r0 = 0; r0 < RL; r0 += 4) {
+        const float4 k4 = *reinterpret_cast<const float4*>(kp + rb * RL + r0);
+        float4 a4 = make_float4(a, a, a, a);
+        if (CHG) a4 = *reinterpret_cast<const float4*>(ap + rb * RL + r0);
+        const float kk4[4] = {k4.x, k4.y, k4.z, k4.w}, aa4[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int vr = (r0 + r) * 8 + rb;
+          float cv[8], s;
+          load_row(vr, cv, s);
+          const float as_ = aa4[r] * s;
+          float y[8];
+#pragma unroll
+          for (int j = 0; j < 8; j += 2) {
+            const float2 r2 = __ffma2_rn(make_float2(cv[j], cv[j + 1]), make_float2(as_, as_),
+                                         __fmul2_rn(make_float2(kk4[r], kk4[r]), make_float2(u[j], u[j + 1])));
+            y[j] = r2.x; y[j + 1] = r2.y;
+          }
+          // the group's absmax over the 4 lanes holding this row of the strip
+          float amax = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) amax = fmax_nan(amax, fabsf(y[j]));
+          amax = fmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+          amax = fmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+          const bool is8 = vr < n8;
+          bool exact_path = false;
+          if (__any_sync(0xffffffffu, is8 && !(amax <= 3.402823466e38f))) {
+            // a non-finite value in some INT8 row group of the warp: the codec's absmax
+            // (NaN ignored) and conversion for this r
+            amax = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(y[j]));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            exact_path = true;
+          }
+          if (is8) {
+            float sc, inv;
+            q8_scales(amax, sc, inv);
+            uint32_t w[2];
+            if (exact_path) {
+              q8_pack<8>(y, inv, w);
+            } else {
+              q8s_pack(y, inv, w);
+            }
+            *reinterpret_cast<uint2*>(dtile + vr * DV + col0) = make_uint2(w[0], w[1]);
+            if (ch == 0) *reinterpret_cast<float*>(dsc8 + (vr * NG + part) * 4) = sc;
+          } else {
+            *reinterpret_cast<uint4*>(dhp + ((vr - n8) * DV + col0) * 2) = StateVec<__nv_bfloat16>::pack(y);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);  // this warp is done with the stage
+  }
+}
+
+template <int RULE, int DK, int DV, typename IT>
+cudaError_t launch_step_q8s(const StepParams& p, cudaStream_t stream) {
+  constexpr int NCW = LA_Q8S_CONSUMER_WARPS / (DV / 32) * (DV / 32);
+  using C = Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, NCW>;
+  const void* fn = reinterpret_cast<const void*>(&step_q8s_kernel<RULE, DK, DV, IT, NCW>);
+  const int per_sm = prepare_kernel(fn, C::kThreads, C::kSmem);
+  if (per_sm <= 0) return cudaErrorInvalidConfiguration;
+  const int64_t ntiles = (int64_t)p.B * p.n_v_heads;
+  const int64_t cap = (int64_t)device_sm_count() * per_sm;
+  const int grid = (int)(ntiles < cap ? ntiles : cap);
+#if LA_STEP_PDL
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, step_q8s_kernel<RULE, DK, DV, IT, NCW>, p);
+  if (e != cudaSuccess) return e;
+#else
+  step_q8s_kernel<RULE, DK, DV, IT, NCW><<<grid, C::kThreads, C::kSmem, stream>>>(p);
+#endif
+  return cudaGetLastError();
+}
+
+// q8 pools: the storage-order kernel when the source and destination share their mask
+// array, the generic step kernel (rows located through each mask) otherwise.
+template <int RULE, int DK, int DV, typename IT>
+cudaError_t launch_step_q8(const StepParams& p, cudaStream_t stream) {
+  if (p.src_mask == p.dst_mask) return launch_step_q8s<RULE, DK, DV, IT>(p, stream);
+  return launch_step<RULE, DK, DV, q8_t, IT, false>(p, stream);
+}
+
+inline StepLaunchFn find_step_q8_table(int rule, int dk, int dv, int io) {
+#define LA_Q8S_CASE(R, K, V)                                                                     \
+  if (rule == R && dk == K && dv == V)                                                           \
+    return io == LA_F32 ? &launch_step_q8<R, K, V, float> : &launch_step_q8<R, K, V, __nv_bfloat16>;
+#define LA_Q8S_SHAPES(R) LA_Q8S_CASE(R, 64, 64) LA_Q8S_CASE(R, 128, 64) LA_Q8S_CASE(R, 128, 128)
+  LA_Q8S_SHAPES(LA_RULE_LINEAR)
+  LA_Q8S_SHAPES(LA_RULE_GATED)
+  LA_Q8S_SHAPES(LA_RULE_DELTA)
+  LA_Q8S_SHAPES(LA_RULE_GATED_DELTA)
+  LA_Q8S_SHAPES(LA_RULE_KDA)
+#undef LA_Q8S_SHAPES
+#undef LA_Q8S_CASE
+  return nullptr;
+}
+
+}  // namespace la

@@ -89,8 +89,9 @@ def _values_of(t, dk, dv, n_hp, mask):
 
 
 @pytest.mark.parametrize("io", [F32, BF16], ids=["f32io", "bf16io"])
-@pytest.mark.parametrize("dk,dv,n_hp", [(64, 64, 8), (128, 64, 0), (128, 128, 16), (128, 128, 32)],
-                         ids=["64x64", "128x64", "128x128", "128x128hp32"])
+@pytest.mark.parametrize("dk,dv,n_hp", [(64, 64, 8), (64, 64, 6), (128, 64, 0), (128, 128, 16), (128, 128, 32),
+                                        (128, 128, 2)],
+                         ids=["64x64", "64x64hp6", "128x64", "128x128", "128x128hp32", "128x128hp2"])
 @pytest.mark.parametrize("rule", ["gated", "gated_delta", "kda"])
 def test_step_q8(rule, dk, dv, n_hp, io):
     inp = W.step_inputs(B=5, n_qk_heads=2, n_v_heads=4, d_k=dk, d_v=dv, rule=rule, n_slots=9, state_dtype=F32,
@@ -115,6 +116,75 @@ def test_step_q8(rule, dk, dv, n_hp, io):
     assert_close(np64(o.cpu()), o_ref, 1e-4 if io == F32 else 2e-2, f"{rule}: outputs")
     untouched = np.setdiff1d(np.arange(9), ws)
     assert torch.equal(after[untouched], before[untouched]), "slots not written keep their bytes"
+
+
+@pytest.mark.parametrize("dst_mask_kind", ["copy", "other"])
+@pytest.mark.parametrize("rule", ["gated_delta", "kda"])
+def test_step_q8_separate_mask_arrays(rule, dst_mask_kind):
+    """Source and destination with their own mask arrays (the kernel that locates rows
+    through each mask): a copy of the source's mask on the same pool, or a second pool with
+    another mask, against the oracle (source decoded through its mask, destination encoded
+    through its own)."""
+    dk, dv, n_hp, n_slots = 128, 128, 16, 9
+    inp = W.step_inputs(B=5, n_qk_heads=2, n_v_heads=4, d_k=dk, d_v=dv, rule=rule, n_slots=n_slots,
+                        state_dtype=F32, io_dtype=BF16, seed=131, slot_map="perm", pool_std=0.3)
+    mask = masks_of(4, dk, n_hp, 11)
+    pool, t = q8_pool(inp.pool, 2, n_hp, mask)
+    src_vals = _values_of(t, dk, dv, n_hp, mask)
+    if dst_mask_kind == "copy":
+        dmask, dt = mask.clone(), t
+        dst = L.Pool.q8(t, 2, dk, dv, n_hp, dmask.cuda())
+    else:
+        dmask = masks_of(4, dk, n_hp, 12)
+        dt = torch.zeros_like(t)
+        dst = L.Pool.q8(dt, 2, dk, dv, n_hp, dmask.cuda())
+    assert dst.mask.data_ptr() != pool.mask.data_ptr()
+    o = torch.empty(5, 4, dv, dtype=BF16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.check(L.la_state_step(rule, pool, dev(inp.read_slot), dst, dev(inp.write_slot), dev(inp.q), dev(inp.k),
+                            dev(inp.v), dev(inp.g), dev(inp.beta), inp.scale, o, err))
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ref, o_ref, e = oracle.step_q8(rule, 2, src_vals, np64(inp.q), np64(inp.k), np64(inp.v), np64(inp.g),
+                                   np64(inp.beta), inp.scale, masks=u32(dmask), io_dtype="bf16",
+                                   read_slot=inp.read_slot.numpy(), write_slot=inp.write_slot.numpy())
+    assert e == 0
+    ws = inp.write_slot.numpy()
+    assert_close(_values_of(dt, dk, dv, n_hp, dmask)[ws], ref[ws], 2e-2, f"{rule}: q8 states ({dst_mask_kind})")
+    assert_close(np64(o.cpu()), o_ref, 2e-2, f"{rule}: outputs ({dst_mask_kind})")
+
+
+def test_step_q8_nonfinite_group_takes_the_codec():
+    """An infinite value input makes every row's group of that column infinite: the codec
+    gives such a group the scale inf and all codes 0 (the infinite value's code is that of
+    NaN), while the other groups of the same rows stay finite and match the oracle."""
+    dk, dv, n_hp = 128, 128, 16
+    inp = W.step_inputs(B=2, n_qk_heads=1, n_v_heads=1, d_k=dk, d_v=dv, rule="gated_delta", n_slots=2,
+                        state_dtype=F32, io_dtype=F32, seed=132, slot_map="perm", pool_std=0.3)
+    inp.v[0, 0, 37] = float("inf")       # column 37: group 1 of request 0
+    mask = masks_of(1, dk, n_hp, 13)
+    pool, t = q8_pool(inp.pool, 1, n_hp, mask)
+    src_vals = _values_of(t, dk, dv, n_hp, mask)
+    o = torch.empty(2, 1, dv, dtype=F32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.check(L.la_state_step("gated_delta", pool, dev(inp.read_slot), pool, dev(inp.write_slot), dev(inp.q),
+                            dev(inp.k), dev(inp.v), dev(inp.g), dev(inp.beta), 1.0, o, err))
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    n8 = dk - n_hp
+    tile = t.cpu()[int(inp.write_slot[0]), 0].numpy()
+    codes = tile[:n8 * dv].view(np.int8).reshape(n8, dv)
+    scales = tile[n8 * dv:n8 * dv + n8 * 4 * 4].view(np.float32).reshape(n8, 4)
+    assert np.all(codes[:, 32:64] == 0) and np.all(np.isinf(scales[:, 1]))
+    assert np.all(np.isfinite(scales[:, [0, 2, 3]]))
+    ref, _, _ = oracle.step_q8("gated_delta", 1, src_vals, np64(inp.q), np64(inp.k), np64(inp.v), np64(inp.g),
+                               np64(inp.beta), 1.0, masks=u32(mask), io_dtype="f32",
+                               read_slot=inp.read_slot.numpy(), write_slot=inp.write_slot.numpy())
+    got = _values_of(t, dk, dv, n_hp, mask)
+    w0, w1 = int(inp.write_slot[0]), int(inp.write_slot[1])
+    finite_cols = np.r_[0:32, 64:128]
+    assert_close(got[w0][:, :, finite_cols], ref[w0][:, :, finite_cols], 2e-2, "finite groups of request 0")
+    assert_close(got[w1], ref[w1], 2e-2, "request 1")
 
 
 @pytest.mark.parametrize("src_kind,dst_kind", [("q8", "q8"), ("f32", "q8"), ("q8", "bf16")])
