@@ -7,11 +7,14 @@
 // Implications) stores a tile's rows in two blocks: the INT8 rows (codes, then one FP32
 // scale per 32 columns) and the BF16 rows, each block in increasing key channel.  With one
 // mask for both tiles a row has the same place in the source and the destination, so the
-// lanes here walk the rows in that storage order: lane block rb takes storage rows
-// 8 r + rb (r = 0 .. d_k / 8 - 1), the INT8 rows first.  At each r all lanes then see the
-// same kind of row (when the number of INT8 rows is a multiple of 8; otherwise one r is
-// mixed), so the warp does not diverge, and the key channel of a row only matters for its
-// key, query and decay, which each warp gathers once per tile into row order.
+// lanes here walk the rows in that storage order.  Each warp owns one 32-column group (a
+// strip) of a tile; lane (rb, hf) holds columns hf * 16 .. hf * 16 + 15 of the strip in the
+// storage rows 16 m + rb (m = 0 .. d_k / 16 - 1), the INT8 rows first.  At each m all lanes
+// then see the same kind of row (when the number of INT8 rows is a multiple of 16;
+// otherwise one m is mixed), so the warp does not diverge, and the key channel of a row
+// only matters for its key, query and decay, which each warp gathers once per tile into
+// row order.  A group's absmax is one shuffle between the two halves, and its scale is
+// computed once per 16 values.
 //
 // Arithmetic (same update and readout as the other step kernels, FP32):
 //  * an INT8 row is held as its exact integer codes and the group scale s; the sums take
@@ -24,6 +27,9 @@
 //    value (rare) takes the codec's own conversion, which sends NaN to 0;
 //  * the pairwise products run as packed FP32 pairs (FFMA2 / FMUL2 / FADD2: the same
 //    correctly rounded results as two scalar operations, half the instructions);
+//  * the column sums S^T k and S^T q meet across the 16 row blocks by recursive halving
+//    (each lane ends with the two sums of one column, which gives that column's u and o);
+//    u goes to the warp's lanes through shared memory;
 //  * two passes over the staged tile (sums, then update and store) instead of holding the
 //    tile in registers: a thread needs few registers, so three tiles are in compute per SM
 //    (twelve consumer warps) to hide the latencies of one warp per tile strip.
@@ -38,14 +44,14 @@ namespace la {
 #endif
 
 // Stage layout of the generic step (StepCfg) with NCW consumer warps, each with its own
-// row-ordered key / query / decay vectors after the stages.
+// row-ordered key / query / decay vectors and a u vector of its strip after the stages.
 template <int DK, int DV, typename IT, bool CHG, int NCW>
 struct Q8sCfg : StepCfg<DK, DV, q8_t, IT, CHG> {
   using Base = StepCfg<DK, DV, q8_t, IT, CHG>;
   static constexpr int kConsumerWarps = NCW;
   static constexpr int kTeams = NCW / Base::kWPT;
   static constexpr int kThreads = (NCW + 1) * 32;
-  static constexpr int kPermFloats = 3 * DK;  // k | q | alpha, in lane-major row order
+  static constexpr int kPermFloats = 3 * DK + 32;  // k | q | alpha (lane-major row order) | u
   static constexpr int kFixed = NCW * kPermFloats * 4 + 12 * ((int)sizeof(StepMeta) + 16) + 64;
   static constexpr int kStages = cmax(2, cmin(12, (227 * 1024 - kFixed) / Base::kStageBytes));
   static constexpr int kOffMeta = kStages * Base::kStageBytes;
@@ -53,7 +59,7 @@ struct Q8sCfg : StepCfg<DK, DV, q8_t, IT, CHG> {
   static constexpr int kOffPerm = round_up(kOffBars + 2 * kStages * 8, 16);
   static constexpr int kSmem = kOffPerm + NCW * kPermFloats * 4;
   static_assert(NCW % Base::kWPT == 0, "whole tiles per team");
-  static_assert(Base::kVec == 8 && Base::kNCH == 4 && Base::kRG == 8, "lanes: 4 x 8 columns by 8 row blocks");
+  static_assert(DV % 32 == 0 && DK % 64 == 0, "32-column strips, 16 row blocks of a multiple of 4 rows");
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
@@ -64,32 +70,36 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
   return r;
 }
 
-// 8 signed codes (little-endian bytes) -> their exact values as floats
-__device__ __forceinline__ void q8s_codes(uint2 w, float* c) {
-  const uint32_t x[2] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u};
+// N signed codes (little-endian bytes of N / 4 words) -> their exact values as floats
+template <int N>
+__device__ __forceinline__ void q8s_codes(const uint32_t* words, float* c) {
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < N / 4; ++i) {
+    const uint32_t x = words[i] ^ 0x80808080u;
 #pragma unroll
-    for (int b = 0; b < 4; ++b)
-      c[4 * i + b] = __uint_as_float(__byte_perm(x[i], 0x4B000000u, 0x7540u | b));
+    for (int b = 0; b < 4; ++b) c[4 * i + b] = __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7540u | b));
+  }
 #pragma unroll
-  for (int e = 0; e < 8; e += 2) {
+  for (int e = 0; e < N; e += 2) {
     const float2 r = __fadd2_rn(make_float2(c[e], c[e + 1]), make_float2(-8388736.0f, -8388736.0f));
-    c[e] = r.x; c[e + 1] = r.y;
+    c[e] = r.x;
+    c[e + 1] = r.y;
   }
 }
 
-// codes rint(y * inv) of 8 finite values with |y| <= the group's absmax, packed into 8 bytes
+// codes rint(y * inv) of N finite values with |y| <= the group's absmax, packed into N bytes
+template <int N>
 __device__ __forceinline__ void q8s_pack(const float* y, float inv, uint32_t* w) {
-  uint32_t b[8];
+  uint32_t b[N];
 #pragma unroll
-  for (int e = 0; e < 8; e += 2) {
+  for (int e = 0; e < N; e += 2) {
     const float2 r = __fadd2_rn(__fmul2_rn(make_float2(y[e], y[e + 1]), make_float2(inv, inv)),
                                 make_float2(12582912.0f, 12582912.0f));
-    b[e] = __float_as_uint(r.x); b[e + 1] = __float_as_uint(r.y);
+    b[e] = __float_as_uint(r.x);
+    b[e + 1] = __float_as_uint(r.y);
   }
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < N / 4; ++i)
     w[i] = __byte_perm(__byte_perm(b[4 * i], b[4 * i + 1], 0x0040u), __byte_perm(b[4 * i + 2], b[4 * i + 3], 0x0040u),
                        0x5410u);
 }
@@ -102,8 +112,9 @@ template <int RULE, int DK, int DV, typename IT, int NCW>
 __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, NCW>::kThreads)
     __maxnreg__(q8s_max_regs(NCW) > 255 ? 255 : q8s_max_regs(NCW)) step_q8s_kernel(const StepParams p) {
   constexpr bool CHG = Rule<RULE>::kChannelGate;
+  constexpr bool PRED = Rule<RULE>::kPredicts;
   using C = Q8sCfg<DK, DV, IT, CHG, NCW>;
-  constexpr int RL = DK / 8;   // rows per lane
+  constexpr int RL = DK / 16;  // rows per lane
   constexpr int NG = DV / 32;  // 32-column groups per row
   extern __shared__ __align__(128) unsigned char smem[];
   StepMeta* meta = reinterpret_cast<StepMeta*>(smem + C::kOffMeta);
@@ -136,17 +147,16 @@ __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, N
 
   const int team = warp / C::kWPT;
   const int part = warp % C::kWPT;
-  const int ch = lane & 3;   // 8-column chunk of the warp's 32-column strip (one group)
-  const int rb = lane >> 2;  // row block: storage rows 8 r + rb
-  const int col0 = part * 32 + ch * 8;
+  const int hf = lane & 1;   // half of the warp's 32-column strip (one group)
+  const int rb = lane >> 1;  // row block: storage rows 16 m + rb
+  const int c0 = part * 32 + hf * 16;
   const int n8 = DK - p.n_hp;
   float* kp = reinterpret_cast<float*>(smem + C::kOffPerm) + warp * C::kPermFloats;
   float* qp = kp + DK;
   float* ap = qp + DK;
+  float* us = ap + DK;  // u of the strip's 32 columns
   unsigned char* dst = static_cast<unsigned char*>(p.dst);
   IT* out = static_cast<IT*>(p.o);
-  const unsigned char* sc8 = nullptr;  // (per tile) the INT8 block's scales
-  const unsigned char* hp = nullptr;   // (per tile) the BF16 rows
 
   for (int64_t it = team; it < n_my; it += C::kTeams) {
     const int stage = (int)(it % C::kStages);
@@ -159,8 +169,8 @@ __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, N
     const StepMeta m = meta[stage];
     if (m.valid) {  // (the same for the whole warp)
       const unsigned char* sb = smem + stage * C::kStageBytes;
-      sc8 = sb + n8 * DV;
-      hp = sc8 + n8 * NG * 4;
+      const unsigned char* sc8 = sb + n8 * DV;      // the INT8 block's scales
+      const unsigned char* hp = sc8 + n8 * NG * 4;  // the BF16 rows
       const IT* qs = reinterpret_cast<const IT*>(sb + C::kTileBytes);
       const IT* ks = reinterpret_cast<const IT*>(sb + C::kOffK);
       const IT* vs = reinterpret_cast<const IT*>(sb + C::kOffV);
@@ -168,8 +178,8 @@ __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, N
       float a, bcoef, c;
       Rule<RULE>::coeffs(m.g, m.beta, a, bcoef, c);
 
-      // key, query (and decay) of each storage row, stored lane-major: row 8 r + rb at
-      // rb * RL + r.  Lane j places key channels j, j + 32, ...; the producer has checked
+      // key, query (and decay) of each storage row, stored lane-major: row 16 m + rb at
+      // rb * RL + m.  Lane j places key channels j, j + 32, ...; the producer has checked
       // that the mask marks exactly n_hp rows, so every place is inside the vectors.
       {
         const int h = (int)((blockIdx.x + it * gridDim.x) % H);
@@ -182,7 +192,7 @@ __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, N
           const int pre = below + __popc(mw & ((1u << lane) - 1u));
           below += __popc(mw);
           const int vr = ((mw >> lane) & 1u) ? n8 + pre : cix - pre;
-          const int pos = (vr & 7) * RL + (vr >> 3);
+          const int pos = (vr & 15) * RL + (vr >> 4);
           kp[pos] = io_load(ks + cix);
           qp[pos] = io_load(qs + cix);
           if (CHG) ap[pos] = as[cix];
@@ -190,69 +200,101 @@ __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, N
         __syncwarp();
       }
 
-      // a storage row of the warp's strip: its 8 values as code, scale (s = 1 for BF16 rows)
+      // a storage row of the lane's 16 columns: values as code, scale (s = 1 for BF16 rows)
       auto load_row = [&](int vr, float* cv, float& s) {
         if (vr < n8) {
-          q8s_codes(*reinterpret_cast<const uint2*>(sb + vr * DV + col0), cv);
+          const uint4 w = *reinterpret_cast<const uint4*>(sb + vr * DV + c0);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+          q8s_codes<16>(ww, cv);
           s = *reinterpret_cast<const float*>(sc8 + (vr * NG + part) * 4);
         } else {
-          StateVec<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(hp + ((vr - n8) * DV + col0) * 2), cv);
+          const uint4* w = reinterpret_cast<const uint4*>(hp + ((vr - n8) * DV + c0) * 2);
+          StateVec<__nv_bfloat16>::unpack(w[0], cv);
+          StateVec<__nv_bfloat16>::unpack(w[1], cv + 8);
           s = 1.0f;
         }
       };
 
       // pass 1: k.q, S^T k and S^T q (kda: the rows' decays scale the keys of both sums)
-      float kq = 0.0f, pp[8], rr[8];
+      float kq = 0.0f, pp[16], rr[16];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) pp[j] = rr[j] = 0.0f;
+      for (int j = 0; j < 16; ++j) pp[j] = rr[j] = 0.0f;
 #pragma unroll
-      for (int r0 = 0; r0 < RL; r0 += 4) {
-        const float4 k4 = *reinterpret_cast<const float4*>(kp + rb * RL + r0);
-        const float4 q4 = *reinterpret_cast<const float4*>(qp + rb * RL + r0);
+      for (int m0 = 0; m0 < RL; m0 += 4) {
+        const float4 k4 = *reinterpret_cast<const float4*>(kp + rb * RL + m0);
+        const float4 q4 = *reinterpret_cast<const float4*>(qp + rb * RL + m0);
         float4 a4 = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
-        if (CHG) a4 = *reinterpret_cast<const float4*>(ap + rb * RL + r0);
+        if (CHG) a4 = *reinterpret_cast<const float4*>(ap + rb * RL + m0);
         const float kk4[4] = {k4.x, k4.y, k4.z, k4.w}, qq4[4] = {q4.x, q4.y, q4.z, q4.w};
         const float aa4[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          float cv[8], s;
-          load_row((r0 + r) * 8 + rb, cv, s);
-          kq = fmaf(kk4[r], qq4[r], kq);
-          const float k1 = s * (CHG ? kk4[r] * aa4[r] : kk4[r]);
-          const float q1 = s * (CHG ? qq4[r] * aa4[r] : qq4[r]);
+        for (int mi = 0; mi < 4; ++mi) {
+          float cv[16], s;
+          load_row((m0 + mi) * 16 + rb, cv, s);
+          kq = fmaf(kk4[mi], qq4[mi], kq);
+          const float k1 = s * (CHG ? kk4[mi] * aa4[mi] : kk4[mi]);
+          const float q1 = s * (CHG ? qq4[mi] * aa4[mi] : qq4[mi]);
 #pragma unroll
-          for (int j = 0; j < 8; j += 2) {
+          for (int j = 0; j < 16; j += 2) {
             const float2 c2 = make_float2(cv[j], cv[j + 1]);
-            if (Rule<RULE>::kPredicts) {
+            if (PRED) {
               const float2 r2 = __ffma2_rn(c2, make_float2(k1, k1), make_float2(pp[j], pp[j + 1]));
-              pp[j] = r2.x; pp[j + 1] = r2.y;
+              pp[j] = r2.x;
+              pp[j + 1] = r2.y;
             }
             const float2 r3 = __ffma2_rn(c2, make_float2(q1, q1), make_float2(rr[j], rr[j + 1]));
-            rr[j] = r3.x; rr[j + 1] = r3.y;
+            rr[j] = r3.x;
+            rr[j + 1] = r3.y;
           }
         }
       }
+      // k.q over the row blocks; the column sums by recursive halving over the row blocks
+      // (lane bits 4 .. 1): the values v = (p_0, r_0, p_1, r_1, ...) (without the p when the
+      // rule does not predict) halve at each step, and lane (rb, hf) ends with column rb
+      // of its half: v[0] = p, v[1] = r (or v[0] = r)
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        kq += __shfl_xor_sync(0xffffffffu, kq, off);
+      for (int off = 2; off < 32; off <<= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+      constexpr int NV = PRED ? 32 : 16;
+      float v[NV];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (Rule<RULE>::kPredicts) pp[j] += __shfl_xor_sync(0xffffffffu, pp[j], off);
-          rr[j] += __shfl_xor_sync(0xffffffffu, rr[j], off);
+      for (int j = 0; j < 16; ++j) {
+        if (PRED) {
+          v[2 * j] = pp[j];
+          v[2 * j + 1] = rr[j];
+        } else {
+          v[j] = rr[j];
         }
       }
-
-      // u = b (v - c p),  o = scale (a r + (k.q) u)
-      float u[8];
-      {
-        float vv[8], o[8];
-        load_f32<IT, 8>(vs + col0, vv);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          u[j] = bcoef * (vv[j] - c * pp[j]);
-          o[j] = p.scale * fmaf(a, rr[j], kq * u[j]);
+      for (int st = 0; st < 4; ++st) {
+        const int half = NV >> (st + 1);
+        const bool upper = (rb >> (3 - st)) & 1;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+          const float send = upper ? v[i] : v[i + half];
+          const float keep = upper ? v[i + half] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16 >> st);
         }
-        if (rb == 0) store_f32<IT, 8>(out + m.o_off + col0, o);
+      }
+      const float pcol = PRED ? v[0] : 0.0f;
+      const float rcol = PRED ? v[1] : v[0];
+
+      // u = b (v - c p),  o = scale (a r + (k.q) u) of column c0 + rb; u to the warp
+      {
+        const int col = c0 + rb;
+        const float uc = bcoef * (io_load(vs + col) - c * pcol);
+        io_store(out + m.o_off + col, p.scale * fmaf(a, rcol, kq * uc));
+        us[hf * 16 + rb] = uc;
+        __syncwarp();
+      }
+      float u[16];
+#pragma unroll
+      for (int j = 0; j < 16; j += 4) {
+        const float4 u4 = *reinterpret_cast<const float4*>(us + hf * 16 + j);
+        u[j] = u4.x;
+        u[j + 1] = u4.y;
+        u[j + 2] = u4.z;
+        u[j + 3] = u4.w;
       }
 
       // pass 2: S' = a S + k u^T, stored in the tile's format at the same storage rows
@@ -260,55 +302,56 @@ __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, N
       unsigned char* dsc8 = dtile + n8 * DV;
       unsigned char* dhp = dsc8 + n8 * NG * 4;
 #pragma unroll
-      for (int r0 = 0; r0 < RL; r0 += 4) {
-        const float4 k4 = *reinterpret_cast<const float4*>(kp + rb * RL + r0);
+      for (int m0 = 0; m0 < RL; m0 += 4) {
+        const float4 k4 = *reinterpret_cast<const float4*>(kp + rb * RL + m0);
         float4 a4 = make_float4(a, a, a, a);
-        if (CHG) a4 = *reinterpret_cast<const float4*>(ap + rb * RL + r0);
+        if (CHG) a4 = *reinterpret_cast<const float4*>(ap + rb * RL + m0);
         const float kk4[4] = {k4.x, k4.y, k4.z, k4.w}, aa4[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int vr = (r0 + r) * 8 + rb;
-          float cv[8], s;
+        for (int mi = 0; mi < 4; ++mi) {
+          const int vr = (m0 + mi) * 16 + rb;
+          float cv[16], s;
           load_row(vr, cv, s);
-          const float as_ = aa4[r] * s;
-          float y[8];
+          const float as_ = aa4[mi] * s;
+          float y[16];
 #pragma unroll
-          for (int j = 0; j < 8; j += 2) {
+          for (int j = 0; j < 16; j += 2) {
             const float2 r2 = __ffma2_rn(make_float2(cv[j], cv[j + 1]), make_float2(as_, as_),
-                                         __fmul2_rn(make_float2(kk4[r], kk4[r]), make_float2(u[j], u[j + 1])));
-            y[j] = r2.x; y[j + 1] = r2.y;
+                                         __fmul2_rn(make_float2(kk4[mi], kk4[mi]), make_float2(u[j], u[j + 1])));
+            y[j] = r2.x;
+            y[j + 1] = r2.y;
           }
-          // the group's absmax over the 4 lanes holding this row of the strip
+          // the group's absmax: this lane's 16 values, then the other half's
           float amax = 0.0f;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) amax = fmax_nan(amax, fabsf(y[j]));
+          for (int j = 0; j < 16; ++j) amax = fmax_nan(amax, fabsf(y[j]));
           amax = fmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-          amax = fmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
           const bool is8 = vr < n8;
           bool exact_path = false;
           if (__any_sync(0xffffffffu, is8 && !(amax <= 3.402823466e38f))) {
             // a non-finite value in some INT8 row group of the warp: the codec's absmax
-            // (NaN ignored) and conversion for this r
+            // (NaN ignored) and conversion for this m
             amax = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(y[j]));
+            for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(y[j]));
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
             exact_path = true;
           }
           if (is8) {
             float sc, inv;
             q8_scales(amax, sc, inv);
-            uint32_t w[2];
+            uint32_t w[4];
             if (exact_path) {
-              q8_pack<8>(y, inv, w);
+              q8_pack<16>(y, inv, w);
             } else {
-              q8s_pack(y, inv, w);
+              q8s_pack<16>(y, inv, w);
             }
-            *reinterpret_cast<uint2*>(dtile + vr * DV + col0) = make_uint2(w[0], w[1]);
-            if (ch == 0) *reinterpret_cast<float*>(dsc8 + (vr * NG + part) * 4) = sc;
+            *reinterpret_cast<uint4*>(dtile + vr * DV + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+            if (hf == 0) *reinterpret_cast<float*>(dsc8 + (vr * NG + part) * 4) = sc;
           } else {
-            *reinterpret_cast<uint4*>(dhp + ((vr - n8) * DV + col0) * 2) = StateVec<__nv_bfloat16>::pack(y);
+            uint4* d = reinterpret_cast<uint4*>(dhp + ((vr - n8) * DV + c0) * 2);
+            d[0] = StateVec<__nv_bfloat16>::pack(y);
+            d[1] = StateVec<__nv_bfloat16>::pack(y + 8);
           }
         }
       }
