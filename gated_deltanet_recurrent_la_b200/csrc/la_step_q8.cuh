@@ -108,7 +108,10 @@ __device__ __forceinline__ void q8s_pack(const float* y, float inv, uint32_t* w)
 // sub-partition with the most warps (the producer's) must fit all of its warps.
 constexpr int q8s_max_regs(int ncw) { return (65536 / 4) / (((ncw + 1 + 3) / 4) * 32) / 8 * 8; }
 
-template <int RULE, int DK, int DV, typename IT, int NCW>
+// NB >= 0: the pool keeps n_hp = 16 NB rows in BF16, so a lane's last NB row steps are the
+// BF16 rows and every row's kind is known at compile time (no branch per row); NB < 0: any
+// even n_hp, each row's kind decided at run time.
+template <int RULE, int DK, int DV, typename IT, int NCW, int NB>
 __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, NCW>::kThreads)
     __maxnreg__(q8s_max_regs(NCW) > 255 ? 255 : q8s_max_regs(NCW)) step_q8s_kernel(const StepParams p) {
   constexpr bool CHG = Rule<RULE>::kChannelGate;
@@ -150,7 +153,7 @@ __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, N
   const int hf = lane & 1;   // half of the warp's 32-column strip (one group)
   const int rb = lane >> 1;  // row block: storage rows 16 m + rb
   const int c0 = part * 32 + hf * 16;
-  const int n8 = DK - p.n_hp;
+  const int n8 = NB >= 0 ? DK - 16 * NB : DK - p.n_hp;
   float* kp = reinterpret_cast<float*>(smem + C::kOffPerm) + warp * C::kPermFloats;
   float* qp = kp + DK;
   float* ap = qp + DK;
@@ -200,9 +203,12 @@ __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, N
         __syncwarp();
       }
 
+      // whether row step ms (storage row 16 ms + rb) is an INT8 row
+      auto int8_row = [&](int ms) { return NB >= 0 ? ms < RL - NB : 16 * ms + rb < n8; };
       // a storage row of the lane's 16 columns: values as code, scale (s = 1 for BF16 rows)
-      auto load_row = [&](int vr, float* cv, float& s) {
-        if (vr < n8) {
+      auto load_row = [&](int ms, float* cv, float& s) {
+        const int vr = 16 * ms + rb;
+        if (int8_row(ms)) {
           const uint4 w = *reinterpret_cast<const uint4*>(sb + vr * DV + c0);
           const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
           q8s_codes<16>(ww, cv);
@@ -230,7 +236,7 @@ __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, N
 #pragma unroll
         for (int mi = 0; mi < 4; ++mi) {
           float cv[16], s;
-          load_row((m0 + mi) * 16 + rb, cv, s);
+          load_row(m0 + mi, cv, s);
           kq = fmaf(kk4[mi], qq4[mi], kq);
           const float k1 = s * (CHG ? kk4[mi] * aa4[mi] : kk4[mi]);
           const float q1 = s * (CHG ? qq4[mi] * aa4[mi] : qq4[mi]);
@@ -297,63 +303,75 @@ __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, N
         u[j + 3] = u4.w;
       }
 
-      // pass 2: S' = a S + k u^T, stored in the tile's format at the same storage rows
+      // pass 2: S' = a S + k u^T, stored in the tile's format at the same storage rows.
+      // The fast form takes each group's absmax keeping NaN and converts codes with the
+      // float trick; if any INT8 group of the warp held a non-finite value, the whole pass
+      // runs again in the codec's form (absmax ignoring NaN, the conversion unit), which
+      // overwrites every store of the first run.
       unsigned char* dtile = dst + m.dst_off;
       unsigned char* dsc8 = dtile + n8 * DV;
       unsigned char* dhp = dsc8 + n8 * NG * 4;
+      auto pass2 = [&](auto exact_tag) {
+        constexpr bool EXACT = decltype(exact_tag)::value;
+        bool bad = false;
 #pragma unroll
-      for (int m0 = 0; m0 < RL; m0 += 4) {
-        const float4 k4 = *reinterpret_cast<const float4*>(kp + rb * RL + m0);
-        float4 a4 = make_float4(a, a, a, a);
-        if (CHG) a4 = *reinterpret_cast<const float4*>(ap + rb * RL + m0);
-        const float kk4[4] = {k4.x, k4.y, k4.z, k4.w}, aa4[4] = {a4.x, a4.y, a4.z, a4.w};
+        for (int m0 = 0; m0 < RL; m0 += 4) {
+          const float4 k4 = *reinterpret_cast<const float4*>(kp + rb * RL + m0);
+          float4 a4 = make_float4(a, a, a, a);
+          if (CHG) a4 = *reinterpret_cast<const float4*>(ap + rb * RL + m0);
+          const float kk4[4] = {k4.x, k4.y, k4.z, k4.w}, aa4[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-        for (int mi = 0; mi < 4; ++mi) {
-          const int vr = (m0 + mi) * 16 + rb;
-          float cv[16], s;
-          load_row(vr, cv, s);
-          const float as_ = aa4[mi] * s;
-          float y[16];
+          for (int mi = 0; mi < 4; ++mi) {
+            const int ms = m0 + mi;
+            const int vr = 16 * ms + rb;
+            float cv[16], s;
+            load_row(ms, cv, s);
+            const float as_ = aa4[mi] * s;
+            float y[16];
 #pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            const float2 r2 = __ffma2_rn(make_float2(cv[j], cv[j + 1]), make_float2(as_, as_),
-                                         __fmul2_rn(make_float2(kk4[mi], kk4[mi]), make_float2(u[j], u[j + 1])));
-            y[j] = r2.x;
-            y[j + 1] = r2.y;
-          }
-          // the group's absmax: this lane's 16 values, then the other half's
-          float amax = 0.0f;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) amax = fmax_nan(amax, fabsf(y[j]));
-          amax = fmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-          const bool is8 = vr < n8;
-          bool exact_path = false;
-          if (__any_sync(0xffffffffu, is8 && !(amax <= 3.402823466e38f))) {
-            // a non-finite value in some INT8 row group of the warp: the codec's absmax
-            // (NaN ignored) and conversion for this m
-            amax = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(y[j]));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-            exact_path = true;
-          }
-          if (is8) {
-            float sc, inv;
-            q8_scales(amax, sc, inv);
-            uint32_t w[4];
-            if (exact_path) {
-              q8_pack<16>(y, inv, w);
-            } else {
-              q8s_pack<16>(y, inv, w);
+            for (int j = 0; j < 16; j += 2) {
+              const float2 r2 = __ffma2_rn(make_float2(cv[j], cv[j + 1]), make_float2(as_, as_),
+                                           __fmul2_rn(make_float2(kk4[mi], kk4[mi]), make_float2(u[j], u[j + 1])));
+              y[j] = r2.x;
+              y[j + 1] = r2.y;
             }
-            *reinterpret_cast<uint4*>(dtile + vr * DV + c0) = make_uint4(w[0], w[1], w[2], w[3]);
-            if (hf == 0) *reinterpret_cast<float*>(dsc8 + (vr * NG + part) * 4) = sc;
-          } else {
-            uint4* d = reinterpret_cast<uint4*>(dhp + ((vr - n8) * DV + c0) * 2);
-            d[0] = StateVec<__nv_bfloat16>::pack(y);
-            d[1] = StateVec<__nv_bfloat16>::pack(y + 8);
+            if (int8_row(ms)) {
+              // the group's absmax: this lane's 16 values, then the other half's (the two
+              // lanes of a row take the same branch; with NB < 0 other rows may not)
+              const unsigned pair = 3u << (lane & ~1);
+              float amax = 0.0f;
+              if (EXACT) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(y[j]));
+                amax = fmaxf(amax, __shfl_xor_sync(pair, amax, 1));
+              } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) amax = fmax_nan(amax, fabsf(y[j]));
+                amax = fmax_nan(amax, __shfl_xor_sync(pair, amax, 1));
+                bad = bad || !(amax <= 3.402823466e38f);
+              }
+              float sc, inv;
+              q8_scales(amax, sc, inv);
+              uint32_t w[4];
+              if (EXACT) {
+                q8_pack<16>(y, inv, w);
+              } else {
+                q8s_pack<16>(y, inv, w);
+              }
+              *reinterpret_cast<uint4*>(dtile + vr * DV + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+              if (hf == 0) *reinterpret_cast<float*>(dsc8 + (vr * NG + part) * 4) = sc;
+            } else {
+              uint4* d = reinterpret_cast<uint4*>(dhp + ((vr - n8) * DV + c0) * 2);
+              d[0] = StateVec<__nv_bfloat16>::pack(y);
+              d[1] = StateVec<__nv_bfloat16>::pack(y + 8);
+            }
           }
         }
+        return bad;
+      };
+      if (__any_sync(0xffffffffu, pass2(std::false_type{}))) {
+        __syncwarp();  // the first run's stores before the second's (same lanes, same addresses)
+        pass2(std::true_type{});
       }
     }
     __syncwarp();
@@ -361,11 +379,11 @@ __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, N
   }
 }
 
-template <int RULE, int DK, int DV, typename IT>
+template <int RULE, int DK, int DV, typename IT, int NB>
 cudaError_t launch_step_q8s(const StepParams& p, cudaStream_t stream) {
   constexpr int NCW = LA_Q8S_CONSUMER_WARPS / (DV / 32) * (DV / 32);
   using C = Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, NCW>;
-  const void* fn = reinterpret_cast<const void*>(&step_q8s_kernel<RULE, DK, DV, IT, NCW>);
+  const void* fn = reinterpret_cast<const void*>(&step_q8s_kernel<RULE, DK, DV, IT, NCW, NB>);
   const int per_sm = prepare_kernel(fn, C::kThreads, C::kSmem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;
   const int64_t ntiles = (int64_t)p.B * p.n_v_heads;
@@ -382,10 +400,10 @@ cudaError_t launch_step_q8s(const StepParams& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, step_q8s_kernel<RULE, DK, DV, IT, NCW>, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, step_q8s_kernel<RULE, DK, DV, IT, NCW, NB>, p);
   if (e != cudaSuccess) return e;
 #else
-  step_q8s_kernel<RULE, DK, DV, IT, NCW><<<grid, C::kThreads, C::kSmem, stream>>>(p);
+  step_q8s_kernel<RULE, DK, DV, IT, NCW, NB><<<grid, C::kThreads, C::kSmem, stream>>>(p);
 #endif
   return cudaGetLastError();
 }
@@ -394,8 +412,14 @@ cudaError_t launch_step_q8s(const StepParams& p, cudaStream_t stream) {
 // array, the generic step kernel (rows located through each mask) otherwise.
 template <int RULE, int DK, int DV, typename IT>
 cudaError_t launch_step_q8(const StepParams& p, cudaStream_t stream) {
-  if (p.src_mask == p.dst_mask) return launch_step_q8s<RULE, DK, DV, IT>(p, stream);
-  return launch_step<RULE, DK, DV, q8_t, IT, false>(p, stream);
+  if (p.src_mask != p.dst_mask) return launch_step<RULE, DK, DV, q8_t, IT, false>(p, stream);
+  // n_hp <= d_k / 4: at most 2 BF16 row steps of 16 rows for d_k = 128, 1 for d_k = 64
+  switch (p.n_hp % 16 == 0 ? p.n_hp / 16 : -1) {
+    case 0: return launch_step_q8s<RULE, DK, DV, IT, 0>(p, stream);
+    case 1: return launch_step_q8s<RULE, DK, DV, IT, 1>(p, stream);
+    case 2: if constexpr (DK >= 128) return launch_step_q8s<RULE, DK, DV, IT, 2>(p, stream);
+    default: return launch_step_q8s<RULE, DK, DV, IT, -1>(p, stream);
+  }
 }
 
 inline StepLaunchFn find_step_q8_table(int rule, int dk, int dv, int io) {
