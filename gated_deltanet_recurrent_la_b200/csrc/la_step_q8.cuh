@@ -31,8 +31,9 @@
 //    (each lane ends with the two sums of one column, which gives that column's u and o);
 //    u goes to the warp's lanes through shared memory;
 //  * two passes over the staged tile (sums, then update and store) instead of holding the
-//    tile in registers: a thread needs few registers, so three tiles are in compute per SM
-//    (twelve consumer warps) to hide the latencies of one warp per tile strip.
+//    tile in registers: a thread needs few registers (at most 96 with 17 warps), so four
+//    tiles are in compute per SM (sixteen consumer warps) to hide the latencies of one warp
+//    per tile strip.
 #pragma once
 
 #include "la_step.cuh"
@@ -40,7 +41,7 @@
 namespace la {
 
 #ifndef LA_Q8S_CONSUMER_WARPS
-#define LA_Q8S_CONSUMER_WARPS 12
+#define LA_Q8S_CONSUMER_WARPS 16
 #endif
 
 // Stage layout of the generic step (StepCfg) with NCW consumer warps, each with its own
@@ -338,7 +339,7 @@ __global__ void __launch_bounds__(Q8sCfg<DK, DV, IT, Rule<RULE>::kChannelGate, N
             if (int8_row(ms)) {
               // the group's absmax: this lane's 16 values, then the other half's (the two
               // lanes of a row take the same branch; with NB < 0 other rows may not)
-              const unsigned pair = 3u << (lane & ~1);
+              const unsigned pair = NB >= 0 ? 0xffffffffu : 3u << (lane & ~1);
               float amax = 0.0f;
               if (EXACT) {
 #pragma unroll
