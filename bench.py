@@ -128,6 +128,7 @@ def kernel_source_hash(files):
 
 KERNEL_SOURCES = {
     "step": ["la_step.cuh", "la_device.cuh"],
+    "step_q8": ["la_step_q8.cuh", "la_step.cuh", "la_device.cuh"],
     "scan": ["la_scan.cuh", "la_device.cuh"],
     "chunk": ["la_chunk.cuh", "la_device.cuh"],
     "chunk_tc": ["la_chunk.cuh", "la_chunk_tc.cuh", "la_umma.cuh", "la_device.cuh"],
@@ -138,6 +139,12 @@ KERNEL_SOURCES = {
                    "la_device.cuh"],
     "pool": ["la_pool.cu"],
 }
+
+
+def step_kernel(workload):
+    """(traffic key, kernel name) of a decode workload's kernel: q8 pools sharing one mask
+    array run the storage-order q8 kernel, every other step the generic step kernel."""
+    return ("step_q8", "la::step_q8s_kernel") if workload == "q8_decode64" else ("step", "la::step_kernel")
 
 
 def recorded_traffic(kernel, workload):
@@ -864,7 +871,7 @@ def measure_row(name, steps, warmup, world, peaks, sm_count, flush=None, ckpt_ev
         row["tokens_per_s"] = run.B / (ms * 1e-3)
         row["state_steps_per_s"] = run.B * inp.n_v_heads / (ms * 1e-3)
         row["roofline"] = {"bound": "hbm", "achieved": row["gb_s"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": row["gb_s"] / peaks["hbm_gbs"], "traffic": recorded_traffic("step", name),
+                           "frac": row["gb_s"] / peaks["hbm_gbs"], "traffic": recorded_traffic(step_kernel(name)[0], name),
                            "peak_source": peaks["source"]}
         row["pct_of_spec_8000"] = 100 * row["gb_s"] / SPEC_HBM_GBS
         if flush is not None:
@@ -973,9 +980,11 @@ def main():
         out["state_steps_per_s"] = world * run.B * inp.n_v_heads / (ms * 1e-3)
         out["ms_per_step_l2_flushed"] = ms_flushed
         out["roofline"] = {"bound": "hbm", "achieved": per_gpu, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": per_gpu / peaks["hbm_gbs"], "traffic": recorded_traffic("step", a.workload),
+                           "frac": per_gpu / peaks["hbm_gbs"],
+                           "traffic": recorded_traffic(step_kernel(a.workload)[0], a.workload),
                            "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] == "measured"
-                           else "fallback 6650 GB/s", "algorithmic_bytes_per_launch": nbytes, "kernel": "la::step_kernel"}
+                           else "fallback 6650 GB/s", "algorithmic_bytes_per_launch": nbytes,
+                           "kernel": step_kernel(a.workload)[1]}
     else:
         alu = fp32_alu_peak_tflops(sm_count, peaks["sm_max_mhz"])
         tf = flops / (ms * 1e-3) / 1e12

@@ -132,6 +132,7 @@ ScanLaunchFn find_scan_conv_bf16io(int rule, int dk, int dv);
 constexpr int kMaxQueryGroup = 8;
 // q8 state storage (d_v a multiple of 32): (64,64), (128,64), (128,128)
 StepLaunchFn find_step_q8(int rule, int dk, int dv, int io);
+StepLaunchFn find_step_q8_f32io(int rule, int dk, int dv);
 StepLaunchFn find_step_qgroups_f32(int rule, int dk, int dv, int io);
 StepLaunchFn find_step_qgroups_bf16(int rule, int dk, int dv, int io);
 ScanLaunchFn find_scan_qgroups_f32io(int rule, int dk, int dv);

@@ -423,10 +423,11 @@ cudaError_t launch_step_q8(const StepParams& p, cudaStream_t stream) {
   }
 }
 
-inline StepLaunchFn find_step_q8_table(int rule, int dk, int dv, int io) {
-#define LA_Q8S_CASE(R, K, V)                                                                     \
-  if (rule == R && dk == K && dv == V)                                                           \
-    return io == LA_F32 ? &launch_step_q8<R, K, V, float> : &launch_step_q8<R, K, V, __nv_bfloat16>;
+// Launcher table of one io type (each io type in its own translation unit).
+template <typename IT>
+StepLaunchFn find_step_q8_table(int rule, int dk, int dv) {
+#define LA_Q8S_CASE(R, K, V) \
+  if (rule == R && dk == K && dv == V) return &launch_step_q8<R, K, V, IT>;
 #define LA_Q8S_SHAPES(R) LA_Q8S_CASE(R, 64, 64) LA_Q8S_CASE(R, 128, 64) LA_Q8S_CASE(R, 128, 128)
   LA_Q8S_SHAPES(LA_RULE_LINEAR)
   LA_Q8S_SHAPES(LA_RULE_GATED)
