@@ -72,7 +72,7 @@ struct StepMeta {
 // CHG: the rule carries a channel-wise gate (kda), d_k FP32 decays staged with the tile.
 // QMAX: query rows a stage holds (1, or kMaxQueryGroup in the query-group direction).
 // CONV: the short causal convolution runs ahead of the step (the stage also holds the
-// tile's convolution history, and each consumer warp a scratch of post-convolution q, k, v).
+// tile's convolution history and weights, and a scratch of its post-convolution q, k, v).
 template <int DK, int DV, typename ST, typename IT, bool CHG = false, int QMAX = 1, bool CONV = false>
 struct StepCfg {
   static constexpr bool kQ8 = std::is_same<ST, q8_t>::value;
@@ -85,7 +85,10 @@ struct StepCfg {
   static constexpr int kRL = DK / kRG;                  // rows per lane
   static constexpr int kConsumerWarps = kWPT > LA_STEP_CONSUMER_WARPS ? kWPT : LA_STEP_CONSUMER_WARPS;
   static constexpr int kTeams = kConsumerWarps / kWPT;  // tiles in compute at once
-  static constexpr int kThreads = (kConsumerWarps + 1) * 32;
+  // CONV: three warps (the q, k and v channels) run the convolution ahead of the consumers
+  static constexpr int kConvWarps = CONV ? 3 : 0;
+  static constexpr int kProducerWarp = kConsumerWarps + kConvWarps;
+  static constexpr int kThreads = (kProducerWarp + 1) * 32;
   // stage room for one tile; q8 tiles hold at most DK / 4 BF16 rows
   static constexpr int kTileBytes = kQ8 ? (int)q8_tile_bytes(DK, DV, DK / 4) : DK * DV * kSB;
   static constexpr int kQKBytes = DK * (int)sizeof(IT);
@@ -101,14 +104,15 @@ struct StepCfg {
   static constexpr int kConvWBytes = CONV ? (2 * DK + DV) * kMaxConvWidth * 4 : 0;
   static constexpr int kCopyBytes = kOffConvW + kConvWBytes;  // with all QMAX query rows, widest convolution
   static constexpr int kStageBytes = round_up(kCopyBytes, 128);
-  static constexpr int kStages = cmax(2, cmin(12, (204 * 1024) / kStageBytes));
+  // CONV, per stage: the tile's post-convolution q | k | v (FP32)
+  static constexpr int kScrFloats = CONV ? 2 * DK + DV : 0;
+  static constexpr int kStages = CONV ? cmax(2, cmin(12, (222 * 1024) / (kStageBytes + kScrFloats * 4)))
+                                      : cmax(2, cmin(12, (204 * 1024) / kStageBytes));
   static constexpr int kOffMeta = kStages * kStageBytes;
   static constexpr int kOffBars = round_up(kOffMeta + kStages * (int)sizeof(StepMeta), 8);
-  static constexpr int kOffScratch = round_up(kOffBars + 2 * kStages * 8, 16);
-  // CONV, per team (the warps of one tile): post-convolution q | k | v, each warp's partial
-  // sums of q^2 and k^2, each warp's arrival flag
-  static constexpr int kScratchFloats = CONV ? 2 * DK + DV + 3 * kWPT : 0;
-  static constexpr int kSmem = kOffScratch + kTeams * kScratchFloats * 4;
+  // barriers per stage: full, empty (and CONV: convolution done)
+  static constexpr int kOffScratch = round_up(kOffBars + (CONV ? 3 : 2) * kStages * 8, 16);
+  static constexpr int kSmem = kOffScratch + kStages * kScrFloats * 4;
 
   static_assert(kNCH >= 1 && kNCH <= 32 && (32 % kNCH) == 0, "strip row must map onto a power-of-two lane group");
   static_assert(kRL >= 1 && DK % kRG == 0, "rows must split evenly over the row blocks");
@@ -118,75 +122,75 @@ struct StepCfg {
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
-// The short causal convolution ahead of the step, for one tile, by the WPT warps of its
-// team, each taking every WPT-th 32-channel block: channel c is y = sum_j w[c][j]
-// x_{t-W+1+j} over the W - 1 staged history inputs and the current input (weights staged
-// with the tile), then SiLU when asked; q and k are then scaled to unit length when asked
-// (the team's partial sums of squares meet in shared memory).  The results land in the
-// team's FP32 scratch [q | k | v] for all of the team's warps.  Each warp writes its
-// channels' new histories (the last W - 1 inputs) to write slot `ws` (skipped when ws < 0).
-// Every warp of the team passes the team barrier (id bar) twice here.
-template <int DK, int DV, typename IT, int WPT>
-__device__ __forceinline__ void conv_operands(const StepParams& p, const unsigned char* xq_s,
-                                              const unsigned char* xk_s, const unsigned char* xv_s,
-                                              const unsigned char* hist_s, const float* w_s, int h, int H, int ws,
-                                              int part, int lane, float* scr, uint32_t bar) {
+// The convolution warps of a CONV step CTA: warp cw takes the q (cw = 0), k (1) or v (2)
+// channels of every tile of the CTA, in order, as soon as its stage has arrived.  Channel c
+// is y = sum_j w[c][j] x_{t-W+1+j} over the W - 1 staged history inputs and the current
+// input (weights staged with the tile), then SiLU when asked; q and k are then scaled to
+// unit length when asked (a warp reduction: one warp holds all of q's or k's channels).
+// The results land in the stage's FP32 scratch, the channels' new histories (the last
+// W - 1 inputs) go to the tile's write slot, and the warp arrives on the stage's
+// convolution barrier, which the consumers wait for.  Skipped tiles only arrive.
+template <int DK, int DV, typename IT, typename C>
+__device__ __forceinline__ void conv_group(const StepParams& p, unsigned char* smem, const StepMeta* meta,
+                                           uint64_t* full, uint64_t* conv_done, int64_t n_my, int cw, int lane) {
   constexpr int CH = 2 * DK + DV;
-  constexpr int kIters = (CH + 32 * WPT - 1) / (32 * WPT);
+  constexpr int kPer = ((DK > DV ? DK : DV) + 31) / 32;  // channels per lane
+  const int H = p.n_v_heads;
   const int W = p.conv_w;
-  const IT* xq = reinterpret_cast<const IT*>(xq_s);
-  const IT* xk = reinterpret_cast<const IT*>(xk_s);
-  const IT* xv = reinterpret_cast<const IT*>(xv_s);
-  const IT* hist = reinterpret_cast<const IT*>(hist_s);
-  float* partial = scr + CH;  // [WPT][2]
-  float sq = 0.0f, sk = 0.0f;
+  const int c_beg = cw == 0 ? 0 : cw == 1 ? DK : 2 * DK;
+  const int n_ch = cw == 2 ? DV : DK;
+  const int x_off = cw == 0 ? C::kTileBytes : cw == 1 ? C::kOffK : C::kOffV;
+  for (int64_t it = 0; it < n_my; ++it) {
+    const int stage = (int)(it % C::kStages);
+    const uint32_t round = (uint32_t)(it / C::kStages);
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], round & 1u, p.wait_ns))) {
+      if (lane == 0) report(p.err, LA_DEVERR_TIMEOUT);
+      return;
+    }
+    const StepMeta m = meta[stage];
+    if (m.valid) {
+      const unsigned char* sb = smem + stage * C::kStageBytes;
+      const IT* x = reinterpret_cast<const IT*>(sb + x_off);
+      const IT* hist = reinterpret_cast<const IT*>(sb + C::kOffHist);
+      const float* wts = reinterpret_cast<const float*>(sb + C::kOffConvW);
+      float* scr = reinterpret_cast<float*>(smem + C::kOffScratch) + stage * C::kScrFloats;
+      const int h = (int)((blockIdx.x + it * gridDim.x) % H);
+      IT* hd = static_cast<IT*>(p.conv_dst) + ((int64_t)m.ws * H + h) * CH * (W - 1);
+      float y[kPer];
+      float ss = 0.0f;
 #pragma unroll
-  for (int it = 0; it < kIters; ++it) {
-    const int c = (part + WPT * it) * 32 + lane;
-    if (c < CH) {
-      const float* w = w_s + c * W;  // staged weights: q channels, then k, then v
-      const float x = io_load(c < DK ? xq + c : c < 2 * DK ? xk + (c - DK) : xv + (c - 2 * DK));
-      float y = w[W - 1] * x;
+      for (int i = 0; i < kPer; ++i) {
+        const int cl = lane + 32 * i;
+        y[i] = 0.0f;
+        if (cl < n_ch) {
+          const int c = c_beg + cl;
+          const float* w = wts + c * W;
+          float acc = w[W - 1] * io_load(x + cl);
 #pragma unroll
-      for (int j = 0; j < kMaxConvWidth - 1; ++j)
-        if (j < W - 1) y = fmaf(w[j], io_load(hist + c * (W - 1) + j), y);
-      if (p.conv_act) y = __fdividef(y, 1.0f + __expf(-y));
-      scr[c] = y;
-      if (c < DK) sq = fmaf(y, y, sq);
-      else if (c < 2 * DK) sk = fmaf(y, y, sk);
-      if (ws >= 0) {
-        IT* hd = static_cast<IT*>(p.conv_dst) + ((int64_t)ws * H + h) * CH * (W - 1);
-        for (int j = 0; j < W - 2; ++j) hd[c * (W - 1) + j] = hist[c * (W - 1) + j + 1];
-        hd[c * (W - 1) + W - 2] = c < DK ? xq[c] : c < 2 * DK ? xk[c - DK] : xv[c - 2 * DK];
+          for (int j = 0; j < kMaxConvWidth - 1; ++j)
+            if (j < W - 1) acc = fmaf(w[j], io_load(hist + c * (W - 1) + j), acc);
+          if (p.conv_act) acc = __fdividef(acc, 1.0f + __expf(-acc));
+          y[i] = acc;
+          ss = fmaf(acc, acc, ss);
+          for (int j = 0; j < W - 2; ++j) hd[c * (W - 1) + j] = hist[c * (W - 1) + j + 1];
+          hd[c * (W - 1) + W - 2] = x[cl];
+        }
+      }
+      float rn = 1.0f;
+      if (cw < 2 && p.conv_l2norm) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        rn = rsqrtf(ss + 1e-6f);
+      }
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int cl = lane + 32 * i;
+        if (cl < n_ch) scr[c_beg + cl] = y[i] * rn;
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&conv_done[stage]);
   }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    sq += __shfl_xor_sync(0xffffffffu, sq, off);
-    sk += __shfl_xor_sync(0xffffffffu, sk, off);
-  }
-  if (lane == 0) {
-    partial[2 * part] = sq;
-    partial[2 * part + 1] = sk;
-  }
-  named_bar_sync(bar, WPT * 32);
-  if (p.conv_l2norm) {
-    sq = 0.0f;
-    sk = 0.0f;
-#pragma unroll
-    for (int w = 0; w < WPT; ++w) {
-      sq += partial[2 * w];
-      sk += partial[2 * w + 1];
-    }
-    const float rq = rsqrtf(sq + 1e-6f), rk = rsqrtf(sk + 1e-6f);
-#pragma unroll
-    for (int it = 0; it < kIters; ++it) {
-      const int c = (part + WPT * it) * 32 + lane;
-      if (c < 2 * DK) scr[c] *= c < DK ? rq : rk;
-    }
-  }
-  named_bar_sync(bar, WPT * 32);
 }
 
 // The producer warp of a step CTA (whose stage layout is C): its lanes fetch the slot ids
@@ -333,6 +337,7 @@ __global__ void __launch_bounds__(
   StepMeta* meta = reinterpret_cast<StepMeta*>(smem + C::kOffMeta);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
   uint64_t* empty = full + C::kStages;
+  uint64_t* conv_done = empty + C::kStages;  // CONV
 
   const int H = p.n_v_heads;
   const int64_t ntiles = (int64_t)p.B * H;
@@ -342,6 +347,7 @@ __global__ void __launch_bounds__(
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], C::kWPT);
+      if (CONV) mbar_init(&conv_done[s], C::kConvWarps);
     }
     mbar_init_fence();
   }
@@ -356,9 +362,15 @@ __global__ void __launch_bounds__(
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  if (warp == C::kConsumerWarps) {
+  if (warp == C::kProducerWarp) {
     step_producer<RULE, DK, DV, ST, IT, QGRP, CONV, C>(p, smem, meta, full, empty, n_my, lane);
     return;
+  }
+  if constexpr (CONV) {
+    if (warp >= C::kConsumerWarps) {
+      conv_group<DK, DV, IT, C>(p, smem, meta, full, conv_done, n_my, warp - C::kConsumerWarps, lane);
+      return;
+    }
   }
 
   // -------------------------------------------------------------------- consumers
@@ -379,36 +391,22 @@ __global__ void __launch_bounds__(
   for (int64_t it = team; it < n_my; it += C::kTeams) {
     const int stage = (int)(it % C::kStages);
     const uint32_t round = (uint32_t)(it / C::kStages);
-    const bool arrived = mbar_wait(&full[stage], round & 1u, p.wait_ns);
-    bool ok = __all_sync(0xffffffffu, arrived);
-    float* scr = nullptr;
-    if constexpr (CONV) {
-      // the team's warps meet at barriers inside the convolution, so they take the
-      // (bounded) arrival decision together: each posts its flag, all read all flags.
-      // This barrier also orders this tile's scratch writes after the previous tile's reads.
-      scr = reinterpret_cast<float*>(smem + C::kOffScratch) + team * C::kScratchFloats;
-      float* flags = scr + 2 * DK + DV + 2 * C::kWPT;
-      if (lane == 0) flags[part] = ok ? 1.0f : 0.0f;
-      named_bar_sync(1 + team, C::kWPT * 32);
-#pragma unroll
-      for (int w = 0; w < C::kWPT; ++w) ok = ok && flags[w] != 0.0f;
-    }
+    bool arrived = mbar_wait(&full[stage], round & 1u, p.wait_ns);
+    if (CONV && arrived) arrived = mbar_wait(&conv_done[stage], round & 1u, p.wait_ns);  // the tile's q, k, v
+    const bool ok = __all_sync(0xffffffffu, arrived);
     if (!ok) {
       if (lane == 0) report(p.err, LA_DEVERR_TIMEOUT);
       return;
     }
     const StepMeta m = meta[stage];
     const unsigned char* sb = smem + stage * C::kStageBytes;
-    // q, k, v of the step: the staged rows, or (CONV) this warp's post-convolution scratch
+    // q, k, v of the step: the staged rows, or (CONV) the stage's post-convolution scratch
     using OT = std::conditional_t<CONV, float, IT>;
     const OT* qs;
     const OT* ks;
     const OT* vs;
     if constexpr (CONV) {
-      conv_operands<DK, DV, IT, C::kWPT>(p, sb + C::kTileBytes, sb + C::kOffK, sb + C::kOffV, sb + C::kOffHist,
-                                         reinterpret_cast<const float*>(sb + C::kOffConvW),
-                                         (int)((blockIdx.x + it * gridDim.x) % H), H, m.valid ? m.ws : -1, part,
-                                         lane, scr, 1 + team);
+      const float* scr = reinterpret_cast<const float*>(smem + C::kOffScratch) + stage * C::kScrFloats;
       qs = scr;
       ks = scr + DK;
       vs = scr + 2 * DK;
