@@ -415,6 +415,8 @@ template <int RULE, int DK, int DV, typename IT>
 cudaError_t launch_step_q8(const StepParams& p, cudaStream_t stream) {
   if (p.src_mask != p.dst_mask) return launch_step<RULE, DK, DV, q8_t, IT, false>(p, stream);
   // n_hp <= d_k / 4: at most 2 BF16 row steps of 16 rows for d_k = 128, 1 for d_k = 64
+  // (with d_k = 64 case 2 cannot occur; were it reached it would fall through to the
+  // kernel that decides each row's kind at run time, which takes any even n_hp)
   switch (p.n_hp % 16 == 0 ? p.n_hp / 16 : -1) {
     case 0: return launch_step_q8s<RULE, DK, DV, IT, 0>(p, stream);
     case 1: return launch_step_q8s<RULE, DK, DV, IT, 1>(p, stream);
