@@ -62,8 +62,12 @@
  *     host): write slots are distinct, and no write slot equals another request's read
  *     slot.  Read slots may repeat; a request may read and write the same slot.
  *   - LA_Q8 pools: la_state_step takes them as source and destination together (equal
- *     n_hp; the masks may differ); the scans take them as source and / or destination;
- *     la_state_scan_chunked and the query-group entry points return LA_ERR_UNSUPPORTED.
+ *     n_hp; the masks may differ, but the step is fastest when both pools use one mask
+ *     array, as an in-place pool does); the token-serial scans and the one-launch chunked
+ *     prefill (la_state_scan_chunked, its checkpointed form, la_state_scan_chunked_qgroups)
+ *     take them as source and / or destination; the two-launch chunked forms, the
+ *     convolution entry points, the kda chunked prefill and la_state_step_qgroups /
+ *     la_state_scan_qgroups return LA_ERR_UNSUPPORTED.
  *   - Pointers to the pool, q, k, v, o and dense buffers must be 16-byte aligned;
  *     g, beta and int32 arrays 4-byte aligned.
  */
